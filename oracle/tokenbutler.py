@@ -1,0 +1,237 @@
+"""Plain fp64 CPU oracle of the TokenButler decode-step hot path.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or run
+this module.  It shares no code with the CUDA path: it is numpy in float64,
+step by step in the order and notation of the sources, with no blocking,
+fusion or reordering.
+
+Sources (cited by page title and section):
+  [MC]  "Meta-Llama-3.1-8B-Instruct-Butler" model card: section "Method"
+        (producer layers, Q_imp, W_K, K_imp, consumer slot, top-x selection
+        with sink prefix and local window, full KV cache kept) and section
+        "Memory requirements" (fixed_<N>pc policy, default 50 %, layer 0 dense,
+        min_sparse_index = sink length, sliding_window).
+  [AB]  "TokenButler: Token Importance is Predictable", abstract (fixed budget,
+        per-token selection, full KV cache preserved).
+  [TS]  TokenSelect README, "Dynamic Token-Level KV Cache Selection" and
+        "Per-head Soft Voting Mechanism".
+
+Readings where the sources leave a step open (each marked "Reading" below):
+  R1  W_K is one D x d' matrix per layer, shared by all KV heads.
+  R2  query head h reads KV head h // (Hq / Hkv).
+  R3  importance scores carry no scale (a scale cannot change a top-k).
+  R4  consumer layer l reads producer G * floor(l / G), slot (l - 1) mod G
+      (non-negative mod); layer 0's slot is never used (layer 0 is dense).
+  R5  budget k = floor(P * L / 100), L counting the current token.
+  R6  the top-k candidates exclude the sink and the window, so the selected
+      set has exactly min(L, s + w + k) tokens.
+  R7  k is clamped to the candidate count; a 100 % budget selects every token.
+  R8  ties in score go to the lower token index; -0.0 equals +0.0.
+  R9  attention uses the real query q, full head dim, scale 1/sqrt(D), over
+      the untouched K/V.
+  R13 prefill row p uses its causal prefix [0, p] with L -> p + 1.
+  R14 soft voting: softmax over all t < L per head, scale 1/sqrt(D), votes
+      summed over all query heads, one set shared by all heads.
+  An empty selected set gives a zero output and lse = -inf.
+
+Parity pins (tests/test_oracle_pins.py) cover every function here; the
+readings R4, R6, R13 and R14 are consistent with the sources but not fixed
+by them (parity unpinned against the pages for those readings).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ------------------------------------------------------------------ layers
+def producer_of(layer: int, G: int) -> int:
+    """[MC] Method: producers sit at layers 0, G, 2G, ...; each predicts for
+    itself and the next G - 1 layers.  Reading R4."""
+    return G * (layer // G)
+
+
+def consumer_slot(layer: int, G: int) -> int:
+    """[MC] Method: a consumer at layer l uses slot (l - 1) mod G of its
+    producer's importance queries.  Reading R4: non-negative mod."""
+    return (layer - 1) % G
+
+
+def importance_queries(q_imp_producer: np.ndarray, layer: int, G: int, B: int, Hq: int,
+                       position: int = 0) -> np.ndarray:
+    """[MC] Method: Q_imp has shape (B*H) x G x L x d'.  Returns the consumer's
+    query per (b, h): q_hat[b, h] = Q_imp[b*Hq + h, slot, position, :]."""
+    slot = consumer_slot(layer, G)
+    q = np.asarray(q_imp_producer, dtype=np.float64)
+    return q[:, slot, position, :].reshape(B, Hq, q.shape[-1])
+
+
+def kv_head_of(h: int, Hq: int, Hkv: int) -> int:
+    """Reading R2: contiguous groups of Hq / Hkv query heads share a KV head."""
+    return h // (Hq // Hkv)
+
+
+def keep_pct_from_policy(policy: str) -> int:
+    """[MC] Memory requirements: "fixed_<N>pc" sparsifies N % of the tokens,
+    i.e. retains 100 - N %."""
+    if not (policy.startswith("fixed_") and policy.endswith("pc")):
+        raise ValueError(f"unsupported policy {policy!r}")
+    n = int(policy[len("fixed_"):-len("pc")])
+    if not 0 <= n <= 100:
+        raise ValueError(f"sparsity {n} % out of range")
+    return 100 - n
+
+
+# ------------------------------------------------------------------ a1: K_imp
+def project_keys(K: np.ndarray, W_K: np.ndarray) -> np.ndarray:
+    """[MC] Method: K_imp = K . W_K on the post-RoPE cached keys (fp64, no
+    rounding).  K: [..., D], W_K: [D, d'] (Reading R1)."""
+    return np.asarray(K, dtype=np.float64) @ np.asarray(W_K, dtype=np.float64)
+
+
+# ------------------------------------------------------------------ a3: scores
+def importance_scores(q_hat: np.ndarray, K_imp: np.ndarray) -> np.ndarray:
+    """[MC] Method: score every cached token with the consumer's importance
+    query: s[t] = q_hat . K_imp[t] (Reading R3: no scale).  q_hat: [d'],
+    K_imp: [L, d']."""
+    return np.asarray(K_imp, dtype=np.float64) @ np.asarray(q_hat, dtype=np.float64)
+
+
+# ------------------------------------------------------------------ a4/a5: select
+def token_budget(L: int, keep_pct: int) -> int:
+    """Reading R5: k = floor(P * L / 100)."""
+    return (keep_pct * L) // 100
+
+
+def select_tokens(scores: np.ndarray, L: int, keep_pct: int, sink: int, window: int) -> np.ndarray:
+    """[MC] Method + Memory requirements: the top-x tokens under a fixed
+    budget, plus the sink prefix (min_sparse_index) and the recent window
+    (sliding_window).  Returns the selected token indices, ascending.
+
+    Candidates are [sink, L - window) (Reading R6); the budget is clamped to
+    their number (R7); order is (score descending, index ascending) (R8)."""
+    s = np.asarray(scores, dtype=np.float64)[:L]
+    sink_set = np.arange(0, min(sink, L), dtype=np.int64)
+    window_set = np.arange(max(L - window, 0), L, dtype=np.int64)
+    cand = np.arange(sink, L - window, dtype=np.int64) if L - window > sink else np.zeros(0, np.int64)
+    k = min(token_budget(L, keep_pct), cand.size)
+    order = np.lexsort((cand, -s[cand]))  # primary key last: score desc, then index asc
+    top = cand[order[:k]]
+    return np.union1d(np.union1d(sink_set, window_set), top).astype(np.int64)
+
+
+# ------------------------------------------------------------------ a6: attention
+def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, scale: float):
+    """[AB] + [MC] Method: exact attention over the selected tokens of the full
+    KV cache: o = sum_{t in Sel} softmax_t(scale * q . K[t]) V[t].  Returns
+    (o, lse) with lse = log sum_{t in Sel} exp(scale * q . K[t]) (natural log).
+    Reading R9: scale = 1/sqrt(D)."""
+    q = np.asarray(q, dtype=np.float64)
+    idx = np.asarray(idx, dtype=np.int64)
+    if idx.size == 0:
+        return np.zeros(q.shape[-1], np.float64), -math.inf
+    Ks = np.asarray(K, dtype=np.float64)[idx]
+    Vs = np.asarray(V, dtype=np.float64)[idx]
+    logits = scale * (Ks @ q)
+    m = logits.max()
+    w = np.exp(logits - m)
+    z = w.sum()
+    return (w @ Vs) / z, m + math.log(z)
+
+
+# ------------------------------------------------------------------ one decode layer
+def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, dense: bool,
+                 K_imp=None, heads=None, batches=None):
+    """One consumer layer's decode step, [MC] Method in order:
+    K_imp = K W_K; consumer slot (l - 1) mod G; score every cached token;
+    top-k + sink + window per query head; attention over the selected tokens.
+    A dense layer (layer 0, [MC] Memory requirements) attends to every token.
+
+    q: [B][Hq][D]; K, V: [B][Hkv][>=L][D]; W_K: [D][d'];
+    q_imp_producer: [(B*Hq)][G][1][d']; L: int or per-sequence list.
+    Returns dicts keyed by (b, h): selected indices, output [D], lse; and the
+    fp64 scores per (b, h) (None for dense layers)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    lens = [L] * B if np.isscalar(L) else list(L)
+    scale = 1.0 / math.sqrt(D)
+    heads = range(Hq) if heads is None else heads
+    batches = range(B) if batches is None else batches
+    sel, out, lse, scores = {}, {}, {}, {}
+    q_hat = None if dense else importance_queries(q_imp_producer, layer, G, B, Hq)
+    for b in batches:
+        Lb = lens[b]
+        kimp_b = {}
+        for h in heads:
+            g = kv_head_of(h, Hq, Hkv)
+            if dense:
+                idx = np.arange(Lb, dtype=np.int64)
+                scores[b, h] = None
+            else:
+                if g not in kimp_b:
+                    kimp_b[g] = (project_keys(K[b, g, :Lb], W_K) if K_imp is None
+                                 else np.asarray(K_imp[b, g, :Lb], dtype=np.float64))
+                s = importance_scores(q_hat[b, h], kimp_b[g])
+                scores[b, h] = s
+                idx = select_tokens(s, Lb, keep_pct, sink, window)
+            sel[b, h] = idx
+            out[b, h], lse[b, h] = attend(q[b, h], K[b, g, :Lb], V[b, g, :Lb], idx, scale)
+    return sel, out, lse, scores
+
+
+# ------------------------------------------------------------------ a7: prefill rows
+def prefill_select(q_hat_rows: np.ndarray, K_imp: np.ndarray, row0: int, keep_pct: int, sink: int,
+                   window: int) -> dict:
+    """Per-row selection of a prefill query chunk (Reading R13): row p of head
+    h scores its causal prefix s_p[t] = q_hat[h, p - row0] . K_imp[g(h), t],
+    t <= p, and selects with L -> p + 1.  q_hat_rows: [Hq][nrows][d'];
+    K_imp: [Hkv][>= row0 + nrows][d'].  Returns {(h, p): indices}."""
+    Hq, nrows, _ = q_hat_rows.shape
+    Hkv = K_imp.shape[0]
+    out = {}
+    for h in range(Hq):
+        g = kv_head_of(h, Hq, Hkv)
+        for r in range(nrows):
+            p = row0 + r
+            s = importance_scores(q_hat_rows[h, r], K_imp[g, :p + 1])
+            out[h, p] = select_tokens(s, p + 1, keep_pct, sink, window)
+    return out
+
+
+# ------------------------------------------------------------------ a8: soft voting
+def softvote_scores(q: np.ndarray, K: np.ndarray, L: int) -> np.ndarray:
+    """[TS] Per-head Soft Voting: per-head criticality a[h, t] = q_h . K[g(h), t]
+    / sqrt(D), normalised by a softmax over the tokens, summed over all heads
+    (Reading R14).  q: [Hq][D]; K: [Hkv][>=L][D].  Returns votes [L]."""
+    q = np.asarray(q, dtype=np.float64)
+    Hq, D = q.shape
+    Hkv = K.shape[0]
+    votes = np.zeros(L, np.float64)
+    for h in range(Hq):
+        a = (np.asarray(K[kv_head_of(h, Hq, Hkv), :L], dtype=np.float64) @ q[h]) / math.sqrt(D)
+        p = np.exp(a - a.max())
+        votes += p / p.sum()
+    return votes
+
+
+def softvote_layer(q, K, V, L, keep_pct, sink, window, batches=None):
+    """[TS] soft-voting variant of one decode layer: one shared selection per
+    sequence from the summed per-head softmaxes, then exact attention per
+    head over that set.  q: [B][Hq][D]; K, V: [B][Hkv][>=L][D]."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    lens = [L] * B if np.isscalar(L) else list(L)
+    batches = range(B) if batches is None else batches
+    sel, out, lse, votes = {}, {}, {}, {}
+    for b in batches:
+        votes[b] = softvote_scores(q[b], K[b], lens[b])
+        sel[b] = select_tokens(votes[b], lens[b], keep_pct, sink, window)
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            out[b, h], lse[b, h] = attend(q[b, h], K[b, g, :lens[b]], V[b, g, :lens[b]], sel[b],
+                                          1.0 / math.sqrt(D))
+    return sel, out, lse, votes
