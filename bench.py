@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the TokenButler hot path on B200.
+
+One step = one decode token through all layers of the workload: for every
+layer, append the new key/value (+ its K_imp row), then layer 0 attends
+densely and every other layer scores all cached tokens with its producer's
+importance query, selects top-k + sink + window per query head and attends
+over the selected tokens.  Default workload: 32 layers, G = 4, B = 4,
+L = 131072 cached tokens per sequence, Llama-3.1-8B shapes (32 query / 8 KV
+heads, D = 128, d' = 32), bf16 caches, keep 30 % + sink 16 + window 64.
+
+Inputs are seeded synthetic tensors made on the device by the shared
+generator; the caches (about 86 GB) are far larger than L2, so no flush is
+needed between steps.  Multi-GPU: independent replicas (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-step latency (us/layer) & KV tokens scored+attended/s; HBM GB/s vs roofline"
+UNIT = "KV head-tokens scored+attended/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--batch", type=int, default=4)
+    ap.add_argument("--length", type=int, default=131072)
+    ap.add_argument("--keep", type=int, default=30)
+    ap.add_argument("--trace-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def workload(args):
+    from query_aware_sparse_decode_b200 import synth as S
+    base = S.DECODE32_B4_L131072
+    wl = base.with_(n_layers=args.layers, B=args.batch, L=args.length, keep_pct=args.keep)
+    if (wl.n_layers, wl.B, wl.L, wl.keep_pct) != (base.n_layers, base.B, base.L, base.keep_pct):
+        wl = wl.with_(name=f"decode{wl.n_layers}_bf16_B{wl.B}_L{wl.L}_keep{wl.keep_pct}")
+    return wl
+
+
+def step_counts(wl):
+    """(scored, attended) head-token pairs of one step."""
+    scored = attended = 0
+    k = (wl.keep_pct * wl.L) // 100
+    sel = min(wl.L, wl.sink + wl.window + min(k, max(wl.L - wl.sink - wl.window, 0)))
+    for layer in range(wl.n_layers):
+        if layer in wl.dense_layers or wl.keep_pct == 100:
+            attended += wl.B * wl.Hq * wl.L
+        else:
+            scored += wl.B * wl.Hq * wl.L
+            attended += wl.B * wl.Hq * sel
+    return scored, attended
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------- ranks
+def max_over_ranks_of(x: float, world: int, device) -> float:
+    """Largest value of `x` over all ranks (timing is the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
+
+
+# ----------------------------------------------------------------------- GPU arm
+def build(wl, max_len, dev):
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    from query_aware_sparse_decode_b200 import tb as TB
+    cfg = TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G, max_len, wl.dtype, wl.keep_pct,
+                         wl.sink, wl.window, dense_layers=wl.dense_layers)
+    ctx = TB.Context(cfg, dev)
+    L0 = wl.L - 1
+    bufs = []
+    for layer in range(wl.n_layers):
+        k = torch.empty((wl.B, wl.Hkv, max_len, wl.D), dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        kimp = torch.empty((wl.B, wl.Hkv, max_len, wl.d_imp), dtype=torch.float32, device=dev)
+        w_raw = S.w_k(wl, layer)
+        w = torch.from_numpy(w_raw.view(np.int16)).view(torch.bfloat16).to(dev)
+        delta = None
+        if layer not in wl.dense_layers:
+            # input recipe: planted keys of layer l stand out for the queries of
+            # slot (l - 1) mod G of producer G * floor(l / G)
+            qi = S.widen(S.q_imp(wl, wl.G * (layer // wl.G), 0), "bf16")
+            qhat = qi[:, (layer - 1) % wl.G, 0, :].reshape(wl.B, wl.Hq, wl.d_imp)
+            delta = torch.from_numpy(S.plant_delta(S.widen(w_raw, "bf16"), qhat, wl.Hkv)).to(dev)
+        S.fill_device(k, S.K_CACHE, layer, 0, wl.B * wl.Hkv, 0, L0, wl.D, max_len * wl.D, wl.D, "bf16",
+                      delta=delta, plant_mod=100 if delta is not None else 0, seed=wl.seed)
+        S.fill_device(v, S.V_CACHE, layer, 0, wl.B * wl.Hkv, 0, L0, wl.D, max_len * wl.D, wl.D, "bf16",
+                      seed=wl.seed)
+        ctx.bind_layer(layer, k, v, kimp, w)
+        ctx.set_seq_lens(layer, [L0] * wl.B)
+        ctx.project_kimp(layer, 0, L0)
+        bufs.append((k, v, kimp, w))
+    torch.cuda.synchronize()
+    return ctx, bufs
+
+
+def step_inputs_host(wl, s):
+    """Pinned host tensors of step s: k_new, v_new [layers][B][Hkv][D],
+    q [layers][B][Hq][D], q_imp [producers][(B*Hq)][G][1][d']."""
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+
+    def t(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+    kn, vn, qq = [], [], []
+    for layer in range(wl.n_layers):
+        k, v = S.kv_new(wl, layer, s)
+        kn.append(k)
+        vn.append(v)
+        qq.append(S.query(wl, layer, s))
+    nprod = (wl.n_layers + wl.G - 1) // wl.G
+    qi = [S.q_imp(wl, p * wl.G, s) for p in range(nprod)]
+    return t(np.stack(kn)), t(np.stack(vn)), t(np.stack(qq)), t(np.stack(qi))
+
+
+def run_step(ctx, wl, L0, inp, out, stream=None):
+    kn, vn, qq, qi = inp
+    for layer in range(wl.n_layers):
+        ctx.set_seq_lens(layer, [L0] * wl.B)
+        ctx.decode_step(layer, kn[layer], vn[layer], qq[layer], qi[layer // wl.G], out[layer], stream)
+
+
+def union_rows(ctx, wl, L0, inp):
+    """Rows of the per-KV-head union of the selected sets (bytes attended) per
+    sparse layer, measured from the library's own selection of one step."""
+    import torch
+    from query_aware_sparse_decode_b200 import tb as TB
+    kn, vn, qq, qi = inp
+    max_len = ctx.cfg.max_len
+    scores = torch.empty((wl.B, wl.Hq, max_len), device=ctx.device)
+    mask = torch.zeros((wl.B, wl.Hq, max_len // 32), dtype=torch.int32, device=ctx.device)
+    gs = wl.Hq // wl.Hkv
+    rows = {}
+    for layer in range(wl.n_layers):
+        if layer in wl.dense_layers:
+            continue
+        ctx.set_seq_lens(layer, [L0 + 1] * wl.B)
+        ctx.score(layer, qi[layer // wl.G], scores)
+        ctx.select(layer, scores, wl.Hq, mask=mask)
+        m = mask.view(wl.B, wl.Hkv, gs, -1)
+        u = m[:, :, 0]
+        for j in range(1, gs):
+            u = u | m[:, :, j]
+        bits = np.unpackbits(u.cpu().numpy().view(np.uint8), bitorder="little")
+        rows[layer] = int(bits.sum())
+    return rows
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from query_aware_sparse_decode_b200 import tb as TB
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workload(args)
+    L0 = wl.L - 1
+    max_len = (wl.L + 255) // 256 * 256
+    if max_len == wl.L:
+        max_len += 256
+    ctx, bufs = build(wl, max_len, dev)
+    stream = torch.cuda.current_stream(dev)
+    nvar = min(args.steps + args.warmup, 4)
+    host_inputs = [step_inputs_host(wl, s) for s in range(nvar)]
+    dev_inputs = [tuple(x.to(dev) for x in h) for h in host_inputs]
+    out = torch.empty((wl.n_layers, wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    scored, attended = step_counts(wl)
+    tokens = scored + attended
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        return max_over_ranks_of(x, world, dev)
+
+    for s in range(args.warmup):
+        run_step(ctx, wl, L0, dev_inputs[s % nvar], out, stream)
+    barrier()
+
+    # ---- device-timed region: inputs resident in HBM
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local_rank)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    n0 = ctx.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for s in range(args.steps):
+        run_step(ctx, wl, L0, dev_inputs[s % nvar], out, stream)
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    launches = ctx.launch_count() - n0
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms / args.steps
+    value = whole_job_rate(tokens, args.steps, world, ms)
+
+    # ---- per-kernel times (trace events inside decode_step, same workload)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(wl.n_layers)]
+    seg = {"append": [], "score": [], "select": [], "attn": [], "combine": [], "attn_dense": []}
+    kn, vn, qq, qi = dev_inputs[0]
+    for s in range(args.trace_steps):
+        for layer in range(wl.n_layers):
+            ctx.trace_events(ev[layer])
+            ctx.set_seq_lens(layer, [L0] * wl.B)
+            ctx.decode_step(layer, kn[layer], vn[layer], qq[layer], qi[layer // wl.G], out[layer], stream)
+        ctx.trace_events(None)
+        torch.cuda.synchronize(dev)
+        for layer in range(wl.n_layers):
+            e = ev[layer]
+            t = [e[i].elapsed_time(e[i + 1]) * 1e3 for i in range(5)]  # us
+            seg["append"].append(t[0])
+            seg["combine"].append(t[4])
+            if layer in wl.dense_layers:
+                seg["attn_dense"].append(t[3])
+            else:
+                seg["score"].append(t[1])
+                seg["select"].append(t[2])
+                seg["attn"].append(t[3])
+    avg = {k: (sum(v) / len(v) if v else 0.0) for k, v in seg.items()}
+
+    # ---- algorithmic bytes
+    urows = union_rows(ctx, wl, L0, dev_inputs[0])
+    sparse_layers = [l for l in range(wl.n_layers) if l not in wl.dense_layers]
+    row_kv = 2 * wl.D * 2                                   # K + V row, bf16
+    kimp_bytes = wl.B * wl.Hkv * wl.L * wl.d_imp * 4         # per sparse layer
+    union_bytes = (sum(urows.values()) / max(len(urows), 1)) * row_kv
+    dense_bytes = wl.B * wl.Hkv * wl.L * row_kv
+    step_bytes = len(sparse_layers) * (kimp_bytes + union_bytes) + (wl.n_layers - len(sparse_layers)) * dense_bytes
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak, peak_src = 6650.0, "fallback"
+    if os.path.exists(peaks_path):
+        with open(peaks_path) as f:
+            peak, peak_src = float(json.load(f)["hbm_gbs"]), "measured"
+    attn_gbs = union_bytes / (avg["attn"] * 1e-6) / 1e9 if avg["attn"] else None
+    score_gbs = kimp_bytes / (avg["score"] * 1e-6) / 1e9 if avg["score"] else None
+    pair_gbs = ((kimp_bytes + union_bytes) / ((avg["score"] + avg["attn"]) * 1e-6) / 1e9
+                if avg["attn"] else None)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dbuf = tuple(torch.empty_like(x) for x in dev_inputs[0])
+        h2d = sum(x.numel() * x.element_size() for x in host_inputs[0])
+        d2h = out.numel() * out.element_size()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(args.steps):
+            for dst, src in zip(dbuf, host_inputs[s % nvar]):
+                dst.copy_(src, non_blocking=True)
+            run_step(ctx, wl, L0, dbuf, out, stream)
+            out_host.copy_(out, non_blocking=True)
+        f1.record(stream)
+        barrier()
+        ems = max_over_ranks(f0.elapsed_time(f1))
+        e2e = {"value": whole_job_rate(tokens, args.steps, world, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems / args.steps}
+
+    status = ctx.check_status()
+    if status:
+        raise RuntimeError(f"device status flags {status:#x}")
+    return dict(wl=wl, value=value, ms_step=ms_step, clk=clk, launches=launches, avg=avg, urows=urows,
+                union_bytes=union_bytes, kimp_bytes=kimp_bytes, step_bytes=step_bytes, peak=peak,
+                peak_src=peak_src, attn_gbs=attn_gbs, score_gbs=score_gbs, pair_gbs=pair_gbs, e2e=e2e,
+                scored=scored, attended=attended)
+
+
+# ----------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(wl, seconds: float):
+    """Times the fp64 oracle on whole (layer, sequence) slabs of the workload
+    (score, select, attend for all query heads; inputs regenerated on the host
+    and excluded from the timing) until about `seconds` of oracle work."""
+    from oracle import tokenbutler as O
+    from query_aware_sparse_decode_b200 import synth as S
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    L0 = wl.L - 1
+    elapsed, tokens, slabs = 0.0, 0, []
+    sparse_layers = [l for l in range(wl.n_layers) if l not in wl.dense_layers] or [0]
+    i = 0
+    while (elapsed < seconds or i == 0) and i < 16:
+        layer = sparse_layers[(1 + 7 * i) % len(sparse_layers)]
+        b = i % wl.B
+        W = S.widen(S.w_k(wl, layer), wl.dtype)
+        qi = S.widen(S.q_imp(wl, O.producer_of(layer, wl.G), 0), wl.dtype)
+        qhat = O.importance_queries(qi, layer, wl.G, wl.B, wl.Hq)
+        delta = S.plant_delta(W, qhat, wl.Hkv)
+        K = S.widen(S.kv_cache_host(wl, layer, S.K_CACHE, 0, L0, delta, b_range=(b, 1)), wl.dtype)
+        V = S.widen(S.kv_cache_host(wl, layer, S.V_CACHE, 0, L0, b_range=(b, 1)), wl.dtype)
+        kn, vn = S.kv_new(wl, layer, 0)
+        K = np.concatenate([K, S.widen(kn, wl.dtype)[b][:, None]], axis=1)[None]
+        V = np.concatenate([V, S.widen(vn, wl.dtype)[b][:, None]], axis=1)[None]
+        Kimp = O.project_keys(K, W)
+        q = S.widen(S.query(wl, layer, 0), wl.dtype)[b:b + 1]
+        qi_b = qi.reshape(wl.B, wl.Hq, wl.G, 1, wl.d_imp)[b]
+        t0 = time.perf_counter()
+        sel, _, _, _ = O.decode_layer(q, K, V, W, qi_b, layer, wl.G, wl.L, wl.keep_pct, wl.sink, wl.window,
+                                      dense=False, K_imp=Kimp)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        tokens += wl.Hq * wl.L + sum(len(v) for v in sel.values())
+        slabs.append((layer, b))
+        i += 1
+    return {"value": tokens / elapsed, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(slabs)} (layer, sequence) slabs of {wl.name}: score + select + attend for all "
+                      f"{wl.Hq} query heads at L={wl.L}, fp64 numpy, {elapsed:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    wl = workload(args)
+    vals = []
+    for s in range(args.warmup + args.steps):
+        r = oracle_sample(wl, seconds=0.0)  # one slab per step
+        if s >= args.warmup:
+            vals.append(r)
+    value = statistics.mean(v["value"] for v in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "layers": wl.n_layers, "keep_pct": wl.keep_pct,
+                       "sink": wl.sink, "window": wl.window},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": "each step: " + vals[0]["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- main
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    r = gpu_arm(args, rank, world, local_rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(r["wl"], args.cpu_seconds)
+    if rank == 0:
+        wl = r["wl"]
+        avg = r["avg"]
+        attn_launch_bytes = r["union_bytes"]
+        line = {
+            "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "layers": wl.n_layers, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                       "D": wl.D, "d_imp": wl.d_imp, "G": wl.G, "L": wl.L, "keep_pct": wl.keep_pct,
+                       "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (caches of all layers, no flush)"},
+            "us_per_layer": r["ms_step"] * 1e3 / wl.n_layers,
+            "tokens_scored_per_step": r["scored"], "tokens_attended_per_step": r["attended"],
+            "hbm_gbs_step": r["step_bytes"] / (r["ms_step"] * 1e-3) / 1e9,
+            "roofline": {"kernel": "butler_sparse_attn (sparse layers)", "bound": "hbm",
+                         "achieved": r["attn_gbs"], "peak": r["peak"], "unit": "GB/s",
+                         "frac": (r["attn_gbs"] / r["peak"]) if r["attn_gbs"] else None, "traffic": None,
+                         "bytes_per_launch": attn_launch_bytes, "peak_source": r["peak_src"]},
+            "roofline_score_plus_attn": {"achieved": r["pair_gbs"], "peak": r["peak"], "unit": "GB/s",
+                                         "frac": (r["pair_gbs"] / r["peak"]) if r["pair_gbs"] else None},
+            "roofline_score": {"achieved": r["score_gbs"], "peak": r["peak"], "unit": "GB/s",
+                               "frac": (r["score_gbs"] / r["peak"]) if r["score_gbs"] else None,
+                               "bytes_per_launch": r["kimp_bytes"]},
+            "kernel_us": avg,
+            "union_rows_per_layer": (sum(r["urows"].values()) / max(len(r["urows"]), 1)),
+            "gpu_launches": r["launches"],
+            "clocks": r["clk"],
+            "e2e": r["e2e"],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

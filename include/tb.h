@@ -1,0 +1,224 @@
+/*
+ * tb.h — C ABI of the TokenButler decode-step hot path on B200 (sm_100a).
+ *
+ * Each decode step of a consumer layer l:
+ *   1. appends the new token's key/value and its importance key
+ *      K_imp = K . W_K  (model card "Meta-Llama-3.1-8B-Instruct-Butler",
+ *      section "Method": learned projection of the real post-RoPE keys);
+ *   2. scores every cached token with the importance query that the layer's
+ *      producer (layer G*floor(l/G)) emitted in slot (l - 1) mod G
+ *      (same section: producers at layers 0, G, 2G, ...);
+ *   3. keeps, per query head, the top-k tokens under a fixed budget plus a
+ *      sink prefix and a recent local window (same section; budget policy
+ *      fixed_<N>pc, min_sparse_index and sliding_window in section
+ *      "Memory requirements"; layer 0 dense);
+ *   4. runs exact attention over only the kept tokens of the untouched full
+ *      KV cache (model card introduction; TokenButler abstract: "fixed
+ *      budget while preserving the full KV cache").
+ * The soft-voting variant (TokenSelect README, "Per-head Soft Voting
+ * Mechanism") replaces 2-3 by one ranking shared by all heads: per-head
+ * softmax of q . K / sqrt(D), summed over the heads.
+ *
+ * Conventions
+ *   - Ownership: the caller owns every buffer (caches, W_K, queries, outputs,
+ *     workspace).  The library never allocates or frees device memory; a
+ *     tb_ctx is a small host object that records pointers and lengths.
+ *   - Pointers named *_cache, q*, k_new, v_new, out, scores, idx, count, mask,
+ *     lse and the workspace are DEVICE pointers; *_host arguments are host
+ *     pointers.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - All compute calls are asynchronous on `stream`.  Argument and shape
+ *     errors are detected on the host and returned synchronously before
+ *     anything is launched; TB_ERR_CUDA reports a launch error.  Errors seen
+ *     by a kernel set bits of a device status word, read by tb_check_status()
+ *     after a synchronisation.  Nothing aborts, traps or throws.
+ *   - Layouts are dense and row-major (last index fastest):
+ *       K cache, V cache   [B][Hkv][max_len][D]   kv_dtype
+ *       K_imp cache        [B][Hkv][max_len][d']  fp32 (always)
+ *       W_K                [D][d']                kv_dtype
+ *       q_imp (producer)   [(B*Hq)][G][n][d']     kv_dtype  (model card: (B.H) x G x L x d')
+ *       q, out             [B][Hq][D]             kv_dtype
+ *       k_new, v_new       [B][Hkv][D]            kv_dtype
+ *       scores             [B][Hq][max_len]       fp32
+ *       mask (per head)    [B][Hq][max_len/32]    uint32, bit t%32 of word t/32
+ *       mask (shared)      [B][max_len/32]        uint32  (soft voting)
+ *       idx                [B][Hq][idx_cap]       int32, ascending
+ *       count, lse         [B][Hq]                int32 / fp32
+ *     Every device pointer must be 16-byte aligned; max_len must be a
+ *     multiple of 256.
+ *   - Query head h reads KV head h / (Hq / Hkv).
+ *   - Sequence b of layer l holds len[l][b] tokens (tb_set_seq_lens /
+ *     tb_append_kv); the decode query sits at position len - 1.
+ *   - Selection (per query head, per sequence, L = len):
+ *       k = floor(keep_pct * L / 100); candidates C = [sink, L - window);
+ *       Sel = [0, min(sink, L)) U top_min(k,|C|)(C) U [max(L - window, 0), L)
+ *     top-k orders by (score descending, index ascending); -0.0 == +0.0;
+ *     NaN scores are outside the contract.
+ *   - A tb_ctx is not re-entrant across concurrent streams.
+ */
+#ifndef TB_H
+#define TB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TB_API __attribute__((visibility("default")))
+#else
+#define TB_API
+#endif
+
+typedef enum {
+  TB_OK = 0,
+  TB_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, negative size        */
+  TB_ERR_SHAPE = 2,         /* shape/alignment not supported                */
+  TB_ERR_CAPACITY = 3,      /* a sequence would exceed max_len              */
+  TB_ERR_WORKSPACE = 4,     /* workspace missing or too small               */
+  TB_ERR_CUDA = 5,          /* CUDA runtime / launch error                  */
+  TB_ERR_DEVICE_STATUS = 6, /* a kernel flagged an error (tb_check_status)  */
+  TB_ERR_UNSUPPORTED = 7,   /* valid request this build does not implement  */
+  TB_ERR_STATE = 8          /* layer not bound / lengths not set            */
+} tb_status;
+
+typedef enum { TB_BF16 = 0, TB_F32 = 1 } tb_dtype;
+typedef enum { TB_BUTLER = 0, TB_SOFTVOTE = 1 } tb_variant;
+typedef enum { TB_MASK_PER_HEAD = 0, TB_MASK_SHARED = 1, TB_MASK_DENSE = 2 } tb_mask_mode;
+
+/* device status word bits (tb_check_status) */
+#define TB_DEV_ERR_INDEX 0x1u     /* a gathered index was outside [0, len)    */
+#define TB_DEV_ERR_COUNT 0x2u     /* a selected-set size differed from k      */
+#define TB_DEV_ERR_TIMEOUT 0x4u   /* a bounded wait gave up                   */
+
+#define TB_MAX_BATCH 128
+#define TB_MAX_LAYERS 64
+
+typedef struct tb_config {
+  int n_layers;              /* decoder layers, 1..TB_MAX_LAYERS                          */
+  int batch;                 /* B, 1..TB_MAX_BATCH                                        */
+  int n_q_heads;             /* Hq                                                        */
+  int n_kv_heads;            /* Hkv; Hq % Hkv == 0, Hq/Hkv in {1,2,4,8}                   */
+  int head_dim;              /* D in {64, 128}                                            */
+  int d_imp;                 /* d' in {16, 32}                                            */
+  int producer_freq;         /* G >= 1 (model card "Method")                              */
+  int max_len;               /* cache capacity per sequence, multiple of 256             */
+  int kv_dtype;              /* tb_dtype of K, V, W_K, q, q_imp, out                       */
+  int keep_pct;              /* P: 100 - N of the fixed_<N>pc policy, 0..100              */
+  int sink;                  /* min_sparse_index: always-kept prefix length               */
+  int window;                /* sliding_window: always-kept recent tokens                 */
+  uint64_t dense_layer_mask; /* bit l set: layer l attends densely (layer 0 by default)   */
+  int variant;               /* tb_variant                                                */
+} tb_config;
+
+typedef struct tb_ctx tb_ctx;
+
+/* Bytes of device workspace tb_init needs for `cfg` (host-only, no CUDA call). */
+TB_API tb_status tb_workspace_size(const tb_config* cfg, size_t* bytes);
+
+/* Validate `cfg` and create a context on the current CUDA device.
+ * `workspace`: caller-owned device buffer of >= tb_workspace_size bytes,
+ * 256-byte aligned, alive until tb_destroy.  Its contents need no
+ * initialisation.  *out receives a host object freed by tb_destroy. */
+TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes, tb_ctx** out);
+
+/* Register layer `layer`'s caller-owned caches and W_K (device pointers,
+ * layouts above).  All lengths of the layer start at 0. */
+TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
+                               const void* w_k);
+
+/* Set / read the per-sequence lengths of a layer (host arrays of `batch`
+ * int32).  Used after the caller filled the caches by a prefill. */
+TB_API tb_status tb_set_seq_lens(tb_ctx* ctx, int layer, const int32_t* lens_host);
+TB_API tb_status tb_get_seq_lens(const tb_ctx* ctx, int layer, int32_t* lens_host);
+
+/* Runtime budget setters: the model card's set_token_sparsity() /
+ * min_sparse_index / sliding_window knobs ("Memory requirements"). */
+TB_API tb_status tb_set_budget(tb_ctx* ctx, int keep_pct, int sink, int window);
+
+/* a1 — model card "Method", K_imp = K . W_K, decode side.  Writes k_new and
+ * v_new ([B][Hkv][D]) at position len[b] of every sequence, computes that
+ * row's K_imp in fp32, then increments len[b] (host-side bookkeeping at
+ * enqueue time).  TB_ERR_CAPACITY if a sequence is full. */
+TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, void* stream);
+
+/* a1' — model card "Method", K_imp = K . W_K, prefill side: computes K_imp
+ * rows [start, start + count) of every (b, KV head) from the cached K.
+ * bf16 caches run on the tensor cores (tcgen05, fp32 accumulation); fp32
+ * caches use fp32 FMA (no TF32). */
+TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, void* stream);
+
+/* a2 + a3 — model card "Method": scores[b][h][t] = q_hat[b][h] . K_imp[b][g(h)][t]
+ * for t < len[b], with q_hat[b][h] = q_imp_producer[b*Hq + h][(layer-1) mod G][0][:]
+ * (fp32 FMA, no scale).  `q_imp_producer`: [(B*Hq)][G][1][d'] of producer
+ * G*floor(layer/G).  Entries t >= len[b] are left untouched. */
+TB_API tb_status tb_score(tb_ctx* ctx, int layer, const void* q_imp_producer, float* scores, void* stream);
+
+/* a4 + a5 — model card "Method" / "Memory requirements": per (b, h) row of
+ * `scores` ([B][Hq][max_len], or [B][max_len] when `rows_per_seq` is 1 for a
+ * shared ranking), selects Sel as in the header comment, with the budget of
+ * the context.  Outputs (each may be NULL, not all):
+ *   idx   [B][rows][idx_cap] ascending indices (TB_ERR_SHAPE if idx_cap is
+ *         smaller than the largest selected set),
+ *   count [B][rows] selected-set sizes,
+ *   mask  [B][rows][max_len/32] bitmask; words past ceil(len/32) untouched.
+ * Bit-exact: the choice depends only on the fp32 score values. */
+TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows_per_seq, int32_t* idx,
+                           int idx_cap, int32_t* count, uint32_t* mask, void* stream);
+
+/* a6 — exact attention over a selected set of the untouched cache:
+ * out[b][h] = sum_{t in Sel} softmax_t(q[b][h] . K[b][g(h)][t] / sqrt(D)) V[b][g(h)][t]
+ * (fp32 accumulation).  `mask_mode`: TB_MASK_PER_HEAD (mask [B][Hq][max_len/32]),
+ * TB_MASK_SHARED (mask [B][max_len/32], one set per sequence) or
+ * TB_MASK_DENSE (mask NULL: every token t < len, the layer-0 / 100 % path).
+ * `lse` (optional, [B][Hq] fp32): natural log of the softmax denominator;
+ * an empty set gives out = 0 and lse = -inf.  Split-K over token chunks with
+ * an fp32 log-sum-exp merge; each K/V row is read once per KV head. */
+TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mask_mode,
+                                void* out, float* lse, void* stream);
+
+/* a1..a6 for one layer: append, then (dense layer or 100 % budget) dense
+ * attention, else score, select and sparse attention (TB_BUTLER) or soft
+ * voting with a shared set (TB_SOFTVOTE; q_imp_producer unused).  Uses the
+ * workspace for scores, masks and split partials. */
+TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, const void* q,
+                                const void* q_imp_producer, void* out, void* stream);
+
+/* a7 — prefill rows of a consumer layer: for positions p in
+ * [row0, row0 + nrows) and every (b, h), scores the causal prefix
+ * s_p[t] = q_hat[b][h][p] . K_imp[b][g(h)][t], t <= p, and selects with
+ * L -> p + 1.  `q_imp_rows`: [(B*Hq)][G][nrows][d'] (positions row0..), slot
+ * (layer-1) mod G.  `row_masks`: [B][Hq][nrows][words_per_row] uint32 with
+ * words_per_row >= ceil((row0 + nrows)/32); every word is written.
+ * Requires len[b] >= row0 + nrows (K_imp rows present). */
+TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_rows, int row0, int nrows,
+                                   uint32_t* row_masks, int words_per_row, void* stream);
+
+/* a8 — TokenSelect soft voting: votes[b][t] = sum_h softmax_t(q[b][h] . K[b][g(h)][t] / sqrt(D))
+ * over t < len[b] (fp32), written to `votes` ([B][max_len]).  Select with
+ * tb_select(rows_per_seq = 1) and attend with TB_MASK_SHARED. */
+TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream);
+
+/* Tracing: when `events` is non-NULL, tb_decode_step records the six
+ * cudaEvent_t events[0..5] on its stream before the append, after the
+ * append, after scoring, after selection, after the split attention kernel
+ * and after the combine (points that a layer skips are recorded at the same
+ * place).  `n_events` must be 6; NULL disables tracing. */
+TB_API tb_status tb_trace_events(tb_ctx* ctx, void* const* events, int n_events);
+
+/* Number of kernel launches this context has issued (a running total). */
+TB_API tb_status tb_launch_count(const tb_ctx* ctx, uint64_t* count);
+
+/* After a synchronisation: reads and clears the device status word.
+ * Returns TB_ERR_DEVICE_STATUS if any bit was set (*flags gets them). */
+TB_API tb_status tb_check_status(tb_ctx* ctx, uint32_t* flags);
+
+TB_API const char* tb_status_string(tb_status s);
+TB_API void tb_destroy(tb_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TB_H */

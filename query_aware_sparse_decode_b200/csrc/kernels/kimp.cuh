@@ -1,0 +1,86 @@
+// butler_kimp_project, CUDA-core parts: the fused decode append (new K/V row
+// + its K_imp row) and the fp32-FMA prefill projection used for fp32 caches.
+// Model card "Meta-Llama-3.1-8B-Instruct-Butler", section "Method":
+// K_imp = K . W_K with one learned D x d' matrix per layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace tb {
+
+struct AppendParams {
+  const void* k_new;  // [B][Hkv][D]
+  const void* v_new;  // [B][Hkv][D]
+  void* k_cache;      // [B][Hkv][max_len][D]
+  void* v_cache;
+  float* kimp;        // [B][Hkv][max_len][d']
+  const void* w_k;    // [D][d']
+  int Hkv, D, dimp, max_len;
+  int pos[kMaxBatch];  // row written for sequence b (its length before the append)
+};
+
+// grid (Hkv, B), block D threads.  K_imp accumulates in fp32, d = 0..D-1.
+template <typename T>
+__global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
+  __shared__ float krow[128];
+  const int g = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const size_t src = ((size_t)b * p.Hkv + g) * p.D + d;
+  const size_t row = ((size_t)b * p.Hkv + g) * p.max_len + p.pos[b];
+  const T kv = reinterpret_cast<const T*>(p.k_new)[src];
+  reinterpret_cast<T*>(p.k_cache)[row * p.D + d] = kv;
+  reinterpret_cast<T*>(p.v_cache)[row * p.D + d] = reinterpret_cast<const T*>(p.v_new)[src];
+  krow[d] = to_f32(kv);
+  __syncthreads();
+  if (d < p.dimp) {
+    const T* w = reinterpret_cast<const T*>(p.w_k);
+    float acc = 0.f;
+    for (int e = 0; e < p.D; ++e) acc = fmaf(krow[e], to_f32(w[e * p.dimp + d]), acc);
+    p.kimp[row * p.dimp + d] = acc;
+  }
+}
+
+struct ProjectParams {
+  const void* k_cache;  // [B][Hkv][max_len][D]
+  float* kimp;          // [B][Hkv][max_len][d']
+  const void* w_k;      // [D][d']
+  int Hkv, max_len, start, count;
+};
+
+// fp32-FMA projection of rows [start, start+count) of every (b, g).
+// grid (ceil(count/32), Hkv, B), block 256: 32 rows x d' outputs per block.
+constexpr int kProjRows = 32;
+template <typename T, int D, int DIMP>
+__global__ void __launch_bounds__(256) project_fma_kernel(const ProjectParams p) {
+  constexpr int ROWS = kProjRows;
+  constexpr int OUT_PER_THREAD = ROWS * DIMP / 256;  // 4 (d'=32) or 2 (d'=16)
+  __shared__ float ks[ROWS][D + 1];
+  __shared__ float ws[D][DIMP];
+  const int g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int r0 = p.start + blockIdx.x * ROWS;
+  const size_t base = ((size_t)b * p.Hkv + g) * p.max_len;
+  const T* K = reinterpret_cast<const T*>(p.k_cache);
+  const T* W = reinterpret_cast<const T*>(p.w_k);
+  for (int i = tid; i < D * DIMP; i += 256) ws[i / DIMP][i % DIMP] = to_f32(W[i]);
+  const int rend = min(ROWS, p.start + p.count - r0);
+  for (int i = tid; i < ROWS * D; i += 256) {
+    const int r = i / D, d = i % D;
+    ks[r][d] = r < rend ? to_f32(K[(base + r0 + r) * D + d]) : 0.f;
+  }
+  __syncthreads();
+  const int r = tid / (256 / ROWS);                          // 8 threads per row
+  const int j0 = (tid % (256 / ROWS)) * OUT_PER_THREAD;
+  float acc[OUT_PER_THREAD];
+#pragma unroll
+  for (int j = 0; j < OUT_PER_THREAD; ++j) acc[j] = 0.f;
+  for (int d = 0; d < D; ++d) {
+    const float kv = ks[r][d];
+#pragma unroll
+    for (int j = 0; j < OUT_PER_THREAD; ++j) acc[j] = fmaf(kv, ws[d][j0 + j], acc[j]);
+  }
+  if (r < rend) {
+#pragma unroll
+    for (int j = 0; j < OUT_PER_THREAD; ++j) p.kimp[(base + r0 + r) * DIMP + j0 + j] = acc[j];
+  }
+}
+
+}  // namespace tb

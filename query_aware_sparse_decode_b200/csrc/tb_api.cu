@@ -1,0 +1,592 @@
+// C ABI of the TokenButler decode-step hot path (declared in include/tb.h):
+// host-side validation, workspace layout, per-layer bookkeeping and
+// stream-ordered kernel launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "kernels/attn.cuh"
+#include "kernels/common.cuh"
+#include "kernels/kimp.cuh"
+#include "kernels/score.cuh"
+#include "kernels/select.cuh"
+#include "tb.h"
+
+using namespace tb;
+
+namespace {
+
+struct LayerState {
+  void* k = nullptr;
+  void* v = nullptr;
+  float* kimp = nullptr;
+  const void* wk = nullptr;
+  bool bound = false;
+  CUtensorMap kimp_map;
+  int lens[TB_MAX_BATCH];
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t status, hist, scores, mask, part_o, part_ml, votes, total;
+  int max_splits;
+};
+
+WsLayout layout_of(const tb_config& c) {
+  WsLayout w{};
+  const size_t B = c.batch, Hq = c.n_q_heads, Lm = c.max_len;
+  w.max_splits = (int)((Lm + 255) / 256);
+  size_t off = 0;
+  w.status = off;  off += align256(256);
+  w.hist = off;    off += align256(B * Hq * kHistBins * 4);
+  w.scores = off;  off += align256(B * Hq * Lm * 4);
+  w.mask = off;    off += align256(B * Hq * (Lm / 32) * 4);
+  w.part_o = off;  off += align256(B * Hq * (size_t)w.max_splits * c.head_dim * 4);
+  w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
+  w.votes = off;   off += align256(B * Lm * 4);
+  w.total = off;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct tb_ctx {
+  tb_config cfg;
+  int device = 0;
+  int num_sms = 148;
+  char* ws = nullptr;
+  WsLayout lay;
+  uint32_t* status = nullptr;
+  uint32_t* hist = nullptr;
+  float* scores = nullptr;
+  uint32_t* mask = nullptr;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  float* votes = nullptr;
+  cudaEvent_t trace[6] = {};
+  bool tracing = false;
+  unsigned long long launches = 0;
+  LayerState layers[TB_MAX_LAYERS];
+};
+
+static void trace_point(tb_ctx* ctx, int i, cudaStream_t st) {
+  if (ctx->tracing) cudaEventRecord(ctx->trace[i], st);
+}
+
+// ------------------------------------------------------------------ validation
+static tb_status check_config(const tb_config* c) {
+  if (!c) return TB_ERR_INVALID_ARG;
+  if (c->n_layers < 1 || c->n_layers > TB_MAX_LAYERS) return TB_ERR_SHAPE;
+  if (c->batch < 1 || c->batch > TB_MAX_BATCH) return TB_ERR_SHAPE;
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) return TB_ERR_SHAPE;
+  const int gs = c->n_q_heads / c->n_kv_heads;
+  if (gs != 1 && gs != 2 && gs != 4 && gs != 8) return TB_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return TB_ERR_UNSUPPORTED;
+  if (c->d_imp != 16 && c->d_imp != 32) return TB_ERR_UNSUPPORTED;
+  if (c->producer_freq < 1) return TB_ERR_SHAPE;
+  if (c->max_len < 256 || c->max_len % 256) return TB_ERR_SHAPE;
+  if ((long long)c->batch * c->n_kv_heads * c->max_len >= (1LL << 31)) return TB_ERR_SHAPE;
+  if ((long long)c->batch * c->n_q_heads * c->max_len >= (1LL << 40)) return TB_ERR_SHAPE;
+  if (c->kv_dtype != TB_BF16 && c->kv_dtype != TB_F32) return TB_ERR_INVALID_ARG;
+  if (c->keep_pct < 0 || c->keep_pct > 100 || c->sink < 0 || c->window < 0) return TB_ERR_INVALID_ARG;
+  if (c->variant != TB_BUTLER && c->variant != TB_SOFTVOTE) return TB_ERR_INVALID_ARG;
+  return TB_OK;
+}
+
+static tb_status check_layer(const tb_ctx* ctx, int layer) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
+  if (!ctx->layers[layer].bound) return TB_ERR_STATE;
+  return TB_OK;
+}
+
+static tb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TB_OK : TB_ERR_CUDA; }
+
+static int max_len_of(const LayerState& ls, int B) {
+  int m = 0;
+  for (int b = 0; b < B; ++b) m = std::max(m, ls.lens[b]);
+  return m;
+}
+
+// ------------------------------------------------------------------ launches
+static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
+                              cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  ScoreParams p{};
+  p.q_imp = q_imp;
+  p.scores = scores;
+  p.hist = hist;
+  p.status = ctx->status;
+  p.G = c.producer_freq;
+  p.slot = ((layer - 1) % c.producer_freq + c.producer_freq) % c.producer_freq;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.max_len = c.max_len;
+  p.sink = c.sink;
+  p.window = c.window;
+  p.tile_base[0] = 0;
+  for (int b = 0; b < TB_MAX_BATCH; ++b) {
+    const int L = b < c.batch ? ls.lens[b] : 0;
+    p.lens[b] = L;
+    p.tile_base[b + 1] = p.tile_base[b] + c.n_kv_heads * ((L + kScoreTile - 1) / kScoreTile);
+  }
+  p.total_tiles = p.tile_base[TB_MAX_BATCH];
+  if (hist) {
+    const size_t n = (size_t)c.batch * c.n_q_heads * kHistBins;
+    zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(hist, n);
+    ++ctx->launches;
+  }
+  if (p.total_tiles == 0) return cuda_status(cudaGetLastError());
+  const int grid = std::min(p.total_tiles, ctx->num_sms);
+  const int gs = c.n_q_heads / c.n_kv_heads;
+  const size_t smem = 1024 + (size_t)kScoreStages * kScoreTile * c.d_imp * 4 + kScoreStages * 8 +
+                      (hist ? (size_t)gs * kHistBins * 4 : 0);
+#define TB_SCORE_CASE(T, DI, GSV)                                                                          \
+  if (c.d_imp == DI && gs == GSV) {                                                                        \
+    if (hist) {                                                                                            \
+      auto k = score_kernel<T, DI, GSV, true>;                                                             \
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
+      k<<<grid, kScoreTile, smem, st>>>(ls.kimp_map, p);                                                   \
+      ++ctx->launches;                                                                                     \
+    } else {                                                                                               \
+      auto k = score_kernel<T, DI, GSV, false>;                                                            \
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
+      k<<<grid, kScoreTile, smem, st>>>(ls.kimp_map, p);                                                   \
+      ++ctx->launches;                                                                                     \
+    }                                                                                                      \
+    return cuda_status(cudaGetLastError());                                                                \
+  }
+  if (c.kv_dtype == TB_BF16) {
+    TB_SCORE_CASE(__nv_bfloat16, 32, 4)
+    TB_SCORE_CASE(__nv_bfloat16, 32, 2)
+    TB_SCORE_CASE(__nv_bfloat16, 32, 1)
+    TB_SCORE_CASE(__nv_bfloat16, 16, 4)
+    TB_SCORE_CASE(__nv_bfloat16, 16, 2)
+    TB_SCORE_CASE(__nv_bfloat16, 16, 1)
+  } else {
+    TB_SCORE_CASE(float, 32, 4)
+    TB_SCORE_CASE(float, 32, 2)
+    TB_SCORE_CASE(float, 32, 1)
+    TB_SCORE_CASE(float, 16, 4)
+    TB_SCORE_CASE(float, 16, 2)
+    TB_SCORE_CASE(float, 16, 1)
+  }
+#undef TB_SCORE_CASE
+  return TB_ERR_UNSUPPORTED;
+}
+
+static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, const uint32_t* hist1, int rows,
+                               int32_t* idx, int idx_cap, int32_t* count, uint32_t* mask, cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  SelectParams p{};
+  p.scores = scores;
+  p.hist1 = hist1;
+  p.idx = idx;
+  p.count = count;
+  p.mask = mask;
+  p.status = ctx->status;
+  p.row_stride = c.max_len;
+  p.rows_per_seq = rows;
+  p.idx_cap = idx_cap;
+  p.mask_words = c.max_len / 32;
+  p.keep_pct = c.keep_pct;
+  p.sink = c.sink;
+  p.window = c.window;
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
+  dim3 grid(rows, c.batch);
+  select_kernel<<<grid, kSelThreads, 0, st>>>(p);
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
+static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mode, void* out,
+                             float* lse, cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  const int maxL = max_len_of(ls, c.batch);
+  const int gs = c.n_q_heads / c.n_kv_heads;
+  AttnParams p{};
+  p.k_cache = ls.k;
+  p.v_cache = ls.v;
+  p.q = q;
+  p.mask = mask;
+  p.part_o = ctx->part_o;
+  p.part_ml = ctx->part_ml;
+  p.status = ctx->status;
+  p.mask_mode = mode;
+  p.mask_words = c.max_len / 32;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.max_len = c.max_len;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
+  // chunking: about four CTAs per SM over the whole grid
+  const int groups = c.batch * c.n_kv_heads;
+  const int want_split = std::max(1, (4 * ctx->num_sms + groups - 1) / groups);
+  int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
+  chunk = std::min(kAttnMaxChunk, std::max(256, (chunk + 255) / 256 * 256));
+  p.chunk = chunk;
+  p.nsplit = std::max(1, (maxL + chunk - 1) / chunk);
+  if (p.nsplit > ctx->lay.max_splits) return TB_ERR_WORKSPACE;
+  if (maxL > 0) {
+    dim3 grid(p.nsplit, c.n_kv_heads, c.batch);
+#define TB_ATTN_CASE(DV, GSV)                                                                               \
+  if (c.head_dim == DV && gs == GSV) {                                                                      \
+    if (c.kv_dtype == TB_BF16) {                                                                            \
+      auto k = attn_bf16_kernel<DV, GSV>;                                                                   \
+      const int smem = attn_bf16_smem_bytes<DV>();                                                          \
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
+      k<<<grid, kAttnThreads, smem, st>>>(p);                                                               \
+    } else {                                                                                                \
+      auto k = attn_f32_kernel<DV, GSV>;                                                                    \
+      const int smem = attn_f32_smem_bytes<DV>();                                                           \
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
+      k<<<grid, kAttnThreads, smem, st>>>(p);                                                               \
+    }                                                                                                       \
+  } else
+    TB_ATTN_CASE(128, 4) TB_ATTN_CASE(128, 2) TB_ATTN_CASE(128, 1) TB_ATTN_CASE(128, 8)
+    TB_ATTN_CASE(64, 4) TB_ATTN_CASE(64, 2) TB_ATTN_CASE(64, 1) TB_ATTN_CASE(64, 8)
+    return TB_ERR_UNSUPPORTED;
+#undef TB_ATTN_CASE
+    ++ctx->launches;
+    tb_status s = cuda_status(cudaGetLastError());
+    if (s != TB_OK) return s;
+  }
+  trace_point(ctx, 4, st);
+  CombineParams cp{};
+  cp.part_o = ctx->part_o;
+  cp.part_ml = ctx->part_ml;
+  cp.out = out;
+  cp.lse = lse;
+  cp.Hq = c.n_q_heads;
+  cp.D = c.head_dim;
+  cp.chunk = chunk;
+  cp.nsplit = p.nsplit;
+  for (int b = 0; b < c.batch; ++b) cp.lens[b] = ls.lens[b];
+  dim3 grid(c.n_q_heads, c.batch);
+  if (c.kv_dtype == TB_BF16)
+    combine_kernel<__nv_bfloat16><<<grid, c.head_dim, 0, st>>>(cp);
+  else
+    combine_kernel<float><<<grid, c.head_dim, 0, st>>>(cp);
+  ++ctx->launches;
+  trace_point(ctx, 5, st);
+  return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------------------ C ABI
+extern "C" {
+
+TB_API tb_status tb_workspace_size(const tb_config* cfg, size_t* bytes) {
+  if (!bytes) return TB_ERR_INVALID_ARG;
+  tb_status s = check_config(cfg);
+  if (s != TB_OK) return s;
+  *bytes = layout_of(*cfg).total;
+  return TB_OK;
+}
+
+TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes, tb_ctx** out) {
+  if (!out) return TB_ERR_INVALID_ARG;
+  *out = nullptr;
+  tb_status s = check_config(cfg);
+  if (s != TB_OK) return s;
+  const WsLayout lay = layout_of(*cfg);
+  if (!workspace || ws_bytes < lay.total) return TB_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return TB_ERR_WORKSPACE;
+  tb_ctx* ctx = new (std::nothrow) tb_ctx();
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  ctx->cfg = *cfg;
+  ctx->lay = lay;
+  if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
+    delete ctx;
+    return TB_ERR_CUDA;
+  }
+  ctx->ws = static_cast<char*>(workspace);
+  ctx->status = reinterpret_cast<uint32_t*>(ctx->ws + lay.status);
+  ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
+  ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
+  ctx->mask = reinterpret_cast<uint32_t*>(ctx->ws + lay.mask);
+  ctx->part_o = reinterpret_cast<float*>(ctx->ws + lay.part_o);
+  ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
+  ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
+  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
+    delete ctx;
+    return TB_ERR_CUDA;
+  }
+  *out = ctx;
+  return TB_OK;
+}
+
+TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
+                               const void* w_k) {
+  if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
+  if (!k_cache || !v_cache || !kimp_cache || !w_k) return TB_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kimp_cache) || !aligned16(w_k)) return TB_ERR_SHAPE;
+  const tb_config& c = ctx->cfg;
+  LayerState& ls = ctx->layers[layer];
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return TB_ERR_CUDA;
+  cuuint64_t gdim[2] = {(cuuint64_t)c.d_imp, (cuuint64_t)c.batch * c.n_kv_heads * c.max_len};
+  cuuint64_t gstride[1] = {(cuuint64_t)c.d_imp * 4};
+  cuuint32_t box[2] = {(cuuint32_t)c.d_imp, (cuuint32_t)kScoreTile};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(&ls.kimp_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, kimp_cache, gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   c.d_imp == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return TB_ERR_CUDA;
+  ls.k = k_cache;
+  ls.v = v_cache;
+  ls.kimp = kimp_cache;
+  ls.wk = w_k;
+  std::memset(ls.lens, 0, sizeof(ls.lens));
+  ls.bound = true;
+  return TB_OK;
+}
+
+TB_API tb_status tb_set_seq_lens(tb_ctx* ctx, int layer, const int32_t* lens_host) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!lens_host) return TB_ERR_INVALID_ARG;
+  for (int b = 0; b < ctx->cfg.batch; ++b)
+    if (lens_host[b] < 0 || lens_host[b] > ctx->cfg.max_len) return TB_ERR_CAPACITY;
+  for (int b = 0; b < ctx->cfg.batch; ++b) ctx->layers[layer].lens[b] = lens_host[b];
+  return TB_OK;
+}
+
+TB_API tb_status tb_get_seq_lens(const tb_ctx* ctx, int layer, int32_t* lens_host) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!lens_host) return TB_ERR_INVALID_ARG;
+  for (int b = 0; b < ctx->cfg.batch; ++b) lens_host[b] = ctx->layers[layer].lens[b];
+  return TB_OK;
+}
+
+TB_API tb_status tb_set_budget(tb_ctx* ctx, int keep_pct, int sink, int window) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  if (keep_pct < 0 || keep_pct > 100 || sink < 0 || window < 0) return TB_ERR_INVALID_ARG;
+  ctx->cfg.keep_pct = keep_pct;
+  ctx->cfg.sink = sink;
+  ctx->cfg.window = window;
+  return TB_OK;
+}
+
+TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!k_new || !v_new) return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  LayerState& ls = ctx->layers[layer];
+  for (int b = 0; b < c.batch; ++b)
+    if (ls.lens[b] >= c.max_len) return TB_ERR_CAPACITY;
+  AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_cache = ls.k;
+  p.v_cache = ls.v;
+  p.kimp = ls.kimp;
+  p.w_k = ls.wk;
+  p.Hkv = c.n_kv_heads;
+  p.D = c.head_dim;
+  p.dimp = c.d_imp;
+  p.max_len = c.max_len;
+  for (int b = 0; b < c.batch; ++b) p.pos[b] = ls.lens[b];
+  dim3 grid(c.n_kv_heads, c.batch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c.kv_dtype == TB_BF16)
+    append_kernel<__nv_bfloat16><<<grid, c.head_dim, 0, st>>>(p);
+  else
+    append_kernel<float><<<grid, c.head_dim, 0, st>>>(p);
+  ++ctx->launches;
+  s = cuda_status(cudaGetLastError());
+  if (s != TB_OK) return s;
+  for (int b = 0; b < c.batch; ++b) ls.lens[b] += 1;
+  return TB_OK;
+}
+
+TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  const tb_config& c = ctx->cfg;
+  if (start < 0 || count < 0 || (long long)start + count > c.max_len) return TB_ERR_CAPACITY;
+  if (count == 0) return TB_OK;
+  const LayerState& ls = ctx->layers[layer];
+  ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count};
+  dim3 grid((count + kProjRows - 1) / kProjRows, c.n_kv_heads, c.batch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define TB_PROJ_CASE(T, DV, DI) \
+  if (c.head_dim == DV && c.d_imp == DI) project_fma_kernel<T, DV, DI><<<grid, 256, 0, st>>>(p); else
+  if (c.kv_dtype == TB_BF16) {
+    TB_PROJ_CASE(__nv_bfloat16, 128, 32) TB_PROJ_CASE(__nv_bfloat16, 128, 16) TB_PROJ_CASE(__nv_bfloat16, 64, 32)
+    TB_PROJ_CASE(__nv_bfloat16, 64, 16) return TB_ERR_UNSUPPORTED;
+  } else {
+    TB_PROJ_CASE(float, 128, 32) TB_PROJ_CASE(float, 128, 16) TB_PROJ_CASE(float, 64, 32)
+    TB_PROJ_CASE(float, 64, 16) return TB_ERR_UNSUPPORTED;
+  }
+#undef TB_PROJ_CASE
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
+TB_API tb_status tb_score(tb_ctx* ctx, int layer, const void* q_imp_producer, float* scores, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!q_imp_producer || !scores) return TB_ERR_INVALID_ARG;
+  if (!aligned16(scores)) return TB_ERR_SHAPE;
+  return launch_score(ctx, layer, q_imp_producer, scores, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows_per_seq, int32_t* idx,
+                           int idx_cap, int32_t* count, uint32_t* mask, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  const tb_config& c = ctx->cfg;
+  if (!scores || (!idx && !count && !mask)) return TB_ERR_INVALID_ARG;
+  if (rows_per_seq != c.n_q_heads && rows_per_seq != 1) return TB_ERR_SHAPE;
+  if (!aligned16(scores)) return TB_ERR_SHAPE;
+  if (idx) {
+    const LayerState& ls = ctx->layers[layer];
+    for (int b = 0; b < c.batch; ++b) {
+      const long long L = ls.lens[b];
+      const long long nc = std::max(0LL, L - c.window - c.sink);
+      const long long k = std::min((long long)c.keep_pct * L / 100, nc);
+      const long long sink_n = std::min<long long>(c.sink, L);
+      const long long win_lo = std::max(L - c.window, sink_n);
+      if (sink_n + (L - win_lo) + k > idx_cap) return TB_ERR_SHAPE;
+    }
+  }
+  return launch_select(ctx, layer, scores, nullptr, rows_per_seq, idx, idx_cap, count, mask,
+                       static_cast<cudaStream_t>(stream));
+}
+
+TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mask_mode,
+                                void* out, float* lse, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!q || !out) return TB_ERR_INVALID_ARG;
+  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE)
+    return TB_ERR_INVALID_ARG;
+  if (mask_mode != TB_MASK_DENSE && !mask) return TB_ERR_INVALID_ARG;
+  if (!aligned16(q)) return TB_ERR_SHAPE;
+  return launch_attn(ctx, layer, q, mask, mask_mode, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, const void* q,
+                                const void* q_imp_producer, void* out, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  const tb_config& c = ctx->cfg;
+  if (!k_new || !v_new || !q || !out) return TB_ERR_INVALID_ARG;
+  const bool dense = ((c.dense_layer_mask >> layer) & 1ull) || c.keep_pct >= 100;
+  if (!dense && c.variant == TB_BUTLER && !q_imp_producer) return TB_ERR_INVALID_ARG;
+  if (!aligned16(q)) return TB_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  trace_point(ctx, 0, st);
+  s = tb_append_kv(ctx, layer, k_new, v_new, stream);
+  if (s != TB_OK) return s;
+  trace_point(ctx, 1, st);
+  if (dense) {
+    trace_point(ctx, 2, st);
+    trace_point(ctx, 3, st);
+    return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
+  }
+  if (c.variant == TB_SOFTVOTE) return TB_ERR_UNSUPPORTED;
+  s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
+  if (s != TB_OK) return s;
+  trace_point(ctx, 2, st);
+  s = launch_select(ctx, layer, ctx->scores, ctx->hist, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+  if (s != TB_OK) return s;
+  trace_point(ctx, 3, st);
+  return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
+}
+
+TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_rows, int row0, int nrows,
+                                   uint32_t* row_masks, int words_per_row, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  (void)q_imp_rows; (void)row0; (void)nrows; (void)row_masks; (void)words_per_row; (void)stream;
+  return TB_ERR_UNSUPPORTED;
+}
+
+TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  (void)q; (void)votes; (void)stream;
+  return TB_ERR_UNSUPPORTED;
+}
+
+TB_API tb_status tb_trace_events(tb_ctx* ctx, void* const* events, int n_events) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  if (!events) {
+    ctx->tracing = false;
+    return TB_OK;
+  }
+  if (n_events != 6) return TB_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i) {
+    if (!events[i]) return TB_ERR_INVALID_ARG;
+    ctx->trace[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  ctx->tracing = true;
+  return TB_OK;
+}
+
+TB_API tb_status tb_launch_count(const tb_ctx* ctx, uint64_t* count) {
+  if (!ctx || !count) return TB_ERR_INVALID_ARG;
+  *count = ctx->launches;
+  return TB_OK;
+}
+
+TB_API tb_status tb_check_status(tb_ctx* ctx, uint32_t* flags) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ctx->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return TB_ERR_CUDA;
+  if (v && cudaMemset(ctx->status, 0, sizeof(v)) != cudaSuccess) return TB_ERR_CUDA;
+  if (flags) *flags = v;
+  return v ? TB_ERR_DEVICE_STATUS : TB_OK;
+}
+
+TB_API const char* tb_status_string(tb_status s) {
+  switch (s) {
+    case TB_OK: return "ok";
+    case TB_ERR_INVALID_ARG: return "invalid argument";
+    case TB_ERR_SHAPE: return "unsupported shape or alignment";
+    case TB_ERR_CAPACITY: return "sequence length exceeds cache capacity";
+    case TB_ERR_WORKSPACE: return "workspace missing or too small";
+    case TB_ERR_CUDA: return "CUDA error";
+    case TB_ERR_DEVICE_STATUS: return "a kernel reported an error";
+    case TB_ERR_UNSUPPORTED: return "not supported by this build";
+    case TB_ERR_STATE: return "layer not bound";
+  }
+  return "unknown status";
+}
+
+TB_API void tb_destroy(tb_ctx* ctx) { delete ctx; }
+
+}  // extern "C"

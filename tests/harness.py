@@ -1,0 +1,134 @@
+"""Shared set-up for the GPU parity tests: seeded inputs (from the generator
+module), device buffers, a bound context, and comparison helpers.  Expected
+values come only from the oracle."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from oracle import tokenbutler as O
+from query_aware_sparse_decode_b200 import synth as S
+from query_aware_sparse_decode_b200 import tb as TB
+
+
+def tdtype(wl):
+    return torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+
+
+def to_dev(arr: np.ndarray, wl) -> torch.Tensor:
+    if wl.dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).cuda()
+
+
+def round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+@dataclass
+class LayerData:
+    layer: int
+    W: np.ndarray          # [D][d'] float64
+    qimp: np.ndarray       # producer tensor [(B*Hq)][G][1][d'] float64
+    qhat: np.ndarray | None  # consumer queries [B][Hq][d'] float64 (None for dense layers)
+    q: np.ndarray          # [B][Hq][D] float64
+    K: np.ndarray          # [B][Hkv][Lfill][D] float64
+    V: np.ndarray
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    kimp: torch.Tensor
+    w_k: torch.Tensor
+    q_imp_dev: torch.Tensor
+    q_dev: torch.Tensor
+
+
+def config_of(wl, max_len=None, keep_pct=None, variant=TB.TB_BUTLER) -> TB.Config:
+    return TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G,
+                          max_len if max_len is not None else round_up(wl.max_len + 1, 256), wl.dtype,
+                          wl.keep_pct if keep_pct is None else keep_pct, wl.sink, wl.window,
+                          dense_layers=wl.dense_layers, variant=variant)
+
+
+def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerData:
+    """Generates layer `layer` on the host, uploads it and binds it with the
+    given per-sequence lengths (rows [0, len[b]) filled)."""
+    B, Hq, Hkv, D, dimp, G = wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G
+    Lmax = ctx.cfg.max_len
+    Lfill = max(lens)
+    W_raw = S.w_k(wl, layer)
+    W = S.widen(W_raw, wl.dtype)
+    prod = O.producer_of(layer, G)
+    qimp_raw = S.q_imp(wl, prod, step)
+    qimp = S.widen(qimp_raw, wl.dtype)
+    dense = layer in wl.dense_layers
+    qhat = None if dense else O.importance_queries(qimp, layer, G, B, Hq)
+    delta = None if dense or wl.plant == "none" else S.plant_delta(W, qhat, Hkv)
+    K_raw = S.kv_cache_host(wl, layer, S.K_CACHE, 0, Lfill, delta).reshape(B, Hkv, Lfill, D)
+    V_raw = S.kv_cache_host(wl, layer, S.V_CACHE, 0, Lfill).reshape(B, Hkv, Lfill, D)
+    q_raw = S.query(wl, layer, step)
+    k_cache = torch.zeros((B, Hkv, Lmax, D), dtype=tdtype(wl), device="cuda")
+    v_cache = torch.zeros_like(k_cache)
+    k_cache[:, :, :Lfill] = to_dev(K_raw, wl)
+    v_cache[:, :, :Lfill] = to_dev(V_raw, wl)
+    kimp = torch.zeros((B, Hkv, Lmax, dimp), dtype=torch.float32, device="cuda")
+    w_k = to_dev(W_raw, wl)
+    ctx.bind_layer(layer, k_cache, v_cache, kimp, w_k)
+    ctx.set_seq_lens(layer, lens)
+    return LayerData(layer, W, qimp, qhat, S.widen(q_raw, wl.dtype), S.widen(K_raw, wl.dtype),
+                     S.widen(V_raw, wl.dtype), k_cache, v_cache, kimp, w_k, to_dev(qimp_raw, wl), to_dev(q_raw, wl))
+
+
+def mask_from_sets(sets: dict, B: int, rows: int, Lmax: int) -> torch.Tensor:
+    """uint32-as-int32 bitmask [B][rows][Lmax/32] from {(b, r): indices}."""
+    m = np.zeros((B, rows, Lmax // 32), dtype=np.uint32)
+    for (b, r), idx in sets.items():
+        idx = np.asarray(idx, dtype=np.int64)
+        np.bitwise_or.at(m[b, r], idx // 32, (np.uint32(1) << (idx % 32).astype(np.uint32)))
+    return torch.from_numpy(m.view(np.int32)).cuda()
+
+
+def sets_from_mask(mask: torch.Tensor, lens) -> dict:
+    m = mask.cpu().numpy().view(np.uint32)
+    out = {}
+    B, rows, _ = m.shape
+    for b in range(B):
+        L = lens[b]
+        for r in range(rows):
+            bits = np.unpackbits(m[b, r].view(np.uint8), bitorder="little")[:L]
+            out[b, r] = np.nonzero(bits)[0]
+    return out
+
+
+def assert_close_rows(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "") -> float:
+    """fp32: max-abs <= 2e-3; bf16: max-abs <= 1e-2 * max|ref| per row.
+    Returns the worst ratio error / allowed."""
+    err = np.abs(got - ref)
+    if dtype == "f32":
+        allowed = 2e-3
+        worst = float(err.max() / allowed)
+    else:
+        allowed = 1e-2 * np.maximum(np.abs(ref).max(axis=-1, keepdims=True), 1e-30)
+        worst = float((err / allowed).max())
+    assert worst <= 1.0, f"{what}: error {worst:.3f} x tolerance"
+    return worst
+
+
+def tie_band_ok(gpu_set, ref_set, scores64, L, keep_pct, sink, window) -> bool:
+    """Selected sets agree except on tokens whose oracle score lies within
+    1e-4 * max|score| of the k-th candidate score."""
+    g, r = set(np.asarray(gpu_set).tolist()), set(np.asarray(ref_set).tolist())
+    if g == r:
+        return True
+    if len(g) != len(r):
+        return False
+    cand = np.arange(sink, L - window) if L - window > sink else np.zeros(0, np.int64)
+    k = min(O.token_budget(L, keep_pct), cand.size)
+    if k == 0:
+        return False
+    sc = scores64[cand]
+    kth = np.sort(sc)[::-1][k - 1]
+    band = 1e-4 * np.abs(scores64[:L]).max()
+    return all(abs(scores64[t] - kth) <= band for t in g ^ r)

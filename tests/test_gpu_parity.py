@@ -1,0 +1,260 @@
+"""GPU parity of the CUDA hot path (through the C ABI) against the fp64 oracle.
+
+Criteria: K_imp within fp32 dot-product rounding; scores max-rel 1e-5;
+selection bit-exact on identical fp32 scores; end-to-end selected sets equal
+except for tokens within 1e-4 * max|score| of the k-th score; attention
+max-abs 2e-3 (fp32) / 1e-2 relative (bf16)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tokenbutler as O
+from query_aware_sparse_decode_b200 import synth as S
+from query_aware_sparse_decode_b200 import tb as TB
+
+from harness import (assert_close_rows, config_of, make_layer, mask_from_sets, round_up, sets_from_mask, tdtype,
+                     tie_band_ok, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+SMALL_BF16 = S.Workload("small_bf16", n_layers=1, B=2, Hq=8, Hkv=2, D=128, d_imp=32, G=1, L=3000, dtype="bf16",
+                        keep_pct=30, sink=16, window=64)
+SMALL_D64 = S.Workload("small_bf16_d64", n_layers=1, B=1, Hq=8, Hkv=4, D=64, d_imp=16, G=1, L=1500, dtype="bf16",
+                       keep_pct=50, sink=4, window=16)
+RAGGED = S.Workload("ragged_bf16", n_layers=1, B=4, Hq=8, Hkv=2, D=128, d_imp=32, G=1, L=2300, dtype="bf16",
+                    keep_pct=30, sink=16, window=64, lens=(2300, 1, 70, 1027))
+
+
+def _kimp_tol(K, W):
+    return 8e-6 * (np.abs(K) @ np.abs(W)) + 1e-30
+
+
+# --------------------------------------------------------------------------- a1'
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
+def test_project_kimp_matches_fp64(wl):
+    ctx = TB.Context(config_of(wl))
+    lens = wl.seq_lens
+    ld = make_layer(ctx, wl, 0, lens)
+    ctx.project_kimp(0, 0, max(lens))
+    torch.cuda.synchronize()
+    got = ld.kimp.cpu().numpy().astype(np.float64)
+    for b, L in enumerate(lens):
+        ref = O.project_keys(ld.K[b, :, :L], ld.W)
+        assert np.all(np.abs(got[b, :, :L] - ref) <= _kimp_tol(ld.K[b, :, :L], ld.W))
+    assert ctx.check_status() == 0
+
+
+# --------------------------------------------------------------------------- a1
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16], ids=lambda w: w.name)
+def test_append_writes_rows_and_kimp(wl):
+    ctx = TB.Context(config_of(wl))
+    lens = wl.seq_lens
+    ld = make_layer(ctx, wl, 0, lens)
+    k_raw, v_raw = S.kv_new(wl, 0, step=3)
+    ctx.append_kv(0, to_dev(k_raw, wl), to_dev(v_raw, wl))
+    torch.cuda.synchronize()
+    assert ctx.seq_lens(0) == [L + 1 for L in lens]
+    k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
+    kc = ld.k_cache.float().cpu().numpy()
+    vc = ld.v_cache.float().cpu().numpy()
+    kimp = ld.kimp.cpu().numpy().astype(np.float64)
+    for b, L in enumerate(lens):
+        assert np.array_equal(kc[b, :, L], k64[b]) and np.array_equal(vc[b, :, L], v64[b])
+        ref = O.project_keys(k64[b], ld.W)
+        assert np.all(np.abs(kimp[b, :, L] - ref) <= _kimp_tol(k64[b], ld.W))
+
+
+# --------------------------------------------------------------------------- a2 + a3
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED,
+                                S.TINY_F32.with_(name="tiny_G4_layer6", n_layers=8, G=4)], ids=lambda w: w.name)
+def test_score_matches_oracle(wl):
+    ctx = TB.Context(config_of(wl))
+    lens = wl.seq_lens
+    layer = wl.n_layers - 2 if wl.n_layers > 1 else 0
+    ld = make_layer(ctx, wl, layer, lens)
+    ctx.project_kimp(layer, 0, max(lens))
+    scores = torch.full((wl.B, wl.Hq, ctx.cfg.max_len), float("nan"), device="cuda")
+    ctx.score(layer, ld.q_imp_dev, scores)
+    torch.cuda.synchronize()
+    s = scores.cpu().numpy().astype(np.float64)
+    gs = wl.Hq // wl.Hkv
+    for b, L in enumerate(lens):
+        for h in range(wl.Hq):
+            ref = O.importance_scores(ld.qhat[b, h], O.project_keys(ld.K[b, h // gs, :L], ld.W))
+            if L:
+                assert np.max(np.abs(s[b, h, :L] - ref)) <= 1e-5 * np.max(np.abs(ref))
+            assert np.all(np.isnan(s[b, h, L:]))      # entries past len are untouched
+
+
+# --------------------------------------------------------------------------- a4 + a5
+def _synthetic_scores(B, rows, Lmax, quant, seed_layer):
+    x = S.fill_host(20, seed_layer, 0, B * rows, 0, Lmax, 1, "f32").reshape(B, rows, Lmax)
+    if quant:
+        x = (np.round(x * quant) / quant).astype(np.float32)   # many exact ties
+        x[..., ::7] = np.float32(-0.0)                          # -0.0 vs +0.0 ties
+        x[..., 3::11] = np.float32(0.0)
+    return x
+
+
+@pytest.mark.parametrize("case", [
+    dict(lens=(512,), keep=50, sink=4, window=16, quant=0),
+    dict(lens=(3000, 2999), keep=30, sink=16, window=64, quant=4),
+    dict(lens=(4096, 100, 80, 1), keep=50, sink=16, window=64, quant=2),
+    dict(lens=(9000,), keep=10, sink=0, window=0, quant=1),
+    dict(lens=(777, 0), keep=100, sink=3, window=5, quant=8),
+    dict(lens=(20000,), keep=0, sink=16, window=64, quant=0),
+    dict(lens=(70000,), keep=30, sink=16, window=64, quant=16),
+], ids=lambda c: f"L{c['lens']}-k{c['keep']}-q{c['quant']}")
+def test_select_bit_exact_on_identical_scores(case):
+    lens, rows = case["lens"], 4
+    B = len(lens)
+    wl = S.Workload("sel", n_layers=1, B=B, Hq=rows, Hkv=1, D=64, d_imp=16, G=1, L=max(lens), dtype="f32",
+                    keep_pct=case["keep"], sink=case["sink"], window=case["window"], plant="none", lens=lens)
+    cfg = config_of(wl)
+    Lmax = cfg.max_len
+    ctx = TB.Context(cfg)
+    dummy = torch.zeros((B, 1, Lmax, 64), device="cuda")
+    ctx.bind_layer(0, dummy, dummy.clone(), torch.zeros((B, 1, Lmax, 16), device="cuda"),
+                   torch.zeros((64, 16), device="cuda"))
+    ctx.set_seq_lens(0, lens)
+    sc = _synthetic_scores(B, rows, Lmax, case["quant"], len(lens) * 100 + case["keep"])
+    cap = max(lens) if max(lens) else 1
+    idx = torch.full((B, rows, cap), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B, rows), -1, dtype=torch.int32, device="cuda")
+    mask = torch.zeros((B, rows, Lmax // 32), dtype=torch.int32, device="cuda")
+    ctx.select(0, torch.from_numpy(sc).cuda(), rows, idx=idx, count=cnt, mask=mask)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    got_sets = sets_from_mask(mask, lens)
+    for b, L in enumerate(lens):
+        for r in range(rows):
+            ref = O.select_tokens(sc[b, r].astype(np.float64), L, case["keep"], case["sink"], case["window"])
+            assert cnt[b, r] == ref.size
+            assert np.array_equal(idx[b, r, :ref.size], ref)
+            assert np.array_equal(got_sets[b, r], ref)
+
+
+# --------------------------------------------------------------------------- a6
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
+def test_sparse_attn_on_oracle_sets(wl):
+    ctx = TB.Context(config_of(wl))
+    lens = wl.seq_lens
+    ld = make_layer(ctx, wl, 0, lens)
+    gs = wl.Hq // wl.Hkv
+    scale = 1.0 / math.sqrt(wl.D)
+    sets = {}
+    for b, L in enumerate(lens):
+        for h in range(wl.Hq):
+            s = O.importance_scores(ld.qhat[b, h], O.project_keys(ld.K[b, h // gs, :L], ld.W))
+            sets[b, h] = O.select_tokens(s, L, wl.keep_pct, wl.sink, wl.window)
+    mask = mask_from_sets(sets, wl.B, wl.Hq, ctx.cfg.max_len)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    ctx.sparse_attn(0, ld.q_dev, mask, TB.TB_MASK_PER_HEAD, out, lse)
+    out_d = torch.empty_like(out)
+    lse_d = torch.empty_like(lse)
+    ctx.sparse_attn(0, ld.q_dev, None, TB.TB_MASK_DENSE, out_d, lse_d)
+    torch.cuda.synchronize()
+    o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+    od, ldn = out_d.float().cpu().numpy(), lse_d.cpu().numpy()
+    for b, L in enumerate(lens):
+        for h in range(wl.Hq):
+            ref, ref_lse = O.attend(ld.q[b, h], ld.K[b, h // gs, :L], ld.V[b, h // gs, :L], sets[b, h], scale)
+            assert_close_rows(o[b, h][None], ref[None], wl.dtype, f"sparse b{b} h{h}")
+            assert abs(l[b, h] - ref_lse) <= 1e-3 * max(1.0, abs(ref_lse))
+            refd, refd_lse = O.attend(ld.q[b, h], ld.K[b, h // gs, :L], ld.V[b, h // gs, :L], np.arange(L), scale)
+            assert_close_rows(od[b, h][None], refd[None], wl.dtype, f"dense b{b} h{h}")
+            assert abs(ldn[b, h] - refd_lse) <= 1e-3 * max(1.0, abs(refd_lse))
+
+
+def test_sparse_attn_empty_set_and_single_token():
+    wl = SMALL_BF16.with_(B=1)
+    ctx = TB.Context(config_of(wl))
+    ld = make_layer(ctx, wl, 0, (wl.L,))
+    sets = {(0, h): (np.array([], np.int64) if h % 2 == 0 else np.array([1234])) for h in range(wl.Hq)}
+    out = torch.empty((1, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, wl.Hq), device="cuda")
+    ctx.sparse_attn(0, ld.q_dev, mask_from_sets(sets, 1, wl.Hq, ctx.cfg.max_len), TB.TB_MASK_PER_HEAD, out, lse)
+    torch.cuda.synchronize()
+    o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(wl.Hq):
+        if h % 2 == 0:
+            assert np.all(o[0, h] == 0) and l[0, h] == -np.inf
+        else:
+            assert np.array_equal(o[0, h], ld.V[0, h // 4, 1234])   # bf16 value row, exact
+
+
+# --------------------------------------------------------------------------- a1..a6 end to end
+def _decode_e2e(wl, layer=0):
+    cfg = config_of(wl)
+    ctx = TB.Context(cfg)
+    lens0 = [L - 1 for L in wl.seq_lens]
+    ld = make_layer(ctx, wl, layer, lens0)
+    ctx.project_kimp(layer, 0, max(lens0))
+    k_raw, v_raw = S.kv_new(wl, layer)
+    k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+    ctx.decode_step(layer, k_dev, v_dev, ld.q_dev, ld.q_imp_dev, out)
+    # the same step through the separate calls, keeping the selection
+    lens = ctx.seq_lens(layer)
+    scores = torch.empty((wl.B, wl.Hq, cfg.max_len), device="cuda")
+    mask = torch.zeros((wl.B, wl.Hq, cfg.max_len // 32), dtype=torch.int32, device="cuda")
+    out2 = torch.empty_like(out)
+    dense = layer in wl.dense_layers or wl.keep_pct == 100
+    if dense:
+        ctx.sparse_attn(layer, ld.q_dev, None, TB.TB_MASK_DENSE, out2)
+    else:
+        ctx.score(layer, ld.q_imp_dev, scores)
+        ctx.select(layer, scores, wl.Hq, mask=mask)
+        ctx.sparse_attn(layer, ld.q_dev, mask, TB.TB_MASK_PER_HEAD, out2)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    assert torch.equal(out, out2)
+    # oracle on the full cache (prefill rows + the appended token)
+    K = np.concatenate([ld.K, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
+    V = np.concatenate([ld.V, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
+    k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
+    for b, L in enumerate(lens):
+        K[b, :, L - 1], V[b, :, L - 1] = k64[b], v64[b]
+    sel, ref, _, sc = O.decode_layer(ld.q, K, V, ld.W, ld.qimp, layer, wl.G, lens, wl.keep_pct, wl.sink,
+                                     wl.window, dense=dense)
+    o = out.float().cpu().numpy()
+    got_sets = None if dense else sets_from_mask(mask, lens)
+    mism = 0
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            if not dense:
+                assert tie_band_ok(got_sets[b, h], sel[b, h], sc[b, h], lens[b], wl.keep_pct, wl.sink, wl.window)
+                if not np.array_equal(got_sets[b, h], sel[b, h]):
+                    mism += 1
+                    continue   # output compared only where the two sets agree
+            assert_close_rows(o[b, h][None], ref[b, h][None], wl.dtype, f"b{b} h{h}")
+    assert mism <= max(1, wl.B * wl.Hq // 20)
+    return ctx, sel, got_sets
+
+
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
+def test_decode_step_end_to_end(wl):
+    _decode_e2e(wl)
+
+
+def test_planted_tokens_selected_tiny_f32():
+    wl = S.TINY_F32
+    _, _, got = _decode_e2e(wl)
+    planted = set(S.plant_list8(wl, 0).tolist())
+    for h in range(wl.Hq):
+        assert planted <= set(got[0, h].tolist())
+        assert got[0, h].size == 256 + 4 + 16
+
+
+def test_full_budget_equals_dense():
+    _decode_e2e(SMALL_BF16.with_(keep_pct=100))
+    _decode_e2e(SMALL_BF16.with_(dense_layers=(0,)))
+
+
+@pytest.mark.parametrize("keep", [50, 100])
+def test_llama8b_L32768_end_to_end(keep):
+    _decode_e2e(S.LLAMA8B_L32K.with_(keep_pct=keep))
