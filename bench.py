@@ -53,7 +53,7 @@ def parse():
 
 def workload(args):
     from query_aware_sparse_decode_b200 import synth as S
-    base = S.DECODE32_B4_L131072
+    base = S.DECODE32_B4_L128K
     wl = base.with_(n_layers=args.layers, B=args.batch, L=args.length, keep_pct=args.keep)
     if (wl.n_layers, wl.B, wl.L, wl.keep_pct) != (base.n_layers, base.B, base.L, base.keep_pct):
         wl = wl.with_(name=f"decode{wl.n_layers}_bf16_B{wl.B}_L{wl.L}_keep{wl.keep_pct}")

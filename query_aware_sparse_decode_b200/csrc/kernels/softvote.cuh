@@ -1,0 +1,185 @@
+// Soft-voting variant of the selection (TokenSelect README, "Dynamic
+// Token-Level KV Cache Selection" and "Per-head Soft Voting Mechanism"):
+//
+//   a[h][t] = q[b][h] . K[b][g(h)][t] / sqrt(D),   t < len[b]
+//   p[h][t] = softmax_t(a[h][.]),   votes[b][t] = sum_h p[h][t]
+//
+// One shared ranking per sequence; the selection then reuses the top-k
+// kernel on `votes` (one row per sequence) and the sparse attention kernel in
+// shared-mask mode.
+//
+// softvote_logits: HBM stream over K (each row read once per KV head and
+// shared by the group's query heads), contiguous 16-token tiles gathered by
+// cp.async into a swizzled ring, q . K^T on mma.sync (bf16 in, fp32
+// accumulate); writes the logits in the log2 domain and one (max, sum of
+// 2^(a - max)) pair per head and chunk.
+// softvote_reduce: merges the chunk pairs into each head's (M, Z) and sums
+// 2^(a - M) / Z over the heads for every token (logits are L2-resident).
+#pragma once
+
+#include "attn.cuh"
+#include "common.cuh"
+
+namespace tb {
+
+constexpr int kVoteChunk = 2048;  // tokens per CTA of the logits pass
+
+struct VoteParams {
+  const void* k_cache;  // [B][Hkv][max_len][D] bf16
+  const void* q;        // [B][Hq][D] bf16
+  float* logits;        // [B][Hq][max_len], log2 domain
+  float* stats;         // [B][Hq][nchunk][2]
+  float* votes;         // [B][max_len]
+  int Hq, Hkv, max_len, nchunk;
+  float scale_log2;
+  int lens[kMaxBatch];
+};
+
+template <int D, int GS>
+__global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const VoteParams p) {
+  constexpr int ROWB = D * 2;
+  constexpr int NCH = D / 8;
+  constexpr int STAGE = kAttnTile * ROWB;  // K only
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int L = p.lens[b];
+  const int t0 = chunk * kVoteChunk;
+  if (t0 >= L) return;
+  const int t1 = min(t0 + kVoteChunk, L);
+  const int n = t1 - t0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = lane >> 2, tq = lane & 3;
+  const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.max_len * ROWB;
+
+  uint32_t qa[KSTEPS][2];
+  {
+    const __nv_bfloat16* qrow =
+        reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * GS + (grp < GS ? grp : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const int dim = (4 * (kk / 2) + tq) * 8 + (kk % 2) * 4;
+      qa[kk][0] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim) : 0u;
+      qa[kk][1] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim + 2) : 0u;
+    }
+  }
+  float m_run = kNegInf, l_run = 0.f;
+  const int ntiles = (n + kAttnTile - 1) / kAttnTile;
+  const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  uint8_t* my_ring = smem + warp * kAttnStages * STAGE;
+  auto issue = [&](int it) {
+    const int tile = warp + it * kAttnWarps;
+    uint8_t* sb = my_ring + (it % kAttnStages) * STAGE;
+#pragma unroll
+    for (int c = lane; c < kAttnTile * NCH; c += 32) {
+      const int row = c / NCH, part = c % NCH;
+      const int tok = min(t0 + tile * kAttnTile + row, t1 - 1);  // clamp the ragged tail
+      cp_async_16(sb + row * ROWB + ((part ^ (row & 7)) << 4), Kb + (size_t)tok * ROWB + part * 16);
+    }
+  };
+#pragma unroll
+  for (int s = 0; s < kAttnStages - 1; ++s) {
+    if (s < my_n) issue(s);
+    cp_async_commit();
+  }
+  const size_t lrow = ((size_t)b * p.Hq + g * GS + (grp < GS ? grp : 0)) * p.max_len;
+  for (int it = 0; it < my_n; ++it) {
+    if (it + kAttnStages - 1 < my_n) issue(it + kAttnStages - 1);
+    cp_async_commit();
+    cp_async_wait<kAttnStages - 1>();
+    __syncwarp();
+    const uint8_t* Ks = my_ring + (it % kAttnStages) * STAGE;
+    const int tile = warp + it * kAttnWarps;
+    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int c = 4 * i + tq;
+      const uint4 k0 = *reinterpret_cast<const uint4*>(Ks + grp * ROWB + ((c ^ (grp & 7)) << 4));
+      const uint4 k1 = *reinterpret_cast<const uint4*>(Ks + (grp + 8) * ROWB + ((c ^ (grp & 7)) << 4));
+      mma_16816(acc0, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k0.x, k0.y);
+      mma_16816(acc0, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k0.z, k0.w);
+      mma_16816(acc1, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k1.x, k1.y);
+      mma_16816(acc1, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k1.z, k1.w);
+    }
+    const int tb0 = t0 + tile * kAttnTile;
+    const int ta = tb0 + 2 * tq, tc = tb0 + 2 * tq + 8;
+    const bool real = grp < GS;
+    const float s0 = real && ta < t1 ? acc0[0] * p.scale_log2 : kNegInf;
+    const float s1 = real && ta + 1 < t1 ? acc0[1] * p.scale_log2 : kNegInf;
+    const float s2 = real && tc < t1 ? acc1[0] * p.scale_log2 : kNegInf;
+    const float s3 = real && tc + 1 < t1 ? acc1[1] * p.scale_log2 : kNegInf;
+    if (real) {
+      if (ta + 1 < t1) {
+        *reinterpret_cast<float2*>(p.logits + lrow + ta) = make_float2(s0, s1);
+      } else if (ta < t1) {
+        p.logits[lrow + ta] = s0;
+      }
+      if (tc + 1 < t1) {
+        *reinterpret_cast<float2*>(p.logits + lrow + tc) = make_float2(s2, s3);
+      } else if (tc < t1) {
+        p.logits[lrow + tc] = s2;
+      }
+    }
+    float mt = fmaxf(fmaxf(s0, s1), fmaxf(s2, s3));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+    const float m_new = fmaxf(m_run, mt);
+    if (m_new != kNegInf) {
+      l_run = l_run * exp2f(m_run - m_new) + exp2f(s0 - m_new) + exp2f(s1 - m_new) + exp2f(s2 - m_new) +
+              exp2f(s3 - m_new);
+      m_run = m_new;
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  __syncthreads();
+  float* wm = reinterpret_cast<float*>(smem);
+  float* wl = wm + kAttnWarps * GS;
+  if (grp < GS && tq == 0) {
+    wm[warp * GS + grp] = m_run;
+    wl[warp * GS + grp] = l_run;
+  }
+  __syncthreads();
+  if (tid < GS) {
+    float M = kNegInf;
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, wm[w * GS + tid]);
+    float l = 0.f;
+    if (M != kNegInf)
+      for (int w = 0; w < kAttnWarps; ++w)
+        if (wm[w * GS + tid] != kNegInf) l += wl[w * GS + tid] * exp2f(wm[w * GS + tid] - M);
+    const size_t ph = (((size_t)b * p.Hq + g * GS + tid) * p.nchunk + chunk) * 2;
+    p.stats[ph] = M;
+    p.stats[ph + 1] = l;
+  }
+}
+
+// grid (ceil(max len / 1024), B), block 256: votes for 1024 tokens per CTA.
+__global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
+  __shared__ float sM[256], sInvZ[256];
+  const int b = blockIdx.y;
+  const int L = p.lens[b];
+  const int t_begin = blockIdx.x * 1024;
+  if (t_begin >= L) return;
+  const int nch = (L + kVoteChunk - 1) / kVoteChunk;
+  for (int h = threadIdx.x; h < p.Hq; h += blockDim.x) {
+    const float* st = p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2;
+    float M = kNegInf;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, st[2 * c]);
+    float Z = 0.f;
+    for (int c = 0; c < nch; ++c)
+      if (st[2 * c] != kNegInf) Z += st[2 * c + 1] * exp2f(st[2 * c] - M);
+    sM[h] = M;
+    sInvZ[h] = 1.f / Z;
+  }
+  __syncthreads();
+  for (int t = t_begin + threadIdx.x; t < min(t_begin + 1024, L); t += blockDim.x) {
+    float v = 0.f;
+    for (int h = 0; h < p.Hq; ++h)
+      v += exp2f(p.logits[((size_t)b * p.Hq + h) * p.max_len + t] - sM[h]) * sInvZ[h];
+    p.votes[(size_t)b * p.max_len + t] = v;
+  }
+}
+
+}  // namespace tb

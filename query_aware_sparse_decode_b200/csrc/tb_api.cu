@@ -15,6 +15,7 @@
 #include "kernels/kimp.cuh"
 #include "kernels/score.cuh"
 #include "kernels/select.cuh"
+#include "kernels/softvote.cuh"
 #include "tb.h"
 
 using namespace tb;
@@ -34,7 +35,7 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, scores, mask, part_o, part_ml, votes, total;
+  size_t status, hist, scores, mask, part_o, part_ml, votes, vstats, total;
   int max_splits;
 };
 
@@ -50,6 +51,7 @@ WsLayout layout_of(const tb_config& c) {
   w.part_o = off;  off += align256(B * Hq * (size_t)w.max_splits * c.head_dim * 4);
   w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
   w.votes = off;   off += align256(B * Lm * 4);
+  w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteChunk - 1) / kVoteChunk) * 2 * 4);
   w.total = off;
   return w;
 }
@@ -88,6 +90,7 @@ struct tb_ctx {
   float* part_o = nullptr;
   float* part_ml = nullptr;
   float* votes = nullptr;
+  float* vstats = nullptr;
   cudaEvent_t trace[6] = {};
   bool tracing = false;
   unsigned long long launches = 0;
@@ -300,6 +303,46 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   return cuda_status(cudaGetLastError());
 }
 
+static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* votes, cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  if (c.kv_dtype != TB_BF16) return TB_ERR_UNSUPPORTED;
+  const int maxL = max_len_of(ls, c.batch);
+  if (maxL == 0) return TB_OK;
+  const int gs = c.n_q_heads / c.n_kv_heads;
+  VoteParams p{};
+  p.k_cache = ls.k;
+  p.q = q;
+  p.logits = ctx->scores;
+  p.stats = ctx->vstats;
+  p.votes = votes;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.max_len = c.max_len;
+  p.nchunk = (c.max_len + kVoteChunk - 1) / kVoteChunk;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
+  dim3 grid((maxL + kVoteChunk - 1) / kVoteChunk, c.n_kv_heads, c.batch);
+#define TB_VOTE_CASE(DV, GSV)                                                                 \
+  if (c.head_dim == DV && gs == GSV) {                                                        \
+    auto k = softvote_logits_kernel<DV, GSV>;                                                 \
+    const int smem = kAttnWarps * kAttnStages * kAttnTile * DV * 2;                           \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);               \
+    k<<<grid, kAttnThreads, smem, st>>>(p);                                                   \
+  } else
+  TB_VOTE_CASE(128, 4) TB_VOTE_CASE(128, 2) TB_VOTE_CASE(128, 1) TB_VOTE_CASE(128, 8)
+  TB_VOTE_CASE(64, 4) TB_VOTE_CASE(64, 2) TB_VOTE_CASE(64, 1) TB_VOTE_CASE(64, 8)
+  return TB_ERR_UNSUPPORTED;
+#undef TB_VOTE_CASE
+  ++ctx->launches;
+  tb_status s = cuda_status(cudaGetLastError());
+  if (s != TB_OK) return s;
+  dim3 g2((maxL + 1023) / 1024, c.batch);
+  softvote_reduce_kernel<<<g2, 256, 0, st>>>(p);
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -336,6 +379,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->part_o = reinterpret_cast<float*>(ctx->ws + lay.part_o);
   ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
   ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
+  ctx->vstats = reinterpret_cast<float*>(ctx->ws + lay.vstats);
   if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return TB_ERR_CUDA;
@@ -517,7 +561,15 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
   }
-  if (c.variant == TB_SOFTVOTE) return TB_ERR_UNSUPPORTED;
+  if (c.variant == TB_SOFTVOTE) {
+    s = launch_softvote(ctx, layer, q, ctx->votes, st);
+    if (s != TB_OK) return s;
+    trace_point(ctx, 2, st);
+    s = launch_select(ctx, layer, ctx->votes, nullptr, 1, nullptr, 0, nullptr, ctx->mask, st);
+    if (s != TB_OK) return s;
+    trace_point(ctx, 3, st);
+    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
+  }
   s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 2, st);
@@ -538,8 +590,9 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
 TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream) {
   tb_status s = check_layer(ctx, layer);
   if (s != TB_OK) return s;
-  (void)q; (void)votes; (void)stream;
-  return TB_ERR_UNSUPPORTED;
+  if (!q || !votes) return TB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(votes)) return TB_ERR_SHAPE;
+  return launch_softvote(ctx, layer, q, votes, static_cast<cudaStream_t>(stream));
 }
 
 TB_API tb_status tb_trace_events(tb_ctx* ctx, void* const* events, int n_events) {
