@@ -382,6 +382,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
 }
 
 // ---------------------------------------------------------------- combine
+constexpr int kMaxSplits = 1024;
+
 struct CombineParams {
   const float* part_o;
   const float* part_ml;
@@ -391,29 +393,56 @@ struct CombineParams {
   int lens[kMaxBatch];
 };
 
-// grid (Hq, B), block D threads: merge the split partials of one head.
+// grid (Hq, B), block D threads: fp32 log-sum-exp merge of one head's split
+// partials.  The split weights 2^(m_s - M) sit in shared memory; each thread
+// then sums its output dimension over the splits with independent loads.
 template <typename T>
-__global__ void combine_kernel(const CombineParams p) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+  __shared__ float wts[kMaxSplits];
+  __shared__ float red[4];
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
+  const int lane = d & 31, warp = d >> 5, nw = nt >> 5;
   const int L = p.lens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
   const size_t ph = ((size_t)b * p.Hq + h) * p.nsplit;
   float M = kNegInf;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, p.part_ml[(ph + s) * 2]);
-  float o = 0.f, l = 0.f;
-  if (M != kNegInf) {
-    for (int s = 0; s < ns; ++s) {
-      const float m = p.part_ml[(ph + s) * 2];
-      if (m == kNegInf) continue;
-      const float f = exp2f(m - M);
-      l += f * p.part_ml[(ph + s) * 2 + 1];
-      o += f * p.part_o[(ph + s) * p.D + d];
-    }
-    o /= l;
+  for (int s = d; s < ns; s += nt) {
+    const float m = p.part_ml[(ph + s) * 2];
+    wts[s] = m;
+    M = fmaxf(M, m);
   }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+  for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
+  float lsum = 0.f;
+  for (int s = d; s < ns; s += nt) {
+    const float m = wts[s];
+    const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
+    wts[s] = f;
+    lsum += f * p.part_ml[(ph + s) * 2 + 1];
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();
+  lsum = 0.f;
+  for (int w = 0; w < nw; ++w) lsum += red[w];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* po = p.part_o + ph * p.D + d;
+  int s = 0;
+  for (; s + 4 <= ns; s += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] += wts[s + u] * po[(size_t)(s + u) * p.D];
+  }
+  for (; s < ns; ++s) acc[0] += wts[s] * po[(size_t)s * p.D];
+  const float o = M == kNegInf ? 0.f : ((acc[0] + acc[1]) + (acc[2] + acc[3])) / lsum;
   reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * p.D + d] = from_f32<T>(o);
   if (p.lse != nullptr && d == 0)
-    p.lse[(size_t)b * p.Hq + h] = M == kNegInf ? kNegInf : (M + log2f(l)) * 0.69314718055994531f;
+    p.lse[(size_t)b * p.Hq + h] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
 }
 
 }  // namespace tb

@@ -11,6 +11,7 @@
 namespace tb {
 
 constexpr int kMaxBatch = TB_MAX_BATCH;
+constexpr int kHistBins = 2048;  // 11-bit first radix digit of the selection
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------ order keys
@@ -101,6 +102,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitCycles) return false;
   }
   return true;
+}
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+// Bounded rendezvous of `nwarps` warps on an mbarrier initialised with count
+// nwarps: lane 0 of each warp arrives, every lane waits for the phase to
+// complete.  `phase` is the caller's running phase counter.  Returns false
+// after the time limit.
+__device__ __forceinline__ bool warps_sync_bounded(uint64_t* bar, uint32_t& phase) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cta(bar);
+  const bool ok = mbar_wait(bar, phase & 1);
+  ++phase;
+  return __all_sync(0xffffffffu, ok);
 }
 // 2-D tiled TMA load (no multicast) completing on `bar`
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {

@@ -19,23 +19,38 @@ struct AppendParams {
   int pos[kMaxBatch];  // row written for sequence b (its length before the append)
 };
 
-// grid (Hkv, B), block D threads.  K_imp accumulates in fp32, d = 0..D-1.
+// grid (Hkv, B), block 128 threads: writes the K and V rows, then
+// K_imp[j] = sum_d K[d] W_K[d][j] in fp32 with W_K staged in shared memory;
+// 128 / d' threads share each output column (partial sums over D / parts
+// dimensions, added in a fixed order).
 template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   __shared__ float krow[128];
-  const int g = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const size_t src = ((size_t)b * p.Hkv + g) * p.D + d;
+  __shared__ float wsm[128 * 32];
+  __shared__ float part[128];
+  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const size_t src = ((size_t)b * p.Hkv + g) * p.D;
   const size_t row = ((size_t)b * p.Hkv + g) * p.max_len + p.pos[b];
-  const T kv = reinterpret_cast<const T*>(p.k_new)[src];
-  reinterpret_cast<T*>(p.k_cache)[row * p.D + d] = kv;
-  reinterpret_cast<T*>(p.v_cache)[row * p.D + d] = reinterpret_cast<const T*>(p.v_new)[src];
-  krow[d] = to_f32(kv);
+  const T* W = reinterpret_cast<const T*>(p.w_k);
+  for (int e = tid; e < p.D * p.dimp; e += 128) wsm[e] = to_f32(W[e]);
+  if (tid < p.D) {
+    const T kv = reinterpret_cast<const T*>(p.k_new)[src + tid];
+    reinterpret_cast<T*>(p.k_cache)[row * p.D + tid] = kv;
+    reinterpret_cast<T*>(p.v_cache)[row * p.D + tid] = reinterpret_cast<const T*>(p.v_new)[src + tid];
+    krow[tid] = to_f32(kv);
+  }
   __syncthreads();
-  if (d < p.dimp) {
-    const T* w = reinterpret_cast<const T*>(p.w_k);
-    float acc = 0.f;
-    for (int e = 0; e < p.D; ++e) acc = fmaf(krow[e], to_f32(w[e * p.dimp + d]), acc);
-    p.kimp[row * p.dimp + d] = acc;
+  const int parts = 128 / p.dimp;          // 4 (d'=32) or 8 (d'=16)
+  const int j = tid % p.dimp, q = tid / p.dimp;
+  const int span = p.D / parts;
+  float acc = 0.f;
+  for (int d = q * span; d < (q + 1) * span; ++d) acc = fmaf(krow[d], wsm[d * p.dimp + j], acc);
+  part[tid] = acc;
+  __syncthreads();
+  if (tid < p.dimp) {
+    float sum = 0.f;
+    for (int i = 0; i < parts; ++i) sum += part[i * p.dimp + tid];
+    p.kimp[row * p.dimp + tid] = sum;
   }
 }
 

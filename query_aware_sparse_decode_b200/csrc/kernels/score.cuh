@@ -5,11 +5,13 @@
 //
 // HBM stream over K_imp (d' fp32 = 64 or 128 bytes per token and KV head),
 // read once per KV head and shared by the Hq/Hkv query heads of the group.
-// Persistent CTAs (one per SM) walk a contiguous range of 256-token tiles;
-// each tile is brought in by one TMA 2-D load (128B/64B swizzle, so the
-// thread-per-token reads below are bank-conflict free) through a 4-stage
-// mbarrier ring.  Optionally accumulates, per query-head row, the histogram
-// of the top 11 bits of the order key over the candidate range
+// Persistent CTAs (one per SM) walk a contiguous range of 256-token tiles.
+// Thread 0 feeds a 4-stage ring with one TMA 2-D load per tile (128B/64B
+// swizzle, so the thread-per-token reads are bank-conflict free), guarded by
+// full/empty mbarriers; each of the 8 warps owns 32 tokens of every tile and
+// releases a stage as soon as it has read it.  Optionally the warps
+// accumulate, per query-head row, the
+// histogram of the top 11 bits of the order key over the candidate range
 // [sink, len - window): the first radix digit of the selection.
 #pragma once
 
@@ -17,9 +19,9 @@
 
 namespace tb {
 
-constexpr int kScoreTile = 256;   // tokens per TMA box / threads per CTA
+constexpr int kScoreTile = 256;   // tokens per TMA box (one per consumer thread)
 constexpr int kScoreStages = 4;
-constexpr int kHistBins = 2048;   // 11-bit first digit
+constexpr int kScoreThreads = kScoreTile;   // 8 warps, one token per thread
 
 struct ScoreParams {
   const void* q_imp;  // [(B*Hq)][G][1][d'] of the producer, kv dtype
@@ -42,14 +44,17 @@ __device__ __forceinline__ int swz_offset(int row, int j) {
 }
 
 template <typename T, int DIMP, int GS, bool HIST>
-__global__ void __launch_bounds__(kScoreTile, 1)
+__global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap kimp_map, const ScoreParams p) {
   constexpr int STAGE_BYTES = kScoreTile * DIMP * 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScoreStages * STAGE_BYTES);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(full + kScoreStages);  // [GS][2048] when HIST
-  __shared__ int s_abort;
+  uint64_t* empty = full + kScoreStages;
+  uint64_t* flush = empty + kScoreStages;                              // warp rendezvous
+  uint32_t* hist = reinterpret_cast<uint32_t*>(flush + 1);             // [GS][2048] when HIST
+  __shared__ int s_abort_store;
+  volatile int* s_abort = &s_abort_store;
 
   const int tid = threadIdx.x;
   const int begin = (int)(((long long)blockIdx.x * p.total_tiles) / gridDim.x);
@@ -58,12 +63,16 @@ __global__ void __launch_bounds__(kScoreTile, 1)
   if (n <= 0) return;
 
   if (tid == 0) {
-    for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kScoreStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kScoreThreads / 32);  // one arrival per warp
+    }
+    mbar_init(flush, kScoreThreads / 32);
     mbar_fence_init();
-    s_abort = 0;
+    *s_abort = 0;
   }
   if (HIST)
-    for (int i = tid; i < GS * kHistBins; i += kScoreTile) hist[i] = 0;
+    for (int i = tid; i < GS * kHistBins; i += kScoreThreads) hist[i] = 0;
   __syncthreads();
 
   // tile gt -> (b, g, tile); b advances monotonically over the range
@@ -74,47 +83,58 @@ __global__ void __launch_bounds__(kScoreTile, 1)
     g = local / nt;
     tile = local - g * nt;
   };
-  auto issue = [&](int i) {
-    int b = 0, g, tile;
-    decode(begin + i, b, g, tile);
-    const int st = i % kScoreStages;
+  // thread 0 feeds the ring: tile j into stage j % stages once every warp has
+  // released that stage's previous tile
+  int pb = 0, issued = 0;
+  auto issue = [&](int j) -> bool {
+    const int st = j % kScoreStages;
+    if (!mbar_wait(&empty[st], ((j / kScoreStages) & 1) ^ 1)) return false;
+    int g, tile;
+    decode(begin + j, pb, g, tile);
     mbar_expect_tx(&full[st], STAGE_BYTES);
-    tma_load_2d(smem + st * STAGE_BYTES, &kimp_map, 0, (b * p.Hkv + g) * p.max_len + tile * kScoreTile, &full[st]);
+    tma_load_2d(smem + st * STAGE_BYTES, &kimp_map, 0, (pb * p.Hkv + g) * p.max_len + tile * kScoreTile, &full[st]);
+    issued = j + 1;
+    return true;
   };
   if (tid == 0)
-    for (int i = 0; i < min(kScoreStages, n); ++i) issue(i);
+    for (int j = 0; j < kScoreStages - 1 && j < n; ++j) (void)issue(j);
 
   float q[GS][DIMP];
   int cur_b = -1, cur_g = -1, b = 0;
+  uint32_t fphase = 0;
   for (int i = 0; i < n; ++i) {
+    if (tid == 0 && i + kScoreStages - 1 < n && !*s_abort)
+      if (!issue(i + kScoreStages - 1)) *s_abort = 1;
     int g, tile;
     decode(begin + i, b, g, tile);
     if (b != cur_b || g != cur_g) {
       if (HIST && cur_b >= 0) {  // flush the previous group's histograms
-        __syncthreads();
-        for (int e = tid; e < GS * kHistBins; e += kScoreTile) {
+        if (!warps_sync_bounded(flush, fphase)) *s_abort = 1;
+        if (*s_abort) break;
+        for (int e = tid; e < GS * kHistBins; e += kScoreThreads) {
           const uint32_t c = hist[e];
           if (c) {
             atomicAdd(&p.hist[((size_t)cur_b * p.Hq + cur_g * GS + e / kHistBins) * kHistBins + e % kHistBins], c);
             hist[e] = 0;
           }
         }
+        if (!warps_sync_bounded(flush, fphase)) *s_abort = 1;
+        if (*s_abort) break;
       }
       cur_b = b;
       cur_g = g;
       const T* qi = reinterpret_cast<const T*>(p.q_imp);
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh) {
-        const T* row = qi + (((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP;
+        const T* qrow = qi + (((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP;
 #pragma unroll
-        for (int j = 0; j < DIMP; ++j) q[hh][j] = to_f32(row[j]);
+        for (int j = 0; j < DIMP; ++j) q[hh][j] = to_f32(qrow[j]);
       }
     }
     const int st = i % kScoreStages;
-    if (!mbar_wait(&full[st], (i / kScoreStages) & 1)) s_abort = i + 1;
-    __syncthreads();
-    if (s_abort) break;
-
+    const bool ok = mbar_wait(&full[st], (i / kScoreStages) & 1);
+    if (__any_sync(0xffffffffu, !ok)) *s_abort = 1;
+    if (*s_abort) break;
     const uint8_t* sb = smem + st * STAGE_BYTES;
     float kv[DIMP];
 #pragma unroll
@@ -125,42 +145,33 @@ __global__ void __launch_bounds__(kScoreTile, 1)
       kv[4 * j + 2] = v.z;
       kv[4 * j + 3] = v.w;
     }
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive_cta(&empty[st]);  // this warp is done with the stage
     const int L = p.lens[b];
     const int t = tile * kScoreTile + tid;
+    const bool cand = HIST && t >= p.sink && t < L - p.window;
 #pragma unroll
     for (int hh = 0; hh < GS; ++hh) {
       float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < DIMP; ++j) acc = fmaf(q[hh][j], kv[j], acc);
       if (t < L) p.scores[((size_t)b * p.Hq + g * GS + hh) * p.max_len + t] = acc;
-      if (HIST) {
-        const bool cand = t >= p.sink && t < L - p.window;
-        const uint32_t bin = cand ? (order_key(acc) >> 21) : 0xFFFFFFFFu;
-        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-        if (cand && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[hh * kHistBins + bin], __popc(peers));
-      }
+      if (cand) atomicAdd(&hist[hh * kHistBins + (order_key(acc) >> 21)], 1u);
     }
-    __syncthreads();  // stage fully consumed
-    if (tid == 0 && i + kScoreStages < n) issue(i + kScoreStages);
   }
-
-  if (s_abort) {
-    if (tid == 0) {
-      atomicOr(p.status, TB_DEV_ERR_TIMEOUT);
-      // wait (bounded) for the loads still in flight before leaving
-      const int i0 = s_abort - 1;
-      for (int j = i0; j < n && j < i0 + kScoreStages; ++j)
-        (void)mbar_wait(&full[j % kScoreStages], (j / kScoreStages) & 1);
-    }
-    return;
-  }
-  if (HIST) {
-    __syncthreads();
-    for (int e = tid; e < GS * kHistBins; e += kScoreTile) {
+  if (HIST && !*s_abort && warps_sync_bounded(flush, fphase)) {
+    for (int e = tid; e < GS * kHistBins; e += kScoreThreads) {
       const uint32_t c = hist[e];
       if (c) atomicAdd(&p.hist[((size_t)cur_b * p.Hq + cur_g * GS + e / kHistBins) * kHistBins + e % kHistBins], c);
     }
   }
+  if (tid == 0 && *s_abort) {
+    atomicOr(p.status, TB_DEV_ERR_TIMEOUT);
+    // loads in flight must land before the CTA leaves
+    for (int j = max(0, issued - kScoreStages); j < issued; ++j)
+      (void)mbar_wait(&full[j % kScoreStages], (j / kScoreStages) & 1);
+  }
+  __syncthreads();
 }
 
 // zero the first-digit histograms before a fused score pass

@@ -8,14 +8,21 @@
 //   Sel = [0, min(sink, L)) U top_min(k, |C|)(C) U [max(L - window, 0), L),
 //   order (score desc, index asc), -0.0 == +0.0.
 //
-// One 1024-thread CTA per row.  The k-th largest order key T is found by a
-// three-digit radix select (11 + 11 + 10 bits): shared-memory histograms
-// filled with warp-aggregated atomics (__match_any_sync + popc), each digit
-// chosen by a block-wide suffix scan.  The first digit's histogram can come
-// from the score kernel.  A final ordered sweep keeps keys > T and the
-// lowest-index `quota` keys == T, writing the ascending index list and the
-// bitmask with ballot/shuffle packing; the sink and window are merged in the
-// same sweep, so the output is ascending by construction.
+// One 1024-thread CTA per row; scores are read as monotone uint32 order keys.
+// Fast path (one ordered sweep of the row):
+//   1. first-digit histogram (top 11 key bits) of the candidates - from the
+//      score kernel, else built here - gives the threshold bin b1 and how
+//      many keys lie above it;
+//   2. the sweep sets, in a shared-memory copy of the row bitmask, every
+//      token surely kept (sink, window, digit > b1) and appends the
+//      candidates of bin b1, in index order (block scan), to a shared buffer;
+//   3. the remaining two digits are resolved on that buffer only; ties at the
+//      final key go to the lowest indices (the buffer is in index order);
+//   4. the bitmask, the count and optionally the ascending index list are
+//      written out from shared memory.
+// Fallback (bin b1 larger than the buffer, or rows beyond the shared bitmask):
+// three radix sweeps over the row with warp-aggregated histograms, then an
+// ordered ballot/scan compaction.
 #pragma once
 
 #include "common.cuh"
@@ -23,6 +30,9 @@
 namespace tb {
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelCap = 16384;       // candidate buffer entries (key + index)
+constexpr int kSelMaskWords = 8192;  // shared bitmask words: rows up to 262144 tokens
+constexpr int kSelSmemBytes = kHistBins * 4 + kSelCap * 8 + kSelMaskWords * 4;
 
 struct SelectParams {
   const float* scores;     // row r of sequence b at (b * rows_per_seq + r) * row_stride
@@ -68,8 +78,18 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint3
   __syncthreads();
 }
 
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
 __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectParams p) {
-  __shared__ uint32_t hist[kHistBins];
+  extern __shared__ __align__(16) uint32_t sel_smem[];
+  uint32_t* hist = sel_smem;                           // [2048]
+  uint32_t* ckey = hist + kHistBins;                   // [kSelCap]
+  uint32_t* cidx = ckey + kSelCap;                     // [kSelCap]
+  uint32_t* smask = cidx + kSelCap;                    // [kSelMaskWords]
   __shared__ uint32_t scan_sm[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
@@ -81,43 +101,199 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   const int lo = p.sink, hi = L - p.window;
   const int nc = hi > lo ? hi - lo : 0;
   const int k = (int)min((long long)p.keep_pct * L / 100, (long long)nc);
+  const int lwords = (L + 31) >> 5;
+  const size_t orow = (size_t)row;
 
-  // ---- radix select of the k-th largest key among the candidates
-  uint32_t T = 0, quota = 0;
-  int mode = 0;  // 0: no candidate kept, 1: all kept, 2: threshold T + quota ties
+  int mode = 0;  // 0: no candidate kept, 1: all kept, 2: threshold + quota ties
   if (k == nc && k > 0) mode = 1;
-  if (k > 0 && k < nc) {
-    mode = 2;
-    uint32_t prefix = 0, kk = (uint32_t)k;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int nbits = pass == 2 ? 10 : 11;
-      const int pshift = pass == 1 ? 21 : 10;  // compare key >> pshift with prefix (passes 1, 2)
-      if (pass == 0 && p.hist1 != nullptr) {
-        for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
-        __syncthreads();
-      } else {
-        for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
-        for (int base = lo & ~3; base < hi; base += 4 * kSelThreads) {
-          const int t0 = base + 4 * tid;
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (t0 < hi) v = *reinterpret_cast<const float4*>(s + t0);
+  if (k > 0 && k < nc) mode = 2;
+
+  // ---- first digit: histogram of the candidates' top 11 key bits
+  int b1 = 0;
+  uint32_t k1 = 0, n1 = 0;
+  if (mode == 2) {
+    if (p.hist1 != nullptr) {
+      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
+    } else {
+      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (int base = lo & ~3; base < hi; base += 4 * kSelThreads) {
+        const int t0 = base + 4 * tid;
+        if (t0 < hi) {
+          const float4 v = *reinterpret_cast<const float4*>(s + t0);
           const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int t = t0 + j;
-            const uint32_t key = order_key(vv[j]);
-            const bool in = t >= lo && t < hi && (pass == 0 || (key >> pshift) == prefix);
-            const uint32_t bin = in ? ((key >> shift) & ((1u << nbits) - 1)) : 0xFFFFFFFFu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+          for (int j = 0; j < 4; ++j)
+            if (t0 + j >= lo && t0 + j < hi) atomicAdd(&hist[order_key(vv[j]) >> 21], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    find_bin<2>(hist, (uint32_t)k, scan_sm, &s_bin, &s_above);
+    b1 = s_bin;
+    k1 = (uint32_t)k - s_above;
+    n1 = hist[b1];
+    __syncthreads();
+  }
+  const bool fast = lwords <= kSelMaskWords && (mode != 2 || n1 <= (uint32_t)kSelCap);
+
+  uint32_t T = 0, quota = 0;
+  if (fast) {
+    // ---- one ordered sweep: sure bits into the shared mask, bin-b1 candidates into the buffer
+    uint32_t nbuf = 0;
+    for (int base = 0; base < L; base += 4 * kSelThreads) {
+      const int t0 = base + 4 * tid;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mode == 2 && t0 < L) v = *reinterpret_cast<const float4*>(s + t0);
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t keepbits = 0, cbits = 0, keys[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = t0 + j;
+        keys[j] = order_key(vv[j]);
+        if (t >= L) continue;
+        const bool cand = t >= lo && t < hi;
+        bool keep = !cand || mode == 1;
+        if (cand && mode == 2) {
+          const uint32_t d1 = keys[j] >> 21;
+          if (d1 > (uint32_t)b1) keep = true;
+          else if (d1 == (uint32_t)b1) cbits |= 1u << j;
+        }
+        if (keep) keepbits |= 1u << j;
+      }
+      uint32_t word = keepbits << ((lane & 7) * 4);
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      const int w = (base >> 5) + (tid >> 3);
+      if ((lane & 7) == 0 && w < lwords) smask[w] = word;
+      if (mode == 2) {
+        uint32_t total;
+        uint32_t pos = nbuf + block_excl_scan<kSelThreads>(__popc(cbits), total, scan_sm);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (cbits & (1u << j)) {
+            if (pos < (uint32_t)kSelCap) {
+              ckey[pos] = keys[j];
+              cidx[pos] = (uint32_t)(t0 + j);
+            }
+            ++pos;
           }
+        nbuf += total;
+      }
+    }
+    __syncthreads();
+    if (mode == 2 && nbuf != n1) {  // histogram and scores disagree: flag it, stay in bounds
+      if (tid == 0) atomicOr(p.status, TB_DEV_ERR_COUNT);
+      nbuf = min(nbuf, (uint32_t)kSelCap);
+    }
+
+    if (mode == 2) {
+      // ---- digits 2 and 3 on the buffer
+      uint32_t prefix = (uint32_t)b1, kk = k1;
+#pragma unroll 1
+      for (int pass = 1; pass < 3; ++pass) {
+        const int shift = pass == 1 ? 10 : 0;
+        const int nbits = pass == 1 ? 11 : 10;
+        const int pshift = pass == 1 ? 21 : 10;
+        for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < (int)nbuf; i += kSelThreads) {
+          const uint32_t key = ckey[i];
+          if ((key >> pshift) == prefix) atomicAdd(&hist[(key >> shift) & ((1u << nbits) - 1)], 1u);
         }
         __syncthreads();
+        if (pass == 1)
+          find_bin<2>(hist, kk, scan_sm, &s_bin, &s_above);
+        else
+          find_bin<1>(hist, kk, scan_sm, &s_bin, &s_above);
+        kk -= s_above;
+        prefix = (prefix << nbits) | (uint32_t)s_bin;
+        __syncthreads();
       }
-      if (pass < 2)
+      T = prefix;
+      quota = kk;
+      // ---- keys above T, and the first `quota` ties in index (= buffer) order
+      uint32_t tie_base = 0;
+      for (int base = 0; base < (int)nbuf; base += kSelThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < (int)nbuf ? ckey[i] : 0u;
+        const bool tie = i < (int)nbuf && key == T;
+        uint32_t total;
+        const uint32_t rank = tie_base + block_excl_scan<kSelThreads>(tie ? 1u : 0u, total, scan_sm);
+        if (i < (int)nbuf && (key > T || (tie && rank < quota))) {
+          const uint32_t t = cidx[i];
+          atomicOr(&smask[t >> 5], 1u << (t & 31));
+        }
+        tie_base += total;
+      }
+      __syncthreads();
+    }
+
+    // ---- write out: mask, count, ascending index list
+    uint32_t cnt_local = 0;
+    for (int w = tid; w < lwords; w += kSelThreads) {
+      const uint32_t m = smask[w];
+      if (p.mask != nullptr) p.mask[orow * p.mask_words + w] = m;
+      cnt_local += __popc(m);
+    }
+    uint32_t total_cnt;
+    (void)block_excl_scan<kSelThreads>(cnt_local, total_cnt, scan_sm);
+    if (p.idx != nullptr) {
+      // thread owns consecutive words [w0, w1)
+      const int per = (lwords + kSelThreads - 1) / kSelThreads;
+      const int w0 = min(lwords, tid * per), w1 = min(lwords, w0 + per);
+      uint32_t mine = 0;
+      for (int w = w0; w < w1; ++w) mine += __popc(smask[w]);
+      uint32_t tot;
+      uint32_t pos = block_excl_scan<kSelThreads>(mine, tot, scan_sm);
+      for (int w = w0; w < w1; ++w) {
+        uint32_t m = smask[w];
+        while (m) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1u;
+          if ((int)pos < p.idx_cap) p.idx[orow * p.idx_cap + pos] = w * 32 + j;
+          ++pos;
+        }
+      }
+    }
+    if (tid == 0) {
+      if (p.count != nullptr) p.count[orow] = (int32_t)total_cnt;
+      const int sink_n = min(p.sink, L);
+      const int win_lo = max(L - p.window, sink_n);
+      if (total_cnt != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
+    }
+    return;
+  }
+
+  // ================================================================ fallback
+  if (mode == 2) {
+    uint32_t prefix = (uint32_t)b1, kk = k1;
+#pragma unroll 1
+    for (int pass = 1; pass < 3; ++pass) {
+      const int shift = pass == 1 ? 10 : 0;
+      const int nbits = pass == 1 ? 11 : 10;
+      const int pshift = pass == 1 ? 21 : 10;
+      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (int base = lo & ~3; base < hi; base += 4 * kSelThreads) {
+        const int t0 = base + 4 * tid;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t0 < hi) v = *reinterpret_cast<const float4*>(s + t0);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = t0 + j;
+          const uint32_t key = order_key(vv[j]);
+          const bool in = t >= lo && t < hi && (key >> pshift) == prefix;
+          if (!__any_sync(0xffffffffu, in)) continue;
+          const uint32_t bin = in ? ((key >> shift) & ((1u << nbits) - 1)) : 0xFFFFFFFFu;
+          const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+          if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+      }
+      __syncthreads();
+      if (pass == 1)
         find_bin<2>(hist, kk, scan_sm, &s_bin, &s_above);
       else
         find_bin<1>(hist, kk, scan_sm, &s_bin, &s_above);
@@ -131,14 +307,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 
   // ---- ordered sweep over [0, L): sink, kept candidates, window
   uint32_t out_base = 0, tie_base = 0;
-  const size_t orow = (size_t)row;
   for (int base = 0; base < L; base += 4 * kSelThreads) {
     const int t0 = base + 4 * tid;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (mode == 2 && t0 < L) v = *reinterpret_cast<const float4*>(s + t0);
     const float vv[4] = {v.x, v.y, v.z, v.w};
     uint32_t forced = 0, tie = 0;  // bit j: element t0 + j
-    uint32_t nsel = 0, ntie = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = t0 + j;
@@ -155,8 +329,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
       }
       if (keep) forced |= 1u << j;
     }
-    nsel = __popc(forced);
-    ntie = __popc(tie);
+    const uint32_t nsel = __popc(forced), ntie = __popc(tie);
     uint32_t total;
     const uint32_t ex = block_excl_scan<kSelThreads>(nsel | (ntie << 16), total, scan_sm);
     const uint32_t ex_sel = ex & 0xFFFFu, ex_tie = ex >> 16;

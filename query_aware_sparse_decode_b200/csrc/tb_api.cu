@@ -13,6 +13,8 @@
 #include "kernels/attn.cuh"
 #include "kernels/common.cuh"
 #include "kernels/kimp.cuh"
+#include "kernels/prefill.cuh"
+#include "kernels/project_tc.cuh"
 #include "kernels/score.cuh"
 #include "kernels/select.cuh"
 #include "kernels/softvote.cuh"
@@ -29,6 +31,7 @@ struct LayerState {
   const void* wk = nullptr;
   bool bound = false;
   CUtensorMap kimp_map;
+  CUtensorMap k_map;  // bf16 caches: K rows, 64-column boxes of 128 rows, 128B swizzle
   int lens[TB_MAX_BATCH];
 };
 
@@ -168,19 +171,19 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   if (p.total_tiles == 0) return cuda_status(cudaGetLastError());
   const int grid = std::min(p.total_tiles, ctx->num_sms);
   const int gs = c.n_q_heads / c.n_kv_heads;
-  const size_t smem = 1024 + (size_t)kScoreStages * kScoreTile * c.d_imp * 4 + kScoreStages * 8 +
+  const size_t smem = 1024 + (size_t)kScoreStages * kScoreTile * c.d_imp * 4 + (2 * kScoreStages + 1) * 8 +
                       (hist ? (size_t)gs * kHistBins * 4 : 0);
 #define TB_SCORE_CASE(T, DI, GSV)                                                                          \
   if (c.d_imp == DI && gs == GSV) {                                                                        \
     if (hist) {                                                                                            \
       auto k = score_kernel<T, DI, GSV, true>;                                                             \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      k<<<grid, kScoreTile, smem, st>>>(ls.kimp_map, p);                                                   \
+      k<<<grid, kScoreThreads, smem, st>>>(ls.kimp_map, p);                                                   \
       ++ctx->launches;                                                                                     \
     } else {                                                                                               \
       auto k = score_kernel<T, DI, GSV, false>;                                                            \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      k<<<grid, kScoreTile, smem, st>>>(ls.kimp_map, p);                                                   \
+      k<<<grid, kScoreThreads, smem, st>>>(ls.kimp_map, p);                                                   \
       ++ctx->launches;                                                                                     \
     }                                                                                                      \
     return cuda_status(cudaGetLastError());                                                                \
@@ -224,7 +227,8 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, cons
   p.window = c.window;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   dim3 grid(rows, c.batch);
-  select_kernel<<<grid, kSelThreads, 0, st>>>(p);
+  cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmemBytes);
+  select_kernel<<<grid, kSelThreads, kSelSmemBytes, st>>>(p);
   ++ctx->launches;
   return cuda_status(cudaGetLastError());
 }
@@ -257,6 +261,7 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   chunk = std::min(kAttnMaxChunk, std::max(256, (chunk + 255) / 256 * 256));
   p.chunk = chunk;
   p.nsplit = std::max(1, (maxL + chunk - 1) / chunk);
+  if (p.nsplit > kMaxSplits) return TB_ERR_UNSUPPORTED;
   if (p.nsplit > ctx->lay.max_splits) return TB_ERR_WORKSPACE;
   if (maxL > 0) {
     dim3 grid(p.nsplit, c.n_kv_heads, c.batch);
@@ -406,6 +411,15 @@ TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_ca
                    c.d_imp == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return TB_ERR_CUDA;
+  if (c.kv_dtype == TB_BF16) {
+    cuuint64_t kdim[2] = {(cuuint64_t)c.head_dim, (cuuint64_t)c.batch * c.n_kv_heads * c.max_len};
+    cuuint64_t kstride[1] = {(cuuint64_t)c.head_dim * 2};
+    cuuint32_t kbox[2] = {64, (cuuint32_t)kTcRows};
+    r = enc(&ls.k_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_cache, kdim, kstride, kbox, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return TB_ERR_CUDA;
+  }
   ls.k = k_cache;
   ls.v = v_cache;
   ls.kimp = kimp_cache;
@@ -465,9 +479,9 @@ TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const v
   dim3 grid(c.n_kv_heads, c.batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c.kv_dtype == TB_BF16)
-    append_kernel<__nv_bfloat16><<<grid, c.head_dim, 0, st>>>(p);
+    append_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(p);
   else
-    append_kernel<float><<<grid, c.head_dim, 0, st>>>(p);
+    append_kernel<float><<<grid, 128, 0, st>>>(p);
   ++ctx->launches;
   s = cuda_status(cudaGetLastError());
   if (s != TB_OK) return s;
@@ -482,18 +496,36 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
   if (start < 0 || count < 0 || (long long)start + count > c.max_len) return TB_ERR_CAPACITY;
   if (count == 0) return TB_OK;
   const LayerState& ls = ctx->layers[layer];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c.kv_dtype == TB_BF16) {
+    ProjectTcParams tp{};
+    tp.w_k = ls.wk;
+    tp.kimp = ls.kimp;
+    tp.status = ctx->status;
+    tp.max_len = c.max_len;
+    tp.start = start;
+    tp.count = count;
+    tp.tiles_per_slab = (count + kTcRows - 1) / kTcRows;
+    tp.total_tiles = tp.tiles_per_slab * c.batch * c.n_kv_heads;
+    const int grid = std::min(tp.total_tiles, ctx->num_sms);
+#define TB_TC_CASE(DV, DI)                                                              \
+  if (c.head_dim == DV && c.d_imp == DI) {                                              \
+    auto k = project_tc_kernel<DV, DI>;                                                 \
+    const int smem = project_tc_smem_bytes<DV>();                                       \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);         \
+    k<<<grid, kTcThreads, smem, st>>>(ls.k_map, tp);                                    \
+  } else
+    TB_TC_CASE(128, 32) TB_TC_CASE(128, 16) TB_TC_CASE(64, 32) TB_TC_CASE(64, 16) return TB_ERR_UNSUPPORTED;
+#undef TB_TC_CASE
+    ++ctx->launches;
+    return cuda_status(cudaGetLastError());
+  }
   ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count};
   dim3 grid((count + kProjRows - 1) / kProjRows, c.n_kv_heads, c.batch);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define TB_PROJ_CASE(T, DV, DI) \
   if (c.head_dim == DV && c.d_imp == DI) project_fma_kernel<T, DV, DI><<<grid, 256, 0, st>>>(p); else
-  if (c.kv_dtype == TB_BF16) {
-    TB_PROJ_CASE(__nv_bfloat16, 128, 32) TB_PROJ_CASE(__nv_bfloat16, 128, 16) TB_PROJ_CASE(__nv_bfloat16, 64, 32)
-    TB_PROJ_CASE(__nv_bfloat16, 64, 16) return TB_ERR_UNSUPPORTED;
-  } else {
-    TB_PROJ_CASE(float, 128, 32) TB_PROJ_CASE(float, 128, 16) TB_PROJ_CASE(float, 64, 32)
-    TB_PROJ_CASE(float, 64, 16) return TB_ERR_UNSUPPORTED;
-  }
+  TB_PROJ_CASE(float, 128, 32) TB_PROJ_CASE(float, 128, 16) TB_PROJ_CASE(float, 64, 32)
+  TB_PROJ_CASE(float, 64, 16) return TB_ERR_UNSUPPORTED;
 #undef TB_PROJ_CASE
   ++ctx->launches;
   return cuda_status(cudaGetLastError());
@@ -583,8 +615,50 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
                                    uint32_t* row_masks, int words_per_row, void* stream) {
   tb_status s = check_layer(ctx, layer);
   if (s != TB_OK) return s;
-  (void)q_imp_rows; (void)row0; (void)nrows; (void)row_masks; (void)words_per_row; (void)stream;
-  return TB_ERR_UNSUPPORTED;
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  if (!q_imp_rows || !row_masks) return TB_ERR_INVALID_ARG;
+  if (row0 < 0 || nrows < 0) return TB_ERR_INVALID_ARG;
+  if (nrows == 0) return TB_OK;
+  const long long need = (long long)row0 + nrows;
+  if (need > c.max_len) return TB_ERR_CAPACITY;
+  if (words_per_row < (need + 31) / 32) return TB_ERR_SHAPE;
+  for (int b = 0; b < c.batch; ++b)
+    if (ls.lens[b] < need) return TB_ERR_STATE;  // K_imp rows of the prefix must exist
+  const size_t smem = (size_t)need * 4;
+  if (smem > 200 * 1024) return TB_ERR_UNSUPPORTED;  // row scores live in shared memory
+  PrefillParams p{};
+  p.q_imp = q_imp_rows;
+  p.kimp = ls.kimp;
+  p.masks = row_masks;
+  p.status = ctx->status;
+  p.G = c.producer_freq;
+  p.slot = ((layer - 1) % c.producer_freq + c.producer_freq) % c.producer_freq;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.max_len = c.max_len;
+  p.row0 = row0;
+  p.nrows = nrows;
+  p.words_per_row = words_per_row;
+  p.keep_pct = c.keep_pct;
+  p.sink = c.sink;
+  p.window = c.window;
+  dim3 grid(nrows, c.n_q_heads, c.batch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define TB_PF_CASE(T, DI)                                                               \
+  if (c.d_imp == DI) {                                                                  \
+    auto k = prefill_select_kernel<T, DI>;                                              \
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+    k<<<grid, kSelThreads, smem, st>>>(p);                                              \
+  } else
+  if (c.kv_dtype == TB_BF16) {
+    TB_PF_CASE(__nv_bfloat16, 32) TB_PF_CASE(__nv_bfloat16, 16) return TB_ERR_UNSUPPORTED;
+  } else {
+    TB_PF_CASE(float, 32) TB_PF_CASE(float, 16) return TB_ERR_UNSUPPORTED;
+  }
+#undef TB_PF_CASE
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
 }
 
 TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream) {

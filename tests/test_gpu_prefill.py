@@ -1,0 +1,101 @@
+"""GPU parity of the prefill importance path: K_imp = K . W_K on the tensor
+cores (tcgen05, bf16 operands, fp32 accumulation) and the per-row causal
+selection of a prefill query chunk, against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import tokenbutler as O
+from query_aware_sparse_decode_b200 import synth as S
+from query_aware_sparse_decode_b200 import tb as TB
+
+from harness import config_of, make_layer, round_up, sets_from_mask, tie_band_ok, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _kimp_tol(K, W):
+    return 8e-6 * (np.abs(K) @ np.abs(W)) + 1e-30
+
+
+@pytest.mark.parametrize("start,count", [(0, 32768), (5, 1000), (32640, 100)])
+def test_tcgen05_projection_prefill_scale(start, count):
+    """One layer of the prefill workload: B=1, 8 KV heads, 32768 cached rows,
+    D=128 -> d'=32; rows checked against fp64 on every KV head."""
+    wl = S.PREFILL_L32K.with_(n_layers=1, dense_layers=())
+    ctx = TB.Context(config_of(wl, max_len=32768 + 256))
+    B, Hkv, D = wl.B, wl.Hkv, wl.D
+    K_raw = S.kv_cache_host(wl, 0, S.K_CACHE, 0, 32768).reshape(B, Hkv, 32768, D)
+    W_raw = S.w_k(wl, 0)
+    k = torch.zeros((B, Hkv, ctx.cfg.max_len, D), dtype=torch.bfloat16, device="cuda")
+    k[:, :, :32768] = to_dev(K_raw, wl)
+    kimp = torch.full((B, Hkv, ctx.cfg.max_len, wl.d_imp), float("nan"), device="cuda")
+    ctx.bind_layer(0, k, torch.zeros_like(k), kimp, to_dev(W_raw, wl))
+    ctx.set_seq_lens(0, [32768])
+    ctx.project_kimp(0, start, count)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    got = kimp.cpu().numpy().astype(np.float64)
+    K = S.widen(K_raw, wl.dtype)
+    W = S.widen(W_raw, wl.dtype)
+    for g in range(Hkv):
+        ref = O.project_keys(K[0, g, start:start + count], W)
+        assert np.all(np.abs(got[0, g, start:start + count] - ref) <= _kimp_tol(K[0, g, start:start + count], W))
+        assert np.all(np.isnan(got[0, g, :start])) and np.all(np.isnan(got[0, g, start + count:]))
+
+
+PF_SMALL = S.Workload("prefill_small", n_layers=8, B=2, Hq=8, Hkv=2, D=128, d_imp=32, G=4, L=3000, dtype="bf16",
+                      keep_pct=50, sink=16, window=64, dense_layers=(0,))
+
+
+def _prefill_case(wl, layer, row0, nrows, heads=None, rows=None):
+    cfg = config_of(wl, max_len=round_up(wl.L, 256))
+    ctx = TB.Context(cfg)
+    ld = make_layer(ctx, wl, layer, [wl.L] * wl.B)
+    ctx.project_kimp(layer, 0, wl.L)
+    prod = O.producer_of(layer, wl.G)
+    qrows_raw = S.q_imp(wl, prod, rows=(row0, nrows))
+    wpr = (row0 + nrows + 31) // 32
+    masks = torch.zeros((wl.B, wl.Hq, nrows, wpr), dtype=torch.int32, device="cuda")
+    ctx.select_prefill(layer, to_dev(qrows_raw, wl), row0, nrows, masks)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    qrows = S.widen(qrows_raw, wl.dtype).reshape(wl.B, wl.Hq, wl.G, nrows, wl.d_imp)
+    slot = O.consumer_slot(layer, wl.G)
+    m = masks.cpu().numpy().view(np.uint32)
+    gs = wl.Hq // wl.Hkv
+    full = heads is None and rows is None
+    heads = range(wl.Hq) if heads is None else heads
+    rows = range(nrows) if rows is None else rows
+    exact = checked = 0
+    for b in range(wl.B):
+        Kimp = O.project_keys(ld.K[b], ld.W)
+        ref = O.prefill_select(qrows[b, :, slot], Kimp, row0, wl.keep_pct, wl.sink, wl.window) if full else None
+        for h in heads:
+            for r in rows:
+                p = row0 + r
+                bits = np.unpackbits(m[b, h, r].view(np.uint8), bitorder="little")
+                assert not bits[p + 1:].any()          # causal: nothing after the row's position
+                got = np.nonzero(bits[:p + 1])[0]
+                s = O.importance_scores(qrows[b, h, slot, r], Kimp[h // gs, :p + 1])
+                want = ref[h, p] if full else O.select_tokens(s, p + 1, wl.keep_pct, wl.sink, wl.window)
+                assert tie_band_ok(got, want, s, p + 1, wl.keep_pct, wl.sink, wl.window)
+                exact += np.array_equal(got, want)
+                checked += 1
+    assert exact >= 0.95 * checked
+
+
+def test_prefill_rows_small():
+    _prefill_case(PF_SMALL, layer=5, row0=2936, nrows=64)
+
+
+def test_prefill_rows_short_prefix_and_edges():
+    # rows 0..99: prefixes shorter than sink + window, then growing budgets
+    _prefill_case(PF_SMALL.with_(L=400, B=1), layer=4, row0=0, nrows=100)
+
+
+def test_prefill_rows_llama8b_L32768_sampled():
+    """The prefill workload's chunk (last 1024 positions of 32768): 4 heads x
+    64 sampled rows checked against the oracle."""
+    wl = S.PREFILL_L32K.with_(n_layers=2)
+    _prefill_case(wl, layer=1, row0=32768 - 1024, nrows=1024, heads=[0, 9, 18, 31], rows=range(0, 1024, 16))
