@@ -33,6 +33,9 @@ struct AttnParams {
   const uint32_t* mask;  // per mask_mode
   float* part_o;         // [B][Hq][nsplit][D]
   float* part_ml;        // [B][Hq][nsplit][2]: running max (log2 domain), sum
+  uint32_t* tickets;     // [B][Hkv] split-completion counters (zero between calls)
+  void* out;             // [B][Hq][D] kv dtype
+  float* lse;            // [B][Hq] or nullptr
   uint32_t* status;
   int mask_mode, mask_words;
   int Hq, Hkv, max_len, chunk, nsplit;
@@ -125,6 +128,89 @@ __device__ __forceinline__ void write_partial(const AttnParams& p, int b, int g,
   }
 }
 
+
+// The last CTA of (b, g) to finish merges the split partials of the group's
+// heads with an fp32 log-sum-exp and writes out / lse.  Completion is counted
+// with an atomic ticket after a fence (no CTA waits on another); the ticket
+// is reset for the next call by the merging CTA.  Partials are read through
+// L2 (they were written by other SMs).
+constexpr int kMaxSplits = 1024;
+
+template <typename T, int D, int GS>
+__device__ __forceinline__ void merge_if_last(const AttnParams& p, int b, int g, int L, float* wts) {
+  __shared__ int s_last;
+  __shared__ float red[kAttnWarps];
+  __threadfence();
+  __syncthreads();
+  const int ns = (L + p.chunk - 1) / p.chunk;
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(&p.tickets[b * p.Hkv + g], 1u);
+    s_last = prev == (uint32_t)(ns - 1);
+    if (s_last) p.tickets[b * p.Hkv + g] = 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int hh = 0; hh < GS; ++hh) {
+    const int h = g * GS + hh;
+    const size_t ph = ((size_t)b * p.Hq + h) * p.nsplit;
+    float M = kNegInf;
+    for (int sp = tid; sp < ns; sp += kAttnThreads) {
+      const float m = __ldcg(p.part_ml + (ph + sp) * 2);
+      wts[sp] = m;
+      M = fmaxf(M, m);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < kAttnWarps; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    float lsum = 0.f;
+    for (int sp = tid; sp < ns; sp += kAttnThreads) {
+      const float m = wts[sp];
+      const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
+      wts[sp] = f;
+      lsum += f * __ldcg(p.part_ml + (ph + sp) * 2 + 1);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    if (lane == 0) red[warp] = lsum;
+    __syncthreads();
+    lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) lsum += red[w];
+    for (int d = tid; d < D; d += kAttnThreads) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* po = p.part_o + ph * D + d;
+      int sp = 0;
+      for (; sp + 4 <= ns; sp += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] += wts[sp + u] * __ldcg(po + (size_t)(sp + u) * D);
+      }
+      for (; sp < ns; ++sp) acc[0] += wts[sp] * __ldcg(po + (size_t)sp * D);
+      const float o = M == kNegInf ? 0.f : ((acc[0] + acc[1]) + (acc[2] + acc[3])) / lsum;
+      reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * D + d] = from_f32<T>(o);
+    }
+    if (p.lse != nullptr && tid == 0)
+      p.lse[(size_t)b * p.Hq + h] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
+    __syncthreads();
+  }
+}
+
+// An empty sequence has no split to merge: split 0 writes out = 0, lse = -inf.
+template <typename T, int D, int GS>
+__device__ __forceinline__ void write_empty(const AttnParams& p, int b, int g) {
+  for (int e = threadIdx.x; e < GS * D; e += kAttnThreads) {
+    const int h = g * GS + e / D;
+    reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * D + e % D] = from_f32<T>(0.f);
+    if (p.lse != nullptr && e % D == 0) p.lse[(size_t)b * p.Hq + h] = kNegInf;
+  }
+}
+
 // ---------------------------------------------------------------- bf16 / mma.sync
 template <int D>
 constexpr int attn_bf16_smem_bytes() {
@@ -149,6 +235,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.lens[b];
   const int t0 = split * p.chunk;
+  if (L == 0 && split == 0) write_empty<__nv_bfloat16, D, GS>(p, b, g);
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
   const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
@@ -301,13 +388,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
+  merge_if_last<__nv_bfloat16, D, GS>(p, b, g, L, wo + kAttnWarps * GS * D);
 }
 
 // ---------------------------------------------------------------- fp32 / FMA
 constexpr int kListBytes = ((kAttnMaxChunk + kAttnTile) * 5 + 15) / 16 * 16;
 template <int D>
 constexpr int attn_f32_smem_bytes() {
-  return kListBytes + kAttnWarps * 8 * (D + 2) * 4;
+  return kListBytes + kAttnWarps * 8 * (D + 2) * 4 + 1024 * 4;  // + split weights of the merge
 }
 
 // fp32 caches: one warp per token at a time, lane owns dims lane + 32 j.
@@ -325,6 +413,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.lens[b];
   const int t0 = split * p.chunk;
+  if (L == 0 && split == 0) write_empty<float, D, GS>(p, b, g);
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
   const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
@@ -379,70 +468,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
-}
-
-// ---------------------------------------------------------------- combine
-constexpr int kMaxSplits = 1024;
-
-struct CombineParams {
-  const float* part_o;
-  const float* part_ml;
-  void* out;   // [B][Hq][D] kv dtype
-  float* lse;  // [B][Hq] or nullptr
-  int Hq, D, chunk, nsplit;
-  int lens[kMaxBatch];
-};
-
-// grid (Hq, B), block D threads: fp32 log-sum-exp merge of one head's split
-// partials.  The split weights 2^(m_s - M) sit in shared memory; each thread
-// then sums its output dimension over the splits with independent loads.
-template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
-  __shared__ float wts[kMaxSplits];
-  __shared__ float red[4];
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
-  const int lane = d & 31, warp = d >> 5, nw = nt >> 5;
-  const int L = p.lens[b];
-  const int ns = (L + p.chunk - 1) / p.chunk;
-  const size_t ph = ((size_t)b * p.Hq + h) * p.nsplit;
-  float M = kNegInf;
-  for (int s = d; s < ns; s += nt) {
-    const float m = p.part_ml[(ph + s) * 2];
-    wts[s] = m;
-    M = fmaxf(M, m);
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  M = red[0];
-  for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-  float lsum = 0.f;
-  for (int s = d; s < ns; s += nt) {
-    const float m = wts[s];
-    const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
-    wts[s] = f;
-    lsum += f * p.part_ml[(ph + s) * 2 + 1];
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if (lane == 0) red[warp] = lsum;
-  __syncthreads();
-  lsum = 0.f;
-  for (int w = 0; w < nw; ++w) lsum += red[w];
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* po = p.part_o + ph * p.D + d;
-  int s = 0;
-  for (; s + 4 <= ns; s += 4) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] += wts[s + u] * po[(size_t)(s + u) * p.D];
-  }
-  for (; s < ns; ++s) acc[0] += wts[s] * po[(size_t)s * p.D];
-  const float o = M == kNegInf ? 0.f : ((acc[0] + acc[1]) + (acc[2] + acc[3])) / lsum;
-  reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * p.D + d] = from_f32<T>(o);
-  if (p.lse != nullptr && d == 0)
-    p.lse[(size_t)b * p.Hq + h] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
+  merge_if_last<float, D, GS>(p, b, g, L, wo + kAttnWarps * GS * D);
 }
 
 }  // namespace tb

@@ -157,4 +157,40 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t& total,
   return base + x - v;
 }
 
+// Exclusive prefix sums of two fields at once (same contract as
+// block_excl_scan; `sm` holds >= 32 uint2).
+template <int NT>
+__device__ __forceinline__ uint2 block_excl_scan2(uint2 v, uint2& total, uint2* sm) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint2 x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t a = __shfl_up_sync(0xffffffffu, x.x, o), c = __shfl_up_sync(0xffffffffu, x.y, o);
+    if (lane >= o) {
+      x.x += a;
+      x.y += c;
+    }
+  }
+  if (lane == 31) sm[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint2 w = lane < NW ? sm[lane] : make_uint2(0u, 0u);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t a = __shfl_up_sync(0xffffffffu, w.x, o), c = __shfl_up_sync(0xffffffffu, w.y, o);
+      if (lane >= o) {
+        w.x += a;
+        w.y += c;
+      }
+    }
+    if (lane < NW) sm[lane] = w;
+  }
+  __syncthreads();
+  const uint2 base = warp ? sm[warp - 1] : make_uint2(0u, 0u);
+  total = sm[NW - 1];
+  __syncthreads();
+  return make_uint2(base.x + x.x - v.x, base.y + x.y - v.y);
+}
+
 }  // namespace tb

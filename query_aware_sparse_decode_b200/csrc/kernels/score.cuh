@@ -8,7 +8,8 @@
 // Persistent CTAs (one per SM) walk a contiguous range of 256-token tiles.
 // Thread 0 feeds a 4-stage ring with one TMA 2-D load per tile (128B/64B
 // swizzle, so the thread-per-token reads are bank-conflict free), guarded by
-// full/empty mbarriers; each of the 8 warps owns 32 tokens of every tile and
+// full/empty mbarriers; thread (half, t) of the 16 warps scores token t of
+// every tile for one half of the group's query heads, and each warp
 // releases a stage as soon as it has read it.  Optionally the warps
 // accumulate, per query-head row, the
 // histogram of the top 11 bits of the order key over the candidate range
@@ -21,7 +22,7 @@ namespace tb {
 
 constexpr int kScoreTile = 256;   // tokens per TMA box (one per consumer thread)
 constexpr int kScoreStages = 4;
-constexpr int kScoreThreads = kScoreTile;   // 8 warps, one token per thread
+constexpr int kScoreThreads = 2 * kScoreTile;  // 16 warps: (token, half of the group's heads) per thread
 
 struct ScoreParams {
   const void* q_imp;  // [(B*Hq)][G][1][d'] of the producer, kv dtype
@@ -99,7 +100,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   if (tid == 0)
     for (int j = 0; j < kScoreStages - 1 && j < n; ++j) (void)issue(j);
 
-  float q[GS][DIMP];
+  constexpr int HPT = (GS + 1) / 2;                     // heads of this thread: the group split in two halves
+  const int row = tid % kScoreTile;                      // token of the tile
+  const int h0 = (tid / kScoreTile) * HPT;               // first head (within the group) of this thread
+  const bool active_heads = h0 < GS;
+  float q[HPT][DIMP];
   int cur_b = -1, cur_g = -1, b = 0;
   uint32_t fphase = 0;
   for (int i = 0; i < n; ++i) {
@@ -125,8 +130,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       cur_g = g;
       const T* qi = reinterpret_cast<const T*>(p.q_imp);
 #pragma unroll
-      for (int hh = 0; hh < GS; ++hh) {
-        const T* qrow = qi + (((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP;
+      for (int hh = 0; hh < HPT; ++hh) {
+        const T* qrow = qi + (((size_t)b * p.Hq + g * GS + (active_heads ? h0 + hh : 0)) * p.G + p.slot) * DIMP;
 #pragma unroll
         for (int j = 0; j < DIMP; ++j) q[hh][j] = to_f32(qrow[j]);
       }
@@ -139,7 +144,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     float kv[DIMP];
 #pragma unroll
     for (int j = 0; j < DIMP / 4; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(sb + swz_offset<DIMP>(tid, j));
+      const float4 v = *reinterpret_cast<const float4*>(sb + swz_offset<DIMP>(row, j));
       kv[4 * j] = v.x;
       kv[4 * j + 1] = v.y;
       kv[4 * j + 2] = v.z;
@@ -147,16 +152,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     __syncwarp();
     if ((tid & 31) == 0) mbar_arrive_cta(&empty[st]);  // this warp is done with the stage
+    if (!active_heads) continue;
     const int L = p.lens[b];
-    const int t = tile * kScoreTile + tid;
+    const int t = tile * kScoreTile + row;
     const bool cand = HIST && t >= p.sink && t < L - p.window;
 #pragma unroll
-    for (int hh = 0; hh < GS; ++hh) {
+    for (int hh = 0; hh < HPT; ++hh) {
       float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < DIMP; ++j) acc = fmaf(q[hh][j], kv[j], acc);
-      if (t < L) p.scores[((size_t)b * p.Hq + g * GS + hh) * p.max_len + t] = acc;
-      if (cand) atomicAdd(&hist[hh * kHistBins + (order_key(acc) >> 21)], 1u);
+      if (t < L) p.scores[((size_t)b * p.Hq + g * GS + h0 + hh) * p.max_len + t] = acc;
+      if (cand) atomicAdd(&hist[(h0 + hh) * kHistBins + (order_key(acc) >> 21)], 1u);
     }
   }
   if (HIST && !*s_abort && warps_sync_bounded(flush, fphase)) {

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   uint32_t* cidx = ckey + kSelCap;                     // [kSelCap]
   uint32_t* smask = cidx + kSelCap;                    // [kSelMaskWords]
   __shared__ uint32_t scan_sm[32];
+  __shared__ uint2 scan2_sm[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
 
@@ -139,48 +140,78 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 
   uint32_t T = 0, quota = 0;
   if (fast) {
-    // ---- one ordered sweep: sure bits into the shared mask, bin-b1 candidates into the buffer
+    // ---- one ordered sweep: sure bits into the shared mask, bin-b1 candidates
+    // into the buffer.  An iteration covers 4 chunks of 4096 tokens; thread
+    // tid owns tokens 4*tid..4*tid+3 of every chunk (coalesced float4 loads),
+    // and the next iteration's loads are issued before this one is processed.
+    constexpr int CH = 4;
+    constexpr int ITER = CH * 4 * kSelThreads;
     uint32_t nbuf = 0;
-    for (int base = 0; base < L; base += 4 * kSelThreads) {
-      const int t0 = base + 4 * tid;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (mode == 2 && t0 < L) v = *reinterpret_cast<const float4*>(s + t0);
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-      uint32_t keepbits = 0, cbits = 0, keys[4];
+    float4 cur[CH], nxt[CH];
+    auto load_iter = [&](int base, float4 (&dst)[CH]) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = t0 + j;
-        keys[j] = order_key(vv[j]);
-        if (t >= L) continue;
-        const bool cand = t >= lo && t < hi;
-        bool keep = !cand || mode == 1;
-        if (cand && mode == 2) {
-          const uint32_t d1 = keys[j] >> 21;
-          if (d1 > (uint32_t)b1) keep = true;
-          else if (d1 == (uint32_t)b1) cbits |= 1u << j;
-        }
-        if (keep) keepbits |= 1u << j;
+      for (int c = 0; c < CH; ++c) {
+        const int t0 = base + c * 4 * kSelThreads + 4 * tid;
+        dst[c] = (mode == 2 && t0 < L) ? *reinterpret_cast<const float4*>(s + t0) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      uint32_t word = keepbits << ((lane & 7) * 4);
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      const int w = (base >> 5) + (tid >> 3);
-      if ((lane & 7) == 0 && w < lwords) smask[w] = word;
-      if (mode == 2) {
-        uint32_t total;
-        uint32_t pos = nbuf + block_excl_scan<kSelThreads>(__popc(cbits), total, scan_sm);
+    };
+    load_iter(0, cur);
+    for (int base = 0; base < L; base += ITER) {
+      if (base + ITER < L) load_iter(base + ITER, nxt);
+      uint32_t cbits[CH];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (cbits & (1u << j)) {
-            if (pos < (uint32_t)kSelCap) {
-              ckey[pos] = keys[j];
-              cidx[pos] = (uint32_t)(t0 + j);
-            }
-            ++pos;
+      for (int c = 0; c < CH; ++c) {
+        const int t0 = base + c * 4 * kSelThreads + 4 * tid;
+        const float vv[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
+        uint32_t keepbits = 0;
+        cbits[c] = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = t0 + j;
+          if (t >= L) continue;
+          const bool cand = t >= lo && t < hi;
+          bool keep = !cand || mode == 1;
+          if (cand && mode == 2) {
+            const uint32_t d1 = order_key(vv[j]) >> 21;
+            if (d1 > (uint32_t)b1) keep = true;
+            else if (d1 == (uint32_t)b1) cbits[c] |= 1u << j;
           }
-        nbuf += total;
+          if (keep) keepbits |= 1u << j;
+        }
+        uint32_t word = keepbits << ((lane & 7) * 4);
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        const int w = ((base + c * 4 * kSelThreads) >> 5) + (tid >> 3);
+        if ((lane & 7) == 0 && w < lwords) smask[w] = word;
       }
+      if (mode == 2) {
+        uint2 tot;
+        const uint2 ex = block_excl_scan2<kSelThreads>(
+            make_uint2(__popc(cbits[0]) | (__popc(cbits[1]) << 16), __popc(cbits[2]) | (__popc(cbits[3]) << 16)),
+            tot, scan2_sm);
+        const uint32_t t0c = tot.x & 0xFFFFu, t1c = tot.x >> 16, t2c = tot.y & 0xFFFFu, t3c = tot.y >> 16;
+        const uint32_t start[CH] = {nbuf + (ex.x & 0xFFFFu), nbuf + t0c + (ex.x >> 16),
+                                    nbuf + t0c + t1c + (ex.y & 0xFFFFu), nbuf + t0c + t1c + t2c + (ex.y >> 16)};
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          uint32_t pos = start[c];
+          const int t0 = base + c * 4 * kSelThreads + 4 * tid;
+          const float vv[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (cbits[c] & (1u << j)) {
+              if (pos < (uint32_t)kSelCap) {
+                ckey[pos] = order_key(vv[j]);
+                cidx[pos] = (uint32_t)(t0 + j);
+              }
+              ++pos;
+            }
+        }
+        nbuf += t0c + t1c + t2c + t3c;
+      }
+#pragma unroll
+      for (int c = 0; c < CH; ++c) cur[c] = nxt[c];
     }
     __syncthreads();
     if (mode == 2 && nbuf != n1) {  // histogram and scores disagree: flag it, stay in bounds

@@ -258,3 +258,23 @@ def test_full_budget_equals_dense():
 @pytest.mark.parametrize("keep", [50, 100])
 def test_llama8b_L32768_end_to_end(keep):
     _decode_e2e(S.LLAMA8B_L32K.with_(keep_pct=keep))
+
+
+def test_attention_on_an_empty_sequence_and_repeated_calls():
+    """A sequence with no cached token yields out = 0 and lse = -inf; the
+    split tickets reset themselves, so back-to-back calls agree."""
+    wl = SMALL_BF16.with_(lens=(1500, 0))
+    ctx = TB.Context(config_of(wl))
+    ld = make_layer(ctx, wl, 0, wl.seq_lens)
+    outs = []
+    for _ in range(3):
+        out = torch.full((wl.B, wl.Hq, wl.D), 7.0, dtype=torch.bfloat16, device="cuda")
+        lse = torch.zeros((wl.B, wl.Hq), device="cuda")
+        ctx.sparse_attn(0, ld.q_dev, None, TB.TB_MASK_DENSE, out, lse)
+        outs.append((out, lse))
+    torch.cuda.synchronize()
+    for out, lse in outs:
+        assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+        assert torch.equal(out, outs[0][0]) and torch.equal(lse, outs[0][1])
+    ref, ref_lse = O.attend(ld.q[0, 0], ld.K[0, 0, :1500], ld.V[0, 0, :1500], np.arange(1500), 1 / math.sqrt(wl.D))
+    assert_close_rows(outs[0][0][0, 0].float().cpu().numpy()[None], ref[None], "bf16")
