@@ -33,7 +33,8 @@
  *     after a synchronisation.  Nothing aborts, traps or throws.
  *   - Layouts are dense and row-major (last index fastest):
  *       K cache, V cache   [B][Hkv][max_len][D]   kv_dtype
- *       K_imp cache        [B][Hkv][max_len][d']  fp32 (always)
+ *       K_imp cache        [B][Hkv][d'][max_len]  fp32 (always), dimension-major:
+ *                          the tokens of one importance dimension are contiguous
  *       W_K                [D][d']                kv_dtype
  *       q_imp (producer)   [(B*Hq)][G][n][d']     kv_dtype  (model card: (B.H) x G x L x d')
  *       q, out             [B][Hq][D]             kv_dtype

@@ -132,14 +132,15 @@ __device__ __forceinline__ void write_partial(const AttnParams& p, int b, int g,
 // The last CTA of (b, g) to finish merges the split partials of the group's
 // heads with an fp32 log-sum-exp and writes out / lse.  Completion is counted
 // with an atomic ticket after a fence (no CTA waits on another); the ticket
-// is reset for the next call by the merging CTA.  Partials are read through
-// L2 (they were written by other SMs).
-constexpr int kMaxSplits = 1024;
+// is reset for the next call by the merging CTA.  Two dependent load phases:
+// the (m, l) pairs of every head and split, then the partial rows as float4.
+// Partials are read through L2 (they were written by other SMs).
+constexpr int kMaxSplits = 512;
 
 template <typename T, int D, int GS>
-__device__ __forceinline__ void merge_if_last(const AttnParams& p, int b, int g, int L, float* wts) {
+__device__ __forceinline__ void merge_if_last(const AttnParams& p, int b, int g, int L, float* scratch) {
   __shared__ int s_last;
-  __shared__ float red[kAttnWarps];
+  __shared__ float sM[GS], sL[GS];
   __threadfence();
   __syncthreads();
   const int ns = (L + p.chunk - 1) / p.chunk;
@@ -152,53 +153,59 @@ __device__ __forceinline__ void merge_if_last(const AttnParams& p, int b, int g,
   if (!s_last) return;
   __threadfence();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int hh = 0; hh < GS; ++hh) {
-    const int h = g * GS + hh;
-    const size_t ph = ((size_t)b * p.Hq + h) * p.nsplit;
+  float* wts = scratch;            // [GS][ns]: m, then the weights 2^(m - M)
+  float* lls = scratch + GS * ns;  // [GS][ns]
+  const size_t ph0 = ((size_t)b * p.Hq + g * GS) * p.nsplit;
+  for (int e = tid; e < GS * ns; e += kAttnThreads) {
+    const int hh = e / ns, sp = e - hh * ns;
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (ph0 + (size_t)hh * p.nsplit + sp) * 2));
+    wts[e] = v.x;
+    lls[e] = v.y;
+  }
+  __syncthreads();
+  for (int hh = warp; hh < GS; hh += kAttnWarps) {
     float M = kNegInf;
-    for (int sp = tid; sp < ns; sp += kAttnThreads) {
-      const float m = __ldcg(p.part_ml + (ph + sp) * 2);
-      wts[sp] = m;
-      M = fmaxf(M, m);
-    }
+    for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, wts[hh * ns + sp]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = red[0];
-#pragma unroll
-    for (int w = 1; w < kAttnWarps; ++w) M = fmaxf(M, red[w]);
-    __syncthreads();
     float lsum = 0.f;
-    for (int sp = tid; sp < ns; sp += kAttnThreads) {
-      const float m = wts[sp];
+    for (int sp = lane; sp < ns; sp += 32) {
+      const float m = wts[hh * ns + sp];
       const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
-      wts[sp] = f;
-      lsum += f * __ldcg(p.part_ml + (ph + sp) * 2 + 1);
+      wts[hh * ns + sp] = f;
+      lsum += f * lls[hh * ns + sp];
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    if (lane == 0) red[warp] = lsum;
-    __syncthreads();
-    lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) lsum += red[w];
-    for (int d = tid; d < D; d += kAttnThreads) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const float* po = p.part_o + ph * D + d;
-      int sp = 0;
-      for (; sp + 4 <= ns; sp += 4) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] += wts[sp + u] * __ldcg(po + (size_t)(sp + u) * D);
-      }
-      for (; sp < ns; ++sp) acc[0] += wts[sp] * __ldcg(po + (size_t)sp * D);
-      const float o = M == kNegInf ? 0.f : ((acc[0] + acc[1]) + (acc[2] + acc[3])) / lsum;
-      reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * D + d] = from_f32<T>(o);
+    if (lane == 0) {
+      sM[hh] = M;
+      sL[hh] = lsum;
     }
-    if (p.lse != nullptr && tid == 0)
-      p.lse[(size_t)b * p.Hq + h] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
-    __syncthreads();
   }
+  __syncthreads();
+  for (int e = tid; e < GS * (D / 4); e += kAttnThreads) {
+    const int hh = e / (D / 4), d4 = e - hh * (D / 4);
+    const float* po = p.part_o + (ph0 + (size_t)hh * p.nsplit) * D + 4 * d4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < ns; ++sp) {
+      const float w = wts[hh * ns + sp];
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(po + (size_t)sp * D));
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    const bool empty_set = sM[hh] == kNegInf;
+    const float inv = empty_set ? 0.f : 1.f / sL[hh];
+    T* dst = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + g * GS + hh) * D + 4 * d4;
+    dst[0] = from_f32<T>(acc.x * inv);
+    dst[1] = from_f32<T>(acc.y * inv);
+    dst[2] = from_f32<T>(acc.z * inv);
+    dst[3] = from_f32<T>(acc.w * inv);
+  }
+  if (p.lse != nullptr && tid < GS)
+    p.lse[(size_t)b * p.Hq + g * GS + tid] =
+        sM[tid] == kNegInf ? kNegInf : (sM[tid] + log2f(sL[tid])) * 0.69314718055994531f;
 }
 
 // An empty sequence has no split to merge: split 0 writes out = 0, lse = -inf.
@@ -388,14 +395,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
-  merge_if_last<__nv_bfloat16, D, GS>(p, b, g, L, wo + kAttnWarps * GS * D);
+  merge_if_last<__nv_bfloat16, D, GS>(p, b, g, L, reinterpret_cast<float*>(ring));
 }
 
 // ---------------------------------------------------------------- fp32 / FMA
 constexpr int kListBytes = ((kAttnMaxChunk + kAttnTile) * 5 + 15) / 16 * 16;
 template <int D>
 constexpr int attn_f32_smem_bytes() {
-  return kListBytes + kAttnWarps * 8 * (D + 2) * 4 + 1024 * 4;  // + split weights of the merge
+  // per-warp states, or the merge's (m, l) table of up to 8 heads x kMaxSplits
+  return kListBytes + (kAttnWarps * 8 * (D + 2) * 4 > 2 * 8 * kMaxSplits * 4 ? kAttnWarps * 8 * (D + 2) * 4
+                                                                            : 2 * 8 * kMaxSplits * 4);
 }
 
 // fp32 caches: one warp per token at a time, lane owns dims lane + 32 j.
@@ -468,7 +477,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
-  merge_if_last<float, D, GS>(p, b, g, L, wo + kAttnWarps * GS * D);
+  merge_if_last<float, D, GS>(p, b, g, L, wm);
 }
 
 }  // namespace tb

@@ -28,7 +28,7 @@ constexpr int kTcThreads = 192;
 
 struct ProjectTcParams {
   const void* w_k;  // [D][d'] bf16
-  float* kimp;      // [B][Hkv][max_len][d']
+  float* kimp;      // [B][Hkv][d'][max_len] (dimension-major)
   uint32_t* status;
   int max_len, start, count;
   int tiles_per_slab, total_tiles;
@@ -169,10 +169,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ntiles = p.total_tiles > (int)blockIdx.x
                          ? (p.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
                          : 0;
-  auto tile_of = [&](int j, int& row0, int& valid) {
+  // tile j of this CTA: K rows [t0, t0 + valid) of slab (b * Hkv + g); row0 is
+  // the same row in the flattened [B*Hkv*max_len][D] view used by TMA
+  auto tile_of = [&](int j, int& row0, int& valid, int& slab, int& t0) {
     const int i = blockIdx.x + j * gridDim.x;
-    const int slab = i / p.tiles_per_slab, tt = i % p.tiles_per_slab;
-    row0 = slab * p.max_len + p.start + tt * kTcRows;
+    slab = i / p.tiles_per_slab;
+    const int tt = i % p.tiles_per_slab;
+    t0 = p.start + tt * kTcRows;
+    row0 = slab * p.max_len + t0;
     valid = min(kTcRows, p.count - tt * kTcRows);
   };
 
@@ -184,8 +188,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *s_abort = 1;
           break;
         }
-        int row0, valid;
-        tile_of(j, row0, valid);
+        int row0, valid, slab, t0;
+        tile_of(j, row0, valid, slab, t0);
         mbar_expect_tx(&full[st], A_STAGE);
 #pragma unroll
         for (int a = 0; a < ATOMS; ++a) tma_load_2d(A + st * A_STAGE + a * A_ATOM, &kmap, a * 64, row0, &full[st]);
@@ -237,13 +241,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cta(&acce[acc]);
-      int row0, valid;
-      tile_of(j, row0, valid);
+      int row0, valid, slab, t0;
+      tile_of(j, row0, valid, slab, t0);
       const int r = quarter * 32 + lane;
       if (r < valid) {
-        float4* dst = reinterpret_cast<float4*>(p.kimp + ((size_t)row0 + r) * DIMP);
+        // dimension-major store: for each column the warp writes 32 consecutive tokens
+        float* dst = p.kimp + (size_t)slab * DIMP * p.max_len + t0 + r;
 #pragma unroll
-        for (int c = 0; c < DIMP / 4; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        for (int c = 0; c < DIMP; ++c) dst[(size_t)c * p.max_len] = v[c];
       }
     }
   }

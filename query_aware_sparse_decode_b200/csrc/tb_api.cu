@@ -30,7 +30,6 @@ struct LayerState {
   float* kimp = nullptr;
   const void* wk = nullptr;
   bool bound = false;
-  CUtensorMap kimp_map;
   CUtensorMap k_map;  // bf16 caches: K rows, 64-column boxes of 128 rows, 128B swizzle
   int lens[TB_MAX_BATCH];
 };
@@ -148,9 +147,9 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const LayerState& ls = ctx->layers[layer];
   ScoreParams p{};
   p.q_imp = q_imp;
+  p.kimp = ls.kimp;
   p.scores = scores;
   p.hist = hist;
-  p.status = ctx->status;
   p.G = c.producer_freq;
   p.slot = ((layer - 1) % c.producer_freq + c.producer_freq) % c.producer_freq;
   p.Hq = c.n_q_heads;
@@ -158,52 +157,47 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.max_len = c.max_len;
   p.sink = c.sink;
   p.window = c.window;
-  p.tile_base[0] = 0;
-  for (int b = 0; b < TB_MAX_BATCH; ++b) {
-    const int L = b < c.batch ? ls.lens[b] : 0;
-    p.lens[b] = L;
-    p.tile_base[b + 1] = p.tile_base[b] + c.n_kv_heads * ((L + kScoreTile - 1) / kScoreTile);
-  }
-  p.total_tiles = p.tile_base[TB_MAX_BATCH];
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   if (hist) {
     const size_t n = (size_t)c.batch * c.n_q_heads * kHistBins;
     zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(hist, n);
     ++ctx->launches;
   }
-  if (p.total_tiles == 0) return cuda_status(cudaGetLastError());
-  const int grid = std::min(p.total_tiles, ctx->num_sms);
+  const int maxL = max_len_of(ls, c.batch);
+  if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
-  const size_t smem = 1024 + (size_t)kScoreStages * kScoreTile * c.d_imp * 4 + (2 * kScoreStages + 1) * 8 +
-                      (hist ? (size_t)gs * kHistBins * 4 : 0);
-#define TB_SCORE_CASE(T, DI, GSV)                                                                          \
-  if (c.d_imp == DI && gs == GSV) {                                                                        \
-    if (hist) {                                                                                            \
-      auto k = score_kernel<T, DI, GSV, true>;                                                             \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      k<<<grid, kScoreThreads, smem, st>>>(ls.kimp_map, p);                                                   \
-      ++ctx->launches;                                                                                     \
-    } else {                                                                                               \
-      auto k = score_kernel<T, DI, GSV, false>;                                                            \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                     \
-      k<<<grid, kScoreThreads, smem, st>>>(ls.kimp_map, p);                                                   \
-      ++ctx->launches;                                                                                     \
-    }                                                                                                      \
-    return cuda_status(cudaGetLastError());                                                                \
+  const size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
+  dim3 grid((maxL + kScoreChunk - 1) / kScoreChunk, c.n_kv_heads, c.batch);
+#define TB_SCORE_CASE(T, DI, GSV)                                                            \
+  if (c.d_imp == DI && gs == GSV) {                                                          \
+    if (hist) {                                                                              \
+      auto k = score_kernel<T, DI, GSV, true>;                                               \
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);       \
+      k<<<grid, kScoreThreads, smem, st>>>(p);                                               \
+    } else {                                                                                 \
+      score_kernel<T, DI, GSV, false><<<grid, kScoreThreads, 0, st>>>(p);                    \
+    }                                                                                        \
+    ++ctx->launches;                                                                         \
+    return cuda_status(cudaGetLastError());                                                  \
   }
   if (c.kv_dtype == TB_BF16) {
     TB_SCORE_CASE(__nv_bfloat16, 32, 4)
     TB_SCORE_CASE(__nv_bfloat16, 32, 2)
     TB_SCORE_CASE(__nv_bfloat16, 32, 1)
+    TB_SCORE_CASE(__nv_bfloat16, 32, 8)
     TB_SCORE_CASE(__nv_bfloat16, 16, 4)
     TB_SCORE_CASE(__nv_bfloat16, 16, 2)
     TB_SCORE_CASE(__nv_bfloat16, 16, 1)
+    TB_SCORE_CASE(__nv_bfloat16, 16, 8)
   } else {
     TB_SCORE_CASE(float, 32, 4)
     TB_SCORE_CASE(float, 32, 2)
     TB_SCORE_CASE(float, 32, 1)
+    TB_SCORE_CASE(float, 32, 8)
     TB_SCORE_CASE(float, 16, 4)
     TB_SCORE_CASE(float, 16, 2)
     TB_SCORE_CASE(float, 16, 1)
+    TB_SCORE_CASE(float, 16, 8)
   }
 #undef TB_SCORE_CASE
   return TB_ERR_UNSUPPORTED;
@@ -263,6 +257,7 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   const int groups = c.batch * c.n_kv_heads;
   const int want_split = std::max(1, (4 * ctx->num_sms + groups - 1) / groups);
   int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
+  chunk = std::max(chunk, (maxL + kMaxSplits - 1) / kMaxSplits);  // at most kMaxSplits splits
   chunk = std::min(kAttnMaxChunk, std::max(256, (chunk + 255) / 256 * 256));
   p.chunk = chunk;
   p.nsplit = std::max(1, (maxL + chunk - 1) / chunk);
@@ -393,15 +388,8 @@ TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_ca
   LayerState& ls = ctx->layers[layer];
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return TB_ERR_CUDA;
-  cuuint64_t gdim[2] = {(cuuint64_t)c.d_imp, (cuuint64_t)c.batch * c.n_kv_heads * c.max_len};
-  cuuint64_t gstride[1] = {(cuuint64_t)c.d_imp * 4};
-  cuuint32_t box[2] = {(cuuint32_t)c.d_imp, (cuuint32_t)kScoreTile};
   cuuint32_t estride[2] = {1, 1};
-  CUresult r = enc(&ls.kimp_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, kimp_cache, gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   c.d_imp == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return TB_ERR_CUDA;
+  CUresult r = CUDA_SUCCESS;
   if (c.kv_dtype == TB_BF16) {
     cuuint64_t kdim[2] = {(cuuint64_t)c.head_dim, (cuuint64_t)c.batch * c.n_kv_heads * c.max_len};
     cuuint64_t kstride[1] = {(cuuint64_t)c.head_dim * 2};

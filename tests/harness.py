@@ -73,7 +73,7 @@ def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerDat
     v_cache = torch.zeros_like(k_cache)
     k_cache[:, :, :Lfill] = to_dev(K_raw, wl)
     v_cache[:, :, :Lfill] = to_dev(V_raw, wl)
-    kimp = torch.zeros((B, Hkv, Lmax, dimp), dtype=torch.float32, device="cuda")
+    kimp = torch.zeros((B, Hkv, dimp, Lmax), dtype=torch.float32, device="cuda")  # dimension-major
     w_k = to_dev(W_raw, wl)
     ctx.bind_layer(layer, k_cache, v_cache, kimp, w_k)
     ctx.set_seq_lens(layer, lens)
