@@ -158,7 +158,7 @@ def build(wl, max_len, dev):
     for layer in range(wl.n_layers):
         k = torch.empty((wl.B, wl.Hkv, max_len, wl.D), dtype=torch.bfloat16, device=dev)
         v = torch.empty_like(k)
-        kimp = torch.empty((wl.B, wl.Hkv, wl.d_imp, max_len), dtype=torch.float32, device=dev)
+        kimp = torch.empty((wl.B, wl.Hkv, max_len // 256, wl.d_imp, 256), dtype=torch.float32, device=dev)
         w_raw = S.w_k(wl, layer)
         w = torch.from_numpy(w_raw.view(np.int16)).view(torch.bfloat16).to(dev)
         delta = None

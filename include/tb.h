@@ -33,8 +33,9 @@
  *     after a synchronisation.  Nothing aborts, traps or throws.
  *   - Layouts are dense and row-major (last index fastest):
  *       K cache, V cache   [B][Hkv][max_len][D]   kv_dtype
- *       K_imp cache        [B][Hkv][d'][max_len]  fp32 (always), dimension-major:
- *                          the tokens of one importance dimension are contiguous
+ *       K_imp cache        [B][Hkv][max_len/256][d'][256]  fp32 (always): tiles of
+ *                          256 tokens, each contiguous and dimension-major
+ *                          (element (b, g, t, j) at tile t/256, row j, column t%256)
  *       W_K                [D][d']                kv_dtype
  *       q_imp (producer)   [(B*Hq)][G][n][d']     kv_dtype  (model card: (B.H) x G x L x d')
  *       q, out             [B][Hq][D]             kv_dtype

@@ -33,9 +33,6 @@ struct AttnParams {
   const uint32_t* mask;  // per mask_mode
   float* part_o;         // [B][Hq][nsplit][D]
   float* part_ml;        // [B][Hq][nsplit][2]: running max (log2 domain), sum
-  uint32_t* tickets;     // [B][Hkv] split-completion counters (zero between calls)
-  void* out;             // [B][Hq][D] kv dtype
-  float* lse;            // [B][Hq] or nullptr
   uint32_t* status;
   int mask_mode, mask_words;
   int Hq, Hkv, max_len, chunk, nsplit;
@@ -129,94 +126,7 @@ __device__ __forceinline__ void write_partial(const AttnParams& p, int b, int g,
 }
 
 
-// The last CTA of (b, g) to finish merges the split partials of the group's
-// heads with an fp32 log-sum-exp and writes out / lse.  Completion is counted
-// with an atomic ticket after a fence (no CTA waits on another); the ticket
-// is reset for the next call by the merging CTA.  Two dependent load phases:
-// the (m, l) pairs of every head and split, then the partial rows as float4.
-// Partials are read through L2 (they were written by other SMs).
 constexpr int kMaxSplits = 512;
-
-template <typename T, int D, int GS>
-__device__ __forceinline__ void merge_if_last(const AttnParams& p, int b, int g, int L, float* scratch) {
-  __shared__ int s_last;
-  __shared__ float sM[GS], sL[GS];
-  __threadfence();
-  __syncthreads();
-  const int ns = (L + p.chunk - 1) / p.chunk;
-  if (threadIdx.x == 0) {
-    const uint32_t prev = atomicAdd(&p.tickets[b * p.Hkv + g], 1u);
-    s_last = prev == (uint32_t)(ns - 1);
-    if (s_last) p.tickets[b * p.Hkv + g] = 0u;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* wts = scratch;            // [GS][ns]: m, then the weights 2^(m - M)
-  float* lls = scratch + GS * ns;  // [GS][ns]
-  const size_t ph0 = ((size_t)b * p.Hq + g * GS) * p.nsplit;
-  for (int e = tid; e < GS * ns; e += kAttnThreads) {
-    const int hh = e / ns, sp = e - hh * ns;
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (ph0 + (size_t)hh * p.nsplit + sp) * 2));
-    wts[e] = v.x;
-    lls[e] = v.y;
-  }
-  __syncthreads();
-  for (int hh = warp; hh < GS; hh += kAttnWarps) {
-    float M = kNegInf;
-    for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, wts[hh * ns + sp]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float lsum = 0.f;
-    for (int sp = lane; sp < ns; sp += 32) {
-      const float m = wts[hh * ns + sp];
-      const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
-      wts[hh * ns + sp] = f;
-      lsum += f * lls[hh * ns + sp];
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    if (lane == 0) {
-      sM[hh] = M;
-      sL[hh] = lsum;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < GS * (D / 4); e += kAttnThreads) {
-    const int hh = e / (D / 4), d4 = e - hh * (D / 4);
-    const float* po = p.part_o + (ph0 + (size_t)hh * p.nsplit) * D + 4 * d4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < ns; ++sp) {
-      const float w = wts[hh * ns + sp];
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(po + (size_t)sp * D));
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
-    }
-    const bool empty_set = sM[hh] == kNegInf;
-    const float inv = empty_set ? 0.f : 1.f / sL[hh];
-    T* dst = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + g * GS + hh) * D + 4 * d4;
-    dst[0] = from_f32<T>(acc.x * inv);
-    dst[1] = from_f32<T>(acc.y * inv);
-    dst[2] = from_f32<T>(acc.z * inv);
-    dst[3] = from_f32<T>(acc.w * inv);
-  }
-  if (p.lse != nullptr && tid < GS)
-    p.lse[(size_t)b * p.Hq + g * GS + tid] =
-        sM[tid] == kNegInf ? kNegInf : (sM[tid] + log2f(sL[tid])) * 0.69314718055994531f;
-}
-
-// An empty sequence has no split to merge: split 0 writes out = 0, lse = -inf.
-template <typename T, int D, int GS>
-__device__ __forceinline__ void write_empty(const AttnParams& p, int b, int g) {
-  for (int e = threadIdx.x; e < GS * D; e += kAttnThreads) {
-    const int h = g * GS + e / D;
-    reinterpret_cast<T*>(p.out)[((size_t)b * p.Hq + h) * D + e % D] = from_f32<T>(0.f);
-    if (p.lse != nullptr && e % D == 0) p.lse[(size_t)b * p.Hq + h] = kNegInf;
-  }
-}
 
 // ---------------------------------------------------------------- bf16 / mma.sync
 template <int D>
@@ -242,7 +152,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.lens[b];
   const int t0 = split * p.chunk;
-  if (L == 0 && split == 0) write_empty<__nv_bfloat16, D, GS>(p, b, g);
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
   const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
@@ -395,16 +304,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
-  merge_if_last<__nv_bfloat16, D, GS>(p, b, g, L, reinterpret_cast<float*>(ring));
 }
 
 // ---------------------------------------------------------------- fp32 / FMA
 constexpr int kListBytes = ((kAttnMaxChunk + kAttnTile) * 5 + 15) / 16 * 16;
 template <int D>
 constexpr int attn_f32_smem_bytes() {
-  // per-warp states, or the merge's (m, l) table of up to 8 heads x kMaxSplits
-  return kListBytes + (kAttnWarps * 8 * (D + 2) * 4 > 2 * 8 * kMaxSplits * 4 ? kAttnWarps * 8 * (D + 2) * 4
-                                                                            : 2 * 8 * kMaxSplits * 4);
+  return kListBytes + kAttnWarps * 8 * (D + 2) * 4;
 }
 
 // fp32 caches: one warp per token at a time, lane owns dims lane + 32 j.
@@ -422,7 +328,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.lens[b];
   const int t0 = split * p.chunk;
-  if (L == 0 && split == 0) write_empty<float, D, GS>(p, b, g);
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
   const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
@@ -477,7 +382,76 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
-  merge_if_last<float, D, GS>(p, b, g, L, wm);
+}
+
+// ---------------------------------------------------------------- combine
+struct CombineParams {
+  const float* part_o;
+  const float* part_ml;
+  void* out;   // [B][Hq][D] kv dtype
+  float* lse;  // [B][Hq] or nullptr
+  int B, Hq, chunk, nsplit;
+  int lens[kMaxBatch];
+};
+
+// fp32 log-sum-exp merge of the split partials: one warp per (b, h), four
+// per CTA.  Two dependent load phases: every split's (m, l), then the partial
+// rows (each lane owns D/32 consecutive dimensions).  An empty set gives
+// out = 0 and lse = -inf.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+  constexpr int DPL = D / 32;
+  __shared__ float sw[4][kMaxSplits];
+  __shared__ float sl[4][kMaxSplits];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x * 4 + warp;
+  if (bh >= p.B * p.Hq) return;
+  const int b = bh / p.Hq;
+  const int L = p.lens[b];
+  const int ns = (L + p.chunk - 1) / p.chunk;
+  const size_t ph = (size_t)bh * p.nsplit;
+  float M = kNegInf;
+  for (int sp = lane; sp < ns; sp += 32) {
+    const float2 v = *reinterpret_cast<const float2*>(p.part_ml + (ph + sp) * 2);
+    sw[warp][sp] = v.x;
+    sl[warp][sp] = v.y;
+    M = fmaxf(M, v.x);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float lsum = 0.f;
+  for (int sp = lane; sp < ns; sp += 32) {
+    const float m = sw[warp][sp];
+    const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
+    sw[warp][sp] = f;
+    lsum += f * sl[warp][sp];
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  __syncwarp();
+  float acc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+  const float* po = p.part_o + ph * D + lane * DPL;
+  for (int sp = 0; sp < ns; ++sp) {
+    const float w = sw[warp][sp];
+    if constexpr (DPL == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)sp * D);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+    }
+  }
+  const float inv = M == kNegInf ? 0.f : 1.f / lsum;
+  T* dst = reinterpret_cast<T*>(p.out) + (size_t)bh * D + lane * DPL;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) dst[i] = from_f32<T>(acc[i] * inv);
+  if (p.lse != nullptr && lane == 0) p.lse[bh] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
 }
 
 }  // namespace tb

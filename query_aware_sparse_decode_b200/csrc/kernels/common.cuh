@@ -12,6 +12,14 @@ namespace tb {
 
 constexpr int kMaxBatch = TB_MAX_BATCH;
 constexpr int kHistBins = 2048;  // 11-bit first radix digit of the selection
+
+// K_imp cache layout [B][Hkv][max_len/256][d'][256]: tiles of 256 tokens, each
+// a contiguous block, dimension-major inside the tile.  Element (slab, j, t)
+// with slab = b * Hkv + g:
+constexpr int kKimpTile = 256;
+__host__ __device__ __forceinline__ size_t kimp_index(size_t slab, int j, int t, int dimp, int max_len) {
+  return slab * (size_t)max_len * dimp + (size_t)(t >> 8) * dimp * kKimpTile + (size_t)j * kKimpTile + (t & 255);
+}
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // ------------------------------------------------------------ order keys

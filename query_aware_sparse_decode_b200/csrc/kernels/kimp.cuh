@@ -13,7 +13,7 @@ struct AppendParams {
   const void* v_new;  // [B][Hkv][D]
   void* k_cache;      // [B][Hkv][max_len][D]
   void* v_cache;
-  float* kimp;        // [B][Hkv][d'][max_len] (dimension-major)
+  float* kimp;        // [B][Hkv][max_len/256][d'][256] (kimp_index)
   const void* w_k;    // [D][d']
   int Hkv, D, dimp, max_len;
   int pos[kMaxBatch];  // row written for sequence b (its length before the append)
@@ -50,13 +50,13 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   if (tid < p.dimp) {
     float sum = 0.f;
     for (int i = 0; i < parts; ++i) sum += part[i * p.dimp + tid];
-    p.kimp[(((size_t)b * p.Hkv + g) * p.dimp + tid) * p.max_len + p.pos[b]] = sum;
+    p.kimp[kimp_index((size_t)b * p.Hkv + g, tid, p.pos[b], p.dimp, p.max_len)] = sum;
   }
 }
 
 struct ProjectParams {
   const void* k_cache;  // [B][Hkv][max_len][D]
-  float* kimp;          // [B][Hkv][d'][max_len] (dimension-major)
+  float* kimp;          // [B][Hkv][max_len/256][d'][256] (kimp_index)
   const void* w_k;      // [D][d']
   int Hkv, max_len, start, count;
 };
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(256) project_fma_kernel(const ProjectParams p)
   if (r < rend) {
     const size_t slab = (size_t)b * p.Hkv + g;
 #pragma unroll
-    for (int j = 0; j < OUT_PER_THREAD; ++j) p.kimp[(slab * DIMP + j0 + j) * p.max_len + r0 + r] = acc[j];
+    for (int j = 0; j < OUT_PER_THREAD; ++j) p.kimp[kimp_index(slab, j0 + j, r0 + r, DIMP, p.max_len)] = acc[j];
   }
 }
 

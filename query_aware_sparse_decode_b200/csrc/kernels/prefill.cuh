@@ -19,7 +19,7 @@ namespace tb {
 
 struct PrefillParams {
   const void* q_imp;   // [(B*Hq)][G][nrows][d'] kv dtype
-  const float* kimp;   // [B][Hkv][d'][max_len] (dimension-major)
+  const float* kimp;   // [B][Hkv][max_len/256][d'][256] (kimp_index)
   uint32_t* masks;     // [B][Hq][nrows][words_per_row]
   uint32_t* status;
   int G, slot, Hq, Hkv, max_len, row0, nrows, words_per_row;
@@ -43,11 +43,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) prefill_select_kernel(const Pr
     q[tid] = to_f32(reinterpret_cast<const TQ*>(p.q_imp)[((((size_t)b * p.Hq + h) * p.G + p.slot) * p.nrows + r) * DIMP +
                                                          tid]);
   __syncthreads();
-  const float* K = p.kimp + ((size_t)b * p.Hkv + g) * DIMP * p.max_len;
+  const size_t slab = (size_t)b * p.Hkv + g;
   for (int t = tid; t < L; t += kSelThreads) {
+    const float* K = p.kimp + kimp_index(slab, 0, t, DIMP, p.max_len);
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < DIMP; ++j) acc = fmaf(q[j], K[(size_t)j * p.max_len + t], acc);
+    for (int j = 0; j < DIMP; ++j) acc = fmaf(q[j], K[j * kKimpTile], acc);
     srow[t] = acc;
   }
   __syncthreads();

@@ -28,7 +28,7 @@ constexpr int kTcThreads = 192;
 
 struct ProjectTcParams {
   const void* w_k;  // [D][d'] bf16
-  float* kimp;      // [B][Hkv][d'][max_len] (dimension-major)
+  float* kimp;      // [B][Hkv][max_len/256][d'][256] (kimp_index)
   uint32_t* status;
   int max_len, start, count;
   int tiles_per_slab, total_tiles;
@@ -245,10 +245,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tile_of(j, row0, valid, slab, t0);
       const int r = quarter * 32 + lane;
       if (r < valid) {
-        // dimension-major store: for each column the warp writes 32 consecutive tokens
-        float* dst = p.kimp + (size_t)slab * DIMP * p.max_len + t0 + r;
+        // for each column the warp writes 32 consecutive tokens of one tile
+        float* dst = p.kimp + kimp_index(slab, 0, t0 + r, DIMP, p.max_len);
 #pragma unroll
-        for (int c = 0; c < DIMP; ++c) dst[(size_t)c * p.max_len] = v[c];
+        for (int c = 0; c < DIMP; ++c) dst[c * kKimpTile] = v[c];
       }
     }
   }

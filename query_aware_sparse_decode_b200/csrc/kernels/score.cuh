@@ -3,8 +3,8 @@
 // "Method": a consumer scores every cached token with its producer's
 // importance query, slot (l - 1) mod G).
 //
-// HBM stream over K_imp, which is stored dimension-major ([b][g][j][t]: the
-// tokens of one importance dimension are contiguous), read once per KV head
+// HBM stream over K_imp, stored as contiguous 256-token tiles, dimension-major
+// inside a tile ([b][g][t/256][j][t%256], see kimp_index), read once per KV head
 // and shared by the Hq/Hkv query heads of the group.  A thread scores four
 // consecutive tokens: d' independent, coalesced 16-byte loads per group of
 // four tokens, fp32 FMA in dimension order j = 0..d'-1, the group's query
@@ -25,7 +25,7 @@ constexpr int kScoreChunk = kScoreThreads * 4 * kScoreIters;    // tokens per CT
 
 struct ScoreParams {
   const void* q_imp;   // [(B*Hq)][G][1][d'] of the producer, kv dtype
-  const float* kimp;   // [B][Hkv][d'][max_len]
+  const float* kimp;   // [B][Hkv][max_len/256][d'][256]
   float* scores;       // [B][Hq][max_len]
   uint32_t* hist;      // [B*Hq][2048] or nullptr
   int G, slot, Hq, Hkv, max_len;
@@ -50,18 +50,19 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
     for (int e = tid; e < GS * kHistBins; e += kScoreThreads) hist[e] = 0;
   __syncthreads();
 
-  const float* K = p.kimp + ((size_t)b * p.Hkv + g) * DIMP * p.max_len;
+  const size_t slab = (size_t)b * p.Hkv + g;
   float* S = p.scores + ((size_t)b * p.Hq + g * GS) * p.max_len;
 #pragma unroll 1
   for (int it = 0; it < kScoreIters; ++it) {
     const int t0 = t_base + it * 4 * kScoreThreads + 4 * tid;
     if (t0 < L) {
+      const float* K = p.kimp + kimp_index(slab, 0, t0, DIMP, p.max_len);
       float acc[GS][4];
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh) acc[hh][0] = acc[hh][1] = acc[hh][2] = acc[hh][3] = 0.f;
-#pragma unroll 8
+#pragma unroll
       for (int j = 0; j < DIMP; ++j) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(K + (size_t)j * p.max_len + t0));
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(K + j * kKimpTile));
 #pragma unroll
         for (int hh = 0; hh < GS; ++hh) {
           const float qv = qs[j][hh];

@@ -78,6 +78,12 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint3
   __syncthreads();
 }
 
+// Inverse of order_key (for keys of finite floats).
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -141,77 +147,84 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   uint32_t T = 0, quota = 0;
   if (fast) {
     // ---- one ordered sweep: sure bits into the shared mask, bin-b1 candidates
-    // into the buffer.  An iteration covers 4 chunks of 4096 tokens; thread
-    // tid owns tokens 4*tid..4*tid+3 of every chunk (coalesced float4 loads),
-    // and the next iteration's loads are issued before this one is processed.
-    constexpr int CH = 4;
-    constexpr int ITER = CH * 4 * kSelThreads;
+    // into the buffer.  Lane = token: an iteration covers STEPS x 1024 tokens,
+    // step j of warp w holds tokens base + j*1024 + w*32 + lane, so a ballot
+    // is one mask word.  The threshold-bin test is two float compares against
+    // the bin's boundary values (the key map is monotone; -0.0 == +0.0 holds
+    // for both).  Candidates keep index order through a (step, warp) prefix.
+    constexpr int STEPS = 16;
+    constexpr int ITER = STEPS * kSelThreads;
+    const int warp = tid >> 5;
+    const float f_lo = key_to_float((uint32_t)b1 << 21);         // smallest key of bin b1
+    const float f_hi = key_to_float(((uint32_t)b1 + 1u) << 21);  // smallest key above bin b1
+    const bool hi_open = b1 == (int)(kHistBins - 1);             // no key lies above the top bin
     uint32_t nbuf = 0;
-    float4 cur[CH], nxt[CH];
-    auto load_iter = [&](int base, float4 (&dst)[CH]) {
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int t0 = base + c * 4 * kSelThreads + 4 * tid;
-        dst[c] = (mode == 2 && t0 < L) ? *reinterpret_cast<const float4*>(s + t0) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    };
-    load_iter(0, cur);
+    uint32_t* wcnt = hist;  // [STEPS][32] candidate counts per (step, warp); hist is free during the sweep
     for (int base = 0; base < L; base += ITER) {
-      if (base + ITER < L) load_iter(base + ITER, nxt);
-      uint32_t cbits[CH];
+      float v[STEPS];
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int t0 = base + c * 4 * kSelThreads + 4 * tid;
-        const float vv[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
-        uint32_t keepbits = 0;
-        cbits[c] = 0;
+      for (int j = 0; j < STEPS; ++j) {
+        const int t = base + j * kSelThreads + tid;
+        v[j] = (mode == 2 && t < L) ? s[t] : 0.f;
+      }
+      uint32_t cmask[STEPS];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int t = t0 + j;
-          if (t >= L) continue;
-          const bool cand = t >= lo && t < hi;
-          bool keep = !cand || mode == 1;
-          if (cand && mode == 2) {
-            const uint32_t d1 = order_key(vv[j]) >> 21;
-            if (d1 > (uint32_t)b1) keep = true;
-            else if (d1 == (uint32_t)b1) cbits[c] |= 1u << j;
-          }
-          if (keep) keepbits |= 1u << j;
+      for (int j = 0; j < STEPS; ++j) {
+        const int t = base + j * kSelThreads + tid;
+        const bool in = t < L;
+        const bool cand = t >= lo && t < hi;
+        bool keep = in && (!cand || mode == 1);
+        bool c = false;
+        if (mode == 2 && in && cand) {
+          const bool above = !hi_open && v[j] >= f_hi;
+          keep = above;
+          c = !above && v[j] >= f_lo;
         }
-        uint32_t word = keepbits << ((lane & 7) * 4);
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        const int w = ((base + c * 4 * kSelThreads) >> 5) + (tid >> 3);
-        if ((lane & 7) == 0 && w < lwords) smask[w] = word;
+        const uint32_t word = __ballot_sync(0xffffffffu, keep);
+        const int w = (base + j * kSelThreads) / 32 + warp;
+        if (lane == 0 && w < lwords) smask[w] = word;
+        cmask[j] = __ballot_sync(0xffffffffu, c);
       }
       if (mode == 2) {
-        uint2 tot;
-        const uint2 ex = block_excl_scan2<kSelThreads>(
-            make_uint2(__popc(cbits[0]) | (__popc(cbits[1]) << 16), __popc(cbits[2]) | (__popc(cbits[3]) << 16)),
-            tot, scan2_sm);
-        const uint32_t t0c = tot.x & 0xFFFFu, t1c = tot.x >> 16, t2c = tot.y & 0xFFFFu, t3c = tot.y >> 16;
-        const uint32_t start[CH] = {nbuf + (ex.x & 0xFFFFu), nbuf + t0c + (ex.x >> 16),
-                                    nbuf + t0c + t1c + (ex.y & 0xFFFFu), nbuf + t0c + t1c + t2c + (ex.y >> 16)};
+        __syncthreads();  // previous users of wcnt are done
+        if (lane < STEPS) {
+          uint32_t cnt = 0;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          uint32_t pos = start[c];
-          const int t0 = base + c * 4 * kSelThreads + 4 * tid;
-          const float vv[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (cbits[c] & (1u << j)) {
-              if (pos < (uint32_t)kSelCap) {
-                ckey[pos] = order_key(vv[j]);
-                cidx[pos] = (uint32_t)(t0 + j);
-              }
-              ++pos;
-            }
+          for (int j = 0; j < STEPS; ++j) cnt = j == lane ? __popc(cmask[j]) : cnt;
+          wcnt[lane * 32 + warp] = cnt;
         }
-        nbuf += t0c + t1c + t2c + t3c;
-      }
+        __syncthreads();
+        if (warp < STEPS) {  // warp j: exclusive prefix over the 32 warps of step j
+          const uint32_t c = wcnt[warp * 32 + lane];
+          uint32_t x = c;
 #pragma unroll
-      for (int c = 0; c < CH; ++c) cur[c] = nxt[c];
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          wcnt[warp * 32 + lane] = x - c;
+          if (lane == 31) scan_sm[warp] = x;  // step total
+        }
+        __syncthreads();
+        uint32_t step_base[STEPS];
+        uint32_t run = nbuf;
+#pragma unroll
+        for (int j = 0; j < STEPS; ++j) {
+          step_base[j] = run;
+          run += scan_sm[j];
+        }
+#pragma unroll
+        for (int j = 0; j < STEPS; ++j) {
+          if (cmask[j] & (1u << lane)) {
+            const uint32_t pos = step_base[j] + wcnt[j * 32 + warp] + __popc(cmask[j] & lanemask_lt());
+            if (pos < (uint32_t)kSelCap) {
+              ckey[pos] = order_key(v[j]);
+              cidx[pos] = (uint32_t)(base + j * kSelThreads + tid);
+            }
+          }
+        }
+        nbuf = run;
+      }
     }
     __syncthreads();
     if (mode == 2 && nbuf != n1) {  // histogram and scores disagree: flag it, stay in bounds

@@ -37,7 +37,7 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, tickets, hist, scores, mask, part_o, part_ml, votes, vstats, total;
+  size_t status, hist, scores, mask, part_o, part_ml, votes, vstats, total;
   int max_splits;
 };
 
@@ -47,7 +47,6 @@ WsLayout layout_of(const tb_config& c) {
   w.max_splits = (int)((Lm + 255) / 256);
   size_t off = 0;
   w.status = off;  off += align256(256);
-  w.tickets = off; off += align256(B * c.n_kv_heads * 4);
   w.hist = off;    off += align256(B * Hq * kHistBins * 4);
   w.scores = off;  off += align256(B * Hq * Lm * 4);
   w.mask = off;    off += align256(B * Hq * (Lm / 32) * 4);
@@ -87,7 +86,6 @@ struct tb_ctx {
   char* ws = nullptr;
   WsLayout lay;
   uint32_t* status = nullptr;
-  uint32_t* tickets = nullptr;
   uint32_t* hist = nullptr;
   float* scores = nullptr;
   uint32_t* mask = nullptr;
@@ -242,9 +240,6 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   p.mask = mask;
   p.part_o = ctx->part_o;
   p.part_ml = ctx->part_ml;
-  p.tickets = ctx->tickets;
-  p.out = out;
-  p.lse = lse;
   p.status = ctx->status;
   p.mask_mode = mode;
   p.mask_words = c.max_len / 32;
@@ -288,7 +283,26 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
     if (s != TB_OK) return s;
   }
   trace_point(ctx, 4, st);
-  trace_point(ctx, 5, st);  // the split merge runs inside the attention kernel
+  CombineParams cp{};
+  cp.part_o = ctx->part_o;
+  cp.part_ml = ctx->part_ml;
+  cp.out = out;
+  cp.lse = lse;
+  cp.B = c.batch;
+  cp.Hq = c.n_q_heads;
+  cp.chunk = chunk;
+  cp.nsplit = p.nsplit;
+  for (int b = 0; b < c.batch; ++b) cp.lens[b] = ls.lens[b];
+  const unsigned cgrid = (unsigned)((c.batch * c.n_q_heads + 3) / 4);
+  if (c.kv_dtype == TB_BF16) {
+    if (c.head_dim == 128) combine_kernel<__nv_bfloat16, 128><<<cgrid, 128, 0, st>>>(cp);
+    else combine_kernel<__nv_bfloat16, 64><<<cgrid, 128, 0, st>>>(cp);
+  } else {
+    if (c.head_dim == 128) combine_kernel<float, 128><<<cgrid, 128, 0, st>>>(cp);
+    else combine_kernel<float, 64><<<cgrid, 128, 0, st>>>(cp);
+  }
+  ++ctx->launches;
+  trace_point(ctx, 5, st);
   return cuda_status(cudaGetLastError());
 }
 
@@ -362,7 +376,6 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   }
   ctx->ws = static_cast<char*>(workspace);
   ctx->status = reinterpret_cast<uint32_t*>(ctx->ws + lay.status);
-  ctx->tickets = reinterpret_cast<uint32_t*>(ctx->ws + lay.tickets);
   ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
   ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
   ctx->mask = reinterpret_cast<uint32_t*>(ctx->ws + lay.mask);
@@ -370,8 +383,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
   ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
   ctx->vstats = reinterpret_cast<float*>(ctx->ws + lay.vstats);
-  // status word and split tickets start at zero (the attention kernel resets its tickets)
-  if (cudaMemset(ctx->ws, 0, lay.hist) != cudaSuccess) {
+  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return TB_ERR_CUDA;
   }

@@ -73,12 +73,23 @@ def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerDat
     v_cache = torch.zeros_like(k_cache)
     k_cache[:, :, :Lfill] = to_dev(K_raw, wl)
     v_cache[:, :, :Lfill] = to_dev(V_raw, wl)
-    kimp = torch.zeros((B, Hkv, dimp, Lmax), dtype=torch.float32, device="cuda")  # dimension-major
+    kimp = kimp_alloc(B, Hkv, dimp, Lmax)
     w_k = to_dev(W_raw, wl)
     ctx.bind_layer(layer, k_cache, v_cache, kimp, w_k)
     ctx.set_seq_lens(layer, lens)
     return LayerData(layer, W, qimp, qhat, S.widen(q_raw, wl.dtype), S.widen(K_raw, wl.dtype),
                      S.widen(V_raw, wl.dtype), k_cache, v_cache, kimp, w_k, to_dev(qimp_raw, wl), to_dev(q_raw, wl))
+
+
+def kimp_alloc(B, Hkv, dimp, Lmax, fill=0.0) -> torch.Tensor:
+    """K_imp cache in the library's layout: 256-token tiles, dimension-major inside."""
+    return torch.full((B, Hkv, Lmax // 256, dimp, 256), fill, dtype=torch.float32, device="cuda")
+
+
+def kimp_rows(kimp: torch.Tensor) -> np.ndarray:
+    """[B][Hkv][Lmax][d'] float64 view of a K_imp cache."""
+    B, Hkv, nt, dimp, _ = kimp.shape
+    return kimp.permute(0, 1, 2, 4, 3).reshape(B, Hkv, nt * 256, dimp).cpu().numpy().astype(np.float64)
 
 
 def mask_from_sets(sets: dict, B: int, rows: int, Lmax: int) -> torch.Tensor:

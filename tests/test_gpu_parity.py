@@ -14,8 +14,8 @@ from oracle import tokenbutler as O
 from query_aware_sparse_decode_b200 import synth as S
 from query_aware_sparse_decode_b200 import tb as TB
 
-from harness import (assert_close_rows, config_of, make_layer, mask_from_sets, round_up, sets_from_mask, tdtype,
-                     tie_band_ok, to_dev)
+from harness import (assert_close_rows, config_of, kimp_alloc, kimp_rows, make_layer, mask_from_sets, round_up,
+                     sets_from_mask, tdtype, tie_band_ok, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +39,7 @@ def test_project_kimp_matches_fp64(wl):
     ld = make_layer(ctx, wl, 0, lens)
     ctx.project_kimp(0, 0, max(lens))
     torch.cuda.synchronize()
-    got = ld.kimp.cpu().numpy().astype(np.float64).transpose(0, 1, 3, 2)  # -> [B][Hkv][t][d']
+    got = kimp_rows(ld.kimp)
     for b, L in enumerate(lens):
         ref = O.project_keys(ld.K[b, :, :L], ld.W)
         assert np.all(np.abs(got[b, :, :L] - ref) <= _kimp_tol(ld.K[b, :, :L], ld.W))
@@ -59,7 +59,7 @@ def test_append_writes_rows_and_kimp(wl):
     k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
     kc = ld.k_cache.float().cpu().numpy()
     vc = ld.v_cache.float().cpu().numpy()
-    kimp = ld.kimp.cpu().numpy().astype(np.float64).transpose(0, 1, 3, 2)
+    kimp = kimp_rows(ld.kimp)
     for b, L in enumerate(lens):
         assert np.array_equal(kc[b, :, L], k64[b]) and np.array_equal(vc[b, :, L], v64[b])
         ref = O.project_keys(k64[b], ld.W)
@@ -116,7 +116,7 @@ def test_select_bit_exact_on_identical_scores(case):
     Lmax = cfg.max_len
     ctx = TB.Context(cfg)
     dummy = torch.zeros((B, 1, Lmax, 64), device="cuda")
-    ctx.bind_layer(0, dummy, dummy.clone(), torch.zeros((B, 1, 16, Lmax), device="cuda"),
+    ctx.bind_layer(0, dummy, dummy.clone(), kimp_alloc(B, 1, 16, Lmax),
                    torch.zeros((64, 16), device="cuda"))
     ctx.set_seq_lens(0, lens)
     sc = _synthetic_scores(B, rows, Lmax, case["quant"], len(lens) * 100 + case["keep"])

@@ -9,7 +9,7 @@ from oracle import tokenbutler as O
 from query_aware_sparse_decode_b200 import synth as S
 from query_aware_sparse_decode_b200 import tb as TB
 
-from harness import config_of, make_layer, round_up, sets_from_mask, tie_band_ok, to_dev
+from harness import config_of, kimp_alloc, kimp_rows, make_layer, round_up, sets_from_mask, tie_band_ok, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -29,13 +29,13 @@ def test_tcgen05_projection_prefill_scale(start, count):
     W_raw = S.w_k(wl, 0)
     k = torch.zeros((B, Hkv, ctx.cfg.max_len, D), dtype=torch.bfloat16, device="cuda")
     k[:, :, :32768] = to_dev(K_raw, wl)
-    kimp = torch.full((B, Hkv, wl.d_imp, ctx.cfg.max_len), float("nan"), device="cuda")
+    kimp = kimp_alloc(B, Hkv, wl.d_imp, ctx.cfg.max_len, float("nan"))
     ctx.bind_layer(0, k, torch.zeros_like(k), kimp, to_dev(W_raw, wl))
     ctx.set_seq_lens(0, [32768])
     ctx.project_kimp(0, start, count)
     torch.cuda.synchronize()
     assert ctx.check_status() == 0
-    got = kimp.cpu().numpy().astype(np.float64).transpose(0, 1, 3, 2)  # -> [B][Hkv][t][d']
+    got = kimp_rows(kimp)
     K = S.widen(K_raw, wl.dtype)
     W = S.widen(W_raw, wl.dtype)
     for g in range(Hkv):
