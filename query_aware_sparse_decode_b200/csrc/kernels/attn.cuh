@@ -433,6 +433,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
   const float* po = p.part_o + ph * D + lane * DPL;
+#pragma unroll 8
   for (int sp = 0; sp < ns; ++sp) {
     const float w = sw[warp][sp];
     if constexpr (DPL == 4) {

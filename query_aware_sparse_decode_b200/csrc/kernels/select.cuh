@@ -8,38 +8,45 @@
 //   Sel = [0, min(sink, L)) U top_min(k, |C|)(C) U [max(L - window, 0), L),
 //   order (score desc, index asc), -0.0 == +0.0.
 //
-// One 1024-thread CTA per row; scores are read as monotone uint32 order keys.
-// Fast path (one ordered sweep of the row):
-//   1. first-digit histogram (top 11 key bits) of the candidates - from the
-//      score kernel, else built here - gives the threshold bin b1 and how
-//      many keys lie above it;
-//   2. the sweep sets, in a shared-memory copy of the row bitmask, every
-//      token surely kept (sink, window, digit > b1) and appends the
-//      candidates of bin b1, in index order (block scan), to a shared buffer;
-//   3. the remaining two digits are resolved on that buffer only; ties at the
-//      final key go to the lowest indices (the buffer is in index order);
-//   4. the bitmask, the count and optionally the ascending index list are
-//      written out from shared memory.
-// Fallback (bin b1 larger than the buffer, or rows beyond the shared bitmask):
-// three radix sweeps over the row with warp-aggregated histograms, then an
-// ordered ballot/scan compaction.
+// Scores are compared as monotone uint32 order keys; the k-th largest key is
+// found digit by digit (11 + 11 + 10 bits).
+//   hist     (standalone calls only) first-digit histogram of the candidates;
+//            the decode step gets it from the score kernel instead.
+//   scatter  many CTAs per row, 8192 tokens each: from the first-digit
+//            histogram every CTA derives the threshold bin b1; lane = token,
+//            a ballot is one mask word: sink, window and keys above b1 are
+//            written to the row bitmask, keys in b1 are appended (CTA-local
+//            buffer, one global atomic per CTA) to the row's candidate list.
+//   resolve  one CTA per row: the candidates (a few percent of the row) are
+//            loaded into shared memory, digits 2 and 3 give the k-th key T,
+//            and ties at T go to the lowest indices (a radix select on the
+//            index when more ties than needed); their mask bits are set.
+//            Then the count check and, if asked, the ascending index list.
+// A row whose threshold bin holds more candidates than the buffer falls back
+// to three radix sweeps over the whole row and an ordered ballot/scan
+// compaction, all inside the resolve CTA.
 #pragma once
 
 #include "common.cuh"
 
 namespace tb {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSelCap = 16384;       // candidate buffer entries (key + index)
-constexpr int kSelMaskWords = 8192;  // shared bitmask words: rows up to 262144 tokens
-constexpr int kSelSmemBytes = kHistBins * 4 + kSelCap * 8 + kSelMaskWords * 4;
+constexpr int kSelThreads = 1024;   // resolve (and prefill) CTAs
+constexpr int kScatThreads = 256;   // scatter / histogram CTAs
+constexpr int kSelChunk = 8192;     // tokens per scatter CTA
+constexpr int kSelCap = 16384;      // candidates per row
+constexpr int kScatCap = 4096;      // candidates staged per scatter CTA before the global append
+constexpr int kResolveSmem = kHistBins * 4 + kSelCap * 8;
+constexpr int kScatSmem = kHistBins * 4 + kScatCap * 8;
 
 struct SelectParams {
-  const float* scores;     // row r of sequence b at (b * rows_per_seq + r) * row_stride
-  const uint32_t* hist1;   // [B*rows][2048] first-digit histograms, or nullptr
-  int32_t* idx;            // [B*rows][idx_cap] or nullptr
-  int32_t* count;          // [B*rows] or nullptr
-  uint32_t* mask;          // [B*rows][mask_words] or nullptr
+  const float* scores;    // row r of sequence b at (b * rows_per_seq + r) * row_stride
+  uint32_t* hist1;        // [B*rows][2048] first-digit histograms of the candidates
+  uint32_t* cand;         // [B*rows][kSelCap][2]: (key, token) of threshold-bin candidates
+  uint32_t* ccount;       // [B*rows] candidates appended (zero before the scatter)
+  int32_t* idx;           // [B*rows][idx_cap] or nullptr
+  int32_t* count;         // [B*rows] or nullptr
+  uint32_t* mask;         // [B*rows][mask_words] (always written)
   uint32_t* status;
   long long row_stride;
   int rows_per_seq, idx_cap, mask_words;
@@ -48,11 +55,11 @@ struct SelectParams {
 };
 
 // Find the bin b (scanning from the top) where the running count reaches k:
-// sum(bins > b) < k <= sum(bins >= b).  NB bins, PER = NB / 1024 per thread.
-template <int PER>
+// sum(bins > b) < k <= sum(bins >= b).  NB = PER * NT bins.
+template <int PER, int NT = kSelThreads>
 __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint32_t* scan_sm, int* out_bin,
                                          uint32_t* out_above) {
-  constexpr int NB = PER * kSelThreads;
+  constexpr int NB = PER * NT;
   const int tid = threadIdx.x;
   uint32_t c[PER];
   uint32_t local = 0;
@@ -62,7 +69,7 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint3
     local += c[j];
   }
   uint32_t total;
-  const uint32_t excl = block_excl_scan<kSelThreads>(local, total, scan_sm);
+  const uint32_t excl = block_excl_scan<NT>(local, total, scan_sm);
   if (excl < k && k <= excl + local) {
     uint32_t run = excl;
 #pragma unroll
@@ -78,7 +85,7 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint3
   __syncthreads();
 }
 
-// Inverse of order_key (for keys of finite floats).
+// Inverse of order_key (keys of finite floats).
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
   return __uint_as_float(u);
@@ -90,209 +97,252 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectParams p) {
-  extern __shared__ __align__(16) uint32_t sel_smem[];
-  uint32_t* hist = sel_smem;                           // [2048]
-  uint32_t* ckey = hist + kHistBins;                   // [kSelCap]
-  uint32_t* cidx = ckey + kSelCap;                     // [kSelCap]
-  uint32_t* smask = cidx + kSelCap;                    // [kSelMaskWords]
-  __shared__ uint32_t scan_sm[32];
-  __shared__ uint2 scan2_sm[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
+struct RowShape {
+  int L, lo, hi, k, mode;  // mode 0: no candidate kept, 1: all kept, 2: top-k by key
+};
+__device__ __forceinline__ RowShape row_shape(const SelectParams& p, int b) {
+  RowShape r;
+  r.L = p.lens[b];
+  r.lo = p.sink;
+  r.hi = r.L - p.window;
+  const int nc = r.hi > r.lo ? r.hi - r.lo : 0;
+  r.k = (int)min((long long)p.keep_pct * r.L / 100, (long long)nc);
+  r.mode = (r.k > 0 && r.k < nc) ? 2 : (r.k == nc && r.k > 0 ? 1 : 0);
+  return r;
+}
 
-  const int r = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-  const int L = p.lens[b];
+// ---------------------------------------------------------------- hist
+// grid (chunks, rows, B): first-digit histogram of the candidates of a chunk.
+__global__ void __launch_bounds__(kScatThreads) select_hist_kernel(const SelectParams p) {
+  __shared__ uint32_t hist[kHistBins];
+  const int chunk = blockIdx.x, r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const RowShape rs = row_shape(p, b);
+  const int t_begin = chunk * kSelChunk;
+  if (rs.mode != 2 || t_begin >= rs.L) return;
   const long long row = (long long)b * p.rows_per_seq + r;
   const float* s = p.scores + row * p.row_stride;
-  const int lo = p.sink, hi = L - p.window;
-  const int nc = hi > lo ? hi - lo : 0;
-  const int k = (int)min((long long)p.keep_pct * L / 100, (long long)nc);
-  const int lwords = (L + 31) >> 5;
-  const size_t orow = (size_t)row;
+  for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = 0;
+  __syncthreads();
+  const int t_end = min(t_begin + kSelChunk, rs.L);
+  for (int t = t_begin + tid; t < t_end; t += kScatThreads)
+    if (t >= rs.lo && t < rs.hi) atomicAdd(&hist[order_key(s[t]) >> 21], 1u);
+  __syncthreads();
+  for (int i = tid; i < kHistBins; i += kScatThreads)
+    if (hist[i]) atomicAdd(&p.hist1[row * kHistBins + i], hist[i]);
+}
 
-  int mode = 0;  // 0: no candidate kept, 1: all kept, 2: threshold + quota ties
-  if (k == nc && k > 0) mode = 1;
-  if (k > 0 && k < nc) mode = 2;
-
-  // ---- first digit: histogram of the candidates' top 11 key bits
-  int b1 = 0;
-  uint32_t k1 = 0, n1 = 0;
-  if (mode == 2) {
-    if (p.hist1 != nullptr) {
-      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
-    } else {
-      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
-      __syncthreads();
-      for (int base = lo & ~3; base < hi; base += 4 * kSelThreads) {
-        const int t0 = base + 4 * tid;
-        if (t0 < hi) {
-          const float4 v = *reinterpret_cast<const float4*>(s + t0);
-          const float vv[4] = {v.x, v.y, v.z, v.w};
+// ---------------------------------------------------------------- scatter
+// grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
+// of the CTA's chunk, 32 tokens (one mask word) per step.
+__global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) uint32_t scat_smem[];
+  uint32_t* hist = scat_smem;               // [2048]
+  uint32_t* lkey = hist + kHistBins;        // [kScatCap]
+  uint32_t* lidx = lkey + kScatCap;         // [kScatCap]
+  __shared__ uint32_t scan_sm[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above, s_n, s_base;
+  const int chunk = blockIdx.x, r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const RowShape rs = row_shape(p, b);
+  const int t_begin = chunk * kSelChunk;
+  if (t_begin >= rs.L) return;
+  const long long row = (long long)b * p.rows_per_seq + r;
+  const float* s = p.scores + row * p.row_stride;
+  float f_lo = 0.f, f_hi = 0.f;
+  bool hi_open = false;
+  if (rs.mode == 2) {
+    for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = p.hist1[row * kHistBins + i];
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    find_bin<kHistBins / kScatThreads, kScatThreads>(hist, (uint32_t)rs.k, scan_sm, &s_bin, &s_above);
+    f_lo = key_to_float((uint32_t)s_bin << 21);           // smallest key of the threshold bin
+    f_hi = key_to_float(((uint32_t)s_bin + 1u) << 21);    // smallest key above it
+    hi_open = s_bin == kHistBins - 1;
+  }
+  constexpr int STEPS = 8;  // loads in flight per thread
+  const int wt0 = t_begin + warp * 1024;
+#pragma unroll 1
+  for (int s0 = 0; s0 < 32; s0 += STEPS) {
+    float v[STEPS];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (t0 + j >= lo && t0 + j < hi) atomicAdd(&hist[order_key(vv[j]) >> 21], 1u);
+    for (int u = 0; u < STEPS; ++u) {
+      const int t = wt0 + (s0 + u) * 32 + lane;
+      v[u] = (rs.mode == 2 && t < rs.L) ? s[t] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < STEPS; ++u) {
+      const int tw = wt0 + (s0 + u) * 32;
+      const int t = tw + lane;
+      const bool in = t < rs.L;
+      const bool cand = t >= rs.lo && t < rs.hi;
+      bool keep = in && (!cand || rs.mode == 1);
+      bool c = false;
+      if (rs.mode == 2 && in && cand) {
+        const bool above = !hi_open && v[u] >= f_hi;
+        keep = above;
+        c = !above && v[u] >= f_lo;
+      }
+      const uint32_t word = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0 && tw < rs.L) p.mask[row * p.mask_words + (tw >> 5)] = word;
+      const uint32_t cm = __ballot_sync(0xffffffffu, c);
+      if (cm) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&s_n, (uint32_t)__popc(cm));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (c) {
+          const uint32_t pos = base + __popc(cm & lanemask_lt());
+          if (pos < (uint32_t)kScatCap) {
+            lkey[pos] = order_key(v[u]);
+            lidx[pos] = (uint32_t)t;
+          }
         }
       }
     }
+  }
+  if (rs.mode != 2) return;
+  __syncthreads();
+  const uint32_t n = min(s_n, (uint32_t)kScatCap);
+  if (tid == 0) {
+    s_base = atomicAdd(&p.ccount[row], s_n);
+    if (s_n > (uint32_t)kScatCap) atomicOr(p.status, TB_DEV_ERR_COUNT);
+  }
+  __syncthreads();
+  uint32_t* dst = p.cand + (size_t)row * kSelCap * 2;
+  for (uint32_t i = tid; i < n; i += kScatThreads) {
+    const uint32_t pos = s_base + i;
+    if (pos < (uint32_t)kSelCap) *reinterpret_cast<uint2*>(dst + 2 * pos) = make_uint2(lkey[i], lidx[i]);
+  }
+}
+
+// ---------------------------------------------------------------- resolve
+// Radix select of the `k` largest among the eligible entries of a shared
+// array, one digit at a time (digits of 11, 11 and 10 bits over a 32-bit
+// key), from pass `first_pass` with `prefix` the digits already fixed.
+// Warp-aggregated shared atomics keep heavily repeated keys cheap.
+template <class Key>
+__device__ __forceinline__ void smem_radix(int n, Key key_of, int first_pass, uint32_t prefix, uint32_t k,
+                                           uint32_t* hist, uint32_t* scan_sm, int* s_bin, uint32_t* s_above,
+                                           uint32_t& T, uint32_t& quota) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t kk = k;
+#pragma unroll 1
+  for (int pass = first_pass; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nbits = pass == 2 ? 10 : 11;
+    const int pshift = pass == 1 ? 21 : 10;
+    for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += kSelThreads) {
+      const int i = base + tid;
+      bool in = false;
+      uint32_t key = 0;
+      if (i < n) in = key_of(i, key);
+      in = in && (pass == 0 || (key >> pshift) == prefix);
+      const uint32_t bin = in ? ((key >> shift) & ((1u << nbits) - 1)) : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    }
+    __syncthreads();
+    if (pass < 2)
+      find_bin<2>(hist, kk, scan_sm, s_bin, s_above);
+    else
+      find_bin<1>(hist, kk, scan_sm, s_bin, s_above);
+    kk -= *s_above;
+    prefix = (prefix << nbits) | (uint32_t)*s_bin;
+    __syncthreads();
+  }
+  T = prefix;
+  quota = kk;
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) uint32_t res_smem[];
+  uint32_t* hist = res_smem;            // [2048]
+  uint32_t* ckey = hist + kHistBins;    // [kSelCap]
+  uint32_t* cidx = ckey + kSelCap;      // [kSelCap]
+  __shared__ uint32_t scan_sm[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  const int r = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const RowShape rs = row_shape(p, b);
+  const int L = rs.L, lo = rs.lo, hi = rs.hi, k = rs.k, mode = rs.mode;
+  const long long row = (long long)b * p.rows_per_seq + r;
+  const size_t orow = (size_t)row;
+  const float* s = p.scores + row * p.row_stride;
+  const int lwords = (L + 31) >> 5;
+
+  bool fallback = false;
+  int b1 = 0;
+  uint32_t k1 = 0, n1 = 0;
+  if (mode == 2) {
+    for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
     __syncthreads();
     find_bin<2>(hist, (uint32_t)k, scan_sm, &s_bin, &s_above);
     b1 = s_bin;
     k1 = (uint32_t)k - s_above;
     n1 = hist[b1];
     __syncthreads();
+    fallback = n1 > (uint32_t)kSelCap;
   }
-  const bool fast = lwords <= kSelMaskWords && (mode != 2 || n1 <= (uint32_t)kSelCap);
 
-  uint32_t T = 0, quota = 0;
-  if (fast) {
-    // ---- one ordered sweep: sure bits into the shared mask, bin-b1 candidates
-    // into the buffer.  Lane = token: an iteration covers STEPS x 1024 tokens,
-    // step j of warp w holds tokens base + j*1024 + w*32 + lane, so a ballot
-    // is one mask word.  The threshold-bin test is two float compares against
-    // the bin's boundary values (the key map is monotone; -0.0 == +0.0 holds
-    // for both).  Candidates keep index order through a (step, warp) prefix.
-    constexpr int STEPS = 16;
-    constexpr int ITER = STEPS * kSelThreads;
-    const int warp = tid >> 5;
-    const float f_lo = key_to_float((uint32_t)b1 << 21);         // smallest key of bin b1
-    const float f_hi = key_to_float(((uint32_t)b1 + 1u) << 21);  // smallest key above bin b1
-    const bool hi_open = b1 == (int)(kHistBins - 1);             // no key lies above the top bin
-    uint32_t nbuf = 0;
-    uint32_t* wcnt = hist;  // [STEPS][32] candidate counts per (step, warp); hist is free during the sweep
-    for (int base = 0; base < L; base += ITER) {
-      float v[STEPS];
-#pragma unroll
-      for (int j = 0; j < STEPS; ++j) {
-        const int t = base + j * kSelThreads + tid;
-        v[j] = (mode == 2 && t < L) ? s[t] : 0.f;
-      }
-      uint32_t cmask[STEPS];
-#pragma unroll
-      for (int j = 0; j < STEPS; ++j) {
-        const int t = base + j * kSelThreads + tid;
-        const bool in = t < L;
-        const bool cand = t >= lo && t < hi;
-        bool keep = in && (!cand || mode == 1);
-        bool c = false;
-        if (mode == 2 && in && cand) {
-          const bool above = !hi_open && v[j] >= f_hi;
-          keep = above;
-          c = !above && v[j] >= f_lo;
-        }
-        const uint32_t word = __ballot_sync(0xffffffffu, keep);
-        const int w = (base + j * kSelThreads) / 32 + warp;
-        if (lane == 0 && w < lwords) smask[w] = word;
-        cmask[j] = __ballot_sync(0xffffffffu, c);
-      }
-      if (mode == 2) {
-        __syncthreads();  // previous users of wcnt are done
-        if (lane < STEPS) {
-          uint32_t cnt = 0;
-#pragma unroll
-          for (int j = 0; j < STEPS; ++j) cnt = j == lane ? __popc(cmask[j]) : cnt;
-          wcnt[lane * 32 + warp] = cnt;
-        }
-        __syncthreads();
-        if (warp < STEPS) {  // warp j: exclusive prefix over the 32 warps of step j
-          const uint32_t c = wcnt[warp * 32 + lane];
-          uint32_t x = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-          }
-          wcnt[warp * 32 + lane] = x - c;
-          if (lane == 31) scan_sm[warp] = x;  // step total
-        }
-        __syncthreads();
-        uint32_t step_base[STEPS];
-        uint32_t run = nbuf;
-#pragma unroll
-        for (int j = 0; j < STEPS; ++j) {
-          step_base[j] = run;
-          run += scan_sm[j];
-        }
-#pragma unroll
-        for (int j = 0; j < STEPS; ++j) {
-          if (cmask[j] & (1u << lane)) {
-            const uint32_t pos = step_base[j] + wcnt[j * 32 + warp] + __popc(cmask[j] & lanemask_lt());
-            if (pos < (uint32_t)kSelCap) {
-              ckey[pos] = order_key(v[j]);
-              cidx[pos] = (uint32_t)(base + j * kSelThreads + tid);
-            }
-          }
-        }
-        nbuf = run;
-      }
-    }
-    __syncthreads();
-    if (mode == 2 && nbuf != n1) {  // histogram and scores disagree: flag it, stay in bounds
-      if (tid == 0) atomicOr(p.status, TB_DEV_ERR_COUNT);
-      nbuf = min(nbuf, (uint32_t)kSelCap);
-    }
-
+  if (!fallback) {
     if (mode == 2) {
-      // ---- digits 2 and 3 on the buffer
-      uint32_t prefix = (uint32_t)b1, kk = k1;
-#pragma unroll 1
-      for (int pass = 1; pass < 3; ++pass) {
-        const int shift = pass == 1 ? 10 : 0;
-        const int nbits = pass == 1 ? 11 : 10;
-        const int pshift = pass == 1 ? 21 : 10;
-        for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < (int)nbuf; i += kSelThreads) {
-          const uint32_t key = ckey[i];
-          if ((key >> pshift) == prefix) atomicAdd(&hist[(key >> shift) & ((1u << nbits) - 1)], 1u);
-        }
-        __syncthreads();
-        if (pass == 1)
-          find_bin<2>(hist, kk, scan_sm, &s_bin, &s_above);
-        else
-          find_bin<1>(hist, kk, scan_sm, &s_bin, &s_above);
-        kk -= s_above;
-        prefix = (prefix << nbits) | (uint32_t)s_bin;
-        __syncthreads();
+      uint32_t n = p.ccount[row];
+      if (n != n1) {  // histogram and scores disagree: flag it, stay in bounds
+        if (tid == 0) atomicOr(p.status, TB_DEV_ERR_COUNT);
+        n = min(n, (uint32_t)kSelCap);
       }
-      T = prefix;
-      quota = kk;
-      // ---- keys above T, and the first `quota` ties in index (= buffer) order
-      uint32_t tie_base = 0;
-      for (int base = 0; base < (int)nbuf; base += kSelThreads) {
-        const int i = base + tid;
-        const uint32_t key = i < (int)nbuf ? ckey[i] : 0u;
-        const bool tie = i < (int)nbuf && key == T;
-        uint32_t total;
-        const uint32_t rank = tie_base + block_excl_scan<kSelThreads>(tie ? 1u : 0u, total, scan_sm);
-        if (i < (int)nbuf && (key > T || (tie && rank < quota))) {
-          const uint32_t t = cidx[i];
-          atomicOr(&smask[t >> 5], 1u << (t & 31));
-        }
-        tie_base += total;
+      const uint32_t* src = p.cand + orow * kSelCap * 2;
+      for (uint32_t i = tid; i < n; i += kSelThreads) {
+        const uint2 e = *reinterpret_cast<const uint2*>(src + 2 * i);
+        ckey[i] = e.x;
+        cidx[i] = e.y;
       }
       __syncthreads();
+      uint32_t T, quota;
+      smem_radix(
+          (int)n,
+          [&](int i, uint32_t& key) {
+            key = ckey[i];
+            return true;
+          },
+          1, (uint32_t)b1, k1, hist, scan_sm, &s_bin, &s_above, T, quota);
+      // ties at T: keep the `quota` lowest indices
+      uint32_t ntie_local = 0;
+      for (uint32_t i = tid; i < n; i += kSelThreads) ntie_local += ckey[i] == T;
+      uint32_t ntie;
+      (void)block_excl_scan<kSelThreads>(ntie_local, ntie, scan_sm);
+      uint32_t J = 0;  // threshold on ~index among the ties when only some of them are kept
+      const bool all_ties = ntie == quota;
+      if (!all_ties) {
+        uint32_t q2;
+        smem_radix(
+            (int)n,
+            [&](int i, uint32_t& key) {
+              key = ~cidx[i];
+              return ckey[i] == T;
+            },
+            0, 0u, quota, hist, scan_sm, &s_bin, &s_above, J, q2);
+      }
+      for (uint32_t i = tid; i < n; i += kSelThreads) {
+        const uint32_t key = ckey[i], t = cidx[i];
+        if (key > T || (key == T && (all_ties || ~t >= J)))
+          atomicOr(&p.mask[orow * p.mask_words + (t >> 5)], 1u << (t & 31));
+      }
+      __threadfence_block();
+      __syncthreads();
     }
-
-    // ---- write out: mask, count, ascending index list
-    uint32_t cnt_local = 0;
-    for (int w = tid; w < lwords; w += kSelThreads) {
-      const uint32_t m = smask[w];
-      if (p.mask != nullptr) p.mask[orow * p.mask_words + w] = m;
-      cnt_local += __popc(m);
-    }
-    uint32_t total_cnt;
-    (void)block_excl_scan<kSelThreads>(cnt_local, total_cnt, scan_sm);
+    // ---- count check and optional ascending index list (mask read back)
+    const int per = (lwords + kSelThreads - 1) / kSelThreads;
+    const int w0 = min(lwords, tid * per), w1 = min(lwords, w0 + per);
+    uint32_t mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(__ldcg(p.mask + orow * p.mask_words + w));
+    uint32_t total;
+    uint32_t pos = block_excl_scan<kSelThreads>(mine, total, scan_sm);
     if (p.idx != nullptr) {
-      // thread owns consecutive words [w0, w1)
-      const int per = (lwords + kSelThreads - 1) / kSelThreads;
-      const int w0 = min(lwords, tid * per), w1 = min(lwords, w0 + per);
-      uint32_t mine = 0;
-      for (int w = w0; w < w1; ++w) mine += __popc(smask[w]);
-      uint32_t tot;
-      uint32_t pos = block_excl_scan<kSelThreads>(mine, tot, scan_sm);
       for (int w = w0; w < w1; ++w) {
-        uint32_t m = smask[w];
+        uint32_t m = __ldcg(p.mask + orow * p.mask_words + w);
         while (m) {
           const int j = __ffs(m) - 1;
           m &= m - 1u;
@@ -302,16 +352,17 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
       }
     }
     if (tid == 0) {
-      if (p.count != nullptr) p.count[orow] = (int32_t)total_cnt;
+      if (p.count != nullptr) p.count[orow] = (int32_t)total;
       const int sink_n = min(p.sink, L);
       const int win_lo = max(L - p.window, sink_n);
-      if (total_cnt != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
+      if (total != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
     }
     return;
   }
 
   // ================================================================ fallback
-  if (mode == 2) {
+  uint32_t T, quota;
+  {
     uint32_t prefix = (uint32_t)b1, kk = k1;
 #pragma unroll 1
     for (int pass = 1; pass < 3; ++pass) {
@@ -354,7 +405,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
   for (int base = 0; base < L; base += 4 * kSelThreads) {
     const int t0 = base + 4 * tid;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (mode == 2 && t0 < L) v = *reinterpret_cast<const float4*>(s + t0);
+    if (t0 < L) v = *reinterpret_cast<const float4*>(s + t0);
     const float vv[4] = {v.x, v.y, v.z, v.w};
     uint32_t forced = 0, tie = 0;  // bit j: element t0 + j
 #pragma unroll
@@ -364,12 +415,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
       const bool cand = t >= lo && t < hi;
       bool keep = !cand;  // sink / window
       if (cand) {
-        if (mode == 1) keep = true;
-        if (mode == 2) {
-          const uint32_t key = order_key(vv[j]);
-          if (key > T) keep = true;
-          else if (key == T) tie |= 1u << j;
-        }
+        const uint32_t key = order_key(vv[j]);
+        if (key > T) keep = true;
+        else if (key == T) tie |= 1u << j;
       }
       if (keep) forced |= 1u << j;
     }
@@ -399,14 +447,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
           ++pos;
         }
     }
-    if (p.mask != nullptr) {
-      uint32_t word = keepbits << ((lane & 7) * 4);
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      const int w = (base >> 5) + (tid >> 3);
-      if ((lane & 7) == 0 && w * 32 < L) p.mask[orow * p.mask_words + w] = word;
-    }
+    uint32_t word = keepbits << ((lane & 7) * 4);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    word |= __shfl_xor_sync(0xffffffffu, word, 4);
+    const int w = (base >> 5) + (tid >> 3);
+    if ((lane & 7) == 0 && w < lwords) p.mask[orow * p.mask_words + w] = word;
     out_base += tot_sel + (min(tie_base + tot_tie, quota) - min(tie_base, quota));
     tie_base += tot_tie;
   }
@@ -414,8 +460,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
     if (p.count != nullptr) p.count[orow] = (int32_t)out_base;
     const int sink_n = min(p.sink, L);
     const int win_lo = max(L - p.window, sink_n);
-    const uint32_t expect = (uint32_t)(sink_n + (L - win_lo) + k);
-    if (out_base != expect) atomicOr(p.status, TB_DEV_ERR_COUNT);
+    if (out_base != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
   }
 }
 

@@ -37,7 +37,7 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, scores, mask, part_o, part_ml, votes, vstats, total;
+  size_t status, hist, ccount, cand, scores, mask, part_o, part_ml, votes, vstats, total;
   int max_splits;
 };
 
@@ -47,7 +47,9 @@ WsLayout layout_of(const tb_config& c) {
   w.max_splits = (int)((Lm + 255) / 256);
   size_t off = 0;
   w.status = off;  off += align256(256);
-  w.hist = off;    off += align256(B * Hq * kHistBins * 4);
+  w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
+  w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters (zeroed together)
+  w.cand = off;    off += align256(B * Hq * (size_t)kSelCap * 8);
   w.scores = off;  off += align256(B * Hq * Lm * 4);
   w.mask = off;    off += align256(B * Hq * (Lm / 32) * 4);
   w.part_o = off;  off += align256(B * Hq * (size_t)w.max_splits * c.head_dim * 4);
@@ -87,6 +89,8 @@ struct tb_ctx {
   WsLayout lay;
   uint32_t* status = nullptr;
   uint32_t* hist = nullptr;
+  uint32_t* ccount = nullptr;
+  uint32_t* cand = nullptr;
   float* scores = nullptr;
   uint32_t* mask = nullptr;
   float* part_o = nullptr;
@@ -156,8 +160,8 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.sink = c.sink;
   p.window = c.window;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  if (hist) {
-    const size_t n = (size_t)c.batch * c.n_q_heads * kHistBins;
+  if (hist) {  // histograms and the selection's candidate counters start at zero
+    const size_t n = (size_t)c.batch * c.n_q_heads * (kHistBins + 1);
     zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(hist, n);
     ++ctx->launches;
   }
@@ -201,16 +205,20 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   return TB_ERR_UNSUPPORTED;
 }
 
-static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, const uint32_t* hist1, int rows,
+// Selection of every row: hist1_ready means the score kernel already built
+// the first-digit histograms (and zeroed the candidate counters).
+static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool hist1_ready, int rows,
                                int32_t* idx, int idx_cap, int32_t* count, uint32_t* mask, cudaStream_t st) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   SelectParams p{};
   p.scores = scores;
-  p.hist1 = hist1;
+  p.hist1 = ctx->hist;
+  p.cand = ctx->cand;
+  p.ccount = ctx->ccount;
   p.idx = idx;
   p.count = count;
-  p.mask = mask;
+  p.mask = mask != nullptr ? mask : ctx->mask;
   p.status = ctx->status;
   p.row_stride = c.max_len;
   p.rows_per_seq = rows;
@@ -220,10 +228,19 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, cons
   p.sink = c.sink;
   p.window = c.window;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  dim3 grid(rows, c.batch);
-  cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmemBytes);
-  select_kernel<<<grid, kSelThreads, kSelSmemBytes, st>>>(p);
-  ++ctx->launches;
+  const int maxL = max_len_of(ls, c.batch);
+  dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
+  if (!hist1_ready) {
+    const size_t n = (size_t)c.batch * c.n_q_heads * (kHistBins + 1);
+    zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(ctx->hist, n);
+    select_hist_kernel<<<cgrid, kScatThreads, 0, st>>>(p);
+    ctx->launches += 2;
+  }
+  cudaFuncSetAttribute(select_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScatSmem);
+  select_scatter_kernel<<<cgrid, kScatThreads, kScatSmem, st>>>(p);
+  cudaFuncSetAttribute(select_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kResolveSmem);
+  select_resolve_kernel<<<dim3(rows, c.batch), kSelThreads, kResolveSmem, st>>>(p);
+  ctx->launches += 2;
   return cuda_status(cudaGetLastError());
 }
 
@@ -377,6 +394,8 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->ws = static_cast<char*>(workspace);
   ctx->status = reinterpret_cast<uint32_t*>(ctx->ws + lay.status);
   ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
+  ctx->ccount = reinterpret_cast<uint32_t*>(ctx->ws + lay.ccount);
+  ctx->cand = reinterpret_cast<uint32_t*>(ctx->ws + lay.cand);
   ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
   ctx->mask = reinterpret_cast<uint32_t*>(ctx->ws + lay.mask);
   ctx->part_o = reinterpret_cast<float*>(ctx->ws + lay.part_o);
@@ -549,7 +568,7 @@ TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows
       if (sink_n + (L - win_lo) + k > idx_cap) return TB_ERR_SHAPE;
     }
   }
-  return launch_select(ctx, layer, scores, nullptr, rows_per_seq, idx, idx_cap, count, mask,
+  return launch_select(ctx, layer, scores, false, rows_per_seq, idx, idx_cap, count, mask,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -588,7 +607,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     s = launch_softvote(ctx, layer, q, ctx->votes, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
-    s = launch_select(ctx, layer, ctx->votes, nullptr, 1, nullptr, 0, nullptr, ctx->mask, st);
+    s = launch_select(ctx, layer, ctx->votes, false, 1, nullptr, 0, nullptr, ctx->mask, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
@@ -596,7 +615,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 2, st);
-  s = launch_select(ctx, layer, ctx->scores, ctx->hist, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+  s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 3, st);
   return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
