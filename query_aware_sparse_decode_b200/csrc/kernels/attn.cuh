@@ -24,7 +24,7 @@ constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kAttnStages = 3;
 constexpr int kAttnTile = 16;        // tokens per mma tile
-constexpr int kAttnMaxChunk = 2048;  // tokens per CTA (multiple of 256)
+constexpr int kAttnMaxChunk = 2048;  // tokens per gather list (a CTA's chunk may span several)
 
 struct AttnParams {
   const void* k_cache;   // [B][Hkv][max_len][D]
@@ -154,7 +154,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const int t0 = split * p.chunk;
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
-  const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 2, tq = lane & 3;
@@ -180,10 +179,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
 #pragma unroll
   for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
   float m_run = kNegInf, l_run = 0.f;
+  uint8_t* my_ring = ring + warp * kAttnStages * STAGE;
 
+  // the CTA's chunk is processed in sub-chunks of up to kAttnMaxChunk tokens
+  // (one gather list each); the softmax state carries across them
+  for (int sc0 = t0; sc0 < t1; sc0 += kAttnMaxChunk) {
+  const int n = build_union_list<GS>(p, b, g, sc0, min(sc0 + kAttnMaxChunk, t1), list_idx, list_hb, scan_sm);
   const int ntiles = n / kAttnTile + (n % kAttnTile ? 1 : 0);
   const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
-  uint8_t* my_ring = ring + warp * kAttnStages * STAGE;
 
   auto issue = [&](int it) {
     const int tile = warp + it * kAttnWarps;
@@ -280,6 +283,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
     __syncwarp();
   }
   cp_async_wait<0>();
+  __syncthreads();  // the gather list and the ring are free for the next sub-chunk
+  }
 
   // ---- merge the four warps through shared memory (reuses the ring)
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -330,7 +335,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   const int t0 = split * p.chunk;
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
-  const int n = build_union_list<GS>(p, b, g, t0, t1, list_idx, list_hb, scan_sm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* Kb = reinterpret_cast<const float*>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.max_len * D;
   const float* Vb = reinterpret_cast<const float*>(p.v_cache) + ((size_t)b * p.Hkv + g) * p.max_len * D;
@@ -345,6 +349,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
       o[hh][j] = 0.f;
     }
   }
+  for (int sc0 = t0; sc0 < t1; sc0 += kAttnMaxChunk) {
+  const int n = build_union_list<GS>(p, b, g, sc0, min(sc0 + kAttnMaxChunk, t1), list_idx, list_hb, scan_sm);
   for (int i = warp; i < n; i += kAttnWarps) {
     const int t = list_idx[i];
     const uint32_t hb = list_hb[i];
@@ -371,6 +377,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
       m[hh] = mn;
     }
   }
+  __syncthreads();  // the gather list is free for the next sub-chunk
+  }
 #pragma unroll
   for (int hh = 0; hh < GS; ++hh) {
     if (lane == 0) {
@@ -394,48 +402,53 @@ struct CombineParams {
   int lens[kMaxBatch];
 };
 
-// fp32 log-sum-exp merge of the split partials: one warp per (b, h), four
-// per CTA.  Two dependent load phases: every split's (m, l), then the partial
-// rows (each lane owns D/32 consecutive dimensions).  An empty set gives
-// out = 0 and lse = -inf.
+// fp32 log-sum-exp merge of the split partials: one CTA per (b, h).  All
+// (m, l) pairs are loaded at once; then each of the four warps sums a
+// quarter of the splits for the whole output row (lane = D/32 consecutive
+// dimensions) and the quarters are added in shared memory.  An empty set
+// gives out = 0 and lse = -inf.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   constexpr int DPL = D / 32;
-  __shared__ float sw[4][kMaxSplits];
-  __shared__ float sl[4][kMaxSplits];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x * 4 + warp;
-  if (bh >= p.B * p.Hq) return;
+  __shared__ float sw[kMaxSplits];
+  __shared__ float sred[4][D];
+  __shared__ float sM[4], sS[4];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int L = p.lens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
   const size_t ph = (size_t)bh * p.nsplit;
   float M = kNegInf;
-  for (int sp = lane; sp < ns; sp += 32) {
-    const float2 v = *reinterpret_cast<const float2*>(p.part_ml + (ph + sp) * 2);
-    sw[warp][sp] = v.x;
-    sl[warp][sp] = v.y;
-    M = fmaxf(M, v.x);
+  for (int sp = tid; sp < ns; sp += 128) {
+    const float m = p.part_ml[(ph + sp) * 2];
+    sw[sp] = m;
+    M = fmaxf(M, m);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) sM[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(sM[0], sM[1]), fmaxf(sM[2], sM[3]));
   float lsum = 0.f;
-  for (int sp = lane; sp < ns; sp += 32) {
-    const float m = sw[warp][sp];
+  for (int sp = tid; sp < ns; sp += 128) {
+    const float m = sw[sp];
     const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
-    sw[warp][sp] = f;
-    lsum += f * sl[warp][sp];
+    sw[sp] = f;
+    lsum += f * p.part_ml[(ph + sp) * 2 + 1];
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  __syncwarp();
+  if (lane == 0) sS[warp] = lsum;
+  __syncthreads();
+  lsum = (sS[0] + sS[1]) + (sS[2] + sS[3]);
   float acc[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
   const float* po = p.part_o + ph * D + lane * DPL;
-#pragma unroll 8
-  for (int sp = 0; sp < ns; ++sp) {
-    const float w = sw[warp][sp];
+#pragma unroll 4
+  for (int sp = warp; sp < ns; sp += 4) {
+    const float w = sw[sp];
     if constexpr (DPL == 4) {
       const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
       acc[0] += w * v.x;
@@ -448,11 +461,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
       acc[1] += w * v.y;
     }
   }
-  const float inv = M == kNegInf ? 0.f : 1.f / lsum;
-  T* dst = reinterpret_cast<T*>(p.out) + (size_t)bh * D + lane * DPL;
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) dst[i] = from_f32<T>(acc[i] * inv);
-  if (p.lse != nullptr && lane == 0) p.lse[bh] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
+  for (int i = 0; i < DPL; ++i) sred[warp][lane * DPL + i] = acc[i];
+  __syncthreads();
+  const float inv = M == kNegInf ? 0.f : 1.f / lsum;
+  for (int d = tid; d < D; d += 128) {
+    const float o = ((sred[0][d] + sred[1][d]) + (sred[2][d] + sred[3][d])) * inv;
+    reinterpret_cast<T*>(p.out)[(size_t)bh * D + d] = from_f32<T>(o);
+  }
+  if (p.lse != nullptr && tid == 0) p.lse[bh] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
 }
 
 }  // namespace tb

@@ -44,6 +44,7 @@ struct SelectParams {
   uint32_t* hist1;        // [B*rows][2048] first-digit histograms of the candidates
   uint32_t* cand;         // [B*rows][kSelCap][2]: (key, token) of threshold-bin candidates
   uint32_t* ccount;       // [B*rows] candidates appended (zero before the scatter)
+  uint4* rowinfo;         // [B*rows] (b1, k1, n1, -): first digit, rank left in it, its count
   int32_t* idx;           // [B*rows][idx_cap] or nullptr
   int32_t* count;         // [B*rows] or nullptr
   uint32_t* mask;         // [B*rows][mask_words] (always written)
@@ -133,7 +134,8 @@ __global__ void __launch_bounds__(kScatThreads) select_hist_kernel(const SelectP
 
 // ---------------------------------------------------------------- scatter
 // grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
-// of the CTA's chunk, 32 tokens (one mask word) per step.
+// of the CTA's chunk; a warp step covers 128 tokens, four consecutive per
+// lane (float4), and lanes 8m..8m+7 form mask word m of the step.
 __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const SelectParams p) {
   extern __shared__ __align__(16) uint32_t scat_smem[];
   uint32_t* hist = scat_smem;               // [2048]
@@ -159,44 +161,77 @@ __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const Sele
     f_lo = key_to_float((uint32_t)s_bin << 21);           // smallest key of the threshold bin
     f_hi = key_to_float(((uint32_t)s_bin + 1u) << 21);    // smallest key above it
     hi_open = s_bin == kHistBins - 1;
+    if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's first digit from here
+      p.rowinfo[row] = make_uint4((uint32_t)s_bin, (uint32_t)rs.k - s_above, hist[s_bin], 0u);
   }
-  constexpr int STEPS = 8;  // loads in flight per thread
+  constexpr int STEPS = 4;  // 16-byte loads in flight per thread
   const int wt0 = t_begin + warp * 1024;
 #pragma unroll 1
-  for (int s0 = 0; s0 < 32; s0 += STEPS) {
-    float v[STEPS];
+  for (int s0 = 0; s0 < 8; s0 += STEPS) {
+    float4 v[STEPS];
 #pragma unroll
     for (int u = 0; u < STEPS; ++u) {
-      const int t = wt0 + (s0 + u) * 32 + lane;
-      v[u] = (rs.mode == 2 && t < rs.L) ? s[t] : 0.f;
+      const int t0 = wt0 + (s0 + u) * 128 + 4 * lane;
+      v[u] = (rs.mode == 2 && t0 < rs.L) ? *reinterpret_cast<const float4*>(s + t0) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < STEPS; ++u) {
-      const int tw = wt0 + (s0 + u) * 32;
-      const int t = tw + lane;
-      const bool in = t < rs.L;
-      const bool cand = t >= rs.lo && t < rs.hi;
-      bool keep = in && (!cand || rs.mode == 1);
-      bool c = false;
-      if (rs.mode == 2 && in && cand) {
-        const bool above = !hi_open && v[u] >= f_hi;
-        keep = above;
-        c = !above && v[u] >= f_lo;
-      }
-      const uint32_t word = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0 && tw < rs.L) p.mask[row * p.mask_words + (tw >> 5)] = word;
-      const uint32_t cm = __ballot_sync(0xffffffffu, c);
-      if (cm) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&s_n, (uint32_t)__popc(cm));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (c) {
-          const uint32_t pos = base + __popc(cm & lanemask_lt());
-          if (pos < (uint32_t)kScatCap) {
-            lkey[pos] = order_key(v[u]);
-            lidx[pos] = (uint32_t)t;
-          }
+      const int tw = wt0 + (s0 + u) * 128;
+      if (tw >= rs.L) break;  // warp-uniform
+      const int t0 = tw + 4 * lane;
+      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t keep = 0, cbits = 0;
+      if (rs.mode == 2 && tw >= rs.lo && tw + 128 <= rs.hi) {
+        // interior step: every token is an in-range candidate
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool above = !hi_open && vv[j] >= f_hi;
+          keep |= (uint32_t)above << j;
+          cbits |= (uint32_t)(!above && vv[j] >= f_lo) << j;
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = t0 + j;
+          const bool in = t < rs.L;
+          const bool cand = t >= rs.lo && t < rs.hi;
+          bool kp = in && (!cand || rs.mode == 1);
+          bool c = false;
+          if (rs.mode == 2 && in && cand) {
+            const bool above = !hi_open && vv[j] >= f_hi;
+            kp = above;
+            c = !above && vv[j] >= f_lo;
+          }
+          keep |= (uint32_t)kp << j;
+          cbits |= (uint32_t)c << j;
+        }
+      }
+      uint32_t word = keep << ((lane & 7) * 4);
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      if ((lane & 7) == 0 && t0 < rs.L) p.mask[row * p.mask_words + (t0 >> 5)] = word;
+      if (__any_sync(0xffffffffu, cbits != 0)) {
+        const uint32_t cnt = __popc(cbits);
+        uint32_t x = cnt;  // inclusive prefix over the lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        uint32_t base = 0;
+        if (lane == 31) base = atomicAdd(&s_n, x);
+        base = __shfl_sync(0xffffffffu, base, 31);
+        uint32_t pos = base + x - cnt;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (cbits & (1u << j)) {
+            if (pos < (uint32_t)kScatCap) {
+              lkey[pos] = order_key(vv[j]);
+              lidx[pos] = (uint32_t)(t0 + j);
+            }
+            ++pos;
+          }
       }
     }
   }
@@ -276,13 +311,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
   int b1 = 0;
   uint32_t k1 = 0, n1 = 0;
   if (mode == 2) {
-    for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
-    __syncthreads();
-    find_bin<2>(hist, (uint32_t)k, scan_sm, &s_bin, &s_above);
-    b1 = s_bin;
-    k1 = (uint32_t)k - s_above;
-    n1 = hist[b1];
-    __syncthreads();
+    const uint4 info = p.rowinfo[row];
+    b1 = (int)info.x;
+    k1 = info.y;
+    n1 = info.z;
     fallback = n1 > (uint32_t)kSelCap;
   }
 

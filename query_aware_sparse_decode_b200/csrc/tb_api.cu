@@ -37,7 +37,7 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, ccount, cand, scores, mask, part_o, part_ml, votes, vstats, total;
+  size_t status, hist, ccount, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats, total;
   int max_splits;
 };
 
@@ -49,6 +49,7 @@ WsLayout layout_of(const tb_config& c) {
   w.status = off;  off += align256(256);
   w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
   w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters (zeroed together)
+  w.rowinfo = off; off += align256(B * Hq * 16);
   w.cand = off;    off += align256(B * Hq * (size_t)kSelCap * 8);
   w.scores = off;  off += align256(B * Hq * Lm * 4);
   w.mask = off;    off += align256(B * Hq * (Lm / 32) * 4);
@@ -91,6 +92,7 @@ struct tb_ctx {
   uint32_t* hist = nullptr;
   uint32_t* ccount = nullptr;
   uint32_t* cand = nullptr;
+  uint4* rowinfo = nullptr;
   float* scores = nullptr;
   uint32_t* mask = nullptr;
   float* part_o = nullptr;
@@ -216,6 +218,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   p.hist1 = ctx->hist;
   p.cand = ctx->cand;
   p.ccount = ctx->ccount;
+  p.rowinfo = ctx->rowinfo;
   p.idx = idx;
   p.count = count;
   p.mask = mask != nullptr ? mask : ctx->mask;
@@ -265,12 +268,11 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   p.max_len = c.max_len;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  // chunking: about four CTAs per SM over the whole grid
+  // chunking: the whole grid is about two full waves of two CTAs per SM
   const int groups = c.batch * c.n_kv_heads;
-  const int want_split = std::max(1, (4 * ctx->num_sms + groups - 1) / groups);
+  const int want_split = std::min(kMaxSplits, std::max(1, (4 * ctx->num_sms) / groups));
   int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
-  chunk = std::max(chunk, (maxL + kMaxSplits - 1) / kMaxSplits);  // at most kMaxSplits splits
-  chunk = std::min(kAttnMaxChunk, std::max(256, (chunk + 255) / 256 * 256));
+  chunk = std::max(256, (chunk + 255) / 256 * 256);
   p.chunk = chunk;
   p.nsplit = std::max(1, (maxL + chunk - 1) / chunk);
   if (p.nsplit > kMaxSplits) return TB_ERR_UNSUPPORTED;
@@ -310,7 +312,7 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   cp.chunk = chunk;
   cp.nsplit = p.nsplit;
   for (int b = 0; b < c.batch; ++b) cp.lens[b] = ls.lens[b];
-  const unsigned cgrid = (unsigned)((c.batch * c.n_q_heads + 3) / 4);
+  const unsigned cgrid = (unsigned)(c.batch * c.n_q_heads);
   if (c.kv_dtype == TB_BF16) {
     if (c.head_dim == 128) combine_kernel<__nv_bfloat16, 128><<<cgrid, 128, 0, st>>>(cp);
     else combine_kernel<__nv_bfloat16, 64><<<cgrid, 128, 0, st>>>(cp);
@@ -396,6 +398,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
   ctx->ccount = reinterpret_cast<uint32_t*>(ctx->ws + lay.ccount);
   ctx->cand = reinterpret_cast<uint32_t*>(ctx->ws + lay.cand);
+  ctx->rowinfo = reinterpret_cast<uint4*>(ctx->ws + lay.rowinfo);
   ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
   ctx->mask = reinterpret_cast<uint32_t*>(ctx->ws + lay.mask);
   ctx->part_o = reinterpret_cast<float*>(ctx->ws + lay.part_o);
