@@ -202,6 +202,36 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
  * tb_select(rows_per_seq = 1) and attend with TB_MASK_SHARED. */
 TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream);
 
+/* ---- allocation-free attention ---------------------------------------------
+ * The model card and the papers have no counterpart to this entry point; it
+ * exists for callers that cannot allocate device memory (a serving loop with
+ * a fixed memory budget that forbids allocation after start-up, a plug-in
+ * whose host process owns all device memory, a runtime that only hands out
+ * streams).  It computes exactly what tb_sparse_attn computes, without a
+ * tb_ctx or a workspace: its split-K partials live in a static device array
+ * of TB_STATIC_SCRATCH_BYTES inside the library, held by every GPU that
+ * loads the library until the process exits.
+ *   - `cache` describes the caller's K/V caches and lengths (host array);
+ *     q, mask, mask_mode, out and lse are as for tb_sparse_attn.
+ *   - TB_ERR_CAPACITY when the partials of the request (B * Hq * splits *
+ *     (D + 2) floats) would not fit in the static array; nothing is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; calls
+ *     that overlap on the GPU (several streams or threads) race on it.
+ *   - It allocates nothing and calls no allocating routine. */
+#define TB_STATIC_SCRATCH_BYTES (8u << 20)
+
+typedef struct tb_cache_view {
+  const void* k_cache;        /* [B][Hkv][max_len][D] device, kv_dtype          */
+  const void* v_cache;        /* [B][Hkv][max_len][D] device, kv_dtype          */
+  int batch, n_q_heads, n_kv_heads, head_dim, max_len, kv_dtype;
+  const int32_t* lens_host;   /* [B] host: tokens per sequence                  */
+} tb_cache_view;
+
+TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, const void* q, const uint32_t* mask,
+                                       int mask_mode, void* out, float* lse, void* stream);
+
 /* Tracing: when `events` is non-NULL, tb_decode_step records the six
  * cudaEvent_t events[0..5] on its stream before the append, after the
  * append, after scoring, after selection, after the split attention kernel

@@ -28,8 +28,8 @@ STATUS_NAMES = {0: "TB_OK", 1: "TB_ERR_INVALID_ARG", 2: "TB_ERR_SHAPE", 3: "TB_E
 # every symbol include/tb.h declares
 EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "tb_get_seq_lens", "tb_set_budget",
            "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
-           "tb_select_prefill", "tb_softvote_scores", "tb_trace_events", "tb_launch_count", "tb_check_status",
-           "tb_status_string", "tb_destroy")
+           "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
+           "tb_check_status", "tb_status_string", "tb_destroy")
 
 
 class TBError(RuntimeError):
@@ -44,6 +44,12 @@ class Config(ctypes.Structure):
                 ("producer_freq", ctypes.c_int), ("max_len", ctypes.c_int), ("kv_dtype", ctypes.c_int),
                 ("keep_pct", ctypes.c_int), ("sink", ctypes.c_int), ("window", ctypes.c_int),
                 ("dense_layer_mask", ctypes.c_uint64), ("variant", ctypes.c_int)]
+
+
+class CacheView(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("batch", ctypes.c_int),
+                ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("max_len", ctypes.c_int), ("kv_dtype", ctypes.c_int), ("lens_host", ctypes.POINTER(ctypes.c_int32))]
 
 
 _lib = None
@@ -72,6 +78,7 @@ def lib():
             "tb_decode_step": [vp, i32, vp, vp, vp, vp, vp, vp],
             "tb_select_prefill": [vp, i32, vp, i32, i32, vp, i32, vp],
             "tb_softvote_scores": [vp, i32, vp, vp, vp],
+            "tb_sparse_attn_static": [P(CacheView), vp, vp, i32, vp, vp, vp],
             "tb_trace_events": [vp, P(vp), i32],
             "tb_launch_count": [vp, P(ctypes.c_uint64)],
             "tb_check_status": [vp, P(ctypes.c_uint32)],
@@ -123,6 +130,19 @@ def workspace_size(cfg: Config) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().tb_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "tb_workspace_size")
     return n.value
+
+
+def sparse_attn_static(k_cache, v_cache, lens, n_q_heads, q, mask, mask_mode, out, lse=None, stream=None) -> None:
+    """tb_sparse_attn_static: the sparse attention without a context or a
+    workspace (its scratch is a static device array inside the library), for
+    callers that cannot allocate device memory.  k_cache, v_cache:
+    [B][Hkv][max_len][D]; lens: per-sequence token counts."""
+    B, Hkv, max_len, D = k_cache.shape
+    arr = (ctypes.c_int32 * B)(*[int(x) for x in lens])
+    view = CacheView(k_cache.data_ptr(), v_cache.data_ptr(), B, n_q_heads, Hkv, D, max_len,
+                     TB_BF16 if k_cache.dtype == torch.bfloat16 else TB_F32, arr)
+    _check(lib().tb_sparse_attn_static(ctypes.byref(view), _ptr(q), _ptr(mask), mask_mode, _ptr(out), _ptr(lse),
+                                       _stream(stream)), "tb_sparse_attn_static")
 
 
 class Context:
