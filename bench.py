@@ -174,10 +174,22 @@ def build(wl, max_len, dev):
                       seed=wl.seed)
         ctx.bind_layer(layer, k, v, kimp, w)
         ctx.set_seq_lens(layer, [L0] * wl.B)
-        ctx.project_kimp(layer, 0, L0)
         bufs.append((k, v, kimp, w))
+    # prefill side of K_imp = K . W_K for every layer (tcgen05 GEMM), timed
     torch.cuda.synchronize()
-    return ctx, bufs
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for layer in range(wl.n_layers):
+        ctx.project_kimp(layer, 0, L0)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / wl.n_layers
+    rows = wl.B * wl.Hkv * L0
+    nbytes = rows * (wl.D * 2 + wl.d_imp * 4)
+    proj = {"kernel": "butler_kimp_project (tcgen05, prefill of the cache)", "us_per_layer": us,
+            "rows_per_layer": rows, "bytes_per_layer": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+            "tflops": 2 * rows * wl.D * wl.d_imp / (us * 1e-6) / 1e12}
+    return ctx, bufs, proj
 
 
 def step_inputs_host(wl, s):
@@ -243,7 +255,7 @@ def gpu_arm(args, rank, world, local_rank):
     max_len = (wl.L + 255) // 256 * 256
     if max_len == wl.L:
         max_len += 256
-    ctx, bufs = build(wl, max_len, dev)
+    ctx, bufs, proj = build(wl, max_len, dev)
     stream = torch.cuda.current_stream(dev)
     nvar = min(args.steps + args.warmup, 4)
     host_inputs = [step_inputs_host(wl, s) for s in range(nvar)]
@@ -351,7 +363,7 @@ def gpu_arm(args, rank, world, local_rank):
     status = ctx.check_status()
     if status:
         raise RuntimeError(f"device status flags {status:#x}")
-    return dict(wl=wl, value=value, ms_step=ms_step, clk=clk, launches=launches, avg=avg, urows=urows,
+    return dict(proj=proj, wl=wl, value=value, ms_step=ms_step, clk=clk, launches=launches, avg=avg, urows=urows,
                 union_bytes=union_bytes, kimp_bytes=kimp_bytes, step_bytes=step_bytes, peak=peak,
                 peak_src=peak_src, attn_gbs=attn_gbs, score_gbs=score_gbs, pair_gbs=pair_gbs, e2e=e2e,
                 scored=scored, attended=attended)
@@ -468,6 +480,7 @@ def main():
                                "frac": (r["score_gbs"] / r["peak"]) if r["score_gbs"] else None,
                                "bytes_per_launch": r["kimp_bytes"]},
             "kernel_us": avg,
+            "prefill_kimp": dict(r["proj"], frac_hbm=r["proj"]["gbs"] / r["peak"]),
             "union_rows_per_layer": (sum(r["urows"].values()) / max(len(r["urows"]), 1)),
             "gpu_launches": r["launches"],
             "clocks": r["clk"],

@@ -134,8 +134,7 @@ __global__ void __launch_bounds__(kScatThreads) select_hist_kernel(const SelectP
 
 // ---------------------------------------------------------------- scatter
 // grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
-// of the CTA's chunk; a warp step covers 128 tokens, four consecutive per
-// lane (float4), and lanes 8m..8m+7 form mask word m of the step.
+// of the CTA's chunk, all loaded up front (8 float4 per lane).
 __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const SelectParams p) {
   extern __shared__ __align__(16) uint32_t scat_smem[];
   uint32_t* hist = scat_smem;               // [2048]
@@ -164,74 +163,76 @@ __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const Sele
     if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's first digit from here
       p.rowinfo[row] = make_uint4((uint32_t)s_bin, (uint32_t)rs.k - s_above, hist[s_bin], 0u);
   }
-  constexpr int STEPS = 4;  // 16-byte loads in flight per thread
+  // a warp step covers 256 tokens: lane owns 8 consecutive tokens (two float4),
+  // lanes 4m..4m+3 form mask word m of the step
+  constexpr int STEPS = 4;
   const int wt0 = t_begin + warp * 1024;
-#pragma unroll 1
-  for (int s0 = 0; s0 < 8; s0 += STEPS) {
-    float4 v[STEPS];
+  float4 v[STEPS][2];
 #pragma unroll
-    for (int u = 0; u < STEPS; ++u) {
-      const int t0 = wt0 + (s0 + u) * 128 + 4 * lane;
-      v[u] = (rs.mode == 2 && t0 < rs.L) ? *reinterpret_cast<const float4*>(s + t0) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+  for (int u = 0; u < STEPS; ++u) {
+    const int t0 = wt0 + u * 256 + 8 * lane;
 #pragma unroll
-    for (int u = 0; u < STEPS; ++u) {
-      const int tw = wt0 + (s0 + u) * 128;
-      if (tw >= rs.L) break;  // warp-uniform
-      const int t0 = tw + 4 * lane;
-      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      uint32_t keep = 0, cbits = 0;
-      if (rs.mode == 2 && tw >= rs.lo && tw + 128 <= rs.hi) {
-        // interior step: every token is an in-range candidate
+    for (int h = 0; h < 2; ++h)
+      v[u][h] = (rs.mode == 2 && t0 + 4 * h < rs.L) ? *reinterpret_cast<const float4*>(s + t0 + 4 * h)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool above = !hi_open && vv[j] >= f_hi;
-          keep |= (uint32_t)above << j;
-          cbits |= (uint32_t)(!above && vv[j] >= f_lo) << j;
-        }
-      } else {
+  for (int u = 0; u < STEPS; ++u) {
+    const int tw = wt0 + u * 256;
+    if (tw >= rs.L) break;  // warp-uniform
+    const int t0 = tw + 8 * lane;
+    const float vv[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w, v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+    uint32_t keep = 0, cbits = 0;
+    if (rs.mode == 2 && tw >= rs.lo && tw + 256 <= rs.hi) {
+      // interior step: every token is an in-range candidate
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int t = t0 + j;
-          const bool in = t < rs.L;
-          const bool cand = t >= rs.lo && t < rs.hi;
-          bool kp = in && (!cand || rs.mode == 1);
-          bool c = false;
-          if (rs.mode == 2 && in && cand) {
-            const bool above = !hi_open && vv[j] >= f_hi;
-            kp = above;
-            c = !above && vv[j] >= f_lo;
-          }
-          keep |= (uint32_t)kp << j;
-          cbits |= (uint32_t)c << j;
-        }
+      for (int j = 0; j < 8; ++j) {
+        keep |= (uint32_t)(vv[j] >= f_hi) << j;
+        cbits |= (uint32_t)(vv[j] >= f_lo) << j;
       }
-      uint32_t word = keep << ((lane & 7) * 4);
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      if ((lane & 7) == 0 && t0 < rs.L) p.mask[row * p.mask_words + (t0 >> 5)] = word;
-      if (__any_sync(0xffffffffu, cbits != 0)) {
-        const uint32_t cnt = __popc(cbits);
-        uint32_t x = cnt;  // inclusive prefix over the lanes
+      if (hi_open) keep = 0;
+      cbits &= ~keep;
+    } else {
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
+      for (int j = 0; j < 8; ++j) {
+        const int t = t0 + j;
+        const bool in = t < rs.L;
+        const bool cand = t >= rs.lo && t < rs.hi;
+        bool kp = in && (!cand || rs.mode == 1);
+        bool c = false;
+        if (rs.mode == 2 && in && cand) {
+          const bool above = !hi_open && vv[j] >= f_hi;
+          kp = above;
+          c = !above && vv[j] >= f_lo;
         }
-        uint32_t base = 0;
-        if (lane == 31) base = atomicAdd(&s_n, x);
-        base = __shfl_sync(0xffffffffu, base, 31);
-        uint32_t pos = base + x - cnt;
+        keep |= (uint32_t)kp << j;
+        cbits |= (uint32_t)c << j;
+      }
+    }
+    uint32_t word = keep << ((lane & 3) * 8);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if ((lane & 3) == 0 && t0 < rs.L) p.mask[row * p.mask_words + (t0 >> 5)] = word;
+    if (__any_sync(0xffffffffu, cbits != 0)) {
+      const uint32_t cnt = __popc(cbits);
+      uint32_t x = cnt;  // inclusive prefix over the lanes
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (cbits & (1u << j)) {
-            if (pos < (uint32_t)kScatCap) {
-              lkey[pos] = order_key(vv[j]);
-              lidx[pos] = (uint32_t)(t0 + j);
-            }
-            ++pos;
-          }
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(&s_n, x);
+      base = __shfl_sync(0xffffffffu, base, 31);
+      uint32_t pos = base + x - cnt;
+      while (cbits) {
+        const int j = __ffs(cbits) - 1;
+        cbits &= cbits - 1u;
+        if (pos < (uint32_t)kScatCap) {
+          lkey[pos] = order_key(vv[j]);
+          lidx[pos] = (uint32_t)(t0 + j);
+        }
+        ++pos;
       }
     }
   }
