@@ -143,3 +143,62 @@ def tie_band_ok(gpu_set, ref_set, scores64, L, keep_pct, sink, window) -> bool:
     kth = np.sort(sc)[::-1][k - 1]
     band = 1e-4 * np.abs(scores64[:L]).max()
     return all(abs(scores64[t] - kth) <= band for t in g ^ r)
+
+
+@dataclass
+class DeviceLayer:
+    """A layer whose caches were made on the device by the shared generator;
+    the oracle regenerates any (b, KV head) slab on the host (same bits)."""
+    wl: object
+    layer: int
+    L0: int
+    W: np.ndarray            # [D][d'] float64
+    qimp: np.ndarray         # producer tensor, float64
+    qhat: np.ndarray | None  # [B][Hq][d'] float64
+    delta: np.ndarray | None  # [B][Hkv][D] float32
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    kimp: torch.Tensor
+    q_imp_dev: torch.Tensor
+    q_dev: torch.Tensor
+    q: np.ndarray            # [B][Hq][D] float64
+
+    def slab(self, which: int, b: int, g: int) -> np.ndarray:
+        """Rows [0, L0) of K (which=K_CACHE) or V of one (b, g), float64 [L0][D]."""
+        wl = self.wl
+        a = b * wl.Hkv + g
+        delta = None
+        mod = 0
+        if which == S.K_CACHE and self.delta is not None:
+            delta, mod = self.delta.reshape(wl.B * wl.Hkv, wl.D), 100
+        raw = S.fill_host(which, self.layer, 0, 1, 0, self.L0, wl.D, wl.dtype, delta=delta, plant_mod=mod,
+                          seed=wl.seed, a0=a)[0]
+        return S.widen(raw, wl.dtype)
+
+
+def make_layer_device(ctx: TB.Context, wl, layer: int, L0: int, step: int = 0) -> DeviceLayer:
+    """Fills rows [0, L0) of every sequence on the device (1 % planted heavy
+    hitters on consumer layers), binds the layer with len = L0 and projects
+    K_imp with the library."""
+    B, Hq, Hkv, D, dimp, G = wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G
+    Lmax = ctx.cfg.max_len
+    W_raw = S.w_k(wl, layer)
+    W = S.widen(W_raw, wl.dtype)
+    qimp_raw = S.q_imp(wl, O.producer_of(layer, G), step)
+    qimp = S.widen(qimp_raw, wl.dtype)
+    dense = layer in wl.dense_layers
+    qhat = None if dense else O.importance_queries(qimp, layer, G, B, Hq)
+    delta = None if dense or wl.plant == "none" else S.plant_delta(W, qhat, Hkv)
+    k = torch.empty((B, Hkv, Lmax, D), dtype=tdtype(wl), device="cuda")
+    v = torch.empty_like(k)
+    dd = None if delta is None else torch.from_numpy(delta.reshape(B * Hkv, D)).cuda()
+    S.fill_device(k, S.K_CACHE, layer, 0, B * Hkv, 0, L0, D, Lmax * D, D, wl.dtype, delta=dd,
+                  plant_mod=100 if dd is not None else 0, seed=wl.seed)
+    S.fill_device(v, S.V_CACHE, layer, 0, B * Hkv, 0, L0, D, Lmax * D, D, wl.dtype, seed=wl.seed)
+    kimp = kimp_alloc(B, Hkv, dimp, Lmax)
+    ctx.bind_layer(layer, k, v, kimp, to_dev(W_raw, wl))
+    ctx.set_seq_lens(layer, [L0] * B)
+    ctx.project_kimp(layer, 0, L0)
+    q_raw = S.query(wl, layer, step)
+    return DeviceLayer(wl, layer, L0, W, qimp, qhat, delta, k, v, kimp, to_dev(qimp_raw, wl), to_dev(q_raw, wl),
+                       S.widen(q_raw, wl.dtype))

@@ -1,0 +1,269 @@
+"""Parity at full size.
+
+Two families of workloads, each with caches generated on the device by the
+counter-based generator:
+
+* the 32-layer decode step at B = 4, L = 131072, G = 4, 30 % kept (the launch
+  configuration the benchmark times: same shapes, same split-K chunking),
+  checked on sampled layers (the dense layer 0 and consumers of every
+  producer slot);
+* the long-context sweep, L = 4096 ... 262144 at 10 / 30 / 50 % kept, for
+  TokenButler and for per-head soft voting (TokenSelect).
+
+The oracle cannot process whole caches of this size in seconds, so it checks
+sampled (sequence, KV head) slabs: it regenerates each slab on the host from
+the same generator (bit-identical rows) and runs its own steps on it.  K_imp
+and scores are compared element by element over the whole slab, the selected
+sets up to the tie band, and attention outputs (and LSE) against the oracle's
+attention over the selected set: the oracle's own set, or the GPU's where the
+two differ only inside the tie band (the output given a set is unique).  Properties that
+hold for every head (set sizes, sink and window membership, and the fused
+step equal to the separate calls) are checked on all heads."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import tokenbutler as O
+from query_aware_sparse_decode_b200 import synth as S
+from query_aware_sparse_decode_b200 import tb as TB
+
+from harness import assert_close_rows, config_of, make_layer_device, sets_from_mask, tdtype, tie_band_ok, to_dev
+
+pytestmark = pytest.mark.gpu
+
+DECODE = S.DECODE32_B4_L128K
+DECODE_LAYERS = (0, 1, 2, 3, 4, 17, 31)   # dense, then slots 0, 1, 2, 3, a middle and the last layer
+DECODE_SAMPLES = ((0, 0), (1, 5), (2, 2), (3, 7))  # (sequence, KV head)
+
+
+def _need_device_bytes(nbytes: int) -> None:
+    free, _ = torch.cuda.mem_get_info()
+    if free < nbytes * 1.25:
+        pytest.skip(f"needs {nbytes / 2**30:.1f} GiB of free device memory, {free / 2**30:.1f} GiB free")
+
+
+def _layer_bytes(wl, max_len: int) -> int:
+    kv = 2 * wl.B * wl.Hkv * max_len * wl.D * (2 if wl.dtype == "bf16" else 4)
+    kimp = wl.B * wl.Hkv * max_len * wl.d_imp * 4
+    scores = wl.B * wl.Hq * max_len * 4
+    return kv + kimp + 2 * scores
+
+
+class _Slabs:
+    """K or V of a device-generated layer seen as [B][Hkv][L][D] float64:
+    rows [0, L - 1) regenerated on the host slab by slab on first use, row
+    L - 1 the token the step appended.  Only the most recent slab is kept."""
+
+    def __init__(self, dl, which: int, new_row: np.ndarray):
+        wl = dl.wl
+        self.dl, self.which, self.new_row = dl, which, new_row
+        self.shape = (wl.B, wl.Hkv, dl.L0 + 1, wl.D)
+        self._key, self._val = None, None
+
+    def slab(self, b: int, g: int) -> np.ndarray:
+        if self._key != (b, g):
+            rows = self.dl.slab(self.which, b, g)
+            self._val = np.concatenate([rows, self.new_row[b, g][None]], axis=0)
+            self._key = (b, g)
+        return self._val
+
+    def __getitem__(self, key):
+        if isinstance(key, tuple) and len(key) == 3:
+            b, g, rows = key
+            return self.slab(b, g)[rows]
+        return _Seq(self, key)
+
+
+class _Seq:
+    """One sequence of a :class:`_Slabs`, seen as [Hkv][L][D]."""
+
+    def __init__(self, slabs: _Slabs, b: int):
+        self.slabs, self.b = slabs, b
+        self.shape = slabs.shape[1:]
+
+    def __getitem__(self, key):
+        g, rows = key
+        return self.slabs.slab(self.b, g)[rows]
+
+
+def _kimp_slab(kimp: torch.Tensor, b: int, g: int, L: int) -> np.ndarray:
+    nt, dimp, tile = kimp.shape[2:]
+    return kimp[b, g].permute(0, 2, 1).reshape(nt * tile, dimp)[:L].cpu().numpy().astype(np.float64)
+
+
+def _check_shape_of_sets(mask: torch.Tensor, lens, keep_pct: int, sink: int, window: int) -> None:
+    """Every row: |set| = sink + window + min(floor(P L / 100), candidates),
+    sink and window inside, nothing at or past len."""
+    m = mask.cpu().numpy().view(np.uint32)
+    B, rows, words = m.shape
+    bits = np.unpackbits(m.reshape(B, rows, words).view(np.uint8), axis=-1, bitorder="little")
+    for b, L in enumerate(lens):
+        cand = max(L - window - sink, 0)
+        want = min(sink, L) + min(window, max(L - min(sink, L), 0)) + min(O.token_budget(L, keep_pct), cand)
+        assert np.all(bits[b, :, :L].sum(axis=-1) == want)
+        assert not bits[b, :, L:].any()
+        assert bits[b, :, :min(sink, L)].all() and bits[b, :, max(L - window, 0):L].all()
+
+
+def _gpu_step(ctx, wl, layer: int, dl, k_dev, v_dev, keep_pct: int) -> dict:
+    """One decode step from len L - 1 at the given budget, fused and through
+    the separate calls (which keep scores and selection)."""
+    cfg = ctx.cfg
+    ctx.set_budget(keep_pct, wl.sink, wl.window)
+    ctx.set_seq_lens(layer, [wl.L - 1] * wl.B)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+    ctx.decode_step(layer, k_dev, v_dev, dl.q_dev, dl.q_imp_dev, out)
+    assert ctx.seq_lens(layer) == [wl.L] * wl.B
+    dense = layer in wl.dense_layers
+    scores = torch.full((wl.B, wl.Hq, cfg.max_len), float("nan"), device="cuda")
+    mask = torch.zeros((wl.B, wl.Hq, cfg.max_len // 32), dtype=torch.int32, device="cuda")
+    out2 = torch.empty_like(out)
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    if dense:
+        ctx.sparse_attn(layer, dl.q_dev, None, TB.TB_MASK_DENSE, out2, lse)
+    else:
+        ctx.score(layer, dl.q_imp_dev, scores)
+        ctx.select(layer, scores, wl.Hq, mask=mask)
+        ctx.sparse_attn(layer, dl.q_dev, mask, TB.TB_MASK_PER_HEAD, out2, lse)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    assert torch.equal(out, out2)
+    if not dense:
+        _check_shape_of_sets(mask, [wl.L] * wl.B, keep_pct, wl.sink, wl.window)
+    return {"out": out.float().cpu().numpy(), "lse": lse.cpu().numpy(), "scores": scores, "mask": mask}
+
+
+def _decode_full(wl, layer: int, samples, keeps=None) -> None:
+    keeps = (wl.keep_pct,) if keeps is None else keeps
+    cfg = config_of(wl)
+    _need_device_bytes(_layer_bytes(wl, cfg.max_len) + len(keeps) * wl.B * wl.Hq * cfg.max_len * 4)
+    ctx = TB.Context(cfg)
+    dl = make_layer_device(ctx, wl, layer, wl.L - 1)
+    k_raw, v_raw = S.kv_new(wl, layer)
+    k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
+    gpu = {P: _gpu_step(ctx, wl, layer, dl, k_dev, v_dev, P) for P in keeps}
+    dense = layer in wl.dense_layers
+    lens = [wl.L] * wl.B
+    # oracle on the sampled (sequence, KV head) slabs
+    K = _Slabs(dl, S.K_CACHE, S.widen(k_raw, wl.dtype))
+    V = _Slabs(dl, S.V_CACHE, S.widen(v_raw, wl.dtype))
+    gs = wl.Hq // wl.Hkv
+    scale = 1.0 / math.sqrt(wl.D)
+    mism = {P: 0 for P in keeps}
+    for b, g in samples:
+        heads = range(g * gs, (g + 1) * gs)
+        Kg = K.slab(b, g)
+        V.slab(b, g)
+        if not dense:
+            kimp = _kimp_slab(dl.kimp, b, g, wl.L)
+            assert np.all(np.abs(kimp - O.project_keys(Kg, dl.W)) <= 8e-6 * (np.abs(Kg) @ np.abs(dl.W)) + 1e-30)
+        for P, r in gpu.items():
+            sel, ref, ref_lse, sc = O.decode_layer(dl.q, K, V, dl.W, dl.qimp, layer, wl.G, lens, P, wl.sink,
+                                                   wl.window, dense=dense, heads=heads, batches=[b])
+            if not dense:
+                got_sets = sets_from_mask(r["mask"][b:b + 1, g * gs:(g + 1) * gs], [wl.L])
+            for h in heads:
+                what = f"layer {layer} keep {P} b{b} h{h}"
+                if not dense:
+                    s = r["scores"][b, h, :wl.L].cpu().numpy().astype(np.float64)
+                    assert np.max(np.abs(s - sc[b, h])) <= 1e-5 * np.max(np.abs(sc[b, h])), what
+                    gset = got_sets[0, h - g * gs]
+                    assert tie_band_ok(gset, sel[b, h], sc[b, h], wl.L, P, wl.sink, wl.window), what
+                    if not np.array_equal(gset, sel[b, h]):
+                        # a different but valid set (inside the tie band):
+                        # the output is still unique given the set
+                        mism[P] += 1
+                        ref[b, h], ref_lse[b, h] = O.attend(dl.q[b, h], Kg, V.slab(b, g), gset, scale)
+                assert_close_rows(r["out"][b, h][None], ref[b, h][None], wl.dtype, what)
+                assert abs(r["lse"][b, h] - ref_lse[b, h]) <= 1e-3 * max(1.0, abs(ref_lse[b, h])), what
+    for P in keeps:
+        assert mism[P] <= len(samples) * gs // 2, f"keep {P}: {mism[P]} sets differ inside the tie band"
+
+
+@pytest.mark.parametrize("layer", DECODE_LAYERS)
+def test_decode32_B4_L131072_sampled_heads(layer):
+    _decode_full(DECODE, layer, DECODE_SAMPLES)
+
+
+@pytest.mark.parametrize("L", S.SWEEP_LENGTHS)
+def test_long_context_sweep_butler(L):
+    wl = S.sweep(L, S.SWEEP_KEEP[0])
+    _decode_full(wl, 0, ((0, 0), (0, wl.Hkv - 1)), keeps=S.SWEEP_KEEP)
+
+
+def _softvote_full(wl, groups, keeps) -> None:
+    """Soft voting on one sequence of length L: votes over every head, the
+    shared set per budget, attention of the heads of the sampled KV groups."""
+    cfg = config_of(wl, variant=TB.TB_SOFTVOTE)
+    _need_device_bytes(_layer_bytes(wl, cfg.max_len))
+    ctx = TB.Context(cfg)
+    dl = make_layer_device(ctx, wl, 0, wl.L - 1)
+    k_raw, v_raw = S.kv_new(wl, 0)
+    k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
+    votes = torch.full((wl.B, cfg.max_len), float("nan"), device="cuda")
+    gpu = {}
+    for P in keeps:
+        ctx.set_budget(P, wl.sink, wl.window)
+        ctx.set_seq_lens(0, [wl.L - 1] * wl.B)
+        out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+        ctx.decode_step(0, k_dev, v_dev, dl.q_dev, None, out)
+        mask = torch.zeros((wl.B, 1, cfg.max_len // 32), dtype=torch.int32, device="cuda")
+        out2 = torch.empty_like(out)
+        ctx.softvote_scores(0, dl.q_dev, votes)
+        ctx.select(0, votes, 1, mask=mask)
+        ctx.sparse_attn(0, dl.q_dev, mask, TB.TB_MASK_SHARED, out2)
+        torch.cuda.synchronize()
+        assert ctx.check_status() == 0
+        assert torch.equal(out, out2)
+        _check_shape_of_sets(mask, [wl.L] * wl.B, P, wl.sink, wl.window)
+        gpu[P] = (sets_from_mask(mask, [wl.L] * wl.B), out.float().cpu().numpy())
+    v = votes.cpu().numpy().astype(np.float64)
+    K = _Slabs(dl, S.K_CACHE, S.widen(k_raw, wl.dtype))
+    V = _Slabs(dl, S.V_CACHE, S.widen(v_raw, wl.dtype))
+    gs = wl.Hq // wl.Hkv
+    scale = 1.0 / math.sqrt(wl.D)
+    for b in range(wl.B):
+        ref_votes = O.softvote_scores(dl.q[b], K[b], wl.L)
+        assert np.max(np.abs(v[b, :wl.L] - ref_votes)) <= 1e-4 * np.max(np.abs(ref_votes))
+        assert abs(v[b, :wl.L].sum() - wl.Hq) <= 1e-3 * wl.Hq
+        sel = {P: O.select_tokens(ref_votes, wl.L, P, wl.sink, wl.window) for P in keeps}
+        for P in keeps:
+            got_sets, _ = gpu[P]
+            assert tie_band_ok(got_sets[b, 0], sel[P], ref_votes, wl.L, P, wl.sink, wl.window), f"keep {P}"
+        for g in groups:
+            Kg, Vg = K.slab(b, g), V.slab(b, g)
+            for P in keeps:
+                got_sets, o = gpu[P]
+                # where the sets differ inside the tie band, the output given
+                # the GPU's (valid) set is still unique
+                use = sel[P] if np.array_equal(got_sets[b, 0], sel[P]) else got_sets[b, 0]
+                for h in range(g * gs, (g + 1) * gs):
+                    ref, _ = O.attend(dl.q[b, h], Kg, Vg, use, scale)
+                    assert_close_rows(o[b, h][None], ref[None], wl.dtype, f"softvote keep {P} b{b} h{h}")
+
+
+@pytest.mark.parametrize("L", S.SWEEP_LENGTHS)
+def test_long_context_sweep_softvote(L):
+    wl = S.sweep(L, S.SWEEP_KEEP[0])
+    _softvote_full(wl, (0, wl.Hkv - 1), S.SWEEP_KEEP)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_device_generator_matches_host_bit_for_bit(dtype):
+    """The premise of the sampled checks: device-filled caches (strided, from
+    a row offset, with planted rows) equal the host's regeneration exactly."""
+    A, t0, t1, C, Lmax = 6, 37, 5000, 128, 5120
+    delta = np.random.default_rng(3).standard_normal((A, C)).astype(np.float32)
+    dev = torch.zeros((A, Lmax, C), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32, device="cuda")
+    S.fill_device(dev, S.K_CACHE, 7, 2, A, t0, t1, C, Lmax * C, C, dtype, delta=torch.from_numpy(delta).cuda(),
+                  plant_mod=100, seed=11)
+    torch.cuda.synchronize()
+    host = S.fill_host(S.K_CACHE, 7, 2, A, t0, t1, C, dtype, delta=delta, plant_mod=100, seed=11)
+    got = dev[:, t0:t1].cpu()
+    got = got.view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else got.numpy()
+    assert np.array_equal(got.view(np.uint8), host.view(np.uint8))
+    assert not dev[:, :t0].any() and not dev[:, t1:].any()
+    one = S.fill_host(S.K_CACHE, 7, 2, 1, t0, t1, C, dtype, delta=delta, plant_mod=100, seed=11, a0=4)
+    assert np.array_equal(one[0].view(np.uint8), host[4].view(np.uint8))
