@@ -48,6 +48,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--table", action="store_true",
+                    help="instead of the step benchmark, print per-kernel times (one JSON line per row) for the "
+                         "8B-shaped L=32768 case, the L=4K..256K sweep of both variants and the prefill path")
+    ap.add_argument("--table-iters", type=int, default=20)
+    ap.add_argument("--table-only", default=None, help="regular expression on the row names to run")
     return ap.parse_args()
 
 
@@ -161,12 +166,13 @@ def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: flo
 
 
 # ----------------------------------------------------------------------- GPU arm
-def build(wl, max_len, dev):
+def build(wl, max_len, dev, variant=None):
     import torch
     from query_aware_sparse_decode_b200 import synth as S
     from query_aware_sparse_decode_b200 import tb as TB
     cfg = TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G, max_len, wl.dtype, wl.keep_pct,
-                         wl.sink, wl.window, dense_layers=wl.dense_layers)
+                         wl.sink, wl.window, dense_layers=wl.dense_layers,
+                         variant=TB.TB_BUTLER if variant is None else variant)
     ctx = TB.Context(cfg, dev)
     L0 = wl.L - 1
     bufs = []
@@ -451,6 +457,172 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------- per-kernel table
+def _pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))]
+
+
+def _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream):
+    """Per-segment times (us) of single decode steps, each bracketed by the
+    library's trace events; with `flush_buf`, L2 is flushed before every step
+    (outside the events) by a 512 MB write followed by a 256 MB read, so the
+    step starts with L2 full of clean, unrelated lines."""
+    import torch
+    kn, vn, qq, qi = inp
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=ctx.device)
+    rows = []
+    for it in range(3 + iters):
+        ctx.set_seq_lens(layer, [wl.L - 1] * wl.B)
+        if flush_buf is not None:
+            flush_buf.add_(1)
+            flush_buf.view(torch.float32)[: 64 << 20].sum()
+        ctx.trace_events(ev)
+        ctx.decode_step(layer, kn, vn, qq, qi, out, stream)
+        ctx.trace_events(None)
+        torch.cuda.synchronize()
+        if it >= 3:
+            rows.append([ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(5)] + [ev[0].elapsed_time(ev[5]) * 1e3])
+    names = ["append", "score", "select", "attn", "combine", "total"]
+    med = {n: statistics.median(r[i] for r in rows) for i, n in enumerate(names)}
+    med["total_p90"] = _pct([r[5] for r in rows], 0.9)
+    return med
+
+
+def _table_case(wl, variant, dev, iters, flush_buf, peak):
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    from query_aware_sparse_decode_b200 import tb as TB
+    max_len = (wl.L + 1 + 255) // 256 * 256
+    ctx, bufs, _ = build(wl, max_len, dev, variant)
+    layer = 0
+    stream = torch.cuda.current_stream(dev)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    kn, vn = S.kv_new(wl, layer)
+    inp = (bf(kn), bf(vn), bf(S.query(wl, layer)), bf(S.q_imp(wl, 0)))
+    cold = _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream)
+    hot = _timed_decode(ctx, wl, layer, inp, iters, None, stream)
+    # algorithmic bytes from the library's own selection of this step
+    ctx.set_seq_lens(layer, [wl.L] * wl.B)
+    dense = wl.keep_pct >= 100 or layer in wl.dense_layers
+    row_kv = 2 * wl.D * 2
+    gs = wl.Hq // wl.Hkv
+    if dense:
+        first, union = 0, wl.B * wl.Hkv * wl.L
+    elif variant == TB.TB_SOFTVOTE:
+        votes = torch.empty((wl.B, max_len), device=dev)
+        mask = torch.zeros((wl.B, 1, max_len // 32), dtype=torch.int32, device=dev)
+        ctx.softvote_scores(layer, inp[2], votes)
+        ctx.select(layer, votes, 1, mask=mask)
+        first = wl.B * wl.Hkv * wl.L * wl.D * 2               # the full K, read for the logits
+        union = int(np.unpackbits(mask.cpu().numpy().view(np.uint8)).sum()) * wl.Hkv
+    else:
+        scores = torch.empty((wl.B, wl.Hq, max_len), device=dev)
+        mask = torch.zeros((wl.B, wl.Hq, max_len // 32), dtype=torch.int32, device=dev)
+        ctx.score(layer, inp[3], scores)
+        ctx.select(layer, scores, wl.Hq, mask=mask)
+        m = mask.view(wl.B, wl.Hkv, gs, -1)
+        u = m[:, :, 0]
+        for j in range(1, gs):
+            u = u | m[:, :, j]
+        first = wl.B * wl.Hkv * wl.L * wl.d_imp * 4           # K_imp
+        union = int(np.unpackbits(u.cpu().numpy().view(np.uint8)).sum())
+    torch.cuda.synchronize()
+    if ctx.check_status():
+        raise RuntimeError("device status flags set")
+    attn_bytes = union * row_kv
+
+    def rates(t):
+        r = {"attn_gbs": attn_bytes / (t["attn"] * 1e-6) / 1e9}
+        if not dense:
+            r["score_gbs"] = first / (t["score"] * 1e-6) / 1e9
+            r["score_plus_attn_gbs"] = (first + attn_bytes) / ((t["score"] + t["attn"]) * 1e-6) / 1e9
+            r["score_plus_attn_frac"] = r["score_plus_attn_gbs"] / peak
+        r["attn_frac"] = r["attn_gbs"] / peak
+        r["step_gbs"] = (first + attn_bytes) / (t["total"] * 1e-6) / 1e9
+        return r
+    line = {"table": "decode", "workload": wl.name, "variant": "softvote" if variant == TB.TB_SOFTVOTE else "butler",
+            "B": wl.B, "L": wl.L, "keep_pct": wl.keep_pct, "dense": dense,
+            "first_pass_bytes": first, "union_rows": union, "attn_bytes": attn_bytes,
+            "us_cold_l2": cold, "us_hot_l2": hot, "rates_cold_l2": rates(cold), "rates_hot_l2": rates(hot),
+            "l2": "cold: 512 MB write + 256 MB read before each step; hot: back-to-back steps",
+            "iters": iters,
+            "peak_gbs": peak}
+    del ctx, bufs
+    torch.cuda.empty_cache()
+    return line
+
+
+def _table_prefill(dev, iters, peak):
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    wl = S.PREFILL_L32K
+    max_len = wl.L + 256
+    # build() fills and projects rows [0, L - 1) of its workload: one more
+    # gives the whole 32768-row prefix of every layer
+    ctx, bufs, proj = build(wl.with_(L=wl.L + 1), max_len, dev)
+    layer, nrows = 1, 1024
+    row0 = wl.L - nrows
+    qrows = S.q_imp(wl, 0, rows=(row0, nrows))
+    qd = torch.from_numpy(np.ascontiguousarray(qrows).view(np.int16)).view(torch.bfloat16).to(dev)
+    wpr = wl.L // 32
+    masks = torch.zeros((wl.B, wl.Hq, nrows, wpr), dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for it in range(3 + iters):
+        e0.record()
+        ctx.select_prefill(layer, qd, row0, nrows, masks)
+        e1.record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            ts.append(e0.elapsed_time(e1) * 1e3)
+    if ctx.check_status():
+        raise RuntimeError("device status flags set")
+    us = statistics.median(ts)
+    elems = wl.B * wl.Hq * sum(row0 + r + 1 for r in range(nrows))
+    line = {"table": "prefill", "workload": wl.name, "kimp_gemm": dict(proj, frac_hbm=proj["gbs"] / peak),
+            "select_prefill": {"rows": nrows, "row0": row0, "us_median": us, "us_p90": _pct(ts, 0.9),
+                               "score_elements": elems, "elements_per_s": elems / (us * 1e-6),
+                               "score_tflops": 2 * wl.d_imp * elems / (us * 1e-6) / 1e12,
+                               "mask_bytes": masks.numel() * 4, "mask_gbs": masks.numel() * 4 / (us * 1e-6) / 1e9}}
+    del ctx, bufs
+    torch.cuda.empty_cache()
+    return line
+
+
+def kernel_table(args):
+    """Per-kernel times for the workloads beside the step benchmark: the
+    8B-shaped L=32768 case (50 % and dense), the long-context sweep of both
+    variants and the prefill importance path.  Prints one JSON line per row."""
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    from query_aware_sparse_decode_b200 import tb as TB
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak = 6650.0
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        with open(peaks_path) as f:
+            peak = float(json.load(f)["hbm_gbs"])
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    cases = [(S.LLAMA8B_L32K, TB.TB_BUTLER), (S.LLAMA8B_L32K.with_(keep_pct=100), TB.TB_BUTLER)]
+    for L in S.SWEEP_LENGTHS:
+        for P in S.SWEEP_KEEP:
+            cases.append((S.sweep(L, P), TB.TB_BUTLER))
+            cases.append((S.sweep(L, P), TB.TB_SOFTVOTE))
+    import re
+    pick = re.compile(args.table_only) if args.table_only else None
+    for wl, variant in cases:
+        name = f"{wl.name}_{'softvote' if variant == TB.TB_SOFTVOTE else 'butler'}"
+        if pick is None or pick.search(name):
+            print(json.dumps(_table_case(wl, variant, dev, args.table_iters, flush_buf, peak)), flush=True)
+    if pick is None or pick.search(S.PREFILL_L32K.name):
+        print(json.dumps(_table_prefill(dev, args.table_iters, peak)), flush=True)
+
+
 # ----------------------------------------------------------------------- main
 def main():
     args = parse()
@@ -459,6 +631,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         reference_arm(args, rank, world)
+        return
+    if args.table:
+        if rank == 0:
+            kernel_table(args)
         return
     import torch
     import torch.distributed as dist

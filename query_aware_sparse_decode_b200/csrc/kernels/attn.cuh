@@ -136,6 +136,8 @@ constexpr int attn_bf16_smem_bytes() {
 
 template <int D, int GS>
 __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnParams p) {
+  pdl_wait();
+  pdl_trigger();
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(GS >= 1 && GS <= 8, "group size");
   constexpr int ROWB = D * 2;                       // bytes per K or V row
@@ -321,6 +323,8 @@ constexpr int attn_f32_smem_bytes() {
 // fp32 caches: one warp per token at a time, lane owns dims lane + 32 j.
 template <int D, int GS>
 __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int DPL = D / 32;
   extern __shared__ __align__(128) uint8_t smem[];
   int32_t* list_idx = reinterpret_cast<int32_t*>(smem);
@@ -403,51 +407,66 @@ struct CombineParams {
 };
 
 // fp32 log-sum-exp merge of the split partials: one CTA per (b, h).  All
-// (m, l) pairs are loaded at once; then each of the four warps sums a
-// quarter of the splits for the whole output row (lane = D/32 consecutive
-// dimensions) and the quarters are added in shared memory.  An empty set
-// gives out = 0 and lse = -inf.
+// (m, l) pairs are loaded at once (one float2 each); then each of the eight
+// warps sums an eighth of the splits for the whole output row (lane = D/32
+// consecutive dimensions, eight split rows in flight per warp) and the
+// eighths are added in shared memory.  An empty set gives out = 0 and
+// lse = -inf.
+constexpr int kCombineThreads = 256;
 template <typename T, int D>
-__global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int DPL = D / 32;
+  constexpr int NW = kCombineThreads / 32;
   __shared__ float sw[kMaxSplits];
-  __shared__ float sred[4][D];
-  __shared__ float sM[4], sS[4];
+  __shared__ float sred[NW][D];
+  __shared__ float sM[NW], sS[NW];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int L = p.lens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
   const size_t ph = (size_t)bh * p.nsplit;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + ph;
   float M = kNegInf;
-  for (int sp = tid; sp < ns; sp += 128) {
-    const float m = p.part_ml[(ph + sp) * 2];
-    sw[sp] = m;
-    M = fmaxf(M, m);
+  float2 mine[(kMaxSplits + kCombineThreads - 1) / kCombineThreads];
+#pragma unroll
+  for (int r = 0; r < (kMaxSplits + kCombineThreads - 1) / kCombineThreads; ++r) {
+    const int sp = tid + r * kCombineThreads;
+    mine[r] = sp < ns ? ml[sp] : make_float2(kNegInf, 0.f);
+    M = fmaxf(M, mine[r].x);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) sM[warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(sM[0], sM[1]), fmaxf(sM[2], sM[3]));
+  M = sM[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, sM[w]);
   float lsum = 0.f;
-  for (int sp = tid; sp < ns; sp += 128) {
-    const float m = sw[sp];
-    const float f = (M == kNegInf || m == kNegInf) ? 0.f : exp2f(m - M);
-    sw[sp] = f;
-    lsum += f * p.part_ml[(ph + sp) * 2 + 1];
+#pragma unroll
+  for (int r = 0; r < (kMaxSplits + kCombineThreads - 1) / kCombineThreads; ++r) {
+    const int sp = tid + r * kCombineThreads;
+    if (sp < ns) {
+      const float f = (M == kNegInf || mine[r].x == kNegInf) ? 0.f : exp2f(mine[r].x - M);
+      sw[sp] = f;
+      lsum += f * mine[r].y;
+    }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
   if (lane == 0) sS[warp] = lsum;
   __syncthreads();
-  lsum = (sS[0] + sS[1]) + (sS[2] + sS[3]);
+  lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) lsum += sS[w];
   float acc[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
   const float* po = p.part_o + ph * D + lane * DPL;
-#pragma unroll 4
-  for (int sp = warp; sp < ns; sp += 4) {
+#pragma unroll 8
+  for (int sp = warp; sp < ns; sp += NW) {
     const float w = sw[sp];
     if constexpr (DPL == 4) {
       const float4 v = *reinterpret_cast<const float4*>(po + (size_t)sp * D);
@@ -465,9 +484,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   for (int i = 0; i < DPL; ++i) sred[warp][lane * DPL + i] = acc[i];
   __syncthreads();
   const float inv = M == kNegInf ? 0.f : 1.f / lsum;
-  for (int d = tid; d < D; d += 128) {
-    const float o = ((sred[0][d] + sred[1][d]) + (sred[2][d] + sred[3][d])) * inv;
-    reinterpret_cast<T*>(p.out)[(size_t)bh * D + d] = from_f32<T>(o);
+  for (int d = tid; d < D; d += kCombineThreads) {
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) o += sred[w][d];
+    reinterpret_cast<T*>(p.out)[(size_t)bh * D + d] = from_f32<T>(o * inv);
   }
   if (p.lse != nullptr && tid == 0) p.lse[bh] = M == kNegInf ? kNegInf : (M + log2f(lsum)) * 0.69314718055994531f;
 }

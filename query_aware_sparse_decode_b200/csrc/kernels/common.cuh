@@ -1,6 +1,8 @@
 // Device helpers shared by the decode hot-path kernels (sm_100a).
 #pragma once
 
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -67,6 +69,16 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 }
 
 // ------------------------------------------------------------ cp.async (LDGSTS)
+// Programmatic dependent launch.  Every kernel of the decode chain starts with
+// pdl_wait() (returns once the stream's preceding kernel has completed and its
+// writes are visible; a no-op for a normal launch) and then pdl_trigger()
+// (lets the next kernel be scheduled onto SMs this grid frees), so the launch
+// latency and prologue of kernel i+1 overlap the tail of kernel i.  All CTAs
+// execute the wait before any global access or early return, which keeps the
+// order of every kernel pair in the stream transitive.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ void cp_async_16(void* smem, const void* gmem) {
@@ -201,4 +213,23 @@ __device__ __forceinline__ uint2 block_excl_scan2(uint2 v, uint2& total, uint2* 
   return make_uint2(base.x + x.x - v.x, base.y + x.y - v.y);
 }
 
+// Host: launch a kernel with programmatic stream serialization allowed (the
+// kernel must begin with pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 }  // namespace tb
+

@@ -25,6 +25,8 @@ struct AppendParams {
 // dimensions, added in a fixed order).
 template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float krow[128];
   __shared__ float wsm[128 * 32];
   __shared__ float part[128];
@@ -32,7 +34,19 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   const size_t src = ((size_t)b * p.Hkv + g) * p.D;
   const size_t row = ((size_t)b * p.Hkv + g) * p.max_len + p.pos[b];
   const T* W = reinterpret_cast<const T*>(p.w_k);
-  for (int e = tid; e < p.D * p.dimp; e += 128) wsm[e] = to_f32(W[e]);
+  const int nw = p.D * p.dimp;
+  constexpr int VEC = 16 / (int)sizeof(T);  // W_K staged with 16-byte loads, all in flight
+  if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && nw % VEC == 0) {
+#pragma unroll 8
+    for (int e = tid * VEC; e < nw; e += 128 * VEC) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(W + e);
+      const T* el = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) wsm[e + i] = to_f32(el[i]);
+    }
+  } else {
+    for (int e = tid; e < nw; e += 128) wsm[e] = to_f32(W[e]);
+  }
   if (tid < p.D) {
     const T kv = reinterpret_cast<const T*>(p.k_new)[src + tid];
     reinterpret_cast<T*>(p.k_cache)[row * p.D + tid] = kv;

@@ -7,9 +7,10 @@
 // inside a tile ([b][g][t/256][j][t%256], see kimp_index), read once per KV head
 // and shared by the Hq/Hkv query heads of the group.  A thread scores four
 // consecutive tokens: d' independent, coalesced 16-byte loads per group of
-// four tokens, fp32 FMA in dimension order j = 0..d'-1, the group's query
-// values broadcast from shared memory.  Small register footprint, high
-// occupancy: latency is hidden by many loads in flight, not by a pipeline.
+// four tokens, written as batches of 16 loads ahead of their FMAs (fp32,
+// dimension order j = 0..d'-1, the group's query values broadcast from
+// shared memory) so that many loads per thread can be in flight.  A CTA covers 1, 2 or 4 groups of
+// 1024 tokens (the launch picks the count so the grid fills the SMs).
 // Optionally each CTA accumulates, per query-head row, the histogram of the
 // top 11 bits of the order key over the candidate range [sink, len - window)
 // (the first radix digit of the selection) and flushes it with global atomics.
@@ -20,8 +21,8 @@
 namespace tb {
 
 constexpr int kScoreThreads = 256;
-constexpr int kScoreIters = 4;                                  // groups of 4 tokens per thread
-constexpr int kScoreChunk = kScoreThreads * 4 * kScoreIters;    // tokens per CTA
+constexpr int kScoreStep = kScoreThreads * 4;   // tokens per CTA iteration (4 per thread)
+constexpr int kScoreLoadBatch = 16;             // float4 loads issued before their FMAs
 
 struct ScoreParams {
   const void* q_imp;   // [(B*Hq)][G][1][d'] of the producer, kv dtype
@@ -30,16 +31,19 @@ struct ScoreParams {
   uint32_t* hist;      // [B*Hq][2048] or nullptr
   int G, slot, Hq, Hkv, max_len;
   int sink, window;
+  int iters;           // CTA iterations of kScoreStep tokens (1, 2 or 4)
   int lens[kMaxBatch];
 };
 
 template <typename T, int DIMP, int GS, bool HIST>
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScoreParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) float qs[DIMP][GS];
   extern __shared__ uint32_t hist[];  // [GS][2048] when HIST
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.lens[b];
-  const int t_base = chunk * kScoreChunk;
+  const int t_base = chunk * kScoreStep * p.iters;
   if (t_base >= L) return;
   const T* qi = reinterpret_cast<const T*>(p.q_imp);
   for (int e = tid; e < DIMP * GS; e += kScoreThreads) {
@@ -52,24 +56,31 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
 
   const size_t slab = (size_t)b * p.Hkv + g;
   float* S = p.scores + ((size_t)b * p.Hq + g * GS) * p.max_len;
+  static_assert(DIMP % kScoreLoadBatch == 0 || DIMP < kScoreLoadBatch, "d' must be a multiple of the batch");
+  constexpr int NB = DIMP < kScoreLoadBatch ? DIMP : kScoreLoadBatch;
 #pragma unroll 1
-  for (int it = 0; it < kScoreIters; ++it) {
-    const int t0 = t_base + it * 4 * kScoreThreads + 4 * tid;
+  for (int it = 0; it < p.iters; ++it) {
+    const int t0 = t_base + it * kScoreStep + 4 * tid;
     if (t0 < L) {
       const float* K = p.kimp + kimp_index(slab, 0, t0, DIMP, p.max_len);
       float acc[GS][4];
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh) acc[hh][0] = acc[hh][1] = acc[hh][2] = acc[hh][3] = 0.f;
 #pragma unroll
-      for (int j = 0; j < DIMP; ++j) {
-        const float4 v = __ldcs(reinterpret_cast<const float4*>(K + j * kKimpTile));
+      for (int j0 = 0; j0 < DIMP; j0 += NB) {
+        float4 v[NB];
 #pragma unroll
-        for (int hh = 0; hh < GS; ++hh) {
-          const float qv = qs[j][hh];
-          acc[hh][0] = fmaf(qv, v.x, acc[hh][0]);
-          acc[hh][1] = fmaf(qv, v.y, acc[hh][1]);
-          acc[hh][2] = fmaf(qv, v.z, acc[hh][2]);
-          acc[hh][3] = fmaf(qv, v.w, acc[hh][3]);
+        for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const float4*>(K + (j0 + jj) * kKimpTile));
+#pragma unroll
+        for (int jj = 0; jj < NB; ++jj) {
+#pragma unroll
+          for (int hh = 0; hh < GS; ++hh) {
+            const float qv = qs[j0 + jj][hh];
+            acc[hh][0] = fmaf(qv, v[jj].x, acc[hh][0]);
+            acc[hh][1] = fmaf(qv, v[jj].y, acc[hh][1]);
+            acc[hh][2] = fmaf(qv, v[jj].z, acc[hh][2]);
+            acc[hh][3] = fmaf(qv, v[jj].w, acc[hh][3]);
+          }
         }
       }
 #pragma unroll
@@ -103,6 +114,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
 
 // zero the first-digit histograms before a fused score pass
 __global__ void zero_u32_kernel(uint32_t* p, size_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
 }
 

@@ -22,9 +22,14 @@
 //            and ties at T go to the lowest indices (a radix select on the
 //            index when more ties than needed); their mask bits are set.
 //            Then the count check and, if asked, the ascending index list.
-// A row whose threshold bin holds more candidates than the buffer falls back
-// to three radix sweeps over the whole row and an ordered ballot/scan
-// compaction, all inside the resolve CTA.
+//   refine   (single-row selections: soft voting) many CTAs per row: when the
+//            threshold bin of the first digit holds more candidates than the
+//            buffer, the second digit is histogrammed over that bin, and the
+//            scatter then splits the row at a 22-bit prefix instead of 11.
+// A row whose threshold bin still holds more candidates than the buffer (or
+// one of whose chunks overflowed its staging buffer) falls back to radix
+// sweeps over the whole row and an ordered ballot/scan compaction, all inside
+// the resolve CTA.
 #pragma once
 
 #include "common.cuh"
@@ -42,9 +47,10 @@ constexpr int kScatSmem = kHistBins * 4 + kScatCap * 8;
 struct SelectParams {
   const float* scores;    // row r of sequence b at (b * rows_per_seq + r) * row_stride
   uint32_t* hist1;        // [B*rows][2048] first-digit histograms of the candidates
+  uint32_t* hist2;        // [B][2048] second-digit histograms (rows_per_seq == 1), or nullptr
   uint32_t* cand;         // [B*rows][kSelCap][2]: (key, token) of threshold-bin candidates
   uint32_t* ccount;       // [B*rows] candidates appended (zero before the scatter)
-  uint4* rowinfo;         // [B*rows] (b1, k1, n1, -): first digit, rank left in it, its count
+  uint4* rowinfo;         // [B*rows] (prefix, rank left in it, its count, digits in the prefix)
   int32_t* idx;           // [B*rows][idx_cap] or nullptr
   int32_t* count;         // [B*rows] or nullptr
   uint32_t* mask;         // [B*rows][mask_words] (always written)
@@ -115,6 +121,8 @@ __device__ __forceinline__ RowShape row_shape(const SelectParams& p, int b) {
 // ---------------------------------------------------------------- hist
 // grid (chunks, rows, B): first-digit histogram of the candidates of a chunk.
 __global__ void __launch_bounds__(kScatThreads) select_hist_kernel(const SelectParams p) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint32_t hist[kHistBins];
   const int chunk = blockIdx.x, r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const RowShape rs = row_shape(p, b);
@@ -132,10 +140,56 @@ __global__ void __launch_bounds__(kScatThreads) select_hist_kernel(const SelectP
     if (hist[i]) atomicAdd(&p.hist1[row * kHistBins + i], hist[i]);
 }
 
+// ---------------------------------------------------------------- refine
+// grid (chunks of kRefChunk tokens, 1, B), one row per sequence: where the
+// first digit's threshold bin holds more candidates than the resolve buffer,
+// histogram the second digit (bits 20..10 of the key) of the keys in that bin.
+constexpr int kRefChunk = 2048;
+__global__ void __launch_bounds__(kScatThreads) select_refine_kernel(const SelectParams p) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t scan_sm[32];
+  __shared__ int s_bin;
+  __shared__ uint32_t s_above;
+  const int chunk = blockIdx.x, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31;
+  const RowShape rs = row_shape(p, b);
+  const int t_begin = chunk * kRefChunk;
+  if (rs.mode != 2 || t_begin >= rs.hi || t_begin + kRefChunk <= rs.lo) return;
+  const long long row = b;
+  for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = p.hist1[row * kHistBins + i];
+  __syncthreads();
+  find_bin<kHistBins / kScatThreads, kScatThreads>(hist, (uint32_t)rs.k, scan_sm, &s_bin, &s_above);
+  const uint32_t b1 = (uint32_t)s_bin;
+  if (hist[b1] <= (uint32_t)kSelCap) return;  // the same decision in every thread
+  __syncthreads();
+  for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = 0;
+  __syncthreads();
+  const float* s = p.scores + row * p.row_stride;
+  const int t_end = min(t_begin + kRefChunk, rs.hi);
+  for (int base = t_begin; base < t_end; base += kScatThreads) {  // warp-uniform bounds
+    const int t = base + tid;
+    bool in = false;
+    uint32_t bin = 0xFFFFFFFFu;
+    if (t >= rs.lo && t < t_end) {
+      const uint32_t key = order_key(s[t]);
+      in = (key >> 21) == b1;
+      if (in) bin = (key >> 10) & (kHistBins - 1);
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+  }
+  __syncthreads();
+  for (int i = tid; i < kHistBins; i += kScatThreads)
+    if (hist[i]) atomicAdd(&p.hist2[row * kHistBins + i], hist[i]);
+}
+
 // ---------------------------------------------------------------- scatter
 // grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
 // of the CTA's chunk, all loaded up front (8 float4 per lane).
-__global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kScatThreads, 5) select_scatter_kernel(const SelectParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint32_t scat_smem[];
   uint32_t* hist = scat_smem;               // [2048]
   uint32_t* lkey = hist + kHistBins;        // [kScatCap]
@@ -152,16 +206,30 @@ __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const Sele
   const float* s = p.scores + row * p.row_stride;
   float f_lo = 0.f, f_hi = 0.f;
   bool hi_open = false;
+  bool collect = false;  // candidates are gathered only when the resolve buffer can hold the bin
   if (rs.mode == 2) {
     for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = p.hist1[row * kHistBins + i];
     if (tid == 0) s_n = 0;
     __syncthreads();
     find_bin<kHistBins / kScatThreads, kScatThreads>(hist, (uint32_t)rs.k, scan_sm, &s_bin, &s_above);
-    f_lo = key_to_float((uint32_t)s_bin << 21);           // smallest key of the threshold bin
-    f_hi = key_to_float(((uint32_t)s_bin + 1u) << 21);    // smallest key above it
-    hi_open = s_bin == kHistBins - 1;
-    if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's first digit from here
-      p.rowinfo[row] = make_uint4((uint32_t)s_bin, (uint32_t)rs.k - s_above, hist[s_bin], 0u);
+    uint32_t prefix = (uint32_t)s_bin, kleft = (uint32_t)rs.k - s_above, nbin = hist[s_bin];
+    int shift = 21;
+    if (p.hist2 != nullptr && nbin > (uint32_t)kSelCap) {  // split the bin by the second digit
+      __syncthreads();
+      for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = p.hist2[(size_t)b * kHistBins + i];
+      __syncthreads();
+      find_bin<kHistBins / kScatThreads, kScatThreads>(hist, kleft, scan_sm, &s_bin, &s_above);
+      prefix = (prefix << 11) | (uint32_t)s_bin;
+      kleft -= s_above;
+      nbin = hist[s_bin];
+      shift = 10;
+    }
+    f_lo = key_to_float(prefix << shift);          // smallest key of the threshold bin
+    f_hi = key_to_float((prefix + 1u) << shift);   // smallest key above it
+    hi_open = prefix == (0xFFFFFFFFu >> shift);
+    collect = nbin <= (uint32_t)kSelCap;
+    if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's prefix from here
+      p.rowinfo[row] = make_uint4(prefix, kleft, nbin, shift == 21 ? 1u : 2u);
   }
   // a warp step covers 256 tokens: lane owns 8 consecutive tokens (two float4),
   // lanes 4m..4m+3 form mask word m of the step
@@ -213,6 +281,7 @@ __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const Sele
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
     word |= __shfl_xor_sync(0xffffffffu, word, 2);
     if ((lane & 3) == 0 && t0 < rs.L) p.mask[row * p.mask_words + (t0 >> 5)] = word;
+    if (!collect) cbits = 0;
     if (__any_sync(0xffffffffu, cbits != 0)) {
       const uint32_t cnt = __popc(cbits);
       uint32_t x = cnt;  // inclusive prefix over the lanes
@@ -236,12 +305,14 @@ __global__ void __launch_bounds__(kScatThreads) select_scatter_kernel(const Sele
       }
     }
   }
-  if (rs.mode != 2) return;
+  if (rs.mode != 2 || !collect) return;
   __syncthreads();
   const uint32_t n = min(s_n, (uint32_t)kScatCap);
   if (tid == 0) {
     s_base = atomicAdd(&p.ccount[row], s_n);
-    if (s_n > (uint32_t)kScatCap) atomicOr(p.status, TB_DEV_ERR_COUNT);
+    // this chunk held more of the bin than its staging buffer: the list is
+    // incomplete, so the resolve CTA takes the whole-row path for this row
+    if (s_n > (uint32_t)kScatCap) atomicOr(&p.ccount[row], 0x80000000u);
   }
   __syncthreads();
   uint32_t* dst = p.cand + (size_t)row * kSelCap * 2;
@@ -293,6 +364,8 @@ __device__ __forceinline__ void smem_radix(int n, Key key_of, int first_pass, ui
 }
 
 __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const SelectParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint32_t res_smem[];
   uint32_t* hist = res_smem;            // [2048]
   uint32_t* ckey = hist + kHistBins;    // [kSelCap]
@@ -309,16 +382,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
   const int lwords = (L + 31) >> 5;
 
   bool fallback = false;
-  int b1 = 0;
-  uint32_t k1 = 0, n1 = 0;
+  uint32_t prefix1 = 0, k1 = 0, n1 = 0;
+  int next_pass = 1;  // digits already fixed by the scatter: 1 or 2
   if (mode == 2) {
     const uint4 info = p.rowinfo[row];
-    b1 = (int)info.x;
+    prefix1 = info.x;
     k1 = info.y;
     n1 = info.z;
+    next_pass = info.w == 2u ? 2 : 1;
     fallback = n1 > (uint32_t)kSelCap;
   }
 
+  if (mode == 2 && !fallback) fallback = (p.ccount[row] >> 31) != 0u;  // a staging buffer overflowed
   if (!fallback) {
     if (mode == 2) {
       uint32_t n = p.ccount[row];
@@ -340,7 +415,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
             key = ckey[i];
             return true;
           },
-          1, (uint32_t)b1, k1, hist, scan_sm, &s_bin, &s_above, T, quota);
+          next_pass, prefix1, k1, hist, scan_sm, &s_bin, &s_above, T, quota);
       // ties at T: keep the `quota` lowest indices
       uint32_t ntie_local = 0;
       for (uint32_t i = tid; i < n; i += kSelThreads) ntie_local += ckey[i] == T;
@@ -396,9 +471,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
   // ================================================================ fallback
   uint32_t T, quota;
   {
-    uint32_t prefix = (uint32_t)b1, kk = k1;
+    uint32_t prefix = prefix1, kk = k1;
 #pragma unroll 1
-    for (int pass = 1; pass < 3; ++pass) {
+    for (int pass = next_pass; pass < 3; ++pass) {
       const int shift = pass == 1 ? 10 : 0;
       const int nbits = pass == 1 ? 11 : 10;
       const int pshift = pass == 1 ? 21 : 10;

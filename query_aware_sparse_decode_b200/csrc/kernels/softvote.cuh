@@ -13,8 +13,12 @@
 // cp.async into a swizzled ring, q . K^T on mma.sync (bf16 in, fp32
 // accumulate); writes the logits in the log2 domain and one (max, sum of
 // 2^(a - max)) pair per head and chunk.
-// softvote_reduce: merges the chunk pairs into each head's (M, Z) and sums
-// 2^(a - M) / Z over the heads for every token (logits are L2-resident).
+// softvote_reduce: merges the chunk pairs into each head's (M, Z) (a warp per
+// head, lanes over the chunks) and sums 2^(a - M) / Z over the heads for four
+// consecutive tokens per thread (logits are L2-resident).  Optionally it also
+// builds the first-digit histogram of the votes over the candidate range
+// [sink, len - window) for the selection that follows (warp-aggregated shared
+// atomics: votes crowd into few bins).
 #pragma once
 
 #include "attn.cuh"
@@ -30,13 +34,17 @@ struct VoteParams {
   float* logits;        // [B][Hq][max_len], log2 domain
   float* stats;         // [B][Hq][nchunk][2]
   float* votes;         // [B][max_len]
+  uint32_t* hist1;      // [B][2048] first-digit histograms of the votes, or nullptr
   int Hq, Hkv, max_len, nchunk;
+  int sink, window;
   float scale_log2;
   int lens[kMaxBatch];
 };
 
 template <int D, int GS>
 __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const VoteParams p) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int ROWB = D * 2;
   constexpr int NCH = D / 8;
   constexpr int STAGE = kAttnTile * ROWB;  // K only
@@ -156,30 +164,78 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
 }
 
 // grid (ceil(max len / 1024), B), block 256: votes for 1024 tokens per CTA.
-__global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
-  __shared__ float sM[256], sInvZ[256];
-  const int b = blockIdx.y;
+constexpr int kVoteMaxHeads = 128;
+__global__ void __launch_bounds__(256, 1) softvote_reduce_kernel(const VoteParams p) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float sM[kVoteMaxHeads], sInvZ[kVoteMaxHeads];
+  __shared__ uint32_t hist[kHistBins];
+  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = p.lens[b];
   const int t_begin = blockIdx.x * 1024;
   if (t_begin >= L) return;
   const int nch = (L + kVoteChunk - 1) / kVoteChunk;
-  for (int h = threadIdx.x; h < p.Hq; h += blockDim.x) {
-    const float* st = p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2;
-    float M = kNegInf;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, st[2 * c]);
-    float Z = 0.f;
-    for (int c = 0; c < nch; ++c)
-      if (st[2 * c] != kNegInf) Z += st[2 * c + 1] * exp2f(st[2 * c] - M);
-    sM[h] = M;
-    sInvZ[h] = 1.f / Z;
+  for (int h = warp; h < p.Hq; h += 8) {
+    const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
+    float m = kNegInf, l = 0.f;
+    for (int c = lane; c < nch; c += 32) {  // per lane: merge its chunks
+      const float2 e = st[c];
+      if (e.x == kNegInf) continue;
+      const float mn = fmaxf(m, e.x);
+      l = l * exp2f(m - mn) + e.y * exp2f(e.x - mn);
+      m = mn;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      const float mn = fmaxf(m, m2);
+      if (mn != kNegInf) {
+        l = (m == kNegInf ? 0.f : l * exp2f(m - mn)) + (m2 == kNegInf ? 0.f : l2 * exp2f(m2 - mn));
+        m = mn;
+      }
+    }
+    if (lane == 0) {
+      sM[h] = m;
+      sInvZ[h] = 1.f / l;
+    }
+  }
+  if (p.hist1 != nullptr)
+    for (int i = tid; i < kHistBins; i += 256) hist[i] = 0;
+  __syncthreads();
+  const int t0 = t_begin + 4 * tid;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (t0 < L) {
+    const float* lg = p.logits + (size_t)b * p.Hq * p.max_len + t0;
+#pragma unroll 8
+    for (int h = 0; h < p.Hq; ++h) {
+      const float4 a = *reinterpret_cast<const float4*>(lg + (size_t)h * p.max_len);
+      const float M = sM[h], iz = sInvZ[h];
+      v[0] += exp2f(a.x - M) * iz;
+      v[1] += exp2f(a.y - M) * iz;
+      v[2] += exp2f(a.z - M) * iz;
+      v[3] += exp2f(a.w - M) * iz;
+    }
+    float* out = p.votes + (size_t)b * p.max_len + t0;
+    if (t0 + 3 < L) {
+      *reinterpret_cast<float4*>(out) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (t0 + u < L) out[u] = v[u];
+    }
+  }
+  if (p.hist1 == nullptr) return;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int t = t0 + u;
+    const bool in = t < L && t >= p.sink && t < L - p.window;
+    const uint32_t bin = in ? (order_key(v[u]) >> 21) : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
   }
   __syncthreads();
-  for (int t = t_begin + threadIdx.x; t < min(t_begin + 1024, L); t += blockDim.x) {
-    float v = 0.f;
-    for (int h = 0; h < p.Hq; ++h)
-      v += exp2f(p.logits[((size_t)b * p.Hq + h) * p.max_len + t] - sM[h]) * sInvZ[h];
-    p.votes[(size_t)b * p.max_len + t] = v;
-  }
+  for (int i = tid; i < kHistBins; i += 256)
+    if (hist[i]) atomicAdd(&p.hist1[(size_t)b * kHistBins + i], hist[i]);
 }
 
 }  // namespace tb

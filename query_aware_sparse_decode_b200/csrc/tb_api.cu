@@ -37,7 +37,7 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, ccount, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats, total;
+  size_t status, hist, ccount, hist2, hist_end, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats, total;
   int max_splits;
 };
 
@@ -48,7 +48,9 @@ WsLayout layout_of(const tb_config& c) {
   size_t off = 0;
   w.status = off;  off += align256(256);
   w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
-  w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters (zeroed together)
+  w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters and the
+  w.hist2 = off;   off += align256(B * kHistBins * 4);   // single-row second-digit histograms
+  w.hist_end = off;                                      // (zeroed together)
   w.rowinfo = off; off += align256(B * Hq * 16);
   w.cand = off;    off += align256(B * Hq * (size_t)kSelCap * 8);
   w.scores = off;  off += align256(B * Hq * Lm * 4);
@@ -91,6 +93,7 @@ struct tb_ctx {
   uint32_t* status = nullptr;
   uint32_t* hist = nullptr;
   uint32_t* ccount = nullptr;
+  uint32_t* hist2 = nullptr;
   uint32_t* cand = nullptr;
   uint4* rowinfo = nullptr;
   float* scores = nullptr;
@@ -145,6 +148,14 @@ static int max_len_of(const LayerState& ls, int B) {
 }
 
 // ------------------------------------------------------------------ launches
+// Zero the selection's histograms and candidate counters (one contiguous
+// workspace range).
+static void launch_zero_hist(tb_ctx* ctx, cudaStream_t st) {
+  const size_t n = (ctx->lay.hist_end - ctx->lay.hist) / 4;
+  launch_pdl(zero_u32_kernel, dim3((unsigned)std::min<size_t>((n + 255) / 256, 1024)), dim3(256), 0, st, ctx->hist, n);
+  ++ctx->launches;
+}
+
 static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
                               cudaStream_t st) {
   const tb_config& c = ctx->cfg;
@@ -162,24 +173,28 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.sink = c.sink;
   p.window = c.window;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  if (hist) {  // histograms and the selection's candidate counters start at zero
-    const size_t n = (size_t)c.batch * c.n_q_heads * (kHistBins + 1);
-    zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(hist, n);
-    ++ctx->launches;
-  }
+  if (hist) launch_zero_hist(ctx, st);  // histograms and candidate counters start at zero
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
   const size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
-  dim3 grid((maxL + kScoreChunk - 1) / kScoreChunk, c.n_kv_heads, c.batch);
+  // the most tokens per CTA (up to 4 steps) that still gives about three
+  // CTAs per SM; short or small batches get one step per CTA
+  int iters = 4;
+  while (iters > 1 && (long long)c.batch * c.n_kv_heads * ((maxL + kScoreStep * iters - 1) / (kScoreStep * iters)) <
+                          3LL * ctx->num_sms)
+    iters >>= 1;
+  p.iters = iters;
+  const int chunk = kScoreStep * iters;
+  dim3 grid((maxL + chunk - 1) / chunk, c.n_kv_heads, c.batch);
 #define TB_SCORE_CASE(T, DI, GSV)                                                            \
   if (c.d_imp == DI && gs == GSV) {                                                          \
     if (hist) {                                                                              \
       auto k = score_kernel<T, DI, GSV, true>;                                               \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);       \
-      k<<<grid, kScoreThreads, smem, st>>>(p);                                               \
+      launch_pdl(k, grid, dim3(kScoreThreads), smem, st, p);                                 \
     } else {                                                                                 \
-      score_kernel<T, DI, GSV, false><<<grid, kScoreThreads, 0, st>>>(p);                    \
+      launch_pdl(score_kernel<T, DI, GSV, false>, grid, dim3(kScoreThreads), 0, st, p);      \
     }                                                                                        \
     ++ctx->launches;                                                                         \
     return cuda_status(cudaGetLastError());                                                  \
@@ -216,6 +231,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   SelectParams p{};
   p.scores = scores;
   p.hist1 = ctx->hist;
+  p.hist2 = rows == 1 ? ctx->hist2 : nullptr;
   p.cand = ctx->cand;
   p.ccount = ctx->ccount;
   p.rowinfo = ctx->rowinfo;
@@ -234,15 +250,19 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   const int maxL = max_len_of(ls, c.batch);
   dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
   if (!hist1_ready) {
-    const size_t n = (size_t)c.batch * c.n_q_heads * (kHistBins + 1);
-    zero_u32_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 1024), 256, 0, st>>>(ctx->hist, n);
-    select_hist_kernel<<<cgrid, kScatThreads, 0, st>>>(p);
-    ctx->launches += 2;
+    launch_zero_hist(ctx, st);
+    launch_pdl(select_hist_kernel, cgrid, dim3(kScatThreads), 0, st, p);
+    ++ctx->launches;
+  }
+  if (rows == 1) {  // one long row per sequence: split a crowded threshold bin further
+    launch_pdl(select_refine_kernel, dim3((std::max(maxL, 1) + kRefChunk - 1) / kRefChunk, 1, c.batch),
+               dim3(kScatThreads), 0, st, p);
+    ++ctx->launches;
   }
   cudaFuncSetAttribute(select_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScatSmem);
-  select_scatter_kernel<<<cgrid, kScatThreads, kScatSmem, st>>>(p);
+  launch_pdl(select_scatter_kernel, cgrid, dim3(kScatThreads), kScatSmem, st, p);
   cudaFuncSetAttribute(select_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kResolveSmem);
-  select_resolve_kernel<<<dim3(rows, c.batch), kSelThreads, kResolveSmem, st>>>(p);
+  launch_pdl(select_resolve_kernel, dim3(rows, c.batch), dim3(kSelThreads), kResolveSmem, st, p);
   ctx->launches += 2;
   return cuda_status(cudaGetLastError());
 }
@@ -285,12 +305,12 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
       auto k = attn_bf16_kernel<DV, GSV>;                                                                   \
       const int smem = attn_bf16_smem_bytes<DV>();                                                          \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
-      k<<<grid, kAttnThreads, smem, st>>>(p);                                                               \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                        \
     } else {                                                                                                \
       auto k = attn_f32_kernel<DV, GSV>;                                                                    \
       const int smem = attn_f32_smem_bytes<DV>();                                                           \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
-      k<<<grid, kAttnThreads, smem, st>>>(p);                                                               \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                        \
     }                                                                                                       \
   } else
     TB_ATTN_CASE(128, 4) TB_ATTN_CASE(128, 2) TB_ATTN_CASE(128, 1) TB_ATTN_CASE(128, 8)
@@ -314,21 +334,27 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   for (int b = 0; b < c.batch; ++b) cp.lens[b] = ls.lens[b];
   const unsigned cgrid = (unsigned)(c.batch * c.n_q_heads);
   if (c.kv_dtype == TB_BF16) {
-    if (c.head_dim == 128) combine_kernel<__nv_bfloat16, 128><<<cgrid, 128, 0, st>>>(cp);
-    else combine_kernel<__nv_bfloat16, 64><<<cgrid, 128, 0, st>>>(cp);
+    if (c.head_dim == 128) launch_pdl(combine_kernel<__nv_bfloat16, 128>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
+    else launch_pdl(combine_kernel<__nv_bfloat16, 64>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
   } else {
-    if (c.head_dim == 128) combine_kernel<float, 128><<<cgrid, 128, 0, st>>>(cp);
-    else combine_kernel<float, 64><<<cgrid, 128, 0, st>>>(cp);
+    if (c.head_dim == 128) launch_pdl(combine_kernel<float, 128>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
+    else launch_pdl(combine_kernel<float, 64>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
   }
   ++ctx->launches;
   trace_point(ctx, 5, st);
   return cuda_status(cudaGetLastError());
 }
 
-static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* votes, cudaStream_t st) {
+static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* votes, uint32_t* hist,
+                                cudaStream_t st) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   if (c.kv_dtype != TB_BF16) return TB_ERR_UNSUPPORTED;
+  if (c.n_q_heads > kVoteMaxHeads) return TB_ERR_UNSUPPORTED;
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return TB_OK;
   const int gs = c.n_q_heads / c.n_kv_heads;
@@ -338,6 +364,9 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   p.logits = ctx->scores;
   p.stats = ctx->vstats;
   p.votes = votes;
+  p.hist1 = hist;
+  p.sink = c.sink;
+  p.window = c.window;
   p.Hq = c.n_q_heads;
   p.Hkv = c.n_kv_heads;
   p.max_len = c.max_len;
@@ -350,7 +379,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
     auto k = softvote_logits_kernel<DV, GSV>;                                                 \
     const int smem = kAttnWarps * kAttnStages * kAttnTile * DV * 2;                           \
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);               \
-    k<<<grid, kAttnThreads, smem, st>>>(p);                                                   \
+    launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                            \
   } else
   TB_VOTE_CASE(128, 4) TB_VOTE_CASE(128, 2) TB_VOTE_CASE(128, 1) TB_VOTE_CASE(128, 8)
   TB_VOTE_CASE(64, 4) TB_VOTE_CASE(64, 2) TB_VOTE_CASE(64, 1) TB_VOTE_CASE(64, 8)
@@ -360,7 +389,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   tb_status s = cuda_status(cudaGetLastError());
   if (s != TB_OK) return s;
   dim3 g2((maxL + 1023) / 1024, c.batch);
-  softvote_reduce_kernel<<<g2, 256, 0, st>>>(p);
+  launch_pdl(softvote_reduce_kernel, g2, dim3(256), 0, st, p);
   ++ctx->launches;
   return cuda_status(cudaGetLastError());
 }
@@ -397,6 +426,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->status = reinterpret_cast<uint32_t*>(ctx->ws + lay.status);
   ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
   ctx->ccount = reinterpret_cast<uint32_t*>(ctx->ws + lay.ccount);
+  ctx->hist2 = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist2);
   ctx->cand = reinterpret_cast<uint32_t*>(ctx->ws + lay.cand);
   ctx->rowinfo = reinterpret_cast<uint4*>(ctx->ws + lay.rowinfo);
   ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
@@ -492,9 +522,9 @@ TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const v
   dim3 grid(c.n_kv_heads, c.batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c.kv_dtype == TB_BF16)
-    append_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(p);
+    launch_pdl(append_kernel<__nv_bfloat16>, grid, dim3(128), 0, st, p);
   else
-    append_kernel<float><<<grid, 128, 0, st>>>(p);
+    launch_pdl(append_kernel<float>, grid, dim3(128), 0, st, p);
   ++ctx->launches;
   s = cuda_status(cudaGetLastError());
   if (s != TB_OK) return s;
@@ -607,10 +637,11 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
   }
   if (c.variant == TB_SOFTVOTE) {
-    s = launch_softvote(ctx, layer, q, ctx->votes, st);
+    launch_zero_hist(ctx, st);
+    s = launch_softvote(ctx, layer, q, ctx->votes, ctx->hist, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
-    s = launch_select(ctx, layer, ctx->votes, false, 1, nullptr, 0, nullptr, ctx->mask, st);
+    s = launch_select(ctx, layer, ctx->votes, true, 1, nullptr, 0, nullptr, ctx->mask, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
@@ -679,7 +710,7 @@ TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float
   if (s != TB_OK) return s;
   if (!q || !votes) return TB_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(votes)) return TB_ERR_SHAPE;
-  return launch_softvote(ctx, layer, q, votes, static_cast<cudaStream_t>(stream));
+  return launch_softvote(ctx, layer, q, votes, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 TB_API tb_status tb_trace_events(tb_ctx* ctx, void* const* events, int n_events) {

@@ -115,12 +115,12 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
       auto k = attn_bf16_kernel<DV, GSV>;                                                     \
       const int smem = attn_bf16_smem_bytes<DV>();                                            \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);             \
-      k<<<grid, kAttnThreads, smem, st>>>(p);                                                 \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                          \
     } else {                                                                                  \
       auto k = attn_f32_kernel<DV, GSV>;                                                      \
       const int smem = attn_f32_smem_bytes<DV>();                                             \
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);             \
-      k<<<grid, kAttnThreads, smem, st>>>(p);                                                 \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                          \
     }                                                                                         \
   } else
   TB_STATIC_ATTN_CASE(128, 4) TB_STATIC_ATTN_CASE(128, 2) TB_STATIC_ATTN_CASE(128, 1) TB_STATIC_ATTN_CASE(128, 8)
@@ -141,11 +141,15 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
   for (int b = 0; b < B; ++b) cp.lens[b] = cache->lens_host[b];
   const unsigned cgrid = (unsigned)(B * Hq);
   if (cache->kv_dtype == TB_BF16) {
-    if (D == 128) combine_kernel<__nv_bfloat16, 128><<<cgrid, 128, 0, st>>>(cp);
-    else combine_kernel<__nv_bfloat16, 64><<<cgrid, 128, 0, st>>>(cp);
+    if (D == 128) launch_pdl(combine_kernel<__nv_bfloat16, 128>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
+    else launch_pdl(combine_kernel<__nv_bfloat16, 64>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
   } else {
-    if (D == 128) combine_kernel<float, 128><<<cgrid, 128, 0, st>>>(cp);
-    else combine_kernel<float, 64><<<cgrid, 128, 0, st>>>(cp);
+    if (D == 128) launch_pdl(combine_kernel<float, 128>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
+    else launch_pdl(combine_kernel<float, 64>, dim3(cgrid), dim3(kCombineThreads), 0, st,
+                    cp);
   }
   return cudaGetLastError() == cudaSuccess ? TB_OK : TB_ERR_CUDA;
 }

@@ -137,6 +137,53 @@ def test_select_bit_exact_on_identical_scores(case):
             assert np.array_equal(got_sets[b, r], ref)
 
 
+def _crowded_scores(kind, L, seed):
+    u = S.fill_host(21, seed, 0, 1, 0, L, 1, "f32").reshape(L).astype(np.float64)
+    u = (u - u.min()) / (u.max() - u.min() + 1e-12)          # in [0, 1)
+    if kind == "one_binade":      # [1, 2): the first digit has 4 occupied bins
+        x = 1.0 + u
+    elif kind == "two_digits":    # [1, 1 + 2**-12): the first two digits leave 2 bins
+        x = 1.0 + np.floor(u * 2048) * 2.0 ** -23
+    else:                         # three values: ties decide almost the whole budget
+        x = np.floor(u * 3) - 1.0
+    return x.astype(np.float32)
+
+
+@pytest.mark.parametrize("kind", ["one_binade", "two_digits", "three_values"])
+@pytest.mark.parametrize("keep", [10, 50])
+def test_single_row_select_on_crowded_bins(kind, keep):
+    """One shared row per sequence (the soft-voting shape) whose top digits
+    leave far more candidates in the threshold bin than the resolve buffer
+    holds: the second-digit refinement and the whole-row fallback must still
+    give exactly the oracle's set (identical fp32 scores)."""
+    lens = (200000, 150001)
+    B = len(lens)
+    wl = S.Workload("sel1", n_layers=1, B=B, Hq=1, Hkv=1, D=64, d_imp=16, G=1, L=max(lens), dtype="f32",
+                    keep_pct=keep, sink=16, window=64, plant="none", lens=lens)
+    cfg = config_of(wl)
+    Lmax = cfg.max_len
+    ctx = TB.Context(cfg)
+    dummy = torch.zeros((B, 1, Lmax, 64), device="cuda")
+    ctx.bind_layer(0, dummy, dummy.clone(), kimp_alloc(B, 1, 16, Lmax), torch.zeros((64, 16), device="cuda"))
+    ctx.set_seq_lens(0, lens)
+    sc = np.zeros((B, Lmax), np.float32)
+    for b, L in enumerate(lens):
+        sc[b, :L] = _crowded_scores(kind, L, 7 + b)
+    idx = torch.full((B, 1, max(lens)), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B, 1), -1, dtype=torch.int32, device="cuda")
+    mask = torch.zeros((B, 1, Lmax // 32), dtype=torch.int32, device="cuda")
+    ctx.select(0, torch.from_numpy(sc).cuda(), 1, idx=idx, count=cnt, mask=mask)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    got_sets = sets_from_mask(mask, lens)
+    for b, L in enumerate(lens):
+        ref = O.select_tokens(sc[b].astype(np.float64), L, keep, wl.sink, wl.window)
+        assert cnt[b, 0] == ref.size
+        assert np.array_equal(idx[b, 0, :ref.size], ref)
+        assert np.array_equal(got_sets[b, 0], ref)
+
+
 # --------------------------------------------------------------------------- a6
 @pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
 def test_sparse_attn_on_oracle_sets(wl):
