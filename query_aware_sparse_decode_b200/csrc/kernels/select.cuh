@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kScatThreads) select_refine_kernel(const Selec
 // ---------------------------------------------------------------- scatter
 // grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
 // of the CTA's chunk, all loaded up front (8 float4 per lane).
-__global__ void __launch_bounds__(kScatThreads, 5) select_scatter_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const SelectParams p) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint32_t scat_smem[];
@@ -204,6 +204,20 @@ __global__ void __launch_bounds__(kScatThreads, 5) select_scatter_kernel(const S
   if (t_begin >= rs.L) return;
   const long long row = (long long)b * p.rows_per_seq + r;
   const float* s = p.scores + row * p.row_stride;
+  // the chunk's scores are requested first, so their latency overlaps the
+  // threshold search below.  A warp step covers 256 tokens: lane owns 8
+  // consecutive tokens (two float4), lanes 4m..4m+3 form mask word m
+  constexpr int STEPS = 4;
+  const int wt0 = t_begin + warp * 1024;
+  float4 v[STEPS][2];
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u) {
+    const int t0 = wt0 + u * 256 + 8 * lane;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      v[u][h] = (rs.mode == 2 && t0 + 4 * h < rs.L) ? *reinterpret_cast<const float4*>(s + t0 + 4 * h)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float f_lo = 0.f, f_hi = 0.f;
   bool hi_open = false;
   bool collect = false;  // candidates are gathered only when the resolve buffer can hold the bin
@@ -230,19 +244,6 @@ __global__ void __launch_bounds__(kScatThreads, 5) select_scatter_kernel(const S
     collect = nbin <= (uint32_t)kSelCap;
     if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's prefix from here
       p.rowinfo[row] = make_uint4(prefix, kleft, nbin, shift == 21 ? 1u : 2u);
-  }
-  // a warp step covers 256 tokens: lane owns 8 consecutive tokens (two float4),
-  // lanes 4m..4m+3 form mask word m of the step
-  constexpr int STEPS = 4;
-  const int wt0 = t_begin + warp * 1024;
-  float4 v[STEPS][2];
-#pragma unroll
-  for (int u = 0; u < STEPS; ++u) {
-    const int t0 = wt0 + u * 256 + 8 * lane;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      v[u][h] = (rs.mode == 2 && t0 + 4 * h < rs.L) ? *reinterpret_cast<const float4*>(s + t0 + 4 * h)
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int u = 0; u < STEPS; ++u) {
@@ -363,6 +364,16 @@ __device__ __forceinline__ void smem_radix(int n, Key key_of, int first_pass, ui
   quota = kk;
 }
 
+// The resolve CTA of a row is the last reader of its histograms and candidate
+// counter: it clears them for the next selection (so no separate zeroing pass
+// precedes the next score kernel).
+__device__ __forceinline__ void clear_row_state(const SelectParams& p, long long row, int b) {
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) p.hist1[row * kHistBins + i] = 0u;
+  if (p.hist2 != nullptr)
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) p.hist2[(size_t)b * kHistBins + i] = 0u;
+  if (threadIdx.x == 0) p.ccount[row] = 0u;
+}
+
 __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const SelectParams p) {
   pdl_wait();
   pdl_trigger();
@@ -465,6 +476,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
       const int win_lo = max(L - p.window, sink_n);
       if (total != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
     }
+    clear_row_state(p, row, b);
     return;
   }
 
@@ -570,6 +582,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
     const int win_lo = max(L - p.window, sink_n);
     if (out_base != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
   }
+  clear_row_state(p, row, b);
 }
 
 }  // namespace tb

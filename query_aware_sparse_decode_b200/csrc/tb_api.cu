@@ -102,6 +102,7 @@ struct tb_ctx {
   float* part_ml = nullptr;
   float* votes = nullptr;
   float* vstats = nullptr;
+  bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last resolve)
   cudaEvent_t trace[6] = {};
   bool tracing = false;
   unsigned long long launches = 0;
@@ -156,6 +157,13 @@ static void launch_zero_hist(tb_ctx* ctx, cudaStream_t st) {
   ++ctx->launches;
 }
 
+// Before a pass that accumulates into the histograms: zero them unless the
+// previous selection's resolve kernels already did.
+static void prepare_hist(tb_ctx* ctx, cudaStream_t st) {
+  if (!ctx->hist_clean) launch_zero_hist(ctx, st);
+  ctx->hist_clean = false;
+}
+
 static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
                               cudaStream_t st) {
   const tb_config& c = ctx->cfg;
@@ -173,7 +181,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.sink = c.sink;
   p.window = c.window;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  if (hist) launch_zero_hist(ctx, st);  // histograms and candidate counters start at zero
+  if (hist) prepare_hist(ctx, st);  // histograms and candidate counters start at zero
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
@@ -250,7 +258,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   const int maxL = max_len_of(ls, c.batch);
   dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
   if (!hist1_ready) {
-    launch_zero_hist(ctx, st);
+    prepare_hist(ctx, st);
     launch_pdl(select_hist_kernel, cgrid, dim3(kScatThreads), 0, st, p);
     ++ctx->launches;
   }
@@ -264,7 +272,9 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   cudaFuncSetAttribute(select_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kResolveSmem);
   launch_pdl(select_resolve_kernel, dim3(rows, c.batch), dim3(kSelThreads), kResolveSmem, st, p);
   ctx->launches += 2;
-  return cuda_status(cudaGetLastError());
+  const tb_status s = cuda_status(cudaGetLastError());
+  if (s == TB_OK) ctx->hist_clean = true;  // every resolve CTA clears its row's state
+  return s;
 }
 
 static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mode, void* out,
@@ -637,7 +647,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
   }
   if (c.variant == TB_SOFTVOTE) {
-    launch_zero_hist(ctx, st);
+    prepare_hist(ctx, st);
     s = launch_softvote(ctx, layer, q, ctx->votes, ctx->hist, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
