@@ -50,6 +50,7 @@ struct SelectParams {
   uint32_t* hist2;        // [B][2048] second-digit histograms (rows_per_seq == 1), or nullptr
   uint32_t* cand;         // [B*rows][kSelCap][2]: (key, token) of threshold-bin candidates
   uint32_t* ccount;       // [B*rows] candidates appended (zero before the scatter)
+  uint32_t* kcount;       // [B*rows] tokens kept by the scatter (zero before the scatter)
   uint4* rowinfo;         // [B*rows] (prefix, rank left in it, its count, digits in the prefix)
   int32_t* idx;           // [B*rows][idx_cap] or nullptr
   int32_t* count;         // [B*rows] or nullptr
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kScatThreads) select_refine_kernel(const Selec
 
 // ---------------------------------------------------------------- scatter
 // grid (chunks, rows, B), 256 threads: warp w owns tokens [w*1024, w*1024+1024)
-// of the CTA's chunk, all loaded up front (8 float4 per lane).
+// of the CTA's chunk, all loaded up front (8 float4 per lane).  The CTA's
+// kept-token count goes to a per-row counter that the resolve kernel checks.
 __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const SelectParams p) {
   pdl_wait();
   pdl_trigger();
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
   uint32_t* lidx = lkey + kScatCap;         // [kScatCap]
   __shared__ uint32_t scan_sm[32];
   __shared__ int s_bin;
-  __shared__ uint32_t s_above, s_n, s_base;
+  __shared__ uint32_t s_above, s_n, s_base, s_kept;
   const int chunk = blockIdx.x, r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const RowShape rs = row_shape(p, b);
@@ -221,9 +223,12 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
   float f_lo = 0.f, f_hi = 0.f;
   bool hi_open = false;
   bool collect = false;  // candidates are gathered only when the resolve buffer can hold the bin
+  if (tid == 0) {
+    s_n = 0;
+    s_kept = 0;
+  }
   if (rs.mode == 2) {
     for (int i = tid; i < kHistBins; i += kScatThreads) hist[i] = p.hist1[row * kHistBins + i];
-    if (tid == 0) s_n = 0;
     __syncthreads();
     find_bin<kHistBins / kScatThreads, kScatThreads>(hist, (uint32_t)rs.k, scan_sm, &s_bin, &s_above);
     uint32_t prefix = (uint32_t)s_bin, kleft = (uint32_t)rs.k - s_above, nbin = hist[s_bin];
@@ -244,7 +249,10 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
     collect = nbin <= (uint32_t)kSelCap;
     if (chunk == 0 && tid == 0)  // the resolve CTA reads the row's prefix from here
       p.rowinfo[row] = make_uint4(prefix, kleft, nbin, shift == 21 ? 1u : 2u);
+  } else {
+    __syncthreads();
   }
+  uint32_t kept = 0;  // tokens of the words this lane stores
 #pragma unroll
   for (int u = 0; u < STEPS; ++u) {
     const int tw = wt0 + u * 256;
@@ -281,7 +289,10 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
     uint32_t word = keep << ((lane & 3) * 8);
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
     word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if ((lane & 3) == 0 && t0 < rs.L) p.mask[row * p.mask_words + (t0 >> 5)] = word;
+    if ((lane & 3) == 0 && t0 < rs.L) {
+      p.mask[row * p.mask_words + (t0 >> 5)] = word;
+      kept += __popc(word);
+    }
     if (!collect) cbits = 0;
     if (__any_sync(0xffffffffu, cbits != 0)) {
       const uint32_t cnt = __popc(cbits);
@@ -306,8 +317,12 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
       }
     }
   }
-  if (rs.mode != 2 || !collect) return;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+  if (lane == 0 && kept) atomicAdd(&s_kept, kept);
   __syncthreads();
+  if (tid == 0 && s_kept) atomicAdd(&p.kcount[row], s_kept);
+  if (rs.mode != 2 || !collect) return;
   const uint32_t n = min(s_n, (uint32_t)kScatCap);
   if (tid == 0) {
     s_base = atomicAdd(&p.ccount[row], s_n);
@@ -371,7 +386,10 @@ __device__ __forceinline__ void clear_row_state(const SelectParams& p, long long
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) p.hist1[row * kHistBins + i] = 0u;
   if (p.hist2 != nullptr)
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) p.hist2[(size_t)b * kHistBins + i] = 0u;
-  if (threadIdx.x == 0) p.ccount[row] = 0u;
+  if (threadIdx.x == 0) {
+    p.ccount[row] = 0u;
+    p.kcount[row] = 0u;
+  }
 }
 
 __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const SelectParams p) {
@@ -452,14 +470,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
       __threadfence_block();
       __syncthreads();
     }
-    // ---- count check and optional ascending index list (mask read back)
-    const int per = (lwords + kSelThreads - 1) / kSelThreads;
-    const int w0 = min(lwords, tid * per), w1 = min(lwords, w0 + per);
-    uint32_t mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(__ldcg(p.mask + orow * p.mask_words + w));
-    uint32_t total;
-    uint32_t pos = block_excl_scan<kSelThreads>(mine, total, scan_sm);
+    // ---- count check and optional ascending index list.  Without a list the
+    // count is the scatter's kept tokens plus the k1 candidates marked here
+    // (exactly k1 by construction); with one, the mask is read back.
+    uint32_t total = 0;
     if (p.idx != nullptr) {
+      const int per = (lwords + kSelThreads - 1) / kSelThreads;
+      const int w0 = min(lwords, tid * per), w1 = min(lwords, w0 + per);
+      uint32_t mine = 0;
+      for (int w = w0; w < w1; ++w) mine += __popc(__ldcg(p.mask + orow * p.mask_words + w));
+      uint32_t pos = block_excl_scan<kSelThreads>(mine, total, scan_sm);
       for (int w = w0; w < w1; ++w) {
         uint32_t m = __ldcg(p.mask + orow * p.mask_words + w);
         while (m) {
@@ -469,6 +489,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
           ++pos;
         }
       }
+    } else {
+      total = p.kcount[row] + (mode == 2 ? k1 : 0u);
     }
     if (tid == 0) {
       if (p.count != nullptr) p.count[orow] = (int32_t)total;
@@ -476,6 +498,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
       const int win_lo = max(L - p.window, sink_n);
       if (total != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
     }
+    __syncthreads();  // every thread has read the counters before they are cleared
     clear_row_state(p, row, b);
     return;
   }

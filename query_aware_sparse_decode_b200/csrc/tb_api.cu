@@ -37,7 +37,8 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, ccount, hist2, hist_end, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats, total;
+  size_t status, hist, ccount, kcount, hist2, hist_end, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats,
+      total;
   int max_splits;
 };
 
@@ -48,8 +49,9 @@ WsLayout layout_of(const tb_config& c) {
   size_t off = 0;
   w.status = off;  off += align256(256);
   w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
-  w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters and the
-  w.hist2 = off;   off += align256(B * kHistBins * 4);   // single-row second-digit histograms
+  w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters, kept-token
+  w.kcount = off;  off += align256(B * Hq * 4);          // counters and the single-row
+  w.hist2 = off;   off += align256(B * kHistBins * 4);   // second-digit histograms
   w.hist_end = off;                                      // (zeroed together)
   w.rowinfo = off; off += align256(B * Hq * 16);
   w.cand = off;    off += align256(B * Hq * (size_t)kSelCap * 8);
@@ -93,6 +95,7 @@ struct tb_ctx {
   uint32_t* status = nullptr;
   uint32_t* hist = nullptr;
   uint32_t* ccount = nullptr;
+  uint32_t* kcount = nullptr;
   uint32_t* hist2 = nullptr;
   uint32_t* cand = nullptr;
   uint4* rowinfo = nullptr;
@@ -242,6 +245,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   p.hist2 = rows == 1 ? ctx->hist2 : nullptr;
   p.cand = ctx->cand;
   p.ccount = ctx->ccount;
+  p.kcount = ctx->kcount;
   p.rowinfo = ctx->rowinfo;
   p.idx = idx;
   p.count = count;
@@ -436,6 +440,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->status = reinterpret_cast<uint32_t*>(ctx->ws + lay.status);
   ctx->hist = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist);
   ctx->ccount = reinterpret_cast<uint32_t*>(ctx->ws + lay.ccount);
+  ctx->kcount = reinterpret_cast<uint32_t*>(ctx->ws + lay.kcount);
   ctx->hist2 = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist2);
   ctx->cand = reinterpret_cast<uint32_t*>(ctx->ws + lay.cand);
   ctx->rowinfo = reinterpret_cast<uint4*>(ctx->ws + lay.rowinfo);
