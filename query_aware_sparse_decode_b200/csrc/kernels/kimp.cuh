@@ -19,18 +19,20 @@ struct AppendParams {
   int pos[kMaxBatch];  // row written for sequence b (its length before the append)
 };
 
-// grid (Hkv, B), block 128 threads: writes the K and V rows, then
+// One appended row of slab (b, g), computed by a CTA of at least 128 threads
+// (all of them call it: it contains barriers): writes the K and V rows, then
 // K_imp[j] = sum_d K[d] W_K[d][j] in fp32 with W_K staged in shared memory;
-// 128 / d' threads share each output column (partial sums over D / parts
-// dimensions, added in a fixed order).
+// the first 128 threads form 128 / d' partial sums per output column (over
+// D / parts dimensions each, ascending) that are added in a fixed order, so
+// the row is the same bits whichever kernel computes it.  `scratch` holds
+// D * d' + 256 floats.
+constexpr int kAppendScratchFloats = 128 * 32 + 256;
 template <typename T>
-__global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ float krow[128];
-  __shared__ float wsm[128 * 32];
-  __shared__ float part[128];
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+__device__ __forceinline__ void append_row(const AppendParams& p, int g, int b, float* scratch) {
+  float* wsm = scratch;             // [D][d']
+  float* krow = scratch + 128 * 32;  // [D]
+  float* part = krow + 128;          // [128]
+  const int tid = threadIdx.x, nt = blockDim.x;
   const size_t src = ((size_t)b * p.Hkv + g) * p.D;
   const size_t row = ((size_t)b * p.Hkv + g) * p.max_len + p.pos[b];
   const T* W = reinterpret_cast<const T*>(p.w_k);
@@ -38,14 +40,14 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   constexpr int VEC = 16 / (int)sizeof(T);  // W_K staged with 16-byte loads, all in flight
   if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && nw % VEC == 0) {
 #pragma unroll 8
-    for (int e = tid * VEC; e < nw; e += 128 * VEC) {
+    for (int e = tid * VEC; e < nw; e += nt * VEC) {
       const uint4 raw = *reinterpret_cast<const uint4*>(W + e);
       const T* el = reinterpret_cast<const T*>(&raw);
 #pragma unroll
       for (int i = 0; i < VEC; ++i) wsm[e + i] = to_f32(el[i]);
     }
   } else {
-    for (int e = tid; e < nw; e += 128) wsm[e] = to_f32(W[e]);
+    for (int e = tid; e < nw; e += nt) wsm[e] = to_f32(W[e]);
   }
   if (tid < p.D) {
     const T kv = reinterpret_cast<const T*>(p.k_new)[src + tid];
@@ -54,18 +56,30 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     krow[tid] = to_f32(kv);
   }
   __syncthreads();
-  const int parts = 128 / p.dimp;          // 4 (d'=32) or 8 (d'=16)
-  const int j = tid % p.dimp, q = tid / p.dimp;
-  const int span = p.D / parts;
-  float acc = 0.f;
-  for (int d = q * span; d < (q + 1) * span; ++d) acc = fmaf(krow[d], wsm[d * p.dimp + j], acc);
-  part[tid] = acc;
+  if (tid < 128) {
+    const int parts = 128 / p.dimp;  // 4 (d'=32) or 8 (d'=16)
+    const int j = tid % p.dimp, q = tid / p.dimp;
+    const int span = p.D / parts;
+    float acc = 0.f;
+    for (int d = q * span; d < (q + 1) * span; ++d) acc = fmaf(krow[d], wsm[d * p.dimp + j], acc);
+    part[tid] = acc;
+  }
   __syncthreads();
   if (tid < p.dimp) {
+    const int parts = 128 / p.dimp;
     float sum = 0.f;
     for (int i = 0; i < parts; ++i) sum += part[i * p.dimp + tid];
     p.kimp[kimp_index((size_t)b * p.Hkv + g, tid, p.pos[b], p.dimp, p.max_len)] = sum;
   }
+}
+
+// grid (Hkv, B), block 128 threads: one appended row per (b, g).
+template <typename T>
+__global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float scratch[kAppendScratchFloats];
+  append_row<T>(p, blockIdx.x, blockIdx.y, scratch);
 }
 
 struct ProjectParams {

@@ -168,7 +168,7 @@ static void prepare_hist(tb_ctx* ctx, cudaStream_t st) {
 }
 
 static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
-                              cudaStream_t st) {
+                              cudaStream_t st, const AppendParams* app = nullptr) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   ScoreParams p{};
@@ -188,7 +188,12 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
-  const size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
+  size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
+  if (hist && app) {  // the fused append uses the histogram space as scratch
+    p.fuse_append = 1;
+    p.app = *app;
+    smem = std::max(smem, (size_t)kAppendScratchFloats * 4);
+  }
   // the most tokens per CTA (up to 4 steps) that still gives about three
   // CTAs per SM; short or small batches get one step per CTA
   int iters = 4;
@@ -514,26 +519,37 @@ TB_API tb_status tb_set_budget(tb_ctx* ctx, int keep_pct, int sink, int window) 
   return TB_OK;
 }
 
+// Parameters of the append of one token per sequence at the current lengths.
+static tb_status append_params(const tb_ctx* ctx, int layer, const void* k_new, const void* v_new,
+                               AppendParams* p) {
+  if (!k_new || !v_new) return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  for (int b = 0; b < c.batch; ++b)
+    if (ls.lens[b] >= c.max_len) return TB_ERR_CAPACITY;
+  *p = AppendParams{};
+  p->k_new = k_new;
+  p->v_new = v_new;
+  p->k_cache = ls.k;
+  p->v_cache = ls.v;
+  p->kimp = ls.kimp;
+  p->w_k = ls.wk;
+  p->Hkv = c.n_kv_heads;
+  p->D = c.head_dim;
+  p->dimp = c.d_imp;
+  p->max_len = c.max_len;
+  for (int b = 0; b < c.batch; ++b) p->pos[b] = ls.lens[b];
+  return TB_OK;
+}
+
 TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, void* stream) {
   tb_status s = check_layer(ctx, layer);
   if (s != TB_OK) return s;
-  if (!k_new || !v_new) return TB_ERR_INVALID_ARG;
   const tb_config& c = ctx->cfg;
   LayerState& ls = ctx->layers[layer];
-  for (int b = 0; b < c.batch; ++b)
-    if (ls.lens[b] >= c.max_len) return TB_ERR_CAPACITY;
-  AppendParams p{};
-  p.k_new = k_new;
-  p.v_new = v_new;
-  p.k_cache = ls.k;
-  p.v_cache = ls.v;
-  p.kimp = ls.kimp;
-  p.w_k = ls.wk;
-  p.Hkv = c.n_kv_heads;
-  p.D = c.head_dim;
-  p.dimp = c.d_imp;
-  p.max_len = c.max_len;
-  for (int b = 0; b < c.batch; ++b) p.pos[b] = ls.lens[b];
+  AppendParams p;
+  s = append_params(ctx, layer, k_new, v_new, &p);
+  if (s != TB_OK) return s;
   dim3 grid(c.n_kv_heads, c.batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c.kv_dtype == TB_BF16)
@@ -643,6 +659,25 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   if (!aligned16(q)) return TB_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   trace_point(ctx, 0, st);
+  if (!dense && c.variant == TB_BUTLER) {
+    // the score kernel appends the token itself (no separate launch)
+    AppendParams app;
+    s = append_params(ctx, layer, k_new, v_new, &app);
+    if (s != TB_OK) return s;
+    LayerState& ls = ctx->layers[layer];
+    for (int b = 0; b < c.batch; ++b) ls.lens[b] += 1;
+    trace_point(ctx, 1, st);
+    s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st, &app);
+    if (s != TB_OK) {
+      for (int b = 0; b < c.batch; ++b) ls.lens[b] -= 1;
+      return s;
+    }
+    trace_point(ctx, 2, st);
+    s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+    if (s != TB_OK) return s;
+    trace_point(ctx, 3, st);
+    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
+  }
   s = tb_append_kv(ctx, layer, k_new, v_new, stream);
   if (s != TB_OK) return s;
   trace_point(ctx, 1, st);
@@ -651,23 +686,15 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
   }
-  if (c.variant == TB_SOFTVOTE) {
-    prepare_hist(ctx, st);
-    s = launch_softvote(ctx, layer, q, ctx->votes, ctx->hist, st);
-    if (s != TB_OK) return s;
-    trace_point(ctx, 2, st);
-    s = launch_select(ctx, layer, ctx->votes, true, 1, nullptr, 0, nullptr, ctx->mask, st);
-    if (s != TB_OK) return s;
-    trace_point(ctx, 3, st);
-    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
-  }
-  s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
+  // soft voting: votes over the full K (the appended row included), one shared set
+  prepare_hist(ctx, st);
+  s = launch_softvote(ctx, layer, q, ctx->votes, ctx->hist, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 2, st);
-  s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+  s = launch_select(ctx, layer, ctx->votes, true, 1, nullptr, 0, nullptr, ctx->mask, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 3, st);
-  return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
+  return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
 }
 
 TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_rows, int row0, int nrows,

@@ -66,6 +66,32 @@ def test_append_writes_rows_and_kimp(wl):
         assert np.all(np.abs(kimp[b, :, L] - ref) <= _kimp_tol(k64[b], ld.W))
 
 
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, RAGGED], ids=lambda w: w.name)
+def test_decode_step_append_matches_append_kernel(wl):
+    """The decode step appends inside its score kernel; the rows it writes
+    must be the very bits the standalone append writes."""
+    lens = [max(L - 1, 0) for L in wl.seq_lens]
+    outs = []
+    for fused in (False, True):
+        ctx = TB.Context(config_of(wl))
+        ld = make_layer(ctx, wl, 0, lens)
+        ctx.project_kimp(0, 0, max(lens))
+        k_raw, v_raw = S.kv_new(wl, 0, step=1)
+        k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
+        if fused:
+            out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+            ctx.decode_step(0, k_dev, v_dev, ld.q_dev, ld.q_imp_dev, out)
+        else:
+            ctx.append_kv(0, k_dev, v_dev)
+        torch.cuda.synchronize()
+        assert ctx.check_status() == 0
+        assert ctx.seq_lens(0) == [L + 1 for L in lens]
+        outs.append((ld.k_cache.clone(), ld.v_cache.clone(), ld.kimp.clone()))
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a.view(torch.int16),
+                           b.view(torch.int32) if b.dtype == torch.float32 else b.view(torch.int16))
+
+
 # --------------------------------------------------------------------------- a2 + a3
 @pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED,
                                 S.TINY_F32.with_(name="tiny_G4_layer6", n_layers=8, G=4)], ids=lambda w: w.name)
@@ -260,10 +286,16 @@ def _decode_e2e(wl, layer=0):
     torch.cuda.synchronize()
     assert ctx.check_status() == 0
     assert torch.equal(out, out2)
+    # the step's own append: K and V rows exact, K_imp row within fp32 rounding
+    k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
+    kc, vc = ld.k_cache.float().cpu().numpy(), ld.v_cache.float().cpu().numpy()
+    kimp_now = kimp_rows(ld.kimp)
+    for b, L in enumerate(lens):
+        assert np.array_equal(kc[b, :, L - 1], k64[b]) and np.array_equal(vc[b, :, L - 1], v64[b])
+        assert np.all(np.abs(kimp_now[b, :, L - 1] - O.project_keys(k64[b], ld.W)) <= _kimp_tol(k64[b], ld.W))
     # oracle on the full cache (prefill rows + the appended token)
     K = np.concatenate([ld.K, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
     V = np.concatenate([ld.V, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
-    k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
     for b, L in enumerate(lens):
         K[b, :, L - 1], V[b, :, L - 1] = k64[b], v64[b]
     sel, ref, _, sc = O.decode_layer(ld.q, K, V, ld.W, ld.qimp, layer, wl.G, lens, wl.keep_pct, wl.sink,
