@@ -135,9 +135,10 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------- DRAM traffic
 # DRAM bytes (read + write) per union K/V row of the sparse attention kernel,
-# from one ncu capture (profiles/attn_bf16_kernel_B2_L131072.md).  Valid only
-# for the kernel source it was measured on; any change makes it null.
-ATTN_TRAFFIC = {"source_sha256_16": "c918de5e67cf05b7", "bytes_per_union_row": 816.714752e6 / 1581259}
+# from one ncu capture of it (B = 2, L = 131072, keep 30 %; summary under
+# profiles/).  Valid only for the kernel source it was measured on; any
+# change makes it null.
+ATTN_TRAFFIC = {"source_sha256_16": "0e7d73ac5fd68159", "bytes_per_union_row": (811.692544e6 + 5.092096e6) / 1581259}
 
 
 def attn_traffic_per_row():

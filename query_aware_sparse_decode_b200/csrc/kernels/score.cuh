@@ -11,16 +11,12 @@
 // dimension order j = 0..d'-1, the group's query values broadcast from
 // shared memory) so that many loads per thread can be in flight.  A CTA covers 1, 2 or 4 groups of
 // 1024 tokens (the launch picks the count so the grid fills the SMs).
-// In the decode step the CTA that scores the new token first appends it (K,
-// V and K_imp rows; the same arithmetic as the append kernel), so the step
-// needs no separate append launch.
 // Optionally each CTA accumulates, per query-head row, the histogram of the
 // top 11 bits of the order key over the candidate range [sink, len - window)
 // (the first radix digit of the selection) and flushes it with global atomics.
 #pragma once
 
 #include "common.cuh"
-#include "kimp.cuh"
 
 namespace tb {
 
@@ -36,9 +32,7 @@ struct ScoreParams {
   int G, slot, Hq, Hkv, max_len;
   int sink, window;
   int iters;           // CTA iterations of kScoreStep tokens (1, 2 or 4)
-  int fuse_append;     // HIST launches only: the CTA holding token app.pos[b] first appends it
   int lens[kMaxBatch];
-  AppendParams app;
 };
 
 template <typename T, int DIMP, int GS, bool HIST>
@@ -55,15 +49,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   for (int e = tid; e < DIMP * GS; e += kScoreThreads) {
     const int j = e / GS, hh = e % GS;
     qs[j][hh] = to_f32(qi[(((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP + j]);
-  }
-  if (HIST && p.fuse_append) {
-    // decode step: the new token's K, V and K_imp rows are written by the CTA
-    // that scores it (hist doubles as scratch), before its own loads below
-    const int pos = p.app.pos[b];
-    if (pos >= t_base && pos < t_base + kScoreStep * p.iters) {
-      append_row<T>(p.app, g, b, reinterpret_cast<float*>(hist));
-      __syncthreads();
-    }
   }
   if (HIST)
     for (int e = tid; e < GS * kHistBins; e += kScoreThreads) hist[e] = 0;

@@ -168,7 +168,7 @@ static void prepare_hist(tb_ctx* ctx, cudaStream_t st) {
 }
 
 static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
-                              cudaStream_t st, const AppendParams* app = nullptr) {
+                              cudaStream_t st) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   ScoreParams p{};
@@ -188,12 +188,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
-  size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
-  if (hist && app) {  // the fused append uses the histogram space as scratch
-    p.fuse_append = 1;
-    p.app = *app;
-    smem = std::max(smem, (size_t)kAppendScratchFloats * 4);
-  }
+  const size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
   // the most tokens per CTA (up to 4 steps) that still gives about three
   // CTAs per SM; short or small batches get one step per CTA
   int iters = 4;
@@ -659,25 +654,6 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   if (!aligned16(q)) return TB_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   trace_point(ctx, 0, st);
-  if (!dense && c.variant == TB_BUTLER) {
-    // the score kernel appends the token itself (no separate launch)
-    AppendParams app;
-    s = append_params(ctx, layer, k_new, v_new, &app);
-    if (s != TB_OK) return s;
-    LayerState& ls = ctx->layers[layer];
-    for (int b = 0; b < c.batch; ++b) ls.lens[b] += 1;
-    trace_point(ctx, 1, st);
-    s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st, &app);
-    if (s != TB_OK) {
-      for (int b = 0; b < c.batch; ++b) ls.lens[b] -= 1;
-      return s;
-    }
-    trace_point(ctx, 2, st);
-    s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
-    if (s != TB_OK) return s;
-    trace_point(ctx, 3, st);
-    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
-  }
   s = tb_append_kv(ctx, layer, k_new, v_new, stream);
   if (s != TB_OK) return s;
   trace_point(ctx, 1, st);
@@ -685,6 +661,15 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     trace_point(ctx, 2, st);
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
+  }
+  if (c.variant == TB_BUTLER) {
+    s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
+    if (s != TB_OK) return s;
+    trace_point(ctx, 2, st);
+    s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+    if (s != TB_OK) return s;
+    trace_point(ctx, 3, st);
+    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
   }
   // soft voting: votes over the full K (the appended row included), one shared set
   prepare_hist(ctx, st);

@@ -68,8 +68,8 @@ def test_append_writes_rows_and_kimp(wl):
 
 @pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, RAGGED], ids=lambda w: w.name)
 def test_decode_step_append_matches_append_kernel(wl):
-    """The decode step appends inside its score kernel; the rows it writes
-    must be the very bits the standalone append writes."""
+    """The rows the decode step appends must be the very bits the standalone
+    append writes (both go through one device routine)."""
     lens = [max(L - 1, 0) for L in wl.seq_lens]
     outs = []
     for fused in (False, True):
