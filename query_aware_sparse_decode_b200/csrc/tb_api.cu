@@ -714,13 +714,21 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
   p.keep_pct = c.keep_pct;
   p.sink = c.sink;
   p.window = c.window;
-  dim3 grid(nrows, c.n_q_heads, c.batch);
+  // rows the blocked kernel hands over to the one-row method are flagged in
+  // the score workspace (B * Hq * nrows words <= B * Hq * max_len floats)
+  p.redo = reinterpret_cast<uint32_t*>(ctx->scores);
+  dim3 grid((nrows + kPfRows - 1) / kPfRows, c.n_q_heads, c.batch);
+  dim3 rgrid((unsigned)std::min<long long>(ctx->num_sms, (long long)c.n_q_heads * nrows), c.batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define TB_PF_CASE(T, DI)                                                               \
   if (c.d_imp == DI) {                                                                  \
-    auto k = prefill_select_kernel<T, DI>;                                              \
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
-    k<<<grid, kSelThreads, smem, st>>>(p);                                              \
+    auto kb = prefill_rows_kernel<T, DI>;                                               \
+    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem);     \
+    kb<<<grid, kPfThreads, kPfSmem, st>>>(p);                                           \
+    auto kr = prefill_redo_kernel<T, DI>;                                               \
+    cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
+    kr<<<rgrid, kSelThreads, smem, st>>>(p);                                            \
+    ctx->launches += 2;                                                                 \
   } else
   if (c.kv_dtype == TB_BF16) {
     TB_PF_CASE(__nv_bfloat16, 32) TB_PF_CASE(__nv_bfloat16, 16) return TB_ERR_UNSUPPORTED;
@@ -728,7 +736,6 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
     TB_PF_CASE(float, 32) TB_PF_CASE(float, 16) return TB_ERR_UNSUPPORTED;
   }
 #undef TB_PF_CASE
-  ++ctx->launches;
   return cuda_status(cudaGetLastError());
 }
 

@@ -99,3 +99,46 @@ def test_prefill_rows_llama8b_L32768_sampled():
     64 sampled rows checked against the oracle."""
     wl = S.PREFILL_L32K.with_(n_layers=2)
     _prefill_case(wl, layer=1, row0=32768 - 1024, nrows=1024, heads=[0, 9, 18, 31], rows=range(0, 1024, 16))
+
+
+def test_prefill_rows_with_massive_ties_take_the_one_row_path():
+    """Keys drawn from three distinct rows: each row's scores take three
+    values, so the threshold prefix holds thousands of equal keys and the
+    blocked kernel hands every row to the one-row method.  Ties go to the
+    lowest indices; the sets must equal the oracle's exactly."""
+    wl = PF_SMALL.with_(B=1, L=2048, n_layers=1, G=1, dense_layers=())
+    cfg = config_of(wl, max_len=round_up(wl.L, 256))
+    ctx = TB.Context(cfg)
+    B, Hkv, D, Lmax = wl.B, wl.Hkv, wl.D, cfg.max_len
+    base = S.fill_host(S.K_CACHE, 0, 0, Hkv, 0, 3, D, "bf16")          # three rows per KV head
+    K_raw = np.stack([base[g][np.arange(wl.L) % 3] for g in range(Hkv)])[None]   # [1][Hkv][L][D]
+    W_raw = S.w_k(wl, 0)
+    k = torch.zeros((B, Hkv, Lmax, D), dtype=torch.bfloat16, device="cuda")
+    k[:, :, :wl.L] = to_dev(K_raw, wl)
+    kimp = kimp_alloc(B, Hkv, wl.d_imp, Lmax)
+    ctx.bind_layer(0, k, torch.zeros_like(k), kimp, to_dev(W_raw, wl))
+    ctx.set_seq_lens(0, [wl.L])
+    ctx.project_kimp(0, 0, wl.L)
+    row0, nrows = wl.L - 40, 40
+    qrows_raw = S.q_imp(wl, 0, rows=(row0, nrows))
+    wpr = (row0 + nrows + 31) // 32
+    masks = torch.full((B, wl.Hq, nrows, wpr), -1, dtype=torch.int32, device="cuda")
+    ctx.select_prefill(0, to_dev(qrows_raw, wl), row0, nrows, masks)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    qrows = S.widen(qrows_raw, wl.dtype).reshape(B, wl.Hq, 1, nrows, wl.d_imp)
+    Kimp = O.project_keys(S.widen(K_raw, "bf16")[0], S.widen(W_raw, "bf16"))
+    ref = O.prefill_select(qrows[0, :, 0], Kimp, row0, wl.keep_pct, wl.sink, wl.window)
+    m = masks.cpu().numpy().view(np.uint32)
+    for h in range(wl.Hq):
+        for r in range(nrows):
+            p = row0 + r
+            bits = np.unpackbits(m[0, h, r].view(np.uint8), bitorder="little")
+            assert not bits[p + 1:].any()
+            assert np.array_equal(np.nonzero(bits[:p + 1])[0], ref[h, p])
+
+
+def test_prefill_rows_blocked_partial_block_and_mixed_budgets():
+    """nrows not a multiple of the 16-row block, rows whose prefixes are
+    shorter than sink + window next to rows with a real top-k."""
+    _prefill_case(PF_SMALL.with_(L=300, B=2), layer=6, row0=50, nrows=37)
