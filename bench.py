@@ -557,10 +557,12 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
     return line
 
 
-def _table_prefill(dev, iters, peak):
+def _table_prefill(dev, iters, peak, n_layers=None):
     import torch
     from query_aware_sparse_decode_b200 import synth as S
     wl = S.PREFILL_L32K
+    if n_layers is not None and n_layers < wl.n_layers:  # a smaller cache set, e.g. for a profiler
+        wl = wl.with_(n_layers=max(2, n_layers))
     max_len = wl.L + 256
     # build() fills and projects rows [0, L - 1) of its workload: one more
     # gives the whole 32768-row prefix of every layer
@@ -621,7 +623,7 @@ def kernel_table(args):
         if pick is None or pick.search(name):
             print(json.dumps(_table_case(wl, variant, dev, args.table_iters, flush_buf, peak)), flush=True)
     if pick is None or pick.search(S.PREFILL_L32K.name):
-        print(json.dumps(_table_prefill(dev, args.table_iters, peak)), flush=True)
+        print(json.dumps(_table_prefill(dev, args.table_iters, peak, args.layers)), flush=True)
 
 
 # ----------------------------------------------------------------------- main

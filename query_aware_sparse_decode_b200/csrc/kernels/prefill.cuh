@@ -228,6 +228,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   __syncthreads();
   const bool any2 = s_any2 != 0;
   const int Lmax = nr > 0 ? p.row0 + r0 + nr : 0;
+  // rows are consecutive positions: row r's candidate range ends at hi0 + r
+  const int hi0 = rhi[0];
+  uint32_t m2 = 0;  // rows that take a top-k
+#pragma unroll
+  for (int r = 0; r < kPfRows; ++r) m2 |= (uint32_t)(rmode[r] == 2) << r;
   const size_t slab = (size_t)b * p.Hkv + g;
   // scores of token t for the 16 rows, j ascending: the same fp32 sums as every
   // other score of the library
@@ -256,14 +261,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     __syncthreads();
     for (int base = 0; base < Lmax; base += kPfThreads) {
       const int t = base + tid;
-      if (t < Lmax) {
+      if (t < Lmax && t >= p.sink) {
         float kv[DIMP];
         kload(t, kv);
-#pragma unroll 1
+#pragma unroll 2
         for (int r = 0; r < kPfRows; ++r) {
-          if (rmode[r] != 2 || t < p.sink || t >= rhi[r]) continue;
-          const float sc = score_row(kv, r);
-          atomicAdd(&hist[r * kHistBins + (order_key(sc) >> 21)], 1u);
+          if (((m2 >> r) & 1u) && t < hi0 + r) {  // row r's candidates end at hi0 + r
+            const float sc = score_row(kv, r);
+            atomicAdd(&hist[r * kHistBins + (order_key(sc) >> 21)], 1u);
+          }
         }
       }
     }
@@ -288,23 +294,24 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     const int t = base + tid;
     float kv[DIMP];
     if (any2 && t < Lmax) kload(t, kv);
-#pragma unroll 1
-    for (int r = 0; r < nr; ++r) {
-      const int L = rL[r], mode = rmode[r];
+#pragma unroll 2
+    for (int r = 0; r < kPfRows; ++r) {
+      if (r >= nr) break;  // uniform
+      const int L = p.row0 + r0 + r + 1;
       const bool in = t < L;
-      const bool cr = t >= p.sink && t < rhi[r];
-      bool keep = in && (!cr || mode == 1);
-      if (mode == 2 && in && cr) {
+      const bool cr = t >= p.sink && t < hi0 + r;
+      bool keep = in && (!cr || rmode[r] == 1);
+      if (((m2 >> r) & 1u) && in && cr) {
         const uint32_t key = order_key(score_row(kv, r));
-        const uint32_t d1 = key >> 21;
-        if (d1 > rb1[r]) {
+        const uint32_t d1 = key >> 21, b1 = rb1[r];
+        if (d1 > b1) {
           keep = true;
-        } else if (d1 == rb1[r]) {
+        } else if (d1 == b1) {
           atomicAdd(&hist[r * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
         }
       }
       const uint32_t word = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0 && (t >> 5) < nwords) {
+      if (lane == 0 && (t >> 5) < nwords) {  // the last chunk may run past the row's words
         mbase[(size_t)r * nwords + (t >> 5)] = word;
         if (word) atomicAdd(&rkept[r], (uint32_t)__popc(word));
       }
@@ -330,15 +337,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // ---- pass 3: keys above the 22-bit prefix into the mask, keys equal to it
   // into the row's list
   if (any2) {
+    uint32_t m3 = 0;  // top-k rows this kernel finishes
+#pragma unroll
+    for (int r = 0; r < kPfRows; ++r) m3 |= (uint32_t)(rmode[r] == 2 && rn2[r] <= (uint32_t)kPfListCap) << r;
     for (int base = 0; base < Lmax; base += kPfThreads) {
       const int t = base + tid;
       float kv[DIMP];
       if (t < Lmax) kload(t, kv);
-#pragma unroll 1
-      for (int r = 0; r < nr; ++r) {
-        if (rmode[r] != 2 || rn2[r] > (uint32_t)kPfListCap) continue;  // uniform
+#pragma unroll 2
+      for (int r = 0; r < kPfRows; ++r) {
+        if (!((m3 >> r) & 1u)) continue;  // uniform
         bool up = false;
-        if (t < Lmax && t >= p.sink && t < rhi[r]) {
+        if (t < Lmax && t >= p.sink && t < hi0 + r) {
           const uint32_t key = order_key(score_row(kv, r));
           if ((key >> 21) == rb1[r]) {
             const uint32_t d2 = (key >> 10) & (kHistBins - 1);
