@@ -176,14 +176,44 @@ __global__ void __launch_bounds__(kSelThreads, 1) prefill_redo_kernel(const Pref
   }
 }
 
-// The blocked method; see the file comment.  grid (ceil(nrows / 16), Hq, B).
+// ---------------------------------------------------------------- blocked
+// TF32 helpers for the score tiles.  A bf16 importance query is exact in TF32.
+// A K_imp value v is carried as hi + lo: hi is v cut to TF32 width and lo the
+// exact remainder v - hi, of which the tensor core reads a TF32-width head.
+// Together they keep at least 21 of v's 24 significand bits, so a tile score
+// differs from the fp32 dot product by about 1e-6 relative: far inside the
+// selection's tie band.  Every pass recomputes the same tiles the same way.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = to_tf32(x);
+  lo = to_tf32(x - __uint_as_float(hi));
+}
+// D += A (16x8, row) * B (8x8, col), TF32 in, fp32 accumulate
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The blocked method; see the file comment.  grid (ceil(nrows / 16), Hq, B),
+// 1024 threads.  The 16 rows are the M dimension of mma.sync m16n8k8 TF32
+// tiles: a warp takes 32 tokens at a time (four n-tiles of 8; one mask word
+// per row), and lane (g, c) = (lane / 4, lane % 4) holds the scores of rows g
+// and g + 8 for tokens 2c and 2c + 1 of each n-tile.
 template <typename TQ, int DIMP>
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const PrefillParams p) {
+  constexpr int KS = DIMP / 8;                        // k-steps of 8 dimensions
+  constexpr bool QSPLIT = sizeof(TQ) == 4;            // fp32 queries need hi + lo too
   extern __shared__ __align__(16) uint32_t pf_smem[];  // hist[16][2048]; in pass 3 the key lists
-  __shared__ __align__(16) float q[kPfRows][DIMP];
-  __shared__ int rL[kPfRows], rhi[kPfRows], rk[kPfRows], rmode[kPfRows];
+  __shared__ int rmode[kPfRows], rk[kPfRows];
   __shared__ uint32_t rb1[kPfRows], rk1[kPfRows], rb2[kPfRows], rk2[kPfRows], rn2[kPfRows], rcnt[kPfRows];
-  __shared__ uint32_t rkept[kPfRows], rabove[kPfRows], rsel[kPfRows];
+  __shared__ uint32_t rkept[kPfRows], rabove[kPfRows];
   __shared__ uint32_t scan_sm[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
@@ -191,6 +221,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   uint32_t* hist = pf_smem;
   uint2* lists = reinterpret_cast<uint2*>(pf_smem);  // [16][kPfListCap], pass 3 only
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, cq = lane & 3;
   const int gs = p.Hq / p.Hkv, g = h / gs;
   const int r0 = blockIdx.x * kPfRows;
   const int nr = min(kPfRows, p.nrows - r0);
@@ -200,76 +231,100 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
   __syncthreads();
   if (tid < kPfRows) {
-    int L = 0, hi = 0, k = 0, mode = 0;
+    int k = 0, mode = 0;
     if (tid < nr) {
-      L = p.row0 + r0 + tid + 1;
-      hi = L - p.window;
+      const int L = p.row0 + r0 + tid + 1;
+      const int hi = L - p.window;
       const int nc = hi > p.sink ? hi - p.sink : 0;
       k = (int)min((long long)p.keep_pct * L / 100, (long long)nc);
       mode = (k > 0 && k < nc) ? 2 : (k == nc && k > 0 ? 1 : 0);
     }
-    rL[tid] = L;
-    rhi[tid] = hi;
     rk[tid] = k;
     rmode[tid] = mode;
     rkept[tid] = 0;
     rabove[tid] = 0;
-    rsel[tid] = 0;
     rcnt[tid] = 0;
     rn2[tid] = 0;
+    rb1[tid] = 0;
+    rb2[tid] = 0;
     if (mode == 2) atomicOr(&s_any2, 1);
-  }
-  for (int e = tid; e < kPfRows * DIMP; e += kPfThreads) {
-    const int r = e / DIMP, j = e % DIMP;
-    q[r][j] = r < nr ? to_f32(reinterpret_cast<const TQ*>(p.q_imp)[((((size_t)b * p.Hq + h) * p.G + p.slot) * p.nrows +
-                                                                      r0 + r) * DIMP + j])
-                     : 0.f;
   }
   __syncthreads();
   const bool any2 = s_any2 != 0;
   const int Lmax = nr > 0 ? p.row0 + r0 + nr : 0;
-  // rows are consecutive positions: row r's candidate range ends at hi0 + r
-  const int hi0 = rhi[0];
-  uint32_t m2 = 0;  // rows that take a top-k
-#pragma unroll
-  for (int r = 0; r < kPfRows; ++r) m2 |= (uint32_t)(rmode[r] == 2) << r;
+  const int L0 = p.row0 + r0 + 1;        // row r covers tokens [0, L0 + r)
+  const int hi0 = L0 - p.window;         // row r's candidates are [sink, hi0 + r)
   const size_t slab = (size_t)b * p.Hkv + g;
-  // scores of token t for the 16 rows, j ascending: the same fp32 sums as every
-  // other score of the library
-  auto kload = [&](int t, float (&kv)[DIMP]) {
-    const float* K = p.kimp + kimp_index(slab, 0, t, DIMP, p.max_len);
+  // A fragments (the 16 rows' importance queries), constant for the kernel
+  uint32_t afr[KS][4], afl[KS][4];
+  {
+    const TQ* qi = reinterpret_cast<const TQ*>(p.q_imp);
+    auto qv = [&](int r, int j) -> float {
+      return r < nr ? to_f32(qi[((((size_t)b * p.Hq + h) * p.G + p.slot) * p.nrows + r0 + r) * DIMP + j]) : 0.f;
+    };
 #pragma unroll
-    for (int j = 0; j < DIMP; ++j) kv[j] = K[j * kKimpTile];
-  };
-  auto score_row = [&](const float (&kv)[DIMP], int r) {
-    float acc = 0.f;
+    for (int ks = 0; ks < KS; ++ks) {
+      const float v[4] = {qv(gq, ks * 8 + cq), qv(gq + 8, ks * 8 + cq), qv(gq, ks * 8 + cq + 4),
+                          qv(gq + 8, ks * 8 + cq + 4)};
 #pragma unroll
-    for (int j = 0; j < DIMP; j += 4) {
-      const float4 qq = *reinterpret_cast<const float4*>(&q[r][j]);
-      acc = fmaf(qq.x, kv[j], acc);
-      acc = fmaf(qq.y, kv[j + 1], acc);
-      acc = fmaf(qq.z, kv[j + 2], acc);
-      acc = fmaf(qq.w, kv[j + 3], acc);
+      for (int e = 0; e < 4; ++e) {
+        if (QSPLIT) {
+          split_tf32(v[e], afr[ks][e], afl[ks][e]);
+        } else {
+          afr[ks][e] = __float_as_uint(v[e]);  // exact
+          afl[ks][e] = 0u;
+        }
+      }
     }
-    return acc;
+  }
+  // scores of the 16 rows for the 32 tokens [t0, t0 + 32): sc[n][i], n-tile n,
+  // i = (row gq, token 2cq), (gq, 2cq+1), (gq+8, 2cq), (gq+8, 2cq+1)
+  auto tile_scores = [&](int t0, float (&sc)[4][4]) {
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+      const int t = t0 + 8 * n + gq;  // the B column this lane loads
+      const bool ok = t < Lmax;
+      const float* K = p.kimp + kimp_index(slab, 0, ok ? t : 0, DIMP, p.max_len);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const float k0 = ok ? K[(ks * 8 + cq) * kKimpTile] : 0.f;
+        const float k1 = ok ? K[(ks * 8 + cq + 4) * kKimpTile] : 0.f;
+        // hi: the value cut to TF32 width; lo: the exact fp32 remainder, of
+        // which the tensor core reads the TF32-width head
+        const uint32_t h0 = __float_as_uint(k0) & 0xFFFFE000u, h1 = __float_as_uint(k1) & 0xFFFFE000u;
+        const uint32_t l0 = __float_as_uint(k0 - __uint_as_float(h0)), l1 = __float_as_uint(k1 - __uint_as_float(h1));
+        mma_tf32_1688(sc[n], afr[ks], h0, h1);
+        mma_tf32_1688(sc[n], afr[ks], l0, l1);
+        if (QSPLIT) mma_tf32_1688(sc[n], afl[ks], h0, h1);
+      }
+    }
   };
+
   uint32_t* mbase = p.masks + (((size_t)b * p.Hq + h) * p.nrows + r0) * p.words_per_row;
+  const int nwords = p.words_per_row;
+  const int nsteps = (Lmax + 31) / 32;
+  const int ra = gq, rb = gq + 8;  // this lane's rows
+  // value i of n-tile n: row (i < 2 ? ra : rb), token t0 + 8 n + 2 cq + (i & 1)
 
   // ---- pass 1: first-digit histograms
   if (any2) {
     for (int e = tid; e < kPfRows * kHistBins; e += kPfThreads) hist[e] = 0u;
     __syncthreads();
-    for (int base = 0; base < Lmax; base += kPfThreads) {
-      const int t = base + tid;
-      if (t < Lmax && t >= p.sink) {
-        float kv[DIMP];
-        kload(t, kv);
-#pragma unroll 2
-        for (int r = 0; r < kPfRows; ++r) {
-          if (((m2 >> r) & 1u) && t < hi0 + r) {  // row r's candidates end at hi0 + r
-            const float sc = score_row(kv, r);
-            atomicAdd(&hist[r * kHistBins + (order_key(sc) >> 21)], 1u);
-          }
+    const bool m2a = rmode[ra] == 2, m2b = rmode[rb] == 2;
+    for (int ws = warp; ws < nsteps; ws += kPfThreads / 32) {
+      const int t0 = ws * 32;
+      float sc[4][4];
+      tile_scores(t0, sc);
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = i < 2 ? ra : rb;
+          const bool m2 = i < 2 ? m2a : m2b;
+          const int t = t0 + 8 * n + 2 * cq + (i & 1);
+          if (m2 && t >= p.sink && t < hi0 + row)
+            atomicAdd(&hist[row * kHistBins + (order_key(sc[n][i]) >> 21)], 1u);
         }
       }
     }
@@ -287,33 +342,54 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     __syncthreads();
   }
 
-  // ---- pass 2: mask words (sink, window, keys above the threshold bin) and
-  // second-digit histograms of the threshold bins; every word of every row
-  const int nwords = p.words_per_row;
-  for (int base = 0; base < nwords * 32; base += kPfThreads) {
-    const int t = base + tid;
-    float kv[DIMP];
-    if (any2 && t < Lmax) kload(t, kv);
-#pragma unroll 2
-    for (int r = 0; r < kPfRows; ++r) {
-      if (r >= nr) break;  // uniform
-      const int L = p.row0 + r0 + r + 1;
-      const bool in = t < L;
-      const bool cr = t >= p.sink && t < hi0 + r;
-      bool keep = in && (!cr || rmode[r] == 1);
-      if (((m2 >> r) & 1u) && in && cr) {
-        const uint32_t key = order_key(score_row(kv, r));
-        const uint32_t d1 = key >> 21, b1 = rb1[r];
-        if (d1 > b1) {
-          keep = true;
-        } else if (d1 == b1) {
-          atomicAdd(&hist[r * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
+  // ---- pass 2: every mask word of every row (sink, window, keys above the
+  // threshold bin), second-digit histograms of the threshold bins
+  {
+    const int mda = rmode[ra], mdb = rmode[rb];
+    const uint32_t b1a = rb1[ra], b1b = rb1[rb];
+    for (int ws = warp; ws < nwords; ws += kPfThreads / 32) {
+      const int t0 = ws * 32;
+      float sc[4][4] = {};
+      if (any2 && t0 < Lmax) tile_scores(t0, sc);  // warp-uniform
+      uint32_t wa = 0, wb = 0;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = i < 2 ? ra : rb, md = i < 2 ? mda : mdb;
+          const int pos = 8 * n + 2 * cq + (i & 1);
+          const int t = t0 + pos;
+          const bool in = t < L0 + row;
+          const bool cr = t >= p.sink && t < hi0 + row;
+          bool keep = in && (!cr || md == 1);
+          if (md == 2 && in && cr) {
+            const uint32_t key = order_key(sc[n][i]);
+            const uint32_t d1 = key >> 21, b1 = i < 2 ? b1a : b1b;
+            if (d1 > b1) {
+              keep = true;
+            } else if (d1 == b1) {
+              atomicAdd(&hist[row * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
+            }
+          }
+          if (keep) {
+            if (i < 2) wa |= 1u << pos;
+            else wb |= 1u << pos;
+          }
         }
       }
-      const uint32_t word = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0 && (t >> 5) < nwords) {  // the last chunk may run past the row's words
-        mbase[(size_t)r * nwords + (t >> 5)] = word;
-        if (word) atomicAdd(&rkept[r], (uint32_t)__popc(word));
+      wa |= __shfl_xor_sync(0xffffffffu, wa, 1);
+      wa |= __shfl_xor_sync(0xffffffffu, wa, 2);
+      wb |= __shfl_xor_sync(0xffffffffu, wb, 1);
+      wb |= __shfl_xor_sync(0xffffffffu, wb, 2);
+      if (cq == 0) {
+        if (ra < nr) {
+          mbase[(size_t)ra * nwords + ws] = wa;
+          if (wa) atomicAdd(&rkept[ra], (uint32_t)__popc(wa));
+        }
+        if (rb < nr) {
+          mbase[(size_t)rb * nwords + ws] = wb;
+          if (wb) atomicAdd(&rkept[rb], (uint32_t)__popc(wb));
+        }
       }
     }
   }
@@ -337,31 +413,42 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // ---- pass 3: keys above the 22-bit prefix into the mask, keys equal to it
   // into the row's list
   if (any2) {
-    uint32_t m3 = 0;  // top-k rows this kernel finishes
+    const bool m3a = rmode[ra] == 2 && rn2[ra] <= (uint32_t)kPfListCap;
+    const bool m3b = rmode[rb] == 2 && rn2[rb] <= (uint32_t)kPfListCap;
+    const uint32_t b1a = rb1[ra], b1b = rb1[rb], b2a = rb2[ra], b2b = rb2[rb];
+    for (int ws = warp; ws < nsteps; ws += kPfThreads / 32) {
+      const int t0 = ws * 32;
+      float sc[4][4];
+      tile_scores(t0, sc);
+      uint32_t ua = 0, ub = 0;
 #pragma unroll
-    for (int r = 0; r < kPfRows; ++r) m3 |= (uint32_t)(rmode[r] == 2 && rn2[r] <= (uint32_t)kPfListCap) << r;
-    for (int base = 0; base < Lmax; base += kPfThreads) {
-      const int t = base + tid;
-      float kv[DIMP];
-      if (t < Lmax) kload(t, kv);
-#pragma unroll 2
-      for (int r = 0; r < kPfRows; ++r) {
-        if (!((m3 >> r) & 1u)) continue;  // uniform
-        bool up = false;
-        if (t < Lmax && t >= p.sink && t < hi0 + r) {
-          const uint32_t key = order_key(score_row(kv, r));
-          if ((key >> 21) == rb1[r]) {
-            const uint32_t d2 = (key >> 10) & (kHistBins - 1);
-            if (d2 > rb2[r]) {
-              up = true;
-            } else if (d2 == rb2[r]) {
-              const uint32_t pos = atomicAdd(&rcnt[r], 1u);
-              if (pos < (uint32_t)kPfListCap) lists[r * kPfListCap + pos] = make_uint2(key, (uint32_t)t);
-            }
+      for (int n = 0; n < 4; ++n) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = i < 2 ? ra : rb;
+          const bool m3 = i < 2 ? m3a : m3b;
+          const int pos = 8 * n + 2 * cq + (i & 1);
+          const int t = t0 + pos;
+          if (!m3 || t < p.sink || t >= hi0 + row) continue;
+          const uint32_t key = order_key(sc[n][i]);
+          if ((key >> 21) != (i < 2 ? b1a : b1b)) continue;
+          const uint32_t d2 = (key >> 10) & (kHistBins - 1), b2 = i < 2 ? b2a : b2b;
+          if (d2 > b2) {
+            if (i < 2) ua |= 1u << pos;
+            else ub |= 1u << pos;
+          } else if (d2 == b2) {
+            const uint32_t slot = atomicAdd(&rcnt[row], 1u);
+            if (slot < (uint32_t)kPfListCap) lists[row * kPfListCap + slot] = make_uint2(key, (uint32_t)t);
           }
         }
-        const uint32_t word = __ballot_sync(0xffffffffu, up);
-        if (lane == 0 && word) atomicOr(&mbase[(size_t)r * nwords + (t >> 5)], word);
+      }
+      ua |= __shfl_xor_sync(0xffffffffu, ua, 1);
+      ua |= __shfl_xor_sync(0xffffffffu, ua, 2);
+      ub |= __shfl_xor_sync(0xffffffffu, ub, 1);
+      ub |= __shfl_xor_sync(0xffffffffu, ub, 2);
+      if (cq == 0) {
+        if (ua) atomicOr(&mbase[(size_t)ra * nwords + ws], ua);
+        if (ub) atomicOr(&mbase[(size_t)rb * nwords + ws], ub);
       }
     }
     __syncthreads();
@@ -386,10 +473,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
 #pragma unroll
       for (int o = 16; o; o >>= 1) nsel += __shfl_xor_sync(0xffffffffu, nsel, o);
       if (lane == 0) {
-        rsel[r] = nsel;
-        // counts: n must equal the histogram's, and kept + above + selected
+        // n must equal the histogram's count, and kept + above + selected
         // must be sink + window + k
-        const int L = rL[r];
+        const int L = L0 + r;
         const int sink_n = min(p.sink, L);
         const int win_lo = max(L - p.window, sink_n);
         if (n != rn2[r] || rkept[r] + rabove[r] + nsel != (uint32_t)(sink_n + (L - win_lo) + rk[r]))
@@ -399,7 +485,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
   // rows of mode 0 / 1: the words of pass 2 are the whole set
   if (tid < nr && rmode[tid] != 2) {
-    const int L = rL[tid];
+    const int L = L0 + tid;
     const int sink_n = min(p.sink, L);
     const int win_lo = max(L - p.window, sink_n);
     if (rkept[tid] != (uint32_t)(sink_n + (L - win_lo) + rk[tid])) atomicOr(p.status, TB_DEV_ERR_COUNT);
