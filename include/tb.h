@@ -86,8 +86,15 @@ typedef enum {
 } tb_status;
 
 typedef enum { TB_BF16 = 0, TB_F32 = 1 } tb_dtype;
-typedef enum { TB_BUTLER = 0, TB_SOFTVOTE = 1 } tb_variant;
-typedef enum { TB_MASK_PER_HEAD = 0, TB_MASK_SHARED = 1, TB_MASK_DENSE = 2 } tb_mask_mode;
+/* TB_BUTLER: one selection per query head (model card "Method").
+ * TB_SOFTVOTE: one selection per sequence from soft votes (TokenSelect README).
+ * TB_BUTLER_GROUP: one selection per KV group: the importance scores of the
+ *   group's Hq/Hkv query heads are summed (fp32, in head order) and the group
+ *   selects once.  This is a GQA-aware option, not a reading of the pages:
+ *   the pages select per head.  Every K/V row the group reads is then used by
+ *   all of its heads, so the attention reads far fewer rows. */
+typedef enum { TB_BUTLER = 0, TB_SOFTVOTE = 1, TB_BUTLER_GROUP = 2 } tb_variant;
+typedef enum { TB_MASK_PER_HEAD = 0, TB_MASK_SHARED = 1, TB_MASK_DENSE = 2, TB_MASK_GROUP = 3 } tb_mask_mode;
 
 /* device status word bits (tb_check_status) */
 #define TB_DEV_ERR_INDEX 0x1u     /* a gathered index was outside [0, len)    */
@@ -154,13 +161,16 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
 /* a2 + a3 — model card "Method": scores[b][h][t] = q_hat[b][h] . K_imp[b][g(h)][t]
  * for t < len[b], with q_hat[b][h] = q_imp_producer[b*Hq + h][(layer-1) mod G][0][:]
  * (fp32 FMA, no scale).  `q_imp_producer`: [(B*Hq)][G][1][d'] of producer
- * G*floor(layer/G).  Entries t >= len[b] are left untouched. */
+ * G*floor(layer/G).  Entries t >= len[b] are left untouched.  With
+ * TB_BUTLER_GROUP the rows are per KV group instead ([B][Hkv][max_len]):
+ * scores[b][g][t] = sum over the group's heads, in head order, of the fp32
+ * per-head scores. */
 TB_API tb_status tb_score(tb_ctx* ctx, int layer, const void* q_imp_producer, float* scores, void* stream);
 
-/* a4 + a5 — model card "Method" / "Memory requirements": per (b, h) row of
- * `scores` ([B][Hq][max_len], or [B][max_len] when `rows_per_seq` is 1 for a
- * shared ranking), selects Sel as in the header comment, with the budget of
- * the context.  Outputs (each may be NULL, not all):
+/* a4 + a5 — model card "Method" / "Memory requirements": per row of `scores`
+ * ([B][rows_per_seq][max_len]; rows_per_seq is Hq for per-head sets, Hkv for
+ * per-group sets, 1 for a shared ranking), selects Sel as in the header
+ * comment, with the budget of the context.  Outputs (each may be NULL, not all):
  *   idx   [B][rows][idx_cap] ascending indices (TB_ERR_SHAPE if idx_cap is
  *         smaller than the largest selected set),
  *   count [B][rows] selected-set sizes,
@@ -172,6 +182,7 @@ TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows
 /* a6 — exact attention over a selected set of the untouched cache:
  * out[b][h] = sum_{t in Sel} softmax_t(q[b][h] . K[b][g(h)][t] / sqrt(D)) V[b][g(h)][t]
  * (fp32 accumulation).  `mask_mode`: TB_MASK_PER_HEAD (mask [B][Hq][max_len/32]),
+ * TB_MASK_GROUP (mask [B][Hkv][max_len/32], one set per KV group),
  * TB_MASK_SHARED (mask [B][max_len/32], one set per sequence) or
  * TB_MASK_DENSE (mask NULL: every token t < len, the layer-0 / 100 % path).
  * `lse` (optional, [B][Hq] fp32): natural log of the softmax denominator;
@@ -181,9 +192,10 @@ TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uin
                                 void* out, float* lse, void* stream);
 
 /* a1..a6 for one layer: append, then (dense layer or 100 % budget) dense
- * attention, else score, select and sparse attention (TB_BUTLER) or soft
- * voting with a shared set (TB_SOFTVOTE; q_imp_producer unused).  Uses the
- * workspace for scores, masks and split partials. */
+ * attention, else score, select and sparse attention (TB_BUTLER per head,
+ * TB_BUTLER_GROUP per KV group) or soft voting with a shared set
+ * (TB_SOFTVOTE; q_imp_producer unused).  Uses the workspace for scores,
+ * masks and split partials. */
 TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, const void* q,
                                 const void* q_imp_producer, void* out, void* stream);
 
@@ -193,7 +205,11 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
  * L -> p + 1.  `q_imp_rows`: [(B*Hq)][G][nrows][d'] (positions row0..), slot
  * (layer-1) mod G.  `row_masks`: [B][Hq][nrows][words_per_row] uint32 with
  * words_per_row >= ceil((row0 + nrows)/32); every word is written.
- * Requires len[b] >= row0 + nrows (K_imp rows present). */
+ * Requires len[b] >= row0 + nrows (K_imp rows present).  Rows are scored in
+ * blocks of 16 on the tensor cores (TF32 with K_imp split into a TF32 head
+ * and its remainder, fp32 accumulation: about 1e-6 relative to the fp32 dot
+ * product); rows with massive ties are redone with fp32 FMA scores.  Always
+ * one selection per query head. */
 TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_rows, int row0, int nrows,
                                    uint32_t* row_masks, int words_per_row, void* stream);
 

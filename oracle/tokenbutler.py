@@ -35,6 +35,12 @@ Readings where the sources leave a step open (each marked "Reading" below):
       summed over all query heads, one set shared by all heads.
   An empty selected set gives a zero output and lse = -inf.
 
+Option beyond the sources (not a reading of them): per-KV-group selection,
+where the importance scores of a group's query heads are summed and the
+group selects once with the same budget, sink, window and tie rules; every
+head of the group then attends over that set (group_scores, decode_layer
+with group=True).
+
 Parity pins (tests/test_oracle_pins.py) cover every function here; the
 readings R4, R6, R13 and R14 are consistent with the sources but not fixed
 by them (parity unpinned against the pages for those readings).
@@ -141,9 +147,21 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, scale: 
     return (w @ Vs) / z, m + math.log(z)
 
 
+# ------------------------------------------------------------------ group option
+def group_scores(q_hat_heads: np.ndarray, K_imp: np.ndarray) -> np.ndarray:
+    """Per-KV-group option: the group's per-head importance scores summed,
+    s_g[t] = sum_h q_hat_h . K_imp[t] (fp64).  q_hat_heads: [GS][d']; K_imp:
+    [L][d']."""
+    q = np.asarray(q_hat_heads, dtype=np.float64)
+    total = np.zeros(np.asarray(K_imp).shape[0], np.float64)
+    for h in range(q.shape[0]):
+        total += importance_scores(q[h], K_imp)
+    return total
+
+
 # ------------------------------------------------------------------ one decode layer
 def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, dense: bool,
-                 K_imp=None, heads=None, batches=None):
+                 K_imp=None, heads=None, batches=None, group: bool = False):
     """One consumer layer's decode step, [MC] Method in order:
     K_imp = K W_K; consumer slot (l - 1) mod G; score every cached token;
     top-k + sink + window per query head; attention over the selected tokens.
@@ -152,7 +170,8 @@ def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, wind
     q: [B][Hq][D]; K, V: [B][Hkv][>=L][D]; W_K: [D][d'];
     q_imp_producer: [(B*Hq)][G][1][d']; L: int or per-sequence list.
     Returns dicts keyed by (b, h): selected indices, output [D], lse; and the
-    fp64 scores per (b, h) (None for dense layers)."""
+    fp64 scores per (b, h) (None for dense layers).  With group=True (the
+    per-KV-group option) the scores and the set are the head's group's."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
     Hkv = K.shape[1]
@@ -174,7 +193,11 @@ def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, wind
                 if g not in kimp_b:
                     kimp_b[g] = (project_keys(K[b, g, :Lb], W_K) if K_imp is None
                                  else np.asarray(K_imp[b, g, :Lb], dtype=np.float64))
-                s = importance_scores(q_hat[b, h], kimp_b[g])
+                if group:
+                    gs = Hq // Hkv
+                    s = group_scores(q_hat[b, g * gs:(g + 1) * gs], kimp_b[g])
+                else:
+                    s = importance_scores(q_hat[b, h], kimp_b[g])
                 scores[b, h] = s
                 idx = select_tokens(s, Lb, keep_pct, sink, window)
             sel[b, h] = idx

@@ -64,6 +64,8 @@ __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int 
         }
       } else if (p.mask_mode == TB_MASK_SHARED) {
         u = p.mask[(size_t)b * p.mask_words + w_base + w];
+      } else if (p.mask_mode == TB_MASK_GROUP) {
+        u = p.mask[((size_t)b * p.Hkv + g) * p.mask_words + w_base + w];
       } else {
         u = 0xFFFFFFFFu;
       }

@@ -11,7 +11,9 @@
 // dimension order j = 0..d'-1, the group's query values broadcast from
 // shared memory) so that many loads per thread can be in flight.  A CTA covers 1, 2 or 4 groups of
 // 1024 tokens (the launch picks the count so the grid fills the SMs).
-// Optionally each CTA accumulates, per query-head row, the histogram of the
+// With GROUPED (one selection per KV group) the group's per-head fp32 scores
+// are added in head order and one row per (b, g) is written instead.
+// Optionally each CTA accumulates, per output row, the histogram of the
 // top 11 bits of the order key over the candidate range [sink, len - window)
 // (the first radix digit of the selection) and flushes it with global atomics.
 #pragma once
@@ -35,12 +37,13 @@ struct ScoreParams {
   int lens[kMaxBatch];
 };
 
-template <typename T, int DIMP, int GS, bool HIST>
+template <typename T, int DIMP, int GS, bool HIST, bool GROUPED = false>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScoreParams p) {
+  constexpr int NR = GROUPED ? 1 : GS;  // output rows per (b, g): per head, or the group's sum
   pdl_wait();
   pdl_trigger();
   __shared__ __align__(16) float qs[DIMP][GS];
-  extern __shared__ uint32_t hist[];  // [GS][2048] when HIST
+  extern __shared__ uint32_t hist[];  // [NR][2048] when HIST
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.lens[b];
   const int t_base = chunk * kScoreStep * p.iters;
@@ -51,11 +54,12 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
     qs[j][hh] = to_f32(qi[(((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP + j]);
   }
   if (HIST)
-    for (int e = tid; e < GS * kHistBins; e += kScoreThreads) hist[e] = 0;
+    for (int e = tid; e < NR * kHistBins; e += kScoreThreads) hist[e] = 0;
   __syncthreads();
 
   const size_t slab = (size_t)b * p.Hkv + g;
-  float* S = p.scores + ((size_t)b * p.Hq + g * GS) * p.max_len;
+  const size_t row0 = GROUPED ? (size_t)b * p.Hkv + g : (size_t)b * p.Hq + g * GS;  // first output row
+  float* S = p.scores + row0 * p.max_len;
   static_assert(DIMP % kScoreLoadBatch == 0 || DIMP < kScoreLoadBatch, "d' must be a multiple of the batch");
   constexpr int NB = DIMP < kScoreLoadBatch ? DIMP : kScoreLoadBatch;
 #pragma unroll 1
@@ -83,8 +87,17 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
           }
         }
       }
+      if (GROUPED) {  // the group's row: per-head fp32 scores added in head order
 #pragma unroll
-      for (int hh = 0; hh < GS; ++hh) {
+        for (int u = 0; u < 4; ++u) {
+          float sum = acc[0][u];
+#pragma unroll
+          for (int hh = 1; hh < GS; ++hh) sum += acc[hh][u];
+          acc[0][u] = sum;
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < NR; ++hh) {
         float* srow = S + (size_t)hh * p.max_len;
         if (t0 + 3 < L) {
           *reinterpret_cast<float4*>(srow + t0) = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
@@ -105,9 +118,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   }
   if (HIST) {
     __syncthreads();
-    for (int e = tid; e < GS * kHistBins; e += kScoreThreads) {
+    for (int e = tid; e < NR * kHistBins; e += kScoreThreads) {
       const uint32_t c = hist[e];
-      if (c) atomicAdd(&p.hist[((size_t)b * p.Hq + g * GS + e / kHistBins) * kHistBins + e % kHistBins], c);
+      if (c) atomicAdd(&p.hist[(row0 + e / kHistBins) * kHistBins + e % kHistBins], c);
     }
   }
 }

@@ -132,7 +132,8 @@ static tb_status check_config(const tb_config* c) {
   if ((long long)c->batch * c->n_q_heads * c->max_len >= (1LL << 40)) return TB_ERR_SHAPE;
   if (c->kv_dtype != TB_BF16 && c->kv_dtype != TB_F32) return TB_ERR_INVALID_ARG;
   if (c->keep_pct < 0 || c->keep_pct > 100 || c->sink < 0 || c->window < 0) return TB_ERR_INVALID_ARG;
-  if (c->variant != TB_BUTLER && c->variant != TB_SOFTVOTE) return TB_ERR_INVALID_ARG;
+  if (c->variant != TB_BUTLER && c->variant != TB_SOFTVOTE && c->variant != TB_BUTLER_GROUP)
+    return TB_ERR_INVALID_ARG;
   return TB_OK;
 }
 
@@ -188,7 +189,8 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const int maxL = max_len_of(ls, c.batch);
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
-  const size_t smem = hist ? (size_t)gs * kHistBins * 4 : 0;
+  const bool grouped = c.variant == TB_BUTLER_GROUP;
+  const size_t smem = hist ? (size_t)(grouped ? 1 : gs) * kHistBins * 4 : 0;
   // the most tokens per CTA (up to 4 steps) that still gives about three
   // CTAs per SM; short or small batches get one step per CTA
   int iters = 4;
@@ -198,17 +200,14 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.iters = iters;
   const int chunk = kScoreStep * iters;
   dim3 grid((maxL + chunk - 1) / chunk, c.n_kv_heads, c.batch);
-#define TB_SCORE_CASE(T, DI, GSV)                                                            \
-  if (c.d_imp == DI && gs == GSV) {                                                          \
-    if (hist) {                                                                              \
-      auto k = score_kernel<T, DI, GSV, true>;                                               \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);       \
-      launch_pdl(k, grid, dim3(kScoreThreads), smem, st, p);                                 \
-    } else {                                                                                 \
-      launch_pdl(score_kernel<T, DI, GSV, false>, grid, dim3(kScoreThreads), 0, st, p);      \
-    }                                                                                        \
-    ++ctx->launches;                                                                         \
-    return cuda_status(cudaGetLastError());                                                  \
+#define TB_SCORE_CASE(T, DI, GSV)                                                                    \
+  if (c.d_imp == DI && gs == GSV) {                                                                  \
+    auto k = hist ? (grouped ? score_kernel<T, DI, GSV, true, true> : score_kernel<T, DI, GSV, true, false>) \
+                  : (grouped ? score_kernel<T, DI, GSV, false, true> : score_kernel<T, DI, GSV, false, false>); \
+    if (hist) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
+    launch_pdl(k, grid, dim3(kScoreThreads), smem, st, p);                                           \
+    ++ctx->launches;                                                                                 \
+    return cuda_status(cudaGetLastError());                                                          \
   }
   if (c.kv_dtype == TB_BF16) {
     TB_SCORE_CASE(__nv_bfloat16, 32, 4)
@@ -614,7 +613,7 @@ TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows
   if (s != TB_OK) return s;
   const tb_config& c = ctx->cfg;
   if (!scores || (!idx && !count && !mask)) return TB_ERR_INVALID_ARG;
-  if (rows_per_seq != c.n_q_heads && rows_per_seq != 1) return TB_ERR_SHAPE;
+  if (rows_per_seq != c.n_q_heads && rows_per_seq != c.n_kv_heads && rows_per_seq != 1) return TB_ERR_SHAPE;
   if (!aligned16(scores)) return TB_ERR_SHAPE;
   if (idx) {
     const LayerState& ls = ctx->layers[layer];
@@ -636,7 +635,8 @@ TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uin
   tb_status s = check_layer(ctx, layer);
   if (s != TB_OK) return s;
   if (!q || !out) return TB_ERR_INVALID_ARG;
-  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE)
+  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE &&
+      mask_mode != TB_MASK_GROUP)
     return TB_ERR_INVALID_ARG;
   if (mask_mode != TB_MASK_DENSE && !mask) return TB_ERR_INVALID_ARG;
   if (!aligned16(q)) return TB_ERR_SHAPE;
@@ -650,7 +650,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   const tb_config& c = ctx->cfg;
   if (!k_new || !v_new || !q || !out) return TB_ERR_INVALID_ARG;
   const bool dense = ((c.dense_layer_mask >> layer) & 1ull) || c.keep_pct >= 100;
-  if (!dense && c.variant == TB_BUTLER && !q_imp_producer) return TB_ERR_INVALID_ARG;
+  if (!dense && c.variant != TB_SOFTVOTE && !q_imp_producer) return TB_ERR_INVALID_ARG;
   if (!aligned16(q)) return TB_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   trace_point(ctx, 0, st);
@@ -662,14 +662,16 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, nullptr, TB_MASK_DENSE, out, nullptr, st);
   }
-  if (c.variant == TB_BUTLER) {
+  if (c.variant == TB_BUTLER || c.variant == TB_BUTLER_GROUP) {
+    const bool grouped = c.variant == TB_BUTLER_GROUP;
     s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
-    s = launch_select(ctx, layer, ctx->scores, true, c.n_q_heads, nullptr, 0, nullptr, ctx->mask, st);
+    s = launch_select(ctx, layer, ctx->scores, true, grouped ? c.n_kv_heads : c.n_q_heads, nullptr, 0, nullptr,
+                      ctx->mask, st);
     if (s != TB_OK) return s;
     trace_point(ctx, 3, st);
-    return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, nullptr, st);
+    return launch_attn(ctx, layer, q, ctx->mask, grouped ? TB_MASK_GROUP : TB_MASK_PER_HEAD, out, nullptr, st);
   }
   // soft voting: votes over the full K (the appended row included), one shared set
   prepare_hist(ctx, st);

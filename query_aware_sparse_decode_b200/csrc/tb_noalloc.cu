@@ -66,7 +66,8 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
   if ((gs != 1 && gs != 2 && gs != 4 && gs != 8) || (D != 64 && D != 128)) return TB_ERR_UNSUPPORTED;
   if (max_len < 256 || max_len % 256) return TB_ERR_SHAPE;
   if (cache->kv_dtype != TB_BF16 && cache->kv_dtype != TB_F32) return TB_ERR_INVALID_ARG;
-  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE)
+  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE &&
+      mask_mode != TB_MASK_GROUP)
     return TB_ERR_INVALID_ARG;
   if (mask_mode != TB_MASK_DENSE && !mask) return TB_ERR_INVALID_ARG;
   int maxL = 0;

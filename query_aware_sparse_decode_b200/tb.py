@@ -16,8 +16,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtb.so")
 
 TB_OK = 0
 TB_BF16, TB_F32 = 0, 1
-TB_BUTLER, TB_SOFTVOTE = 0, 1
-TB_MASK_PER_HEAD, TB_MASK_SHARED, TB_MASK_DENSE = 0, 1, 2
+TB_BUTLER, TB_SOFTVOTE, TB_BUTLER_GROUP = 0, 1, 2
+TB_MASK_PER_HEAD, TB_MASK_SHARED, TB_MASK_DENSE, TB_MASK_GROUP = 0, 1, 2, 3
 MAX_BATCH = 128
 MAX_LAYERS = 64
 

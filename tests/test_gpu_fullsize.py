@@ -107,26 +107,28 @@ def _check_shape_of_sets(mask: torch.Tensor, lens, keep_pct: int, sink: int, win
         assert bits[b, :, :min(sink, L)].all() and bits[b, :, max(L - window, 0):L].all()
 
 
-def _gpu_step(ctx, wl, layer: int, dl, k_dev, v_dev, keep_pct: int) -> dict:
+def _gpu_step(ctx, wl, layer: int, dl, k_dev, v_dev, keep_pct: int, group: bool = False) -> dict:
     """One decode step from len L - 1 at the given budget, fused and through
-    the separate calls (which keep scores and selection)."""
+    the separate calls (which keep scores and selection).  With `group`, one
+    set per KV group (rows [B][Hkv])."""
     cfg = ctx.cfg
+    rows = wl.Hkv if group else wl.Hq
     ctx.set_budget(keep_pct, wl.sink, wl.window)
     ctx.set_seq_lens(layer, [wl.L - 1] * wl.B)
     out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
     ctx.decode_step(layer, k_dev, v_dev, dl.q_dev, dl.q_imp_dev, out)
     assert ctx.seq_lens(layer) == [wl.L] * wl.B
     dense = layer in wl.dense_layers
-    scores = torch.full((wl.B, wl.Hq, cfg.max_len), float("nan"), device="cuda")
-    mask = torch.zeros((wl.B, wl.Hq, cfg.max_len // 32), dtype=torch.int32, device="cuda")
+    scores = torch.full((wl.B, rows, cfg.max_len), float("nan"), device="cuda")
+    mask = torch.zeros((wl.B, rows, cfg.max_len // 32), dtype=torch.int32, device="cuda")
     out2 = torch.empty_like(out)
     lse = torch.empty((wl.B, wl.Hq), device="cuda")
     if dense:
         ctx.sparse_attn(layer, dl.q_dev, None, TB.TB_MASK_DENSE, out2, lse)
     else:
         ctx.score(layer, dl.q_imp_dev, scores)
-        ctx.select(layer, scores, wl.Hq, mask=mask)
-        ctx.sparse_attn(layer, dl.q_dev, mask, TB.TB_MASK_PER_HEAD, out2, lse)
+        ctx.select(layer, scores, rows, mask=mask)
+        ctx.sparse_attn(layer, dl.q_dev, mask, TB.TB_MASK_GROUP if group else TB.TB_MASK_PER_HEAD, out2, lse)
     torch.cuda.synchronize()
     assert ctx.check_status() == 0
     assert torch.equal(out, out2)
@@ -135,15 +137,15 @@ def _gpu_step(ctx, wl, layer: int, dl, k_dev, v_dev, keep_pct: int) -> dict:
     return {"out": out.float().cpu().numpy(), "lse": lse.cpu().numpy(), "scores": scores, "mask": mask}
 
 
-def _decode_full(wl, layer: int, samples, keeps=None) -> None:
+def _decode_full(wl, layer: int, samples, keeps=None, group: bool = False) -> None:
     keeps = (wl.keep_pct,) if keeps is None else keeps
-    cfg = config_of(wl)
+    cfg = config_of(wl, variant=TB.TB_BUTLER_GROUP if group else TB.TB_BUTLER)
     _need_device_bytes(_layer_bytes(wl, cfg.max_len) + len(keeps) * wl.B * wl.Hq * cfg.max_len * 4)
     ctx = TB.Context(cfg)
     dl = make_layer_device(ctx, wl, layer, wl.L - 1)
     k_raw, v_raw = S.kv_new(wl, layer)
     k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
-    gpu = {P: _gpu_step(ctx, wl, layer, dl, k_dev, v_dev, P) for P in keeps}
+    gpu = {P: _gpu_step(ctx, wl, layer, dl, k_dev, v_dev, P, group) for P in keeps}
     dense = layer in wl.dense_layers
     lens = [wl.L] * wl.B
     # oracle on the sampled (sequence, KV head) slabs
@@ -161,15 +163,17 @@ def _decode_full(wl, layer: int, samples, keeps=None) -> None:
             assert np.all(np.abs(kimp - O.project_keys(Kg, dl.W)) <= 8e-6 * (np.abs(Kg) @ np.abs(dl.W)) + 1e-30)
         for P, r in gpu.items():
             sel, ref, ref_lse, sc = O.decode_layer(dl.q, K, V, dl.W, dl.qimp, layer, wl.G, lens, P, wl.sink,
-                                                   wl.window, dense=dense, heads=heads, batches=[b])
+                                                   wl.window, dense=dense, heads=heads, batches=[b], group=group)
             if not dense:
-                got_sets = sets_from_mask(r["mask"][b:b + 1, g * gs:(g + 1) * gs], [wl.L])
+                got_sets = (sets_from_mask(r["mask"][b:b + 1, g:g + 1], [wl.L]) if group
+                            else sets_from_mask(r["mask"][b:b + 1, g * gs:(g + 1) * gs], [wl.L]))
             for h in heads:
                 what = f"layer {layer} keep {P} b{b} h{h}"
                 if not dense:
-                    s = r["scores"][b, h, :wl.L].cpu().numpy().astype(np.float64)
+                    srow = g if group else h
+                    s = r["scores"][b, srow, :wl.L].cpu().numpy().astype(np.float64)
                     assert np.max(np.abs(s - sc[b, h])) <= 1e-5 * np.max(np.abs(sc[b, h])), what
-                    gset = got_sets[0, h - g * gs]
+                    gset = got_sets[0, 0 if group else h - g * gs]
                     assert tie_band_ok(gset, sel[b, h], sc[b, h], wl.L, P, wl.sink, wl.window), what
                     if not np.array_equal(gset, sel[b, h]):
                         # a different but valid set (inside the tie band):
@@ -185,6 +189,12 @@ def _decode_full(wl, layer: int, samples, keeps=None) -> None:
 @pytest.mark.parametrize("layer", DECODE_LAYERS)
 def test_decode32_B4_L131072_sampled_heads(layer):
     _decode_full(DECODE, layer, DECODE_SAMPLES)
+
+
+@pytest.mark.parametrize("L", (16384, 131072, 262144))
+def test_long_context_sweep_group_selection(L):
+    wl = S.sweep(L, S.SWEEP_KEEP[0])
+    _decode_full(wl, 0, ((0, 0), (0, wl.Hkv - 1)), keeps=S.SWEEP_KEEP, group=True)
 
 
 @pytest.mark.parametrize("L", S.SWEEP_LENGTHS)

@@ -315,6 +315,60 @@ def _decode_e2e(wl, layer=0):
     return ctx, sel, got_sets
 
 
+def _decode_e2e_group(wl, layer=0):
+    """The per-KV-group option: one set per (b, g) from the group's summed
+    scores, attended by every head of the group."""
+    cfg = config_of(wl, variant=TB.TB_BUTLER_GROUP)
+    ctx = TB.Context(cfg)
+    lens0 = [L - 1 for L in wl.seq_lens]
+    ld = make_layer(ctx, wl, layer, lens0)
+    ctx.project_kimp(layer, 0, max(lens0))
+    k_raw, v_raw = S.kv_new(wl, layer)
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+    ctx.decode_step(layer, to_dev(k_raw, wl), to_dev(v_raw, wl), ld.q_dev, ld.q_imp_dev, out)
+    lens = ctx.seq_lens(layer)
+    scores = torch.full((wl.B, wl.Hkv, cfg.max_len), float("nan"), device="cuda")
+    mask = torch.zeros((wl.B, wl.Hkv, cfg.max_len // 32), dtype=torch.int32, device="cuda")
+    out2 = torch.empty_like(out)
+    ctx.score(layer, ld.q_imp_dev, scores)
+    ctx.select(layer, scores, wl.Hkv, mask=mask)
+    ctx.sparse_attn(layer, ld.q_dev, mask, TB.TB_MASK_GROUP, out2)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    assert torch.equal(out, out2)
+    K = np.concatenate([ld.K, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
+    V = np.concatenate([ld.V, np.zeros((wl.B, wl.Hkv, 1, wl.D))], axis=2)
+    k64, v64 = S.widen(k_raw, wl.dtype), S.widen(v_raw, wl.dtype)
+    for b, L in enumerate(lens):
+        K[b, :, L - 1], V[b, :, L - 1] = k64[b], v64[b]
+    sel, ref, _, sc = O.decode_layer(ld.q, K, V, ld.W, ld.qimp, layer, wl.G, lens, wl.keep_pct, wl.sink,
+                                     wl.window, dense=False, group=True)
+    got_sets = sets_from_mask(mask, lens)
+    s_gpu = scores.cpu().numpy().astype(np.float64)
+    o = out.float().cpu().numpy()
+    gs = wl.Hq // wl.Hkv
+    scale = 1.0 / math.sqrt(wl.D)
+    mism = 0
+    for b, L in enumerate(lens):
+        for g in range(wl.Hkv):
+            lead = g * gs
+            if L:
+                assert np.max(np.abs(s_gpu[b, g, :L] - sc[b, lead])) <= 1e-5 * np.max(np.abs(sc[b, lead]))
+            gset = got_sets[b, g]
+            assert tie_band_ok(gset, sel[b, lead], sc[b, lead], L, wl.keep_pct, wl.sink, wl.window)
+            if not np.array_equal(gset, sel[b, lead]):
+                mism += 1
+            for h in range(lead, lead + gs):
+                want, _ = O.attend(ld.q[b, h], K[b, g, :L], V[b, g, :L], gset, scale)
+                assert_close_rows(o[b, h][None], want[None], wl.dtype, f"group b{b} h{h}")
+    assert mism <= max(1, wl.B * wl.Hkv // 10)
+
+
+@pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
+def test_group_selection_decode_step(wl):
+    _decode_e2e_group(wl)
+
+
 @pytest.mark.parametrize("wl", [S.TINY_F32, SMALL_BF16, SMALL_D64, RAGGED], ids=lambda w: w.name)
 def test_decode_step_end_to_end(wl):
     _decode_e2e(wl)

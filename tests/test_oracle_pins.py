@@ -380,3 +380,41 @@ def test_softvote_layer_shares_one_set_over_heads():
     for h in range(4):
         o, _ = O.attend(q[0, h], K[0, h // 2], V[0, h // 2], sel[0], 0.25)
         assert np.allclose(out[0, h], o, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- per-group option
+def test_group_scores_one_head_is_the_head_and_sum_is_the_summed_query():
+    rng = np.random.default_rng(11)
+    K_imp = rng.standard_normal((40, 6))
+    q1 = rng.standard_normal((1, 6))
+    assert np.array_equal(O.group_scores(q1, K_imp), O.importance_scores(q1[0], K_imp))
+    q4 = rng.standard_normal((4, 6))
+    # textbook loops over the summed query (the scores are linear in q)
+    qsum = [sum(q4[h, j] for h in range(4)) for j in range(6)]
+    want = np.array([sum(qsum[j] * K_imp[t, j] for j in range(6)) for t in range(40)])
+    assert np.allclose(O.group_scores(q4, K_imp), want, rtol=1e-13, atol=1e-13)
+
+
+def test_group_selection_shares_one_set_per_group_and_equals_per_head_for_equal_queries():
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, D, dimp, L, G = 1, 8, 2, 16, 4, 300, 1
+    q = rng.standard_normal((B, Hq, D))
+    K = rng.standard_normal((B, Hkv, L, D))
+    V = rng.standard_normal((B, Hkv, L, D))
+    W = rng.standard_normal((D, dimp))
+    qi = rng.standard_normal((B * Hq, G, 1, dimp))
+    sel, out, _, sc = O.decode_layer(q, K, V, W, qi, 1, G, L, 30, 4, 16, dense=False, group=True)
+    gs = Hq // Hkv
+    for h in range(Hq):
+        lead = (h // gs) * gs
+        assert np.array_equal(sel[0, h], sel[0, lead])            # one set per group
+        assert np.array_equal(sc[0, h], sc[0, lead])
+        ref, _ = O.attend(q[0, h], K[0, h // gs], V[0, h // gs], sel[0, h], 1 / math.sqrt(D))
+        assert np.allclose(out[0, h], ref)
+    # every head of a group with the same importance query: the group sum is a
+    # positive multiple of each head's scores, so the sets are the per-head sets
+    qi_same = np.repeat(qi.reshape(B, Hkv, gs, G, 1, dimp)[:, :, :1], gs, axis=2).reshape(B * Hq, G, 1, dimp)
+    sel_g, _, _, _ = O.decode_layer(q, K, V, W, qi_same, 1, G, L, 30, 4, 16, dense=False, group=True)
+    sel_h, _, _, _ = O.decode_layer(q, K, V, W, qi_same, 1, G, L, 30, 4, 16, dense=False)
+    for h in range(Hq):
+        assert np.array_equal(sel_g[0, h], sel_h[0, h])
