@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=4)
     ap.add_argument("--length", type=int, default=131072)
     ap.add_argument("--keep", type=int, default=30)
+    ap.add_argument("--variant", choices=["butler", "group"], default="butler",
+                    help="per-head selection (the pages' method, default) or the per-KV-group option")
     ap.add_argument("--trace-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -62,7 +64,14 @@ def workload(args):
     wl = base.with_(n_layers=args.layers, B=args.batch, L=args.length, keep_pct=args.keep)
     if (wl.n_layers, wl.B, wl.L, wl.keep_pct) != (base.n_layers, base.B, base.L, base.keep_pct):
         wl = wl.with_(name=f"decode{wl.n_layers}_bf16_B{wl.B}_L{wl.L}_keep{wl.keep_pct}")
+    if getattr(args, "variant", "butler") == "group":
+        wl = wl.with_(name=wl.name + "_group_select")
     return wl
+
+
+def variant_code(args):
+    from query_aware_sparse_decode_b200 import tb as TB
+    return TB.TB_BUTLER_GROUP if getattr(args, "variant", "butler") == "group" else TB.TB_BUTLER
 
 
 def step_counts(wl):
@@ -138,7 +147,7 @@ class ClockSampler:
 # from one ncu capture of it (B = 2, L = 131072, keep 30 %; summary under
 # profiles/).  Valid only for the kernel source it was measured on; any
 # change makes it null.
-ATTN_TRAFFIC = {"source_sha256_16": "0e7d73ac5fd68159", "bytes_per_union_row": (811.692544e6 + 5.092096e6) / 1581259}
+ATTN_TRAFFIC = {"source_sha256_16": "81ae913471f38008", "bytes_per_union_row": (811.698176e6 + 4.206336e6) / 1581259}
 
 
 def attn_traffic_per_row():
@@ -249,8 +258,10 @@ def union_rows(ctx, wl, L0, inp):
     from query_aware_sparse_decode_b200 import tb as TB
     kn, vn, qq, qi = inp
     max_len = ctx.cfg.max_len
-    scores = torch.empty((wl.B, wl.Hq, max_len), device=ctx.device)
-    mask = torch.zeros((wl.B, wl.Hq, max_len // 32), dtype=torch.int32, device=ctx.device)
+    group = ctx.cfg.variant == TB.TB_BUTLER_GROUP
+    nrow = wl.Hkv if group else wl.Hq
+    scores = torch.empty((wl.B, nrow, max_len), device=ctx.device)
+    mask = torch.zeros((wl.B, nrow, max_len // 32), dtype=torch.int32, device=ctx.device)
     gs = wl.Hq // wl.Hkv
     rows = {}
     for layer in range(wl.n_layers):
@@ -258,11 +269,14 @@ def union_rows(ctx, wl, L0, inp):
             continue
         ctx.set_seq_lens(layer, [L0 + 1] * wl.B)
         ctx.score(layer, qi[layer // wl.G], scores)
-        ctx.select(layer, scores, wl.Hq, mask=mask)
-        m = mask.view(wl.B, wl.Hkv, gs, -1)
-        u = m[:, :, 0]
-        for j in range(1, gs):
-            u = u | m[:, :, j]
+        ctx.select(layer, scores, nrow, mask=mask)
+        if group:  # one set per group already
+            u = mask
+        else:
+            m = mask.view(wl.B, wl.Hkv, gs, -1)
+            u = m[:, :, 0]
+            for j in range(1, gs):
+                u = u | m[:, :, j]
         bits = np.unpackbits(u.cpu().numpy().view(np.uint8), bitorder="little")
         rows[layer] = int(bits.sum())
     return rows
@@ -279,7 +293,7 @@ def gpu_arm(args, rank, world, local_rank):
     max_len = (wl.L + 255) // 256 * 256
     if max_len == wl.L:
         max_len += 256
-    ctx, bufs, proj = build(wl, max_len, dev)
+    ctx, bufs, proj = build(wl, max_len, dev, variant_code(args))
     stream = torch.cuda.current_stream(dev)
     nvar = min(args.steps + args.warmup, 4)
     host_inputs = [step_inputs_host(wl, s) for s in range(nvar)]
@@ -394,7 +408,7 @@ def gpu_arm(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------- CPU oracle leg
-def oracle_sample(wl, seconds: float):
+def oracle_sample(wl, seconds: float, group: bool = False):
     """Times the fp64 oracle on whole (layer, sequence) slabs of the workload
     (score, select, attend for all query heads; inputs regenerated on the host
     and excluded from the timing) until about `seconds` of oracle work."""
@@ -426,7 +440,7 @@ def oracle_sample(wl, seconds: float):
         qi_b = qi.reshape(wl.B, wl.Hq, wl.G, 1, wl.d_imp)[b]
         t0 = time.perf_counter()
         sel, _, _, _ = O.decode_layer(q, K, V, W, qi_b, layer, wl.G, wl.L, wl.keep_pct, wl.sink, wl.window,
-                                      dense=False, K_imp=Kimp)
+                                      dense=False, K_imp=Kimp, group=group)
         dt = time.perf_counter() - t0
         elapsed += dt
         tokens += wl.Hq * wl.L + sum(len(v) for v in sel.values())
@@ -443,7 +457,7 @@ def reference_arm(args, rank, world):
     wl = workload(args)
     vals = []
     for s in range(args.warmup + args.steps):
-        r = oracle_sample(wl, seconds=0.0)  # one slab per step
+        r = oracle_sample(wl, seconds=0.0, group=args.variant == "group")  # one slab per step
         if s >= args.warmup:
             vals.append(r)
     value = statistics.mean(v["value"] for v in vals)
@@ -491,6 +505,11 @@ def _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream):
     return med
 
 
+def _variant_name(variant):
+    from query_aware_sparse_decode_b200 import tb as TB
+    return {TB.TB_SOFTVOTE: "softvote", TB.TB_BUTLER_GROUP: "group"}.get(variant, "butler")
+
+
 def _table_case(wl, variant, dev, iters, flush_buf, peak):
     import torch
     from query_aware_sparse_decode_b200 import synth as S
@@ -521,14 +540,19 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
         first = wl.B * wl.Hkv * wl.L * wl.D * 2               # the full K, read for the logits
         union = int(np.unpackbits(mask.cpu().numpy().view(np.uint8)).sum()) * wl.Hkv
     else:
-        scores = torch.empty((wl.B, wl.Hq, max_len), device=dev)
-        mask = torch.zeros((wl.B, wl.Hq, max_len // 32), dtype=torch.int32, device=dev)
+        group = variant == TB.TB_BUTLER_GROUP
+        nrow = wl.Hkv if group else wl.Hq
+        scores = torch.empty((wl.B, nrow, max_len), device=dev)
+        mask = torch.zeros((wl.B, nrow, max_len // 32), dtype=torch.int32, device=dev)
         ctx.score(layer, inp[3], scores)
-        ctx.select(layer, scores, wl.Hq, mask=mask)
-        m = mask.view(wl.B, wl.Hkv, gs, -1)
-        u = m[:, :, 0]
-        for j in range(1, gs):
-            u = u | m[:, :, j]
+        ctx.select(layer, scores, nrow, mask=mask)
+        if group:
+            u = mask
+        else:
+            m = mask.view(wl.B, wl.Hkv, gs, -1)
+            u = m[:, :, 0]
+            for j in range(1, gs):
+                u = u | m[:, :, j]
         first = wl.B * wl.Hkv * wl.L * wl.d_imp * 4           # K_imp
         union = int(np.unpackbits(u.cpu().numpy().view(np.uint8)).sum())
     torch.cuda.synchronize()
@@ -545,7 +569,7 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
         r["attn_frac"] = r["attn_gbs"] / peak
         r["step_gbs"] = (first + attn_bytes) / (t["total"] * 1e-6) / 1e9
         return r
-    line = {"table": "decode", "workload": wl.name, "variant": "softvote" if variant == TB.TB_SOFTVOTE else "butler",
+    line = {"table": "decode", "workload": wl.name, "variant": _variant_name(variant),
             "B": wl.B, "L": wl.L, "keep_pct": wl.keep_pct, "dense": dense,
             "first_pass_bytes": first, "union_rows": union, "attn_bytes": attn_bytes,
             "us_cold_l2": cold, "us_hot_l2": hot, "rates_cold_l2": rates(cold), "rates_hot_l2": rates(hot),
@@ -616,10 +640,11 @@ def kernel_table(args):
         for P in S.SWEEP_KEEP:
             cases.append((S.sweep(L, P), TB.TB_BUTLER))
             cases.append((S.sweep(L, P), TB.TB_SOFTVOTE))
+            cases.append((S.sweep(L, P), TB.TB_BUTLER_GROUP))
     import re
     pick = re.compile(args.table_only) if args.table_only else None
     for wl, variant in cases:
-        name = f"{wl.name}_{'softvote' if variant == TB.TB_SOFTVOTE else 'butler'}"
+        name = f"{wl.name}_{_variant_name(variant)}"
         if pick is None or pick.search(name):
             print(json.dumps(_table_case(wl, variant, dev, args.table_iters, flush_buf, peak)), flush=True)
     if pick is None or pick.search(S.PREFILL_L32K.name):
@@ -649,7 +674,7 @@ def main():
     r = gpu_arm(args, rank, world, local_rank)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(r["wl"], args.cpu_seconds)
+        cpu = oracle_sample(r["wl"], args.cpu_seconds, group=args.variant == "group")
     if rank == 0:
         wl = r["wl"]
         avg = r["avg"]
@@ -661,6 +686,7 @@ def main():
             "config": {"workload": wl.name, "layers": wl.n_layers, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv,
                        "D": wl.D, "d_imp": wl.d_imp, "G": wl.G, "L": wl.L, "keep_pct": wl.keep_pct,
                        "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
+                       "selection": "per_kv_group" if args.variant == "group" else "per_query_head",
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (caches of all layers, no flush)"},
             "us_per_layer": r["ms_step"] * 1e3 / wl.n_layers,
