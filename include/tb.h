@@ -218,6 +218,16 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
  * tb_select(rows_per_seq = 1) and attend with TB_MASK_SHARED. */
 TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream);
 
+/* Failure-detection self-test (no counterpart on the pages).  Launches one
+ * CTA that waits on an mbarrier expecting one arrival, with the same bounded
+ * wait the pipelined kernels use (the tensor-core K_imp projection).  With
+ * `arrive` != 0 the CTA arrives itself and the wait completes; with 0 nothing
+ * arrives, the wait gives up after `cycles` SM cycles (1 .. 2e10) and sets
+ * TB_DEV_ERR_TIMEOUT in the status word read by tb_check_status.  Neither
+ * case faults, traps or hangs; the context stays usable.  TB_ERR_INVALID_ARG
+ * for a NULL context or `cycles` out of range. */
+TB_API tb_status tb_selftest_bounded_wait(tb_ctx* ctx, long long cycles, int arrive, void* stream);
+
 /* ---- allocation-free attention ---------------------------------------------
  * The model card and the papers have no counterpart to this entry point; it
  * exists for callers that cannot allocate device memory (a serving loop with

@@ -770,6 +770,32 @@ TB_API tb_status tb_launch_count(const tb_ctx* ctx, uint64_t* count) {
   return TB_OK;
 }
 
+// Failure-detection self-test of the library's bounded mbarrier wait
+// (mbar_wait, as used by the pipelined kernels): one mbarrier that expects
+// one arrival.  With `arrive`, thread 0 arrives and the wait
+// completes; otherwise nothing arrives, the wait gives up after `cycles` SM
+// cycles and TB_DEV_ERR_TIMEOUT is recorded.  The CTA then exits normally.
+static __global__ void wait_selftest_kernel(uint32_t* status, long long cycles, int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (arrive) mbar_arrive_cta(&bar);
+    if (!mbar_wait(&bar, 0, cycles)) atomicOr(status, TB_DEV_ERR_TIMEOUT);
+  }
+}
+
+TB_API tb_status tb_selftest_bounded_wait(tb_ctx* ctx, long long cycles, int arrive, void* stream) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  if (cycles < 1 || cycles > 20000000000LL) return TB_ERR_INVALID_ARG;  // at most about ten seconds
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctx->status, cycles, arrive ? 1 : 0);
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
 TB_API tb_status tb_check_status(tb_ctx* ctx, uint32_t* flags) {
   if (!ctx) return TB_ERR_INVALID_ARG;
   uint32_t v = 0;

@@ -29,7 +29,7 @@ STATUS_NAMES = {0: "TB_OK", 1: "TB_ERR_INVALID_ARG", 2: "TB_ERR_SHAPE", 3: "TB_E
 EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "tb_get_seq_lens", "tb_set_budget",
            "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
            "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
-           "tb_check_status", "tb_status_string", "tb_destroy")
+           "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait")
 
 
 class TBError(RuntimeError):
@@ -84,6 +84,7 @@ def lib():
             "tb_check_status": [vp, P(ctypes.c_uint32)],
             "tb_status_string": [i32],
             "tb_destroy": [vp],
+            "tb_selftest_bounded_wait": [vp, ctypes.c_longlong, i32, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -219,6 +220,12 @@ class Context:
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().tb_trace_events(self._h, arr, len(events)), "tb_trace_events")
         self._trace = events
+
+    def selftest_bounded_wait(self, cycles: int, arrive: bool, stream=None) -> None:
+        """Launch the bounded-wait self-test (see include/tb.h); read the
+        outcome with check_status() after a synchronisation."""
+        _check(lib().tb_selftest_bounded_wait(self._h, int(cycles), 1 if arrive else 0, _stream(stream)),
+               "tb_selftest_bounded_wait")
 
     def launch_count(self) -> int:
         n = ctypes.c_uint64(0)
