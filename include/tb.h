@@ -218,6 +218,40 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
  * tb_select(rows_per_seq = 1) and attend with TB_MASK_SHARED. */
 TB_API tb_status tb_softvote_scores(tb_ctx* ctx, int layer, const void* q, float* votes, void* stream);
 
+/* ---- amortised selection ----------------------------------------------------
+ * TokenButler abstract (importance predicted at intervals, neighbouring tokens
+ * fetched) and TokenSelect README ("Selection Cache": consecutive similar
+ * queries share selection results).  The pages fix none of the parameters.
+ * With a cache bound to a layer and tb_set_reuse(interval > 0), every decode
+ * step of that layer decides per selection row (query head, or KV group with
+ * TB_BUTLER_GROUP) whether to reuse the row's cached selection:
+ *   reuse  iff  the row takes a real top-k now (0 < k < candidates), the
+ *               cache holds a top-k selected at length len0 > 0,
+ *               len - len0 <= interval, and
+ *               cos(q_hat_now, q_hat_cached) >= tau (fp32; for a group, its
+ *               heads' importance queries summed in head order).
+ * A reused row's set is the cached top-k (the cached mask inside
+ * [sink, len0 - window)), widened by `radius` tokens on each side, kept inside
+ * [sink, len - window), plus the current sink and window; its scores and
+ * selection are not computed (a KV group whose rows all reuse is not scored).
+ * Other rows select afresh and refill the cache.  The count check of reused
+ * rows is skipped (their size is the cached top-k's). */
+
+/* Bytes of one layer's selection cache for `cfg`. */
+TB_API tb_status tb_selection_cache_size(const tb_config* cfg, size_t* bytes);
+/* Bind a caller-owned, zero-filled, 256-byte aligned device buffer of at least
+ * tb_selection_cache_size bytes as layer `layer`'s selection cache (NULL
+ * unbinds).  TB_ERR_UNSUPPORTED for TB_SOFTVOTE. */
+TB_API tb_status tb_bind_selection_cache(tb_ctx* ctx, int layer, void* cache, size_t bytes);
+/* Reuse parameters: tau in [-1, 1], interval >= 0 tokens (0 turns reuse off),
+ * radius in [0, 31]. */
+TB_API tb_status tb_set_reuse(tb_ctx* ctx, float tau, int interval, int radius);
+
+/* Copy the selection masks of the last sparse tb_decode_step, [B][rows][max_len/32]
+ * uint32 (rows: Hq, or Hkv with TB_BUTLER_GROUP), into a caller device buffer
+ * of >= `bytes` bytes (stream-ordered; words past ceil(len/32) are stale). */
+TB_API tb_status tb_copy_step_masks(tb_ctx* ctx, uint32_t* dst, size_t bytes, void* stream);
+
 /* Failure-detection self-test (no counterpart on the pages).  Launches one
  * CTA that waits on an mbarrier expecting one arrival, with the same bounded
  * wait the pipelined kernels use (the tensor-core K_imp projection).  With

@@ -35,6 +35,15 @@ Readings where the sources leave a step open (each marked "Reading" below):
       summed over all query heads, one set shared by all heads.
   An empty selected set gives a zero output and lse = -inf.
 
+  R18 amortised selection (TokenButler abstract: prediction interval with
+      neighbour fetching; TokenSelect README, "Selection Cache"): a row reuses
+      its cached top-k when it takes a real top-k now, the cache holds a top-k
+      chosen at length len0 > 0 with len - len0 <= interval, and the cosine of
+      the current and cached importance queries is >= tau; the reused set is
+      the cached top-k widened by `radius` tokens each side, kept inside the
+      current candidates, plus the current sink and window (reuse_decision,
+      reused_set).  The pages fix none of these numbers.
+
 Option beyond the sources (not a reading of them): per-KV-group selection,
 where the importance scores of a group's query heads are summed and the
 group selects once with the same budget, sink, window and tie rules; every
@@ -157,6 +166,38 @@ def group_scores(q_hat_heads: np.ndarray, K_imp: np.ndarray) -> np.ndarray:
     for h in range(q.shape[0]):
         total += importance_scores(q[h], K_imp)
     return total
+
+
+# ------------------------------------------------------------------ amortised selection
+def reuse_decision(q_now, q_cached, L: int, len0: int, interval: int, tau: float, keep_pct: int, sink: int,
+                   window: int) -> bool:
+    """Reading R18: whether a row reuses its cached selection this step."""
+    cand = L - window - sink if L - window > sink else 0
+    k = min(token_budget(L, keep_pct), cand)
+    if not (0 < k < cand):
+        return False
+    if len0 <= 0 or L < len0 or L - len0 > interval:
+        return False
+    a = np.asarray(q_now, dtype=np.float64)
+    c = np.asarray(q_cached, dtype=np.float64)
+    na, nc = math.sqrt(float(a @ a)), math.sqrt(float(c @ c))
+    if na == 0.0 or nc == 0.0:
+        return False
+    return float(a @ c) / (na * nc) >= tau
+
+
+def reused_set(cached: np.ndarray, len0: int, L: int, sink: int, window: int, radius: int) -> np.ndarray:
+    """Reading R18: the set a reusing row attends to at length L."""
+    cached = np.asarray(cached, dtype=np.int64)
+    topk = cached[(cached >= sink) & (cached < len0 - window)]
+    widened = set(topk.tolist())
+    for d in range(1, radius + 1):
+        widened.update((topk - d).tolist())
+        widened.update((topk + d).tolist())
+    keep = {t for t in widened if sink <= t < L - window}
+    keep.update(range(0, min(sink, L)))
+    keep.update(range(max(L - window, 0), L))
+    return np.array(sorted(keep), dtype=np.int64)
 
 
 # ------------------------------------------------------------------ one decode layer

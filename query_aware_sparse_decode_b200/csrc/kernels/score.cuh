@@ -34,6 +34,7 @@ struct ScoreParams {
   int G, slot, Hq, Hkv, max_len;
   int sink, window;
   int iters;           // CTA iterations of kScoreStep tokens (1, 2 or 4)
+  const uint32_t* reuse;  // [B*rows] amortised selection: rows that skip scoring, or null
   int lens[kMaxBatch];
 };
 
@@ -48,6 +49,13 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   const int L = p.lens[b];
   const int t_base = chunk * kScoreStep * p.iters;
   if (t_base >= L) return;
+  if (p.reuse != nullptr) {  // every row of this group reuses its cached selection: nothing to score
+    const size_t r0 = GROUPED ? (size_t)b * p.Hkv + g : (size_t)b * p.Hq + g * GS;
+    bool all = true;
+#pragma unroll
+    for (int hh = 0; hh < NR; ++hh) all = all && p.reuse[r0 + hh] != 0u;
+    if (all) return;
+  }
   const T* qi = reinterpret_cast<const T*>(p.q_imp);
   for (int e = tid; e < DIMP * GS; e += kScoreThreads) {
     const int j = e / GS, hh = e % GS;

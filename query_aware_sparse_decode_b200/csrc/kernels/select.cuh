@@ -33,6 +33,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "reuse.cuh"
 
 namespace tb {
 
@@ -59,6 +60,11 @@ struct SelectParams {
   long long row_stride;
   int rows_per_seq, idx_cap, mask_words;
   int keep_pct, sink, window;
+  // amortised selection (decode step only; all null otherwise)
+  const uint32_t* reuse;  // [B*rows] 1: this row reuses its cached selection
+  const int32_t* sc_len;  // [B*rows] length of the cached selection
+  uint32_t* sc_mask;      // [B*rows][mask_words] cached masks (refilled by fresh rows)
+  int reuse_radius;
   int lens[kMaxBatch];
 };
 
@@ -205,6 +211,37 @@ __global__ void __launch_bounds__(kScatThreads, 4) select_scatter_kernel(const S
   const int t_begin = chunk * kSelChunk;
   if (t_begin >= rs.L) return;
   const long long row = (long long)b * p.rows_per_seq + r;
+  if (p.reuse != nullptr && p.reuse[row]) {
+    // the row reuses its cached selection: cached top-k (widened by the
+    // radius) inside the current candidates, plus the current sink and window
+    const uint32_t* cm = p.sc_mask + row * p.mask_words;
+    const int hi_prev = p.sc_len[row] - p.window, lo = p.sink;
+    auto topk = [&](int w) -> uint32_t {
+      return (w < 0 || w >= p.mask_words) ? 0u : (cm[w] & range_bits(w * 32, lo, hi_prev));
+    };
+    uint32_t kept = 0;
+    const int w_end = min((t_begin + kSelChunk) >> 5, (rs.L + 31) >> 5);
+    for (int w = (t_begin >> 5) + tid; w < w_end; w += kScatThreads) {
+      uint32_t x = topk(w);
+      if (p.reuse_radius > 0) {
+        const uint32_t prev = topk(w - 1), next = topk(w + 1);
+        const uint64_t below = ((uint64_t)x << 32) | prev;  // tokens 32(w-1) .. 32w+31
+        const uint64_t above = ((uint64_t)next << 32) | x;  // tokens 32w .. 32(w+1)+31
+        uint32_t d = x;
+        for (int sft = 1; sft <= p.reuse_radius; ++sft)
+          d |= (uint32_t)(below >> (32 - sft)) | (uint32_t)(above >> sft);
+        x = d;
+      }
+      const uint32_t word = (x & range_bits(w * 32, lo, rs.hi)) | range_bits(w * 32, 0, min(p.sink, rs.L)) |
+                            range_bits(w * 32, max(rs.L - p.window, 0), rs.L);
+      p.mask[row * p.mask_words + w] = word;
+      kept += __popc(word);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+    if (lane == 0 && kept) atomicAdd(&p.kcount[row], kept);
+    return;
+  }
   const float* s = p.scores + row * p.row_stride;
   // the chunk's scores are requested first, so their latency overlaps the
   // threshold search below.  A warp step covers 256 tokens: lane owns 8
@@ -404,11 +441,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
   __shared__ uint32_t s_above;
   const int r = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
   const RowShape rs = row_shape(p, b);
-  const int L = rs.L, lo = rs.lo, hi = rs.hi, k = rs.k, mode = rs.mode;
+  const int L = rs.L, lo = rs.lo, hi = rs.hi, k = rs.k;
   const long long row = (long long)b * p.rows_per_seq + r;
+  const bool reused = p.reuse != nullptr && p.reuse[row] != 0u;
+  const int mode = reused ? 0 : rs.mode;  // a reused row's mask is complete after the scatter
   const size_t orow = (size_t)row;
   const float* s = p.scores + row * p.row_stride;
   const int lwords = (L + 31) >> 5;
+  // a fresh selection of a row with a selection cache refills it below
+  const bool refill = p.reuse != nullptr && !reused && rs.mode == 2;
 
   bool fallback = false;
   uint32_t prefix1 = 0, k1 = 0, n1 = 0;
@@ -496,8 +537,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
       if (p.count != nullptr) p.count[orow] = (int32_t)total;
       const int sink_n = min(p.sink, L);
       const int win_lo = max(L - p.window, sink_n);
-      if (total != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
+      // a reused set has the cached top-k's size, not this step's k
+      if (!reused && total != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
     }
+    if (refill)
+      for (int w = tid; w < lwords; w += kSelThreads) p.sc_mask[orow * p.mask_words + w] = __ldcg(p.mask + orow * p.mask_words + w);
     __syncthreads();  // every thread has read the counters before they are cleared
     clear_row_state(p, row, b);
     return;
@@ -604,6 +648,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
     const int sink_n = min(p.sink, L);
     const int win_lo = max(L - p.window, sink_n);
     if (out_base != (uint32_t)(sink_n + (L - win_lo) + k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
+  }
+  if (refill) {
+    __syncthreads();  // the mask words written above
+    for (int w = tid; w < lwords; w += kSelThreads) p.sc_mask[orow * p.mask_words + w] = __ldcg(p.mask + orow * p.mask_words + w);
   }
   clear_row_state(p, row, b);
 }

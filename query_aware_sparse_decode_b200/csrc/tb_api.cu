@@ -14,6 +14,7 @@
 #include "kernels/common.cuh"
 #include "kernels/kimp.cuh"
 #include "kernels/prefill.cuh"
+#include "kernels/reuse.cuh"
 #include "kernels/project_tc.cuh"
 #include "kernels/score.cuh"
 #include "kernels/select.cuh"
@@ -32,13 +33,17 @@ struct LayerState {
   bool bound = false;
   CUtensorMap k_map;  // bf16 caches: K rows, 64-column boxes of 128 rows, 128B swizzle
   int lens[TB_MAX_BATCH];
+  // selection cache (amortised selection), caller-owned, or null
+  float* sc_q = nullptr;        // [B*rows][d'] importance query of the cached set
+  int32_t* sc_len = nullptr;    // [B*rows] length at which it was selected (0: empty)
+  uint32_t* sc_mask = nullptr;  // [B*rows][max_len/32] the cached mask
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
   size_t status, hist, ccount, kcount, hist2, hist_end, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats,
-      total;
+      reuse, total;
   int max_splits;
 };
 
@@ -61,6 +66,7 @@ WsLayout layout_of(const tb_config& c) {
   w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
   w.votes = off;   off += align256(B * Lm * 4);
   w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteChunk - 1) / kVoteChunk) * 2 * 4);
+  w.reuse = off;   off += align256(B * Hq * 4);         // per-row reuse decisions of the step
   w.total = off;
   return w;
 }
@@ -106,6 +112,10 @@ struct tb_ctx {
   float* votes = nullptr;
   float* vstats = nullptr;
   bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last resolve)
+  uint32_t* reuse = nullptr;
+  float reuse_tau = 0.f;     // amortised selection: cosine threshold,
+  int reuse_interval = 0;    // at most this many tokens since the cached selection (0: off),
+  int reuse_radius = 0;      // neighbours t +- 1..r of the cached top-k kept as well
   cudaEvent_t trace[6] = {};
   bool tracing = false;
   unsigned long long launches = 0;
@@ -169,7 +179,7 @@ static void prepare_hist(tb_ctx* ctx, cudaStream_t st) {
 }
 
 static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* scores, uint32_t* hist,
-                              cudaStream_t st) {
+                              cudaStream_t st, const uint32_t* reuse = nullptr) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   ScoreParams p{};
@@ -184,6 +194,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   p.max_len = c.max_len;
   p.sink = c.sink;
   p.window = c.window;
+  p.reuse = reuse;
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   if (hist) prepare_hist(ctx, st);  // histograms and candidate counters start at zero
   const int maxL = max_len_of(ls, c.batch);
@@ -235,7 +246,8 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
 // Selection of every row: hist1_ready means the score kernel already built
 // the first-digit histograms (and zeroed the candidate counters).
 static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool hist1_ready, int rows,
-                               int32_t* idx, int idx_cap, int32_t* count, uint32_t* mask, cudaStream_t st) {
+                               int32_t* idx, int idx_cap, int32_t* count, uint32_t* mask, cudaStream_t st,
+                               bool use_cache = false) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   SelectParams p{};
@@ -257,6 +269,12 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   p.keep_pct = c.keep_pct;
   p.sink = c.sink;
   p.window = c.window;
+  if (use_cache) {
+    p.reuse = ctx->reuse;
+    p.sc_len = ls.sc_len;
+    p.sc_mask = ls.sc_mask;
+    p.reuse_radius = ctx->reuse_radius;
+  }
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   const int maxL = max_len_of(ls, c.batch);
   dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
@@ -449,6 +467,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
   ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
   ctx->vstats = reinterpret_cast<float*>(ctx->ws + lay.vstats);
+  ctx->reuse = reinterpret_cast<uint32_t*>(ctx->ws + lay.reuse);
   if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return TB_ERR_CUDA;
@@ -510,6 +529,68 @@ TB_API tb_status tb_set_budget(tb_ctx* ctx, int keep_pct, int sink, int window) 
   ctx->cfg.keep_pct = keep_pct;
   ctx->cfg.sink = sink;
   ctx->cfg.window = window;
+  return TB_OK;
+}
+
+// ------------------------------------------------------------------ amortised selection
+static int sel_rows(const tb_config& c) { return c.variant == TB_BUTLER_GROUP ? c.n_kv_heads : c.n_q_heads; }
+
+struct SelCacheLayout {
+  size_t q, len, mask, total;
+};
+static SelCacheLayout sel_cache_layout(const tb_config& c) {
+  const size_t R = (size_t)c.batch * sel_rows(c);
+  SelCacheLayout l{};
+  size_t off = 0;
+  l.q = off;    off += align256(R * c.d_imp * 4);
+  l.len = off;  off += align256(R * 4);
+  l.mask = off; off += align256(R * (size_t)(c.max_len / 32) * 4);
+  l.total = off;
+  return l;
+}
+
+TB_API tb_status tb_selection_cache_size(const tb_config* cfg, size_t* bytes) {
+  if (!bytes) return TB_ERR_INVALID_ARG;
+  const tb_status s = check_config(cfg);
+  if (s != TB_OK) return s;
+  *bytes = sel_cache_layout(*cfg).total;
+  return TB_OK;
+}
+
+TB_API tb_status tb_bind_selection_cache(tb_ctx* ctx, int layer, void* cache, size_t bytes) {
+  if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
+  LayerState& ls = ctx->layers[layer];
+  if (!cache) {
+    ls.sc_q = nullptr;
+    ls.sc_len = nullptr;
+    ls.sc_mask = nullptr;
+    return TB_OK;
+  }
+  if (ctx->cfg.variant == TB_SOFTVOTE) return TB_ERR_UNSUPPORTED;
+  const SelCacheLayout l = sel_cache_layout(ctx->cfg);
+  if (bytes < l.total) return TB_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(cache) & 255u) != 0) return TB_ERR_SHAPE;
+  char* c = static_cast<char*>(cache);
+  ls.sc_q = reinterpret_cast<float*>(c + l.q);
+  ls.sc_len = reinterpret_cast<int32_t*>(c + l.len);
+  ls.sc_mask = reinterpret_cast<uint32_t*>(c + l.mask);
+  return TB_OK;
+}
+
+TB_API tb_status tb_copy_step_masks(tb_ctx* ctx, uint32_t* dst, size_t bytes, void* stream) {
+  if (!ctx || !dst) return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  const size_t need = (size_t)c.batch * sel_rows(c) * (size_t)(c.max_len / 32) * 4;
+  if (bytes < need) return TB_ERR_SHAPE;
+  return cuda_status(cudaMemcpyAsync(dst, ctx->mask, need, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+}
+
+TB_API tb_status tb_set_reuse(tb_ctx* ctx, float tau, int interval, int radius) {
+  if (!ctx) return TB_ERR_INVALID_ARG;
+  if (!(tau >= -1.f && tau <= 1.f) || interval < 0 || radius < 0 || radius > 31) return TB_ERR_INVALID_ARG;
+  ctx->reuse_tau = tau;
+  ctx->reuse_interval = interval;
+  ctx->reuse_radius = radius;
   return TB_OK;
 }
 
@@ -643,6 +724,39 @@ TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uin
   return launch_attn(ctx, layer, q, mask, mask_mode, out, lse, static_cast<cudaStream_t>(stream));
 }
 
+// Amortised selection: per-row reuse decisions of this step (see reuse.cuh).
+static tb_status launch_reuse_decide(tb_ctx* ctx, int layer, const void* q_imp, cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  ReuseParams p{};
+  p.q_imp = q_imp;
+  p.sc_q = ls.sc_q;
+  p.sc_len = ls.sc_len;
+  p.reuse = ctx->reuse;
+  p.G = c.producer_freq;
+  p.slot = ((layer - 1) % c.producer_freq + c.producer_freq) % c.producer_freq;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.rows_per_seq = sel_rows(c);
+  p.nrows_total = c.batch * p.rows_per_seq;
+  p.tau = ctx->reuse_tau;
+  p.interval = ctx->reuse_interval;
+  p.keep_pct = c.keep_pct;
+  p.sink = c.sink;
+  p.window = c.window;
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
+  const dim3 grid((p.nrows_total + 7) / 8);
+  if (c.kv_dtype == TB_BF16) {
+    if (c.d_imp == 32) launch_pdl(reuse_decide_kernel<__nv_bfloat16, 32>, grid, dim3(256), 0, st, p);
+    else launch_pdl(reuse_decide_kernel<__nv_bfloat16, 16>, grid, dim3(256), 0, st, p);
+  } else {
+    if (c.d_imp == 32) launch_pdl(reuse_decide_kernel<float, 32>, grid, dim3(256), 0, st, p);
+    else launch_pdl(reuse_decide_kernel<float, 16>, grid, dim3(256), 0, st, p);
+  }
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
 TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, const void* q,
                                 const void* q_imp_producer, void* out, void* stream) {
   tb_status s = check_layer(ctx, layer);
@@ -664,11 +778,17 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   }
   if (c.variant == TB_BUTLER || c.variant == TB_BUTLER_GROUP) {
     const bool grouped = c.variant == TB_BUTLER_GROUP;
-    s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st);
+    const LayerState& ls = ctx->layers[layer];
+    const bool cached = ls.sc_q != nullptr && ctx->reuse_interval > 0;
+    if (cached) {
+      s = launch_reuse_decide(ctx, layer, q_imp_producer, st);
+      if (s != TB_OK) return s;
+    }
+    s = launch_score(ctx, layer, q_imp_producer, ctx->scores, ctx->hist, st, cached ? ctx->reuse : nullptr);
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
     s = launch_select(ctx, layer, ctx->scores, true, grouped ? c.n_kv_heads : c.n_q_heads, nullptr, 0, nullptr,
-                      ctx->mask, st);
+                      ctx->mask, st, cached);
     if (s != TB_OK) return s;
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, ctx->mask, grouped ? TB_MASK_GROUP : TB_MASK_PER_HEAD, out, nullptr, st);

@@ -29,7 +29,8 @@ STATUS_NAMES = {0: "TB_OK", 1: "TB_ERR_INVALID_ARG", 2: "TB_ERR_SHAPE", 3: "TB_E
 EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "tb_get_seq_lens", "tb_set_budget",
            "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
            "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
-           "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait")
+           "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait", "tb_selection_cache_size",
+           "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks")
 
 
 class TBError(RuntimeError):
@@ -85,6 +86,10 @@ def lib():
             "tb_status_string": [i32],
             "tb_destroy": [vp],
             "tb_selftest_bounded_wait": [vp, ctypes.c_longlong, i32, vp],
+            "tb_selection_cache_size": [P(Config), P(sz)],
+            "tb_bind_selection_cache": [vp, i32, vp, sz],
+            "tb_set_reuse": [vp, ctypes.c_float, i32, i32],
+            "tb_copy_step_masks": [vp, vp, sz, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -220,6 +225,29 @@ class Context:
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().tb_trace_events(self._h, arr, len(events)), "tb_trace_events")
         self._trace = events
+
+    def selection_cache(self, layer: int):
+        """Allocate (zero-filled) and bind layer `layer`'s selection cache;
+        returns the tensor, which must stay alive while bound."""
+        n = ctypes.c_size_t(0)
+        _check(lib().tb_selection_cache_size(ctypes.byref(self.cfg), ctypes.byref(n)), "tb_selection_cache_size")
+        buf = torch.zeros(n.value + 256, dtype=torch.uint8, device=self.device)
+        off = (-buf.data_ptr()) % 256
+        view = buf[off:off + n.value]
+        _check(lib().tb_bind_selection_cache(self._h, layer, ctypes.c_void_p(view.data_ptr()), n.value),
+               "tb_bind_selection_cache")
+        self._keep[("selection_cache", layer)] = buf
+        return view
+
+    def step_masks(self, rows: int, stream=None):
+        """The last sparse decode step's selection masks, [B][rows][max_len/32] int32."""
+        out = torch.zeros((self.cfg.batch, rows, self.cfg.max_len // 32), dtype=torch.int32, device=self.device)
+        _check(lib().tb_copy_step_masks(self._h, ctypes.c_void_p(out.data_ptr()), out.numel() * 4, _stream(stream)),
+               "tb_copy_step_masks")
+        return out
+
+    def set_reuse(self, tau: float, interval: int, radius: int = 0) -> None:
+        _check(lib().tb_set_reuse(self._h, ctypes.c_float(tau), interval, radius), "tb_set_reuse")
 
     def selftest_bounded_wait(self, cycles: int, arrive: bool, stream=None) -> None:
         """Launch the bounded-wait self-test (see include/tb.h); read the

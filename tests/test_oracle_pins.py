@@ -418,3 +418,35 @@ def test_group_selection_shares_one_set_per_group_and_equals_per_head_for_equal_
     sel_h, _, _, _ = O.decode_layer(q, K, V, W, qi_same, 1, G, L, 30, 4, 16, dense=False)
     for h in range(Hq):
         assert np.array_equal(sel_g[0, h], sel_h[0, h])
+
+
+# --------------------------------------------------------------------------- amortised selection (R18)
+def test_reuse_decision_rules():
+    q = np.array([1.0, 0.0, 0.0])
+    near = np.array([1.0, 0.1, 0.0])            # cos 0.995
+    far = np.array([0.0, 1.0, 0.0])             # cos 0
+    args = dict(interval=4, tau=0.9, keep_pct=30, sink=4, window=16)
+    assert O.reuse_decision(q, near, 200, 198, **args)
+    assert not O.reuse_decision(q, far, 200, 198, **args)
+    assert not O.reuse_decision(q, near, 200, 195, **args)          # older than the interval
+    assert not O.reuse_decision(q, near, 200, 0, **args)            # empty cache
+    assert not O.reuse_decision(q, near, 15, 14, **args)            # no top-k at this length
+    assert not O.reuse_decision(np.zeros(3), near, 200, 198, **args)
+    assert O.reuse_decision(q, q, 200, 200, **args)                 # same step, same query
+    assert not O.reuse_decision(q, near, 200, 198, **dict(args, keep_pct=100))  # 100 %: all candidates
+
+
+def test_reused_set_keeps_cached_topk_window_and_sink_with_neighbours():
+    sink, window = 2, 4
+    len0, L = 40, 42
+    topk = np.array([5, 9, 20, 33])               # 33 = len0 - window - 3, still a candidate then
+    cached = np.concatenate([np.arange(sink), topk, np.arange(len0 - window, len0)])
+    got = O.reused_set(cached, len0, L, sink, window, radius=0)
+    want = np.concatenate([np.arange(sink), topk, np.arange(L - window, L)])
+    assert np.array_equal(got, want)
+    # cached window tokens (36..39) are not top-k: only 38, 39 stay, as window of L = 42
+    got2 = O.reused_set(cached, len0, L, sink, window, radius=2)
+    want2 = sorted(set(range(sink)) | {3, 4, 5, 6, 7, 8, 9, 10, 11, 18, 19, 20, 21, 22, 31, 32, 33, 34, 35}
+                   | set(range(L - window, L)))
+    assert np.array_equal(got2, np.array(want2))
+    assert got2.min() >= 0 and got2.max() < L
