@@ -46,6 +46,12 @@ def parse():
     ap.add_argument("--keep", type=int, default=30)
     ap.add_argument("--variant", choices=["butler", "group"], default="butler",
                     help="per-head selection (the pages' method, default) or the per-KV-group option")
+    ap.add_argument("--reuse", default=None, metavar="TAU,INTERVAL,RADIUS",
+                    help="amortised selection: reuse a row's cached top-k when cos >= TAU and it is at most "
+                         "INTERVAL tokens old, widened by RADIUS neighbours; the step then advances the length by "
+                         "one token per decode step and the importance queries drift (see --drift)")
+    ap.add_argument("--drift", type=float, default=0.05,
+                    help="with --reuse: importance query of step s = q(0) + DRIFT * noise(s)")
     ap.add_argument("--trace-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -66,6 +72,8 @@ def workload(args):
         wl = wl.with_(name=f"decode{wl.n_layers}_bf16_B{wl.B}_L{wl.L}_keep{wl.keep_pct}")
     if getattr(args, "variant", "butler") == "group":
         wl = wl.with_(name=wl.name + "_group_select")
+    if getattr(args, "reuse", None):
+        wl = wl.with_(name=wl.name + f"_reuse{args.reuse.replace(',', '_')}_drift{args.drift:g}")
     return wl
 
 
@@ -225,9 +233,11 @@ def build(wl, max_len, dev, variant=None):
     return ctx, bufs, proj
 
 
-def step_inputs_host(wl, s):
+def step_inputs_host(wl, s, drift=None):
     """Pinned host tensors of step s: k_new, v_new [layers][B][Hkv][D],
-    q [layers][B][Hq][D], q_imp [producers][(B*Hq)][G][1][d']."""
+    q [layers][B][Hq][D], q_imp [producers][(B*Hq)][G][1][d'].  With `drift`,
+    q_imp of step s is q_imp(0) + drift * noise(s) (bf16), so consecutive
+    steps' importance queries stay close."""
     import torch
     from query_aware_sparse_decode_b200 import synth as S
 
@@ -240,11 +250,18 @@ def step_inputs_host(wl, s):
         vn.append(v)
         qq.append(S.query(wl, layer, s))
     nprod = (wl.n_layers + wl.G - 1) // wl.G
-    qi = [S.q_imp(wl, p * wl.G, s) for p in range(nprod)]
+    if drift is None:
+        qi = [S.q_imp(wl, p * wl.G, s) for p in range(nprod)]
+    else:
+        qi = [S.f32_to_bf16_bits((S.widen(S.q_imp(wl, p * wl.G, 0), "bf16") +
+                                  drift * S.widen(S.q_imp(wl, p * wl.G, 1000 + s), "bf16")).astype(np.float32))
+              for p in range(nprod)]
     return t(np.stack(kn)), t(np.stack(vn)), t(np.stack(qq)), t(np.stack(qi))
 
 
 def run_step(ctx, wl, L0, inp, out, stream=None):
+    """One decode step of every layer at length L0 + 1 (the new token goes to
+    position L0)."""
     kn, vn, qq, qi = inp
     for layer in range(wl.n_layers):
         ctx.set_seq_lens(layer, [L0] * wl.B)
@@ -296,7 +313,25 @@ def gpu_arm(args, rank, world, local_rank):
     ctx, bufs, proj = build(wl, max_len, dev, variant_code(args))
     stream = torch.cuda.current_stream(dev)
     nvar = min(args.steps + args.warmup, 4)
-    host_inputs = [step_inputs_host(wl, s) for s in range(nvar)]
+    drift = None
+    if args.reuse:  # amortised selection: caches bound, queries drifting, the length advancing
+        tau, interval, radius = args.reuse.split(",")
+        for layer in range(wl.n_layers):
+            ctx.selection_cache(layer)
+        ctx.set_reuse(float(tau), int(interval), int(radius))
+        drift = args.drift
+    host_inputs = [step_inputs_host(wl, s, drift) for s in range(nvar)]
+    pos = {"n": 0}
+
+    def next_L0():
+        """Position of the step's new token: fixed, or advancing by one per
+        step when selections are cached (max_len leaves 255 tokens of room)."""
+        if not args.reuse:
+            return L0
+        pos["n"] += 1
+        if pos["n"] >= max_len - wl.L:
+            raise RuntimeError("--reuse runs out of cache room: use fewer steps")
+        return L0 + pos["n"]
     dev_inputs = [tuple(x.to(dev) for x in h) for h in host_inputs]
     out = torch.empty((wl.n_layers, wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
     scored, attended = step_counts(wl)
@@ -311,7 +346,7 @@ def gpu_arm(args, rank, world, local_rank):
         return max_over_ranks_of(x, world, dev)
 
     for s in range(args.warmup):
-        run_step(ctx, wl, L0, dev_inputs[s % nvar], out, stream)
+        run_step(ctx, wl, next_L0(), dev_inputs[s % nvar], out, stream)
     barrier()
 
     # ---- device-timed region: inputs resident in HBM
@@ -326,7 +361,7 @@ def gpu_arm(args, rank, world, local_rank):
     barrier()
     e0.record(stream)
     for s in range(args.steps):
-        run_step(ctx, wl, L0, dev_inputs[s % nvar], out, stream)
+        run_step(ctx, wl, next_L0(), dev_inputs[s % nvar], out, stream)
     e1.record(stream)
     barrier()
     clk = clocks.stop()
@@ -340,9 +375,10 @@ def gpu_arm(args, rank, world, local_rank):
     seg = {"append": [], "score": [], "select": [], "attn": [], "combine": [], "attn_dense": []}
     kn, vn, qq, qi = dev_inputs[0]
     for s in range(args.trace_steps):
+        Ls = next_L0()
         for layer in range(wl.n_layers):
             ctx.trace_events(ev[layer])
-            ctx.set_seq_lens(layer, [L0] * wl.B)
+            ctx.set_seq_lens(layer, [Ls] * wl.B)
             ctx.decode_step(layer, kn[layer], vn[layer], qq[layer], qi[layer // wl.G], out[layer], stream)
         ctx.trace_events(None)
         torch.cuda.synchronize(dev)
@@ -390,7 +426,7 @@ def gpu_arm(args, rank, world, local_rank):
         for s in range(args.steps):
             for dst, src in zip(dbuf, host_inputs[s % nvar]):
                 dst.copy_(src, non_blocking=True)
-            run_step(ctx, wl, L0, dbuf, out, stream)
+            run_step(ctx, wl, next_L0(), dbuf, out, stream)
             out_host.copy_(out, non_blocking=True)
         f1.record(stream)
         barrier()
@@ -687,6 +723,10 @@ def main():
                        "D": wl.D, "d_imp": wl.d_imp, "G": wl.G, "L": wl.L, "keep_pct": wl.keep_pct,
                        "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
                        "selection": "per_kv_group" if args.variant == "group" else "per_query_head",
+                       "reuse": (None if not args.reuse else
+                                 {"tau,interval,radius": args.reuse, "drift": args.drift,
+                                  "note": "the length advances one token per step; scored and attended "
+                                          "counts are those of a fresh step at L"}),
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (caches of all layers, no flush)"},
             "us_per_layer": r["ms_step"] * 1e3 / wl.n_layers,
