@@ -137,6 +137,21 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
 TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
                                const void* w_k);
 
+/* Paged K/V caches (serving layouts; SURVEY's next row on page-table gathers).
+ * Register layer `layer` with K and V page pools [num_pages][Hkv][page_size][D]
+ * (kv_dtype) and a device page table `page_table` [B][max_pages] int32: token
+ * t of sequence b, KV head g, is row t % page_size of page
+ * page_table[b][t / page_size].  page_size: a power of two >= 16;
+ * max_pages * page_size >= max_len; num_pages * Hkv * page_size < 2^31.  The
+ * table is read by the kernels, so the caller may remap pages between calls
+ * (stream-ordered).  K_imp stays a dense per-sequence cache as above.  Every
+ * call works on paged layers; the K_imp projection of paged bf16 caches uses
+ * fp32 FMA instead of the tensor cores (a TMA tile may not cross pages).
+ * Lengths start at 0. */
+TB_API tb_status tb_bind_layer_paged(tb_ctx* ctx, int layer, void* k_pool, void* v_pool, int num_pages,
+                                     const int32_t* page_table, int page_size, int max_pages, float* kimp_cache,
+                                     const void* w_k);
+
 /* Set / read the per-sequence lengths of a layer (host arrays of `batch`
  * int32).  Used after the caller filled the caches by a prefill. */
 TB_API tb_status tb_set_seq_lens(tb_ctx* ctx, int layer, const int32_t* lens_host);

@@ -27,8 +27,9 @@ constexpr int kAttnTile = 16;        // tokens per mma tile
 constexpr int kAttnMaxChunk = 2048;  // tokens per gather list (a CTA's chunk may span several)
 
 struct AttnParams {
-  const void* k_cache;   // [B][Hkv][max_len][D]
+  const void* k_cache;   // [B][Hkv][max_len][D], or a page pool (KvLayout)
   const void* v_cache;
+  KvLayout kl;
   const void* q;         // [B][Hq][D]
   const uint32_t* mask;  // per mask_mode
   float* part_o;         // [B][Hq][nsplit][D]
@@ -40,8 +41,9 @@ struct AttnParams {
   int lens[kMaxBatch];
 };
 
-// Builds the CTA's gather list: ascending union tokens of [t0, t1) with a
-// head bitmask each; pads to a multiple of 16 with (t0, no head).
+// Builds the CTA's gather list: the cache rows of the ascending union tokens
+// of [t0, t1) with a head bitmask each; pads to a multiple of 16 with
+// (row of t0, no head).
 template <int GS>
 __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int g, int t0, int t1, int32_t* list_idx,
                                                 uint8_t* list_hb, uint32_t* scan_sm) {
@@ -83,7 +85,7 @@ __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int 
 #pragma unroll
         for (int hh = 0; hh < GS; ++hh) hb |= ((hm[hh] >> j) & 1u) << hh;
       }
-      list_idx[pos] = t0 + 32 * w + j;
+      list_idx[pos] = (int32_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, t0 + 32 * w + j);  // the token's cache row
       list_hb[pos] = (uint8_t)hb;
       ++pos;
     }
@@ -91,7 +93,7 @@ __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int 
   }
   const int padded = (base + kAttnTile - 1) / kAttnTile * kAttnTile;
   for (int i = base + tid; i < padded; i += kAttnThreads) {
-    list_idx[i] = t0;
+    list_idx[i] = (int32_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, t0);
     list_hb[i] = 0;
   }
   __syncthreads();
@@ -161,8 +163,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 2, tq = lane & 3;
-  const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.max_len * ROWB;
-  const uint8_t* Vb = reinterpret_cast<const uint8_t*>(p.v_cache) + ((size_t)b * p.Hkv + g) * p.max_len * ROWB;
+  // gather lists hold cache rows (dense or paged), so the bases are the caches'
+  const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache);
+  const uint8_t* Vb = reinterpret_cast<const uint8_t*>(p.v_cache);
 
   // A fragments of Q (rows = the group's heads; rows >= GS and 8..15 are 0).
   // Logical k (2tq + {0,1}) of k-step kk maps to dims (4(kk/2)+tq)*8 + (kk%2)*4 + {0,1},
@@ -342,8 +345,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_f32_kernel(const AttnParams
   if (t0 >= L) return;
   const int t1 = min(t0 + p.chunk, L);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* Kb = reinterpret_cast<const float*>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.max_len * D;
-  const float* Vb = reinterpret_cast<const float*>(p.v_cache) + ((size_t)b * p.Hkv + g) * p.max_len * D;
+  const float* Kb = reinterpret_cast<const float*>(p.k_cache);  // list entries are cache rows
+  const float* Vb = reinterpret_cast<const float*>(p.v_cache);
   float q[GS][DPL], o[GS][DPL], m[GS], l[GS];
 #pragma unroll
   for (int hh = 0; hh < GS; ++hh) {

@@ -24,6 +24,23 @@ __host__ __device__ __forceinline__ size_t kimp_index(size_t slab, int j, int t,
 }
 constexpr float kNegInf = -__builtin_huge_valf();
 
+// ------------------------------------------------------------ K/V row layout
+// Dense caches: slab (b, g) is rows [(b*Hkv + g)*max_len, ... + max_len) of
+// [B][Hkv][max_len][D].  Paged caches: a pool [pages][Hkv][page_size][D] and
+// a page table [B][max_pages] of page ids; token t of (b, g) is row
+// (page_table[b][t / page_size]*Hkv + g)*page_size + t % page_size of the
+// pool (page_size a power of two).  Rows are counted in units of D elements.
+struct KvLayout {
+  const int32_t* page_table;  // null: dense
+  int page_size, page_shift, max_pages;
+};
+__device__ __forceinline__ uint32_t kv_row(const KvLayout& kl, int b, int g, int Hkv, int max_len, int t) {
+  if (kl.page_table == nullptr) return ((uint32_t)b * Hkv + g) * (uint32_t)max_len + (uint32_t)t;
+  const int page = kl.page_table[(size_t)b * kl.max_pages + (t >> kl.page_shift)];
+  return ((uint32_t)page * Hkv + g) * (uint32_t)kl.page_size + (uint32_t)(t & (kl.page_size - 1));
+}
+
+
 // ------------------------------------------------------------ order keys
 // Monotone map of fp32 onto uint32 (larger score -> larger key); -0.0 is
 // folded onto +0.0 first so that the two compare equal.

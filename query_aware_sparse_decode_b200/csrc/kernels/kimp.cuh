@@ -16,6 +16,7 @@ struct AppendParams {
   float* kimp;        // [B][Hkv][max_len/256][d'][256] (kimp_index)
   const void* w_k;    // [D][d']
   int Hkv, D, dimp, max_len;
+  KvLayout kl;         // dense or paged K/V caches
   int pos[kMaxBatch];  // row written for sequence b (its length before the append)
 };
 
@@ -34,7 +35,7 @@ __device__ __forceinline__ void append_row(const AppendParams& p, int g, int b, 
   float* part = krow + 128;          // [128]
   const int tid = threadIdx.x, nt = blockDim.x;
   const size_t src = ((size_t)b * p.Hkv + g) * p.D;
-  const size_t row = ((size_t)b * p.Hkv + g) * p.max_len + p.pos[b];
+  const size_t row = kv_row(p.kl, b, g, p.Hkv, p.max_len, p.pos[b]);
   const T* W = reinterpret_cast<const T*>(p.w_k);
   const int nw = p.D * p.dimp;
   constexpr int VEC = 16 / (int)sizeof(T);  // W_K staged with 16-byte loads, all in flight
@@ -83,10 +84,11 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
 }
 
 struct ProjectParams {
-  const void* k_cache;  // [B][Hkv][max_len][D]
+  const void* k_cache;  // [B][Hkv][max_len][D], or a page pool (KvLayout)
   float* kimp;          // [B][Hkv][max_len/256][d'][256] (kimp_index)
   const void* w_k;      // [D][d']
   int Hkv, max_len, start, count;
+  KvLayout kl;
 };
 
 // fp32-FMA projection of rows [start, start+count) of every (b, g).
@@ -98,16 +100,18 @@ __global__ void __launch_bounds__(256) project_fma_kernel(const ProjectParams p)
   constexpr int OUT_PER_THREAD = ROWS * DIMP / 256;  // 4 (d'=32) or 2 (d'=16)
   __shared__ float ks[ROWS][D + 1];
   __shared__ float ws[D][DIMP];
+  __shared__ uint32_t krow[ROWS];  // cache rows of the block's tokens
   const int g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int r0 = p.start + blockIdx.x * ROWS;
-  const size_t base = ((size_t)b * p.Hkv + g) * p.max_len;
   const T* K = reinterpret_cast<const T*>(p.k_cache);
   const T* W = reinterpret_cast<const T*>(p.w_k);
   for (int i = tid; i < D * DIMP; i += 256) ws[i / DIMP][i % DIMP] = to_f32(W[i]);
   const int rend = min(ROWS, p.start + p.count - r0);
+  if (tid < ROWS) krow[tid] = tid < rend ? kv_row(p.kl, b, g, p.Hkv, p.max_len, r0 + tid) : 0u;
+  __syncthreads();
   for (int i = tid; i < ROWS * D; i += 256) {
     const int r = i / D, d = i % D;
-    ks[r][d] = r < rend ? to_f32(K[(base + r0 + r) * D + d]) : 0.f;
+    ks[r][d] = r < rend ? to_f32(K[(size_t)krow[r] * D + d]) : 0.f;
   }
   __syncthreads();
   const int r = tid / (256 / ROWS);                          // 8 threads per row

@@ -29,7 +29,8 @@ namespace tb {
 constexpr int kVoteChunk = 2048;  // tokens per CTA of the logits pass
 
 struct VoteParams {
-  const void* k_cache;  // [B][Hkv][max_len][D] bf16
+  const void* k_cache;  // [B][Hkv][max_len][D] bf16, or a page pool (KvLayout)
+  KvLayout kl;
   const void* q;        // [B][Hq][D] bf16
   float* logits;        // [B][Hq][max_len], log2 domain
   float* stats;         // [B][Hq][nchunk][2]
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   const int n = t1 - t0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 2, tq = lane & 3;
-  const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.max_len * ROWB;
+  const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache);  // rows via kv_row
 
   uint32_t qa[KSTEPS][2];
   {
@@ -82,7 +83,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     for (int c = lane; c < kAttnTile * NCH; c += 32) {
       const int row = c / NCH, part = c % NCH;
       const int tok = min(t0 + tile * kAttnTile + row, t1 - 1);  // clamp the ragged tail
-      cp_async_16(sb + row * ROWB + ((part ^ (row & 7)) << 4), Kb + (size_t)tok * ROWB + part * 16);
+      cp_async_16(sb + row * ROWB + ((part ^ (row & 7)) << 4),
+                  Kb + (size_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, tok) * ROWB + part * 16);
     }
   };
 #pragma unroll

@@ -33,6 +33,7 @@ struct LayerState {
   bool bound = false;
   CUtensorMap k_map;  // bf16 caches: K rows, 64-column boxes of 128 rows, 128B swizzle
   int lens[TB_MAX_BATCH];
+  KvLayout kl{};       // dense (page_table null) or paged K/V caches
   // selection cache (amortised selection), caller-owned, or null
   float* sc_q = nullptr;        // [B*rows][d'] importance query of the cached set
   int32_t* sc_len = nullptr;    // [B*rows] length at which it was selected (0: empty)
@@ -307,6 +308,7 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   AttnParams p{};
   p.k_cache = ls.k;
   p.v_cache = ls.v;
+  p.kl = ls.kl;
   p.q = q;
   p.mask = mask;
   p.part_o = ctx->part_o;
@@ -391,6 +393,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   const int gs = c.n_q_heads / c.n_kv_heads;
   VoteParams p{};
   p.k_cache = ls.k;
+  p.kl = ls.kl;
   p.q = q;
   p.logits = ctx->scores;
   p.stats = ctx->vstats;
@@ -500,6 +503,30 @@ TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_ca
   ls.v = v_cache;
   ls.kimp = kimp_cache;
   ls.wk = w_k;
+  ls.kl = KvLayout{};
+  std::memset(ls.lens, 0, sizeof(ls.lens));
+  ls.bound = true;
+  return TB_OK;
+}
+
+TB_API tb_status tb_bind_layer_paged(tb_ctx* ctx, int layer, void* k_pool, void* v_pool, int num_pages,
+                                     const int32_t* page_table, int page_size, int max_pages, float* kimp_cache,
+                                     const void* w_k) {
+  if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
+  if (!k_pool || !v_pool || !page_table || !kimp_cache || !w_k) return TB_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(kimp_cache) || !aligned16(w_k)) return TB_ERR_SHAPE;
+  const tb_config& c = ctx->cfg;
+  if (page_size < 16 || (page_size & (page_size - 1)) != 0 || num_pages < 1 || max_pages < 1) return TB_ERR_SHAPE;
+  if ((long long)max_pages * page_size < c.max_len) return TB_ERR_SHAPE;
+  if ((long long)num_pages * c.n_kv_heads * page_size >= (1LL << 31)) return TB_ERR_SHAPE;
+  LayerState& ls = ctx->layers[layer];
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  ls.k = k_pool;
+  ls.v = v_pool;
+  ls.kimp = kimp_cache;
+  ls.wk = w_k;
+  ls.kl = KvLayout{page_table, page_size, shift, max_pages};
   std::memset(ls.lens, 0, sizeof(ls.lens));
   ls.bound = true;
   return TB_OK;
@@ -609,6 +636,7 @@ static tb_status append_params(const tb_ctx* ctx, int layer, const void* k_new, 
   p->v_cache = ls.v;
   p->kimp = ls.kimp;
   p->w_k = ls.wk;
+  p->kl = ls.kl;
   p->Hkv = c.n_kv_heads;
   p->D = c.head_dim;
   p->dimp = c.d_imp;
@@ -646,7 +674,7 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
   if (count == 0) return TB_OK;
   const LayerState& ls = ctx->layers[layer];
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (c.kv_dtype == TB_BF16) {
+  if (c.kv_dtype == TB_BF16 && ls.kl.page_table == nullptr) {
     ProjectTcParams tp{};
     tp.w_k = ls.wk;
     tp.kimp = ls.kimp;
@@ -669,12 +697,18 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
     ++ctx->launches;
     return cuda_status(cudaGetLastError());
   }
-  ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count};
+  // fp32 caches, and paged caches of either type (a TMA tile may not cross pages): fp32 FMA
+  ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count, ls.kl};
   dim3 grid((count + kProjRows - 1) / kProjRows, c.n_kv_heads, c.batch);
 #define TB_PROJ_CASE(T, DV, DI) \
   if (c.head_dim == DV && c.d_imp == DI) project_fma_kernel<T, DV, DI><<<grid, 256, 0, st>>>(p); else
-  TB_PROJ_CASE(float, 128, 32) TB_PROJ_CASE(float, 128, 16) TB_PROJ_CASE(float, 64, 32)
-  TB_PROJ_CASE(float, 64, 16) return TB_ERR_UNSUPPORTED;
+  if (c.kv_dtype == TB_BF16) {
+    TB_PROJ_CASE(__nv_bfloat16, 128, 32) TB_PROJ_CASE(__nv_bfloat16, 128, 16) TB_PROJ_CASE(__nv_bfloat16, 64, 32)
+    TB_PROJ_CASE(__nv_bfloat16, 64, 16) return TB_ERR_UNSUPPORTED;
+  } else {
+    TB_PROJ_CASE(float, 128, 32) TB_PROJ_CASE(float, 128, 16) TB_PROJ_CASE(float, 64, 32)
+    TB_PROJ_CASE(float, 64, 16) return TB_ERR_UNSUPPORTED;
+  }
 #undef TB_PROJ_CASE
   ++ctx->launches;
   return cuda_status(cudaGetLastError());

@@ -30,7 +30,7 @@ EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "
            "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
            "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
            "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait", "tb_selection_cache_size",
-           "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks")
+           "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks", "tb_bind_layer_paged")
 
 
 class TBError(RuntimeError):
@@ -90,6 +90,7 @@ def lib():
             "tb_bind_selection_cache": [vp, i32, vp, sz],
             "tb_set_reuse": [vp, ctypes.c_float, i32, i32],
             "tb_copy_step_masks": [vp, vp, sz, vp],
+            "tb_bind_layer_paged": [vp, i32, vp, vp, i32, vp, i32, i32, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -225,6 +226,14 @@ class Context:
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().tb_trace_events(self._h, arr, len(events)), "tb_trace_events")
         self._trace = events
+
+    def bind_layer_paged(self, layer, k_pool, v_pool, page_table, kimp_cache, w_k) -> None:
+        """k_pool, v_pool: [pages][Hkv][page_size][D]; page_table: [B][max_pages] int32 (device)."""
+        num_pages, _, page_size, _ = k_pool.shape
+        max_pages = page_table.shape[1]
+        _check(lib().tb_bind_layer_paged(self._h, layer, _ptr(k_pool), _ptr(v_pool), num_pages, _ptr(page_table),
+                                         page_size, max_pages, _ptr(kimp_cache), _ptr(w_k)), "tb_bind_layer_paged")
+        self._keep[layer] = (k_pool, v_pool, page_table, kimp_cache, w_k)
 
     def selection_cache(self, layer: int):
         """Allocate (zero-filled) and bind layer `layer`'s selection cache;
