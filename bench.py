@@ -50,6 +50,9 @@ def parse():
                     help="amortised selection: reuse a row's cached top-k when cos >= TAU and it is at most "
                          "INTERVAL tokens old, widened by RADIUS neighbours; the step then advances the length by "
                          "one token per decode step and the importance queries drift (see --drift)")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="paged K/V caches: pages of this many tokens (a power of two >= 16) placed in a shuffled "
+                         "pool, addressed through a page table; 0 (default) keeps dense caches")
     ap.add_argument("--drift", type=float, default=0.05,
                     help="with --reuse: importance query of step s = q(0) + DRIFT * noise(s)")
     ap.add_argument("--trace-steps", type=int, default=3)
@@ -74,7 +77,34 @@ def workload(args):
         wl = wl.with_(name=wl.name + "_group_select")
     if getattr(args, "reuse", None):
         wl = wl.with_(name=wl.name + f"_reuse{args.reuse.replace(',', '_')}_drift{args.drift:g}")
+    if getattr(args, "page_size", 0):
+        wl = wl.with_(name=wl.name + f"_paged{args.page_size}")
     return wl
+
+
+def page_caches(ctx, wl, bufs, page, max_len, dev):
+    """Re-bind every layer with its K/V rows moved into a pool of shuffled
+    pages and a page table (K_imp and W_K stay as they are)."""
+    import torch
+    npg = max_len // page
+    g = torch.Generator(device="cpu").manual_seed(1234)
+    for layer, (k, v, kimp, w) in enumerate(bufs):
+        perm = torch.randperm(wl.B * npg, generator=g)
+        pools = []
+        for x in (k, v):
+            staged = x.view(wl.B, wl.Hkv, npg, page, wl.D).permute(0, 2, 1, 3, 4).reshape(wl.B * npg, wl.Hkv, page,
+                                                                                         wl.D)
+            pool = torch.empty_like(staged)
+            pool[perm.to(dev)] = staged
+            del staged
+            pools.append(pool)
+        table = perm.view(wl.B, npg).to(torch.int32).to(dev)
+        lens = ctx.seq_lens(layer)
+        ctx.bind_layer_paged(layer, pools[0], pools[1], table, kimp, w)
+        ctx.set_seq_lens(layer, lens)
+        bufs[layer] = (pools[0], pools[1], kimp, w, table)
+        del k, v
+    torch.cuda.empty_cache()
 
 
 def variant_code(args):
@@ -155,7 +185,7 @@ class ClockSampler:
 # from one ncu capture of it (B = 2, L = 131072, keep 30 %; summary under
 # profiles/).  Valid only for the kernel source it was measured on; any
 # change makes it null.
-ATTN_TRAFFIC = {"source_sha256_16": "81ae913471f38008", "bytes_per_union_row": (811.698176e6 + 4.206336e6) / 1581259}
+ATTN_TRAFFIC = {"source_sha256_16": "12fe4df7a7e9e7e7", "bytes_per_union_row": (811.743232e6 + 5.543168e6) / 1581259}
 
 
 def attn_traffic_per_row():
@@ -311,6 +341,10 @@ def gpu_arm(args, rank, world, local_rank):
     if max_len == wl.L:
         max_len += 256
     ctx, bufs, proj = build(wl, max_len, dev, variant_code(args))
+    if args.page_size:
+        if max_len % args.page_size:
+            raise SystemExit("--page-size must divide the cache capacity")
+        page_caches(ctx, wl, bufs, args.page_size, max_len, dev)
     stream = torch.cuda.current_stream(dev)
     nvar = min(args.steps + args.warmup, 4)
     drift = None
@@ -723,6 +757,7 @@ def main():
                        "D": wl.D, "d_imp": wl.d_imp, "G": wl.G, "L": wl.L, "keep_pct": wl.keep_pct,
                        "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
                        "selection": "per_kv_group" if args.variant == "group" else "per_query_head",
+                       "kv_layout": f"paged, {args.page_size}-token pages" if args.page_size else "dense",
                        "reuse": (None if not args.reuse else
                                  {"tau,interval,radius": args.reuse, "drift": args.drift,
                                   "note": "the length advances one token per step; scored and attended "

@@ -137,7 +137,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
 TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
                                const void* w_k);
 
-/* Paged K/V caches (serving layouts; SURVEY's next row on page-table gathers).
+/* Paged K/V caches (serving layouts: the attention's page-table gather).
  * Register layer `layer` with K and V page pools [num_pages][Hkv][page_size][D]
  * (kv_dtype) and a device page table `page_table` [B][max_pages] int32: token
  * t of sequence b, KV head g, is row t % page_size of page
