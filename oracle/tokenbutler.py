@@ -50,6 +50,10 @@ group selects once with the same budget, sink, window and tie rules; every
 head of the group then attends over that set (group_scores, decode_layer
 with group=True).
 
+Option beyond the sources: a bf16 K_imp cache (round_to_bf16,
+project_keys with storage="bf16"): K_imp is rounded once, from its exact
+value, to the nearest bfloat16 (ties to even) and scored as stored.
+
 Parity pins (tests/test_oracle_pins.py) cover every function here; the
 readings R4, R6, R13 and R14 are consistent with the sources but not fixed
 by them (parity unpinned against the pages for those readings).
@@ -100,10 +104,24 @@ def keep_pct_from_policy(policy: str) -> int:
 
 
 # ------------------------------------------------------------------ a1: K_imp
-def project_keys(K: np.ndarray, W_K: np.ndarray) -> np.ndarray:
+def project_keys(K: np.ndarray, W_K: np.ndarray, storage: str = "f64") -> np.ndarray:
     """[MC] Method: K_imp = K . W_K on the post-RoPE cached keys (fp64, no
-    rounding).  K: [..., D], W_K: [D, d'] (Reading R1)."""
-    return np.asarray(K, dtype=np.float64) @ np.asarray(W_K, dtype=np.float64)
+    rounding).  K: [..., D], W_K: [D, d'] (Reading R1).  storage="bf16": the
+    bf16 K_imp cache option, each exact value rounded once to bfloat16."""
+    kimp = np.asarray(K, dtype=np.float64) @ np.asarray(W_K, dtype=np.float64)
+    return round_to_bf16(kimp) if storage == "bf16" else kimp
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value (8 significant bits, fp32's exponent range),
+    ties to the even significand, returned as float64.  For finite |x| below
+    the largest bfloat16; below 2^-126 the quantum is fixed at 2^-133
+    (subnormal bfloat16)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m * 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                 # subnormal range: fixed quantum 2^-133
+    q = np.ldexp(1.0, e - 8)                # one unit in the 8th significant bit
+    return np.rint(x / q) * q               # np.rint rounds half to even; x / q is exact
 
 
 # ------------------------------------------------------------------ a3: scores
@@ -202,7 +220,7 @@ def reused_set(cached: np.ndarray, len0: int, L: int, sink: int, window: int, ra
 
 # ------------------------------------------------------------------ one decode layer
 def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, dense: bool,
-                 K_imp=None, heads=None, batches=None, group: bool = False):
+                 K_imp=None, heads=None, batches=None, group: bool = False, kimp_storage: str = "f64"):
     """One consumer layer's decode step, [MC] Method in order:
     K_imp = K W_K; consumer slot (l - 1) mod G; score every cached token;
     top-k + sink + window per query head; attention over the selected tokens.
@@ -212,7 +230,8 @@ def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, wind
     q_imp_producer: [(B*Hq)][G][1][d']; L: int or per-sequence list.
     Returns dicts keyed by (b, h): selected indices, output [D], lse; and the
     fp64 scores per (b, h) (None for dense layers).  With group=True (the
-    per-KV-group option) the scores and the set are the head's group's."""
+    per-KV-group option) the scores and the set are the head's group's.
+    kimp_storage="bf16": scores are taken on the bf16-rounded K_imp."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
     Hkv = K.shape[1]
@@ -232,7 +251,7 @@ def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, wind
                 scores[b, h] = None
             else:
                 if g not in kimp_b:
-                    kimp_b[g] = (project_keys(K[b, g, :Lb], W_K) if K_imp is None
+                    kimp_b[g] = (project_keys(K[b, g, :Lb], W_K, kimp_storage) if K_imp is None
                                  else np.asarray(K_imp[b, g, :Lb], dtype=np.float64))
                 if group:
                     gs = Hq // Hkv

@@ -450,3 +450,65 @@ def test_reused_set_keeps_cached_topk_window_and_sink_with_neighbours():
                    | set(range(L - window, L)))
     assert np.array_equal(got2, np.array(want2))
     assert got2.min() >= 0 and got2.max() < L
+
+
+# ------------------------------------------------------------ bf16 K_imp storage
+def test_round_to_bf16_closed_forms():
+    """Nearest bfloat16 with ties to the even significand (8 significant
+    bits: spacing 2^-7 on [1, 2)), rounded once from the exact value."""
+    r = O.round_to_bf16
+    cases = [
+        (1.0 + 2.0 ** -8, 1.0),                          # tie between 1 and 1 + 2^-7: even is 1
+        (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),          # tie between 1 + 2^-7 (odd) and 1 + 2^-6 (even)
+        (1.0 + 2.0 ** -8 + 2.0 ** -40, 1.0 + 2.0 ** -7),  # just above the tie: one rounding, not two
+        (-(1.0 + 2.0 ** -8), -1.0),                      # sign-symmetric
+        (255.5, 256.0),                                  # 255.5 is a tie on [128, 256): 255 odd -> 256
+        (254.5, 254.0),                                  # tie: 254 even
+        (3.0 * 2.0 ** 100, 3.0 * 2.0 ** 100),            # representable values are kept
+        (1.3 * 2.0 ** -130, 10 * 2.0 ** -133),           # subnormal: quantum 2^-133
+    ]
+    for x, want in cases:
+        assert r(np.array(x)) == want, x
+    z = r(np.array([0.0, -0.0]))
+    assert z[0] == 0 and not np.signbit(z[0]) and np.signbit(z[1])
+
+
+def test_round_to_bf16_equals_library_cast_on_fp32_values():
+    """On values an fp32 holds exactly, rounding once equals the library's
+    round-to-nearest-even fp32 -> bf16 conversion."""
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(200000) * 10.0 ** rng.integers(-30, 30, 200000),
+                        np.float32(1.0) + np.arange(-4096, 4096) * np.float32(2.0 ** -23)]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_to_bf16(x.astype(np.float64)), want)
+
+
+def test_bf16_storage_rounds_the_sum_not_the_terms():
+    """K = [1, 2^-8], W_K = [[1], [1]]: the exact K_imp 1 + 2^-8 is a tie and
+    stores as 1.0; rounding each term (or none) would give 1 + 2^-8."""
+    K = np.array([[1.0, 2.0 ** -8]])
+    W = np.array([[1.0], [1.0]])
+    assert O.project_keys(K, W)[0, 0] == 1.0 + 2.0 ** -8
+    assert O.project_keys(K, W, "bf16")[0, 0] == 1.0
+    K2 = np.array([[1.0, 2.0 ** -8 + 2.0 ** -30]])
+    assert O.project_keys(K2, W, "bf16")[0, 0] == 1.0 + 2.0 ** -7
+
+
+def test_bf16_storage_decides_the_selection_in_decode_layer():
+    """Two candidates whose exact scores differ by less than half a bf16 step
+    tie after storage, and the tie goes to the lower index (R8): the stored
+    precision must reach the selection."""
+    B, Hq, Hkv, D, dimp, G = 1, 1, 1, 2, 1, 1
+    W = np.array([[1.0], [0.0]])
+    K = np.zeros((B, Hkv, 2, D))
+    K[0, 0, 0, 0] = 1.0
+    K[0, 0, 1, 0] = 1.0 + 2.0 ** -9
+    V = np.arange(B * Hkv * 2 * D, dtype=np.float64).reshape(B, Hkv, 2, D)
+    q = np.ones((B, Hq, D))
+    qimp = np.ones((B * Hq, G, 1, dimp))
+    args = (q, K, V, W, qimp, 1, G, 2, 50, 0, 0)
+    sel64, *_ = O.decode_layer(*args, dense=False)
+    sel16, out16, _, sc16 = O.decode_layer(*args, dense=False, kimp_storage="bf16")
+    assert sel64[0, 0].tolist() == [1]
+    assert sel16[0, 0].tolist() == [0] and sc16[0, 0].tolist() == [1.0, 1.0]
+    assert np.array_equal(out16[0, 0], V[0, 0, 0])
