@@ -50,6 +50,8 @@ def parse():
                     help="amortised selection: reuse a row's cached top-k when cos >= TAU and it is at most "
                          "INTERVAL tokens old, widened by RADIUS neighbours; the step then advances the length by "
                          "one token per decode step and the importance queries drift (see --drift)")
+    ap.add_argument("--kimp", choices=["f32", "bf16"], default="f32",
+                    help="K_imp cache precision: fp32 (default) or the bf16 option (half the score stream)")
     ap.add_argument("--page-size", type=int, default=0,
                     help="paged K/V caches: pages of this many tokens (a power of two >= 16) placed in a shuffled "
                          "pool, addressed through a page table; 0 (default) keeps dense caches")
@@ -79,6 +81,8 @@ def workload(args):
         wl = wl.with_(name=wl.name + f"_reuse{args.reuse.replace(',', '_')}_drift{args.drift:g}")
     if getattr(args, "page_size", 0):
         wl = wl.with_(name=wl.name + f"_paged{args.page_size}")
+    if getattr(args, "kimp", "f32") == "bf16":
+        wl = wl.with_(name=wl.name + "_kimpbf16")
     return wl
 
 
@@ -214,20 +218,25 @@ def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: flo
 
 
 # ----------------------------------------------------------------------- GPU arm
-def build(wl, max_len, dev, variant=None):
+def kimp_elem_bytes(cfg) -> int:
+    """Bytes of one K_imp element: fp32, or bf16 with the bf16 K_imp option."""
+    return 2 if cfg.kimp_bf16 else 4
+
+
+def build(wl, max_len, dev, variant=None, kimp_dtype="f32"):
     import torch
     from query_aware_sparse_decode_b200 import synth as S
     from query_aware_sparse_decode_b200 import tb as TB
     cfg = TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G, max_len, wl.dtype, wl.keep_pct,
                          wl.sink, wl.window, dense_layers=wl.dense_layers,
-                         variant=TB.TB_BUTLER if variant is None else variant)
+                         variant=TB.TB_BUTLER if variant is None else variant, kimp_dtype=kimp_dtype)
     ctx = TB.Context(cfg, dev)
     L0 = wl.L - 1
     bufs = []
     for layer in range(wl.n_layers):
         k = torch.empty((wl.B, wl.Hkv, max_len, wl.D), dtype=torch.bfloat16, device=dev)
         v = torch.empty_like(k)
-        kimp = torch.empty((wl.B, wl.Hkv, max_len // 256, wl.d_imp, 256), dtype=torch.float32, device=dev)
+        kimp = TB.kimp_cache(cfg, dev)
         w_raw = S.w_k(wl, layer)
         w = torch.from_numpy(w_raw.view(np.int16)).view(torch.bfloat16).to(dev)
         delta = None
@@ -256,7 +265,7 @@ def build(wl, max_len, dev, variant=None):
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / wl.n_layers
     rows = wl.B * wl.Hkv * L0
-    nbytes = rows * (wl.D * 2 + wl.d_imp * 4)
+    nbytes = rows * (wl.D * 2 + wl.d_imp * kimp_elem_bytes(cfg))
     proj = {"kernel": "butler_kimp_project (tcgen05, prefill of the cache)", "us_per_layer": us,
             "rows_per_layer": rows, "bytes_per_layer": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
             "tflops": 2 * rows * wl.D * wl.d_imp / (us * 1e-6) / 1e12}
@@ -340,7 +349,7 @@ def gpu_arm(args, rank, world, local_rank):
     max_len = (wl.L + 255) // 256 * 256
     if max_len == wl.L:
         max_len += 256
-    ctx, bufs, proj = build(wl, max_len, dev, variant_code(args))
+    ctx, bufs, proj = build(wl, max_len, dev, variant_code(args), args.kimp)
     if args.page_size:
         if max_len % args.page_size:
             raise SystemExit("--page-size must divide the cache capacity")
@@ -433,7 +442,7 @@ def gpu_arm(args, rank, world, local_rank):
     urows = union_rows(ctx, wl, L0, dev_inputs[0])
     sparse_layers = [l for l in range(wl.n_layers) if l not in wl.dense_layers]
     row_kv = 2 * wl.D * 2                                   # K + V row, bf16
-    kimp_bytes = wl.B * wl.Hkv * wl.L * wl.d_imp * 4         # per sparse layer
+    kimp_bytes = wl.B * wl.Hkv * wl.L * wl.d_imp * kimp_elem_bytes(ctx.cfg)   # per sparse layer
     union_bytes = (sum(urows.values()) / max(len(urows), 1)) * row_kv
     dense_bytes = wl.B * wl.Hkv * wl.L * row_kv
     step_bytes = len(sparse_layers) * (kimp_bytes + union_bytes) + (wl.n_layers - len(sparse_layers)) * dense_bytes
@@ -478,7 +487,7 @@ def gpu_arm(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------- CPU oracle leg
-def oracle_sample(wl, seconds: float, group: bool = False):
+def oracle_sample(wl, seconds: float, group: bool = False, kimp: str = "f32"):
     """Times the fp64 oracle on whole (layer, sequence) slabs of the workload
     (score, select, attend for all query heads; inputs regenerated on the host
     and excluded from the timing) until about `seconds` of oracle work."""
@@ -505,7 +514,7 @@ def oracle_sample(wl, seconds: float, group: bool = False):
         kn, vn = S.kv_new(wl, layer, 0)
         K = np.concatenate([K, S.widen(kn, wl.dtype)[b][:, None]], axis=1)[None]
         V = np.concatenate([V, S.widen(vn, wl.dtype)[b][:, None]], axis=1)[None]
-        Kimp = O.project_keys(K, W)
+        Kimp = O.project_keys(K, W, "bf16" if kimp == "bf16" else "f64")
         q = S.widen(S.query(wl, layer, 0), wl.dtype)[b:b + 1]
         qi_b = qi.reshape(wl.B, wl.Hq, wl.G, 1, wl.d_imp)[b]
         t0 = time.perf_counter()
@@ -527,7 +536,7 @@ def reference_arm(args, rank, world):
     wl = workload(args)
     vals = []
     for s in range(args.warmup + args.steps):
-        r = oracle_sample(wl, seconds=0.0, group=args.variant == "group")  # one slab per step
+        r = oracle_sample(wl, seconds=0.0, group=args.variant == "group", kimp=args.kimp)  # one slab per step
         if s >= args.warmup:
             vals.append(r)
     value = statistics.mean(v["value"] for v in vals)
@@ -623,7 +632,7 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
             u = m[:, :, 0]
             for j in range(1, gs):
                 u = u | m[:, :, j]
-        first = wl.B * wl.Hkv * wl.L * wl.d_imp * 4           # K_imp
+        first = wl.B * wl.Hkv * wl.L * wl.d_imp * kimp_elem_bytes(ctx.cfg)   # K_imp
         union = int(np.unpackbits(u.cpu().numpy().view(np.uint8)).sum())
     torch.cuda.synchronize()
     if ctx.check_status():
@@ -744,7 +753,7 @@ def main():
     r = gpu_arm(args, rank, world, local_rank)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(r["wl"], args.cpu_seconds, group=args.variant == "group")
+        cpu = oracle_sample(r["wl"], args.cpu_seconds, group=args.variant == "group", kimp=args.kimp)
     if rank == 0:
         wl = r["wl"]
         avg = r["avg"]
@@ -758,6 +767,7 @@ def main():
                        "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
                        "selection": "per_kv_group" if args.variant == "group" else "per_query_head",
                        "kv_layout": f"paged, {args.page_size}-token pages" if args.page_size else "dense",
+                       "kimp_cache": args.kimp,
                        "reuse": (None if not args.reuse else
                                  {"tau,interval,radius": args.reuse, "drift": args.drift,
                                   "note": "the length advances one token per step; scored and attended "

@@ -33,9 +33,10 @@
  *     after a synchronisation.  Nothing aborts, traps or throws.
  *   - Layouts are dense and row-major (last index fastest):
  *       K cache, V cache   [B][Hkv][max_len][D]   kv_dtype
- *       K_imp cache        [B][Hkv][max_len/256][d'][256]  fp32 (always): tiles of
- *                          256 tokens, each contiguous and dimension-major
- *                          (element (b, g, t, j) at tile t/256, row j, column t%256)
+ *       K_imp cache        [B][Hkv][max_len/256][d'][256]  fp32, or bf16 when
+ *                          cfg.kimp_bf16 = 1: tiles of 256 tokens, each
+ *                          contiguous and dimension-major (element (b, g, t, j)
+ *                          at tile t/256, row j, column t%256)
  *       W_K                [D][d']                kv_dtype
  *       q_imp (producer)   [(B*Hq)][G][n][d']     kv_dtype  (model card: (B.H) x G x L x d')
  *       q, out             [B][Hq][D]             kv_dtype
@@ -119,6 +120,11 @@ typedef struct tb_config {
   int window;                /* sliding_window: always-kept recent tokens                 */
   uint64_t dense_layer_mask; /* bit l set: layer l attends densely (layer 0 by default)   */
   int variant;               /* tb_variant                                                */
+  int kimp_bf16;             /* 0: fp32 K_imp cache (default); 1: bf16 K_imp cache, every
+                                K_imp value computed in fp32 and rounded to nearest even
+                                (halves the score stream; kv_dtype TB_BF16 only, else
+                                TB_ERR_UNSUPPORTED).  Option beyond the pages, which do not
+                                state the cache's precision                               */
 } tb_config;
 
 typedef struct tb_ctx tb_ctx;
@@ -134,7 +140,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
 
 /* Register layer `layer`'s caller-owned caches and W_K (device pointers,
  * layouts above).  All lengths of the layer start at 0. */
-TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
+TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, void* kimp_cache,
                                const void* w_k);
 
 /* Paged K/V caches (serving layouts: the attention's page-table gather).
@@ -149,7 +155,7 @@ TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_ca
  * fp32 FMA instead of the tensor cores (a TMA tile may not cross pages).
  * Lengths start at 0. */
 TB_API tb_status tb_bind_layer_paged(tb_ctx* ctx, int layer, void* k_pool, void* v_pool, int num_pages,
-                                     const int32_t* page_table, int page_size, int max_pages, float* kimp_cache,
+                                     const int32_t* page_table, int page_size, int max_pages, void* kimp_cache,
                                      const void* w_k);
 
 /* Set / read the per-sequence lengths of a layer (host arrays of `batch`
@@ -163,19 +169,20 @@ TB_API tb_status tb_set_budget(tb_ctx* ctx, int keep_pct, int sink, int window);
 
 /* a1 — model card "Method", K_imp = K . W_K, decode side.  Writes k_new and
  * v_new ([B][Hkv][D]) at position len[b] of every sequence, computes that
- * row's K_imp in fp32, then increments len[b] (host-side bookkeeping at
+ * row's K_imp in fp32 (stored in the cache's type), then increments len[b] (host-side bookkeeping at
  * enqueue time).  TB_ERR_CAPACITY if a sequence is full. */
 TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, void* stream);
 
 /* a1' — model card "Method", K_imp = K . W_K, prefill side: computes K_imp
  * rows [start, start + count) of every (b, KV head) from the cached K.
  * bf16 caches run on the tensor cores (tcgen05, fp32 accumulation); fp32
- * caches use fp32 FMA (no TF32). */
+ * caches use fp32 FMA (no TF32).  A bf16 K_imp cache receives each fp32
+ * result rounded to nearest even. */
 TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, void* stream);
 
 /* a2 + a3 — model card "Method": scores[b][h][t] = q_hat[b][h] . K_imp[b][g(h)][t]
  * for t < len[b], with q_hat[b][h] = q_imp_producer[b*Hq + h][(layer-1) mod G][0][:]
- * (fp32 FMA, no scale).  `q_imp_producer`: [(B*Hq)][G][1][d'] of producer
+ * (fp32 FMA on the stored K_imp values, no scale).  `q_imp_producer`: [(B*Hq)][G][1][d'] of producer
  * G*floor(layer/G).  Entries t >= len[b] are left untouched.  With
  * TB_BUTLER_GROUP the rows are per KV group instead ([B][Hkv][max_len]):
  * scores[b][g][t] = sum over the group's heads, in head order, of the fp32
@@ -221,9 +228,10 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
  * (layer-1) mod G.  `row_masks`: [B][Hq][nrows][words_per_row] uint32 with
  * words_per_row >= ceil((row0 + nrows)/32); every word is written.
  * Requires len[b] >= row0 + nrows (K_imp rows present).  Rows are scored in
- * blocks of 16 on the tensor cores (TF32 with K_imp split into a TF32 head
+ * blocks of 16 on the tensor cores (TF32 with an fp32 K_imp split into a TF32 head
  * and its remainder, fp32 accumulation: about 1e-6 relative to the fp32 dot
- * product); rows with massive ties are redone with fp32 FMA scores.  Always
+ * product; a bf16 K_imp is exact in TF32 and needs no split); rows with
+ * massive ties are redone with fp32 FMA scores.  Always
  * one selection per query head. */
 TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_rows, int row0, int nrows,
                                    uint32_t* row_masks, int words_per_row, void* stream);

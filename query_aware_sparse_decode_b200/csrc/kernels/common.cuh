@@ -74,6 +74,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// K_imp cache elements: fp32, or bf16 (the fp32 value rounded to nearest,
+// ties to even) when the context stores K_imp in bf16.
+__device__ __forceinline__ void store_kimp(void* base, size_t i, float v, bool bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(base)[i] = v;
+}
+
 // ------------------------------------------------------------ mma.sync
 // D(16x8, f32) += A(16x16, bf16, row) * B(16x8, bf16, col)
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -1,5 +1,7 @@
 // butler_kimp_project, CUDA-core parts: the fused decode append (new K/V row
 // + its K_imp row) and the fp32-FMA prefill projection used for fp32 caches.
+// K_imp is computed in fp32 and stored as fp32, or rounded to bf16 when the
+// context keeps a bf16 K_imp cache.
 // Model card "Meta-Llama-3.1-8B-Instruct-Butler", section "Method":
 // K_imp = K . W_K with one learned D x d' matrix per layer.
 #pragma once
@@ -13,9 +15,10 @@ struct AppendParams {
   const void* v_new;  // [B][Hkv][D]
   void* k_cache;      // [B][Hkv][max_len][D]
   void* v_cache;
-  float* kimp;        // [B][Hkv][max_len/256][d'][256] (kimp_index)
+  void* kimp;         // [B][Hkv][max_len/256][d'][256] (kimp_index), fp32 or bf16
   const void* w_k;    // [D][d']
   int Hkv, D, dimp, max_len;
+  int kimp_bf16;       // K_imp elements are bf16
   KvLayout kl;         // dense or paged K/V caches
   int pos[kMaxBatch];  // row written for sequence b (its length before the append)
 };
@@ -70,7 +73,7 @@ __device__ __forceinline__ void append_row(const AppendParams& p, int g, int b, 
     const int parts = 128 / p.dimp;
     float sum = 0.f;
     for (int i = 0; i < parts; ++i) sum += part[i * p.dimp + tid];
-    p.kimp[kimp_index((size_t)b * p.Hkv + g, tid, p.pos[b], p.dimp, p.max_len)] = sum;
+    store_kimp(p.kimp, kimp_index((size_t)b * p.Hkv + g, tid, p.pos[b], p.dimp, p.max_len), sum, p.kimp_bf16);
   }
 }
 
@@ -85,10 +88,11 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
 
 struct ProjectParams {
   const void* k_cache;  // [B][Hkv][max_len][D], or a page pool (KvLayout)
-  float* kimp;          // [B][Hkv][max_len/256][d'][256] (kimp_index)
+  void* kimp;           // [B][Hkv][max_len/256][d'][256] (kimp_index), fp32 or bf16
   const void* w_k;      // [D][d']
   int Hkv, max_len, start, count;
   KvLayout kl;
+  int kimp_bf16;
 };
 
 // fp32-FMA projection of rows [start, start+count) of every (b, g).
@@ -127,7 +131,8 @@ __global__ void __launch_bounds__(256) project_fma_kernel(const ProjectParams p)
   if (r < rend) {
     const size_t slab = (size_t)b * p.Hkv + g;
 #pragma unroll
-    for (int j = 0; j < OUT_PER_THREAD; ++j) p.kimp[kimp_index(slab, j0 + j, r0 + r, DIMP, p.max_len)] = acc[j];
+    for (int j = 0; j < OUT_PER_THREAD; ++j)
+      store_kimp(p.kimp, kimp_index(slab, j0 + j, r0 + r, DIMP, p.max_len), acc[j], p.kimp_bf16);
   }
 }
 

@@ -35,7 +35,7 @@ constexpr int kPfSmem = kPfRows * kHistBins * 4;
 
 struct PrefillParams {
   const void* q_imp;   // [(B*Hq)][G][nrows][d'] kv dtype
-  const float* kimp;   // [B][Hkv][max_len/256][d'][256] (kimp_index)
+  const void* kimp;    // [B][Hkv][max_len/256][d'][256] (kimp_index), KT elements
   uint32_t* masks;     // [B][Hq][nrows][words_per_row]
   uint32_t* status;
   uint32_t* redo;      // [B][Hq][nrows]: 1 where the blocked kernel left the row to the one-row method
@@ -48,7 +48,7 @@ struct PrefillParams {
 // largest order key is found by three radix digits, and an ordered sweep
 // writes the row's mask words (ties at the threshold go to the lowest
 // indices through a block scan).
-template <typename TQ, int DIMP>
+template <typename TQ, typename KT, int DIMP>
 __device__ void prefill_one_row(const PrefillParams& p, int b, int h, int r, float* srow, uint32_t* hist,
                                 uint32_t* scan_sm, int* s_bin_p, uint32_t* s_above_p, float* q) {
   int& s_bin = *s_bin_p;
@@ -63,10 +63,10 @@ __device__ void prefill_one_row(const PrefillParams& p, int b, int h, int r, flo
   __syncthreads();
   const size_t slab = (size_t)b * p.Hkv + g;
   for (int t = tid; t < L; t += kSelThreads) {
-    const float* K = p.kimp + kimp_index(slab, 0, t, DIMP, p.max_len);
+    const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t, DIMP, p.max_len);
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < DIMP; ++j) acc = fmaf(q[j], K[j * kKimpTile], acc);
+    for (int j = 0; j < DIMP; ++j) acc = fmaf(q[j], to_f32(K[j * kKimpTile]), acc);
     srow[t] = acc;
   }
   __syncthreads();
@@ -148,7 +148,7 @@ __device__ void prefill_one_row(const PrefillParams& p, int b, int h, int r, flo
 // flags of its rows (strided by gridDim.x) in one parallel load, then runs the
 // one-row method on the flagged ones.  Dynamic smem: `need` floats of row
 // scores.
-template <typename TQ, int DIMP>
+template <typename TQ, typename KT, int DIMP>
 __global__ void __launch_bounds__(kSelThreads, 1) prefill_redo_kernel(const PrefillParams p) {
   extern __shared__ float srow[];
   __shared__ uint32_t hist[kHistBins];
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) prefill_redo_kernel(const Pref
     const int n = n_todo;
     for (int j = 0; j < n; ++j) {
       const int hr = todo[j];
-      prefill_one_row<TQ, DIMP>(p, b, hr / p.nrows, hr % p.nrows, srow, hist, scan_sm, &s_bin, &s_above, q);
+      prefill_one_row<TQ, KT, DIMP>(p, b, hr / p.nrows, hr % p.nrows, srow, hist, scan_sm, &s_bin, &s_above, q);
     }
     __syncthreads();
   }
@@ -206,10 +206,11 @@ __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)
 // tiles: a warp takes 32 tokens at a time (four n-tiles of 8; one mask word
 // per row), and lane (g, c) = (lane / 4, lane % 4) holds the scores of rows g
 // and g + 8 for tokens 2c and 2c + 1 of each n-tile.
-template <typename TQ, int DIMP>
+template <typename TQ, typename KT, int DIMP>
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const PrefillParams p) {
   constexpr int KS = DIMP / 8;                        // k-steps of 8 dimensions
   constexpr bool QSPLIT = sizeof(TQ) == 4;            // fp32 queries need hi + lo too
+  constexpr bool KBF16 = sizeof(KT) == 2;             // bf16 K_imp: exact in TF32
   extern __shared__ __align__(16) uint32_t pf_smem[];  // hist[16][2048]; in pass 3 the key lists
   __shared__ int rmode[kPfRows], rk[kPfRows];
   __shared__ uint32_t rb1[kPfRows], rk1[kPfRows], rb2[kPfRows], rk2[kPfRows], rn2[kPfRows], rcnt[kPfRows];
@@ -285,17 +286,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
       sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
       const int t = t0 + 8 * n + gq;  // the B column this lane loads
       const bool ok = t < Lmax;
-      const float* K = p.kimp + kimp_index(slab, 0, ok ? t : 0, DIMP, p.max_len);
+      const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, ok ? t : 0, DIMP, p.max_len);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        const float k0 = ok ? K[(ks * 8 + cq) * kKimpTile] : 0.f;
-        const float k1 = ok ? K[(ks * 8 + cq + 4) * kKimpTile] : 0.f;
+        const float k0 = ok ? to_f32(K[(ks * 8 + cq) * kKimpTile]) : 0.f;
+        const float k1 = ok ? to_f32(K[(ks * 8 + cq + 4) * kKimpTile]) : 0.f;
         // hi: the value cut to TF32 width; lo: the exact fp32 remainder, of
-        // which the tensor core reads the TF32-width head
+        // which the tensor core reads the TF32-width head.  A bf16 K_imp has
+        // 8 significant bits, so it is exact in TF32 and has no remainder.
         const uint32_t h0 = __float_as_uint(k0) & 0xFFFFE000u, h1 = __float_as_uint(k1) & 0xFFFFE000u;
-        const uint32_t l0 = __float_as_uint(k0 - __uint_as_float(h0)), l1 = __float_as_uint(k1 - __uint_as_float(h1));
         mma_tf32_1688(sc[n], afr[ks], h0, h1);
-        mma_tf32_1688(sc[n], afr[ks], l0, l1);
+        if (!KBF16) {
+          const uint32_t l0 = __float_as_uint(k0 - __uint_as_float(h0));
+          const uint32_t l1 = __float_as_uint(k1 - __uint_as_float(h1));
+          mma_tf32_1688(sc[n], afr[ks], l0, l1);
+        }
         if (QSPLIT) mma_tf32_1688(sc[n], afl[ks], h0, h1);
       }
     }

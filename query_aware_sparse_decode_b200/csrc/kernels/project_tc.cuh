@@ -28,10 +28,11 @@ constexpr int kTcThreads = 192;
 
 struct ProjectTcParams {
   const void* w_k;  // [D][d'] bf16
-  float* kimp;      // [B][Hkv][max_len/256][d'][256] (kimp_index)
+  void* kimp;       // [B][Hkv][max_len/256][d'][256] (kimp_index), fp32 or bf16
   uint32_t* status;
   int max_len, start, count;
   int tiles_per_slab, total_tiles;
+  int kimp_bf16;    // store K_imp rounded to bf16
 };
 
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
@@ -246,9 +247,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int r = quarter * 32 + lane;
       if (r < valid) {
         // for each column the warp writes 32 consecutive tokens of one tile
-        float* dst = p.kimp + kimp_index(slab, 0, t0 + r, DIMP, p.max_len);
+        const size_t dst = kimp_index(slab, 0, t0 + r, DIMP, p.max_len);
+        if (p.kimp_bf16) {
+          __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(p.kimp) + dst;
 #pragma unroll
-        for (int c = 0; c < DIMP; ++c) dst[c * kKimpTile] = v[c];
+          for (int c = 0; c < DIMP; ++c) k16[c * kKimpTile] = __float2bfloat16_rn(v[c]);
+        } else {
+          float* k32 = reinterpret_cast<float*>(p.kimp) + dst;
+#pragma unroll
+          for (int c = 0; c < DIMP; ++c) k32[c * kKimpTile] = v[c];
+        }
       }
     }
   }

@@ -5,12 +5,13 @@
 //
 // HBM stream over K_imp, stored as contiguous 256-token tiles, dimension-major
 // inside a tile ([b][g][t/256][j][t%256], see kimp_index), read once per KV head
-// and shared by the Hq/Hkv query heads of the group.  A thread scores four
-// consecutive tokens: d' independent, coalesced 16-byte loads per group of
-// four tokens, written as batches of 16 loads ahead of their FMAs (fp32,
-// dimension order j = 0..d'-1, the group's query values broadcast from
-// shared memory) so that many loads per thread can be in flight.  A CTA covers 1, 2 or 4 groups of
-// 1024 tokens (the launch picks the count so the grid fills the SMs).
+// and shared by the Hq/Hkv query heads of the group.  A thread scores the
+// consecutive tokens of one 16-byte load per dimension (four fp32 or eight
+// bf16 K_imp values): d' independent, coalesced loads, written as batches of
+// up to 16 loads ahead of their FMAs (fp32, dimension order j = 0..d'-1, the
+// group's query values broadcast from shared memory) so that many loads per
+// thread can be in flight.  A CTA covers 1, 2 or 4 steps of 256 threads' tokens
+// (the launch picks the count so the grid fills the SMs).
 // With GROUPED (one selection per KV group) the group's per-head fp32 scores
 // are added in head order and one row per (b, g) is written instead.
 // Optionally each CTA accumulates, per output row, the histogram of the
@@ -23,31 +24,51 @@
 namespace tb {
 
 constexpr int kScoreThreads = 256;
-constexpr int kScoreStep = kScoreThreads * 4;   // tokens per CTA iteration (4 per thread)
-constexpr int kScoreLoadBatch = 16;             // float4 loads issued before their FMAs
+constexpr int kScoreLoadBatch = 16;  // 16-byte loads issued before their FMAs
+// tokens per CTA iteration: one 16-byte load of KT elements per thread and dimension
+template <typename KT>
+constexpr int score_step() { return kScoreThreads * (16 / (int)sizeof(KT)); }
 
 struct ScoreParams {
   const void* q_imp;   // [(B*Hq)][G][1][d'] of the producer, kv dtype
-  const float* kimp;   // [B][Hkv][max_len/256][d'][256]
+  const void* kimp;    // [B][Hkv][max_len/256][d'][256], KT elements
   float* scores;       // [B][Hq][max_len]
   uint32_t* hist;      // [B*Hq][2048] or nullptr
   int G, slot, Hq, Hkv, max_len;
   int sink, window;
-  int iters;           // CTA iterations of kScoreStep tokens (1, 2 or 4)
+  int iters;           // CTA iterations of score_step<KT>() tokens (1, 2 or 4)
   const uint32_t* reuse;  // [B*rows] amortised selection: rows that skip scoring, or null
   int lens[kMaxBatch];
 };
 
-template <typename T, int DIMP, int GS, bool HIST, bool GROUPED = false>
+// The 16 bytes of one load as fp32 values (bf16 widened exactly).
+__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[4]) {
+  x[0] = __uint_as_float(v.x);
+  x[1] = __uint_as_float(v.y);
+  x[2] = __uint_as_float(v.z);
+  x[3] = __uint_as_float(v.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <typename T, typename KT, int DIMP, int GS, bool HIST, bool GROUPED = false>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScoreParams p) {
   constexpr int NR = GROUPED ? 1 : GS;  // output rows per (b, g): per head, or the group's sum
+  constexpr int TPT = 16 / (int)sizeof(KT);  // tokens per thread and step
+  constexpr int STEP = score_step<KT>();
   pdl_wait();
   pdl_trigger();
   __shared__ __align__(16) float qs[DIMP][GS];
   extern __shared__ uint32_t hist[];  // [NR][2048] when HIST
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.lens[b];
-  const int t_base = chunk * kScoreStep * p.iters;
+  const int t_base = chunk * STEP * p.iters;
   if (t_base >= L) return;
   if (p.reuse != nullptr) {  // every row of this group reuses its cached selection: nothing to score
     const size_t r0 = GROUPED ? (size_t)b * p.Hkv + g : (size_t)b * p.Hq + g * GS;
@@ -68,36 +89,40 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   const size_t slab = (size_t)b * p.Hkv + g;
   const size_t row0 = GROUPED ? (size_t)b * p.Hkv + g : (size_t)b * p.Hq + g * GS;  // first output row
   float* S = p.scores + row0 * p.max_len;
-  static_assert(DIMP % kScoreLoadBatch == 0 || DIMP < kScoreLoadBatch, "d' must be a multiple of the batch");
-  constexpr int NB = DIMP < kScoreLoadBatch ? DIMP : kScoreLoadBatch;
+  // loads in flight per batch: 16, or 8 when the accumulators are many
+  constexpr int NB0 = GS * TPT > 32 ? kScoreLoadBatch / 2 : kScoreLoadBatch;
+  static_assert(DIMP % NB0 == 0 || DIMP < NB0, "d' must be a multiple of the batch");
+  constexpr int NB = DIMP < NB0 ? DIMP : NB0;
 #pragma unroll 1
   for (int it = 0; it < p.iters; ++it) {
-    const int t0 = t_base + it * kScoreStep + 4 * tid;
+    const int t0 = t_base + it * STEP + TPT * tid;
     if (t0 < L) {
-      const float* K = p.kimp + kimp_index(slab, 0, t0, DIMP, p.max_len);
-      float acc[GS][4];
+      const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t0, DIMP, p.max_len);
+      float acc[GS][TPT];
 #pragma unroll
-      for (int hh = 0; hh < GS; ++hh) acc[hh][0] = acc[hh][1] = acc[hh][2] = acc[hh][3] = 0.f;
+      for (int hh = 0; hh < GS; ++hh)
+#pragma unroll
+        for (int u = 0; u < TPT; ++u) acc[hh][u] = 0.f;
 #pragma unroll
       for (int j0 = 0; j0 < DIMP; j0 += NB) {
-        float4 v[NB];
+        uint4 v[NB];
 #pragma unroll
-        for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const float4*>(K + (j0 + jj) * kKimpTile));
+        for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const uint4*>(K + (j0 + jj) * kKimpTile));
 #pragma unroll
         for (int jj = 0; jj < NB; ++jj) {
+          float kv[TPT];
+          unpack16(v[jj], kv);
 #pragma unroll
           for (int hh = 0; hh < GS; ++hh) {
             const float qv = qs[j0 + jj][hh];
-            acc[hh][0] = fmaf(qv, v[jj].x, acc[hh][0]);
-            acc[hh][1] = fmaf(qv, v[jj].y, acc[hh][1]);
-            acc[hh][2] = fmaf(qv, v[jj].z, acc[hh][2]);
-            acc[hh][3] = fmaf(qv, v[jj].w, acc[hh][3]);
+#pragma unroll
+            for (int u = 0; u < TPT; ++u) acc[hh][u] = fmaf(qv, kv[u], acc[hh][u]);
           }
         }
       }
       if (GROUPED) {  // the group's row: per-head fp32 scores added in head order
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < TPT; ++u) {
           float sum = acc[0][u];
 #pragma unroll
           for (int hh = 1; hh < GS; ++hh) sum += acc[hh][u];
@@ -107,16 +132,19 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
 #pragma unroll
       for (int hh = 0; hh < NR; ++hh) {
         float* srow = S + (size_t)hh * p.max_len;
-        if (t0 + 3 < L) {
-          *reinterpret_cast<float4*>(srow + t0) = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
+        if (t0 + TPT - 1 < L) {
+#pragma unroll
+          for (int u = 0; u < TPT; u += 4)
+            *reinterpret_cast<float4*>(srow + t0 + u) =
+                make_float4(acc[hh][u], acc[hh][u + 1], acc[hh][u + 2], acc[hh][u + 3]);
         } else {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
+          for (int u = 0; u < TPT; ++u)
             if (t0 + u < L) srow[t0 + u] = acc[hh][u];
         }
         if (HIST) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < TPT; ++u) {
             const int t = t0 + u;
             if (t >= p.sink && t < L - p.window) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
           }

@@ -28,7 +28,7 @@ namespace {
 struct LayerState {
   void* k = nullptr;
   void* v = nullptr;
-  float* kimp = nullptr;
+  void* kimp = nullptr;  // fp32 or bf16 (cfg.kimp_bf16)
   const void* wk = nullptr;
   bool bound = false;
   CUtensorMap k_map;  // bf16 caches: K rows, 64-column boxes of 128 rows, 128B swizzle
@@ -145,6 +145,8 @@ static tb_status check_config(const tb_config* c) {
   if (c->keep_pct < 0 || c->keep_pct > 100 || c->sink < 0 || c->window < 0) return TB_ERR_INVALID_ARG;
   if (c->variant != TB_BUTLER && c->variant != TB_SOFTVOTE && c->variant != TB_BUTLER_GROUP)
     return TB_ERR_INVALID_ARG;
+  if (c->kimp_bf16 != 0 && c->kimp_bf16 != 1) return TB_ERR_INVALID_ARG;
+  if (c->kimp_bf16 && c->kv_dtype != TB_BF16) return TB_ERR_UNSUPPORTED;
   return TB_OK;
 }
 
@@ -205,41 +207,41 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const size_t smem = hist ? (size_t)(grouped ? 1 : gs) * kHistBins * 4 : 0;
   // the most tokens per CTA (up to 4 steps) that still gives about three
   // CTAs per SM; short or small batches get one step per CTA
+  const int step = c.kimp_bf16 ? score_step<__nv_bfloat16>() : score_step<float>();
   int iters = 4;
-  while (iters > 1 && (long long)c.batch * c.n_kv_heads * ((maxL + kScoreStep * iters - 1) / (kScoreStep * iters)) <
+  while (iters > 1 && (long long)c.batch * c.n_kv_heads * ((maxL + step * iters - 1) / (step * iters)) <
                           3LL * ctx->num_sms)
     iters >>= 1;
   p.iters = iters;
-  const int chunk = kScoreStep * iters;
+  const int chunk = step * iters;
   dim3 grid((maxL + chunk - 1) / chunk, c.n_kv_heads, c.batch);
-#define TB_SCORE_CASE(T, DI, GSV)                                                                    \
+#define TB_SCORE_CASE(T, KT, DI, GSV)                                                                \
   if (c.d_imp == DI && gs == GSV) {                                                                  \
-    auto k = hist ? (grouped ? score_kernel<T, DI, GSV, true, true> : score_kernel<T, DI, GSV, true, false>) \
-                  : (grouped ? score_kernel<T, DI, GSV, false, true> : score_kernel<T, DI, GSV, false, false>); \
+    auto k = hist ? (grouped ? score_kernel<T, KT, DI, GSV, true, true> : score_kernel<T, KT, DI, GSV, true, false>) \
+                  : (grouped ? score_kernel<T, KT, DI, GSV, false, true>                             \
+                             : score_kernel<T, KT, DI, GSV, false, false>);                          \
     if (hist) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
     launch_pdl(k, grid, dim3(kScoreThreads), smem, st, p);                                           \
     ++ctx->launches;                                                                                 \
     return cuda_status(cudaGetLastError());                                                          \
   }
-  if (c.kv_dtype == TB_BF16) {
-    TB_SCORE_CASE(__nv_bfloat16, 32, 4)
-    TB_SCORE_CASE(__nv_bfloat16, 32, 2)
-    TB_SCORE_CASE(__nv_bfloat16, 32, 1)
-    TB_SCORE_CASE(__nv_bfloat16, 32, 8)
-    TB_SCORE_CASE(__nv_bfloat16, 16, 4)
-    TB_SCORE_CASE(__nv_bfloat16, 16, 2)
-    TB_SCORE_CASE(__nv_bfloat16, 16, 1)
-    TB_SCORE_CASE(__nv_bfloat16, 16, 8)
+#define TB_SCORE_CASES(T, KT)                                                                        \
+  TB_SCORE_CASE(T, KT, 32, 4)                                                                        \
+  TB_SCORE_CASE(T, KT, 32, 2)                                                                        \
+  TB_SCORE_CASE(T, KT, 32, 1)                                                                        \
+  TB_SCORE_CASE(T, KT, 32, 8)                                                                        \
+  TB_SCORE_CASE(T, KT, 16, 4)                                                                        \
+  TB_SCORE_CASE(T, KT, 16, 2)                                                                        \
+  TB_SCORE_CASE(T, KT, 16, 1)                                                                        \
+  TB_SCORE_CASE(T, KT, 16, 8)
+  if (c.kv_dtype == TB_BF16 && c.kimp_bf16) {
+    TB_SCORE_CASES(__nv_bfloat16, __nv_bfloat16)
+  } else if (c.kv_dtype == TB_BF16) {
+    TB_SCORE_CASES(__nv_bfloat16, float)
   } else {
-    TB_SCORE_CASE(float, 32, 4)
-    TB_SCORE_CASE(float, 32, 2)
-    TB_SCORE_CASE(float, 32, 1)
-    TB_SCORE_CASE(float, 32, 8)
-    TB_SCORE_CASE(float, 16, 4)
-    TB_SCORE_CASE(float, 16, 2)
-    TB_SCORE_CASE(float, 16, 1)
-    TB_SCORE_CASE(float, 16, 8)
+    TB_SCORE_CASES(float, float)
   }
+#undef TB_SCORE_CASES
 #undef TB_SCORE_CASE
   return TB_ERR_UNSUPPORTED;
 }
@@ -479,7 +481,7 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   return TB_OK;
 }
 
-TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, float* kimp_cache,
+TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_cache, void* kimp_cache,
                                const void* w_k) {
   if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
   if (!k_cache || !v_cache || !kimp_cache || !w_k) return TB_ERR_INVALID_ARG;
@@ -510,7 +512,7 @@ TB_API tb_status tb_bind_layer(tb_ctx* ctx, int layer, void* k_cache, void* v_ca
 }
 
 TB_API tb_status tb_bind_layer_paged(tb_ctx* ctx, int layer, void* k_pool, void* v_pool, int num_pages,
-                                     const int32_t* page_table, int page_size, int max_pages, float* kimp_cache,
+                                     const int32_t* page_table, int page_size, int max_pages, void* kimp_cache,
                                      const void* w_k) {
   if (!ctx || layer < 0 || layer >= ctx->cfg.n_layers) return TB_ERR_INVALID_ARG;
   if (!k_pool || !v_pool || !page_table || !kimp_cache || !w_k) return TB_ERR_INVALID_ARG;
@@ -637,6 +639,7 @@ static tb_status append_params(const tb_ctx* ctx, int layer, const void* k_new, 
   p->kimp = ls.kimp;
   p->w_k = ls.wk;
   p->kl = ls.kl;
+  p->kimp_bf16 = c.kimp_bf16;
   p->Hkv = c.n_kv_heads;
   p->D = c.head_dim;
   p->dimp = c.d_imp;
@@ -684,6 +687,7 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
     tp.count = count;
     tp.tiles_per_slab = (count + kTcRows - 1) / kTcRows;
     tp.total_tiles = tp.tiles_per_slab * c.batch * c.n_kv_heads;
+    tp.kimp_bf16 = c.kimp_bf16;
     const int grid = std::min(tp.total_tiles, ctx->num_sms);
 #define TB_TC_CASE(DV, DI)                                                              \
   if (c.head_dim == DV && c.d_imp == DI) {                                              \
@@ -698,7 +702,7 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
     return cuda_status(cudaGetLastError());
   }
   // fp32 caches, and paged caches of either type (a TMA tile may not cross pages): fp32 FMA
-  ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count, ls.kl};
+  ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count, ls.kl, c.kimp_bf16};
   dim3 grid((count + kProjRows - 1) / kProjRows, c.n_kv_heads, c.batch);
 #define TB_PROJ_CASE(T, DV, DI) \
   if (c.head_dim == DV && c.d_imp == DI) project_fma_kernel<T, DV, DI><<<grid, 256, 0, st>>>(p); else
@@ -876,20 +880,22 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
   dim3 grid((nrows + kPfRows - 1) / kPfRows, c.n_q_heads, c.batch);
   dim3 rgrid((unsigned)std::min<long long>(ctx->num_sms, (long long)c.n_q_heads * nrows), c.batch);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-#define TB_PF_CASE(T, DI)                                                               \
+#define TB_PF_CASE(T, KT, DI)                                                           \
   if (c.d_imp == DI) {                                                                  \
-    auto kb = prefill_rows_kernel<T, DI>;                                               \
+    auto kb = prefill_rows_kernel<T, KT, DI>;                                           \
     cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem);     \
     kb<<<grid, kPfThreads, kPfSmem, st>>>(p);                                           \
-    auto kr = prefill_redo_kernel<T, DI>;                                               \
+    auto kr = prefill_redo_kernel<T, KT, DI>;                                           \
     cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
     kr<<<rgrid, kSelThreads, smem, st>>>(p);                                            \
     ctx->launches += 2;                                                                 \
   } else
-  if (c.kv_dtype == TB_BF16) {
-    TB_PF_CASE(__nv_bfloat16, 32) TB_PF_CASE(__nv_bfloat16, 16) return TB_ERR_UNSUPPORTED;
+  if (c.kv_dtype == TB_BF16 && c.kimp_bf16) {
+    TB_PF_CASE(__nv_bfloat16, __nv_bfloat16, 32) TB_PF_CASE(__nv_bfloat16, __nv_bfloat16, 16) return TB_ERR_UNSUPPORTED;
+  } else if (c.kv_dtype == TB_BF16) {
+    TB_PF_CASE(__nv_bfloat16, float, 32) TB_PF_CASE(__nv_bfloat16, float, 16) return TB_ERR_UNSUPPORTED;
   } else {
-    TB_PF_CASE(float, 32) TB_PF_CASE(float, 16) return TB_ERR_UNSUPPORTED;
+    TB_PF_CASE(float, float, 32) TB_PF_CASE(float, float, 16) return TB_ERR_UNSUPPORTED;
   }
 #undef TB_PF_CASE
   return cuda_status(cudaGetLastError());

@@ -44,7 +44,7 @@ class Config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("d_imp", ctypes.c_int),
                 ("producer_freq", ctypes.c_int), ("max_len", ctypes.c_int), ("kv_dtype", ctypes.c_int),
                 ("keep_pct", ctypes.c_int), ("sink", ctypes.c_int), ("window", ctypes.c_int),
-                ("dense_layer_mask", ctypes.c_uint64), ("variant", ctypes.c_int)]
+                ("dense_layer_mask", ctypes.c_uint64), ("variant", ctypes.c_int), ("kimp_bf16", ctypes.c_int)]
 
 
 class CacheView(ctypes.Structure):
@@ -124,13 +124,23 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 def make_config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, d_imp, producer_freq, max_len, kv_dtype,
-                keep_pct, sink, window, dense_layers=(0,), variant=TB_BUTLER) -> Config:
+                keep_pct, sink, window, dense_layers=(0,), variant=TB_BUTLER, kimp_dtype="f32") -> Config:
+    """kimp_dtype: "f32" (default) or "bf16" (a bf16 K_imp cache; bf16 K/V only)."""
     mask = 0
     for l in dense_layers:
         mask |= 1 << l
+    if kimp_dtype not in ("f32", "bf16"):
+        raise ValueError(f"kimp_dtype must be 'f32' or 'bf16', not {kimp_dtype!r}")
     return Config(n_layers, batch, n_q_heads, n_kv_heads, head_dim, d_imp, producer_freq, max_len,
                   TB_BF16 if kv_dtype in ("bf16", TB_BF16, torch.bfloat16) else TB_F32, keep_pct, sink, window,
-                  mask, variant)
+                  mask, variant, 1 if kimp_dtype == "bf16" else 0)
+
+
+def kimp_cache(cfg: Config, device="cuda", fill=0.0) -> torch.Tensor:
+    """A K_imp cache for `cfg` in the library's layout [B][Hkv][max_len/256][d'][256]
+    (256-token tiles, dimension-major inside), fp32 or bf16 as cfg says."""
+    dt = torch.bfloat16 if cfg.kimp_bf16 else torch.float32
+    return torch.full((cfg.batch, cfg.n_kv_heads, cfg.max_len // 256, cfg.d_imp, 256), fill, dtype=dt, device=device)
 
 
 def workspace_size(cfg: Config) -> int:
@@ -166,7 +176,13 @@ class Context:
         self._keep = {}  # tensors bound to layers stay alive with the context
 
     # -------------------------------------------------------------- setup
+    def _kimp_type_ok(self, kimp_cache) -> None:
+        want = torch.bfloat16 if self.cfg.kimp_bf16 else torch.float32
+        if kimp_cache.dtype != want:
+            raise TypeError(f"K_imp cache must be {want} for this config, got {kimp_cache.dtype}")
+
     def bind_layer(self, layer: int, k_cache, v_cache, kimp_cache, w_k) -> None:
+        self._kimp_type_ok(kimp_cache)
         _check(lib().tb_bind_layer(self._h, layer, _ptr(k_cache), _ptr(v_cache), _ptr(kimp_cache), _ptr(w_k)),
                "tb_bind_layer")
         self._keep[layer] = (k_cache, v_cache, kimp_cache, w_k)
@@ -229,6 +245,7 @@ class Context:
 
     def bind_layer_paged(self, layer, k_pool, v_pool, page_table, kimp_cache, w_k) -> None:
         """k_pool, v_pool: [pages][Hkv][page_size][D]; page_table: [B][max_pages] int32 (device)."""
+        self._kimp_type_ok(kimp_cache)
         num_pages, _, page_size, _ = k_pool.shape
         max_pages = page_table.shape[1]
         _check(lib().tb_bind_layer_paged(self._h, layer, _ptr(k_pool), _ptr(v_pool), num_pages, _ptr(page_table),

@@ -45,11 +45,11 @@ class LayerData:
     q_dev: torch.Tensor
 
 
-def config_of(wl, max_len=None, keep_pct=None, variant=TB.TB_BUTLER) -> TB.Config:
+def config_of(wl, max_len=None, keep_pct=None, variant=TB.TB_BUTLER, kimp_dtype="f32") -> TB.Config:
     return TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G,
                           max_len if max_len is not None else round_up(wl.max_len + 1, 256), wl.dtype,
                           wl.keep_pct if keep_pct is None else keep_pct, wl.sink, wl.window,
-                          dense_layers=wl.dense_layers, variant=variant)
+                          dense_layers=wl.dense_layers, variant=variant, kimp_dtype=kimp_dtype)
 
 
 def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerData:
@@ -73,7 +73,7 @@ def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerDat
     v_cache = torch.zeros_like(k_cache)
     k_cache[:, :, :Lfill] = to_dev(K_raw, wl)
     v_cache[:, :, :Lfill] = to_dev(V_raw, wl)
-    kimp = kimp_alloc(B, Hkv, dimp, Lmax)
+    kimp = TB.kimp_cache(ctx.cfg)
     w_k = to_dev(W_raw, wl)
     ctx.bind_layer(layer, k_cache, v_cache, kimp, w_k)
     ctx.set_seq_lens(layer, lens)
@@ -81,15 +81,61 @@ def make_layer(ctx: TB.Context, wl, layer: int, lens, step: int = 0) -> LayerDat
                      S.widen(V_raw, wl.dtype), k_cache, v_cache, kimp, w_k, to_dev(qimp_raw, wl), to_dev(q_raw, wl))
 
 
-def kimp_alloc(B, Hkv, dimp, Lmax, fill=0.0) -> torch.Tensor:
+def kimp_alloc(B, Hkv, dimp, Lmax, fill=0.0, dtype=torch.float32) -> torch.Tensor:
     """K_imp cache in the library's layout: 256-token tiles, dimension-major inside."""
-    return torch.full((B, Hkv, Lmax // 256, dimp, 256), fill, dtype=torch.float32, device="cuda")
+    return torch.full((B, Hkv, Lmax // 256, dimp, 256), fill, dtype=dtype, device="cuda")
 
 
 def kimp_rows(kimp: torch.Tensor) -> np.ndarray:
-    """[B][Hkv][Lmax][d'] float64 view of a K_imp cache."""
+    """[B][Hkv][Lmax][d'] float64 view of a K_imp cache (fp32 or bf16)."""
     B, Hkv, nt, dimp, _ = kimp.shape
-    return kimp.permute(0, 1, 2, 4, 3).reshape(B, Hkv, nt * 256, dimp).cpu().numpy().astype(np.float64)
+    return kimp.permute(0, 1, 2, 4, 3).reshape(B, Hkv, nt * 256, dimp).float().cpu().numpy().astype(np.float64)
+
+
+KIMP_REL = 8e-6   # fp32 dot-product error bound of a K_imp element, relative to sum_d |K_d W_dj| (D <= 128)
+
+
+def bf16_kimp_bounds(K: np.ndarray, W: np.ndarray):
+    """The bfloat16 values a kernel may store for K_imp = K W: it rounds an
+    fp32 dot product within KIMP_REL * sum|K_d W_dj| of the exact value, and
+    rounding is monotone, so its value lies between the oracle's rounding of
+    the two ends of that interval (equal ends: one possible value)."""
+    x = np.asarray(K, np.float64) @ np.asarray(W, np.float64)
+    tol = KIMP_REL * (np.abs(K) @ np.abs(W)) + 1e-30
+    return O.round_to_bf16(x - tol), O.round_to_bf16(x + tol)
+
+
+def bf16_kimp_ok(got: np.ndarray, K: np.ndarray, W: np.ndarray) -> bool:
+    """A kernel's bf16 K_imp is the oracle's rounding of the exact K W,
+    or, where the fp32 error interval straddles a rounding midpoint, the
+    bfloat16 neighbour on the other side."""
+    lo, hi = bf16_kimp_bounds(K, W)
+    return bool(((got >= lo) & (got <= hi)).all())
+
+
+def bf16_score_slack(qabs: np.ndarray, K: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Per-token bound [L] on how far a score over a kernel's bf16 K_imp may
+    sit from the same score over the oracle's: sum_j |q_j| (hi_j - lo_j).
+    qabs: [d'] absolute importance query (a group's: the sum of |q| over
+    its heads)."""
+    lo, hi = bf16_kimp_bounds(K, W)
+    return (hi - lo) @ np.asarray(qabs, np.float64)
+
+
+def paged_copy(ld, wl, max_len, page, seed):
+    """Pool [pages][Hkv][page][D] holding the dense caches' rows in shuffled
+    pages (plus unused spare pages), and the page table [B][max_len/page]."""
+    per_seq = max_len // page
+    n_pages = wl.B * per_seq + 5
+    perm = np.random.default_rng(seed).permutation(n_pages)[: wl.B * per_seq].reshape(wl.B, per_seq)
+    kpool = torch.zeros((n_pages, wl.Hkv, page, wl.D), dtype=ld.k_cache.dtype, device="cuda")
+    vpool = torch.zeros_like(kpool)
+    for b in range(wl.B):
+        for i in range(per_seq):
+            kpool[perm[b, i]] = ld.k_cache[b, :, i * page:(i + 1) * page]
+            vpool[perm[b, i]] = ld.v_cache[b, :, i * page:(i + 1) * page]
+    table = torch.from_numpy(perm.astype(np.int32)).cuda()
+    return kpool, vpool, table
 
 
 def mask_from_sets(sets: dict, B: int, rows: int, Lmax: int) -> torch.Tensor:
@@ -127,9 +173,10 @@ def assert_close_rows(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = 
     return worst
 
 
-def tie_band_ok(gpu_set, ref_set, scores64, L, keep_pct, sink, window) -> bool:
+def tie_band_ok(gpu_set, ref_set, scores64, L, keep_pct, sink, window, slack=None) -> bool:
     """Selected sets agree except on tokens whose oracle score lies within
-    1e-4 * max|score| of the k-th candidate score."""
+    1e-4 * max|score| of the k-th candidate score (plus, with a bf16 K_imp,
+    the token's own slack and the largest slack: `slack` [L])."""
     g, r = set(np.asarray(gpu_set).tolist()), set(np.asarray(ref_set).tolist())
     if g == r:
         return True
@@ -142,7 +189,10 @@ def tie_band_ok(gpu_set, ref_set, scores64, L, keep_pct, sink, window) -> bool:
     sc = scores64[cand]
     kth = np.sort(sc)[::-1][k - 1]
     band = 1e-4 * np.abs(scores64[:L]).max()
-    return all(abs(scores64[t] - kth) <= band for t in g ^ r)
+    if slack is None:
+        return all(abs(scores64[t] - kth) <= band for t in g ^ r)
+    smax = float(np.max(slack[:L]))
+    return all(abs(scores64[t] - kth) <= band + slack[t] + smax for t in g ^ r)
 
 
 @dataclass
@@ -195,7 +245,7 @@ def make_layer_device(ctx: TB.Context, wl, layer: int, L0: int, step: int = 0) -
     S.fill_device(k, S.K_CACHE, layer, 0, B * Hkv, 0, L0, D, Lmax * D, D, wl.dtype, delta=dd,
                   plant_mod=100 if dd is not None else 0, seed=wl.seed)
     S.fill_device(v, S.V_CACHE, layer, 0, B * Hkv, 0, L0, D, Lmax * D, D, wl.dtype, seed=wl.seed)
-    kimp = kimp_alloc(B, Hkv, dimp, Lmax)
+    kimp = TB.kimp_cache(ctx.cfg)
     ctx.bind_layer(layer, k, v, kimp, to_dev(W_raw, wl))
     ctx.set_seq_lens(layer, [L0] * B)
     ctx.project_kimp(layer, 0, L0)

@@ -9,29 +9,13 @@ import torch
 from query_aware_sparse_decode_b200 import synth as S
 from query_aware_sparse_decode_b200 import tb as TB
 
-from harness import config_of, kimp_alloc, make_layer, sets_from_mask, tdtype, to_dev
+from harness import config_of, kimp_alloc, make_layer, paged_copy, sets_from_mask, tdtype, to_dev
 
 pytestmark = pytest.mark.gpu
 
 WL = S.Workload("paged_bf16", n_layers=1, B=2, Hq=8, Hkv=2, D=128, d_imp=32, G=1, L=3000, dtype="bf16",
                 keep_pct=30, sink=16, window=64, lens=(3000, 1777))
 PAGE = 64
-
-
-def _paged_copy(ld, wl, max_len, page, seed):
-    """Pool [pages][Hkv][page][D] holding the dense caches' rows in shuffled
-    pages (plus unused spare pages), and the page table [B][max_len/page]."""
-    per_seq = max_len // page
-    n_pages = wl.B * per_seq + 5
-    perm = np.random.default_rng(seed).permutation(n_pages)[: wl.B * per_seq].reshape(wl.B, per_seq)
-    kpool = torch.zeros((n_pages, wl.Hkv, page, wl.D), dtype=ld.k_cache.dtype, device="cuda")
-    vpool = torch.zeros_like(kpool)
-    for b in range(wl.B):
-        for i in range(per_seq):
-            kpool[perm[b, i]] = ld.k_cache[b, :, i * page:(i + 1) * page]
-            vpool[perm[b, i]] = ld.v_cache[b, :, i * page:(i + 1) * page]
-    table = torch.from_numpy(perm.astype(np.int32)).cuda()
-    return kpool, vpool, table
 
 
 @pytest.mark.parametrize("variant", [TB.TB_BUTLER, TB.TB_BUTLER_GROUP, TB.TB_SOFTVOTE],
@@ -43,7 +27,7 @@ def test_paged_equals_dense_bit_for_bit(variant):
     lens0 = [L - 1 for L in wl.seq_lens]
     ld = make_layer(dense, wl, 0, lens0)
     paged = TB.Context(cfg)
-    kpool, vpool, table = _paged_copy(ld, wl, cfg.max_len, PAGE, 5)
+    kpool, vpool, table = paged_copy(ld, wl, cfg.max_len, PAGE, 5)
     kimp_p = kimp_alloc(wl.B, wl.Hkv, wl.d_imp, cfg.max_len)
     paged.bind_layer_paged(0, kpool, vpool, table, kimp_p, ld.w_k)
     paged.set_seq_lens(0, lens0)
@@ -82,7 +66,7 @@ def test_paged_attention_and_selection_match_dense_on_identical_kimp():
     ld = make_layer(dense, wl, 0, lens0)
     dense.project_kimp(0, 0, max(lens0))
     paged = TB.Context(cfg)
-    kpool, vpool, table = _paged_copy(ld, wl, cfg.max_len, PAGE, 9)
+    kpool, vpool, table = paged_copy(ld, wl, cfg.max_len, PAGE, 9)
     kimp_p = ld.kimp.clone()
     paged.bind_layer_paged(0, kpool, vpool, table, kimp_p, ld.w_k)
     paged.set_seq_lens(0, lens0)
