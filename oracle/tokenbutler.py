@@ -50,6 +50,13 @@ group selects once with the same budget, sink, window and tie rules; every
 head of the group then attends over that set (group_scores, decode_layer
 with group=True).
 
+  R19 sequence-sharded decode (beyond the sources, which run one device):
+      rank r holds the contiguous tokens [t0_r, t1_r), ranks in token order;
+      the selection is the unsharded one (global budget from the global
+      length, ties at the threshold to the lower index, hence to the lower
+      rank), and the output merges the ranks' attention over their parts of
+      the set by log-sum-exp (merge_partials, decode_layer_sharded).
+
 Option beyond the sources: a bf16 K_imp cache (round_to_bf16,
 project_keys with storage="bf16"): K_imp is rounded once, from its exact
 value, to the nearest bfloat16 (ties to even) and scored as stored.
@@ -263,6 +270,52 @@ def decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, wind
             sel[b, h] = idx
             out[b, h], lse[b, h] = attend(q[b, h], K[b, g, :Lb], V[b, g, :Lb], idx, scale)
     return sel, out, lse, scores
+
+
+# ------------------------------------------------------------------ sequence sharding (R19)
+def merge_partials(outs, lses):
+    """Attention over a set split into disjoint parts, from each part's
+    normalised output o_r and log-sum-exp lse_r: weights exp(lse_r - lse)
+    with lse = log sum_r exp(lse_r).  Parts with lse_r = -inf (empty) carry
+    no weight; when every part is empty the result is a zero output and
+    lse = -inf (as for an empty set)."""
+    lses = np.asarray(lses, dtype=np.float64)
+    outs = np.asarray(outs, dtype=np.float64)
+    if np.all(np.isneginf(lses)):
+        return np.zeros(outs.shape[1:]), -math.inf
+    m = lses[~np.isneginf(lses)].max()
+    w = np.where(np.isneginf(lses), 0.0, np.exp(lses - m))
+    total = w.sum()
+    return (w[:, None] * outs).sum(axis=0) / total, m + math.log(total)
+
+
+def decode_layer_sharded(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, bounds,
+                         group: bool = False, kimp_storage: str = "f64"):
+    """Reading R19: the decode step of one layer with the tokens split over
+    ranks, bounds = [(t0_r, t1_r)] contiguous and in order.  The selected set
+    is the unsharded step's; rank r attends over its part of it and the parts
+    are merged (merge_partials).  Returns (sel, out, lse, parts) with parts
+    {(b, h): [indices of rank r]}."""
+    sel, _, _, _ = decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, dense=False,
+                                group=group, kimp_storage=kimp_storage)
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    lens = [L] * B if np.isscalar(L) else list(L)
+    scale = 1.0 / math.sqrt(D)
+    out, lse, parts = {}, {}, {}
+    for (b, h), idx in sel.items():
+        g = kv_head_of(h, Hq, Hkv)
+        pieces, outs, lses = [], [], []
+        for t0, t1 in bounds:
+            mine = idx[(idx >= t0) & (idx < t1)]
+            o_r, l_r = attend(q[b, h], K[b, g, :lens[b]], V[b, g, :lens[b]], mine, scale)
+            pieces.append(mine)
+            outs.append(o_r)
+            lses.append(l_r)
+        out[b, h], lse[b, h] = merge_partials(outs, lses)
+        parts[b, h] = pieces
+    return sel, out, lse, parts
 
 
 # ------------------------------------------------------------------ a7: prefill rows

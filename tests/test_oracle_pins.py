@@ -512,3 +512,55 @@ def test_bf16_storage_decides_the_selection_in_decode_layer():
     assert sel64[0, 0].tolist() == [1]
     assert sel16[0, 0].tolist() == [0] and sc16[0, 0].tolist() == [1.0, 1.0]
     assert np.array_equal(out16[0, 0], V[0, 0, 0])
+
+
+# ------------------------------------------------------------ sequence sharding (R19)
+def test_merge_partials_equals_attention_over_the_union():
+    """Splitting a set into disjoint parts and merging the parts' outputs by
+    their log-sum-exp is attention over the whole set (softmax identity)."""
+    rng = np.random.default_rng(19)
+    q, K, V = rng.standard_normal(64), rng.standard_normal((300, 64)), rng.standard_normal((300, 64))
+    idx = np.sort(rng.choice(300, 120, replace=False))
+    parts = [idx[idx < 90], idx[(idx >= 90) & (idx < 90)], idx[(idx >= 90) & (idx < 250)], idx[idx >= 250]]
+    assert parts[1].size == 0
+    res = [O.attend(q, K, V, p, 0.125) for p in parts]
+    o, lse = O.merge_partials([r[0] for r in res], [r[1] for r in res])
+    o_all, lse_all = O.attend(q, K, V, idx, 0.125)
+    assert np.allclose(o, o_all, rtol=0, atol=1e-12) and math.isclose(lse, lse_all, rel_tol=1e-13)
+    # the merge is symmetric in its parts
+    o2, lse2 = O.merge_partials([r[0] for r in res[::-1]], [r[1] for r in res[::-1]])
+    assert np.allclose(o2, o, atol=1e-14) and math.isclose(lse2, lse, rel_tol=1e-15)
+
+
+def test_merge_partials_special_cases():
+    o = np.arange(4.0)
+    got, lse = O.merge_partials([o], [1.5])                       # one part: itself
+    assert np.array_equal(got, o) and lse == 1.5
+    got, lse = O.merge_partials([np.zeros(4), o], [-math.inf, 0.0])  # an empty part carries no weight
+    assert np.array_equal(got, o) and lse == 0.0
+    got, lse = O.merge_partials([np.zeros(4), np.zeros(4)], [-math.inf, -math.inf])
+    assert np.array_equal(got, np.zeros(4)) and lse == -math.inf    # every part empty: as an empty set
+    # two equal-mass parts average: lse = l + log 2
+    got, lse = O.merge_partials([np.ones(4), 3 * np.ones(4)], [0.7, 0.7])
+    assert np.allclose(got, 2.0) and math.isclose(lse, 0.7 + math.log(2.0))
+
+
+@pytest.mark.parametrize("group", [False, True])
+def test_sharded_decode_equals_unsharded(group):
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, L, D, dimp, G = 2, 4, 2, 700, 32, 8, 1
+    q, K, V, W, qimp = _layer_inputs(rng, B, Hq, Hkv, L, D, dimp, G)
+    lens = [700, 455]
+    args = (q, K, V, W, qimp, 1, G, lens, 30, 8, 32)
+    sel, out, lse, _ = O.decode_layer(*args, dense=False, group=group)
+    bounds = [(0, 200), (200, 420), (420, 700)]
+    sel_s, out_s, lse_s, parts = O.decode_layer_sharded(*args, bounds, group=group)
+    for key in sel:
+        assert np.array_equal(sel_s[key], sel[key])
+        assert np.allclose(out_s[key], out[key], atol=1e-12) and math.isclose(lse_s[key], lse[key], rel_tol=1e-12)
+        pieces = parts[key]
+        assert np.array_equal(np.concatenate(pieces), sel[key])      # disjoint, in rank order, covering the set
+        for (t0, t1), p in zip(bounds, pieces):
+            assert p.size == 0 or (p.min() >= t0 and p.max() < t1)
+    # sequence 1 ends inside rank 2's range; rank 2 still holds its window
+    assert parts[1, 0][2].size > 0
