@@ -315,6 +315,53 @@ typedef struct tb_cache_view {
 TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, const void* q, const uint32_t* mask,
                                        int mask_mode, void* out, float* lse, void* stream);
 
+/* ---- Sequence-sharded decode (one long sequence over several ranks).
+ * Beyond the pages, which decode on one device: each rank's context holds,
+ * for every sequence, the contiguous global tokens [t0, t0 + len[b]) of its
+ * caches (ranks in token order; appends go to the rank holding the end).
+ * One step selects exactly the one-device set (model card "Method": top-x
+ * under the global budget k = min(floor(P * L / 100), candidates), sink,
+ * window, ties to the lower index) and merges the ranks' attention over
+ * their parts by log-sum-exp.  Per layer and step, on every rank:
+ *   tb_shard_set(layer, t0, global lengths)
+ *   tb_score(...)                          local scores (rows: Hq, or Hkv with TB_BUTLER_GROUP)
+ *   for pass in 0, 1:  tb_shard_hist -> sum the histograms over ranks -> tb_shard_pick(n_ranks = 1)
+ *   pass 2:            tb_shard_hist -> gather the histograms in rank order -> tb_shard_pick(R, rank)
+ *   tb_shard_mask                          this rank's mask words
+ *   tb_sparse_attn_partial                 fp32 partial output and lse
+ *   gather the partials in rank order -> tb_merge_partials
+ * The collectives are the caller's (NCCL through torch.distributed in the
+ * Python binding).  TB_ERR_UNSUPPORTED for TB_SOFTVOTE.  Buffers (device,
+ * caller-owned):
+ *   hist   [B*rows][2048] uint32 (pass 2: gathered [R][B*rows][2048])
+ *   state  [B*rows][4] uint32: threshold key, counts, mode, quota
+ *   mask   [B][rows][max_len/32] uint32 (words of this rank's local tokens)
+ *   part   [B*Hq*D + B*Hq] fp32: output rows, then natural-log lse
+ * A summed histogram holding fewer keys than the budget sets
+ * TB_DEV_ERR_COUNT and leaves that row without its top-k. */
+TB_API tb_status tb_shard_set(tb_ctx* ctx, int layer, int t0, const int32_t* global_lens_host);
+/* zeroes `hist` and accumulates this rank's histogram of radix digit `pass`
+ * (0: top 11 bits of the order key, 1: next 11, 2: low 10) over its
+ * candidates, restricted by `state` to the digits found so far (pass > 0) */
+TB_API tb_status tb_shard_hist(tb_ctx* ctx, int layer, const float* scores, int pass, const uint32_t* state,
+                               uint32_t* hist, void* stream);
+/* from the histogram summed over ranks (passes 0, 1; n_ranks = 1) or the
+ * gathered per-rank histograms (pass 2; n_ranks = R, this rank's index),
+ * the row's digit of the k-th largest key; pass 2 also sets the quota of
+ * keys equal to the threshold this rank keeps */
+TB_API tb_status tb_shard_pick(tb_ctx* ctx, int layer, int pass, const uint32_t* hist, int n_ranks, int rank,
+                               uint32_t* state, void* stream);
+TB_API tb_status tb_shard_mask(tb_ctx* ctx, int layer, const float* scores, const uint32_t* state, uint32_t* mask,
+                               void* stream);
+/* tb_sparse_attn writing fp32 output rows and lse into `part` (layout above) */
+TB_API tb_status tb_sparse_attn_partial(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mask_mode,
+                                        float* part, void* stream);
+/* out[b][h] = sum_r exp(lse_r - lse) o_r over `n_parts` consecutive `part`
+ * blocks (lse_r = -inf: no weight; all empty: zero output, lse -inf);
+ * `lse` [B][Hq] may be NULL */
+TB_API tb_status tb_merge_partials(tb_ctx* ctx, const float* parts, int n_parts, void* out, float* lse,
+                                   void* stream);
+
 /* Tracing: when `events` is non-NULL, tb_decode_step records the six
  * cudaEvent_t events[0..5] on its stream before the append, after the
  * append, after scoring, after selection, after the split attention kernel

@@ -18,6 +18,7 @@
 #include "kernels/project_tc.cuh"
 #include "kernels/score.cuh"
 #include "kernels/select.cuh"
+#include "kernels/shard.cuh"
 #include "kernels/softvote.cuh"
 #include "tb.h"
 
@@ -38,6 +39,10 @@ struct LayerState {
   float* sc_q = nullptr;        // [B*rows][d'] importance query of the cached set
   int32_t* sc_len = nullptr;    // [B*rows] length at which it was selected (0: empty)
   uint32_t* sc_mask = nullptr;  // [B*rows][max_len/32] the cached mask
+  // sequence sharding: this layer's caches hold global tokens [shard_t0, shard_t0 + lens[b])
+  bool shard_on = false;
+  int shard_t0 = 0;
+  int glen[TB_MAX_BATCH];
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -302,7 +307,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
 }
 
 static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mode, void* out,
-                             float* lse, cudaStream_t st) {
+                             float* lse, cudaStream_t st, bool out_f32 = false) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   const int maxL = max_len_of(ls, c.batch);
@@ -368,7 +373,7 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   cp.nsplit = p.nsplit;
   for (int b = 0; b < c.batch; ++b) cp.lens[b] = ls.lens[b];
   const unsigned cgrid = (unsigned)(c.batch * c.n_q_heads);
-  if (c.kv_dtype == TB_BF16) {
+  if (c.kv_dtype == TB_BF16 && !out_f32) {
     if (c.head_dim == 128) launch_pdl(combine_kernel<__nv_bfloat16, 128>, dim3(cgrid), dim3(kCombineThreads), 0, st,
                     cp);
     else launch_pdl(combine_kernel<__nv_bfloat16, 64>, dim3(cgrid), dim3(kCombineThreads), 0, st,
@@ -983,3 +988,141 @@ TB_API const char* tb_status_string(tb_status s) {
 TB_API void tb_destroy(tb_ctx* ctx) { delete ctx; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ sequence sharding
+static tb_status shard_params(const tb_ctx* ctx, int layer, ShardParams* p) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  if (c.variant == TB_SOFTVOTE) return TB_ERR_UNSUPPORTED;
+  if (!ls.shard_on) return TB_ERR_STATE;
+  *p = ShardParams{};
+  p->status = ctx->status;
+  p->rows = sel_rows(c);
+  p->total_rows = c.batch * p->rows;
+  p->max_len = c.max_len;
+  p->keep_pct = c.keep_pct;
+  p->sink = c.sink;
+  p->window = c.window;
+  p->t0 = ls.shard_t0;
+  for (int b = 0; b < c.batch; ++b) {
+    p->nloc[b] = ls.lens[b];
+    p->glen[b] = ls.glen[b];
+  }
+  return TB_OK;
+}
+
+TB_API tb_status tb_shard_set(tb_ctx* ctx, int layer, int t0, const int32_t* global_lens) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!global_lens || t0 < 0) return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  if (c.variant == TB_SOFTVOTE) return TB_ERR_UNSUPPORTED;
+  LayerState& ls = ctx->layers[layer];
+  for (int b = 0; b < c.batch; ++b)
+    if ((long long)t0 + ls.lens[b] > global_lens[b] || global_lens[b] < 0) return TB_ERR_STATE;
+  ls.shard_on = true;
+  ls.shard_t0 = t0;
+  for (int b = 0; b < c.batch; ++b) ls.glen[b] = global_lens[b];
+  return TB_OK;
+}
+
+static unsigned shard_chunks(const tb_ctx* ctx, const ShardParams& p, int tok) {
+  int m = 1;
+  for (int b = 0; b < ctx->cfg.batch; ++b) m = std::max(m, p.nloc[b]);
+  return (unsigned)((m + tok - 1) / tok);
+}
+
+TB_API tb_status tb_shard_hist(tb_ctx* ctx, int layer, const float* scores, int pass, const uint32_t* state,
+                               uint32_t* hist, void* stream) {
+  ShardParams p;
+  tb_status s = shard_params(ctx, layer, &p);
+  if (s != TB_OK) return s;
+  if (!scores || !hist || (pass > 0 && !state) || pass < 0 || pass > 2) return TB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  p.scores = scores;
+  p.state = reinterpret_cast<uint4*>(const_cast<uint32_t*>(state));
+  p.hist = hist;
+  p.pass = pass;
+  const size_t n = (size_t)p.total_rows * kHistBins;
+  launch_pdl(zero_u32_kernel, dim3((unsigned)std::min<size_t>((n + 255) / 256, 1024)), dim3(256), 0, st, hist, n);
+  launch_pdl(shard_hist_kernel, dim3(shard_chunks(ctx, p, kShardHistTok), p.total_rows), dim3(kShardThreads), 0, st,
+             p);
+  ctx->launches += 2;
+  return cuda_status(cudaGetLastError());
+}
+
+TB_API tb_status tb_shard_pick(tb_ctx* ctx, int layer, int pass, const uint32_t* hist, int n_ranks, int rank,
+                               uint32_t* state, void* stream) {
+  ShardParams p;
+  tb_status s = shard_params(ctx, layer, &p);
+  if (s != TB_OK) return s;
+  if (!hist || !state || pass < 0 || pass > 2) return TB_ERR_INVALID_ARG;
+  if (n_ranks < 1 || rank < 0 || rank >= n_ranks || (pass < 2 && n_ranks != 1)) return TB_ERR_INVALID_ARG;
+  p.hist_in = hist;
+  p.state = reinterpret_cast<uint4*>(state);
+  p.pass = pass;
+  p.n_ranks = n_ranks;
+  p.rank = rank;
+  launch_pdl(shard_pick_kernel, dim3((unsigned)((p.total_rows + 7) / 8)), dim3(kShardThreads), 0,
+             static_cast<cudaStream_t>(stream), p);
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
+TB_API tb_status tb_shard_mask(tb_ctx* ctx, int layer, const float* scores, const uint32_t* state, uint32_t* mask,
+                               void* stream) {
+  ShardParams p;
+  tb_status s = shard_params(ctx, layer, &p);
+  if (s != TB_OK) return s;
+  if (!scores || !state || !mask) return TB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  p.scores = scores;
+  p.state = reinterpret_cast<uint4*>(const_cast<uint32_t*>(state));
+  p.mask = mask;
+  launch_pdl(shard_mask_kernel, dim3(shard_chunks(ctx, p, kShardMaskTok), p.total_rows), dim3(kShardThreads), 0, st,
+             p);
+  launch_pdl(shard_ties_kernel, dim3((unsigned)p.total_rows), dim3(kShardThreads), 0, st, p);
+  ctx->launches += 2;
+  return cuda_status(cudaGetLastError());
+}
+
+TB_API tb_status tb_sparse_attn_partial(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mask_mode,
+                                        float* part, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!q || !part) return TB_ERR_INVALID_ARG;
+  if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_GROUP &&
+      mask_mode != TB_MASK_DENSE)
+    return TB_ERR_INVALID_ARG;
+  if (mask_mode != TB_MASK_DENSE && !mask) return TB_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(part)) return TB_ERR_SHAPE;
+  const tb_config& c = ctx->cfg;
+  float* lse = part + (size_t)c.batch * c.n_q_heads * c.head_dim;
+  return launch_attn(ctx, layer, q, mask, mask_mode, part, lse, static_cast<cudaStream_t>(stream), true);
+}
+
+TB_API tb_status tb_merge_partials(tb_ctx* ctx, const float* parts, int n_parts, void* out, float* lse,
+                                   void* stream) {
+  if (!ctx || !parts || !out || n_parts < 1) return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  MergeParams p{};
+  p.parts = parts;
+  p.rows = c.batch * c.n_q_heads;
+  p.part_stride = (size_t)p.rows * (c.head_dim + 1);
+  p.out = out;
+  p.lse = lse;
+  p.n_parts = n_parts;
+  const dim3 grid((unsigned)((p.rows + 3) / 4));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c.kv_dtype == TB_BF16) {
+    if (c.head_dim == 128) launch_pdl(merge_partials_kernel<__nv_bfloat16, 128>, grid, dim3(128), 0, st, p);
+    else launch_pdl(merge_partials_kernel<__nv_bfloat16, 64>, grid, dim3(128), 0, st, p);
+  } else {
+    if (c.head_dim == 128) launch_pdl(merge_partials_kernel<float, 128>, grid, dim3(128), 0, st, p);
+    else launch_pdl(merge_partials_kernel<float, 64>, grid, dim3(128), 0, st, p);
+  }
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}

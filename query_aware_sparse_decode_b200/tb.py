@@ -30,7 +30,8 @@ EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "
            "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
            "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
            "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait", "tb_selection_cache_size",
-           "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks", "tb_bind_layer_paged")
+           "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks", "tb_bind_layer_paged", "tb_shard_set",
+           "tb_shard_hist", "tb_shard_pick", "tb_shard_mask", "tb_sparse_attn_partial", "tb_merge_partials")
 
 
 class TBError(RuntimeError):
@@ -91,6 +92,12 @@ def lib():
             "tb_set_reuse": [vp, ctypes.c_float, i32, i32],
             "tb_copy_step_masks": [vp, vp, sz, vp],
             "tb_bind_layer_paged": [vp, i32, vp, vp, i32, vp, i32, i32, vp, vp],
+            "tb_shard_set": [vp, i32, i32, P(ctypes.c_int32)],
+            "tb_shard_hist": [vp, i32, vp, i32, vp, vp, vp],
+            "tb_shard_pick": [vp, i32, i32, vp, i32, i32, vp, vp],
+            "tb_shard_mask": [vp, i32, vp, vp, vp, vp],
+            "tb_sparse_attn_partial": [vp, i32, vp, vp, i32, vp, vp],
+            "tb_merge_partials": [vp, vp, i32, vp, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -274,6 +281,31 @@ class Context:
 
     def set_reuse(self, tau: float, interval: int, radius: int = 0) -> None:
         _check(lib().tb_set_reuse(self._h, ctypes.c_float(tau), interval, radius), "tb_set_reuse")
+
+    # ---- sequence-sharded decode (the step sequence is in shard.py)
+    def shard_set(self, layer: int, t0: int, global_lens) -> None:
+        arr = (ctypes.c_int32 * self.cfg.batch)(*[int(x) for x in global_lens])
+        _check(lib().tb_shard_set(self._h, layer, int(t0), arr), "tb_shard_set")
+
+    def shard_hist(self, layer, scores, pass_, state, hist, stream=None) -> None:
+        _check(lib().tb_shard_hist(self._h, layer, _ptr(scores), pass_, _ptr(state), _ptr(hist), _stream(stream)),
+               "tb_shard_hist")
+
+    def shard_pick(self, layer, pass_, hist, n_ranks, rank, state, stream=None) -> None:
+        _check(lib().tb_shard_pick(self._h, layer, pass_, _ptr(hist), n_ranks, rank, _ptr(state), _stream(stream)),
+               "tb_shard_pick")
+
+    def shard_mask(self, layer, scores, state, mask, stream=None) -> None:
+        _check(lib().tb_shard_mask(self._h, layer, _ptr(scores), _ptr(state), _ptr(mask), _stream(stream)),
+               "tb_shard_mask")
+
+    def sparse_attn_partial(self, layer, q, mask, mask_mode, part, stream=None) -> None:
+        _check(lib().tb_sparse_attn_partial(self._h, layer, _ptr(q), _ptr(mask), mask_mode, _ptr(part),
+                                            _stream(stream)), "tb_sparse_attn_partial")
+
+    def merge_partials(self, parts, n_parts, out, lse=None, stream=None) -> None:
+        _check(lib().tb_merge_partials(self._h, _ptr(parts), n_parts, _ptr(out), _ptr(lse), _stream(stream)),
+               "tb_merge_partials")
 
     def selftest_bounded_wait(self, cycles: int, arrive: bool, stream=None) -> None:
         """Launch the bounded-wait self-test (see include/tb.h); read the

@@ -49,3 +49,69 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks_of(3.5, 1, None) == 3.5
     assert bench.whole_job_rate(10, 2, 1, 1000.0) == 20.0
+
+
+# ------------------------------------------------ sequence-sharded step exchanges
+def _fake_step(rank, world, log):
+    """The exchange pattern of shard_step with stand-in tensors: a summed
+    histogram, then a gather in rank order."""
+    h = torch.full((3, 2048), rank + 1, dtype=torch.int32)
+    h[0, rank] += 100
+    yield ("sum", h)
+    log.append(h.clone())
+    src = torch.arange(5, dtype=torch.float32) + 10 * rank
+    dst = torch.empty((world, 5))
+    yield ("gather", src, dst)
+    log.append(dst.clone())
+
+
+def _shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from query_aware_sparse_decode_b200.shard import TorchCollectives
+    log = []
+    TorchCollectives().run(_fake_step(rank, world, log))
+    q.put((rank, [t.tolist() for t in log]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _expected(world):
+    from query_aware_sparse_decode_b200.shard import run_lockstep
+    logs = [[] for _ in range(world)]
+    run_lockstep(_fake_step(r, world, logs[r]) for r in range(world))
+    return logs
+
+
+def test_shard_exchanges_torch_distributed_world2_match_lockstep():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    want = _expected(2)
+    for r in range(2):
+        assert res[r] == [t.tolist() for t in want[r]]
+    hsum, gathered = want[0]
+    assert hsum[0, 0].item() == 103 and hsum[0, 1].item() == 103 and hsum[1, 5].item() == 3
+    assert gathered[1].tolist() == [10.0, 11.0, 12.0, 13.0, 14.0]      # rank order
+
+
+def test_lockstep_rejects_ranks_out_of_step():
+    from query_aware_sparse_decode_b200.shard import run_lockstep
+
+    def a():
+        yield ("sum", torch.zeros(2, dtype=torch.int32))
+
+    def b():
+        yield ("gather", torch.zeros(2), torch.zeros((2, 2)))
+
+    with pytest.raises(RuntimeError):
+        run_lockstep([a(), b()])
+    with pytest.raises(RuntimeError):
+        run_lockstep([a(), iter(())])
