@@ -699,6 +699,98 @@ def _table_prefill(dev, iters, peak, n_layers=None):
     return line
 
 
+def _table_shard(wl, ranks_list, dev, iters, flush_buf, variant=None):
+    """Sequence-sharded decode of one layer with R ranks emulated on this GPU
+    in lock step (each rank its own context and caches, ranks in token
+    order, the last one appending).  Per rank: the device time of its own
+    kernels between the exchanges (median over steps); the exchanges, done
+    here by in-process copies, are excluded and reported as bytes, since
+    across GPUs they are NCCL collectives over NVLink."""
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    from query_aware_sparse_decode_b200 import tb as TB
+    from query_aware_sparse_decode_b200.shard import ShardBuffers, exchange_in_process, sel_rows, shard_step
+    variant = TB.TB_BUTLER if variant is None else variant
+    L0 = wl.L - 1
+    max_len = (wl.L + 1 + 255) // 256 * 256
+    full, bufs, _ = build(wl, max_len, dev, variant)
+    k_full, v_full, kimp_full, w = bufs[0]
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    kn, vn = S.kv_new(wl, 0)
+    kn, vn, qq, qi = bf(kn), bf(vn), bf(S.query(wl, 0)), bf(S.q_imp(wl, 0))
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    rows_out = []
+    for R in ranks_list:
+        per = (L0 + R - 1) // R
+        starts = [r * per for r in range(R)]
+        ranks = []
+        for r in range(R):
+            t0 = starts[r]
+            n = (starts[r + 1] if r + 1 < R else L0) - t0
+            cap = (n + 2 + 255) // 256 * 256
+            cfg = TB.make_config(1, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G, cap, "bf16", wl.keep_pct, wl.sink,
+                                 wl.window, dense_layers=(), variant=variant)
+            ctx = TB.Context(cfg, dev)
+            k = torch.zeros((wl.B, wl.Hkv, cap, wl.D), dtype=torch.bfloat16, device=dev)
+            v = torch.zeros_like(k)
+            k[:, :, :n] = k_full[:, :, t0:t0 + n]
+            v[:, :, :n] = v_full[:, :, t0:t0 + n]
+            kimp = TB.kimp_cache(cfg, dev)
+            ctx.bind_layer(0, k, v, kimp, w)
+            ctx.set_seq_lens(0, [n] * wl.B)
+            ctx.project_kimp(0, 0, n)
+            ranks.append((ctx, n, t0, ShardBuffers(cfg, R, dev), (k, v, kimp)))
+        stream = torch.cuda.current_stream(dev)
+        per_rank = [[] for _ in range(R)]
+        for it in range(3 + iters):
+            for ctx, n, _, _, _ in ranks:
+                ctx.set_seq_lens(0, [n] * wl.B)
+            if flush_buf is not None:
+                flush_buf.add_(1)
+                flush_buf.view(torch.float32)[: 64 << 20].sum()
+            steps = [shard_step(ctx, 0, r, R, t0, [wl.L] * wl.B, qq, qi, out, sb,
+                                kn if r == R - 1 else None, vn if r == R - 1 else None, stream)
+                     for r, (ctx, _, t0, sb, _) in enumerate(ranks)]
+            evs = [[] for _ in range(R)]
+            # the host issues the ranks' calls one by one; a device-side wait
+            # queued first lets all of them be enqueued before the GPU reaches
+            # them, so the events time the kernels and not the issuing
+            torch.cuda._sleep(100_000_000)
+            while True:
+                ops = []
+                for r, st in enumerate(steps):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    ops.append(next(st, None))
+                    e1.record(stream)
+                    evs[r].append((e0, e1))
+                if all(o is None for o in ops):
+                    break
+                exchange_in_process(ops)
+            torch.cuda.synchronize()
+            for ctx, _, _, _, _ in ranks:
+                if ctx.check_status():
+                    raise RuntimeError("device status flags set")
+            if it >= 3:
+                for r in range(R):
+                    per_rank[r].append(sum(a.elapsed_time(b) for a, b in evs[r]) * 1e3)
+        med = [statistics.median(x) for x in per_rank]
+        nrow = wl.B * sel_rows(ranks[0][0].cfg)
+        part = wl.B * wl.Hq * (wl.D + 1) * 4
+        rows_out.append({"ranks": R, "tokens_per_rank": [n for _, n, _, _, _ in ranks],
+                         "us_per_rank": [round(x, 1) for x in med], "us_slowest_rank": round(max(med), 1),
+                         "exchange_bytes_per_rank": {"hist_sum_2x": 2 * nrow * 2048 * 4,
+                                                     "hist_gather": R * nrow * 2048 * 4,
+                                                     "partials_gather": R * part}})
+        del ranks
+        torch.cuda.empty_cache()
+    return {"table": "sequence_sharded", "workload": wl.name, "variant": _variant_name(variant),
+            "emulated_on": "one GPU, ranks in lock step, calls enqueued behind a device wait",
+            "rows": rows_out}
+
+
 def kernel_table(args):
     """Per-kernel times for the workloads beside the step benchmark: the
     8B-shaped L=32768 case (50 % and dense), the long-context sweep of both
@@ -728,6 +820,10 @@ def kernel_table(args):
             print(json.dumps(_table_case(wl, variant, dev, args.table_iters, flush_buf, peak)), flush=True)
     if pick is None or pick.search(S.PREFILL_L32K.name):
         print(json.dumps(_table_prefill(dev, args.table_iters, peak, args.layers)), flush=True)
+    for L in (131072, 262144):
+        wl = S.sweep(L, 30)
+        if pick is None or pick.search(f"shard_{wl.name}"):
+            print(json.dumps(_table_shard(wl, (1, 2, 4, 8), dev, args.table_iters, flush_buf)), flush=True)
 
 
 # ----------------------------------------------------------------------- main

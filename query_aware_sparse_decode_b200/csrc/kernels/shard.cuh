@@ -30,8 +30,8 @@
 namespace tb {
 
 constexpr int kShardThreads = 256;
-constexpr int kShardHistTok = 8192;  // tokens per CTA of the histogram kernel
-constexpr int kShardMaskTok = 8192;  // tokens per CTA of the mask kernel (8 warps x 32 words)
+constexpr int kShardHistTok = 2048;  // tokens per CTA of the histogram kernel (8 loads per thread)
+constexpr int kShardMaskTok = 2048;  // tokens per CTA of the mask kernel (8 warps x 8 words)
 
 struct ShardParams {
   const float* scores;      // [B][rows][max_len] this rank's scores (local token index)
@@ -89,8 +89,17 @@ __global__ void __launch_bounds__(kShardThreads) shard_hist_kernel(const ShardPa
   for (int i = tid; i < kHistBins; i += kShardThreads) h[i] = 0;
   __syncthreads();
   const float* s = p.scores + (size_t)row * p.max_len;
-  for (int t = t_begin + tid; t < t_end; t += kShardThreads) {
-    const uint32_t key = order_key(s[t]);
+  constexpr int PER = kShardHistTok / kShardThreads;
+  float v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {  // all loads first, coalesced across the block
+    const int t = t_begin + tid + i * kShardThreads;
+    v[i] = t < t_end ? s[t] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    if (t_begin + tid + i * kShardThreads >= t_end) break;
+    const uint32_t key = order_key(v[i]);
     if (p.pass == 0)
       atomicAdd(&h[key >> 21], 1u);
     else if ((key >> match_shift) == match)
@@ -101,18 +110,22 @@ __global__ void __launch_bounds__(kShardThreads) shard_hist_kernel(const ShardPa
     if (h[i]) atomicAdd(&p.hist[(size_t)row * kHistBins + i], h[i]);
 }
 
-// One warp per row: the digit of the current pass that holds the row's k-th
-// largest key (counts summed over ranks).  Pass 0 also sets the row's mode
-// from the global budget k = min(floor(P * L / 100), candidates).  After the
-// last digit the threshold T is known, and the gathered per-rank counts of T
-// give this rank's quota: the keys equal to T still to take, minus those of
-// lower ranks, clamped to this rank's own.  grid ceil(B*rows / 8), block 256.
+// One CTA per row: the digit of the current pass that holds the row's k-th
+// largest key (counts summed over ranks).  Thread t holds the nb/256 bins
+// just below nb - t * nb/256 (thread 0 the highest), loaded at once; a
+// block scan of the per-thread counts from the top finds the thread, and
+// the thread its bin.  Pass 0 also sets the row's mode from the global
+// budget k = min(floor(P * L / 100), candidates).  After the last digit the
+// threshold T is known, and the gathered per-rank counts of T give this
+// rank's quota: the keys equal to T still to take, minus those of lower
+// ranks, clamped to this rank's own.  grid B*rows, block 256.
 __global__ void __launch_bounds__(kShardThreads) shard_pick_kernel(const ShardParams p) {
   pdl_wait();
   pdl_trigger();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (kShardThreads / 32) + warp;
-  if (row >= p.total_rows) return;
+  constexpr int NW = kShardThreads / 32;
+  __shared__ uint32_t wtot[NW];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x;
   const int b = row / p.rows;
   uint4 st;
   if (p.pass == 0) {
@@ -121,7 +134,7 @@ __global__ void __launch_bounds__(kShardThreads) shard_pick_kernel(const ShardPa
     const int k = (int)min((long long)p.keep_pct * L / 100, (long long)cand);
     st = make_uint4(0u, (uint32_t)k, k == 0 ? 0u : (k == cand ? 1u : 2u), 0u);
     if (st.z != 2u) {
-      if (lane == 0) p.state[row] = st;
+      if (tid == 0) p.state[row] = st;
       return;
     }
   } else {
@@ -130,43 +143,56 @@ __global__ void __launch_bounds__(kShardThreads) shard_pick_kernel(const ShardPa
   }
   const uint32_t krem = st.y;
   const int nb = p.pass == 2 ? 1024 : kHistBins;
-  const int per = nb / 32;
+  const int per = nb / kShardThreads;  // 8 or 4
   const int nsum = p.pass == 2 ? p.n_ranks : 1;
   const uint32_t* H = p.hist_in + (size_t)row * kHistBins;
   const size_t rstride = (size_t)p.total_rows * kHistBins;
-  auto count = [&](int bin) {
-    uint32_t c = 0;
-    for (int r = 0; r < nsum; ++r) c += H[r * rstride + bin];
-    return c;
-  };
-  // lane l sums bins [nb - (l + 1) * per, nb - l * per): lane 0 the highest
-  const int bin_hi = nb - lane * per;
-  uint32_t lsum = 0;
-  for (int i = 1; i <= per; ++i) lsum += count(bin_hi - i);
-  uint32_t incl = lsum;
+  const int bin_hi = nb - tid * per;  // this thread: bins [bin_hi - per, bin_hi)
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = 0;
+  for (int r = 0; r < nsum; ++r) {
+    const uint32_t* Hr = H + r * rstride + (bin_hi - per);
+    if (per == 8) {
+      const uint4 a = *reinterpret_cast<const uint4*>(Hr), d = *reinterpret_cast<const uint4*>(Hr + 4);
+      c[0] += a.x, c[1] += a.y, c[2] += a.z, c[3] += a.w, c[4] += d.x, c[5] += d.y, c[6] += d.z, c[7] += d.w;
+    } else {
+      const uint4 a = *reinterpret_cast<const uint4*>(Hr);
+      c[0] += a.x, c[1] += a.y, c[2] += a.z, c[3] += a.w;
+    }
+  }
+  uint32_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mine += c[i];
+  // inclusive scan over threads in order (thread 0 = highest bins)
+  uint32_t incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  const uint32_t excl = incl - lsum;
-  const unsigned ball = __ballot_sync(0xffffffffu, excl < krem && krem <= incl);
-  if (ball == 0u) {  // the summed counts hold fewer than k keys: inconsistent histograms
-    if (lane == 0) {
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) incl += wtot[w];
+  uint32_t total = 0;
+  for (int w = 0; w < NW; ++w) total += wtot[w];
+  const uint32_t excl = incl - mine;
+  if (total < krem) {  // the summed counts hold fewer than k keys: inconsistent histograms
+    if (tid == 0) {
       atomicOr(p.status, TB_DEV_ERR_COUNT);
       st.z = 0u;
       p.state[row] = st;
     }
     return;
   }
-  if (lane != __ffs(ball) - 1) return;
+  if (!(excl < krem && krem <= incl)) return;  // exactly one thread goes on
   uint32_t above = excl;
-  int bin = bin_hi - 1;
-  for (; bin > bin_hi - per; --bin) {
-    const uint32_t c = count(bin);
-    if (above + c >= krem) break;
-    above += c;
+  int i = per - 1;  // c[per - 1] is bin bin_hi - 1, the highest of this thread
+  for (; i > 0; --i) {
+    if (above + c[i] >= krem) break;
+    above += c[i];
   }
+  const int bin = bin_hi - per + i;
   const uint32_t rem = krem - above;  // keys of this digit value still to take (>= 1)
   st.x |= (uint32_t)bin << (p.pass == 0 ? 21 : (p.pass == 1 ? 10 : 0));
   if (p.pass < 2) {
@@ -174,15 +200,16 @@ __global__ void __launch_bounds__(kShardThreads) shard_pick_kernel(const ShardPa
   } else {
     uint32_t before = 0;
     for (int r = 0; r < p.rank; ++r) before += H[r * rstride + bin];
-    const uint32_t mine = H[(size_t)p.rank * rstride + bin];
-    st.y = mine;
-    st.w = rem > before ? min(rem - before, mine) : 0u;
+    const uint32_t own = H[(size_t)p.rank * rstride + bin];
+    st.y = own;
+    st.w = rem > before ? min(rem - before, own) : 0u;
   }
   p.state[row] = st;
 }
 
 // grid (ceil(max local tokens / kShardMaskTok), B*rows), block 256: each warp
-// writes 32 consecutive mask words of its row (one ballot per word).  A word
+// writes 8 consecutive mask words of its row (one ballot per word; the
+// scores of all 8 words are loaded first).  A word
 // holds sink tokens, window tokens, every candidate (mode 1), or candidates
 // whose key is above T, plus those equal to T when the quota is all of this
 // rank's (mode 2).
@@ -193,7 +220,8 @@ __global__ void __launch_bounds__(kShardThreads) shard_mask_kernel(const ShardPa
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = p.nloc[b], L = p.glen[b];
   const int nwords = (n + 31) >> 5;
-  const int w0 = blockIdx.x * (kShardMaskTok / 32) + warp * 32;
+  constexpr int WPW = kShardMaskTok / 32 / (kShardThreads / 32);  // words per warp
+  const int w0 = blockIdx.x * (kShardMaskTok / 32) + warp * WPW;
   if (w0 >= nwords) return;
   const uint4 st = p.state[row];
   const int s_end = min(p.sink, L), w_beg = L - p.window;
@@ -201,8 +229,17 @@ __global__ void __launch_bounds__(kShardThreads) shard_mask_kernel(const ShardPa
   const bool all_eq = st.z == 2u && st.w > 0u && st.w == st.y;
   const float* s = p.scores + (size_t)row * p.max_len;
   uint32_t* m = p.mask + (size_t)row * (p.max_len / 32);
-  const int w1 = min(w0 + 32, nwords);
-  for (int w = w0; w < w1; ++w) {
+  float v[WPW];
+#pragma unroll
+  for (int i = 0; i < WPW; ++i) {
+    const int tl = (w0 + i) * 32 + lane;
+    const int t = p.t0 + tl;
+    v[i] = (st.z == 2u && tl < n && t >= c_lo && t < c_hi) ? s[tl] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < WPW; ++i) {
+    const int w = w0 + i;
+    if (w >= nwords) break;
     const int tl = w * 32 + lane;
     const int t = p.t0 + tl;
     bool keep = false;
@@ -213,7 +250,7 @@ __global__ void __launch_bounds__(kShardThreads) shard_mask_kernel(const ShardPa
         if (st.z == 1u) {
           keep = true;
         } else if (st.z == 2u) {
-          const uint32_t key = order_key(s[tl]);
+          const uint32_t key = order_key(v[i]);
           keep = key > st.x || (all_eq && key == st.x);
         }
       }

@@ -1065,7 +1065,7 @@ TB_API tb_status tb_shard_pick(tb_ctx* ctx, int layer, int pass, const uint32_t*
   p.pass = pass;
   p.n_ranks = n_ranks;
   p.rank = rank;
-  launch_pdl(shard_pick_kernel, dim3((unsigned)((p.total_rows + 7) / 8)), dim3(kShardThreads), 0,
+  launch_pdl(shard_pick_kernel, dim3((unsigned)p.total_rows), dim3(kShardThreads), 0,
              static_cast<cudaStream_t>(stream), p);
   ++ctx->launches;
   return cuda_status(cudaGetLastError());

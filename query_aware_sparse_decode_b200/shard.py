@@ -107,22 +107,26 @@ def run_lockstep(steps) -> None:
     carrying out each exchange between them."""
     steps = list(steps)
     while True:
-        ops = []
-        for s in steps:
-            ops.append(next(s, None))
+        ops = [next(s, None) for s in steps]
         if all(o is None for o in ops):
             return
-        if any(o is None for o in ops) or len({o[0] for o in ops}) != 1:
-            raise RuntimeError("ranks out of step: " + ", ".join("done" if o is None else o[0] for o in ops))
-        if ops[0][0] == "sum":
-            total = ops[0][1].clone()
-            for o in ops[1:]:
-                total += o[1]
-            for o in ops:
-                o[1].copy_(total)
-        elif ops[0][0] == "gather":
-            for o in ops:
-                for r, src in enumerate(ops):
-                    o[2][r].copy_(src[1])
-        else:
-            raise ValueError(f"unknown exchange {ops[0][0]!r}")
+        exchange_in_process(ops)
+
+
+def exchange_in_process(ops) -> None:
+    """One exchange among ranks that share a process: ops[r] is rank r's
+    request, all of the same kind."""
+    if any(o is None for o in ops) or len({o[0] for o in ops}) != 1:
+        raise RuntimeError("ranks out of step: " + ", ".join("done" if o is None else o[0] for o in ops))
+    if ops[0][0] == "sum":
+        total = ops[0][1].clone()
+        for o in ops[1:]:
+            total += o[1]
+        for o in ops:
+            o[1].copy_(total)
+    elif ops[0][0] == "gather":
+        for o in ops:
+            for r, src in enumerate(ops):
+                o[2][r].copy_(src[1])
+    else:
+        raise ValueError(f"unknown exchange {ops[0][0]!r}")
