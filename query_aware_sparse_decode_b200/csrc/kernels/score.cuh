@@ -10,7 +10,9 @@
 // bf16 K_imp values): d' independent, coalesced loads, written as batches of
 // up to 16 loads ahead of their FMAs (fp32, dimension order j = 0..d'-1, the
 // group's query values broadcast from shared memory) so that many loads per
-// thread can be in flight.  A CTA covers 1, 2 or 4 steps of 256 threads' tokens
+// thread can be in flight.  The FMAs run on pairs of consecutive tokens
+// (fma.rn.f32x2: two independent round-to-nearest fp32 FMAs, the bits of two
+// fmaf).  A CTA covers 1, 2 or 4 steps of 256 threads' tokens
 // (the launch picks the count so the grid fills the SMs).
 // With GROUPED (one selection per KV group) the group's per-head fp32 scores
 // are added in head order and one row per (b, g) is written instead.
@@ -41,20 +43,31 @@ struct ScoreParams {
   int lens[kMaxBatch];
 };
 
-// The 16 bytes of one load as fp32 values (bf16 widened exactly).
-__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[4]) {
-  x[0] = __uint_as_float(v.x);
-  x[1] = __uint_as_float(v.y);
-  x[2] = __uint_as_float(v.z);
-  x[3] = __uint_as_float(v.w);
+// Packed fp32 pairs for fma.rn.f32x2.
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
 }
-__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[8]) {
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// The 16 bytes of one load as fp32 pairs of consecutive tokens (bf16
+// widened exactly: the low half of a word is the earlier token).
+__device__ __forceinline__ void unpack16(const uint4& v, uint64_t (&x)[2]) {
+  x[0] = f2_pack(v.x, v.y);
+  x[1] = f2_pack(v.z, v.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& v, uint64_t (&x)[4]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+  for (int i = 0; i < 4; ++i) x[i] = f2_pack(w[i] << 16, w[i] & 0xFFFF0000u);
 }
 
 template <typename T, typename KT, int DIMP, int GS, bool HIST, bool GROUPED = false>
@@ -98,11 +111,11 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
     const int t0 = t_base + it * STEP + TPT * tid;
     if (t0 < L) {
       const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t0, DIMP, p.max_len);
-      float acc[GS][TPT];
+      uint64_t acc2[GS][TPT / 2];  // token pairs (2u, 2u + 1)
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh)
 #pragma unroll
-        for (int u = 0; u < TPT; ++u) acc[hh][u] = 0.f;
+        for (int u = 0; u < TPT / 2; ++u) acc2[hh][u] = 0ull;
 #pragma unroll
       for (int j0 = 0; j0 < DIMP; j0 += NB) {
         uint4 v[NB];
@@ -110,16 +123,22 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
         for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const uint4*>(K + (j0 + jj) * kKimpTile));
 #pragma unroll
         for (int jj = 0; jj < NB; ++jj) {
-          float kv[TPT];
+          uint64_t kv[TPT / 2];
           unpack16(v[jj], kv);
 #pragma unroll
           for (int hh = 0; hh < GS; ++hh) {
-            const float qv = qs[j0 + jj][hh];
+            const uint32_t qb = __float_as_uint(qs[j0 + jj][hh]);
+            const uint64_t qv = f2_pack(qb, qb);
 #pragma unroll
-            for (int u = 0; u < TPT; ++u) acc[hh][u] = fmaf(qv, kv[u], acc[hh][u]);
+            for (int u = 0; u < TPT / 2; ++u) acc2[hh][u] = ffma2(kv[u], qv, acc2[hh][u]);
           }
         }
       }
+      float acc[GS][TPT];
+#pragma unroll
+      for (int hh = 0; hh < GS; ++hh)
+#pragma unroll
+        for (int u = 0; u < TPT / 2; ++u) f2_unpack(acc2[hh][u], acc[hh][2 * u], acc[hh][2 * u + 1]);
       if (GROUPED) {  // the group's row: per-head fp32 scores added in head order
 #pragma unroll
         for (int u = 0; u < TPT; ++u) {
