@@ -290,14 +290,14 @@ def merge_partials(outs, lses):
 
 
 def decode_layer_sharded(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, bounds,
-                         group: bool = False, kimp_storage: str = "f64"):
+                         group: bool = False, kimp_storage: str = "f64", heads=None, batches=None):
     """Reading R19: the decode step of one layer with the tokens split over
     ranks, bounds = [(t0_r, t1_r)] contiguous and in order.  The selected set
     is the unsharded step's; rank r attends over its part of it and the parts
     are merged (merge_partials).  Returns (sel, out, lse, parts) with parts
-    {(b, h): [indices of rank r]}."""
+    {(b, h): [indices of rank r]}.  `heads`, `batches`: as for decode_layer."""
     sel, _, _, _ = decode_layer(q, K, V, W_K, q_imp_producer, layer, G, L, keep_pct, sink, window, dense=False,
-                                group=group, kimp_storage=kimp_storage)
+                                group=group, kimp_storage=kimp_storage, heads=heads, batches=batches)
     q = np.asarray(q, dtype=np.float64)
     B, Hq, D = q.shape
     Hkv = K.shape[1]

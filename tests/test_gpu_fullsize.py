@@ -277,3 +277,76 @@ def test_device_generator_matches_host_bit_for_bit(dtype):
     assert not dev[:, :t0].any() and not dev[:, t1:].any()
     one = S.fill_host(S.K_CACHE, 7, 2, 1, t0, t1, C, dtype, delta=delta, plant_mod=100, seed=11, a0=4)
     assert np.array_equal(one[0].view(np.uint8), host[4].view(np.uint8))
+
+
+# ------------------------------------------------------------ sequence sharding at full size
+@pytest.mark.parametrize("ranks", [4])
+def test_sequence_sharded_L262144(ranks):
+    """One B = 1, L = 262144 layer at 30 % over 4 emulated ranks (lock step on
+    this GPU): the union of the ranks' masks equals the one-context step's
+    bit for bit (identical K_imp rows give identical scores), every rank's
+    merged output equals the one context's within bf16 rounding, and sampled
+    KV heads match the oracle (sets up to the tie band, outputs)."""
+    from query_aware_sparse_decode_b200.shard import ShardBuffers, run_lockstep, shard_step
+    wl = S.sweep(262144, 30)
+    cfg = config_of(wl)
+    _need_device_bytes(2 * _layer_bytes(wl, cfg.max_len))
+    full = TB.Context(cfg)
+    dl = make_layer_device(full, wl, 0, wl.L - 1)
+    L0 = wl.L - 1
+    per = (L0 + ranks - 1) // ranks
+    starts = [r * per for r in range(ranks)]
+    ctxs = []
+    for r in range(ranks):
+        t0 = starts[r]
+        n = (starts[r + 1] if r + 1 < ranks else L0) - t0
+        cap = (n + 2 + 255) // 256 * 256
+        rc = TB.Context(config_of(wl, max_len=cap))
+        k = torch.zeros((wl.B, wl.Hkv, cap, wl.D), dtype=tdtype(wl), device="cuda")
+        v = torch.zeros_like(k)
+        k[:, :, :n] = dl.k_cache[:, :, t0:t0 + n]
+        v[:, :, :n] = dl.v_cache[:, :, t0:t0 + n]
+        kimp = TB.kimp_cache(rc.cfg)
+        rc.bind_layer(0, k, v, kimp, to_dev(S.w_k(wl, 0), wl))
+        rc.set_seq_lens(0, [n] * wl.B)
+        rc.project_kimp(0, 0, n)
+        ctxs.append((rc, t0, ShardBuffers(rc.cfg, ranks), (k, v, kimp)))
+    k_raw, v_raw = S.kv_new(wl, 0)
+    k_dev, v_dev = to_dev(k_raw, wl), to_dev(v_raw, wl)
+    outs = [torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda") for _ in range(ranks)]
+    run_lockstep(shard_step(rc, 0, r, ranks, t0, [wl.L] * wl.B, dl.q_dev, dl.q_imp_dev, outs[r], sb,
+                            k_dev if r == ranks - 1 else None, v_dev if r == ranks - 1 else None)
+                 for r, (rc, t0, sb, _) in enumerate(ctxs))
+    r1 = _gpu_step(full, wl, 0, dl, k_dev, v_dev, wl.keep_pct)
+    for rc, _, _, _ in ctxs:
+        assert rc.check_status() == 0
+    # one-context sets against the union of the ranks' local masks
+    want = sets_from_mask(r1["mask"], [wl.L] * wl.B)
+    got = {}
+    for rc, t0, sb, _ in ctxs:
+        for key, idx in sets_from_mask(sb.mask, rc.seq_lens(0)).items():
+            got.setdefault(key, []).append(idx + t0)
+    for key in want:
+        assert np.array_equal(np.concatenate(got[key]), want[key]), f"row {key}"
+    merged = outs[0].float().cpu().numpy()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    assert_close_rows(merged.reshape(-1, wl.D), r1["out"].reshape(-1, wl.D), wl.dtype, "merged vs one context")
+    # oracle on two sampled KV heads
+    K = _Slabs(dl, S.K_CACHE, S.widen(k_raw, wl.dtype))
+    V = _Slabs(dl, S.V_CACHE, S.widen(v_raw, wl.dtype))
+    gs = wl.Hq // wl.Hkv
+    bounds = [(starts[r], starts[r + 1] if r + 1 < ranks else wl.L) for r in range(ranks)]
+    for g in (0, 5):
+        heads = range(g * gs, (g + 1) * gs)
+        K.slab(0, g)
+        V.slab(0, g)
+        sel, ref, _, _ = O.decode_layer_sharded(dl.q, K, V, dl.W, dl.qimp, 0, wl.G, [wl.L], wl.keep_pct,
+                                                wl.sink, wl.window, bounds, heads=heads, batches=[0])
+        _, _, _, sc = O.decode_layer(dl.q, K, V, dl.W, dl.qimp, 0, wl.G, [wl.L], wl.keep_pct, wl.sink, wl.window,
+                                     dense=False, heads=heads, batches=[0])
+        for h in heads:
+            gset = np.concatenate(got[0, h])
+            assert tie_band_ok(gset, sel[0, h], sc[0, h], wl.L, wl.keep_pct, wl.sink, wl.window), f"h{h}"
+            if np.array_equal(gset, sel[0, h]):
+                assert_close_rows(merged[0, h][None], ref[0, h][None], wl.dtype, f"h{h}")
