@@ -195,18 +195,23 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const int ntiles = n / kAttnTile + (n % kAttnTile ? 1 : 0);
   const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
 
+  // A lane copies the same 16-byte pieces of its rows from K and from V: the
+  // rows' cache indices are read from the list once, before the copies.
+  constexpr int PER = kAttnTile * NCH / 32;  // pieces per lane and tensor
   auto issue = [&](int it) {
     const int tile = warp + it * kAttnWarps;
     uint8_t* sb = my_ring + (it % kAttnStages) * STAGE;
+    int tok[PER];
 #pragma unroll
-    for (int c = lane; c < 2 * kAttnTile * NCH; c += 32) {
-      const int tensor = c / (kAttnTile * NCH);
-      const int rc = c % (kAttnTile * NCH);
-      const int row = rc / NCH, part = rc % NCH;
-      const int tok = list_idx[tile * kAttnTile + row];
-      const uint8_t* src = (tensor ? Vb : Kb) + (size_t)tok * ROWB + part * 16;
-      uint8_t* dst = sb + tensor * kAttnTile * ROWB + row * ROWB + ((part ^ (row & 7)) << 4);
-      cp_async_16(dst, src);
+    for (int i = 0; i < PER; ++i) tok[i] = list_idx[tile * kAttnTile + (lane + 32 * i) / NCH];
+#pragma unroll
+    for (int tensor = 0; tensor < 2; ++tensor) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int rc = lane + 32 * i, row = rc / NCH, part = rc % NCH;
+        cp_async_16(sb + tensor * kAttnTile * ROWB + row * ROWB + ((part ^ (row & 7)) << 4),
+                    (tensor ? Vb : Kb) + (size_t)tok[i] * ROWB + part * 16);
+      }
     }
   };
 #pragma unroll

@@ -14,8 +14,8 @@
 // accumulate); writes the logits in the log2 domain and one (max, sum of
 // 2^(a - max)) pair per head and chunk.
 // softvote_reduce: merges the chunk pairs into each head's (M, Z) (a warp per
-// head, lanes over the chunks) and sums 2^(a - M) / Z over the heads for four
-// consecutive tokens per thread (logits are L2-resident).  Optionally it also
+// head, lanes over the chunks) and sums 2^(a - M) / Z over the heads, one
+// token per thread (logits are L2-resident).  Optionally it also
 // builds the first-digit histogram of the votes over the candidate range
 // [sink, len - window) for the selection that follows (warp-aggregated shared
 // atomics: votes crowd into few bins).
@@ -76,15 +76,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   const int ntiles = (n + kAttnTile - 1) / kAttnTile;
   const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
   uint8_t* my_ring = smem + warp * kAttnStages * STAGE;
+  // A tile's 16 tokens are consecutive cache rows: tiles start at multiples of
+  // 16 and pages hold a power of two >= 16 tokens, so one row lookup per tile
+  // serves all of them (rows past the ragged end repeat the last token).
   auto issue = [&](int it) {
     const int tile = warp + it * kAttnWarps;
     uint8_t* sb = my_ring + (it % kAttnStages) * STAGE;
+    const int tt = t0 + tile * kAttnTile;
+    const int last = t1 - 1 - tt;
+    const uint8_t* base = Kb + (size_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, tt) * ROWB;
 #pragma unroll
     for (int c = lane; c < kAttnTile * NCH; c += 32) {
       const int row = c / NCH, part = c % NCH;
-      const int tok = min(t0 + tile * kAttnTile + row, t1 - 1);  // clamp the ragged tail
-      cp_async_16(sb + row * ROWB + ((part ^ (row & 7)) << 4),
-                  Kb + (size_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, tok) * ROWB + part * 16);
+      cp_async_16(sb + row * ROWB + ((part ^ (row & 7)) << 4), base + min(row, last) * ROWB + part * 16);
     }
   };
 #pragma unroll
@@ -165,17 +169,26 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   }
 }
 
-// grid (ceil(max len / 1024), B), block 256: votes for 1024 tokens per CTA.
+// grid (ceil(max len / 256), B), block 256: one token per thread.  The
+// token's logits of the first kVotePrefetch heads are requested before the
+// CTA merges the chunk statistics, so their latency overlaps the merge.
 constexpr int kVoteMaxHeads = 128;
-__global__ void __launch_bounds__(256, 1) softvote_reduce_kernel(const VoteParams p) {
+constexpr int kVoteReduceTok = 256;
+constexpr int kVotePrefetch = 32;
+__global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sM[kVoteMaxHeads], sInvZ[kVoteMaxHeads];
   __shared__ uint32_t hist[kHistBins];
   const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = p.lens[b];
-  const int t_begin = blockIdx.x * 1024;
+  const int t_begin = blockIdx.x * kVoteReduceTok;
   if (t_begin >= L) return;
+  const int t = t_begin + tid;
+  const float* lg = p.logits + (size_t)b * p.Hq * p.max_len + t;
+  float a[kVotePrefetch];
+#pragma unroll
+  for (int h = 0; h < kVotePrefetch; ++h) a[h] = (h < p.Hq && t < L) ? lg[(size_t)h * p.max_len] : 0.f;
   const int nch = (L + kVoteChunk - 1) / kVoteChunk;
   for (int h = warp; h < p.Hq; h += 8) {
     const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
@@ -204,37 +217,19 @@ __global__ void __launch_bounds__(256, 1) softvote_reduce_kernel(const VoteParam
   if (p.hist1 != nullptr)
     for (int i = tid; i < kHistBins; i += 256) hist[i] = 0;
   __syncthreads();
-  const int t0 = t_begin + 4 * tid;
-  float v[4] = {0.f, 0.f, 0.f, 0.f};
-  if (t0 < L) {
-    const float* lg = p.logits + (size_t)b * p.Hq * p.max_len + t0;
-#pragma unroll 8
-    for (int h = 0; h < p.Hq; ++h) {
-      const float4 a = *reinterpret_cast<const float4*>(lg + (size_t)h * p.max_len);
-      const float M = sM[h], iz = sInvZ[h];
-      v[0] += exp2f(a.x - M) * iz;
-      v[1] += exp2f(a.y - M) * iz;
-      v[2] += exp2f(a.z - M) * iz;
-      v[3] += exp2f(a.w - M) * iz;
-    }
-    float* out = p.votes + (size_t)b * p.max_len + t0;
-    if (t0 + 3 < L) {
-      *reinterpret_cast<float4*>(out) = make_float4(v[0], v[1], v[2], v[3]);
-    } else {
+  float v = 0.f;  // sum over the heads in head order
+  if (t < L) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (t0 + u < L) out[u] = v[u];
-    }
+    for (int h = 0; h < kVotePrefetch; ++h)
+      if (h < p.Hq) v += exp2f(a[h] - sM[h]) * sInvZ[h];
+    for (int h = kVotePrefetch; h < p.Hq; ++h) v += exp2f(lg[(size_t)h * p.max_len] - sM[h]) * sInvZ[h];
+    p.votes[(size_t)b * p.max_len + t] = v;
   }
   if (p.hist1 == nullptr) return;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int t = t0 + u;
-    const bool in = t < L && t >= p.sink && t < L - p.window;
-    const uint32_t bin = in ? (order_key(v[u]) >> 21) : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-    if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-  }
+  const bool in = t < L && t >= p.sink && t < L - p.window;
+  const uint32_t bin = in ? (order_key(v) >> 21) : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+  if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
   __syncthreads();
   for (int i = tid; i < kHistBins; i += 256)
     if (hist[i]) atomicAdd(&p.hist1[(size_t)b * kHistBins + i], hist[i]);

@@ -429,7 +429,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   ++ctx->launches;
   tb_status s = cuda_status(cudaGetLastError());
   if (s != TB_OK) return s;
-  dim3 g2((maxL + 1023) / 1024, c.batch);
+  dim3 g2((maxL + kVoteReduceTok - 1) / kVoteReduceTok, c.batch);
   launch_pdl(softvote_reduce_kernel, g2, dim3(256), 0, st, p);
   ++ctx->launches;
   return cuda_status(cudaGetLastError());
