@@ -26,7 +26,9 @@
 
 namespace tb {
 
-constexpr int kVoteChunk = 2048;  // tokens per CTA of the logits pass
+// Tokens per CTA of the logits pass: chosen per launch (a multiple of 16, at
+// least kVoteMinChunk) so that the grid is about four CTAs per SM in one wave.
+constexpr int kVoteMinChunk = 256;
 
 struct VoteParams {
   const void* k_cache;  // [B][Hkv][max_len][D] bf16, or a page pool (KvLayout)
@@ -36,7 +38,8 @@ struct VoteParams {
   float* stats;         // [B][Hq][nchunk][2]
   float* votes;         // [B][max_len]
   uint32_t* hist1;      // [B][2048] first-digit histograms of the votes, or nullptr
-  int Hq, Hkv, max_len, nchunk;
+  int Hq, Hkv, max_len, nchunk;  // nchunk: stride of the chunk statistics, >= max_len / chunk
+  int chunk;                     // tokens per CTA of the logits pass
   int sink, window;
   float scale_log2;
   int lens[kMaxBatch];
@@ -53,9 +56,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   extern __shared__ __align__(128) uint8_t smem[];
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int L = p.lens[b];
-  const int t0 = chunk * kVoteChunk;
+  const int t0 = chunk * p.chunk;
   if (t0 >= L) return;
-  const int t1 = min(t0 + kVoteChunk, L);
+  const int t1 = min(t0 + p.chunk, L);
   const int n = t1 - t0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 2, tq = lane & 3;
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p
   float a[kVotePrefetch];
 #pragma unroll
   for (int h = 0; h < kVotePrefetch; ++h) a[h] = (h < p.Hq && t < L) ? lg[(size_t)h * p.max_len] : 0.f;
-  const int nch = (L + kVoteChunk - 1) / kVoteChunk;
+  const int nch = (L + p.chunk - 1) / p.chunk;
   for (int h = warp; h < p.Hq; h += 8) {
     const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
     float m = kNegInf, l = 0.f;

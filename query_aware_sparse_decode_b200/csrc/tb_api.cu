@@ -71,7 +71,7 @@ WsLayout layout_of(const tb_config& c) {
   w.part_o = off;  off += align256(B * Hq * (size_t)w.max_splits * c.head_dim * 4);
   w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
   w.votes = off;   off += align256(B * Lm * 4);
-  w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteChunk - 1) / kVoteChunk) * 2 * 4);
+  w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteMinChunk - 1) / kVoteMinChunk) * 2 * 4);
   w.reuse = off;   off += align256(B * Hq * 4);         // per-row reuse decisions of the step
   w.total = off;
   return w;
@@ -411,10 +411,15 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   p.Hq = c.n_q_heads;
   p.Hkv = c.n_kv_heads;
   p.max_len = c.max_len;
-  p.nchunk = (c.max_len + kVoteChunk - 1) / kVoteChunk;
+  p.nchunk = (c.max_len + kVoteMinChunk - 1) / kVoteMinChunk;
+  {  // about four CTAs per SM in one wave, whatever B and L
+    const int nsplit = std::max(1, 4 * ctx->num_sms / (c.batch * c.n_kv_heads));
+    const int chunk = ((maxL + nsplit - 1) / nsplit + 15) / 16 * 16;
+    p.chunk = std::max(kVoteMinChunk, chunk);
+  }
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  dim3 grid((maxL + kVoteChunk - 1) / kVoteChunk, c.n_kv_heads, c.batch);
+  dim3 grid((maxL + p.chunk - 1) / p.chunk, c.n_kv_heads, c.batch);
 #define TB_VOTE_CASE(DV, GSV)                                                                 \
   if (c.head_dim == DV && gs == GSV) {                                                        \
     auto k = softvote_logits_kernel<DV, GSV>;                                                 \
