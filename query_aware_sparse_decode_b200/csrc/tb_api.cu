@@ -328,9 +328,14 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   p.max_len = c.max_len;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  // chunking: the whole grid is about two full waves of two CTAs per SM
+  // chunking: the whole grid is about two full waves of two CTAs per SM, or
+  // one wave when two would leave CTAs with short chunks (fewer than 3584
+  // tokens: the list build, the ring's fill and the partial write then weigh
+  // more than the second wave's balance gains)
   const int groups = c.batch * c.n_kv_heads;
-  const int want_split = std::min(kMaxSplits, std::max(1, (4 * ctx->num_sms) / groups));
+  int want_split = std::min(kMaxSplits, std::max(1, (4 * ctx->num_sms) / groups));
+  if ((std::max(maxL, 1) + want_split - 1) / want_split < 3584)
+    want_split = std::min(kMaxSplits, std::max(1, (2 * ctx->num_sms) / groups));
   int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
   chunk = std::max(256, (chunk + 255) / 256 * 256);
   p.chunk = chunk;
