@@ -77,7 +77,26 @@ def test_null_context_calls_fail_cleanly():
     assert L.tb_set_budget(None, 30, 16, 64) == 1
     assert L.tb_check_status(None, None) == 1
     assert L.tb_trace_events(None, None, 0) == 1
+    assert L.tb_shard_set(None, 0, 0, None) == 1
+    assert L.tb_shard_hist(None, 0, None, 0, None, None, None) == 1
+    assert L.tb_shard_pick(None, 0, 0, None, 1, 0, None, None) == 1
+    assert L.tb_shard_mask(None, 0, None, None, None, None) == 1
+    assert L.tb_sparse_attn_partial(None, 0, None, None, 0, None, None) == 1
+    assert L.tb_merge_partials(None, None, 1, None, None, None) == 1
+    assert L.tb_bind_layer_paged(None, 0, None, None, 1, None, 64, 1, None, None) == 1
+    assert L.tb_set_reuse(None, 0.9, 3, 0) == 1
     L.tb_destroy(None)
+
+
+def test_kimp_storage_option_validation():
+    """bf16 K_imp needs bf16 caches; the flag is 0 or 1."""
+    assert _ws(_cfg(kimp_dtype="bf16"))[0] == 0
+    assert _ws(_cfg(kimp_dtype="bf16", kv_dtype="f32"))[0] == 7
+    cfg = _cfg()
+    cfg.kimp_bf16 = 2
+    assert TB.lib().tb_workspace_size(ctypes.byref(cfg), ctypes.byref(ctypes.c_size_t(0))) == 1
+    with pytest.raises(ValueError):
+        _cfg(kimp_dtype="fp8")
 
 
 def test_status_strings():
