@@ -163,6 +163,51 @@ def test_select_bit_exact_on_identical_scores(case):
             assert np.array_equal(got_sets[b, r], ref)
 
 
+@pytest.mark.parametrize("case", [
+    dict(lens=(512,), keep=50, sink=4, window=16, quant=0, kind=None),
+    dict(lens=(3000, 2999), keep=30, sink=16, window=64, quant=4, kind=None),
+    dict(lens=(4096, 100, 80, 1), keep=50, sink=16, window=64, quant=2, kind=None),
+    dict(lens=(9000,), keep=10, sink=0, window=0, quant=1, kind=None),
+    dict(lens=(777, 0), keep=100, sink=3, window=5, quant=8, kind=None),
+    dict(lens=(16384, 12000), keep=30, sink=16, window=64, quant=0, kind="three_values"),
+    dict(lens=(16000,), keep=50, sink=16, window=64, quant=0, kind="two_digits"),
+], ids=lambda c: f"L{c['lens']}-k{c['keep']}-q{c['quant']}-{c['kind']}")
+def test_short_row_select_bit_exact_on_identical_scores(case):
+    """Rows of at most 16384 tokens without an index list take the one-CTA-
+    per-row selection: exact sets and counts on identical fp32 scores,
+    including quantised scores (-0.0 against +0.0) and rows where ties at
+    the threshold decide most of the budget (an ordered quota)."""
+    lens, rows = case["lens"], 4
+    B = len(lens)
+    wl = S.Workload("selr", n_layers=1, B=B, Hq=rows, Hkv=1, D=64, d_imp=16, G=1, L=max(lens), dtype="f32",
+                    keep_pct=case["keep"], sink=case["sink"], window=case["window"], plant="none", lens=lens)
+    cfg = config_of(wl)
+    Lmax = cfg.max_len
+    ctx = TB.Context(cfg)
+    dummy = torch.zeros((B, 1, Lmax, 64), device="cuda")
+    ctx.bind_layer(0, dummy, dummy.clone(), kimp_alloc(B, 1, 16, Lmax), torch.zeros((64, 16), device="cuda"))
+    ctx.set_seq_lens(0, lens)
+    if case["kind"] is None:
+        sc = _synthetic_scores(B, rows, Lmax, case["quant"], len(lens) * 100 + case["keep"] + 7)
+    else:
+        sc = np.zeros((B, rows, Lmax), np.float32)
+        for b, L in enumerate(lens):
+            for r in range(rows):
+                sc[b, r, :L] = _crowded_scores(case["kind"], L, 31 + 4 * b + r)
+    cnt = torch.full((B, rows), -1, dtype=torch.int32, device="cuda")
+    mask = torch.zeros((B, rows, Lmax // 32), dtype=torch.int32, device="cuda")
+    ctx.select(0, torch.from_numpy(sc).cuda(), rows, count=cnt, mask=mask)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    cnt = cnt.cpu().numpy()
+    got_sets = sets_from_mask(mask, lens)
+    for b, L in enumerate(lens):
+        for r in range(rows):
+            ref = O.select_tokens(sc[b, r].astype(np.float64), L, case["keep"], case["sink"], case["window"])
+            assert cnt[b, r] == ref.size, f"b{b} r{r}"
+            assert np.array_equal(got_sets[b, r], ref), f"b{b} r{r}"
+
+
 def _crowded_scores(kind, L, seed):
     u = S.fill_host(21, seed, 0, 1, 0, L, 1, "f32").reshape(L).astype(np.float64)
     u = (u - u.min()) / (u.max() - u.min() + 1e-12)          # in [0, 1)
