@@ -164,7 +164,7 @@ __device__ __forceinline__ bool warps_sync_bounded(uint64_t* bar, uint32_t& phas
   ++phase;
   return __all_sync(0xffffffffu, ok);
 }
-// 2-D tiled TMA load (no multicast) completing on `bar`
+// 2-D tiled TMA load into this CTA's shared memory only, completing on `bar`
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(

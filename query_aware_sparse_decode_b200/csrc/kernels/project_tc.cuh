@@ -5,7 +5,7 @@
 // GEMM with M = cached rows (tiles of 128), N = d' (32 or 16), K = D (128 or
 // 64), bf16 operands and fp32 accumulation in tensor memory.
 //   warp 0      TMA producer: K tiles (128 rows x 64 columns per box, 128B
-//               swizzle) into a 4-stage shared-memory ring; no multicast.
+//               swizzle) into a 4-stage shared-memory ring of this CTA only.
 //   warp 1      one thread issues tcgen05.mma (kind::f16, M=128) per 16-wide
 //               K step and commits to the ring's "empty" and the
 //               accumulator's "full" mbarriers.
