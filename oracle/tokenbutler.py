@@ -62,8 +62,10 @@ project_keys with storage="bf16"): K_imp is rounded once, from its exact
 value, to the nearest bfloat16 (ties to even) and scored as stored.
 
 Parity pins (tests/test_oracle_pins.py) cover every function here; the
-readings R4, R6, R13 and R14 are consistent with the sources but not fixed
-by them (parity unpinned against the pages for those readings).
+readings R4, R6, R13, R14 and R18 are consistent with the sources but not
+fixed by them (parity unpinned against the pages for those readings), and
+R19 and the two options go beyond the sources (pinned by identities:
+equality with the unsharded step, the softmax split, single rounding).
 """
 from __future__ import annotations
 
