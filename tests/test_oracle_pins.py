@@ -1,7 +1,9 @@
 """Pins of the fp64 oracle against what the sources and the mathematics fix:
 hand-typed values from the model card, textbook special cases, library
 routines (torch float64 scaled_dot_product_attention), brute force on tiny
-inputs and invariants.  CPU only."""
+inputs and invariants.  Every pin runs on both statements of the oracle:
+the numpy one (oracle/tokenbutler.py) and the C++ one (oracle/tokenbutler.cpp
+through oracle/native.py).  CPU only."""
 import itertools
 import math
 import os
@@ -10,9 +12,16 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import tokenbutler as O
+from oracle import native as _native
+from oracle import tokenbutler as _numpy_oracle
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(params=["numpy", "cpp"])
+def O(request):
+    """The oracle under test."""
+    return _numpy_oracle if request.param == "numpy" else _native
 
 
 def _rows(name, tag=None):
@@ -30,7 +39,7 @@ def _rows(name, tag=None):
 
 
 # ----------------------------------------------------------------- layers / slots
-def test_slot_map_matches_model_card_table():
+def test_slot_map_matches_model_card_table(O):
     rows = _rows("slot_map_G4.txt")
     assert len(rows) == 32
     for layer, prod, slot in rows:
@@ -38,7 +47,7 @@ def test_slot_map_matches_model_card_table():
         assert O.consumer_slot(int(layer), 4) == int(slot)
 
 
-def test_each_producer_serves_itself_and_next_G_minus_1_layers_with_distinct_slots():
+def test_each_producer_serves_itself_and_next_G_minus_1_layers_with_distinct_slots(O):
     for G in (1, 2, 3, 4, 8):
         for p in range(0, 64, G):
             layers = range(p, p + G)
@@ -46,7 +55,7 @@ def test_each_producer_serves_itself_and_next_G_minus_1_layers_with_distinct_slo
             assert sorted(O.consumer_slot(l, G) for l in layers) == list(range(G))
 
 
-def test_importance_query_layout_picks_slot_and_position():
+def test_importance_query_layout_picks_slot_and_position(O):
     # Q_imp is (B*H) x G x L x d' (model card, Method).  B=1, Hq=2, G=2, 3 positions, d'=2.
     q = np.arange(1 * 2 * 2 * 3 * 2, dtype=np.float64).reshape(2, 2, 3, 2)
     # layer 2 reads slot (2-1) mod 2 = 1; head 1 is row 1
@@ -57,14 +66,14 @@ def test_importance_query_layout_picks_slot_and_position():
     assert qh[0, 0].tolist() == [10.0, 11.0]   # ((0*2+1)*3+2)*2 = 10
 
 
-def test_gqa_head_map():
+def test_gqa_head_map(O):
     assert [O.kv_head_of(h, 32, 8) for h in range(8)] == [0, 0, 0, 0, 1, 1, 1, 1]
     assert O.kv_head_of(31, 32, 8) == 7
     assert [O.kv_head_of(h, 4, 2) for h in range(4)] == [0, 0, 1, 1]
 
 
 # ----------------------------------------------------------------- budget
-def test_policy_and_budget_golden():
+def test_policy_and_budget_golden(O):
     for name, pct in _rows("budget.txt", "policy"):
         assert O.keep_pct_from_policy(name) == int(pct)
     for L, pct, k in _rows("budget.txt", "budget"):
@@ -73,7 +82,7 @@ def test_policy_and_budget_golden():
         O.keep_pct_from_policy("topk_50")
 
 
-def test_budget_floor_and_limits():
+def test_budget_floor_and_limits(O):
     assert O.token_budget(131072, 30) == 39321      # floor(39321.6)
     assert O.token_budget(7, 50) == 3
     assert O.token_budget(0, 50) == 0
@@ -82,7 +91,7 @@ def test_budget_floor_and_limits():
 
 
 # ----------------------------------------------------------------- K_imp and scores
-def test_project_keys_special_cases():
+def test_project_keys_special_cases(O):
     rng = np.random.default_rng(1)
     K = rng.standard_normal((5, 7, 8))
     W = np.zeros((8, 3))
@@ -95,7 +104,7 @@ def test_project_keys_special_cases():
     assert np.all(out[..., [0, 2]] == 0)
 
 
-def test_project_keys_is_linear_and_matches_loops_on_tiny():
+def test_project_keys_is_linear_and_matches_loops_on_tiny(O):
     rng = np.random.default_rng(2)
     K = rng.standard_normal((4, 6))
     W = rng.standard_normal((6, 3))
@@ -105,7 +114,7 @@ def test_project_keys_is_linear_and_matches_loops_on_tiny():
     assert np.allclose(O.project_keys(K + K2, W), O.project_keys(K, W) + O.project_keys(K2, W), atol=1e-12)
 
 
-def test_scores_basis_query_reads_one_coordinate():
+def test_scores_basis_query_reads_one_coordinate(O):
     rng = np.random.default_rng(3)
     Kimp = rng.standard_normal((9, 4))
     for j in range(4):
@@ -117,7 +126,7 @@ def test_scores_basis_query_reads_one_coordinate():
 
 
 # ----------------------------------------------------------------- selection
-def test_select_hand_example():
+def test_select_hand_example(O):
     s = np.array([9, 1, 5, 5, 2, 7, 5, 0, 3, 4], dtype=np.float64)
     # L=10, sink 1, window 2: candidates are tokens 1..7.
     # 50 %: k = 5 -> scores 7(t5), 5(t2), 5(t3), 5(t6), 2(t4)
@@ -140,7 +149,7 @@ def _brute_force_top(s, cand, k):
 
 
 @pytest.mark.parametrize("seed", range(12))
-def test_select_matches_brute_force_on_tiny_rows(seed):
+def test_select_matches_brute_force_on_tiny_rows(O, seed):
     rng = np.random.default_rng(seed)
     L = int(rng.integers(1, 13))
     s = rng.integers(-3, 4, size=L).astype(np.float64)   # small integers: many exact ties, exact sums
@@ -158,7 +167,7 @@ def test_select_matches_brute_force_on_tiny_rows(seed):
 @pytest.mark.parametrize("L,pct,sink,window", [(4096, 50, 16, 64), (4096, 30, 16, 64), (1000, 10, 4, 16),
                                                 (80, 50, 16, 64), (70, 50, 16, 64), (1, 50, 16, 64),
                                                 (0, 50, 4, 4), (333, 100, 0, 0), (333, 50, 0, 0)])
-def test_select_invariants(L, pct, sink, window):
+def test_select_invariants(O, L, pct, sink, window):
     rng = np.random.default_rng(L + pct)
     s = np.round(rng.standard_normal(L) * 4) / 4          # quantised: exact ties
     sel = O.select_tokens(s, L, pct, sink, window)
@@ -180,14 +189,14 @@ def test_select_invariants(L, pct, sink, window):
             assert max(tied_in) < min(tied_out)
 
 
-def test_select_negative_zero_equals_positive_zero():
+def test_select_negative_zero_equals_positive_zero(O):
     s = np.array([0.0, -0.0, 0.0, -0.0, -1.0])
     assert O.select_tokens(s, 5, 40, 0, 0).tolist() == [0, 1]
     s = np.array([-0.0, 0.0, -0.0, 0.0, -1.0])
     assert O.select_tokens(s, 5, 40, 0, 0).tolist() == [0, 1]
 
 
-def test_select_invariant_under_softmax_and_positive_affine_maps():
+def test_select_invariant_under_softmax_and_positive_affine_maps(O):
     rng = np.random.default_rng(7)
     s = rng.standard_normal(4096) * 3
     base = O.select_tokens(s, 4096, 30, 16, 64)
@@ -206,7 +215,7 @@ def _sdpa64(q, K, V):
     return out[0, 0, 0].numpy()
 
 
-def test_attend_equals_library_attention_on_all_tokens():
+def test_attend_equals_library_attention_on_all_tokens(O):
     rng = np.random.default_rng(4)
     q, K, V = rng.standard_normal(64), rng.standard_normal((300, 64)), rng.standard_normal((300, 64))
     o, lse = O.attend(q, K, V, np.arange(300), 1 / 8)
@@ -214,7 +223,7 @@ def test_attend_equals_library_attention_on_all_tokens():
     assert math.isclose(lse, float(np.log(np.exp(K @ q / 8).sum())), rel_tol=1e-12)
 
 
-def test_attend_textbook_loops_on_tiny():
+def test_attend_textbook_loops_on_tiny(O):
     rng = np.random.default_rng(5)
     q, K, V = rng.standard_normal(3), rng.standard_normal((5, 3)), rng.standard_normal((5, 3))
     idx = [0, 2, 3]
@@ -225,7 +234,7 @@ def test_attend_textbook_loops_on_tiny():
     assert math.isclose(lse, math.log(sum(w)), rel_tol=1e-12)
 
 
-def test_attend_special_cases():
+def test_attend_special_cases(O):
     rng = np.random.default_rng(6)
     q, K, V = rng.standard_normal(16), rng.standard_normal((50, 16)), rng.standard_normal((50, 16))
     o, _ = O.attend(q, K, V, np.array([17]), 0.25)          # one token: its value row
@@ -238,7 +247,7 @@ def test_attend_special_cases():
     assert np.all(o == 0) and lse == -math.inf
 
 
-def test_attend_order_free_and_lse_merge():
+def test_attend_order_free_and_lse_merge(O):
     rng = np.random.default_rng(8)
     q, K, V = rng.standard_normal(32), rng.standard_normal((200, 32)), rng.standard_normal((200, 32))
     a, b = np.arange(0, 200, 3), np.arange(1, 200, 3)
@@ -263,7 +272,7 @@ def _layer_inputs(rng, B, Hq, Hkv, L, D, dimp, G):
     return q, K, V, W, qi
 
 
-def test_full_budget_equals_dense_gqa_attention_from_library():
+def test_full_budget_equals_dense_gqa_attention_from_library(O):
     rng = np.random.default_rng(9)
     B, Hq, Hkv, L, D = 2, 8, 2, 96, 32
     q, K, V, W, qi = _layer_inputs(rng, B, Hq, Hkv, L, D, 8, 4)
@@ -282,7 +291,7 @@ def test_full_budget_equals_dense_gqa_attention_from_library():
     assert all(np.allclose(out_d[k], out[k], atol=1e-12) for k in out)
 
 
-def test_sparse_layer_uses_consumer_slot_and_own_kv_head():
+def test_sparse_layer_uses_consumer_slot_and_own_kv_head(O):
     rng = np.random.default_rng(10)
     B, Hq, Hkv, L, D, dimp, G = 1, 4, 2, 64, 16, 4, 4
     q, K, V, W, qi = _layer_inputs(rng, B, Hq, Hkv, L, D, dimp, G)
@@ -296,7 +305,7 @@ def test_sparse_layer_uses_consumer_slot_and_own_kv_head():
         assert sel[0, h].size == 2 + 4 + 32
 
 
-def test_ragged_lengths_per_sequence():
+def test_ragged_lengths_per_sequence(O):
     rng = np.random.default_rng(11)
     q, K, V, W, qi = _layer_inputs(rng, 3, 4, 2, 50, 16, 4, 1)
     lens = [50, 17, 1]
@@ -307,7 +316,7 @@ def test_ragged_lengths_per_sequence():
             assert sel[b, h].max() == Lb - 1
 
 
-def test_planted_tokens_are_selected_tiny_f32():
+def test_planted_tokens_are_selected_tiny_f32(O):
     from query_aware_sparse_decode_b200 import synth as S
     wl = S.TINY_F32
     W = S.w_k(wl, 0)
@@ -330,7 +339,7 @@ def test_planted_tokens_are_selected_tiny_f32():
 
 
 # ----------------------------------------------------------------- prefill rows
-def test_prefill_rows_are_causal_and_match_brute_force():
+def test_prefill_rows_are_causal_and_match_brute_force(O):
     rng = np.random.default_rng(12)
     Hq, Hkv, dimp, row0, nrows = 2, 1, 3, 5, 6
     Kimp = np.round(rng.standard_normal((Hkv, row0 + nrows, dimp)) * 2) / 2
@@ -348,7 +357,7 @@ def test_prefill_rows_are_causal_and_match_brute_force():
 
 
 # ----------------------------------------------------------------- soft voting
-def test_softvote_votes_sum_to_heads_and_equal_keys_vote_uniformly():
+def test_softvote_votes_sum_to_heads_and_equal_keys_vote_uniformly(O):
     rng = np.random.default_rng(13)
     q, K = rng.standard_normal((8, 16)), rng.standard_normal((2, 40, 16))
     v = O.softvote_scores(q, K, 40)
@@ -357,7 +366,7 @@ def test_softvote_votes_sum_to_heads_and_equal_keys_vote_uniformly():
     assert np.allclose(O.softvote_scores(q, Ku, 40), 8.0 / 40, atol=1e-14)
 
 
-def test_softvote_two_tokens_closed_form_and_single_head_reduction():
+def test_softvote_two_tokens_closed_form_and_single_head_reduction(O):
     D = 16
     q = np.zeros((1, D))
     q[0, 0] = 1.0
@@ -372,7 +381,7 @@ def test_softvote_two_tokens_closed_form_and_single_head_reduction():
     assert np.array_equal(O.select_tokens(v1, 500, 30, 4, 8), O.select_tokens(K1[0] @ q1[0], 500, 30, 4, 8))
 
 
-def test_softvote_layer_shares_one_set_over_heads():
+def test_softvote_layer_shares_one_set_over_heads(O):
     rng = np.random.default_rng(15)
     q, K, V = rng.standard_normal((1, 4, 16)), rng.standard_normal((1, 2, 64, 16)), rng.standard_normal((1, 2, 64, 16))
     sel, out, _, votes = O.softvote_layer(q, K, V, 64, 30, 2, 4)
@@ -383,7 +392,7 @@ def test_softvote_layer_shares_one_set_over_heads():
 
 
 # --------------------------------------------------------------------------- per-group option
-def test_group_scores_one_head_is_the_head_and_sum_is_the_summed_query():
+def test_group_scores_one_head_is_the_head_and_sum_is_the_summed_query(O):
     rng = np.random.default_rng(11)
     K_imp = rng.standard_normal((40, 6))
     q1 = rng.standard_normal((1, 6))
@@ -395,7 +404,7 @@ def test_group_scores_one_head_is_the_head_and_sum_is_the_summed_query():
     assert np.allclose(O.group_scores(q4, K_imp), want, rtol=1e-13, atol=1e-13)
 
 
-def test_group_selection_shares_one_set_per_group_and_equals_per_head_for_equal_queries():
+def test_group_selection_shares_one_set_per_group_and_equals_per_head_for_equal_queries(O):
     rng = np.random.default_rng(12)
     B, Hq, Hkv, D, dimp, L, G = 1, 8, 2, 16, 4, 300, 1
     q = rng.standard_normal((B, Hq, D))
@@ -421,7 +430,7 @@ def test_group_selection_shares_one_set_per_group_and_equals_per_head_for_equal_
 
 
 # --------------------------------------------------------------------------- amortised selection (R18)
-def test_reuse_decision_rules():
+def test_reuse_decision_rules(O):
     q = np.array([1.0, 0.0, 0.0])
     near = np.array([1.0, 0.1, 0.0])            # cos 0.995
     far = np.array([0.0, 1.0, 0.0])             # cos 0
@@ -436,7 +445,7 @@ def test_reuse_decision_rules():
     assert not O.reuse_decision(q, near, 200, 198, **dict(args, keep_pct=100))  # 100 %: all candidates
 
 
-def test_reused_set_keeps_cached_topk_window_and_sink_with_neighbours():
+def test_reused_set_keeps_cached_topk_window_and_sink_with_neighbours(O):
     sink, window = 2, 4
     len0, L = 40, 42
     topk = np.array([5, 9, 20, 33])               # 33 = len0 - window - 3, still a candidate then
@@ -453,7 +462,7 @@ def test_reused_set_keeps_cached_topk_window_and_sink_with_neighbours():
 
 
 # ------------------------------------------------------------ bf16 K_imp storage
-def test_round_to_bf16_closed_forms():
+def test_round_to_bf16_closed_forms(O):
     """Nearest bfloat16 with ties to the even significand (8 significant
     bits: spacing 2^-7 on [1, 2)), rounded once from the exact value."""
     r = O.round_to_bf16
@@ -473,7 +482,7 @@ def test_round_to_bf16_closed_forms():
     assert z[0] == 0 and not np.signbit(z[0]) and np.signbit(z[1])
 
 
-def test_round_to_bf16_equals_library_cast_on_fp32_values():
+def test_round_to_bf16_equals_library_cast_on_fp32_values(O):
     """On values an fp32 holds exactly, rounding once equals the library's
     round-to-nearest-even fp32 -> bf16 conversion."""
     rng = np.random.default_rng(7)
@@ -483,7 +492,7 @@ def test_round_to_bf16_equals_library_cast_on_fp32_values():
     assert np.array_equal(O.round_to_bf16(x.astype(np.float64)), want)
 
 
-def test_bf16_storage_rounds_the_sum_not_the_terms():
+def test_bf16_storage_rounds_the_sum_not_the_terms(O):
     """K = [1, 2^-8], W_K = [[1], [1]]: the exact K_imp 1 + 2^-8 is a tie and
     stores as 1.0; rounding each term (or none) would give 1 + 2^-8."""
     K = np.array([[1.0, 2.0 ** -8]])
@@ -494,7 +503,7 @@ def test_bf16_storage_rounds_the_sum_not_the_terms():
     assert O.project_keys(K2, W, "bf16")[0, 0] == 1.0 + 2.0 ** -7
 
 
-def test_bf16_storage_decides_the_selection_in_decode_layer():
+def test_bf16_storage_decides_the_selection_in_decode_layer(O):
     """Two candidates whose exact scores differ by less than half a bf16 step
     tie after storage, and the tie goes to the lower index (R8): the stored
     precision must reach the selection."""
@@ -515,7 +524,7 @@ def test_bf16_storage_decides_the_selection_in_decode_layer():
 
 
 # ------------------------------------------------------------ sequence sharding (R19)
-def test_merge_partials_equals_attention_over_the_union():
+def test_merge_partials_equals_attention_over_the_union(O):
     """Splitting a set into disjoint parts and merging the parts' outputs by
     their log-sum-exp is attention over the whole set (softmax identity)."""
     rng = np.random.default_rng(19)
@@ -532,7 +541,7 @@ def test_merge_partials_equals_attention_over_the_union():
     assert np.allclose(o2, o, atol=1e-14) and math.isclose(lse2, lse, rel_tol=1e-15)
 
 
-def test_merge_partials_special_cases():
+def test_merge_partials_special_cases(O):
     o = np.arange(4.0)
     got, lse = O.merge_partials([o], [1.5])                       # one part: itself
     assert np.array_equal(got, o) and lse == 1.5
@@ -546,7 +555,7 @@ def test_merge_partials_special_cases():
 
 
 @pytest.mark.parametrize("group", [False, True])
-def test_sharded_decode_equals_unsharded(group):
+def test_sharded_decode_equals_unsharded(O, group):
     rng = np.random.default_rng(23)
     B, Hq, Hkv, L, D, dimp, G = 2, 4, 2, 700, 32, 8, 1
     q, K, V, W, qimp = _layer_inputs(rng, B, Hq, Hkv, L, D, dimp, G)
