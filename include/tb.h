@@ -271,7 +271,7 @@ TB_API tb_status tb_bind_selection_cache(tb_ctx* ctx, int layer, void* cache, si
 TB_API tb_status tb_set_reuse(tb_ctx* ctx, float tau, int interval, int radius);
 
 /* Copy the selection masks of the last sparse tb_decode_step, [B][rows][max_len/32]
- * uint32 (rows: Hq, or Hkv with TB_BUTLER_GROUP), into a caller device buffer
+ * uint32 (rows: Hq, Hkv with TB_BUTLER_GROUP, 1 with TB_SOFTVOTE), into a caller device buffer
  * of >= `bytes` bytes (stream-ordered; words past ceil(len/32) are stale). */
 TB_API tb_status tb_copy_step_masks(tb_ctx* ctx, uint32_t* dst, size_t bytes, void* stream);
 
@@ -297,9 +297,14 @@ TB_API tb_status tb_selftest_bounded_wait(tb_ctx* ctx, long long cycles, int arr
  *   - `cache` describes the caller's K/V caches and lengths (host array);
  *     q, mask, mask_mode, out and lse are as for tb_sparse_attn.
  *   - TB_ERR_CAPACITY when the partials of the request (B * Hq * splits *
- *     (D + 2) floats) would not fit in the static array; nothing is launched.
+ *     (D + 2) floats) would not fit in the static array; TB_ERR_SHAPE when
+ *     B * Hkv * max_len >= 2^31 or B * Hq * max_len >= 2^40 (the limits of a
+ *     context); nothing is launched in either case.  The split count is the
+ *     one tb_sparse_attn picks for the same lengths.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept until the process exits: after cudaDeviceReset of
+ *     a device, do not call this entry point on that device again.
  *   - All calls share the array and it keeps the last call's contents; calls
  *     that overlap on the GPU (several streams or threads) race on it.
  *   - It allocates nothing and calls no allocating routine. */

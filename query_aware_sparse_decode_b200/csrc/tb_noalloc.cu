@@ -17,7 +17,10 @@
 // partial before the merge reads it).  Calls that overlap on the GPU (other
 // streams, other host threads) race on it.  The device address of the array
 // is looked up once per device, on the first call made with that device
-// current; make that first call before any stream capture.
+// current; make that first call before any stream capture.  The address is
+// kept for the life of the process: after cudaDeviceReset (which unloads the
+// library's device code) it no longer names the array, so a process that
+// resets a device must not call this entry point on it again.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -25,6 +28,7 @@
 #include <mutex>
 
 #include "kernels/attn.cuh"
+#include "kernels/attn_split.cuh"
 #include "tb.h"
 
 using namespace tb;
@@ -65,6 +69,10 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
   const int gs = Hq / Hkv;
   if ((gs != 1 && gs != 2 && gs != 4 && gs != 8) || (D != 64 && D != 128)) return TB_ERR_UNSUPPORTED;
   if (max_len < 256 || max_len % 256) return TB_ERR_SHAPE;
+  // the gather lists hold 32-bit cache row numbers, and score-sized row
+  // offsets must fit 40 bits: the same limits as a context's configuration
+  if ((long long)B * Hkv * max_len >= (1LL << 31)) return TB_ERR_SHAPE;
+  if ((long long)B * Hq * max_len >= (1LL << 40)) return TB_ERR_SHAPE;
   if (cache->kv_dtype != TB_BF16 && cache->kv_dtype != TB_F32) return TB_ERR_INVALID_ARG;
   if (mask_mode != TB_MASK_PER_HEAD && mask_mode != TB_MASK_SHARED && mask_mode != TB_MASK_DENSE &&
       mask_mode != TB_MASK_GROUP)
@@ -81,12 +89,9 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
   tb_status s = scratch_for_current_device(&scratch, &num_sms);
   if (s != TB_OK) return s;
 
-  // the same chunking rule as tb_sparse_attn: about two waves of two CTAs per SM
-  const int groups = B * Hkv;
-  const int want_split = std::min(kMaxSplits, std::max(1, (4 * num_sms) / groups));
-  int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
-  chunk = std::max(256, (chunk + 255) / 256 * 256);
-  const int nsplit = std::max(1, (maxL + chunk - 1) / chunk);
+  // the chunking rule of tb_sparse_attn (attn_split)
+  int chunk = 0, nsplit = 0;
+  if (!attn_split(num_sms, B * Hkv, maxL, &chunk, &nsplit)) return TB_ERR_UNSUPPORTED;
   const size_t part_o_floats = (size_t)B * Hq * nsplit * D;
   const size_t part_ml_floats = (size_t)B * Hq * nsplit * 2;
   if ((part_o_floats + part_ml_floats) * sizeof(float) > kStaticScratchBytes) return TB_ERR_CAPACITY;
@@ -115,13 +120,15 @@ extern "C" TB_API tb_status tb_sparse_attn_static(const tb_cache_view* cache, co
     if (cache->kv_dtype == TB_BF16) {                                                         \
       auto k = attn_bf16_kernel<DV, GSV>;                                                     \
       const int smem = attn_bf16_smem_bytes<DV>();                                            \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);             \
-      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                          \
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+        return TB_ERR_CUDA;                                                                   \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                   \
     } else {                                                                                  \
       auto k = attn_f32_kernel<DV, GSV>;                                                      \
       const int smem = attn_f32_smem_bytes<DV>();                                             \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);             \
-      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                          \
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+        return TB_ERR_CUDA;                                                                   \
+      launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                   \
     }                                                                                         \
   } else
   TB_STATIC_ATTN_CASE(128, 4) TB_STATIC_ATTN_CASE(128, 2) TB_STATIC_ATTN_CASE(128, 1) TB_STATIC_ATTN_CASE(128, 8)

@@ -3,8 +3,9 @@
 It serves callers that cannot allocate device memory (fixed-budget serving
 loops, plug-ins in a host process that owns all device memory): it needs no
 context and no workspace because its split partials live in a static device
-array inside the library.  Its results must match tb_sparse_attn's, call
-after call, and requests too large for the static array must be refused.
+array inside the library.  Its results must match the oracle's attention
+over the same sets and tb_sparse_attn's, call after call, and requests too
+large for the static array or for 32-bit cache rows must be refused.
 This file is collected last so that a failure here leaves every other test
 already run."""
 import math
@@ -52,11 +53,20 @@ def test_static_attention_matches_context_attention_twice(mode):
         got.append((out, lse))
     torch.cuda.synchronize()
     r, rl = ref.float().cpu().numpy(), ref_lse.cpu().numpy()
+    # the oracle's attention over the same sets (every token for the dense mode)
+    sets = _sets(ld, wl) if mode == TB.TB_MASK_PER_HEAD else None
+    scale = 1.0 / math.sqrt(wl.D)
+    gs = wl.Hq // wl.Hkv
     for out, lse in got:
         o, l = out.float().cpu().numpy(), lse.cpu().numpy()
-        for b in range(wl.B):
-            assert_close_rows(o[b], r[b], "bf16", f"static b{b}")
+        for b, L in enumerate(wl.seq_lens):
+            assert_close_rows(o[b], r[b], "bf16", f"static vs context b{b}")
             assert np.all(np.abs(l[b] - rl[b]) <= 1e-3 * np.maximum(1.0, np.abs(rl[b])))
+            for h in range(wl.Hq):
+                idx = sets[b, h] if sets is not None else np.arange(L)
+                want, want_lse = O.attend(ld.q[b, h], ld.K[b, h // gs, :L], ld.V[b, h // gs, :L], idx, scale)
+                assert_close_rows(o[b, h][None], want[None], "bf16", f"static vs oracle b{b} h{h}")
+                assert abs(l[b, h] - want_lse) <= 1e-3 * max(1.0, abs(want_lse))
 
 
 def test_static_attention_refuses_requests_beyond_its_scratch():
@@ -71,3 +81,18 @@ def test_static_attention_refuses_requests_beyond_its_scratch():
     st = TB.lib().tb_sparse_attn_static(TB.ctypes.byref(view), TB.ctypes.c_void_p(small.data_ptr()), None,
                                         TB.TB_MASK_DENSE, TB.ctypes.c_void_p(out.data_ptr()), None, None)
     assert st == 3  # TB_ERR_CAPACITY
+
+
+def test_static_attention_refuses_more_cache_rows_than_32_bits_hold():
+    # B * Hkv * max_len >= 2^31: the gather lists hold 32-bit cache rows, so
+    # the request is refused before any launch (a context refuses it too)
+    B, Hq, Hkv, D, max_len = 128, 8, 8, 128, 1 << 21
+    assert B * Hkv * max_len >= 1 << 31
+    small = torch.zeros(16, dtype=torch.bfloat16, device="cuda")  # never read
+    k = small.as_strided((B, Hkv, max_len, D), (0, 0, 0, 0))
+    out = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    arr = (TB.ctypes.c_int32 * B)(*([10] * B))
+    view = TB.CacheView(k.data_ptr(), k.data_ptr(), B, Hq, Hkv, D, max_len, TB.TB_BF16, arr)
+    st = TB.lib().tb_sparse_attn_static(TB.ctypes.byref(view), TB.ctypes.c_void_p(small.data_ptr()), None,
+                                        TB.TB_MASK_DENSE, TB.ctypes.c_void_p(out.data_ptr()), None, None)
+    assert st == 2  # TB_ERR_SHAPE
