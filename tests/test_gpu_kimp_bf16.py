@@ -8,7 +8,9 @@ exact value: those elements may hold the neighbouring bfloat16 value
 (harness.bf16_kimp_bounds), and scores over them may move by that step
 times |q_j| (harness.bf16_score_slack).  Everything else is compared as for
 the fp32 cache: scores within fp32 accumulation, sets within the tie band,
-outputs where the sets agree."""
+outputs against the oracle's attention over the GPU's set."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -132,10 +134,11 @@ def _decode(wl, group):
             slack = bf16_score_slack(qabs, K[b, g, :L], ld.W)
             assert tie_band_ok(got[b, r], sel[b, h], sc[b, h], L, wl.keep_pct, wl.sink, wl.window, slack), \
                 f"b{b} h{h}"
+            want = ref[b, h]
             if not np.array_equal(got[b, r], sel[b, h]):
                 mism += 1
-                continue
-            assert_close_rows(o[b, h][None], ref[b, h][None], wl.dtype, f"b{b} h{h}")
+                want, _ = O.attend(ld.q[b, h], K[b, g, :L], V[b, g, :L], got[b, r], 1.0 / math.sqrt(wl.D))
+            assert_close_rows(o[b, h][None], want[None], wl.dtype, f"b{b} h{h}")
     assert mism <= max(1, wl.B * wl.Hq // 20)
 
 

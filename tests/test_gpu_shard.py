@@ -2,9 +2,12 @@
 holding a contiguous token range of the same layer, run in lock step
 (shard.run_lockstep; no kernel of one rank waits on another's).  The merged
 step must select the oracle's set (decode_layer_sharded: the one-device
-set) within the tie band, give its output where the sets agree, and, with
+set) within the tie band, give the oracle's attention over the selected set
+(the GPU's own set where the two differ inside the band), and, with
 identical K_imp rows, select exactly what the one-context step selects.
-The oracle never sees a GPU value."""
+The oracle never sees a GPU value other than a selected index set."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -150,10 +153,12 @@ def _run(wl, starts, variant=TB.TB_BUTLER, periodic=None, kimp_dtype="f32", page
                 slack = bf16_score_slack(qabs, K[b, g, :L], ld.W)
             assert tie_band_ok(got[b, r], sel[b, h], sc[b, h], L, wl.keep_pct, wl.sink, wl.window, slack), \
                 f"b{b} h{h}"
+            want = ref[b, h]
             if not np.array_equal(got[b, r], sel[b, h]):
                 mism += 1
-                continue
-            assert_close_rows(o[b, h][None], ref[b, h][None], wl.dtype, f"b{b} h{h}")
+                g = h // gs
+                want, _ = O.attend(ld.q[b, h], K[b, g, :L], V[b, g, :L], got[b, r], 1.0 / math.sqrt(wl.D))
+            assert_close_rows(o[b, h][None], want[None], wl.dtype, f"b{b} h{h}")
     assert mism <= max(1, wl.B * wl.Hq // 20)
     return got, sel, same_kimp
 
