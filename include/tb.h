@@ -180,6 +180,15 @@ TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const v
  * result rounded to nearest even. */
 TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, void* stream);
 
+/* a1' for layers [first_layer, first_layer + n_layers) at once (same rows
+ * [start, start + count) of each): with dense bf16 caches one persistent
+ * tensor-core launch covers every layer's tiles (a prefill of all layers
+ * streams K at the HBM rate instead of paying one short launch per layer);
+ * fp32 or paged caches run tb_project_kimp layer by layer.  Each result
+ * equals tb_project_kimp's bit for bit. */
+TB_API tb_status tb_project_kimp_layers(tb_ctx* ctx, int first_layer, int n_layers, int start, int count,
+                                        void* stream);
+
 /* a2 + a3 — model card "Method": scores[b][h][t] = q_hat[b][h] . K_imp[b][g(h)][t]
  * for t < len[b], with q_hat[b][h] = q_imp_producer[b*Hq + h][(layer-1) mod G][0][:]
  * (fp32 FMA on the stored K_imp values, no scale).  `q_imp_producer`: [(B*Hq)][G][1][d'] of producer
@@ -212,6 +221,17 @@ TB_API tb_status tb_select(tb_ctx* ctx, int layer, const float* scores, int rows
  * an fp32 log-sum-exp merge; each K/V row is read once per KV head. */
 TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uint32_t* mask, int mask_mode,
                                 void* out, float* lse, void* stream);
+
+/* a6 with the selected sets as index lists, the shape tb_select writes:
+ * idx [B][Hq][idx_cap] int32 token indices (each listed once; any order),
+ * count [B][Hq] int32 (device).  The lists are turned into per-head
+ * bitmasks in the context's workspace (what tb_copy_step_masks copies is
+ * then these sets), then tb_sparse_attn runs in TB_MASK_PER_HEAD mode: the
+ * same result as tb_sparse_attn on the equivalent mask.  An index outside
+ * [0, len) is skipped, a count outside [0, idx_cap] is clamped, and either
+ * sets TB_DEV_ERR_INDEX. */
+TB_API tb_status tb_sparse_attn_idx(tb_ctx* ctx, int layer, const void* q, const int32_t* idx, int idx_cap,
+                                    const int32_t* count, void* out, float* lse, void* stream);
 
 /* a1..a6 for one layer: append, then (dense layer or 100 % budget) dense
  * attention, else score, select and sparse attention (TB_BUTLER per head,

@@ -5,15 +5,21 @@
 // GEMM with M = cached rows (tiles of 128), N = d' (32 or 16), K = D (128 or
 // 64), bf16 operands and fp32 accumulation in tensor memory.
 //   warp 0      TMA producer: K tiles (128 rows x 64 columns per box, 128B
-//               swizzle) into a 4-stage shared-memory ring of this CTA only.
+//               swizzle) into a 4-stage shared-memory ring of this CTA only;
+//               it also writes each layer's W_K^T (N x K, K-major) into one
+//               of two shared buffers in the 128B-swizzled canonical layout.
 //   warp 1      one thread issues tcgen05.mma (kind::f16, M=128) per 16-wide
 //               K step and commits to the ring's "empty" and the
 //               accumulator's "full" mbarriers.
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x d' columns each (one row per
 //               thread) and plain 128-byte row stores of fp32 K_imp.
 // Two accumulators in tensor memory let the epilogue of tile j overlap the
-// MMAs of tile j + 1.  W_K^T (N x K, K-major) is written into shared memory
-// once per CTA in the same 128B-swizzled canonical layout.
+// MMAs of tile j + 1.  One launch may cover several layers (a persistent grid
+// over every layer's tiles, layer by layer within a CTA, one tensor map per
+// layer): W_K^T is double-buffered, the producer refills a buffer once the
+// MMA issuer's commit says the MMAs of the layer before last are done, and
+// the MMA issuer waits for a layer's buffer before its first MMA, so a layer
+// change costs no pipeline drain.
 // Every mbarrier wait is bounded; a timeout sets TB_DEV_ERR_TIMEOUT and the
 // CTA winds down (tensor memory is always released).
 #pragma once
@@ -26,12 +32,15 @@ constexpr int kTcStages = 4;
 constexpr int kTcRows = 128;
 constexpr int kTcThreads = 192;
 
+constexpr int kTcMaxLayers = TB_MAX_LAYERS;
+
 struct ProjectTcParams {
-  const void* w_k;  // [D][d'] bf16
-  void* kimp;       // [B][Hkv][max_len/256][d'][256] (kimp_index), fp32 or bf16
+  CUtensorMap kmap[kTcMaxLayers];  // per layer: K rows [B*Hkv*max_len][D], 64-column boxes of 128 rows
+  const void* w_k[kTcMaxLayers];   // per layer: [D][d'] bf16
+  void* kimp[kTcMaxLayers];        // per layer: [B][Hkv][max_len/256][d'][256] (kimp_index), fp32 or bf16
   uint32_t* status;
   int max_len, start, count;
-  int tiles_per_slab, total_tiles;
+  int tiles_per_slab, tiles_per_layer, total_tiles, n_layers;
   int kimp_bf16;    // store K_imp rounded to bf16
 };
 
@@ -95,12 +104,13 @@ __device__ __forceinline__ void tmem_ld_row<16>(uint32_t taddr, float (&v)[16]) 
 
 template <int D>
 constexpr int project_tc_smem_bytes() {
-  return 1024 + kTcStages * kTcRows * D * 2 + 1024 * (D / 64) /*W^T atoms: <= 32 rows x 128 B each*/ * 4 + 256;
+  return 1024 + kTcStages * kTcRows * D * 2 + 2 * 4096 * (D / 64) /*two W^T buffers of <= 32 rows x 128 B per atom*/ +
+         256;
 }
 
 template <int D, int DIMP>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    project_tc_kernel(const __grid_constant__ CUtensorMap kmap, const ProjectTcParams p) {
+    project_tc_kernel(const __grid_constant__ ProjectTcParams p) {
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(DIMP == 16 || DIMP == 32, "importance dim");
   constexpr int ATOMS = D / 64;                       // 128-byte swizzle atoms along K
@@ -116,13 +126,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* A = smem;
-  uint8_t* Bt = smem + kTcStages * A_STAGE;
+  uint8_t* Bt = smem + kTcStages * A_STAGE;  // two W^T buffers of ATOMS * 4096 bytes
   static_assert(B_ATOM <= 4096, "W^T atom");
-  uint64_t* full = reinterpret_cast<uint64_t*>(Bt + ATOMS * 4096);
+  uint64_t* full = reinterpret_cast<uint64_t*>(Bt + 2 * ATOMS * 4096);
   uint64_t* empty = full + kTcStages;
   uint64_t* accf = empty + kTcStages;
   uint64_t* acce = accf + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* wfull = acce + 2;   // W^T buffer written (producer arrives)
+  uint64_t* wfree = wfull + 2;  // MMAs reading a W^T buffer completed (MMA commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfree + 2);
   __shared__ int s_abort_store, s_issued_store, s_consumed_store;
   volatile int* s_abort = &s_abort_store;      // set by any role, polled by all
   volatile int* s_issued = &s_issued_store;    // TMA loads issued (producer)
@@ -139,6 +151,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], 4);
+      mbar_init(&wfull[a], 1);
+      mbar_init(&wfree[a], 1);
     }
     mbar_fence_init();
     *s_abort = 0;
@@ -151,17 +165,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  {
-    const __nv_bfloat16* W = reinterpret_cast<const __nv_bfloat16*>(p.w_k);
-    for (int e = tid; e < D * DIMP; e += kTcThreads) {
-      const int k = e / DIMP, n = e % DIMP;  // W[k][n] -> W^T[n][k]
-      const int atom = k / 64, kc = k % 64;
-      const int chunk = kc / 8;
-      uint8_t* dst = Bt + atom * 4096 + n * 128 + ((chunk ^ (n & 7)) << 4) + (kc % 8) * 2;
-      *reinterpret_cast<__nv_bfloat16*>(dst) = W[e];
-    }
-  }
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -170,10 +173,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ntiles = p.total_tiles > (int)blockIdx.x
                          ? (p.total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
                          : 0;
-  // tile j of this CTA: K rows [t0, t0 + valid) of slab (b * Hkv + g); row0 is
-  // the same row in the flattened [B*Hkv*max_len][D] view used by TMA
+  // tile j of this CTA: K rows [t0, t0 + valid) of slab (b * Hkv + g) of
+  // layer `layer`; row0 is the same row in the flattened [B*Hkv*max_len][D]
+  // view used by TMA.  A CTA's tiles come layer by layer.
+  auto layer_of = [&](int j) { return (int)((blockIdx.x + (long long)j * gridDim.x) / p.tiles_per_layer); };
   auto tile_of = [&](int j, int& row0, int& valid, int& slab, int& t0) {
-    const int i = blockIdx.x + j * gridDim.x;
+    const int i = (int)((blockIdx.x + (long long)j * gridDim.x) % p.tiles_per_layer);
     slab = i / p.tiles_per_slab;
     const int tt = i % p.tiles_per_slab;
     t0 = p.start + tt * kTcRows;
@@ -181,27 +186,77 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     valid = min(kTcRows, p.count - tt * kTcRows);
   };
 
-  if (warp == 0) {
-    if (lane == 0) {  // ---- TMA producer
-      for (int j = 0; j < ntiles && !*s_abort; ++j) {
-        const int st = j % kTcStages;
-        if (!mbar_wait(&empty[st], ((j / kTcStages) & 1) ^ 1)) {
+  if (warp == 0) {  // ---- producer warp: W^T buffers (all lanes), TMA loads (lane 0)
+    int cur = -1, li = -1;  // current layer, its index among this CTA's layers
+    for (int j = 0; j < ntiles; ++j) {
+      if (__any_sync(0xffffffffu, *s_abort != 0)) break;
+      const int layer = layer_of(j);
+      if (layer != cur) {  // this CTA's next layer: fill W^T buffer li & 1
+        cur = layer;
+        ++li;
+        const int s = li & 1;
+        bool ok = li < 2 || mbar_wait(&wfree[s], ((li - 2) >> 1) & 1);  // MMAs of layer li - 2 done
+        if (__any_sync(0xffffffffu, !ok)) {
           *s_abort = 1;
           break;
         }
-        int row0, valid, slab, t0;
-        tile_of(j, row0, valid, slab, t0);
-        mbar_expect_tx(&full[st], A_STAGE);
+        // W [D][d'] bf16 (16-byte aligned): all of a lane's 16-byte pieces are
+        // requested before any is stored, then each piece's eight elements
+        // W[k][n..n+7] go to rows n..n+7 of W^T[n][k]
+        const uint4* W = reinterpret_cast<const uint4*>(p.w_k[layer]);
+        uint8_t* Bs = Bt + s * ATOMS * 4096;
+        constexpr int PIECES = D * DIMP / 8 / 32;  // per lane
+        uint4 w[PIECES];
 #pragma unroll
-        for (int a = 0; a < ATOMS; ++a) tma_load_2d(A + st * A_STAGE + a * A_ATOM, &kmap, a * 64, row0, &full[st]);
-        *s_issued = j + 1;
+        for (int i = 0; i < PIECES; ++i) w[i] = __ldg(W + lane + 32 * i);
+#pragma unroll
+        for (int i = 0; i < PIECES; ++i) {
+          const int e0 = 8 * (lane + 32 * i);
+          const int k = e0 / DIMP, n0 = e0 % DIMP;
+          const int atom = k / 64, kc = k % 64, chunk = kc / 8;
+          const uint32_t wd[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int n = n0 + q;
+            const uint16_t bits = (uint16_t)(wd[q >> 1] >> (16 * (q & 1)));
+            *reinterpret_cast<uint16_t*>(Bs + atom * 4096 + n * 128 + ((chunk ^ (n & 7)) << 4) + (kc % 8) * 2) = bits;
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cta(&wfull[s]);
       }
+      if (lane == 0) {
+        const int st = j % kTcStages;
+        if (!mbar_wait(&empty[st], ((j / kTcStages) & 1) ^ 1)) {
+          *s_abort = 1;
+        } else {
+          int row0, valid, slab, t0;
+          tile_of(j, row0, valid, slab, t0);
+          mbar_expect_tx(&full[st], A_STAGE);
+#pragma unroll
+          for (int a = 0; a < ATOMS; ++a)
+            tma_load_2d(A + st * A_STAGE + a * A_ATOM, &p.kmap[layer], a * 64, row0, &full[st]);
+          *s_issued = j + 1;
+        }
+      }
+      __syncwarp();
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer
-      int last = -1;
+      int last = -1, cur = -1, li = -1;
       for (int j = 0; j < ntiles && !*s_abort; ++j) {
         const int st = j % kTcStages, acc = j & 1;
+        const int layer = layer_of(j);
+        if (layer != cur) {  // first tile of this CTA's next layer
+          if (li >= 0) umma_commit(&wfree[li & 1]);  // buffer of the previous layer free once its MMAs complete
+          cur = layer;
+          ++li;
+          if (!mbar_wait(&wfull[li & 1], (li >> 1) & 1)) {
+            *s_abort = 1;
+            break;
+          }
+        }
         if (!mbar_wait(&full[st], (j / kTcStages) & 1)) {
           *s_abort = 1;
           break;
@@ -212,7 +267,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(A + st * A_STAGE), b0 = smem_u32(Bt);
+        const uint32_t a0 = smem_u32(A + st * A_STAGE), b0 = smem_u32(Bt + (li & 1) * ATOMS * 4096);
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           const uint32_t off = (kk / 4) * A_ATOM + (kk % 4) * 32;
@@ -244,16 +299,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) mbar_arrive_cta(&acce[acc]);
       int row0, valid, slab, t0;
       tile_of(j, row0, valid, slab, t0);
+      const int layer = layer_of(j);
       const int r = quarter * 32 + lane;
       if (r < valid) {
         // for each column the warp writes 32 consecutive tokens of one tile
         const size_t dst = kimp_index(slab, 0, t0 + r, DIMP, p.max_len);
         if (p.kimp_bf16) {
-          __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(p.kimp) + dst;
+          __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(p.kimp[layer]) + dst;
 #pragma unroll
           for (int c = 0; c < DIMP; ++c) k16[c * kKimpTile] = __float2bfloat16_rn(v[c]);
         } else {
-          float* k32 = reinterpret_cast<float*>(p.kimp) + dst;
+          float* k32 = reinterpret_cast<float*>(p.kimp[layer]) + dst;
 #pragma unroll
           for (int c = 0; c < DIMP; ++c) k32[c * kKimpTile] = v[c];
         }

@@ -12,8 +12,9 @@
 // group's query values broadcast from shared memory) so that many loads per
 // thread can be in flight.  The FMAs run on pairs of consecutive tokens
 // (fma.rn.f32x2: two independent round-to-nearest fp32 FMAs, the bits of two
-// fmaf).  A CTA covers 1, 2 or 4 steps of 256 threads' tokens
-// (the launch picks the count so the grid fills the SMs).
+// fmaf).  A CTA covers `chunk` consecutive tokens (a multiple of 32, up to
+// `iters` steps of 256 threads' tokens; the launch uses 1, 2 or 4 whole
+// steps, picking the count so that the grid fills the SMs).
 // With GROUPED (one selection per KV group) the group's per-head fp32 scores
 // are added in head order and one row per (b, g) is written instead.
 // Optionally each CTA accumulates, per output row, the histogram of the
@@ -38,7 +39,8 @@ struct ScoreParams {
   uint32_t* hist;      // [B*Hq][2048] or nullptr
   int G, slot, Hq, Hkv, max_len;
   int sink, window;
-  int iters;           // CTA iterations of score_step<KT>() tokens (1, 2 or 4)
+  int chunk;           // tokens per CTA, a multiple of 32
+  int iters;           // ceil(chunk / score_step<KT>()) iterations
   const uint32_t* reuse;  // [B*rows] amortised selection: rows that skip scoring, or null
   int lens[kMaxBatch];
 };
@@ -81,8 +83,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   extern __shared__ uint32_t hist[];  // [NR][2048] when HIST
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.lens[b];
-  const int t_base = chunk * STEP * p.iters;
+  const int t_base = chunk * p.chunk;
   if (t_base >= L) return;
+  const int t_end = min(t_base + p.chunk, L);  // this CTA's tokens: [t_base, t_end)
   if (p.reuse != nullptr) {  // every row of this group reuses its cached selection: nothing to score
     const size_t r0 = GROUPED ? (size_t)b * p.Hkv + g : (size_t)b * p.Hq + g * GS;
     bool all = true;
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
 #pragma unroll 1
   for (int it = 0; it < p.iters; ++it) {
     const int t0 = t_base + it * STEP + TPT * tid;
-    if (t0 < L) {
+    if (t0 < t_end) {
       const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t0, DIMP, p.max_len);
       uint64_t acc2[GS][TPT / 2];  // token pairs (2u, 2u + 1)
 #pragma unroll

@@ -65,6 +65,9 @@ struct SelectParams {
   const int32_t* sc_len;  // [B*rows] length of the cached selection
   uint32_t* sc_mask;      // [B*rows][mask_words] cached masks (refilled by fresh rows)
   int reuse_radius;
+  // cluster selection (select_cluster_kernel) only
+  uint32_t* ctot;         // [B*rows][2048 + 1024] the cluster's digit-2 and digit-3 totals (zero between selections)
+  uint32_t* cslot;        // [B*rows][32] per-CTA tie counts (0..15) and kept counts (16..31)
   int lens[kMaxBatch];
 };
 

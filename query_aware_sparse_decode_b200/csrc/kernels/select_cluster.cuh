@@ -1,0 +1,517 @@
+// butler_topk + butler_merge in one launch: the selection of a row by a
+// thread-block cluster (model card "Meta-Llama-3.1-8B-Instruct-Butler",
+// section "Method": top-x subset under a fixed token budget plus a sink
+// prefix and a recent local window; section "Memory requirements":
+// fixed_<N>pc, min_sparse_index, sliding_window).
+//
+//   k = floor(P * L / 100), candidates C = [sink, L - window),
+//   Sel = [0, min(sink, L)) U top_min(k, |C|)(C) U [max(L - window, 0), L),
+//   order (score desc, index asc), -0.0 == +0.0.
+//
+// A cluster of NC CTAs (NC in 1..16) owns one row; CTA c owns the tokens
+// [c * chunk, (c + 1) * chunk).  Scores are compared as monotone uint32 order
+// keys and the k-th largest key T is found digit by digit (11 + 11 + 10
+// bits).  The row's scores are read from L2 once:
+//   1. digit 1 comes from the first-digit histogram that the score kernel
+//      (or select_hist_kernel) built; every CTA finds the threshold bin b1
+//      while its first score loads are in flight.
+//   2. one pass over the CTA's tokens (16-byte loads, batches of four per
+//      thread double-buffered in registers; scores compared as floats with
+//      the bin's bounds) writes, per 32-token word, "kept for sure" (sink,
+//      window, keys above bin b1) into a shared copy of the CTA's mask words,
+//      and appends the keys of bin b1 (a few percent of the row) to a shared
+//      list while histogramming their second digit.
+//   3. each CTA adds its histogram into the row's total in L2 (atomics);
+//      after a cluster barrier every CTA reads the total back: digit 2, then
+//      digit 3 over the list the same way, give T and the number `quota` of
+//      keys equal to T that are kept.
+//   4. ties at T go to the lowest indices.  When every key equal to T is
+//      kept (the usual case) each CTA keeps its own; otherwise each CTA posts
+//      its count, and after a barrier CTA c keeps the first
+//      clamp(quota - (ties on CTAs < c), 0, its ties) of its own, found by an
+//      ordered scan over a shared tie bitmap.
+//   5. list keys above T and the kept ties are OR-ed into the shared mask
+//      words, which are written once.  The kept counts are added up in L2;
+//      the last CTA to finish (a ticket counter) checks the total, writes the
+//      optional count and clears the row's first-digit histogram and totals,
+//      so the next selection needs no zeroing pass.  With an index list the
+//      counts are posted per CTA instead and a barrier gives every CTA its
+//      offset.
+// The cluster barriers (barrier.cluster arrive/release, wait/acquire) are the
+// only waits between CTAs, and every value they exchange goes through L2; no
+// CTA waits on a flag.  A CTA whose list overflows re-reads its tokens from
+// L2 for steps 3-5 instead; the result is the same.  Rows that keep none or
+// all of their candidates, and rows reusing a cached selection, write their
+// words directly.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "reuse.cuh"
+#include "select.cuh"
+
+namespace tb {
+
+constexpr int kClThreads = 256;
+constexpr int kClWarps = kClThreads / 32;
+constexpr int kClChunkMax = 65536;            // tokens per CTA
+constexpr int kClWordsMax = kClChunkMax / 32;  // mask words per CTA
+constexpr int kClListCap = 4096;              // keys of the threshold bin kept in shared memory
+constexpr int kClMaxCluster = 16;
+constexpr int kClHist3 = 1024;                // bins of the 10-bit last digit
+constexpr int kClBatch = 4;                   // 16-byte loads per thread and batch of the first pass
+constexpr int kClTotWords = kHistBins + kClHist3 + 2;  // per row in ctot: totals, kept count, CTA ticket
+constexpr int kClSlotWords = 2 * kClMaxCluster;    // per row in cslot
+
+struct ClusterSelectSmem {
+  uint32_t mword[kClWordsMax];      // the CTA's mask words
+  uint32_t tbits[kClWordsMax];      // keys equal to T among the CTA's tokens
+  uint2 list[kClListCap];           // (key, token - c0) of the threshold bin's keys
+  uint32_t hist[kHistBins];         // this CTA's digit-2 (then digit-3) histogram
+  uint32_t tot[kHistBins];          // a cluster total read back from L2
+  uint32_t scan[32];
+  uint32_t n_list, pre_ties, ntie_all, last;
+  int bin;
+  uint32_t above;
+};
+constexpr int kClSmem = (int)sizeof(ClusterSelectSmem);
+
+// Host: cluster size and chunk of a selection over rows of at most maxL
+// tokens, `nrows` rows in all.  max_active[i] is how many clusters of 2^i
+// CTAs (1..16) can be resident at once (0: not launchable).  Among the sizes
+// whose CTAs cover a row (nc * kClChunkMax >= L): the largest that keeps all
+// rows' clusters resident in one wave, with at most about four CTAs per SM
+// and at least 256 tokens per CTA; else the smallest covering size that is
+// resident in one wave; else the smallest covering size.  Returns false when
+// no size covers the row.
+inline bool cluster_select_shape(int num_sms, long long nrows, int maxL, const int (&max_active)[5], int* nc_out,
+                                 int* chunk_out) {
+  const long long L = maxL > 1 ? maxL : 1;
+  int pick = 0, one_wave = 0, cover = 0;
+  for (int i = 0; i < 5; ++i) {
+    const int nc = 1 << i;
+    if (max_active[i] < 1 || (long long)nc * kClChunkMax < L) continue;
+    if (!cover) cover = nc;
+    if (nrows > max_active[i]) continue;
+    if (!one_wave) one_wave = nc;
+    if (nrows * nc <= 4LL * num_sms && (L + nc - 1) / nc >= 256) pick = nc;
+  }
+  const int nc = pick ? pick : (one_wave ? one_wave : cover);
+  if (!nc) return false;
+  const long long chunk = ((L + nc - 1) / nc + 255) / 256 * 256;
+  *nc_out = nc;
+  *chunk_out = (int)chunk;
+  return chunk <= kClChunkMax;
+}
+
+// Host: launch with programmatic stream serialization and a cluster of
+// `nc` CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                      int nc, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = nc;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// A cluster total (NB words in L2) read into shared memory, and the bin where
+// the running count from the top reaches k.  A histogram holding fewer than
+// k keys (inconsistent scores, e.g. NaN) records TB_DEV_ERR_COUNT and yields
+// bin 0, so every index stays in bounds.
+template <int NB>
+__device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32_t k, ClusterSelectSmem& sm,
+                                                   uint32_t* status, uint32_t& above) {
+  for (int i = threadIdx.x; i < NB; i += kClThreads) sm.tot[i] = __ldcg(total + i);
+  if (threadIdx.x == 0) {
+    sm.bin = -1;
+    sm.above = 0;
+  }
+  __syncthreads();
+  find_bin<NB / kClThreads, kClThreads>(sm.tot, k, sm.scan, &sm.bin, &sm.above);  // ends with a block barrier
+  const int bin = sm.bin;
+  above = sm.above;
+  if (bin < 0) {
+    if (threadIdx.x == 0) atomicOr(status, TB_DEV_ERR_COUNT);
+    above = 0;
+    return 0u;
+  }
+  return (uint32_t)bin;
+}
+
+// Adds this CTA's histogram into the row's total in L2 (non-empty bins only).
+template <int NB>
+__device__ __forceinline__ void hist_to_total(const uint32_t* hist, uint32_t* total) {
+  for (int i = threadIdx.x; i < NB; i += kClThreads) {
+    const uint32_t v = hist[i];
+    if (v) atomicAdd(total + i, v);
+  }
+}
+
+// Calls f(t, key) for every candidate token t of [a, b) (a a multiple of 4,
+// candidates [lo, hi)), reading the scores with four 16-byte loads per
+// thread in flight.  The row holds max_len >= b scores, a multiple of 256,
+// so every 16-byte load that starts below b stays inside the row.
+template <class F>
+__device__ __forceinline__ void visit_candidates(const float* srow, int a, int b, int lo, int hi, F f) {
+  const int start = max(a, lo) & ~3, end = min(b, hi);
+  for (int base = start; base < end; base += 16 * kClThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t0 = base + 4 * (threadIdx.x + kClThreads * u);
+      v[u] = t0 < end ? __ldcg(reinterpret_cast<const float4*>(srow + t0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t0 = base + 4 * (threadIdx.x + kClThreads * u);
+      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = t0 + j;
+        if (t >= lo && t < end) f(t, order_key(vv[j]));
+      }
+    }
+  }
+}
+
+// grid (NC, rows, B), cluster (NC, 1, 1), kClThreads threads, kClSmem bytes.
+__global__ void __launch_bounds__(kClThreads, 3) select_cluster_kernel(const SelectParams p, int chunk) {
+  pdl_wait();
+  pdl_trigger();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(16) uint8_t cl_raw[];
+  ClusterSelectSmem& sm = *reinterpret_cast<ClusterSelectSmem*>(cl_raw);
+  const int nc = (int)cluster.num_blocks();
+  const int c = (int)cluster.block_rank();
+  const int r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const RowShape rs = row_shape(p, b);
+  const long long row = (long long)b * p.rows_per_seq + r;
+  const int c0 = c * chunk;                    // a multiple of 256: word-aligned
+  const int c1 = min(c0 + chunk, rs.L);
+  const int nw = c1 > c0 ? (c1 - c0 + 31) >> 5 : 0;  // this CTA's words holding tokens < L
+  const bool reused = p.reuse != nullptr && p.reuse[row] != 0u;
+  const bool topk = rs.mode == 2 && !reused;
+  const float* srow = p.scores + row * p.row_stride;
+  uint32_t* tot = p.ctot + row * kClTotWords;   // [2048] digit-2 total, then [1024] digit-3 total
+  uint32_t* slot = p.cslot + row * kClSlotWords;  // [16] tie counts, [16] kept counts
+
+  if (topk) {
+    for (int i = tid; i < nw; i += kClThreads) sm.tbits[i] = 0u;
+    for (int i = tid; i < kHistBins; i += kClThreads) sm.hist[i] = 0u;
+    if (tid == 0) sm.n_list = 0u;
+    // Warp w owns words [wb, we) and walks them in batches of 16 words: lane l
+    // loads the 16 bytes at tokens 32 * (w0 + 4u + l / 8) + 4 * (l % 8),
+    // u = 0..3, so lane group l / 8 holds word w0 + 4u + l / 8.  The next
+    // batch's loads are in flight while this one is processed (two register
+    // batches).
+    const int wpw = (nw + kClWarps - 1) / kClWarps;
+    const int wb = min(warp * wpw, nw), we = min(wb + wpw, nw);
+    float4 va[kClBatch], vb[kClBatch];
+    auto load_batch = [&](float4 (&v)[kClBatch], int w0) {
+#pragma unroll
+      for (int u = 0; u < kClBatch; ++u) {
+        const int w = w0 + 4 * u + (lane >> 3);
+        const int tv = c0 + 32 * w + 4 * (lane & 7);
+        v[u] = (w < we && tv < c1) ? __ldcg(reinterpret_cast<const float4*>(srow + tv))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    if (wb < we) load_batch(va, wb);  // requested first: their latency overlaps the digit-1 search
+    // ---- digit 1 from the row's first-digit histogram; the bin's bounds as floats
+    uint32_t above;
+    const uint32_t b1 = total_find_bin<kHistBins>(p.hist1 + row * kHistBins, (uint32_t)rs.k, sm, p.status, above);
+    const uint32_t kleft = (uint32_t)rs.k - above;
+    const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
+    const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
+    const float f_hi = hi_open ? 0.f : key_to_float((b1 + 1u) << 21);       // smallest key above it
+    // ---- one pass over the CTA's tokens: sure-keep words, the bin's keys, digit-2 histogram.
+    // Float comparisons against the bin's bounds decide the same as the keys
+    // (the key map is monotone and folds -0.0 onto +0.0, as IEEE comparison
+    // does).  A lane's bin members of a batch (bit 4u + j: its load u,
+    // element j) are appended with one warp scan and one shared atomic.
+    auto process = [&](const float4 (&v)[kClBatch], int w0) {
+      const bool interior =
+          w0 + 4 * kClBatch <= we && c0 + 32 * w0 >= rs.lo && c0 + 32 * (w0 + 4 * kClBatch) <= min(rs.hi, c1);
+      uint32_t memb = 0;  // bit 4u + j
+#pragma unroll
+      for (int u = 0; u < kClBatch; ++u) {
+        const int w = w0 + 4 * u + (lane >> 3);
+        const int tv = c0 + 32 * w + 4 * (lane & 7);
+        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t keep = 0, mb = 0;
+        if (interior) {  // every token a valid candidate
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            keep |= (uint32_t)(vv[j] >= f_hi) << j;
+            mb |= (uint32_t)(vv[j] >= f_lo) << j;
+          }
+          if (hi_open) keep = 0;
+          mb &= ~keep;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = tv + j;
+            const bool valid = w < we && t < c1;
+            const bool cand = t >= rs.lo && t < rs.hi;
+            const bool up = !hi_open && vv[j] >= f_hi;
+            keep |= (uint32_t)(valid && (!cand || up)) << j;
+            mb |= (uint32_t)(valid && cand && !up && vv[j] >= f_lo) << j;
+          }
+        }
+        uint32_t word = keep << (4 * (lane & 7));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        if ((lane & 7) == 0 && w < we) sm.mword[w] = word;
+        memb |= mb << (4 * u);
+      }
+      if (!__any_sync(0xffffffffu, memb != 0u)) return;
+      const uint32_t cnt = __popc(memb);
+      uint32_t x = cnt;  // inclusive prefix over the lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(&sm.n_list, x);
+      base = __shfl_sync(0xffffffffu, base, 31);
+      uint32_t pos = base + x - cnt;
+#pragma unroll
+      for (int u = 0; u < kClBatch; ++u) {
+        if (((memb >> (4 * u)) & 0xFu) == 0u) continue;
+        const int tv = c0 + 32 * (w0 + 4 * u + (lane >> 3)) + 4 * (lane & 7);
+        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((memb >> (4 * u + j)) & 1u) {
+            const uint32_t key = order_key(vv[j]);
+            if (pos < (uint32_t)kClListCap) sm.list[pos] = make_uint2(key, (uint32_t)(tv + j - c0));
+            atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
+            ++pos;
+          }
+      }
+    };
+    constexpr int WB = 4 * kClBatch;  // words per batch
+    for (int w0 = wb; w0 < we; w0 += 2 * WB) {
+      if (w0 + WB < we) load_batch(vb, w0 + WB);
+      process(va, w0);
+      if (w0 + WB < we) {
+        if (w0 + 2 * WB < we) load_batch(va, w0 + 2 * WB);
+        process(vb, w0 + WB);
+      }
+    }
+    __syncthreads();
+    hist_to_total<kHistBins>(sm.hist, tot);
+    cluster.sync();  // the row's digit-2 total is complete in L2
+    // ---- digit 2
+    const uint32_t b2 = total_find_bin<kHistBins>(tot, kleft, sm, p.status, above);
+    const uint32_t kleft2 = kleft - above;
+    const uint32_t prefix22 = (b1 << 11) | b2;
+    const uint32_t n_list = sm.n_list;
+    const bool overflow = n_list > (uint32_t)kClListCap;  // the list misses keys: re-read from L2
+    for (int i = tid; i < kClHist3; i += kClThreads) sm.hist[i] = 0u;
+    __syncthreads();
+    if (!overflow) {
+      for (uint32_t i = tid; i < n_list; i += kClThreads) {
+        const uint32_t key = sm.list[i].x;
+        if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
+      }
+    } else {
+      visit_candidates(srow, c0, c1, rs.lo, rs.hi, [&](int, uint32_t key) {
+        if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
+      });
+    }
+    __syncthreads();
+    hist_to_total<kClHist3>(sm.hist, tot + kHistBins);
+    cluster.sync();  // the row's digit-3 total is complete in L2
+    // ---- digit 3: the k-th key T and the number of keys equal to T that are kept
+    const uint32_t b3 = total_find_bin<kClHist3>(tot + kHistBins, kleft2, sm, p.status, above);
+    const uint32_t T = (prefix22 << 10) | b3;
+    const uint32_t quota = kleft2 - above;
+    const uint32_t ntie_all = sm.tot[b3], my_ties = sm.hist[b3];
+    uint32_t q_c = my_ties;  // every key equal to T kept (the usual case: one key at T)
+    if (ntie_all != quota) {  // the same decision in every CTA of the cluster
+      if (tid == 0) slot[c] = my_ties;
+      cluster.sync();  // every CTA's count of keys equal to T is posted
+      if (tid == 0) {  // ties on the CTAs before this one (lower tokens)
+        uint32_t pre = 0;
+        for (int j = 0; j < c; ++j) pre += __ldcg(slot + j);
+        sm.pre_ties = pre;
+      }
+      __syncthreads();
+      const uint32_t pre = sm.pre_ties;
+      q_c = quota > pre ? min(quota - pre, my_ties) : 0u;
+    }
+    // ---- keys of bin b1 above T into the words, keys equal to T into the tie bitmap
+    if (!overflow) {
+      for (uint32_t i = tid; i < n_list; i += kClThreads) {
+        const uint2 e = sm.list[i];
+        if (e.x > T)
+          atomicOr(&sm.mword[e.y >> 5], 1u << (e.y & 31));
+        else if (e.x == T)
+          atomicOr(&sm.tbits[e.y >> 5], 1u << (e.y & 31));
+      }
+    } else {
+      visit_candidates(srow, c0, c1, rs.lo, rs.hi, [&](int t, uint32_t key) {
+        const int o = t - c0;
+        if (key > T && (key >> 21) == b1)
+          atomicOr(&sm.mword[o >> 5], 1u << (o & 31));
+        else if (key == T)
+          atomicOr(&sm.tbits[o >> 5], 1u << (o & 31));
+      });
+    }
+    __syncthreads();
+    // ---- the first q_c ties of this CTA, in token order
+    if (q_c == my_ties) {
+      for (int w = tid; w < nw; w += kClThreads) sm.mword[w] |= sm.tbits[w];
+    } else if (q_c > 0) {  // uniform in the CTA
+      constexpr int WPT = kClWordsMax / kClThreads;
+      const int w0 = tid * WPT;
+      uint32_t cnt = 0;
+#pragma unroll
+      for (int j = 0; j < WPT; ++j)
+        if (w0 + j < nw) cnt += __popc(sm.tbits[w0 + j]);
+      uint32_t total;
+      uint32_t rank = block_excl_scan<kClThreads>(cnt, total, sm.scan);
+#pragma unroll
+      for (int j = 0; j < WPT; ++j) {
+        if (w0 + j >= nw) break;
+        uint32_t x = sm.tbits[w0 + j], keep = 0;
+        while (x && rank < q_c) {
+          const uint32_t low = x & (~x + 1u);
+          keep |= low;
+          x ^= low;
+          ++rank;
+        }
+        sm.mword[w0 + j] |= keep;
+      }
+    }
+  } else {
+    // ---- no top-k to resolve: sink, window and all or none of the
+    // candidates, or the cached top-k of a reusing row (widened by the
+    // radius, kept inside the current candidates)
+    const int sink_hi = min(p.sink, rs.L), win_lo = max(rs.L - p.window, 0);
+    const uint32_t* cm = reused ? p.sc_mask + row * p.mask_words : nullptr;
+    const int hi_prev = reused ? p.sc_len[row] - p.window : 0;
+    auto cached = [&](int gw) -> uint32_t {
+      return (gw < 0 || gw >= p.mask_words) ? 0u : (cm[gw] & range_bits(gw * 32, p.sink, hi_prev));
+    };
+    for (int w = tid; w < nw; w += kClThreads) {
+      const int gw = (c0 >> 5) + w, t0 = gw * 32;
+      uint32_t word = range_bits(t0, 0, sink_hi) | range_bits(t0, win_lo, rs.L);
+      if (reused) {
+        uint32_t x = cached(gw);
+        if (p.reuse_radius > 0) {
+          const uint32_t prev = cached(gw - 1), next = cached(gw + 1);
+          const uint64_t below = ((uint64_t)x << 32) | prev;    // tokens 32(gw-1) .. 32gw+31
+          const uint64_t above_w = ((uint64_t)next << 32) | x;  // tokens 32gw .. 32(gw+1)+31
+          uint32_t d = x;
+          for (int sft = 1; sft <= p.reuse_radius; ++sft)
+            d |= (uint32_t)(below >> (32 - sft)) | (uint32_t)(above_w >> sft);
+          x = d;
+        }
+        word |= x & range_bits(t0, rs.lo, rs.hi);
+      } else if (rs.mode == 1) {
+        word |= range_bits(t0, rs.lo, rs.hi);
+      }
+      sm.mword[w] = word;
+    }
+  }
+
+  // ---- write the words once; post kept counts; count check, count, index list
+  __syncthreads();
+  uint32_t* gm = p.mask + row * p.mask_words + (c0 >> 5);
+  const bool refill = p.reuse != nullptr && !reused && rs.mode == 2;  // a fresh top-k refills the cache
+  uint32_t kept = 0;
+  for (int w = tid; w < nw; w += kClThreads) {
+    const uint32_t x = sm.mword[w];
+    gm[w] = x;
+    if (refill) p.sc_mask[row * p.mask_words + (c0 >> 5) + w] = x;
+    kept += __popc(x);
+  }
+  uint32_t kept_cta;
+  (void)block_excl_scan<kClThreads>(kept, kept_cta, sm.scan);
+  const int sink_n = min(p.sink, rs.L);
+  const uint32_t expect = (uint32_t)(sink_n + (rs.L - max(rs.L - p.window, sink_n)) + rs.k);
+  uint32_t* kept_sum = tot + kHistBins + kClHist3;  // then the CTA ticket
+  if (p.idx == nullptr) {
+    // The last CTA of the row to finish (a ticket taken after this CTA's
+    // count is added; nothing waits on it) checks the total, writes the
+    // count and clears the row's state: every CTA read the histograms and
+    // totals before taking its ticket.
+    if (tid == 0) {
+      atomicAdd(kept_sum, kept_cta);
+      __threadfence();
+      sm.last = atomicAdd(kept_sum + 1, 1u) == (uint32_t)(nc - 1) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (sm.last) {
+      __threadfence();
+      if (tid == 0) {
+        const uint32_t total = __ldcg(kept_sum);
+        if (p.count != nullptr) p.count[row] = (int32_t)total;
+        // a reused set has the cached top-k's size, not this step's k
+        if (!reused && total != expect) atomicOr(p.status, TB_DEV_ERR_COUNT);
+      }
+      __syncthreads();  // the total is read before it is cleared
+      for (int i = tid; i < kHistBins; i += kClThreads) p.hist1[row * kHistBins + i] = 0u;
+      for (int i = tid; i < kClTotWords; i += kClThreads) tot[i] = 0u;
+    }
+    return;
+  }
+  // ---- with an index list: the CTAs' kept counts in order give each CTA's offset
+  if (tid == 0) slot[kClMaxCluster + c] = kept_cta;
+  cluster.sync();  // every CTA's kept count is posted
+  uint32_t total = 0, before = 0;
+  for (int j = 0; j < nc; ++j) {
+    const uint32_t x = __ldcg(slot + kClMaxCluster + j);
+    total += x;
+    if (j < c) before += x;
+  }
+  if (c == 0 && tid == 0) {
+    if (p.count != nullptr) p.count[row] = (int32_t)total;
+    if (!reused && total != expect) atomicOr(p.status, TB_DEV_ERR_COUNT);
+  }
+  {  // ascending indices: this CTA's run starts after the lower CTAs' kept tokens
+    constexpr int WPT = kClWordsMax / kClThreads;
+    const int w0 = tid * WPT;
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int j = 0; j < WPT; ++j)
+      if (w0 + j < nw) cnt += __popc(sm.mword[w0 + j]);
+    uint32_t tot_idx;
+    uint32_t pos = before + block_excl_scan<kClThreads>(cnt, tot_idx, sm.scan);
+#pragma unroll
+    for (int j = 0; j < WPT; ++j) {
+      if (w0 + j >= nw) break;
+      uint32_t x = sm.mword[w0 + j];
+      while (x) {
+        const int bit = __ffs(x) - 1;
+        x &= x - 1u;
+        if (pos < (uint32_t)p.idx_cap) p.idx[row * p.idx_cap + pos] = c0 + 32 * (w0 + j) + bit;
+        ++pos;
+      }
+    }
+  }
+  if (c == 0) {  // every CTA read the histograms and totals before the last cluster barrier
+    for (int i = tid; i < kHistBins; i += kClThreads) p.hist1[row * kHistBins + i] = 0u;
+    for (int i = tid; i < kClTotWords; i += kClThreads) tot[i] = 0u;
+  }
+}
+
+}  // namespace tb

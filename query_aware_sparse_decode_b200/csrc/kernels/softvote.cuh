@@ -12,10 +12,12 @@
 // shared by the group's query heads), contiguous 16-token tiles gathered by
 // cp.async into a swizzled ring, q . K^T on mma.sync (bf16 in, fp32
 // accumulate); writes the logits in the log2 domain and one (max, sum of
-// 2^(a - max)) pair per head and chunk.
-// softvote_reduce: merges the chunk pairs into each head's (M, Z) (a warp per
-// head, lanes over the chunks) and sums 2^(a - M) / Z over the heads, one
-// token per thread (logits are L2-resident).  Optionally it also
+// 2^(a - max)) pair per head and chunk.  The last CTA of a sequence to finish
+// (a device-scope completion counter, fence then count; nothing waits on it)
+// merges the sequence's chunk pairs into each head's (M, 1/Z) and resets the
+// counter for the next launch.
+// softvote_reduce: sums 2^(a - M) / Z over the heads, one token per thread
+// (logits are L2-resident), after one read of the heads' (M, 1/Z).  Optionally it also
 // builds the first-digit histogram of the votes over the candidate range
 // [sink, len - window) for the selection that follows (warp-aggregated shared
 // atomics: votes crowd into few bins).
@@ -36,6 +38,8 @@ struct VoteParams {
   const void* q;        // [B][Hq][D] bf16
   float* logits;        // [B][Hq][max_len], log2 domain
   float* stats;         // [B][Hq][nchunk][2]
+  float* mz;            // [B][Hq][2]: each head's merged max M (log2 domain) and 1/Z
+  uint32_t* done;       // [B] logits CTAs finished (zero between launches)
   float* votes;         // [B][max_len]
   uint32_t* hist1;      // [B][2048] first-digit histograms of the votes, or nullptr
   int Hq, Hkv, max_len, nchunk;  // nchunk: stride of the chunk statistics, >= max_len / chunk
@@ -142,8 +146,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
     const float m_new = fmaxf(m_run, mt);
     if (m_new != kNegInf) {
-      l_run = l_run * exp2f(m_run - m_new) + exp2f(s0 - m_new) + exp2f(s1 - m_new) + exp2f(s2 - m_new) +
-              exp2f(s3 - m_new);
+      // 2^x on the special-function unit (relative error about 2^-22, far
+      // inside the votes' tolerance); 2^-inf = 0
+      l_run = l_run * fast_exp2(m_run - m_new) + fast_exp2(s0 - m_new) + fast_exp2(s1 - m_new) +
+              fast_exp2(s2 - m_new) + fast_exp2(s3 - m_new);
       m_run = m_new;
     }
     __syncwarp();
@@ -170,20 +176,61 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     p.stats[ph] = M;
     p.stats[ph + 1] = l;
   }
+  // ---- the sequence's last CTA merges every chunk's pair into (M, 1/Z) per head
+  __shared__ uint32_t s_last;
+  __threadfence();  // this CTA's pairs are visible device-wide before it is counted
+  __syncthreads();
+  const int nch = (L + p.chunk - 1) / p.chunk;
+  if (tid == 0) s_last = atomicAdd(&p.done[b], 1u) == (uint32_t)(nch * p.Hkv - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // four threads per head (consecutive lanes), each merging every fourth chunk
+  constexpr int TPH = 4;
+  const int sub = tid % TPH;
+  for (int h0 = 0; h0 < p.Hq; h0 += kAttnThreads / TPH) {
+    const int h = h0 + tid / TPH;
+    float m = kNegInf, l = 0.f;
+    if (h < p.Hq) {
+      const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
+#pragma unroll 4
+      for (int c = sub; c < nch; c += TPH) {
+        const float2 e = __ldcg(st + c);
+        if (e.x == kNegInf) continue;
+        const float mn = fmaxf(m, e.x);
+        l = l * exp2f(m - mn) + e.y * exp2f(e.x - mn);
+        m = mn;
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < TPH; o <<= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      const float mn = fmaxf(m, m2);
+      if (mn != kNegInf) {
+        l = (m == kNegInf ? 0.f : l * exp2f(m - mn)) + (m2 == kNegInf ? 0.f : l2 * exp2f(m2 - mn));
+        m = mn;
+      }
+    }
+    if (h < p.Hq && sub == 0) {
+      p.mz[((size_t)b * p.Hq + h) * 2] = m;
+      p.mz[((size_t)b * p.Hq + h) * 2 + 1] = 1.f / l;
+    }
+  }
+  if (tid == 0) p.done[b] = 0u;  // ready for the next launch (stream-ordered after this grid)
 }
 
 // grid (ceil(max len / 256), B), block 256: one token per thread.  The
 // token's logits of the first kVotePrefetch heads are requested before the
-// CTA merges the chunk statistics, so their latency overlaps the merge.
+// CTA reads the heads' (M, 1/Z), so the two latencies overlap.
 constexpr int kVoteMaxHeads = 128;
 constexpr int kVoteReduceTok = 256;
 constexpr int kVotePrefetch = 32;
 __global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
   pdl_wait();
   pdl_trigger();
-  __shared__ float sM[kVoteMaxHeads], sInvZ[kVoteMaxHeads];
+  __shared__ float2 sMZ[kVoteMaxHeads];  // per head: (M, 1/Z)
   __shared__ uint32_t hist[kHistBins];
-  const int b = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
   const int L = p.lens[b];
   const int t_begin = blockIdx.x * kVoteReduceTok;
   if (t_begin >= L) return;
@@ -192,30 +239,9 @@ __global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p
   float a[kVotePrefetch];
 #pragma unroll
   for (int h = 0; h < kVotePrefetch; ++h) a[h] = (h < p.Hq && t < L) ? lg[(size_t)h * p.max_len] : 0.f;
-  const int nch = (L + p.chunk - 1) / p.chunk;
-  for (int h = warp; h < p.Hq; h += 8) {
-    const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
-    float m = kNegInf, l = 0.f;
-    for (int c = lane; c < nch; c += 32) {  // per lane: merge its chunks
-      const float2 e = st[c];
-      if (e.x == kNegInf) continue;
-      const float mn = fmaxf(m, e.x);
-      l = l * exp2f(m - mn) + e.y * exp2f(e.x - mn);
-      m = mn;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
-      const float mn = fmaxf(m, m2);
-      if (mn != kNegInf) {
-        l = (m == kNegInf ? 0.f : l * exp2f(m - mn)) + (m2 == kNegInf ? 0.f : l2 * exp2f(m2 - mn));
-        m = mn;
-      }
-    }
-    if (lane == 0) {
-      sM[h] = m;
-      sInvZ[h] = 1.f / l;
-    }
+  for (int h = tid; h < p.Hq; h += 256) {
+    const float2 mz = reinterpret_cast<const float2*>(p.mz)[(size_t)b * p.Hq + h];
+    sMZ[h] = mz;
   }
   if (p.hist1 != nullptr)
     for (int i = tid; i < kHistBins; i += 256) hist[i] = 0;
@@ -224,8 +250,14 @@ __global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p
   if (t < L) {
 #pragma unroll
     for (int h = 0; h < kVotePrefetch; ++h)
-      if (h < p.Hq) v += exp2f(a[h] - sM[h]) * sInvZ[h];
-    for (int h = kVotePrefetch; h < p.Hq; ++h) v += exp2f(lg[(size_t)h * p.max_len] - sM[h]) * sInvZ[h];
+      if (h < p.Hq) {
+        const float2 mz = sMZ[h];
+        v = fmaf(fast_exp2(a[h] - mz.x), mz.y, v);
+      }
+    for (int h = kVotePrefetch; h < p.Hq; ++h) {
+      const float2 mz = sMZ[h];
+      v = fmaf(fast_exp2(lg[(size_t)h * p.max_len] - mz.x), mz.y, v);
+    }
     p.votes[(size_t)b * p.max_len + t] = v;
   }
   if (p.hist1 == nullptr) return;

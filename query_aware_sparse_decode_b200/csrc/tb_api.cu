@@ -11,6 +11,8 @@
 #include <new>
 
 #include "kernels/attn.cuh"
+#include "kernels/attn_split.cuh"
+#include "kernels/index_mask.cuh"
 #include "kernels/common.cuh"
 #include "kernels/kimp.cuh"
 #include "kernels/prefill.cuh"
@@ -18,6 +20,7 @@
 #include "kernels/project_tc.cuh"
 #include "kernels/score.cuh"
 #include "kernels/select.cuh"
+#include "kernels/select_cluster.cuh"
 #include "kernels/shard.cuh"
 #include "kernels/softvote.cuh"
 #include "tb.h"
@@ -48,8 +51,8 @@ struct LayerState {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t status, hist, ccount, kcount, hist2, hist_end, rowinfo, cand, scores, mask, part_o, part_ml, votes, vstats,
-      reuse, total;
+  size_t status, hist, ccount, kcount, hist2, ctot, hist_end, cslot, rowinfo, cand, scores, mask, part_o, part_ml, votes,
+      vstats, vmz, vdone, reuse, total;
   int max_splits;
 };
 
@@ -62,8 +65,10 @@ WsLayout layout_of(const tb_config& c) {
   w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
   w.ccount = off;  off += align256(B * Hq * 4);          // candidate counters, kept-token
   w.kcount = off;  off += align256(B * Hq * 4);          // counters and the single-row
-  w.hist2 = off;   off += align256(B * kHistBins * 4);   // second-digit histograms
+  w.hist2 = off;   off += align256(B * kHistBins * 4);   // second-digit histograms and the
+  w.ctot = off;    off += align256(B * Hq * (size_t)kClTotWords * 4);  // cluster selection's totals
   w.hist_end = off;                                      // (zeroed together)
+  w.cslot = off;   off += align256(B * Hq * (size_t)kClSlotWords * 4);  // cluster selection's per-CTA counts
   w.rowinfo = off; off += align256(B * Hq * 16);
   w.cand = off;    off += align256(B * Hq * (size_t)kSelCap * 8);
   w.scores = off;  off += align256(B * Hq * Lm * 4);
@@ -72,6 +77,8 @@ WsLayout layout_of(const tb_config& c) {
   w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
   w.votes = off;   off += align256(B * Lm * 4);
   w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteMinChunk - 1) / kVoteMinChunk) * 2 * 4);
+  w.vmz = off;     off += align256(B * Hq * 2 * 4);      // per head: merged soft-vote (M, 1/Z)
+  w.vdone = off;   off += align256(B * 4);               // logits CTAs finished (zeroed at init, self-clearing)
   w.reuse = off;   off += align256(B * Hq * 4);         // per-row reuse decisions of the step
   w.total = off;
   return w;
@@ -117,7 +124,12 @@ struct tb_ctx {
   float* part_ml = nullptr;
   float* votes = nullptr;
   float* vstats = nullptr;
-  bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last resolve)
+  float* vmz = nullptr;
+  uint32_t* vdone = nullptr;
+  bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last selection)
+  int cluster_active[5] = {};  // resident clusters of 1, 2, 4, 8, 16 CTAs of the selection kernel (0: not launchable)
+  uint32_t* ctot = nullptr;
+  uint32_t* cslot = nullptr;
   uint32_t* reuse = nullptr;
   float reuse_tau = 0.f;     // amortised selection: cosine threshold,
   int reuse_interval = 0;    // at most this many tokens since the cached selection (0: off),
@@ -170,6 +182,38 @@ static int max_len_of(const LayerState& ls, int B) {
   return m;
 }
 
+// How many clusters of 1, 2, 4, 8 and 16 CTAs of the cluster selection
+// kernel can be resident at once on this device (0: that size cannot run).
+static void probe_cluster_select(tb_ctx* ctx) {
+  for (int i = 0; i < 5; ++i) ctx->cluster_active[i] = 0;
+  if (cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kClSmem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  for (int i = 0; i < 5; ++i) {
+    const int nc = 1 << i;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, 1, 1);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = kClSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, select_cluster_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      clusters = 0;
+    }
+    ctx->cluster_active[i] = clusters;
+  }
+}
+
 // ------------------------------------------------------------------ launches
 // Zero the selection's histograms and candidate counters (one contiguous
 // workspace range).
@@ -211,7 +255,8 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   const bool grouped = c.variant == TB_BUTLER_GROUP;
   const size_t smem = hist ? (size_t)(grouped ? 1 : gs) * kHistBins * 4 : 0;
   // the most tokens per CTA (up to 4 steps) that still gives about three
-  // CTAs per SM; short or small batches get one step per CTA
+  // CTAs per SM; short or small batches get one step per CTA (a grid sized
+  // to whole waves of exactly balanced chunks measured no faster)
   const int step = c.kimp_bf16 ? score_step<__nv_bfloat16>() : score_step<float>();
   int iters = 4;
   while (iters > 1 && (long long)c.batch * c.n_kv_heads * ((maxL + step * iters - 1) / (step * iters)) <
@@ -219,6 +264,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
     iters >>= 1;
   p.iters = iters;
   const int chunk = step * iters;
+  p.chunk = chunk;
   dim3 grid((maxL + chunk - 1) / chunk, c.n_kv_heads, c.batch);
 #define TB_SCORE_CASE(T, KT, DI, GSV)                                                                \
   if (c.d_imp == DI && gs == GSV) {                                                                  \
@@ -285,6 +331,24 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   }
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   const int maxL = max_len_of(ls, c.batch);
+  int nc = 0, chunk = 0;
+  if (cluster_select_shape(ctx->num_sms, (long long)rows * c.batch, maxL, ctx->cluster_active, &nc, &chunk)) {
+    // one cluster per row: one launch after the first-digit histogram
+    if (!hist1_ready) {
+      dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
+      prepare_hist(ctx, st);
+      launch_pdl(select_hist_kernel, cgrid, dim3(kScatThreads), 0, st, p);
+      ++ctx->launches;
+    }
+    p.ctot = ctx->ctot;
+    p.cslot = ctx->cslot;
+    launch_pdl_cluster(select_cluster_kernel, dim3(nc, rows, c.batch), dim3(kClThreads), (size_t)kClSmem, st, nc, p,
+                       chunk);
+    ++ctx->launches;
+    const tb_status s = cuda_status(cudaGetLastError());
+    if (s == TB_OK) ctx->hist_clean = true;  // CTA 0 of every row clears the row's histogram
+    return s;
+  }
   if (maxL <= kRowMax && !use_cache && idx == nullptr) {  // short rows: one CTA per row, one launch
     cudaFuncSetAttribute(select_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmem);
     launch_pdl(select_row_kernel, dim3(rows, c.batch), dim3(kSelThreads), (size_t)kRowSmem, st, p,
@@ -337,19 +401,9 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
   p.max_len = c.max_len;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c.head_dim));
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
-  // chunking: the whole grid is about two full waves of two CTAs per SM, or
-  // one wave when two would leave CTAs with short chunks (fewer than 3584
-  // tokens: the list build, the ring's fill and the partial write then weigh
-  // more than the second wave's balance gains)
-  const int groups = c.batch * c.n_kv_heads;
-  int want_split = std::min(kMaxSplits, std::max(1, (4 * ctx->num_sms) / groups));
-  if ((std::max(maxL, 1) + want_split - 1) / want_split < 3584)
-    want_split = std::min(kMaxSplits, std::max(1, (2 * ctx->num_sms) / groups));
-  int chunk = (std::max(maxL, 1) + want_split - 1) / want_split;
-  chunk = std::max(256, (chunk + 255) / 256 * 256);
+  int chunk = 0;
+  if (!attn_split(ctx->num_sms, c.batch * c.n_kv_heads, maxL, &chunk, &p.nsplit)) return TB_ERR_UNSUPPORTED;
   p.chunk = chunk;
-  p.nsplit = std::max(1, (maxL + chunk - 1) / chunk);
-  if (p.nsplit > kMaxSplits) return TB_ERR_UNSUPPORTED;
   if (p.nsplit > ctx->lay.max_splits) return TB_ERR_WORKSPACE;
   {
     dim3 grid(p.nsplit, c.n_kv_heads, c.batch);
@@ -418,6 +472,8 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   p.q = q;
   p.logits = ctx->scores;
   p.stats = ctx->vstats;
+  p.mz = ctx->vmz;
+  p.done = ctx->vdone;
   p.votes = votes;
   p.hist1 = hist;
   p.sink = c.sink;
@@ -488,6 +544,8 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->ccount = reinterpret_cast<uint32_t*>(ctx->ws + lay.ccount);
   ctx->kcount = reinterpret_cast<uint32_t*>(ctx->ws + lay.kcount);
   ctx->hist2 = reinterpret_cast<uint32_t*>(ctx->ws + lay.hist2);
+  ctx->ctot = reinterpret_cast<uint32_t*>(ctx->ws + lay.ctot);
+  ctx->cslot = reinterpret_cast<uint32_t*>(ctx->ws + lay.cslot);
   ctx->cand = reinterpret_cast<uint32_t*>(ctx->ws + lay.cand);
   ctx->rowinfo = reinterpret_cast<uint4*>(ctx->ws + lay.rowinfo);
   ctx->scores = reinterpret_cast<float*>(ctx->ws + lay.scores);
@@ -496,11 +554,15 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
   ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
   ctx->vstats = reinterpret_cast<float*>(ctx->ws + lay.vstats);
+  ctx->vmz = reinterpret_cast<float*>(ctx->ws + lay.vmz);
+  ctx->vdone = reinterpret_cast<uint32_t*>(ctx->ws + lay.vdone);
   ctx->reuse = reinterpret_cast<uint32_t*>(ctx->ws + lay.reuse);
-  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
+  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMemset(ctx->vdone, 0, (size_t)cfg->batch * sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return TB_ERR_CUDA;
   }
+  probe_cluster_select(ctx);
   *out = ctx;
   return TB_OK;
 }
@@ -633,7 +695,8 @@ TB_API tb_status tb_bind_selection_cache(tb_ctx* ctx, int layer, void* cache, si
 TB_API tb_status tb_copy_step_masks(tb_ctx* ctx, uint32_t* dst, size_t bytes, void* stream) {
   if (!ctx || !dst) return TB_ERR_INVALID_ARG;
   const tb_config& c = ctx->cfg;
-  const size_t need = (size_t)c.batch * sel_rows(c) * (size_t)(c.max_len / 32) * 4;
+  const int rows = c.variant == TB_SOFTVOTE ? 1 : sel_rows(c);  // soft voting: one shared set per sequence
+  const size_t need = (size_t)c.batch * rows * (size_t)(c.max_len / 32) * 4;
   if (bytes < need) return TB_ERR_SHAPE;
   return cuda_status(cudaMemcpyAsync(dst, ctx->mask, need, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
 }
@@ -693,6 +756,41 @@ TB_API tb_status tb_append_kv(tb_ctx* ctx, int layer, const void* k_new, const v
   return TB_OK;
 }
 
+// One persistent tcgen05 launch projecting rows [start, start + count) of
+// every (b, KV head) of layers [first, first + n) (dense bf16 caches).
+static tb_status launch_project_tc(tb_ctx* ctx, int first, int n, int start, int count, cudaStream_t st) {
+  const tb_config& c = ctx->cfg;
+  ProjectTcParams tp{};  // ~9 KB of kernel parameters (one tensor map per layer)
+  for (int i = 0; i < n; ++i) {
+    const LayerState& ls = ctx->layers[first + i];
+    tp.kmap[i] = ls.k_map;
+    tp.w_k[i] = ls.wk;
+    tp.kimp[i] = ls.kimp;
+  }
+  tp.status = ctx->status;
+  tp.max_len = c.max_len;
+  tp.start = start;
+  tp.count = count;
+  tp.tiles_per_slab = (count + kTcRows - 1) / kTcRows;
+  tp.tiles_per_layer = tp.tiles_per_slab * c.batch * c.n_kv_heads;
+  tp.total_tiles = tp.tiles_per_layer * n;
+  tp.n_layers = n;
+  tp.kimp_bf16 = c.kimp_bf16;
+  const int grid = std::min(tp.total_tiles, ctx->num_sms);
+#define TB_TC_CASE(DV, DI)                                                              \
+  if (c.head_dim == DV && c.d_imp == DI) {                                              \
+    auto k = project_tc_kernel<DV, DI>;                                                 \
+    const int smem = project_tc_smem_bytes<DV>();                                       \
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+      return TB_ERR_CUDA;                                                               \
+    k<<<grid, kTcThreads, smem, st>>>(tp);                                              \
+  } else
+  TB_TC_CASE(128, 32) TB_TC_CASE(128, 16) TB_TC_CASE(64, 32) TB_TC_CASE(64, 16) return TB_ERR_UNSUPPORTED;
+#undef TB_TC_CASE
+  ++ctx->launches;
+  return cuda_status(cudaGetLastError());
+}
+
 TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, void* stream) {
   tb_status s = check_layer(ctx, layer);
   if (s != TB_OK) return s;
@@ -701,30 +799,7 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
   if (count == 0) return TB_OK;
   const LayerState& ls = ctx->layers[layer];
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (c.kv_dtype == TB_BF16 && ls.kl.page_table == nullptr) {
-    ProjectTcParams tp{};
-    tp.w_k = ls.wk;
-    tp.kimp = ls.kimp;
-    tp.status = ctx->status;
-    tp.max_len = c.max_len;
-    tp.start = start;
-    tp.count = count;
-    tp.tiles_per_slab = (count + kTcRows - 1) / kTcRows;
-    tp.total_tiles = tp.tiles_per_slab * c.batch * c.n_kv_heads;
-    tp.kimp_bf16 = c.kimp_bf16;
-    const int grid = std::min(tp.total_tiles, ctx->num_sms);
-#define TB_TC_CASE(DV, DI)                                                              \
-  if (c.head_dim == DV && c.d_imp == DI) {                                              \
-    auto k = project_tc_kernel<DV, DI>;                                                 \
-    const int smem = project_tc_smem_bytes<DV>();                                       \
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);         \
-    k<<<grid, kTcThreads, smem, st>>>(ls.k_map, tp);                                    \
-  } else
-    TB_TC_CASE(128, 32) TB_TC_CASE(128, 16) TB_TC_CASE(64, 32) TB_TC_CASE(64, 16) return TB_ERR_UNSUPPORTED;
-#undef TB_TC_CASE
-    ++ctx->launches;
-    return cuda_status(cudaGetLastError());
-  }
+  if (c.kv_dtype == TB_BF16 && ls.kl.page_table == nullptr) return launch_project_tc(ctx, layer, 1, start, count, st);
   // fp32 caches, and paged caches of either type (a TMA tile may not cross pages): fp32 FMA
   ProjectParams p{ls.k, ls.kimp, ls.wk, c.n_kv_heads, c.max_len, start, count, ls.kl, c.kimp_bf16};
   dim3 grid((count + kProjRows - 1) / kProjRows, c.n_kv_heads, c.batch);
@@ -740,6 +815,29 @@ TB_API tb_status tb_project_kimp(tb_ctx* ctx, int layer, int start, int count, v
 #undef TB_PROJ_CASE
   ++ctx->launches;
   return cuda_status(cudaGetLastError());
+}
+
+TB_API tb_status tb_project_kimp_layers(tb_ctx* ctx, int first_layer, int n_layers, int start, int count,
+                                        void* stream) {
+  if (!ctx || n_layers < 1 || first_layer < 0 || (long long)first_layer + n_layers > ctx->cfg.n_layers)
+    return TB_ERR_INVALID_ARG;
+  const tb_config& c = ctx->cfg;
+  if (start < 0 || count < 0 || (long long)start + count > c.max_len) return TB_ERR_CAPACITY;
+  bool tc = c.kv_dtype == TB_BF16;
+  for (int l = first_layer; l < first_layer + n_layers; ++l) {
+    const tb_status s = check_layer(ctx, l);
+    if (s != TB_OK) return s;
+    tc = tc && ctx->layers[l].kl.page_table == nullptr;
+  }
+  if (count == 0) return TB_OK;
+  if (!tc) {  // fp32 or paged caches: the FMA projection, layer by layer
+    for (int l = first_layer; l < first_layer + n_layers; ++l) {
+      const tb_status s = tb_project_kimp(ctx, l, start, count, stream);
+      if (s != TB_OK) return s;
+    }
+    return TB_OK;
+  }
+  return launch_project_tc(ctx, first_layer, n_layers, start, count, static_cast<cudaStream_t>(stream));
 }
 
 TB_API tb_status tb_score(tb_ctx* ctx, int layer, const void* q_imp_producer, float* scores, void* stream) {
@@ -784,6 +882,31 @@ TB_API tb_status tb_sparse_attn(tb_ctx* ctx, int layer, const void* q, const uin
   if (mask_mode != TB_MASK_DENSE && !mask) return TB_ERR_INVALID_ARG;
   if (!aligned16(q)) return TB_ERR_SHAPE;
   return launch_attn(ctx, layer, q, mask, mask_mode, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+TB_API tb_status tb_sparse_attn_idx(tb_ctx* ctx, int layer, const void* q, const int32_t* idx, int idx_cap,
+                                    const int32_t* count, void* out, float* lse, void* stream) {
+  tb_status s = check_layer(ctx, layer);
+  if (s != TB_OK) return s;
+  if (!q || !idx || !count || !out || idx_cap < 1) return TB_ERR_INVALID_ARG;
+  if (!aligned16(q)) return TB_ERR_SHAPE;
+  const tb_config& c = ctx->cfg;
+  const LayerState& ls = ctx->layers[layer];
+  IndexMaskParams p{};
+  p.idx = idx;
+  p.count = count;
+  p.mask = ctx->mask;
+  p.status = ctx->status;
+  p.Hq = c.n_q_heads;
+  p.idx_cap = idx_cap;
+  p.mask_words = c.max_len / 32;
+  for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  launch_pdl(index_mask_kernel, dim3(c.n_q_heads, c.batch), dim3(kIdxMaskThreads), 0, st, p);
+  ++ctx->launches;
+  s = cuda_status(cudaGetLastError());
+  if (s != TB_OK) return s;
+  return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_PER_HEAD, out, lse, st);
 }
 
 // Amortised selection: per-row reuse decisions of this step (see reuse.cuh).

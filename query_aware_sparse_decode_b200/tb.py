@@ -27,8 +27,8 @@ STATUS_NAMES = {0: "TB_OK", 1: "TB_ERR_INVALID_ARG", 2: "TB_ERR_SHAPE", 3: "TB_E
 
 # every symbol include/tb.h declares
 EXPORTS = ("tb_workspace_size", "tb_init", "tb_bind_layer", "tb_set_seq_lens", "tb_get_seq_lens", "tb_set_budget",
-           "tb_append_kv", "tb_project_kimp", "tb_score", "tb_select", "tb_sparse_attn", "tb_decode_step",
-           "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
+           "tb_append_kv", "tb_project_kimp", "tb_project_kimp_layers", "tb_score", "tb_select", "tb_sparse_attn",
+           "tb_sparse_attn_idx", "tb_decode_step", "tb_select_prefill", "tb_softvote_scores", "tb_sparse_attn_static", "tb_trace_events", "tb_launch_count",
            "tb_check_status", "tb_status_string", "tb_destroy", "tb_selftest_bounded_wait", "tb_selection_cache_size",
            "tb_bind_selection_cache", "tb_set_reuse", "tb_copy_step_masks", "tb_bind_layer_paged", "tb_shard_set",
            "tb_shard_hist", "tb_shard_pick", "tb_shard_mask", "tb_sparse_attn_partial", "tb_merge_partials")
@@ -74,9 +74,11 @@ def lib():
             "tb_set_budget": [vp, i32, i32, i32],
             "tb_append_kv": [vp, i32, vp, vp, vp],
             "tb_project_kimp": [vp, i32, i32, i32, vp],
+            "tb_project_kimp_layers": [vp, i32, i32, i32, i32, vp],
             "tb_score": [vp, i32, vp, vp, vp],
             "tb_select": [vp, i32, vp, i32, vp, i32, vp, vp, vp],
             "tb_sparse_attn": [vp, i32, vp, vp, i32, vp, vp, vp],
+            "tb_sparse_attn_idx": [vp, i32, vp, vp, i32, vp, vp, vp, vp],
             "tb_decode_step": [vp, i32, vp, vp, vp, vp, vp, vp],
             "tb_select_prefill": [vp, i32, vp, i32, i32, vp, i32, vp],
             "tb_softvote_scores": [vp, i32, vp, vp, vp],
@@ -214,6 +216,10 @@ class Context:
     def project_kimp(self, layer, start, count, stream=None) -> None:
         _check(lib().tb_project_kimp(self._h, layer, start, count, _stream(stream)), "tb_project_kimp")
 
+    def project_kimp_layers(self, first_layer, n_layers, start, count, stream=None) -> None:
+        _check(lib().tb_project_kimp_layers(self._h, first_layer, n_layers, start, count, _stream(stream)),
+               "tb_project_kimp_layers")
+
     def score(self, layer, q_imp, scores, stream=None) -> None:
         _check(lib().tb_score(self._h, layer, _ptr(q_imp), _ptr(scores), _stream(stream)), "tb_score")
 
@@ -225,6 +231,11 @@ class Context:
     def sparse_attn(self, layer, q, mask, mask_mode, out, lse=None, stream=None) -> None:
         _check(lib().tb_sparse_attn(self._h, layer, _ptr(q), _ptr(mask), mask_mode, _ptr(out), _ptr(lse),
                                     _stream(stream)), "tb_sparse_attn")
+
+    def sparse_attn_idx(self, layer, q, idx, count, out, lse=None, stream=None) -> None:
+        """Attention over sets given as index lists: idx [B][Hq][cap], count [B][Hq] (int32)."""
+        _check(lib().tb_sparse_attn_idx(self._h, layer, _ptr(q), _ptr(idx), idx.shape[-1], _ptr(count), _ptr(out),
+                                        _ptr(lse), _stream(stream)), "tb_sparse_attn_idx")
 
     def decode_step(self, layer, k_new, v_new, q, q_imp, out, stream=None) -> None:
         _check(lib().tb_decode_step(self._h, layer, _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(q_imp), _ptr(out),
