@@ -257,11 +257,11 @@ def test_single_row_select_on_crowded_bins(kind, keep):
 
 @pytest.mark.parametrize("kind", [None, "two_digits"])
 def test_select_rows_beyond_one_cluster(kind):
-    """Rows longer than 16 CTAs of 32768 tokens (524288) take the many-CTA
-    scatter + resolve path: the same exact sets, counts and index lists on
-    identical fp32 scores (one shared row per sequence, as in soft voting,
-    and quantised per-head rows)."""
-    lens = (600000, 524289)
+    """Rows longer than a cluster of 16 CTAs of 65536 tokens (1048576) take
+    the many-CTA scatter + resolve path: the same exact sets, counts and
+    index lists on identical fp32 scores (one shared row per sequence, as in
+    soft voting, and quantised per-head rows)."""
+    lens = (1100000, 1048577)
     B = len(lens)
     rows = 1 if kind else 2
     keep = 30
@@ -326,6 +326,53 @@ def test_sparse_attn_on_oracle_sets(wl):
             refd, refd_lse = O.attend(ld.q[b, h], ld.K[b, h // gs, :L], ld.V[b, h // gs, :L], np.arange(L), scale)
             assert_close_rows(od[b, h][None], refd[None], wl.dtype, f"dense b{b} h{h}")
             assert abs(ldn[b, h] - refd_lse) <= 1e-3 * max(1.0, abs(refd_lse))
+
+
+def test_sparse_attn_on_index_lists():
+    """tb_sparse_attn_idx (the sets as the ascending index lists and counts
+    that tb_select writes) equals tb_sparse_attn on the same sets' mask bit
+    for bit and the oracle's attention; out-of-range indices are skipped and
+    flagged."""
+    wl = SMALL_BF16
+    ctx = TB.Context(config_of(wl))
+    ld = make_layer(ctx, wl, 0, wl.seq_lens)
+    gs = wl.Hq // wl.Hkv
+    sets = {}
+    for b, L in enumerate(wl.seq_lens):
+        for h in range(wl.Hq):
+            s = O.importance_scores(ld.qhat[b, h], O.project_keys(ld.K[b, h // gs, :L], ld.W))
+            sets[b, h] = O.select_tokens(s, L, wl.keep_pct, wl.sink, wl.window)
+    cap = max(len(v) for v in sets.values()) + 3
+    idx = np.full((wl.B, wl.Hq, cap), -1, np.int32)
+    cnt = np.zeros((wl.B, wl.Hq), np.int32)
+    for (b, h), v in sets.items():
+        idx[b, h, :len(v)] = v
+        cnt[b, h] = len(v)
+    mask = mask_from_sets(sets, wl.B, wl.Hq, ctx.cfg.max_len)
+    outs = []
+    for use_idx in (True, False):
+        out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+        lse = torch.empty((wl.B, wl.Hq), device="cuda")
+        if use_idx:
+            ctx.sparse_attn_idx(0, ld.q_dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out, lse)
+        else:
+            ctx.sparse_attn(0, ld.q_dev, mask, TB.TB_MASK_PER_HEAD, out, lse)
+        outs.append((out, lse))
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    o = outs[0][0].float().cpu().numpy()
+    scale = 1.0 / math.sqrt(wl.D)
+    for (b, h), v in sets.items():
+        L = wl.seq_lens[b]
+        want, _ = O.attend(ld.q[b, h], ld.K[b, h // gs, :L], ld.V[b, h // gs, :L], v, scale)
+        assert_close_rows(o[b, h][None], want[None], wl.dtype, f"b{b} h{h}")
+    # an index past the length: skipped and flagged
+    idx[0, 0, 0] = wl.seq_lens[0] + 5
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=tdtype(wl), device="cuda")
+    ctx.sparse_attn_idx(0, ld.q_dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0x1  # TB_DEV_ERR_INDEX
 
 
 def test_sparse_attn_empty_set_and_single_token():

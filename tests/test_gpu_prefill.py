@@ -9,7 +9,8 @@ from oracle import tokenbutler as O
 from query_aware_sparse_decode_b200 import synth as S
 from query_aware_sparse_decode_b200 import tb as TB
 
-from harness import config_of, kimp_alloc, kimp_rows, make_layer, round_up, sets_from_mask, tie_band_ok, to_dev
+from harness import (bf16_kimp_bounds, config_of, kimp_alloc, kimp_rows, make_layer, round_up, sets_from_mask,
+                     tie_band_ok, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +43,57 @@ def test_tcgen05_projection_prefill_scale(start, count):
         ref = O.project_keys(K[0, g, start:start + count], W)
         assert np.all(np.abs(got[0, g, start:start + count] - ref) <= _kimp_tol(K[0, g, start:start + count], W))
         assert np.all(np.isnan(got[0, g, :start])) and np.all(np.isnan(got[0, g, start + count:]))
+
+
+@pytest.mark.parametrize("kimp_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [(128, 32), (64, 16)], ids=["D128_d32", "D64_d16"])
+def test_tcgen05_projection_over_many_layers_in_one_launch(d, kimp_dtype):
+    """tb_project_kimp_layers: one persistent launch over 6 layers (each its
+    own cache, W_K and K_imp) equals tb_project_kimp layer by layer bit for
+    bit, and the fp64 oracle within the fp32 bound; rows outside
+    [start, start + count) stay untouched.  B=2, 2 KV heads, 3000 rows: a
+    CTA's tiles cross layer boundaries with both W_K^T buffers in use."""
+    D, dimp = d
+    wl = S.Workload("prefill_layers", n_layers=6, B=2, Hq=4, Hkv=2, D=D, d_imp=dimp, G=2, L=3000, dtype="bf16",
+                    keep_pct=50, sink=16, window=64, dense_layers=())
+    cfg = config_of(wl, max_len=3072, kimp_dtype=kimp_dtype)
+    multi, single = TB.Context(cfg), TB.Context(cfg)
+    start, count = 37, 2900
+    kd = torch.bfloat16 if kimp_dtype == "bf16" else torch.float32
+    layers = []
+    for layer in range(wl.n_layers):
+        K_raw = S.kv_cache_host(wl, layer, S.K_CACHE, 0, wl.L).reshape(wl.B, wl.Hkv, wl.L, D)
+        W_raw = S.w_k(wl, layer)
+        k = torch.zeros((wl.B, wl.Hkv, cfg.max_len, D), dtype=torch.bfloat16, device="cuda")
+        k[:, :, :wl.L] = to_dev(K_raw, wl)
+        w = to_dev(W_raw, wl)
+        km = kimp_alloc(wl.B, wl.Hkv, dimp, cfg.max_len, float("nan"), kd)
+        ks = kimp_alloc(wl.B, wl.Hkv, dimp, cfg.max_len, float("nan"), kd)
+        multi.bind_layer(layer, k, torch.zeros_like(k), km, w)
+        single.bind_layer(layer, k, torch.zeros_like(k), ks, w)
+        for ctx in (multi, single):
+            ctx.set_seq_lens(layer, [wl.L] * wl.B)
+        layers.append((K_raw, W_raw, km, ks))
+    multi.project_kimp_layers(0, wl.n_layers, start, count)
+    for layer in range(wl.n_layers):
+        single.project_kimp(layer, start, count)
+    torch.cuda.synchronize()
+    assert multi.check_status() == 0 and single.check_status() == 0
+    for layer, (K_raw, W_raw, km, ks) in enumerate(layers):
+        assert torch.equal(km.view(torch.int16) if kd == torch.bfloat16 else km.view(torch.int32),
+                           ks.view(torch.int16) if kd == torch.bfloat16 else ks.view(torch.int32)), f"layer {layer}"
+        got = kimp_rows(km)
+        K, W = S.widen(K_raw, wl.dtype), S.widen(W_raw, wl.dtype)
+        for b in range(wl.B):
+            for g in range(wl.Hkv):
+                Kr = K[b, g, start:start + count]
+                ref = O.project_keys(Kr, W)
+                if kimp_dtype == "bf16":
+                    lo, hi = bf16_kimp_bounds(Kr, W)
+                    assert np.all((got[b, g, start:start + count] >= lo) & (got[b, g, start:start + count] <= hi))
+                else:
+                    assert np.all(np.abs(got[b, g, start:start + count] - ref) <= _kimp_tol(Kr, W)), f"l{layer}"
+                assert np.all(np.isnan(got[b, g, :start])) and np.all(np.isnan(got[b, g, start + count:]))
 
 
 PF_SMALL = S.Workload("prefill_small", n_layers=8, B=2, Hq=8, Hkv=2, D=128, d_imp=32, G=4, L=3000, dtype="bf16",

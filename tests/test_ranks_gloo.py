@@ -115,3 +115,89 @@ def test_lockstep_rejects_ranks_out_of_step():
         run_lockstep([a(), b()])
     with pytest.raises(RuntimeError):
         run_lockstep([a(), iter(())])
+
+
+# ------------------------------------------------ shard_step itself over torch.distributed
+class _FakeLibrary:
+    """Stands in for a rank's library context on the CPU: every call that
+    shard_step makes records its inputs and writes rank-dependent values into
+    the real ShardBuffers, so the exchanges move the shapes and contents the
+    GPU path moves (no GPU in these tests)."""
+
+    def __init__(self, cfg, rank):
+        self.cfg, self.rank, self.seen = cfg, rank, []
+
+    def append_kv(self, layer, k, v, stream=None):
+        self.seen.append(("append", layer))
+
+    def shard_set(self, layer, t0, glens):
+        self.seen.append(("set", layer, t0, tuple(glens)))
+
+    def score(self, layer, q_imp, scores, stream=None):
+        scores.fill_(float(self.rank + 1))
+
+    def shard_hist(self, layer, scores, p, state, hist, stream=None):
+        hist.zero_()
+        hist[:, 7 * p + self.rank] = 1 + p + 10 * self.rank
+
+    def shard_pick(self, layer, p, hist, n_ranks, rank, state, stream=None):
+        self.seen.append(("pick", p, n_ranks, rank, hist.clone()))
+
+    def shard_mask(self, layer, scores, state, mask, stream=None):
+        mask.fill_(self.rank)
+
+    def sparse_attn_partial(self, layer, q, mask, mode, part, stream=None):
+        part.copy_(torch.arange(part.numel(), dtype=torch.float32) + 1000 * self.rank)
+
+    def merge_partials(self, parts, n, out, lse, stream=None):
+        self.seen.append(("merge", n, parts.clone()))
+
+
+def _shard_step_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from query_aware_sparse_decode_b200 import tb as TB
+    from query_aware_sparse_decode_b200.shard import ShardBuffers, TorchCollectives, shard_step
+    cfg = TB.make_config(2, 2, 8, 2, 64, 16, 1, 512, "bf16", 30, 4, 8, dense_layers=(0,))
+    lib = _FakeLibrary(cfg, rank)
+    bufs = ShardBuffers(cfg, world, torch.device("cpu"))
+    for layer in (0, 1):   # a dense layer (partials only) and a sparse one (all exchanges)
+        TorchCollectives().run(shard_step(lib, layer, rank, world, 256 * rank, [500, 480], None, None, None, bufs,
+                                          "k" if rank == world - 1 else None, "v" if rank == world - 1 else None))
+    q.put((rank, [(s[0],) + tuple(x.tolist() if torch.is_tensor(x) else x for x in s[1:]) for s in lib.seen]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_shard_step_over_torch_distributed_world2_matches_lockstep():
+    """shard_step's own exchange sequence (two summed histograms, a gathered
+    histogram, gathered partials) with the real ShardBuffers shapes, run by
+    TorchCollectives over two gloo processes, hands every library call the
+    same tensors as the one-process lock-step runner, rank order kept."""
+    from query_aware_sparse_decode_b200 import tb as TB
+    from query_aware_sparse_decode_b200.shard import ShardBuffers, run_lockstep, shard_step
+    ctx = mp.get_context("spawn")
+    qu = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_step_worker, args=(r, 2, port, qu)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(qu.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg = TB.make_config(2, 2, 8, 2, 64, 16, 1, 512, "bf16", 30, 4, 8, dense_layers=(0,))
+    libs = [_FakeLibrary(cfg, r) for r in range(2)]
+    bufs = [ShardBuffers(cfg, 2, torch.device("cpu")) for _ in range(2)]
+    for layer in (0, 1):
+        run_lockstep(shard_step(libs[r], layer, r, 2, 256 * r, [500, 480], None, None, None, bufs[r],
+                                "k" if r == 1 else None, "v" if r == 1 else None) for r in range(2))
+    for r in range(2):
+        want = [(s[0],) + tuple(x.tolist() if torch.is_tensor(x) else x for x in s[1:]) for s in libs[r].seen]
+        assert res[r] == want
+    # the summed first digit holds both ranks' counts; the last digit is gathered in rank order
+    picks = [s for s in libs[0].seen if s[0] == "pick"]
+    assert picks[0][4][0, 0].item() == 1 and picks[0][4][0, 1].item() == 11
+    assert picks[2][4].shape == (2, 2 * 8, 2048) and picks[2][4][1, 0, 15].item() == 13
+    merges = [s for s in libs[1].seen if s[0] == "merge"]
+    assert len(merges) == 2 and merges[1][2][1, 0].item() == 1000.0
