@@ -57,9 +57,15 @@ def parse():
                          "pool, addressed through a page table; 0 (default) keeps dense caches")
     ap.add_argument("--drift", type=float, default=0.05,
                     help="with --reuse: importance query of step s = q(0) + DRIFT * noise(s)")
+    ap.add_argument("--shard", action="store_true",
+                    help="sequence-sharded decode: every sequence's tokens split into one contiguous range per rank "
+                         "(ranks in token order, the last one appending), radix histograms and partial outputs "
+                         "exchanged per layer by NCCL collectives; strong scaling of the same workload")
     ap.add_argument("--trace-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-config-rows", action="store_true",
+                    help="leave out the other workloads' rows (8B-shaped L=32768, prefill path, L=128K/256K sweep)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--table", action="store_true",
                     help="instead of the step benchmark, print per-kernel times (one JSON line per row) for the "
@@ -184,6 +190,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def read_peak():
+    """(HBM GB/s, source): the measured copy bandwidth of MEASURED_PEAKS.json,
+    else the pool's earlier measurement (fallback)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def gpu_ident(dev, local_rank: int) -> str:
+    """nvidia-smi's id of the device (its UUID; the local rank otherwise)."""
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(local_rank)
+
+
 # ----------------------------------------------------------------------- DRAM traffic
 # DRAM bytes (read + write) per union K/V row of the sparse attention kernel,
 # from one ncu capture of it (B = 2, L = 131072, keep 30 %; summary under
@@ -253,20 +278,21 @@ def build(wl, max_len, dev, variant=None, kimp_dtype="f32"):
         ctx.bind_layer(layer, k, v, kimp, w)
         ctx.set_seq_lens(layer, [L0] * wl.B)
         bufs.append((k, v, kimp, w))
-    # prefill side of K_imp = K . W_K for every layer (tcgen05 GEMM), timed
-    # after one untimed launch (module load, shared-memory attribute)
+    # prefill side of K_imp = K . W_K for every layer: one persistent tcgen05
+    # launch over all layers, timed after one untimed launch (module load,
+    # shared-memory attribute)
     ctx.project_kimp(0, 0, min(L0, 1024))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for layer in range(wl.n_layers):
-        ctx.project_kimp(layer, 0, L0)
+    ctx.project_kimp_layers(0, wl.n_layers, 0, L0)
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / wl.n_layers
     rows = wl.B * wl.Hkv * L0
     nbytes = rows * (wl.D * 2 + wl.d_imp * kimp_elem_bytes(cfg))
-    proj = {"kernel": "butler_kimp_project (tcgen05, prefill of the cache)", "us_per_layer": us,
+    proj = {"kernel": "butler_kimp_project (tcgen05, prefill of the cache, one launch over all layers)",
+            "us_per_layer": us,
             "rows_per_layer": rows, "bytes_per_layer": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
             "tflops": 2 * rows * wl.D * wl.d_imp / (us * 1e-6) / 1e12}
     return ctx, bufs, proj
@@ -393,11 +419,7 @@ def gpu_arm(args, rank, world, local_rank):
     barrier()
 
     # ---- device-timed region: inputs resident in HBM
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        gpu_id = str(local_rank)
-    clocks = ClockSampler(gpu_id)
+    clocks = ClockSampler(gpu_ident(dev, local_rank))
     clocks.start()
     n0 = ctx.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -446,11 +468,7 @@ def gpu_arm(args, rank, world, local_rank):
     union_bytes = (sum(urows.values()) / max(len(urows), 1)) * row_kv
     dense_bytes = wl.B * wl.Hkv * wl.L * row_kv
     step_bytes = len(sparse_layers) * (kimp_bytes + union_bytes) + (wl.n_layers - len(sparse_layers)) * dense_bytes
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    peak, peak_src = 6650.0, "fallback"
-    if os.path.exists(peaks_path):
-        with open(peaks_path) as f:
-            peak, peak_src = float(json.load(f)["hbm_gbs"]), "measured"
+    peak, peak_src = read_peak()
     attn_gbs = union_bytes / (avg["attn"] * 1e-6) / 1e9 if avg["attn"] else None
     score_gbs = kimp_bytes / (avg["score"] * 1e-6) / 1e9 if avg["score"] else None
     pair_gbs = ((kimp_bytes + union_bytes) / ((avg["score"] + avg["attn"]) * 1e-6) / 1e9
@@ -486,67 +504,235 @@ def gpu_arm(args, rank, world, local_rank):
                 scored=scored, attended=attended)
 
 
-# ----------------------------------------------------------------------- CPU oracle leg
-def oracle_sample(wl, seconds: float, group: bool = False, kimp: str = "f32"):
-    """Times the fp64 oracle on whole (layer, sequence) slabs of the workload
-    (score, select, attend for all query heads; inputs regenerated on the host
-    and excluded from the timing) until about `seconds` of oracle work."""
-    from oracle import tokenbutler as O
+# ----------------------------------------------------------------------- sequence-sharded arm
+def shard_arm(args, rank, world, local_rank):
+    """The workload's decode step with every sequence split by token range
+    over the ranks (include/tb.h, "Sequence-sharded decode"; shard.py gives
+    the call order).  Rank r holds tokens [r * per, (r + 1) * per) of every
+    layer's caches; per layer the ranks exchange two summed radix histograms,
+    one gathered histogram and the gathered fp32 partial outputs with NCCL
+    (one rank: in-process copies).  The total work is fixed: strong scaling."""
+    import torch
+    import torch.distributed as dist
     from query_aware_sparse_decode_b200 import synth as S
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
+    from query_aware_sparse_decode_b200 import tb as TB
+    from query_aware_sparse_decode_b200.shard import ShardBuffers, TorchCollectives, run_lockstep, shard_step
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workload(args)
+    wl = wl.with_(name=wl.name + f"_sharded{world}")
     L0 = wl.L - 1
-    elapsed, tokens, slabs = 0.0, 0, []
+    per = (L0 + world - 1) // world
+    t0 = rank * per
+    n = max(0, min(per, L0 - t0))
+    last = rank == world - 1
+    cap = (n + 2 + 255) // 256 * 256
+    cfg = TB.make_config(wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.D, wl.d_imp, wl.G, cap, wl.dtype, wl.keep_pct, wl.sink,
+                         wl.window, dense_layers=wl.dense_layers)
+    ctx = TB.Context(cfg, dev)
+    bufs = []
+    for layer in range(wl.n_layers):
+        k = torch.empty((wl.B, wl.Hkv, cap, wl.D), dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        w_raw = S.w_k(wl, layer)
+        delta = None
+        if layer not in wl.dense_layers:
+            qi = S.widen(S.q_imp(wl, wl.G * (layer // wl.G), 0), "bf16")
+            qhat = qi[:, (layer - 1) % wl.G, 0, :].reshape(wl.B, wl.Hq, wl.d_imp)
+            delta = torch.from_numpy(S.plant_delta(S.widen(w_raw, "bf16"), qhat, wl.Hkv)).to(dev)
+        if n:
+            S.fill_device(k, S.K_CACHE, layer, 0, wl.B * wl.Hkv, t0, t0 + n, wl.D, cap * wl.D, wl.D, "bf16",
+                          delta=delta, plant_mod=100 if delta is not None else 0, seed=wl.seed, dst_t0=0)
+            S.fill_device(v, S.V_CACHE, layer, 0, wl.B * wl.Hkv, t0, t0 + n, wl.D, cap * wl.D, wl.D, "bf16",
+                          seed=wl.seed, dst_t0=0)
+        kimp = TB.kimp_cache(cfg, dev)
+        ctx.bind_layer(layer, k, v, kimp, torch.from_numpy(w_raw.view(np.int16)).view(torch.bfloat16).to(dev))
+        ctx.set_seq_lens(layer, [n] * wl.B)
+        bufs.append((k, v, kimp))
+    if n:
+        ctx.project_kimp_layers(0, wl.n_layers, 0, n)
+    sb = ShardBuffers(cfg, world, dev)
+    nvar = min(args.steps + args.warmup, 4)
+    host_inputs = [step_inputs_host(wl, s) for s in range(nvar)]
+    dev_inputs = [tuple(x.to(dev) for x in h) for h in host_inputs]
+    out = torch.empty((wl.n_layers, wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    coll = TorchCollectives() if world > 1 else None
+
+    def one_step(inp):
+        kn, vn, qq, qi = inp
+        for layer in range(wl.n_layers):
+            ctx.set_seq_lens(layer, [n] * wl.B)
+            st = shard_step(ctx, layer, rank, world, t0, [wl.L] * wl.B, qq[layer], qi[layer // wl.G], out[layer], sb,
+                            kn[layer] if last else None, vn[layer] if last else None, stream)
+            if coll is not None:
+                coll.run(st)
+            else:
+                run_lockstep([st])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for s in range(args.warmup):
+        one_step(dev_inputs[s % nvar])
+    barrier()
+    clocks = ClockSampler(gpu_ident(dev, local_rank))
+    clocks.start()
+    n0 = ctx.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for s in range(args.steps):
+        one_step(dev_inputs[s % nvar])
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    launches = ctx.launch_count() - n0
+    ms = max_over_ranks_of(e0.elapsed_time(e1), world, dev)
+    scored, attended = step_counts(wl)
+    value = (scored + attended) * args.steps / (ms / 1e3)   # the whole job's fixed work
+    # end to end: this rank's inputs copied in from pinned memory, the merged output read back
+    dbuf = tuple(torch.empty_like(x) for x in dev_inputs[0])
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for s in range(args.steps):
+        for dst, src in zip(dbuf, host_inputs[s % nvar]):
+            dst.copy_(src, non_blocking=True)
+        one_step(dbuf)
+        out_host.copy_(out, non_blocking=True)
+    f1.record(stream)
+    barrier()
+    ems = max_over_ranks_of(f0.elapsed_time(f1), world, dev)
+    status = ctx.check_status()
+    if status:
+        raise RuntimeError(f"device status flags {status:#x}")
+    if rank == 0:
+        peak, peak_src = read_peak()
+        kimp_b = wl.B * wl.Hkv * wl.L * wl.d_imp * 4
+        dense_b = wl.B * wl.Hkv * wl.L * 2 * wl.D * 2
+        nsp = sum(1 for l in range(wl.n_layers) if l not in wl.dense_layers)
+        step_bytes = nsp * kimp_b + (wl.n_layers - nsp) * dense_b
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "layers": wl.n_layers, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                           "D": wl.D, "d_imp": wl.d_imp, "G": wl.G, "L": wl.L, "keep_pct": wl.keep_pct,
+                           "sink": wl.sink, "window": wl.window, "dense_layers": list(wl.dense_layers),
+                           "selection": "per_query_head, sharded by token range", "tokens_per_rank": per,
+                           "parallelism": f"sequence-sharded x{world}",
+                           "l2": "inputs larger than L2 (caches of all layers, no flush)"},
+                "us_per_layer": ms / args.steps * 1e3 / wl.n_layers,
+                "tokens_scored_per_step": scored, "tokens_attended_per_step": attended,
+                "roofline": {"kernel": "a rank's whole sharded step (K_imp of sparse layers + dense K/V; the "
+                                       "attended rows are not counted, a lower bound)", "bound": "hbm",
+                             "achieved": step_bytes / world / (ms / args.steps * 1e-3) / 1e9, "peak": peak,
+                             "unit": "GB/s", "frac": step_bytes / world / (ms / args.steps * 1e-3) / 1e9 / peak,
+                             "traffic": None, "peak_source": peak_src},
+                "gpu_launches": launches, "clocks": clk,
+                "e2e": {"value": (scored + attended) * args.steps / (ems / 1e3), "unit": UNIT,
+                        "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host_inputs[0]),
+                        "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": ems / args.steps},
+                "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- CPU oracle leg
+def _oracle_slab(wl, layer, b, kimp):
+    """Host inputs of one (layer, sequence) slab of the workload at L: the
+    caches with the step's appended token, the queries and the cache's K_imp
+    (projected by the oracle; a decode step finds it in the cache)."""
+    from oracle import native as N
+    from query_aware_sparse_decode_b200 import synth as S
+    L0 = wl.L - 1
+    W = S.widen(S.w_k(wl, layer), wl.dtype)
+    qi = S.widen(S.q_imp(wl, N.producer_of(layer, wl.G), 0), wl.dtype)
+    qhat = N.importance_queries(qi, layer, wl.G, wl.B, wl.Hq)
+    delta = S.plant_delta(W, qhat, wl.Hkv)
+    K = S.widen(S.kv_cache_host(wl, layer, S.K_CACHE, 0, L0, delta, b_range=(b, 1)), wl.dtype)
+    V = S.widen(S.kv_cache_host(wl, layer, S.V_CACHE, 0, L0, b_range=(b, 1)), wl.dtype)
+    kn, vn = S.kv_new(wl, layer, 0)
+    K = np.concatenate([K, S.widen(kn, wl.dtype)[b][:, None]], axis=1)[None]
+    V = np.concatenate([V, S.widen(vn, wl.dtype)[b][:, None]], axis=1)[None]
+    Kimp = N.project_keys(K, W, "bf16" if kimp == "bf16" else "f64")
+    q = S.widen(S.query(wl, layer, 0), wl.dtype)[b:b + 1]
+    qi_b = qi.reshape(wl.B, wl.Hq, wl.G, 1, wl.d_imp)[b]
+    return q, K, V, W, qi_b, Kimp
+
+
+def oracle_sample(wl, seconds: float, group: bool = False, kimp: str = "f64", threads=None, max_runs: int = 64,
+                  n_inputs: int = 2):
+    """Times the C++ fp64 oracle (oracle/tokenbutler.cpp) on whole (layer,
+    sequence) slabs of the workload: the decode step's score, select and
+    attend for all query heads at L (a3-a6), with the cache's K_imp given.
+    `n_inputs` slabs are generated on the host outside the timed region and
+    timed in turn until about `seconds` of oracle work (at least one run,
+    at most `max_runs`), with `threads` OpenMP threads (default: every core)."""
+    from oracle import native as N
+    nproc = os.cpu_count() or 1
+    threads = nproc if threads is None else threads
+    N.set_threads(nproc)  # input preparation on every core
     sparse_layers = [l for l in range(wl.n_layers) if l not in wl.dense_layers] or [0]
-    i = 0
-    while (elapsed < seconds or i == 0) and i < 16:
+    inputs = []
+    for i in range(n_inputs):
         layer = sparse_layers[(1 + 7 * i) % len(sparse_layers)]
-        b = i % wl.B
-        W = S.widen(S.w_k(wl, layer), wl.dtype)
-        qi = S.widen(S.q_imp(wl, O.producer_of(layer, wl.G), 0), wl.dtype)
-        qhat = O.importance_queries(qi, layer, wl.G, wl.B, wl.Hq)
-        delta = S.plant_delta(W, qhat, wl.Hkv)
-        K = S.widen(S.kv_cache_host(wl, layer, S.K_CACHE, 0, L0, delta, b_range=(b, 1)), wl.dtype)
-        V = S.widen(S.kv_cache_host(wl, layer, S.V_CACHE, 0, L0, b_range=(b, 1)), wl.dtype)
-        kn, vn = S.kv_new(wl, layer, 0)
-        K = np.concatenate([K, S.widen(kn, wl.dtype)[b][:, None]], axis=1)[None]
-        V = np.concatenate([V, S.widen(vn, wl.dtype)[b][:, None]], axis=1)[None]
-        Kimp = O.project_keys(K, W, "bf16" if kimp == "bf16" else "f64")
-        q = S.widen(S.query(wl, layer, 0), wl.dtype)[b:b + 1]
-        qi_b = qi.reshape(wl.B, wl.Hq, wl.G, 1, wl.d_imp)[b]
+        inputs.append((layer, _oracle_slab(wl, layer, i % wl.B, kimp)))
+    N.set_threads(threads)
+    elapsed, tokens, runs = 0.0, 0, 0
+    while (elapsed < seconds or runs == 0) and runs < max_runs:
+        layer, (q, K, V, W, qi_b, Kimp) = inputs[runs % n_inputs]
         t0 = time.perf_counter()
-        sel, _, _, _ = O.decode_layer(q, K, V, W, qi_b, layer, wl.G, wl.L, wl.keep_pct, wl.sink, wl.window,
+        sel, _, _, _ = N.decode_layer(q, K, V, W, qi_b, layer, wl.G, wl.L, wl.keep_pct, wl.sink, wl.window,
                                       dense=False, K_imp=Kimp, group=group)
-        dt = time.perf_counter() - t0
-        elapsed += dt
+        elapsed += time.perf_counter() - t0
         tokens += wl.Hq * wl.L + sum(len(v) for v in sel.values())
-        slabs.append((layer, b))
-        i += 1
-    return {"value": tokens / elapsed, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(slabs)} (layer, sequence) slabs of {wl.name}: score + select + attend for all "
-                      f"{wl.Hq} query heads at L={wl.L}, fp64 numpy, {elapsed:.1f} s"}
+        runs += 1
+    return {"value": tokens / elapsed, "unit": UNIT, "threads": threads, "runs": runs, "inputs": n_inputs,
+            "seconds": elapsed}
+
+
+def cpu_baseline(wl, seconds: float, group: bool = False, kimp: str = "f64"):
+    """The oracle single-threaded and on every core of the host (about
+    `seconds` each); the line's value is the all-core rate."""
+    nproc = os.cpu_count() or 1
+    single = oracle_sample(wl, seconds / 2, group, kimp, threads=1, max_runs=2, n_inputs=1)
+    allc = oracle_sample(wl, seconds / 2, group, kimp, threads=nproc)
+    return {"value": allc["value"], "unit": UNIT, "cores": nproc, "kind": "oracle",
+            "sample": f"{allc['runs']} runs over {allc['inputs']} (layer, sequence) slabs of {wl.name} on {nproc} "
+                      f"threads and {single['runs']} on one: score + select + attend (a3-a6) for all {wl.Hq} query "
+                      f"heads at "
+                      f"L={wl.L}, the cache's K_imp projected outside the timed region, C++ fp64 oracle, "
+                      f"{allc['seconds']:.1f} s + {single['seconds']:.1f} s",
+            "single": {"value": single["value"], "threads": 1},
+            "all_core": {"value": allc["value"], "threads": nproc},
+            "cores_nproc": nproc, "omp_num_threads": os.environ.get("OMP_NUM_THREADS")}
 
 
 def reference_arm(args, rank, world):
+    """The oracle as the reference arm: each step one (layer, sequence) slab
+    of the workload on every host core (rank 0 only; other ranks exit)."""
     if rank != 0:
         return
     wl = workload(args)
     vals = []
     for s in range(args.warmup + args.steps):
-        r = oracle_sample(wl, seconds=0.0, group=args.variant == "group", kimp=args.kimp)  # one slab per step
+        r = oracle_sample(wl, seconds=0.0, group=args.variant == "group", kimp=args.kimp, max_runs=1, n_inputs=1)
         if s >= args.warmup:
             vals.append(r)
     value = statistics.mean(v["value"] for v in vals)
+    nproc = os.cpu_count() or 1
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "L": wl.L, "layers": wl.n_layers, "keep_pct": wl.keep_pct,
                        "sink": wl.sink, "window": wl.window},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": "each step: " + vals[0]["sample"]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nproc, "kind": "oracle",
+                             "sample": f"each step: one (layer, sequence) slab of {wl.name}: score + select + "
+                                       f"attend (a3-a6) for all {wl.Hq} query heads at L={wl.L}, the cache's K_imp "
+                                       f"projected outside the timed region, C++ fp64 oracle on {nproc} threads"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -589,7 +775,7 @@ def _variant_name(variant):
     return {TB.TB_SOFTVOTE: "softvote", TB.TB_BUTLER_GROUP: "group"}.get(variant, "butler")
 
 
-def _table_case(wl, variant, dev, iters, flush_buf, peak):
+def _table_case(wl, variant, dev, iters, flush_buf, peak, hot_l2=True):
     import torch
     from query_aware_sparse_decode_b200 import synth as S
     from query_aware_sparse_decode_b200 import tb as TB
@@ -603,7 +789,7 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
     kn, vn = S.kv_new(wl, layer)
     inp = (bf(kn), bf(vn), bf(S.query(wl, layer)), bf(S.q_imp(wl, 0)))
     cold = _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream)
-    hot = _timed_decode(ctx, wl, layer, inp, iters, None, stream)
+    hot = _timed_decode(ctx, wl, layer, inp, iters, None, stream) if hot_l2 else None
     # algorithmic bytes from the library's own selection of this step
     ctx.set_seq_lens(layer, [wl.L] * wl.B)
     dense = wl.keep_pct >= 100 or layer in wl.dense_layers
@@ -651,7 +837,8 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak):
     line = {"table": "decode", "workload": wl.name, "variant": _variant_name(variant),
             "B": wl.B, "L": wl.L, "keep_pct": wl.keep_pct, "dense": dense,
             "first_pass_bytes": first, "union_rows": union, "attn_bytes": attn_bytes,
-            "us_cold_l2": cold, "us_hot_l2": hot, "rates_cold_l2": rates(cold), "rates_hot_l2": rates(hot),
+            "us_cold_l2": cold, "us_hot_l2": hot, "rates_cold_l2": rates(cold),
+            "rates_hot_l2": rates(hot) if hot is not None else None,
             "l2": "cold: 512 MB write + 256 MB read before each step; hot: back-to-back steps",
             "iters": iters,
             "peak_gbs": peak}
@@ -791,6 +978,45 @@ def _table_shard(wl, ranks_list, dev, iters, flush_buf, variant=None):
             "rows": rows_out}
 
 
+def config_rows(dev, iters, peak, n_layers_prefill=32):
+    """The rows of the other workloads carried in the default bench line:
+    the 8B-shaped single layer at L=32768 (50 % and dense), the prefill
+    importance path (K_imp GEMM over 32 layers and the 1024-row causal
+    selection) and the long-context sweep at L = 131072 and 262144 for the
+    TokenButler and soft-voting variants at 10/30/50 %.  Per row: median
+    per-kernel times of 20 single cold-L2 decode steps and the fraction of
+    the HBM peak reached by the first pass (score, or soft-vote logits) plus
+    the attention."""
+    import torch
+    from query_aware_sparse_decode_b200 import synth as S
+    from query_aware_sparse_decode_b200 import tb as TB
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    cases = [(S.LLAMA8B_L32K, TB.TB_BUTLER), (S.LLAMA8B_L32K.with_(keep_pct=100), TB.TB_BUTLER)]
+    for L in (131072, 262144):
+        for P in S.SWEEP_KEEP:
+            cases += [(S.sweep(L, P), TB.TB_BUTLER), (S.sweep(L, P), TB.TB_SOFTVOTE)]
+    rows = []
+    for wl, variant in cases:
+        line = _table_case(wl, variant, dev, iters, flush_buf, peak, hot_l2=False)
+        t, rt = line["us_cold_l2"], line["rates_cold_l2"]
+        rows.append({"workload": line["workload"], "variant": line["variant"], "L": line["L"],
+                     "keep_pct": line["keep_pct"], "dense": line["dense"],
+                     "us": {k: round(t[k], 2) for k in ("score", "select", "attn", "combine", "total")},
+                     "first_pass_bytes": line["first_pass_bytes"], "attn_bytes": line["attn_bytes"],
+                     "pair_frac": (round(rt["score_plus_attn_frac"], 4) if "score_plus_attn_frac" in rt else None),
+                     "attn_frac": round(rt["attn_frac"], 4)})
+    del flush_buf
+    torch.cuda.empty_cache()
+    pf = _table_prefill(dev, iters, peak, n_layers_prefill)
+    prefill = {"kimp_gemm_us_per_layer": round(pf["kimp_gemm"]["us_per_layer"], 2),
+               "kimp_gemm_frac_hbm": round(pf["kimp_gemm"]["frac_hbm"], 4),
+               "kimp_gemm_tflops": round(pf["kimp_gemm"]["tflops"], 1),
+               "select_rows_us": round(pf["select_prefill"]["us_median"], 1),
+               "select_rows_elements_per_s": pf["select_prefill"]["elements_per_s"]}
+    return {"decode_rows": rows, "prefill": prefill, "peak_gbs": peak,
+            "timing": "median of single decode steps, L2 flushed before each (512 MB write, 256 MB read)"}
+
+
 def kernel_table(args):
     """Per-kernel times for the workloads beside the step benchmark: the
     8B-shaped L=32768 case (50 % and dense), the long-context sweep of both
@@ -800,11 +1026,7 @@ def kernel_table(args):
     from query_aware_sparse_decode_b200 import tb as TB
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    peak = 6650.0
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(peaks_path):
-        with open(peaks_path) as f:
-            peak = float(json.load(f)["hbm_gbs"])
+    peak, _ = read_peak()
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     cases = [(S.LLAMA8B_L32K, TB.TB_BUTLER), (S.LLAMA8B_L32K.with_(keep_pct=100), TB.TB_BUTLER)]
     for L in S.SWEEP_LENGTHS:
@@ -846,10 +1068,24 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
+    if args.shard:
+        shard_arm(args, rank, world, local_rank)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     r = gpu_arm(args, rank, world, local_rank)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(r["wl"], args.cpu_seconds, group=args.variant == "group", kimp=args.kimp)
+        cpu = cpu_baseline(r["wl"], args.cpu_seconds, group=args.variant == "group", kimp=args.kimp)
+    extra = None
+    if rank == 0 and world == 1 and not args.no_config_rows:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        clk = ClockSampler(gpu_ident(dev, local_rank))
+        clk.start()
+        extra = config_rows(dev, args.table_iters, r["peak"])
+        extra["clocks"] = clk.stop()
     if rank == 0:
         wl = r["wl"]
         avg = r["avg"]
@@ -891,6 +1127,7 @@ def main():
             "clocks": r["clk"],
             "e2e": r["e2e"],
             "cpu_baseline": cpu,
+            "config_rows": extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -107,14 +107,16 @@ def fill_host(kind: int, layer: int, step: int, A: int, t0: int, t1: int, C: int
 
 def fill_device(tensor, kind: int, layer: int, step: int, A: int, t0: int, t1: int, C: int,
                 stride_a: int, stride_t: int, dtype: str, scale: float = 1.0, delta=None,
-                plant_mod: int = 0, seed: int = 0, stream=None) -> None:
+                plant_mod: int = 0, seed: int = 0, stream=None, dst_t0: int | None = None) -> None:
     """Fill rows t0 <= t < t1 of a device tensor whose element (a, t, c) sits
-    at a*stride_a + t*stride_t + c, with the same bits :func:`fill_host` gives.
-    ``delta`` is a device fp32 tensor [A][C] or None."""
+    at a*stride_a + (t - t0 + dst_t0)*stride_t + c (dst_t0 = t0 by default:
+    row t of the tensor holds row t), with the same bits :func:`fill_host`
+    gives.  ``delta`` is a device fp32 tensor [A][C] or None."""
     import torch
     if stream is None:
         stream = torch.cuda.current_stream().cuda_stream
-    base = tensor.data_ptr() + t0 * stride_t * tensor.element_size()  # element (0, t0)
+    row = t0 if dst_t0 is None else dst_t0
+    base = tensor.data_ptr() + row * stride_t * tensor.element_size()  # element (0, t0)
     rc = _dev_lib().tbs_fill_device(ctypes.c_void_p(base), _DTYPE_CODE[dtype], 0, A, t0, t1, C,
                                     stride_a, stride_t, key(seed, stream_id(kind, layer, step)),
                                     np.float32(scale), None if delta is None else ctypes.c_void_p(delta.data_ptr()),
