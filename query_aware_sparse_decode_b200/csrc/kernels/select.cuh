@@ -659,100 +659,4 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_resolve_kernel(const Se
   clear_row_state(p, row, b);
 }
 
-// ---------------------------------------------------------------- short rows
-// Rows of at most kRowMax tokens: one 1024-thread CTA per row does the whole
-// selection in shared memory, in one launch instead of scatter + resolve
-// (whose global candidate lists and two dependent launches dominate short
-// rows).  The row's order keys are staged in shared memory; the first digit
-// comes from the score kernel's fused histogram when it is ready, the other
-// digits from smem_radix over the staged keys.  Ties at the threshold key go to
-// the lowest indices: when every key equal to T is kept no ordering is needed,
-// otherwise an ordered block scan assigns the quota.  Mask words of the row's
-// tokens, the optional count, the count check and the clearing of the row's
-// histograms and counters follow as in the resolve kernel.  Index lists and
-// amortised selection take the scatter + resolve path.  Above 16384 tokens
-// the many-CTA scatter wins (L = 32768 at B = 1: 29.7 against 23.5 us).
-constexpr int kRowMax = 16384;
-constexpr int kRowSmem = (kRowMax + kHistBins) * 4;
-__global__ void __launch_bounds__(kSelThreads, 1) select_row_kernel(const SelectParams p, int hist1_ready) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) uint32_t row_smem[];
-  uint32_t* keys = row_smem;              // [kRowMax] order keys of the row
-  uint32_t* hist = row_smem + kRowMax;    // [2048]
-  __shared__ uint32_t scan_sm[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
-  const int r = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-  const RowShape rs = row_shape(p, b);
-  const long long row = (long long)b * p.rows_per_seq + r;
-  const float* s = p.scores + row * p.row_stride;
-  uint32_t T = 0, quota = 0;
-  if (rs.mode == 2) {
-    for (int t = rs.lo + tid; t < rs.hi; t += kSelThreads) keys[t] = order_key(s[t]);
-    uint32_t prefix = 0, kk = (uint32_t)rs.k;
-    int first = 0;
-    if (hist1_ready) {  // first digit: the score kernel's histogram of the candidates
-      for (int i = tid; i < kHistBins; i += kSelThreads) hist[i] = p.hist1[row * kHistBins + i];
-      __syncthreads();
-      find_bin<kHistBins / kSelThreads>(hist, kk, scan_sm, &s_bin, &s_above);
-      kk -= s_above;
-      prefix = (uint32_t)s_bin;
-      first = 1;
-    }
-    __syncthreads();
-    smem_radix(
-        rs.hi - rs.lo,
-        [&](int i, uint32_t& key) {
-          key = keys[rs.lo + i];
-          return true;
-        },
-        first, prefix, kk, hist, scan_sm, &s_bin, &s_above, T, quota);
-  }
-  // keys equal to T: all kept (no ordering needed), or the quota lowest indices
-  bool all_ties = true;
-  if (rs.mode == 2) {
-    uint32_t mine = 0;
-    for (int t = rs.lo + tid; t < rs.hi; t += kSelThreads) mine += keys[t] == T;
-    uint32_t ntie;
-    (void)block_excl_scan<kSelThreads>(mine, ntie, scan_sm);
-    all_ties = ntie == quota;
-  }
-  uint32_t* m = p.mask + row * p.mask_words;
-  uint32_t tie_base = 0, count = 0;
-  for (int base = 0; base < rs.L; base += kSelThreads) {
-    const int t = base + tid;
-    bool keep = false, tie = false;
-    if (t < rs.L) {
-      const bool cand = t >= rs.lo && t < rs.hi;
-      keep = !cand || rs.mode == 1;
-      if (cand && rs.mode == 2) {
-        const uint32_t key = keys[t];
-        keep = key > T || (all_ties && key == T);
-        tie = !all_ties && key == T;
-      }
-    }
-    if (!all_ties) {  // uniform in the CTA
-      uint32_t total;
-      const uint32_t ex = block_excl_scan<kSelThreads>(tie ? 1u : 0u, total, scan_sm);
-      if (tie && tie_base + ex < quota) keep = true;
-      tie_base += total;
-    }
-    const uint32_t word = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0 && t < rs.L) {
-      m[t >> 5] = word;
-      count += __popc(word);
-    }
-  }
-  uint32_t total;
-  (void)block_excl_scan<kSelThreads>(count, total, scan_sm);
-  if (tid == 0) {
-    if (p.count != nullptr) p.count[row] = (int32_t)total;
-    const int sink_n = min(p.sink, rs.L);
-    const int win_lo = max(rs.L - p.window, sink_n);
-    if (total != (uint32_t)(sink_n + (rs.L - win_lo) + rs.k)) atomicOr(p.status, TB_DEV_ERR_COUNT);
-  }
-  clear_row_state(p, row, b);
-}
-
 }  // namespace tb

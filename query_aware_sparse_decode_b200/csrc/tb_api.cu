@@ -349,15 +349,8 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
     if (s == TB_OK) ctx->hist_clean = true;  // CTA 0 of every row clears the row's histogram
     return s;
   }
-  if (maxL <= kRowMax && !use_cache && idx == nullptr) {  // short rows: one CTA per row, one launch
-    cudaFuncSetAttribute(select_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmem);
-    launch_pdl(select_row_kernel, dim3(rows, c.batch), dim3(kSelThreads), (size_t)kRowSmem, st, p,
-               hist1_ready ? 1 : 0);
-    ++ctx->launches;
-    const tb_status s = cuda_status(cudaGetLastError());
-    if (s == TB_OK) ctx->hist_clean = true;  // every row CTA clears its row's state
-    return s;
-  }
+  // rows longer than one cluster reaches: many CTAs per row scatter the
+  // threshold bin's candidates, one CTA per row resolves them
   dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
   if (!hist1_ready) {
     prepare_hist(ctx, st);
