@@ -10,9 +10,12 @@
 // row of the group's union is gathered from HBM exactly once and serves all
 // heads (a per-token head bitmask masks the scores).  Rows are gathered by
 // cp.async into an XOR-swizzled shared-memory ring (3 stages per warp).
-// QK^T and PV run on mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the
-// group's heads as the M rows; the online softmax is kept in fp32 in the
-// log2 domain.  Each CTA writes one (m, l, o) partial per head; the combine
+// Both products run on mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the
+// group's heads as the 8 N columns: S^T = K Q^T takes the K tile as A
+// (ldmatrix), O^T = V^T P^T takes the V tile as A (ldmatrix.trans) and P^T
+// as B (movmatrix.trans of the softmax fragment), so a 16-token tile costs
+// D/8 mma whatever the group size.  The online softmax is kept in fp32 in
+// the log2 domain.  Each CTA writes one (m, l, o) partial per head; the combine
 // kernel merges the chunks with an fp32 log-sum-exp.
 #pragma once
 
@@ -147,8 +150,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   constexpr int ROWB = D * 2;                       // bytes per K or V row
   constexpr int NCH = D / 8;                        // 16-byte pieces per row
   constexpr int STAGE = 2 * kAttnTile * ROWB;       // K tile + V tile
-  constexpr int KSTEPS = D / 16;
-  constexpr int NT = D / 8;                         // n-tiles of the output
+  constexpr int KSTEPS = D / 16;                    // k-steps of S^T = K Q^T
+  constexpr int MT = D / 16;                        // m-tiles of O^T = V^T P^T
+  constexpr int RPL = kAttnTile * NCH / 32;         // rows a lane copies per tensor
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   int32_t* list_idx = reinterpret_cast<int32_t*>(smem + kAttnWarps * kAttnStages * STAGE);
@@ -167,26 +171,45 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache);
   const uint8_t* Vb = reinterpret_cast<const uint8_t*>(p.v_cache);
 
-  // A fragments of Q (rows = the group's heads; rows >= GS and 8..15 are 0).
-  // Logical k (2tq + {0,1}) of k-step kk maps to dims (4(kk/2)+tq)*8 + (kk%2)*4 + {0,1},
-  // logical k (2tq + 8 + {0,1}) to the same + {2,3}; K uses the same map.
-  uint32_t qa[KSTEPS][2];
+  // The tile's tokens are the M rows of S^T = K Q^T (A = the K tile, B = Q^T
+  // with the group's heads as its 8 columns, heads >= GS zero) and the K
+  // dimension of O^T = V^T P^T (A = the V tile read transposed, B = P^T):
+  // no mma row is spent on absent heads.  B fragments of Q^T: lane (grp, tq)
+  // holds head grp, dims 16kk + 2tq + {0,1} and 16kk + 8 + 2tq + {0,1}.
+  uint32_t qb[KSTEPS][2];
   {
     const __nv_bfloat16* qrow =
         reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * GS + (grp < GS ? grp : 0)) * D;
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
-      const int dim = (4 * (kk / 2) + tq) * 8 + (kk % 2) * 4;
-      qa[kk][0] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim) : 0u;
-      qa[kk][1] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim + 2) : 0u;
+      qb[kk][0] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq) : 0u;
+      qb[kk][1] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * tq) : 0u;
     }
   }
+  // the two heads (columns 2tq, 2tq+1) whose scores and outputs this lane holds
+  const uint32_t head_bits = ((1u << GS) - 1u) >> (2 * tq) & 3u;
 
-  float o[NT][2];
+  // o[mt][0..1]: dims 16mt + grp, heads 2tq + {0,1}; o[mt][2..3]: dims 16mt + grp + 8
+  float o[MT][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = 0.f;
-  float m_run = kNegInf, l_run = 0.f;
+  for (int j = 0; j < MT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};
   uint8_t* my_ring = ring + warp * kAttnStages * STAGE;
+  const uint32_t ring_u32 = smem_u32(my_ring);
+
+  // ldmatrix row addresses: lane supplies row (lane & 7) of matrix (lane >> 3).
+  // K (S^T A operand): matrix j = tokens 8(j & 1) + r, piece 2kk + (j >> 1).
+  // V (O^T A operand, transposed): matrix j = tokens 8(j >> 1) + r, piece 2mt + (j & 1).
+  // The swizzled piece (c ^ r) of row r is (2kk ^ (c_low ^ r)) for even 2kk.
+  const int lr = lane & 7, lj = lane >> 3;
+  const uint32_t k_row_off = (uint32_t)((lr + 8 * (lj & 1)) * ROWB);
+  const uint32_t k_x = (uint32_t)(((lj >> 1) ^ lr) << 4);
+  const uint32_t v_row_off = (uint32_t)((lr + 8 * (lj >> 1)) * ROWB + kAttnTile * ROWB);
+  const uint32_t v_x = (uint32_t)(((lj & 1) ^ lr) << 4);
+
+  // gather: lane copies piece (lane % NCH) of rows (lane / NCH) * RPL + i of
+  // the tile, from K and from V at the same offset
+  const int g_part = lane % NCH, g_row0 = (lane / NCH) * RPL;
 
   // the CTA's chunk is processed in sub-chunks of up to kAttnMaxChunk tokens
   // (one gather list each); the softmax state carries across them
@@ -195,23 +218,25 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   const int ntiles = n / kAttnTile + (n % kAttnTile ? 1 : 0);
   const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
 
-  // A lane copies the same 16-byte pieces of its rows from K and from V: the
-  // rows' cache indices are read from the list once, before the copies.
-  constexpr int PER = kAttnTile * NCH / 32;  // pieces per lane and tensor
   auto issue = [&](int it) {
     const int tile = warp + it * kAttnWarps;
     uint8_t* sb = my_ring + (it % kAttnStages) * STAGE;
-    int tok[PER];
+    int tok[RPL];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) tok[i] = list_idx[tile * kAttnTile + (lane + 32 * i) / NCH];
+    for (int i = 0; i < RPL; i += 4) {
+      const int4 t4 = *reinterpret_cast<const int4*>(list_idx + tile * kAttnTile + g_row0 + i);
+      tok[i] = t4.x;
+      tok[i + 1] = t4.y;
+      tok[i + 2] = t4.z;
+      tok[i + 3] = t4.w;
+    }
 #pragma unroll
-    for (int tensor = 0; tensor < 2; ++tensor) {
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const int rc = lane + 32 * i, row = rc / NCH, part = rc % NCH;
-        cp_async_16(sb + tensor * kAttnTile * ROWB + row * ROWB + ((part ^ (row & 7)) << 4),
-                    (tensor ? Vb : Kb) + (size_t)tok[i] * ROWB + part * 16);
-      }
+    for (int i = 0; i < RPL; ++i) {
+      const int row = g_row0 + i;
+      const size_t off = (size_t)tok[i] * ROWB + g_part * 16;
+      uint8_t* dst = sb + row * ROWB + ((g_part ^ (row & 7)) << 4);
+      cp_async_16(dst, Kb + off);
+      cp_async_16(dst + kAttnTile * ROWB, Vb + off);
     }
   };
 #pragma unroll
@@ -225,72 +250,63 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
     cp_async_commit();
     cp_async_wait<kAttnStages - 1>();
     __syncwarp();
-    const uint8_t* Ks = my_ring + (it % kAttnStages) * STAGE;
-    const uint8_t* Vs = Ks + kAttnTile * ROWB;
+    const uint32_t st = ring_u32 + (uint32_t)((it % kAttnStages) * STAGE);
     const int tile = warp + it * kAttnWarps;
 
-    // ---- S = Q K^T for tokens 0..7 (acc0) and 8..15 (acc1) of the tile
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- S^T = K Q^T: s[0..1] = tokens grp, s[2..3] = tokens grp + 8; heads 2tq + {0,1}
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      const int c = 4 * i + tq;
-      const uint4 k0 = *reinterpret_cast<const uint4*>(Ks + grp * ROWB + ((c ^ (grp & 7)) << 4));
-      const uint4 k1 = *reinterpret_cast<const uint4*>(Ks + (grp + 8) * ROWB + ((c ^ ((grp + 8) & 7)) << 4));
-      mma_16816(acc0, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k0.x, k0.y);
-      mma_16816(acc0, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k0.z, k0.w);
-      mma_16816(acc1, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k1.x, k1.y);
-      mma_16816(acc1, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k1.z, k1.w);
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(a, st + k_row_off + (((uint32_t)(32 * kk)) ^ k_x));
+      mma_16816(s, a[0], a[1], a[2], a[3], qb[kk][0], qb[kk][1]);
     }
 
-    // ---- masked online softmax (log2 domain) for head row `grp`
-    const uint8_t* hb = list_hb + tile * kAttnTile;
-    const bool real = grp < GS;
-    const float s0 = real && ((hb[2 * tq] >> grp) & 1) ? acc0[0] * p.scale_log2 : kNegInf;
-    const float s1 = real && ((hb[2 * tq + 1] >> grp) & 1) ? acc0[1] * p.scale_log2 : kNegInf;
-    const float s2 = real && ((hb[2 * tq + 8] >> grp) & 1) ? acc1[0] * p.scale_log2 : kNegInf;
-    const float s3 = real && ((hb[2 * tq + 9] >> grp) & 1) ? acc1[1] * p.scale_log2 : kNegInf;
-    float mt = fmaxf(fmaxf(s0, s1), fmaxf(s2, s3));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-    const float m_new = fmaxf(m_run, mt);
-    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f, alpha = 1.f;
-    if (m_new != kNegInf) {
-      alpha = fast_exp2(m_run - m_new);
-      p0 = fast_exp2(s0 - m_new);
-      p1 = fast_exp2(s1 - m_new);
-      p2 = fast_exp2(s2 - m_new);
-      p3 = fast_exp2(s3 - m_new);
+    // ---- masked online softmax (log2 domain) per head column
+    const uint32_t hb0 = list_hb[tile * kAttnTile + grp] >> (2 * tq) & head_bits;
+    const uint32_t hb1 = list_hb[tile * kAttnTile + grp + 8] >> (2 * tq) & head_bits;
+    float x[4];
+    x[0] = (hb0 & 1u) ? s[0] * p.scale_log2 : kNegInf;
+    x[1] = (hb0 & 2u) ? s[1] * p.scale_log2 : kNegInf;
+    x[2] = (hb1 & 1u) ? s[2] * p.scale_log2 : kNegInf;
+    x[3] = (hb1 & 2u) ? s[3] * p.scale_log2 : kNegInf;
+    float mt0 = fmaxf(x[0], x[2]), mt1 = fmaxf(x[1], x[3]);
+#pragma unroll
+    for (int sh = 4; sh < 32; sh <<= 1) {
+      mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, sh));
+      mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, sh));
     }
-    m_run = m_new;
-    l_run = l_run * alpha + (p0 + p1) + (p2 + p3);
+    const float mn0 = fmaxf(m_run[0], mt0), mn1 = fmaxf(m_run[1], mt1);
+    // a head with no kept token so far subtracts 0: every exponent is -inf
+    const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
+    const float al0 = m_run[0] == mu0 ? 1.f : fast_exp2(m_run[0] - mu0);
+    const float al1 = m_run[1] == mu1 ? 1.f : fast_exp2(m_run[1] - mu1);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    const float p0 = fast_exp2(x[0] - mu0), p1 = fast_exp2(x[1] - mu1);
+    const float p2 = fast_exp2(x[2] - mu0), p3 = fast_exp2(x[3] - mu1);
+    l_run[0] = l_run[0] * al0 + (p0 + p2);
+    l_run[1] = l_run[1] * al1 + (p1 + p3);
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      o[j][0] *= alpha;
-      o[j][1] *= alpha;
-    }
-    const uint32_t pa0 = pack_bf16(p0, p1), pa2 = pack_bf16(p2, p3);
-
-    // ---- O += P V: lane holds dims hf*64 + grp*8 + e of tokens 2tq, 2tq+1, 2tq+8, 2tq+9
-#pragma unroll
-    for (int hf = 0; hf < D / 64; ++hf) {
-      const int c = hf * 8 + grp;
-      const int r0 = 2 * tq, r1 = 2 * tq + 1, r2 = 2 * tq + 8, r3 = 2 * tq + 9;
-      const uint4 va = *reinterpret_cast<const uint4*>(Vs + r0 * ROWB + ((c ^ (r0 & 7)) << 4));
-      const uint4 vb = *reinterpret_cast<const uint4*>(Vs + r1 * ROWB + ((c ^ (r1 & 7)) << 4));
-      const uint4 vc = *reinterpret_cast<const uint4*>(Vs + r2 * ROWB + ((c ^ (r2 & 7)) << 4));
-      const uint4 vd = *reinterpret_cast<const uint4*>(Vs + r3 * ROWB + ((c ^ (r3 & 7)) << 4));
-      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-      const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t sel = (e & 1) ? 0x7632u : 0x5410u;
-        const uint32_t b0 = __byte_perm(wa[e >> 1], wb[e >> 1], sel);
-        const uint32_t b1 = __byte_perm(wc[e >> 1], wd[e >> 1], sel);
-        float dd[4] = {o[hf * 8 + e][0], o[hf * 8 + e][1], 0.f, 0.f};
-        mma_16816(dd, pa0, 0u, pa2, 0u, b0, b1);
-        o[hf * 8 + e][0] = dd[0];
-        o[hf * 8 + e][1] = dd[1];
+      for (int j = 0; j < MT; ++j) {
+        o[j][0] *= al0;
+        o[j][1] *= al1;
+        o[j][2] *= al0;
+        o[j][3] *= al1;
       }
+    }
+    // P (tokens x heads, C layout) -> P^T B fragments: b0 = tokens 2tq + {0,1},
+    // b1 = tokens 2tq + 8 + {0,1}, head grp
+    const uint32_t pb0 = movmatrix_trans(pack_bf16(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16(p2, p3));
+
+    // ---- O^T += V^T P^T
+#pragma unroll
+    for (int j = 0; j < MT; ++j) {
+      uint32_t a[4];
+      ldsm_x4_trans(a, st + v_row_off + (((uint32_t)(32 * j)) ^ v_x));
+      mma_16816(o[j], a[0], a[1], a[2], a[3], pb0, pb1);
     }
     __syncwarp();
   }
@@ -299,25 +315,30 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_bf16_kernel(const AttnPa
   }
 
   // ---- merge the four warps through shared memory (reuses the ring)
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+#pragma unroll
+  for (int sh = 4; sh < 32; sh <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], sh);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], sh);
+  }
   __syncthreads();
   float* wm = reinterpret_cast<float*>(ring);
   float* wl = wm + kAttnWarps * GS;
   float* wo = wl + kAttnWarps * GS;
-  if (grp < GS) {
-    if (tq == 0) {
-      wm[warp * GS + grp] = m_run;
-      wl[warp * GS + grp] = l_run;
-    }
 #pragma unroll
-    for (int hf = 0; hf < D / 64; ++hf)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float* dst = wo + (warp * GS + grp) * D + hf * 64 + e;
-        dst[(2 * tq) * 8] = o[hf * 8 + e][0];
-        dst[(2 * tq + 1) * 8] = o[hf * 8 + e][1];
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * tq + e;
+    if (h < GS) {
+      if (grp == 0) {
+        wm[warp * GS + h] = m_run[e];
+        wl[warp * GS + h] = l_run[e];
       }
+      float* dst = wo + (warp * GS + h) * D;
+#pragma unroll
+      for (int j = 0; j < MT; ++j) {
+        dst[16 * j + grp] = o[j][e];
+        dst[16 * j + grp + 8] = o[j][2 + e];
+      }
+    }
   }
   __syncthreads();
   write_partial<D, GS>(p, b, g, split, wm, wl, wo);
