@@ -770,6 +770,75 @@ def _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream):
     return med
 
 
+def _cold_batched(fn, flush, reps=5, k=10):
+    """Device time (us) of one call of `fn` starting with a cold L2 and no
+    launch gap: `k` pairs (flush, fn) queued back to back minus `k` flushes
+    queued alone, the two interleaved `reps` times, median of the
+    differences.  The flush is a 256 MB read, so the call starts with L2 full
+    of clean, unrelated lines; as in a chained decode step, the call's launch
+    is processed while the work before it runs."""
+    import torch
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    fn()
+    flush()
+    torch.cuda.synchronize()
+    diffs = []
+    for _ in range(reps):
+        e[0].record()
+        for _ in range(k):
+            flush()
+        e[1].record()
+        for _ in range(k):
+            flush()
+            fn()
+        e[2].record()
+        torch.cuda.synchronize()
+        diffs.append((e[1].elapsed_time(e[2]) - e[0].elapsed_time(e[1])) * 1e3 / k)
+    return statistics.median(diffs)
+
+
+def _batched_case(ctx, wl, variant, layer, inp, flush_buf, max_len):
+    """Per-call cold-L2 device times (us) of the separate calls of one decode
+    step (score or soft-vote logits + reduce, selection, attention + combine)
+    and of the fused step, with `_cold_batched`."""
+    import torch
+    from query_aware_sparse_decode_b200 import tb as TB
+    kn, vn, qq, qi = inp
+    dev = ctx.device
+    flat = flush_buf.view(torch.float32)[: 64 << 20]
+
+    def flush():
+        flat.sum()
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    gs = wl.Hq // wl.Hkv
+    t = {}
+    dense = wl.keep_pct >= 100 or layer in wl.dense_layers
+    ctx.set_seq_lens(layer, [wl.L] * wl.B)
+    if dense:
+        t["attn"] = _cold_batched(lambda: ctx.sparse_attn(layer, qq, None, TB.TB_MASK_DENSE, out), flush)
+    else:
+        if variant == TB.TB_SOFTVOTE:
+            sc = torch.empty((wl.B, max_len), device=dev)
+            nrow, mode = 1, TB.TB_MASK_SHARED
+            t["score"] = _cold_batched(lambda: ctx.softvote_scores(layer, qq, sc), flush)
+        else:
+            group = variant == TB.TB_BUTLER_GROUP
+            nrow = wl.Hkv if group else wl.Hq
+            mode = TB.TB_MASK_GROUP if group else TB.TB_MASK_PER_HEAD
+            sc = torch.empty((wl.B, nrow, max_len), device=dev)
+            t["score"] = _cold_batched(lambda: ctx.score(layer, qi, sc), flush)
+        mask = torch.zeros((wl.B, nrow, max_len // 32), dtype=torch.int32, device=dev)
+        t["select"] = _cold_batched(lambda: ctx.select(layer, sc, nrow, mask=mask), flush)
+        t["attn"] = _cold_batched(lambda: ctx.sparse_attn(layer, qq, mask, mode, out), flush)
+
+    def step():
+        ctx.set_seq_lens(layer, [wl.L - 1] * wl.B)
+        ctx.decode_step(layer, kn, vn, qq, qi, out)
+    t["step"] = _cold_batched(step, flush)
+    ctx.set_seq_lens(layer, [wl.L] * wl.B)
+    return t
+
+
 def _variant_name(variant):
     from query_aware_sparse_decode_b200 import tb as TB
     return {TB.TB_SOFTVOTE: "softvote", TB.TB_BUTLER_GROUP: "group"}.get(variant, "butler")
@@ -790,6 +859,7 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak, hot_l2=True):
     inp = (bf(kn), bf(vn), bf(S.query(wl, layer)), bf(S.q_imp(wl, 0)))
     cold = _timed_decode(ctx, wl, layer, inp, iters, flush_buf, stream)
     hot = _timed_decode(ctx, wl, layer, inp, iters, None, stream) if hot_l2 else None
+    batched = _batched_case(ctx, wl, variant, layer, inp, flush_buf, max_len)
     # algorithmic bytes from the library's own selection of this step
     ctx.set_seq_lens(layer, [wl.L] * wl.B)
     dense = wl.keep_pct >= 100 or layer in wl.dense_layers
@@ -834,9 +904,15 @@ def _table_case(wl, variant, dev, iters, flush_buf, peak, hot_l2=True):
         r["attn_frac"] = r["attn_gbs"] / peak
         r["step_gbs"] = (first + attn_bytes) / (t["total"] * 1e-6) / 1e9
         return r
+    bt = batched
     line = {"table": "decode", "workload": wl.name, "variant": _variant_name(variant),
             "B": wl.B, "L": wl.L, "keep_pct": wl.keep_pct, "dense": dense,
             "first_pass_bytes": first, "union_rows": union, "attn_bytes": attn_bytes,
+            "us_batched": bt,
+            "batched_attn_frac": attn_bytes / (bt["attn"] * 1e-6) / 1e9 / peak,
+            "batched_pair_frac": (None if dense else
+                                  (first + attn_bytes) / ((bt["score"] + bt["attn"]) * 1e-6) / 1e9 / peak),
+            "batched_step_gbs": (first + attn_bytes) / (bt["step"] * 1e-6) / 1e9,
             "us_cold_l2": cold, "us_hot_l2": hot, "rates_cold_l2": rates(cold),
             "rates_hot_l2": rates(hot) if hot is not None else None,
             "l2": "cold: 512 MB write + 256 MB read before each step; hot: back-to-back steps",
@@ -999,12 +1075,18 @@ def config_rows(dev, iters, peak, n_layers_prefill=32):
     for wl, variant in cases:
         line = _table_case(wl, variant, dev, iters, flush_buf, peak, hot_l2=False)
         t, rt = line["us_cold_l2"], line["rates_cold_l2"]
+        bt = line["us_batched"]
         rows.append({"workload": line["workload"], "variant": line["variant"], "L": line["L"],
                      "keep_pct": line["keep_pct"], "dense": line["dense"],
-                     "us": {k: round(t[k], 2) for k in ("score", "select", "attn", "combine", "total")},
+                     "us": {k: round(v, 2) for k, v in bt.items()},
                      "first_pass_bytes": line["first_pass_bytes"], "attn_bytes": line["attn_bytes"],
-                     "pair_frac": (round(rt["score_plus_attn_frac"], 4) if "score_plus_attn_frac" in rt else None),
-                     "attn_frac": round(rt["attn_frac"], 4)})
+                     "pair_frac": (round(line["batched_pair_frac"], 4) if line["batched_pair_frac"] is not None
+                                   else None),
+                     "attn_frac": round(line["batched_attn_frac"], 4),
+                     "us_traced": {k: round(t[k], 2) for k in ("score", "select", "attn", "combine", "total")},
+                     "pair_frac_traced": (round(rt["score_plus_attn_frac"], 4) if "score_plus_attn_frac" in rt
+                                          else None),
+                     "attn_frac_traced": round(rt["attn_frac"], 4)})
     del flush_buf
     torch.cuda.empty_cache()
     pf = _table_prefill(dev, iters, peak, n_layers_prefill)
@@ -1014,7 +1096,12 @@ def config_rows(dev, iters, peak, n_layers_prefill=32):
                "select_rows_us": round(pf["select_prefill"]["us_median"], 1),
                "select_rows_elements_per_s": pf["select_prefill"]["elements_per_s"]}
     return {"decode_rows": rows, "prefill": prefill, "peak_gbs": peak,
-            "timing": "median of single decode steps, L2 flushed before each (512 MB write, 256 MB read)"}
+            "timing": ("us / pair_frac / attn_frac: per call through the C ABI (score or soft-vote logits + reduce; "
+                       "selection; attention + combine; the fused step), L2 cold (a 256 MB read before each call), "
+                       "launches queued back to back so that no launch gap is counted: 10 (read, call) pairs minus "
+                       "10 reads, median of 5; us_traced / pair_frac_traced: the fused step's segments between "
+                       "trace events (each segment also holds the gap of its launch behind an event), median of "
+                       "single steps, L2 flushed before each (512 MB write, 256 MB read)")}
 
 
 def kernel_table(args):

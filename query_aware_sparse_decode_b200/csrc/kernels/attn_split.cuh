@@ -10,8 +10,8 @@ namespace tb {
 // The grid is about two full waves of two CTAs per SM, or one wave when two
 // would leave CTAs with short chunks (fewer than 3584 tokens: the list build,
 // the ring's fill and the partial write then weigh more than the second
-// wave's balance gains).  Chunks are multiples of 256 tokens.  `groups` is
-// B * Hkv.  Returns false when more than kMaxSplits splits would be needed.
+// wave's balance gains).  Chunks are multiples of 32 tokens (whole mask
+// words), so that the splits fill the wave.  `groups` is B * Hkv.  Returns false when more than kMaxSplits splits would be needed.
 inline bool attn_split(int num_sms, int groups, int maxL, int* chunk_out, int* nsplit_out) {
   const int L = maxL > 1 ? maxL : 1;
   int want = (4 * num_sms) / groups;
@@ -21,8 +21,7 @@ inline bool attn_split(int num_sms, int groups, int maxL, int* chunk_out, int* n
     want = want < 1 ? 1 : (want > kMaxSplits ? kMaxSplits : want);
   }
   int chunk = (L + want - 1) / want;
-  chunk = (chunk + 255) / 256 * 256;
-  if (chunk < 256) chunk = 256;
+  chunk = (chunk + 31) / 32 * 32;
   const int n = (maxL + chunk - 1) / chunk;
   *chunk_out = chunk;
   *nsplit_out = n > 1 ? n : 1;

@@ -10,14 +10,13 @@
 //
 // softvote_logits: HBM stream over K (each row read once per KV head and
 // shared by the group's query heads), contiguous 16-token tiles gathered by
-// cp.async into a swizzled ring, q . K^T on mma.sync (bf16 in, fp32
-// accumulate); writes the logits in the log2 domain and one (max, sum of
-// 2^(a - max)) pair per head and chunk.  The last CTA of a sequence to finish
-// (a device-scope completion counter, fence then count; nothing waits on it)
-// merges the sequence's chunk pairs into each head's (M, 1/Z) and resets the
-// counter for the next launch.
-// softvote_reduce: sums 2^(a - M) / Z over the heads, one token per thread
-// (logits are L2-resident), after one read of the heads' (M, 1/Z).  Optionally it also
+// cp.async into a swizzled ring, K q^T on mma.sync (bf16 in, fp32
+// accumulate; the tile's tokens as the M rows, the group's heads as the N
+// columns); writes the logits in the log2 domain and one (max, sum of
+// 2^(a - max)) pair per head and chunk.
+// softvote_reduce: merges each head's chunk pairs into (M, 1/Z) (every CTA,
+// while its first logits are in flight), then sums 2^(a - M) / Z over the
+// heads, one token per thread (logits are L2-resident).  Optionally it also
 // builds the first-digit histogram of the votes over the candidate range
 // [sink, len - window) for the selection that follows (warp-aggregated shared
 // atomics: votes crowd into few bins).
@@ -31,6 +30,9 @@ namespace tb {
 // Tokens per CTA of the logits pass: chosen per launch (a multiple of 16, at
 // least kVoteMinChunk) so that the grid is about four CTAs per SM in one wave.
 constexpr int kVoteMinChunk = 256;
+constexpr int kVoteStages = 3;  // ring stages per warp of the logits pass (16 K rows each)
+template <int D>
+constexpr int vote_logits_smem() { return kAttnWarps * kVoteStages * kAttnTile * D * 2; }
 
 struct VoteParams {
   const void* k_cache;  // [B][Hkv][max_len][D] bf16, or a page pool (KvLayout)
@@ -38,8 +40,6 @@ struct VoteParams {
   const void* q;        // [B][Hq][D] bf16
   float* logits;        // [B][Hq][max_len], log2 domain
   float* stats;         // [B][Hq][nchunk][2]
-  float* mz;            // [B][Hq][2]: each head's merged max M (log2 domain) and 1/Z
-  uint32_t* done;       // [B] logits CTAs finished (zero between launches)
   float* votes;         // [B][max_len]
   uint32_t* hist1;      // [B][2048] first-digit histograms of the votes, or nullptr
   int Hq, Hkv, max_len, nchunk;  // nchunk: stride of the chunk statistics, >= max_len / chunk
@@ -68,27 +68,41 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   const int grp = lane >> 2, tq = lane & 3;
   const uint8_t* Kb = reinterpret_cast<const uint8_t*>(p.k_cache);  // rows via kv_row
 
-  uint32_t qa[KSTEPS][2];
+  // S^T = K Q^T on mma.sync: the tile's 16 tokens are the M rows (A = the K
+  // tile, ldmatrix), the group's heads the 8 N columns (B = Q^T, heads >= GS
+  // zero).  Lane (grp, tq) holds head grp, dims 16kk + 2tq + {0,1} and
+  // 16kk + 8 + 2tq + {0,1} of Q^T, and receives the logits of tokens grp and
+  // grp + 8 for heads 2tq and 2tq + 1.
+  uint32_t qb[KSTEPS][2];
   {
     const __nv_bfloat16* qrow =
         reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * GS + (grp < GS ? grp : 0)) * D;
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
-      const int dim = (4 * (kk / 2) + tq) * 8 + (kk % 2) * 4;
-      qa[kk][0] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim) : 0u;
-      qa[kk][1] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + dim + 2) : 0u;
+      qb[kk][0] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq) : 0u;
+      qb[kk][1] = grp < GS ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * tq) : 0u;
     }
   }
-  float m_run = kNegInf, l_run = 0.f;
+  // the lane's two heads, and whether each is one of the group's
+  const int hp = 2 * tq;
+  const bool real0 = hp < GS, real1 = hp + 1 < GS;
+  // per lane and head: running max and sum of 2^(a - max) over the lane's tokens
+  float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};
   const int ntiles = (n + kAttnTile - 1) / kAttnTile;
   const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
-  uint8_t* my_ring = smem + warp * kAttnStages * STAGE;
+  uint8_t* my_ring = smem + warp * kVoteStages * STAGE;
+  const uint32_t ring_u32 = smem_u32(my_ring);
+  // ldmatrix rows: lane supplies row (lane & 7) of matrix (lane >> 3) = tokens
+  // 8 (j & 1) + r, piece 2kk + (j >> 1); the swizzled piece is 2kk ^ ((j >> 1) ^ r)
+  const int lr = lane & 7, lj = lane >> 3;
+  const uint32_t k_row_off = (uint32_t)((lr + 8 * (lj & 1)) * ROWB);
+  const uint32_t k_x = (uint32_t)(((lj >> 1) ^ lr) << 4);
   // A tile's 16 tokens are consecutive cache rows: tiles start at multiples of
   // 16 and pages hold a power of two >= 16 tokens, so one row lookup per tile
   // serves all of them (rows past the ragged end repeat the last token).
   auto issue = [&](int it) {
     const int tile = warp + it * kAttnWarps;
-    uint8_t* sb = my_ring + (it % kAttnStages) * STAGE;
+    uint8_t* sb = my_ring + (it % kVoteStages) * STAGE;
     const int tt = t0 + tile * kAttnTile;
     const int last = t1 - 1 - tt;
     const uint8_t* base = Kb + (size_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, tt) * ROWB;
@@ -99,70 +113,79 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     }
   };
 #pragma unroll
-  for (int s = 0; s < kAttnStages - 1; ++s) {
+  for (int s = 0; s < kVoteStages - 1; ++s) {
     if (s < my_n) issue(s);
     cp_async_commit();
   }
-  const size_t lrow = ((size_t)b * p.Hq + g * GS + (grp < GS ? grp : 0)) * p.max_len;
+  float* lrow0 = p.logits + ((size_t)b * p.Hq + g * GS + (real0 ? hp : 0)) * p.max_len;
+  float* lrow1 = p.logits + ((size_t)b * p.Hq + g * GS + (real1 ? hp + 1 : 0)) * p.max_len;
   for (int it = 0; it < my_n; ++it) {
-    if (it + kAttnStages - 1 < my_n) issue(it + kAttnStages - 1);
+    if (it + kVoteStages - 1 < my_n) issue(it + kVoteStages - 1);
     cp_async_commit();
-    cp_async_wait<kAttnStages - 1>();
+    cp_async_wait<kVoteStages - 1>();
     __syncwarp();
-    const uint8_t* Ks = my_ring + (it % kAttnStages) * STAGE;
+    const uint32_t st = ring_u32 + (uint32_t)((it % kVoteStages) * STAGE);
     const int tile = warp + it * kAttnWarps;
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      const int c = 4 * i + tq;
-      const uint4 k0 = *reinterpret_cast<const uint4*>(Ks + grp * ROWB + ((c ^ (grp & 7)) << 4));
-      const uint4 k1 = *reinterpret_cast<const uint4*>(Ks + (grp + 8) * ROWB + ((c ^ (grp & 7)) << 4));
-      mma_16816(acc0, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k0.x, k0.y);
-      mma_16816(acc0, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k0.z, k0.w);
-      mma_16816(acc1, qa[2 * i][0], 0u, qa[2 * i][1], 0u, k1.x, k1.y);
-      mma_16816(acc1, qa[2 * i + 1][0], 0u, qa[2 * i + 1][1], 0u, k1.z, k1.w);
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(a, st + k_row_off + (((uint32_t)(32 * kk)) ^ k_x));
+      mma_16816(s, a[0], a[1], a[2], a[3], qb[kk][0], qb[kk][1]);
     }
-    const int tb0 = t0 + tile * kAttnTile;
-    const int ta = tb0 + 2 * tq, tc = tb0 + 2 * tq + 8;
-    const bool real = grp < GS;
-    const float s0 = real && ta < t1 ? acc0[0] * p.scale_log2 : kNegInf;
-    const float s1 = real && ta + 1 < t1 ? acc0[1] * p.scale_log2 : kNegInf;
-    const float s2 = real && tc < t1 ? acc1[0] * p.scale_log2 : kNegInf;
-    const float s3 = real && tc + 1 < t1 ? acc1[1] * p.scale_log2 : kNegInf;
-    if (real) {
-      if (ta + 1 < t1) {
-        *reinterpret_cast<float2*>(p.logits + lrow + ta) = make_float2(s0, s1);
-      } else if (ta < t1) {
-        p.logits[lrow + ta] = s0;
+    __syncwarp();  // the stage is refilled by the next iteration's copies
+    const int ta = t0 + tile * kAttnTile + grp, tc = ta + 8;
+    // x[0], x[1]: token ta, heads hp, hp + 1; x[2], x[3]: token tc
+    float x[4];
+    x[0] = ta < t1 ? s[0] * p.scale_log2 : kNegInf;
+    x[1] = ta < t1 ? s[1] * p.scale_log2 : kNegInf;
+    x[2] = tc < t1 ? s[2] * p.scale_log2 : kNegInf;
+    x[3] = tc < t1 ? s[3] * p.scale_log2 : kNegInf;
+    if (real0) {
+      if (ta < t1) lrow0[ta] = x[0];
+      if (tc < t1) lrow0[tc] = x[2];
+    }
+    if (real1) {
+      if (ta < t1) lrow1[ta] = x[1];
+      if (tc < t1) lrow1[tc] = x[3];
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float mn = fmaxf(m_run[e], fmaxf(x[e], x[2 + e]));
+      if (mn != kNegInf) {
+        // 2^x on the special-function unit (relative error about 2^-22, far
+        // inside the votes' tolerance); 2^-inf = 0
+        l_run[e] = l_run[e] * fast_exp2(m_run[e] - mn) + fast_exp2(x[e] - mn) + fast_exp2(x[2 + e] - mn);
+        m_run[e] = mn;
       }
-      if (tc + 1 < t1) {
-        *reinterpret_cast<float2*>(p.logits + lrow + tc) = make_float2(s2, s3);
-      } else if (tc < t1) {
-        p.logits[lrow + tc] = s2;
-      }
     }
-    float mt = fmaxf(fmaxf(s0, s1), fmaxf(s2, s3));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-    const float m_new = fmaxf(m_run, mt);
-    if (m_new != kNegInf) {
-      // 2^x on the special-function unit (relative error about 2^-22, far
-      // inside the votes' tolerance); 2^-inf = 0
-      l_run = l_run * fast_exp2(m_run - m_new) + fast_exp2(s0 - m_new) + fast_exp2(s1 - m_new) +
-              fast_exp2(s2 - m_new) + fast_exp2(s3 - m_new);
-      m_run = m_new;
-    }
-    __syncwarp();
   }
   cp_async_wait<0>();
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  // merge the lanes' pairs of each head (the 8 lanes with the same tq)
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m_run[e], o), l2 = __shfl_xor_sync(0xffffffffu, l_run[e], o);
+      const float mn = fmaxf(m_run[e], m2);
+      if (mn != kNegInf) {
+        l_run[e] = (m_run[e] == kNegInf ? 0.f : l_run[e] * exp2f(m_run[e] - mn)) +
+                   (m2 == kNegInf ? 0.f : l2 * exp2f(m2 - mn));
+        m_run[e] = mn;
+      }
+    }
   __syncthreads();
   float* wm = reinterpret_cast<float*>(smem);
   float* wl = wm + kAttnWarps * GS;
-  if (grp < GS && tq == 0) {
-    wm[warp * GS + grp] = m_run;
-    wl[warp * GS + grp] = l_run;
+  if (grp == 0) {
+    if (real0) {
+      wm[warp * GS + hp] = m_run[0];
+      wl[warp * GS + hp] = l_run[0];
+    }
+    if (real1) {
+      wm[warp * GS + hp + 1] = m_run[1];
+      wl[warp * GS + hp + 1] = l_run[1];
+    }
   }
   __syncthreads();
   if (tid < GS) {
@@ -176,20 +199,34 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     p.stats[ph] = M;
     p.stats[ph + 1] = l;
   }
-  // ---- the sequence's last CTA merges every chunk's pair into (M, 1/Z) per head
-  __shared__ uint32_t s_last;
-  __threadfence();  // this CTA's pairs are visible device-wide before it is counted
-  __syncthreads();
+}
+
+// grid (ceil(max len / 256), B), block 256: one token per thread.  The
+// token's logits of the first kVotePrefetch heads are requested before the
+// CTA merges the heads' chunk pairs, so the two latencies overlap.
+constexpr int kVoteMaxHeads = 128;
+constexpr int kVoteReduceTok = 256;
+constexpr int kVotePrefetch = 32;
+__global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float2 sMZ[kVoteMaxHeads];  // per head: (M, 1/Z)
+  __shared__ uint32_t hist[kHistBins];
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int L = p.lens[b];
+  const int t_begin = blockIdx.x * kVoteReduceTok;
+  if (t_begin >= L) return;
+  const int t = t_begin + tid;
+  const float* lg = p.logits + (size_t)b * p.Hq * p.max_len + t;
+  float a[kVotePrefetch];
+#pragma unroll
+  for (int h = 0; h < kVotePrefetch; ++h) a[h] = (h < p.Hq && t < L) ? lg[(size_t)h * p.max_len] : 0.f;
+  // each head's (M, 1/Z) from the logits pass's per-chunk pairs: eight
+  // threads per head, each merging every eighth chunk, then across the eight
   const int nch = (L + p.chunk - 1) / p.chunk;
-  if (tid == 0) s_last = atomicAdd(&p.done[b], 1u) == (uint32_t)(nch * p.Hkv - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // four threads per head (consecutive lanes), each merging every fourth chunk
-  constexpr int TPH = 4;
-  const int sub = tid % TPH;
-  for (int h0 = 0; h0 < p.Hq; h0 += kAttnThreads / TPH) {
-    const int h = h0 + tid / TPH;
+  constexpr int TPH = 8;
+  for (int h0 = 0; h0 < p.Hq; h0 += 256 / TPH) {
+    const int h = h0 + tid / TPH, sub = tid % TPH;
     float m = kNegInf, l = 0.f;
     if (h < p.Hq) {
       const float2* st = reinterpret_cast<const float2*>(p.stats + ((size_t)b * p.Hq + h) * p.nchunk * 2);
@@ -211,37 +248,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
         m = mn;
       }
     }
-    if (h < p.Hq && sub == 0) {
-      p.mz[((size_t)b * p.Hq + h) * 2] = m;
-      p.mz[((size_t)b * p.Hq + h) * 2 + 1] = 1.f / l;
-    }
-  }
-  if (tid == 0) p.done[b] = 0u;  // ready for the next launch (stream-ordered after this grid)
-}
-
-// grid (ceil(max len / 256), B), block 256: one token per thread.  The
-// token's logits of the first kVotePrefetch heads are requested before the
-// CTA reads the heads' (M, 1/Z), so the two latencies overlap.
-constexpr int kVoteMaxHeads = 128;
-constexpr int kVoteReduceTok = 256;
-constexpr int kVotePrefetch = 32;
-__global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ float2 sMZ[kVoteMaxHeads];  // per head: (M, 1/Z)
-  __shared__ uint32_t hist[kHistBins];
-  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-  const int L = p.lens[b];
-  const int t_begin = blockIdx.x * kVoteReduceTok;
-  if (t_begin >= L) return;
-  const int t = t_begin + tid;
-  const float* lg = p.logits + (size_t)b * p.Hq * p.max_len + t;
-  float a[kVotePrefetch];
-#pragma unroll
-  for (int h = 0; h < kVotePrefetch; ++h) a[h] = (h < p.Hq && t < L) ? lg[(size_t)h * p.max_len] : 0.f;
-  for (int h = tid; h < p.Hq; h += 256) {
-    const float2 mz = reinterpret_cast<const float2*>(p.mz)[(size_t)b * p.Hq + h];
-    sMZ[h] = mz;
+    if (h < p.Hq && sub == 0) sMZ[h] = make_float2(m, 1.f / l);
   }
   if (p.hist1 != nullptr)
     for (int i = tid; i < kHistBins; i += 256) hist[i] = 0;

@@ -52,14 +52,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
   size_t status, hist, ccount, kcount, hist2, ctot, hist_end, cslot, rowinfo, cand, scores, mask, part_o, part_ml, votes,
-      vstats, vmz, vdone, reuse, total;
+      vstats, reuse, total;
   int max_splits;
 };
 
 WsLayout layout_of(const tb_config& c) {
   WsLayout w{};
   const size_t B = c.batch, Hq = c.n_q_heads, Lm = c.max_len;
-  w.max_splits = (int)((Lm + 255) / 256);
+  w.max_splits = (int)std::min<size_t>((Lm + 31) / 32, kMaxSplits);  // attention splits: 32-token chunks at least
   size_t off = 0;
   w.status = off;  off += align256(256);
   w.hist = off;    off += B * Hq * kHistBins * 4;        // first-digit histograms, then
@@ -77,8 +77,6 @@ WsLayout layout_of(const tb_config& c) {
   w.part_ml = off; off += align256(B * Hq * (size_t)w.max_splits * 2 * 4);
   w.votes = off;   off += align256(B * Lm * 4);
   w.vstats = off;  off += align256(B * Hq * ((Lm + kVoteMinChunk - 1) / kVoteMinChunk) * 2 * 4);
-  w.vmz = off;     off += align256(B * Hq * 2 * 4);      // per head: merged soft-vote (M, 1/Z)
-  w.vdone = off;   off += align256(B * 4);               // logits CTAs finished (zeroed at init, self-clearing)
   w.reuse = off;   off += align256(B * Hq * 4);         // per-row reuse decisions of the step
   w.total = off;
   return w;
@@ -124,8 +122,6 @@ struct tb_ctx {
   float* part_ml = nullptr;
   float* votes = nullptr;
   float* vstats = nullptr;
-  float* vmz = nullptr;
-  uint32_t* vdone = nullptr;
   bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last selection)
   int cluster_active[5] = {};  // resident clusters of 1, 2, 4, 8, 16 CTAs of the selection kernel (0: not launchable)
   uint32_t* ctot = nullptr;
@@ -465,8 +461,6 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   p.q = q;
   p.logits = ctx->scores;
   p.stats = ctx->vstats;
-  p.mz = ctx->vmz;
-  p.done = ctx->vdone;
   p.votes = votes;
   p.hist1 = hist;
   p.sink = c.sink;
@@ -486,7 +480,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
 #define TB_VOTE_CASE(DV, GSV)                                                                 \
   if (c.head_dim == DV && gs == GSV) {                                                        \
     auto k = softvote_logits_kernel<DV, GSV>;                                                 \
-    const int smem = kAttnWarps * kAttnStages * kAttnTile * DV * 2;                           \
+    const int smem = vote_logits_smem<DV>();                                                  \
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);               \
     launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                            \
   } else
@@ -547,11 +541,8 @@ TB_API tb_status tb_init(const tb_config* cfg, void* workspace, size_t ws_bytes,
   ctx->part_ml = reinterpret_cast<float*>(ctx->ws + lay.part_ml);
   ctx->votes = reinterpret_cast<float*>(ctx->ws + lay.votes);
   ctx->vstats = reinterpret_cast<float*>(ctx->ws + lay.vstats);
-  ctx->vmz = reinterpret_cast<float*>(ctx->ws + lay.vmz);
-  ctx->vdone = reinterpret_cast<uint32_t*>(ctx->ws + lay.vdone);
   ctx->reuse = reinterpret_cast<uint32_t*>(ctx->ws + lay.reuse);
-  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess ||
-      cudaMemset(ctx->vdone, 0, (size_t)cfg->batch * sizeof(uint32_t)) != cudaSuccess) {
+  if (cudaMemset(ctx->status, 0, sizeof(uint32_t)) != cudaSuccess) {
     delete ctx;
     return TB_ERR_CUDA;
   }
