@@ -53,7 +53,7 @@
 
 namespace tb {
 
-constexpr int kClThreads = 256;
+constexpr int kClThreads = 512;
 constexpr int kClWarps = kClThreads / 32;
 constexpr int kClChunkMax = 65536;            // tokens per CTA
 constexpr int kClWordsMax = kClChunkMax / 32;  // mask words per CTA
@@ -188,7 +188,7 @@ __device__ __forceinline__ void visit_candidates(const float* srow, int a, int b
 }
 
 // grid (NC, rows, B), cluster (NC, 1, 1), kClThreads threads, kClSmem bytes.
-__global__ void __launch_bounds__(kClThreads, 3) select_cluster_kernel(const SelectParams p, int chunk) {
+__global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const SelectParams p, int chunk) {
   pdl_wait();
   pdl_trigger();
   namespace cg = cooperative_groups;
