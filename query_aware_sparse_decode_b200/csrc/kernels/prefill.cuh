@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   __shared__ uint32_t scan_sm[32];
   __shared__ int s_bin;
   __shared__ uint32_t s_above;
-  __shared__ int s_any2;
+  __shared__ int s_any2, s_not2, s_big2;
   uint32_t* hist = pf_smem;
   uint2* lists = reinterpret_cast<uint2*>(pf_smem);  // [16][kPfListCap], pass 3 only
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   const int nr = min(kPfRows, p.nrows - r0);
   if (tid == 0) {
     s_any2 = 0;
+    s_not2 = 0;
+    s_big2 = 0;
     s_bin = 0;
   }
   __syncthreads();
@@ -249,9 +251,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     rb1[tid] = 0;
     rb2[tid] = 0;
     if (mode == 2) atomicOr(&s_any2, 1);
+    if (mode != 2) atomicOr(&s_not2, 1);
   }
   __syncthreads();
   const bool any2 = s_any2 != 0;
+  // every one of the 16 rows resolves a top-k (no short or padding rows):
+  // interior tiles then need no per-token range or mode checks
+  const bool all2 = s_not2 == 0;
   const int Lmax = nr > 0 ? p.row0 + r0 + nr : 0;
   const int L0 = p.row0 + r0 + 1;        // row r covers tokens [0, L0 + r)
   const int hi0 = L0 - p.window;         // row r's candidates are [sink, hi0 + r)
@@ -321,6 +327,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
       const int t0 = ws * 32;
       float sc[4][4];
       tile_scores(t0, sc);
+      if (all2 && t0 >= p.sink && t0 + 32 <= hi0) {  // every token a candidate of every row (warp-uniform)
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            atomicAdd(&hist[(i < 2 ? ra : rb) * kHistBins + (order_key(sc[n][i]) >> 21)], 1u);
+        continue;
+      }
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
 #pragma unroll
@@ -357,6 +371,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
       float sc[4][4] = {};
       if (any2 && t0 < Lmax) tile_scores(t0, sc);  // warp-uniform
       uint32_t wa = 0, wb = 0;
+      if (all2 && t0 >= p.sink && t0 + 32 <= hi0) {  // every token a candidate of every row (warp-uniform)
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int pos = 8 * n + 2 * cq + (i & 1);
+            const uint32_t key = order_key(sc[n][i]);
+            const uint32_t d1 = key >> 21, b1 = i < 2 ? b1a : b1b;
+            if (d1 > b1) {
+              if (i < 2) wa |= 1u << pos;
+              else wb |= 1u << pos;
+            } else if (d1 == b1) {
+              atomicAdd(&hist[(i < 2 ? ra : rb) * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
+            }
+          }
+        }
+      } else {
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
 #pragma unroll
@@ -381,6 +412,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
             else wb |= 1u << pos;
           }
         }
+      }
       }
       wa |= __shfl_xor_sync(0xffffffffu, wa, 1);
       wa |= __shfl_xor_sync(0xffffffffu, wa, 2);
@@ -413,6 +445,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     }
   }
   if (tid < nr) p.redo[((size_t)b * p.Hq + h) * p.nrows + r0 + tid] = (rmode[tid] == 2 && rn2[tid] > (uint32_t)kPfListCap);
+  if (tid < kPfRows && rmode[tid] == 2 && rn2[tid] > (uint32_t)kPfListCap) atomicOr(&s_big2, 1);
   __syncthreads();
 
   // ---- pass 3: keys above the 22-bit prefix into the mask, keys equal to it
@@ -421,11 +454,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     const bool m3a = rmode[ra] == 2 && rn2[ra] <= (uint32_t)kPfListCap;
     const bool m3b = rmode[rb] == 2 && rn2[rb] <= (uint32_t)kPfListCap;
     const uint32_t b1a = rb1[ra], b1b = rb1[rb], b2a = rb2[ra], b2b = rb2[rb];
+    const bool all3 = all2 && __all_sync(0xffffffffu, m3a && m3b) && s_big2 == 0;
     for (int ws = warp; ws < nsteps; ws += kPfThreads / 32) {
       const int t0 = ws * 32;
       float sc[4][4];
       tile_scores(t0, sc);
       uint32_t ua = 0, ub = 0;
+      // every token a candidate of every row, every row listed (warp-uniform)
+      const bool inner = all3 && t0 >= p.sink && t0 + 32 <= hi0;
 #pragma unroll
       for (int n = 0; n < 4; ++n) {
 #pragma unroll
@@ -434,7 +470,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
           const bool m3 = i < 2 ? m3a : m3b;
           const int pos = 8 * n + 2 * cq + (i & 1);
           const int t = t0 + pos;
-          if (!m3 || t < p.sink || t >= hi0 + row) continue;
+          if (!inner && (!m3 || t < p.sink || t >= hi0 + row)) continue;
           const uint32_t key = order_key(sc[n][i]);
           if ((key >> 21) != (i < 2 ? b1a : b1b)) continue;
           const uint32_t d2 = (key >> 10) & (kHistBins - 1), b2 = i < 2 ? b2a : b2b;
