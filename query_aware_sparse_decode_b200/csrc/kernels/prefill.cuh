@@ -10,14 +10,18 @@
 // rows share the K_imp prefix, so each K_imp row is read once per block (not
 // once per row) and feeds 16 fp32 dot products, in the same dimension order
 // as every other score in the library.  Scores are recomputed, not stored,
-// in three passes:
+// in two passes, and a third pass works on what the second kept:
 //   1. first-digit (11-bit) histograms of the 16 rows' candidates;
 //   2. mask words of sink, window and keys above each row's threshold bin
-//      (one ballot per row and 32 tokens), and second-digit histograms of
-//      the threshold bins;
-//   3. keys above the 22-bit threshold prefix are OR-ed into the mask, keys
-//      equal to it (a handful per row) are listed in shared memory and
-//      ranked by (key desc, index asc), which also settles ties.
+//      (one ballot per row and 32 tokens), second-digit histograms of the
+//      threshold bins, and (rows under 65536 tokens) each row's keys of its
+//      threshold bin listed in shared memory, up to kPfBinCap per row;
+//   3. from those lists, keys above the 22-bit threshold prefix are OR-ed
+//      into the mask and keys equal to it (a handful per row) are listed and
+//      ranked by (key desc, index asc), which also settles ties.  Rows whose
+//      bin did not fit recompute their tiles for this pass instead.
+// Tiles whose 32 tokens are candidates of all 16 rows skip the per-token
+// range checks.
 // A row whose 22-bit prefix holds more than kPfListCap keys (massive ties) is
 // flagged; prefill_redo_kernel then recomputes it with the one-row method
 // (row scores in shared memory, three radix digits, an ordered sweep).
@@ -31,7 +35,14 @@ namespace tb {
 constexpr int kPfRows = 16;       // rows per CTA of the blocked kernel
 constexpr int kPfThreads = 1024;
 constexpr int kPfListCap = 256;   // keys per row sharing the 22-bit threshold prefix
-constexpr int kPfSmem = kPfRows * kHistBins * 4;
+// Pass 2 keeps each row's keys of its threshold bin in shared memory (with
+// 16-bit second-digit counters, two per word) so that pass 3 works on those
+// lists instead of recomputing the tiles: rows of fewer than 65536 tokens, up
+// to kPfBinCap keys per row.
+constexpr int kPfBinCap = 1280;
+constexpr int kPfHist16Words = kPfRows * kHistBins / 2;
+constexpr int kPfSmem = kPfHist16Words * 4 + kPfRows * kPfBinCap * 8;  // >= the 32-bit first-digit histograms
+static_assert(kPfSmem >= kPfRows * kHistBins * 4, "pass 1 histograms fit");
 
 struct PrefillParams {
   const void* q_imp;   // [(B*Hq)][G][nrows][d'] kv dtype
@@ -201,6 +212,28 @@ __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// find_bin over 2048 bins held as 16-bit counters, two per word (bin 2w in
+// the low half of word w), with kPfThreads threads (one word each).
+__device__ __forceinline__ void find_bin16(const uint32_t* h16, uint32_t k, uint32_t* scan_sm, int* out_bin,
+                                           uint32_t* out_above) {
+  static_assert(kHistBins == 2 * kPfThreads, "one word per thread");
+  const int tid = threadIdx.x;
+  const uint32_t w = h16[kHistBins / 2 - 1 - tid];  // bins 2047 - 2 tid (high half) and 2046 - 2 tid (low half)
+  const uint32_t c0 = w >> 16, c1 = w & 0xFFFFu;
+  uint32_t total;
+  const uint32_t excl = block_excl_scan<kPfThreads>(c0 + c1, total, scan_sm);
+  if (excl < k && k <= excl + c0 + c1) {
+    if (excl + c0 >= k) {
+      *out_bin = kHistBins - 1 - 2 * tid;
+      *out_above = excl;
+    } else {
+      *out_bin = kHistBins - 2 - 2 * tid;
+      *out_above = excl + c0;
+    }
+  }
+  __syncthreads();
+}
+
 // The blocked method; see the file comment.  grid (ceil(nrows / 16), Hq, B),
 // 1024 threads.  The 16 rows are the M dimension of mma.sync m16n8k8 TF32
 // tiles: a warp takes 32 tokens at a time (four n-tiles of 8; one mask word
@@ -211,9 +244,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   constexpr int KS = DIMP / 8;                        // k-steps of 8 dimensions
   constexpr bool QSPLIT = sizeof(TQ) == 4;            // fp32 queries need hi + lo too
   constexpr bool KBF16 = sizeof(KT) == 2;             // bf16 K_imp: exact in TF32
-  extern __shared__ __align__(16) uint32_t pf_smem[];  // hist[16][2048]; in pass 3 the key lists
+  // pass 1: hist[16][2048]; pass 2: 16-bit counters [16][1024] words + bin lists
+  // [16][kPfBinCap] (or 32-bit hist[16][2048] for long rows); pass 3: lists [16][kPfListCap]
+  extern __shared__ __align__(16) uint32_t pf_smem[];
   __shared__ int rmode[kPfRows], rk[kPfRows];
   __shared__ uint32_t rb1[kPfRows], rk1[kPfRows], rb2[kPfRows], rk2[kPfRows], rn2[kPfRows], rcnt[kPfRows];
+  __shared__ uint32_t rbin[kPfRows];  // keys of the threshold bin appended per row (pass 2)
   __shared__ uint32_t rkept[kPfRows], rabove[kPfRows];
   __shared__ uint32_t scan_sm[32];
   __shared__ int s_bin;
@@ -221,6 +257,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   __shared__ int s_any2, s_not2, s_big2;
   uint32_t* hist = pf_smem;
   uint2* lists = reinterpret_cast<uint2*>(pf_smem);  // [16][kPfListCap], pass 3 only
+  uint2* blists = reinterpret_cast<uint2*>(pf_smem + kPfHist16Words);  // [16][kPfBinCap], passes 2-3
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, cq = lane & 3;
   const int gs = p.Hq / p.Hkv, g = h / gs;
@@ -247,6 +284,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     rkept[tid] = 0;
     rabove[tid] = 0;
     rcnt[tid] = 0;
+    rbin[tid] = 0;
     rn2[tid] = 0;
     rb1[tid] = 0;
     rb2[tid] = 0;
@@ -259,6 +297,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // interior tiles then need no per-token range or mode checks
   const bool all2 = s_not2 == 0;
   const int Lmax = nr > 0 ? p.row0 + r0 + nr : 0;
+  const bool lm = Lmax < 65536;  // 16-bit second-digit counters and bin lists in pass 2
   const int L0 = p.row0 + r0 + 1;        // row r covers tokens [0, L0 + r)
   const int hi0 = L0 - p.window;         // row r's candidates are [sink, hi0 + r)
   const size_t slab = (size_t)b * p.Hkv + g;
@@ -362,7 +401,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
 
   // ---- pass 2: every mask word of every row (sink, window, keys above the
-  // threshold bin), second-digit histograms of the threshold bins
+  // threshold bin), second-digit histograms of the threshold bins, and (rows
+  // under 65536 tokens) the threshold bin's keys listed per row
+  auto member = [&](int row, uint32_t key, int t) {
+    const uint32_t d2 = (key >> 10) & (kHistBins - 1);
+    if (lm) {
+      atomicAdd(&hist[row * (kHistBins / 2) + (d2 >> 1)], 1u << ((d2 & 1u) << 4));
+      const uint32_t slot = atomicAdd(&rbin[row], 1u);
+      if (slot < (uint32_t)kPfBinCap) blists[row * kPfBinCap + slot] = make_uint2(key, (uint32_t)t);
+    } else {
+      atomicAdd(&hist[row * kHistBins + d2], 1u);
+    }
+  };
   {
     const int mda = rmode[ra], mdb = rmode[rb];
     const uint32_t b1a = rb1[ra], b1b = rb1[rb];
@@ -383,7 +433,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
               if (i < 2) wa |= 1u << pos;
               else wb |= 1u << pos;
             } else if (d1 == b1) {
-              atomicAdd(&hist[(i < 2 ? ra : rb) * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
+              member(i < 2 ? ra : rb, key, t0 + pos);
             }
           }
         }
@@ -404,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
             if (d1 > b1) {
               keep = true;
             } else if (d1 == b1) {
-              atomicAdd(&hist[row * kHistBins + ((key >> 10) & (kHistBins - 1))], 1u);
+              member(row, key, t);
             }
           }
           if (keep) {
@@ -434,12 +484,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   if (any2) {
     for (int r = 0; r < kPfRows; ++r) {
       if (rmode[r] != 2) continue;
-      find_bin<kHistBins / kPfThreads, kPfThreads>(hist + r * kHistBins, rk1[r], scan_sm, &s_bin, &s_above);
+      if (lm)
+        find_bin16(hist + r * (kHistBins / 2), rk1[r], scan_sm, &s_bin, &s_above);
+      else
+        find_bin<kHistBins / kPfThreads, kPfThreads>(hist + r * kHistBins, rk1[r], scan_sm, &s_bin, &s_above);
       if (tid == 0) {
         rb2[r] = (uint32_t)s_bin;
         rk2[r] = rk1[r] - s_above;
         rabove[r] = s_above;
-        rn2[r] = hist[r * kHistBins + s_bin];
+        rn2[r] = lm ? (hist[r * (kHistBins / 2) + (s_bin >> 1)] >> ((s_bin & 1) << 4)) & 0xFFFFu
+                    : hist[r * kHistBins + s_bin];
       }
       __syncthreads();
     }
@@ -451,11 +505,28 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // ---- pass 3: keys above the 22-bit prefix into the mask, keys equal to it
   // into the row's list
   if (any2) {
-    const bool m3a = rmode[ra] == 2 && rn2[ra] <= (uint32_t)kPfListCap;
-    const bool m3b = rmode[rb] == 2 && rn2[rb] <= (uint32_t)kPfListCap;
+    // a row is resolved from its bin list when the list holds the whole bin
+    auto listed = [&](int r) { return lm && rbin[r] <= (uint32_t)kPfBinCap; };
+    {  // keys of the listed rows' bins above the 22-bit prefix into the mask, keys at it into the row's list
+      for (int e = tid; e < kPfRows * kPfBinCap; e += kPfThreads) {
+        const int r = e / kPfBinCap, i = e % kPfBinCap;
+        if (rmode[r] != 2 || rn2[r] > (uint32_t)kPfListCap || !listed(r) || (uint32_t)i >= rbin[r]) continue;
+        const uint2 x = blists[e];
+        const uint32_t d2 = (x.x >> 10) & (kHistBins - 1);
+        if (d2 > rb2[r]) {
+          atomicOr(&mbase[(size_t)r * nwords + (x.y >> 5)], 1u << (x.y & 31));
+        } else if (d2 == rb2[r]) {
+          const uint32_t slot = atomicAdd(&rcnt[r], 1u);
+          if (slot < (uint32_t)kPfListCap) lists[r * kPfListCap + slot] = x;
+        }
+      }
+    }
+    const bool m3a = rmode[ra] == 2 && rn2[ra] <= (uint32_t)kPfListCap && !listed(ra);
+    const bool m3b = rmode[rb] == 2 && rn2[rb] <= (uint32_t)kPfListCap && !listed(rb);
     const uint32_t b1a = rb1[ra], b1b = rb1[rb], b2a = rb2[ra], b2b = rb2[rb];
     const bool all3 = all2 && __all_sync(0xffffffffu, m3a && m3b) && s_big2 == 0;
-    for (int ws = warp; ws < nsteps; ws += kPfThreads / 32) {
+    const bool any3 = __syncthreads_or(m3a || m3b);  // some row is left to the tile recompute
+    for (int ws = warp; any3 && ws < nsteps; ws += kPfThreads / 32) {
       const int t0 = ws * 32;
       float sc[4][4];
       tile_scores(t0, sc);
