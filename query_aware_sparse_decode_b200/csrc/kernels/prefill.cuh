@@ -33,7 +33,7 @@
 namespace tb {
 
 constexpr int kPfRows = 16;       // rows per CTA of the blocked kernel
-constexpr int kPfThreads = 1024;
+constexpr int kPfThreads = 512;
 constexpr int kPfListCap = 256;   // keys per row sharing the 22-bit threshold prefix
 // Pass 2 keeps each row's keys of its threshold bin in shared memory (with
 // 16-bit second-digit counters, two per word) so that pass 3 works on those
@@ -213,22 +213,33 @@ __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)
 }
 
 // find_bin over 2048 bins held as 16-bit counters, two per word (bin 2w in
-// the low half of word w), with kPfThreads threads (one word each).
+// the low half of word w); a thread takes consecutive words from the top.
 __device__ __forceinline__ void find_bin16(const uint32_t* h16, uint32_t k, uint32_t* scan_sm, int* out_bin,
                                            uint32_t* out_above) {
-  static_assert(kHistBins == 2 * kPfThreads, "one word per thread");
+  constexpr int W = kHistBins / 2 / kPfThreads;  // words per thread
+  static_assert(W * kPfThreads * 2 == kHistBins, "whole words per thread");
   const int tid = threadIdx.x;
-  const uint32_t w = h16[kHistBins / 2 - 1 - tid];  // bins 2047 - 2 tid (high half) and 2046 - 2 tid (low half)
-  const uint32_t c0 = w >> 16, c1 = w & 0xFFFFu;
+  uint32_t c[2 * W];
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < W; ++j) {  // descending bins: the high half of a word first
+    const uint32_t w = h16[kHistBins / 2 - 1 - (tid * W + j)];
+    c[2 * j] = w >> 16;
+    c[2 * j + 1] = w & 0xFFFFu;
+    local += c[2 * j] + c[2 * j + 1];
+  }
   uint32_t total;
-  const uint32_t excl = block_excl_scan<kPfThreads>(c0 + c1, total, scan_sm);
-  if (excl < k && k <= excl + c0 + c1) {
-    if (excl + c0 >= k) {
-      *out_bin = kHistBins - 1 - 2 * tid;
-      *out_above = excl;
-    } else {
-      *out_bin = kHistBins - 2 - 2 * tid;
-      *out_above = excl + c0;
+  const uint32_t excl = block_excl_scan<kPfThreads>(local, total, scan_sm);
+  if (excl < k && k <= excl + local) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int i = 0; i < 2 * W; ++i) {
+      if (run + c[i] >= k) {
+        *out_bin = kHistBins - 1 - (tid * 2 * W + i);
+        *out_above = run;
+        break;
+      }
+      run += c[i];
     }
   }
   __syncthreads();
@@ -325,17 +336,31 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
   // scores of the 16 rows for the 32 tokens [t0, t0 + 32): sc[n][i], n-tile n,
   // i = (row gq, token 2cq), (gq, 2cq+1), (gq+8, 2cq), (gq+8, 2cq+1)
-  auto tile_scores = [&](int t0, float (&sc)[4][4]) {
+  // The B operands of a tile: the K_imp values this lane feeds to the four
+  // n-tiles (token t0 + 8 n + gq, dimensions ks * 8 + cq and + 4), all
+  // requested before the first mma of the tile.
+  using TileK = float[4][KS][2];
+  auto tile_load = [&](int t0, TileK& kv) {
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
-      sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-      const int t = t0 + 8 * n + gq;  // the B column this lane loads
+      const int t = t0 + 8 * n + gq;
       const bool ok = t < Lmax;
       const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, ok ? t : 0, DIMP, p.max_len);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        const float k0 = ok ? to_f32(K[(ks * 8 + cq) * kKimpTile]) : 0.f;
-        const float k1 = ok ? to_f32(K[(ks * 8 + cq + 4) * kKimpTile]) : 0.f;
+        kv[n][ks][0] = ok ? to_f32(K[(ks * 8 + cq) * kKimpTile]) : 0.f;
+        kv[n][ks][1] = ok ? to_f32(K[(ks * 8 + cq + 4) * kKimpTile]) : 0.f;
+      }
+    }
+  };
+  auto tile_mma = [&](const TileK& kv, float (&sc)[4][4]) {
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const float k0 = kv[n][ks][0];
+        const float k1 = kv[n][ks][1];
         // hi: the value cut to TF32 width; lo: the exact fp32 remainder, of
         // which the tensor core reads the TF32-width head.  A bf16 K_imp has
         // 8 significant bits, so it is exact in TF32 and has no remainder.
@@ -349,6 +374,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
         if (QSPLIT) mma_tf32_1688(sc[n], afl[ks], h0, h1);
       }
     }
+  };
+  auto tile_scores = [&](int t0, float (&sc)[4][4]) {
+    TileK kv;
+    tile_load(t0, kv);
+    tile_mma(kv, sc);
   };
 
   uint32_t* mbase = p.masks + (((size_t)b * p.Hq + h) * p.nrows + r0) * p.words_per_row;
@@ -565,8 +595,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     }
     __syncthreads();
     // rank each listed key by (key desc, index asc): the first rk2 are kept
-    if (warp < nr && rmode[warp] == 2 && rn2[warp] <= (uint32_t)kPfListCap) {
-      const int r = warp;
+    for (int r = warp; r < nr; r += kPfThreads / 32) {
+      if (rmode[r] != 2 || rn2[r] > (uint32_t)kPfListCap) continue;
       const uint32_t n = min(rcnt[r], (uint32_t)kPfListCap);
       const uint2* lst = lists + r * kPfListCap;
       uint32_t nsel = 0;
