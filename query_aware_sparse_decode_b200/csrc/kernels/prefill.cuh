@@ -212,37 +212,47 @@ __device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// find_bin over 2048 bins held as 16-bit counters, two per word (bin 2w in
-// the low half of word w); a thread takes consecutive words from the top.
-__device__ __forceinline__ void find_bin16(const uint32_t* h16, uint32_t k, uint32_t* scan_sm, int* out_bin,
-                                           uint32_t* out_above) {
-  constexpr int W = kHistBins / 2 / kPfThreads;  // words per thread
-  static_assert(W * kPfThreads * 2 == kHistBins, "whole words per thread");
-  const int tid = threadIdx.x;
-  uint32_t c[2 * W];
+// find_bin for one row by one warp: lane l sums bins 2047 - 64 l - j
+// (j = 0..63; read in a lane-skewed order, so no two lanes hit one bank),
+// a warp scan gives each lane the count above its range, and the lane whose
+// range holds the k-th key walks it from the top.  PACKED: 16-bit counters,
+// two per word (bin 2w in the low half of word w).  bin = -1 when the
+// histogram holds fewer than k keys.
+template <bool PACKED>
+__device__ __forceinline__ void warp_find_bin(const uint32_t* hist, uint32_t k, int& bin, uint32_t& above) {
+  const int lane = threadIdx.x & 31;
+  auto count = [&](int b) -> uint32_t {
+    return PACKED ? (hist[b >> 1] >> ((b & 1) << 4)) & 0xFFFFu : hist[b];
+  };
   uint32_t local = 0;
+#pragma unroll 8
+  for (int j = 0; j < 64; ++j) local += count(kHistBins - 1 - (64 * lane + ((j + lane) & 63)));
+  uint32_t incl = local;
 #pragma unroll
-  for (int j = 0; j < W; ++j) {  // descending bins: the high half of a word first
-    const uint32_t w = h16[kHistBins / 2 - 1 - (tid * W + j)];
-    c[2 * j] = w >> 16;
-    c[2 * j + 1] = w & 0xFFFFu;
-    local += c[2 * j] + c[2 * j + 1];
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  uint32_t total;
-  const uint32_t excl = block_excl_scan<kPfThreads>(local, total, scan_sm);
-  if (excl < k && k <= excl + local) {
+  const uint32_t excl = incl - local;
+  const uint32_t holder = __ballot_sync(0xffffffffu, excl < k && k <= incl);
+  int fb = -1;
+  uint32_t fa = 0;
+  if (holder != 0u && lane == __ffs(holder) - 1) {
     uint32_t run = excl;
-#pragma unroll
-    for (int i = 0; i < 2 * W; ++i) {
-      if (run + c[i] >= k) {
-        *out_bin = kHistBins - 1 - (tid * 2 * W + i);
-        *out_above = run;
+    for (int j = 0; j < 64; ++j) {
+      const int b = kHistBins - 1 - (64 * lane + j);
+      const uint32_t c = count(b);
+      if (run + c >= k) {
+        fb = b;
+        fa = run;
         break;
       }
-      run += c[i];
+      run += c;
     }
   }
-  __syncthreads();
+  const int src = holder != 0u ? __ffs(holder) - 1 : 0;
+  bin = __shfl_sync(0xffffffffu, fb, src);
+  above = __shfl_sync(0xffffffffu, fa, src);
 }
 
 // The blocked method; see the file comment.  grid (ceil(nrows / 16), Hq, B),
@@ -262,9 +272,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   __shared__ uint32_t rb1[kPfRows], rk1[kPfRows], rb2[kPfRows], rk2[kPfRows], rn2[kPfRows], rcnt[kPfRows];
   __shared__ uint32_t rbin[kPfRows];  // keys of the threshold bin appended per row (pass 2)
   __shared__ uint32_t rkept[kPfRows], rabove[kPfRows];
-  __shared__ uint32_t scan_sm[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above;
   __shared__ int s_any2, s_not2, s_big2;
   uint32_t* hist = pf_smem;
   uint2* lists = reinterpret_cast<uint2*>(pf_smem);  // [16][kPfListCap], pass 3 only
@@ -278,7 +285,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
     s_any2 = 0;
     s_not2 = 0;
     s_big2 = 0;
-    s_bin = 0;
   }
   __syncthreads();
   if (tid < kPfRows) {
@@ -417,15 +423,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
       }
     }
     __syncthreads();
-    for (int r = 0; r < kPfRows; ++r) {
-      if (rmode[r] != 2) continue;  // uniform: shared value
-      find_bin<kHistBins / kPfThreads, kPfThreads>(hist + r * kHistBins, (uint32_t)rk[r], scan_sm, &s_bin, &s_above);
-      if (tid == 0) {
-        rb1[r] = (uint32_t)s_bin;
-        rk1[r] = (uint32_t)rk[r] - s_above;
+    static_assert(kPfThreads / 32 >= kPfRows, "a warp per row");
+    if (warp < kPfRows && rmode[warp] == 2) {  // the 16 rows' threshold bins at once
+      int bin;
+      uint32_t ab;
+      warp_find_bin<false>(hist + warp * kHistBins, (uint32_t)rk[warp], bin, ab);
+      if (lane == 0) {
+        if (bin < 0) {  // inconsistent scores: count error, indices kept in bounds
+          atomicOr(p.status, TB_DEV_ERR_COUNT);
+          bin = 0;
+          ab = 0;
+        }
+        rb1[warp] = (uint32_t)bin;
+        rk1[warp] = (uint32_t)rk[warp] - ab;
       }
-      __syncthreads();
     }
+    __syncthreads();
     for (int e = tid; e < kPfRows * kHistBins; e += kPfThreads) hist[e] = 0u;
     __syncthreads();
   }
@@ -512,21 +525,28 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
   __syncthreads();
   if (any2) {
-    for (int r = 0; r < kPfRows; ++r) {
-      if (rmode[r] != 2) continue;
+    if (warp < kPfRows && rmode[warp] == 2) {
+      const int r = warp;
+      int bin;
+      uint32_t ab;
       if (lm)
-        find_bin16(hist + r * (kHistBins / 2), rk1[r], scan_sm, &s_bin, &s_above);
+        warp_find_bin<true>(hist + r * (kHistBins / 2), rk1[r], bin, ab);
       else
-        find_bin<kHistBins / kPfThreads, kPfThreads>(hist + r * kHistBins, rk1[r], scan_sm, &s_bin, &s_above);
-      if (tid == 0) {
-        rb2[r] = (uint32_t)s_bin;
-        rk2[r] = rk1[r] - s_above;
-        rabove[r] = s_above;
-        rn2[r] = lm ? (hist[r * (kHistBins / 2) + (s_bin >> 1)] >> ((s_bin & 1) << 4)) & 0xFFFFu
-                    : hist[r * kHistBins + s_bin];
+        warp_find_bin<false>(hist + r * kHistBins, rk1[r], bin, ab);
+      if (lane == 0) {
+        if (bin < 0) {
+          atomicOr(p.status, TB_DEV_ERR_COUNT);
+          bin = 0;
+          ab = 0;
+        }
+        rb2[r] = (uint32_t)bin;
+        rk2[r] = rk1[r] - ab;
+        rabove[r] = ab;
+        rn2[r] = lm ? (hist[r * (kHistBins / 2) + (bin >> 1)] >> ((bin & 1) << 4)) & 0xFFFFu
+                    : hist[r * kHistBins + bin];
       }
-      __syncthreads();
     }
+    __syncthreads();
   }
   if (tid < nr) p.redo[((size_t)b * p.Hq + h) * p.nrows + r0 + tid] = (rmode[tid] == 2 && rn2[tid] > (uint32_t)kPfListCap);
   if (tid < kPfRows && rmode[tid] == 2 && rn2[tid] > (uint32_t)kPfListCap) atomicOr(&s_big2, 1);
