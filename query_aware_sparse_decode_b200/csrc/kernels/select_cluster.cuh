@@ -53,8 +53,11 @@
 
 namespace tb {
 
-constexpr int kClThreads = 512;
-constexpr int kClWarps = kClThreads / 32;
+// Threads per CTA: 512 (two CTAs per SM) when the rows' clusters need more
+// than one CTA per SM, 1024 (one per SM) when they fit one wave of one CTA
+// per SM (few rows: every SM then runs one 32-warp CTA)
+constexpr int kClThreadsMany = 512;
+constexpr int kClThreadsFew = 1024;
 constexpr int kClChunkMax = 65536;            // tokens per CTA
 constexpr int kClWordsMax = kClChunkMax / 32;  // mask words per CTA
 constexpr int kClListCap = 4096;              // keys of the threshold bin kept in shared memory
@@ -131,16 +134,16 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
 // the running count from the top reaches k.  A histogram holding fewer than
 // k keys (inconsistent scores, e.g. NaN) records TB_DEV_ERR_COUNT and yields
 // bin 0, so every index stays in bounds.
-template <int NB>
+template <int NT, int NB>
 __device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32_t k, ClusterSelectSmem& sm,
                                                    uint32_t* status, uint32_t& above) {
-  for (int i = threadIdx.x; i < NB; i += kClThreads) sm.tot[i] = __ldcg(total + i);
+  for (int i = threadIdx.x; i < NB; i += NT) sm.tot[i] = __ldcg(total + i);
   if (threadIdx.x == 0) {
     sm.bin = -1;
     sm.above = 0;
   }
   __syncthreads();
-  find_bin<NB / kClThreads, kClThreads>(sm.tot, k, sm.scan, &sm.bin, &sm.above);  // ends with a block barrier
+  find_bin<NB / NT, NT>(sm.tot, k, sm.scan, &sm.bin, &sm.above);  // ends with a block barrier
   const int bin = sm.bin;
   above = sm.above;
   if (bin < 0) {
@@ -152,9 +155,9 @@ __device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32
 }
 
 // Adds this CTA's histogram into the row's total in L2 (non-empty bins only).
-template <int NB>
+template <int NT, int NB>
 __device__ __forceinline__ void hist_to_total(const uint32_t* hist, uint32_t* total) {
-  for (int i = threadIdx.x; i < NB; i += kClThreads) {
+  for (int i = threadIdx.x; i < NB; i += NT) {
     const uint32_t v = hist[i];
     if (v) atomicAdd(total + i, v);
   }
@@ -164,19 +167,19 @@ __device__ __forceinline__ void hist_to_total(const uint32_t* hist, uint32_t* to
 // candidates [lo, hi)), reading the scores with four 16-byte loads per
 // thread in flight.  The row holds max_len >= b scores, a multiple of 256,
 // so every 16-byte load that starts below b stays inside the row.
-template <class F>
+template <int NT, class F>
 __device__ __forceinline__ void visit_candidates(const float* srow, int a, int b, int lo, int hi, F f) {
   const int start = max(a, lo) & ~3, end = min(b, hi);
-  for (int base = start; base < end; base += 16 * kClThreads) {
+  for (int base = start; base < end; base += 16 * NT) {
     float4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int t0 = base + 4 * (threadIdx.x + kClThreads * u);
+      const int t0 = base + 4 * (threadIdx.x + NT * u);
       v[u] = t0 < end ? __ldcg(reinterpret_cast<const float4*>(srow + t0)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int t0 = base + 4 * (threadIdx.x + kClThreads * u);
+      const int t0 = base + 4 * (threadIdx.x + NT * u);
       const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -187,8 +190,11 @@ __device__ __forceinline__ void visit_candidates(const float* srow, int a, int b
   }
 }
 
-// grid (NC, rows, B), cluster (NC, 1, 1), kClThreads threads, kClSmem bytes.
-__global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const SelectParams p, int chunk) {
+// grid (NC, rows, B), cluster (NC, 1, 1), NT threads, kClSmem bytes.
+template <int NT>
+__global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const SelectParams p, int chunk) {
+  constexpr int kClThreads = NT;
+  constexpr int kClWarps = NT / 32;
   pdl_wait();
   pdl_trigger();
   namespace cg = cooperative_groups;
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const Sel
     if (wb < we) load_batch(va, wb);  // requested first: their latency overlaps the digit-1 search
     // ---- digit 1 from the row's first-digit histogram; the bin's bounds as floats
     uint32_t above;
-    const uint32_t b1 = total_find_bin<kHistBins>(p.hist1 + row * kHistBins, (uint32_t)rs.k, sm, p.status, above);
+    const uint32_t b1 = total_find_bin<NT, kHistBins>(p.hist1 + row * kHistBins, (uint32_t)rs.k, sm, p.status, above);
     const uint32_t kleft = (uint32_t)rs.k - above;
     const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
     const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
@@ -316,10 +322,10 @@ __global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const Sel
       }
     }
     __syncthreads();
-    hist_to_total<kHistBins>(sm.hist, tot);
+    hist_to_total<NT, kHistBins>(sm.hist, tot);
     cluster.sync();  // the row's digit-2 total is complete in L2
     // ---- digit 2
-    const uint32_t b2 = total_find_bin<kHistBins>(tot, kleft, sm, p.status, above);
+    const uint32_t b2 = total_find_bin<NT, kHistBins>(tot, kleft, sm, p.status, above);
     const uint32_t kleft2 = kleft - above;
     const uint32_t prefix22 = (b1 << 11) | b2;
     const uint32_t n_list = sm.n_list;
@@ -332,15 +338,15 @@ __global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const Sel
         if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
       }
     } else {
-      visit_candidates(srow, c0, c1, rs.lo, rs.hi, [&](int, uint32_t key) {
+      visit_candidates<NT>(srow, c0, c1, rs.lo, rs.hi, [&](int, uint32_t key) {
         if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
       });
     }
     __syncthreads();
-    hist_to_total<kClHist3>(sm.hist, tot + kHistBins);
+    hist_to_total<NT, kClHist3>(sm.hist, tot + kHistBins);
     cluster.sync();  // the row's digit-3 total is complete in L2
     // ---- digit 3: the k-th key T and the number of keys equal to T that are kept
-    const uint32_t b3 = total_find_bin<kClHist3>(tot + kHistBins, kleft2, sm, p.status, above);
+    const uint32_t b3 = total_find_bin<NT, kClHist3>(tot + kHistBins, kleft2, sm, p.status, above);
     const uint32_t T = (prefix22 << 10) | b3;
     const uint32_t quota = kleft2 - above;
     const uint32_t ntie_all = sm.tot[b3], my_ties = sm.hist[b3];
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kClThreads, 2) select_cluster_kernel(const Sel
           atomicOr(&sm.tbits[e.y >> 5], 1u << (e.y & 31));
       }
     } else {
-      visit_candidates(srow, c0, c1, rs.lo, rs.hi, [&](int t, uint32_t key) {
+      visit_candidates<NT>(srow, c0, c1, rs.lo, rs.hi, [&](int t, uint32_t key) {
         const int o = t - c0;
         if (key > T && (key >> 21) == b1)
           atomicOr(&sm.mword[o >> 5], 1u << (o & 31));

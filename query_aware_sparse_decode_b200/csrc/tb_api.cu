@@ -123,7 +123,10 @@ struct tb_ctx {
   float* votes = nullptr;
   float* vstats = nullptr;
   bool hist_clean = false;  // histograms and counters known to be zero (cleared by the last selection)
-  int cluster_active[5] = {};  // resident clusters of 1, 2, 4, 8, 16 CTAs of the selection kernel (0: not launchable)
+  // resident clusters of 1, 2, 4, 8, 16 CTAs of the selection kernel (0: not launchable), for its
+  // 512-thread and its 1024-thread CTAs
+  int cluster_active[5] = {};
+  int cluster_active_few[5] = {};
   uint32_t* ctot = nullptr;
   uint32_t* cslot = nullptr;
   uint32_t* reuse = nullptr;
@@ -180,11 +183,12 @@ static int max_len_of(const LayerState& ls, int B) {
 
 // How many clusters of 1, 2, 4, 8 and 16 CTAs of the cluster selection
 // kernel can be resident at once on this device (0: that size cannot run).
-static void probe_cluster_select(tb_ctx* ctx) {
-  for (int i = 0; i < 5; ++i) ctx->cluster_active[i] = 0;
-  if (cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kClSmem) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+template <int NT>
+static void probe_cluster_select_nt(int (&active)[5]) {
+  auto k = select_cluster_kernel<NT>;
+  for (int i = 0; i < 5; ++i) active[i] = 0;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kClSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
     return;
   }
@@ -192,7 +196,7 @@ static void probe_cluster_select(tb_ctx* ctx) {
     const int nc = 1 << i;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nc, 1, 1);
-    cfg.blockDim = dim3(kClThreads);
+    cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = kClSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -202,12 +206,17 @@ static void probe_cluster_select(tb_ctx* ctx) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, select_cluster_kernel, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&clusters, k, &cfg) != cudaSuccess) {
       cudaGetLastError();
       clusters = 0;
     }
-    ctx->cluster_active[i] = clusters;
+    active[i] = clusters;
   }
+}
+
+static void probe_cluster_select(tb_ctx* ctx) {
+  probe_cluster_select_nt<kClThreadsMany>(ctx->cluster_active);
+  probe_cluster_select_nt<kClThreadsFew>(ctx->cluster_active_few);
 }
 
 // ------------------------------------------------------------------ launches
@@ -328,7 +337,13 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   for (int b = 0; b < c.batch; ++b) p.lens[b] = ls.lens[b];
   const int maxL = max_len_of(ls, c.batch);
   int nc = 0, chunk = 0;
-  if (cluster_select_shape(ctx->num_sms, (long long)rows * c.batch, maxL, ctx->cluster_active, &nc, &chunk)) {
+  // 1024-thread CTAs when the rows' clusters fit one wave of one CTA per SM
+  const long long nrows = (long long)rows * c.batch;
+  bool few = cluster_select_shape(ctx->num_sms, nrows, maxL, ctx->cluster_active_few, &nc, &chunk);
+  int ci = 0;
+  while (few && (1 << ci) < nc) ++ci;
+  few = few && nrows * nc <= ctx->num_sms && nrows <= ctx->cluster_active_few[ci];
+  if (few || cluster_select_shape(ctx->num_sms, nrows, maxL, ctx->cluster_active, &nc, &chunk)) {
     // one cluster per row: one launch after the first-digit histogram
     if (!hist1_ready) {
       dim3 cgrid((std::max(maxL, 1) + kSelChunk - 1) / kSelChunk, rows, c.batch);
@@ -338,8 +353,12 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
     }
     p.ctot = ctx->ctot;
     p.cslot = ctx->cslot;
-    launch_pdl_cluster(select_cluster_kernel, dim3(nc, rows, c.batch), dim3(kClThreads), (size_t)kClSmem, st, nc, p,
-                       chunk);
+    if (few)
+      launch_pdl_cluster(select_cluster_kernel<kClThreadsFew>, dim3(nc, rows, c.batch), dim3(kClThreadsFew),
+                         (size_t)kClSmem, st, nc, p, chunk);
+    else
+      launch_pdl_cluster(select_cluster_kernel<kClThreadsMany>, dim3(nc, rows, c.batch), dim3(kClThreadsMany),
+                         (size_t)kClSmem, st, nc, p, chunk);
     ++ctx->launches;
     const tb_status s = cuda_status(cudaGetLastError());
     if (s == TB_OK) ctx->hist_clean = true;  // CTA 0 of every row clears the row's histogram
