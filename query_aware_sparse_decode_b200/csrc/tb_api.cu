@@ -276,7 +276,8 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
     auto k = hist ? (grouped ? score_kernel<T, KT, DI, GSV, true, true> : score_kernel<T, KT, DI, GSV, true, false>) \
                   : (grouped ? score_kernel<T, KT, DI, GSV, false, true>                             \
                              : score_kernel<T, KT, DI, GSV, false, false>);                          \
-    if (hist) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
+    if (hist && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+      return TB_ERR_CUDA;                                                                            \
     launch_pdl(k, grid, dim3(kScoreThreads), smem, st, p);                                           \
     ++ctx->launches;                                                                                 \
     return cuda_status(cudaGetLastError());                                                          \
@@ -377,9 +378,13 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
                dim3(kScatThreads), 0, st, p);
     ++ctx->launches;
   }
-  cudaFuncSetAttribute(select_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScatSmem);
+  if (cudaFuncSetAttribute(select_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScatSmem) !=
+      cudaSuccess)
+    return TB_ERR_CUDA;
   launch_pdl(select_scatter_kernel, cgrid, dim3(kScatThreads), kScatSmem, st, p);
-  cudaFuncSetAttribute(select_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kResolveSmem);
+  if (cudaFuncSetAttribute(select_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kResolveSmem) !=
+      cudaSuccess)
+    return TB_ERR_CUDA;
   launch_pdl(select_resolve_kernel, dim3(rows, c.batch), dim3(kSelThreads), kResolveSmem, st, p);
   ctx->launches += 2;
   const tb_status s = cuda_status(cudaGetLastError());
@@ -420,12 +425,14 @@ static tb_status launch_attn(tb_ctx* ctx, int layer, const void* q, const uint32
     if (c.kv_dtype == TB_BF16) {                                                                            \
       auto k = attn_bf16_kernel<DV, GSV>;                                                                   \
       const int smem = attn_bf16_smem_bytes<DV>();                                                          \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+        return TB_ERR_CUDA;                                                                          \
       launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                        \
     } else {                                                                                                \
       auto k = attn_f32_kernel<DV, GSV>;                                                                    \
       const int smem = attn_f32_smem_bytes<DV>();                                                           \
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                           \
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) \
+        return TB_ERR_CUDA;                                                                          \
       launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                                        \
     }                                                                                                       \
   } else
@@ -500,7 +507,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
   if (c.head_dim == DV && gs == GSV) {                                                        \
     auto k = softvote_logits_kernel<DV, GSV>;                                                 \
     const int smem = vote_logits_smem<DV>();                                                  \
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);               \
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return TB_ERR_CUDA; \
     launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                            \
   } else
   TB_VOTE_CASE(128, 4) TB_VOTE_CASE(128, 2) TB_VOTE_CASE(128, 1) TB_VOTE_CASE(128, 8)
@@ -1033,10 +1040,12 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
 #define TB_PF_CASE(T, KT, DI)                                                           \
   if (c.d_imp == DI) {                                                                  \
     auto kb = prefill_rows_kernel<T, KT, DI>;                                           \
-    cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem);     \
+    if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem) != cudaSuccess) \
+      return TB_ERR_CUDA;                                                                            \
     kb<<<grid, kPfThreads, kPfSmem, st>>>(p);                                           \
     auto kr = prefill_redo_kernel<T, KT, DI>;                                           \
-    cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);   \
+    if (cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+      return TB_ERR_CUDA;                                                                            \
     kr<<<rgrid, kSelThreads, smem, st>>>(p);                                            \
     ctx->launches += 2;                                                                 \
   } else
