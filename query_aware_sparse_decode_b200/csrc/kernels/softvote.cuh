@@ -30,9 +30,11 @@ namespace tb {
 // Tokens per CTA of the logits pass: chosen per launch (a multiple of 16, at
 // least kVoteMinChunk) so that the grid is about four CTAs per SM in one wave.
 constexpr int kVoteMinChunk = 256;
+constexpr int kVoteWarps = 4;   // warps per CTA of the logits pass
+constexpr int kVoteThreads = kVoteWarps * 32;
 constexpr int kVoteStages = 3;  // ring stages per warp of the logits pass (16 K rows each)
 template <int D>
-constexpr int vote_logits_smem() { return kAttnWarps * kVoteStages * kAttnTile * D * 2; }
+constexpr int vote_logits_smem() { return kVoteWarps * kVoteStages * kAttnTile * D * 2; }
 
 struct VoteParams {
   const void* k_cache;  // [B][Hkv][max_len][D] bf16, or a page pool (KvLayout)
@@ -50,7 +52,7 @@ struct VoteParams {
 };
 
 template <int D, int GS>
-__global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const VoteParams p) {
+__global__ void __launch_bounds__(kVoteThreads, 2) softvote_logits_kernel(const VoteParams p) {
   pdl_wait();
   pdl_trigger();
   constexpr int ROWB = D * 2;
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   // per lane and head: running max and sum of 2^(a - max) over the lane's tokens
   float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};
   const int ntiles = (n + kAttnTile - 1) / kAttnTile;
-  const int my_n = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  const int my_n = ntiles > warp ? (ntiles - warp + kVoteWarps - 1) / kVoteWarps : 0;
   uint8_t* my_ring = smem + warp * kVoteStages * STAGE;
   const uint32_t ring_u32 = smem_u32(my_ring);
   // ldmatrix rows: lane supplies row (lane & 7) of matrix (lane >> 3) = tokens
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   // 16 and pages hold a power of two >= 16 tokens, so one row lookup per tile
   // serves all of them (rows past the ragged end repeat the last token).
   auto issue = [&](int it) {
-    const int tile = warp + it * kAttnWarps;
+    const int tile = warp + it * kVoteWarps;
     uint8_t* sb = my_ring + (it % kVoteStages) * STAGE;
     const int tt = t0 + tile * kAttnTile;
     const int last = t1 - 1 - tt;
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     cp_async_wait<kVoteStages - 1>();
     __syncwarp();
     const uint32_t st = ring_u32 + (uint32_t)((it % kVoteStages) * STAGE);
-    const int tile = warp + it * kAttnWarps;
+    const int tile = warp + it * kVoteWarps;
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
     }
   __syncthreads();
   float* wm = reinterpret_cast<float*>(smem);
-  float* wl = wm + kAttnWarps * GS;
+  float* wl = wm + kVoteWarps * GS;
   if (grp == 0) {
     if (real0) {
       wm[warp * GS + hp] = m_run[0];
@@ -190,10 +192,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) softvote_logits_kernel(const 
   __syncthreads();
   if (tid < GS) {
     float M = kNegInf;
-    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, wm[w * GS + tid]);
+    for (int w = 0; w < kVoteWarps; ++w) M = fmaxf(M, wm[w * GS + tid]);
     float l = 0.f;
     if (M != kNegInf)
-      for (int w = 0; w < kAttnWarps; ++w)
+      for (int w = 0; w < kVoteWarps; ++w)
         if (wm[w * GS + tid] != kNegInf) l += wl[w * GS + tid] * exp2f(wm[w * GS + tid] - M);
     const size_t ph = (((size_t)b * p.Hq + g * GS + tid) * p.nchunk + chunk) * 2;
     p.stats[ph] = M;

@@ -508,7 +508,7 @@ static tb_status launch_softvote(tb_ctx* ctx, int layer, const void* q, float* v
     auto k = softvote_logits_kernel<DV, GSV>;                                                 \
     const int smem = vote_logits_smem<DV>();                                                  \
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return TB_ERR_CUDA; \
-    launch_pdl(k, grid, dim3(kAttnThreads), smem, st, p);                            \
+    launch_pdl(k, grid, dim3(kVoteThreads), smem, st, p);                            \
   } else
   TB_VOTE_CASE(128, 4) TB_VOTE_CASE(128, 2) TB_VOTE_CASE(128, 1) TB_VOTE_CASE(128, 8)
   TB_VOTE_CASE(64, 4) TB_VOTE_CASE(64, 2) TB_VOTE_CASE(64, 1) TB_VOTE_CASE(64, 8)
