@@ -12,6 +12,7 @@
 
 #include "kernels/attn.cuh"
 #include "kernels/attn_split.cuh"
+#include "kernels/combine.cuh"
 #include "kernels/index_mask.cuh"
 #include "kernels/common.cuh"
 #include "kernels/kimp.cuh"

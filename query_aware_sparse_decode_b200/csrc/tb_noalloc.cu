@@ -29,6 +29,7 @@
 
 #include "kernels/attn.cuh"
 #include "kernels/attn_split.cuh"
+#include "kernels/combine.cuh"
 #include "tb.h"
 
 using namespace tb;
