@@ -247,7 +247,9 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
  * L -> p + 1.  `q_imp_rows`: [(B*Hq)][G][nrows][d'] (positions row0..), slot
  * (layer-1) mod G.  `row_masks`: [B][Hq][nrows][words_per_row] uint32 with
  * words_per_row >= ceil((row0 + nrows)/32); every word is written.
- * Requires len[b] >= row0 + nrows (K_imp rows present).  Rows are scored in
+ * Requires len[b] >= row0 + nrows (K_imp rows present) and
+ * row0 + nrows <= 51200 (a row's fp32 scores fit 200 KB of shared memory for
+ * the massive-ties method), else TB_ERR_UNSUPPORTED.  Rows are scored in
  * blocks of 16 on the tensor cores (TF32 with an fp32 K_imp split into a TF32 head
  * and its remainder, fp32 accumulation: about 1e-6 relative to the fp32 dot
  * product; a bf16 K_imp is exact in TF32 and needs no split); rows with

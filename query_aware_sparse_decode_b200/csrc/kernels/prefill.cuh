@@ -14,8 +14,8 @@
 //   1. first-digit (11-bit) histograms of the 16 rows' candidates;
 //   2. mask words of sink, window and keys above each row's threshold bin
 //      (one ballot per row and 32 tokens), second-digit histograms of the
-//      threshold bins, and (rows under 65536 tokens) each row's keys of its
-//      threshold bin listed in shared memory, up to kPfBinCap per row;
+//      threshold bins, and each row's keys of its threshold bin listed in
+//      shared memory, up to kPfBinCap per row;
 //   3. from those lists, keys above the 22-bit threshold prefix are OR-ed
 //      into the mask and keys equal to it (a handful per row) are listed and
 //      ranked by (key desc, index asc), which also settles ties.  Rows whose
@@ -35,10 +35,14 @@ namespace tb {
 constexpr int kPfRows = 16;       // rows per CTA of the blocked kernel
 constexpr int kPfThreads = 512;
 constexpr int kPfListCap = 256;   // keys per row sharing the 22-bit threshold prefix
+// Prefixes the prefill selection accepts: the one-row method keeps a row's
+// fp32 scores in 200 KB of shared memory.  Below 65536 tokens, so a 16-bit
+// counter holds any bin's count.
+constexpr int kPfMaxPrefix = 200 * 1024 / 4;
+static_assert(kPfMaxPrefix < 65536, "16-bit second-digit counters");
 // Pass 2 keeps each row's keys of its threshold bin in shared memory (with
 // 16-bit second-digit counters, two per word) so that pass 3 works on those
-// lists instead of recomputing the tiles: rows of fewer than 65536 tokens, up
-// to kPfBinCap keys per row.
+// lists instead of recomputing the tiles: up to kPfBinCap keys per row.
 constexpr int kPfBinCap = 1280;
 constexpr int kPfHist16Words = kPfRows * kHistBins / 2;
 constexpr int kPfSmem = kPfHist16Words * 4 + kPfRows * kPfBinCap * 8;  // >= the 32-bit first-digit histograms
@@ -314,7 +318,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // interior tiles then need no per-token range or mode checks
   const bool all2 = s_not2 == 0;
   const int Lmax = nr > 0 ? p.row0 + r0 + nr : 0;
-  const bool lm = Lmax < 65536;  // 16-bit second-digit counters and bin lists in pass 2
   const int L0 = p.row0 + r0 + 1;        // row r covers tokens [0, L0 + r)
   const int hi0 = L0 - p.window;         // row r's candidates are [sink, hi0 + r)
   const size_t slab = (size_t)b * p.Hkv + g;
@@ -444,17 +447,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   }
 
   // ---- pass 2: every mask word of every row (sink, window, keys above the
-  // threshold bin), second-digit histograms of the threshold bins, and (rows
-  // under 65536 tokens) the threshold bin's keys listed per row
+  // threshold bin), second-digit histograms of the threshold bins (16-bit
+  // counters), and the threshold bin's keys listed per row
   auto member = [&](int row, uint32_t key, int t) {
     const uint32_t d2 = (key >> 10) & (kHistBins - 1);
-    if (lm) {
-      atomicAdd(&hist[row * (kHistBins / 2) + (d2 >> 1)], 1u << ((d2 & 1u) << 4));
-      const uint32_t slot = atomicAdd(&rbin[row], 1u);
-      if (slot < (uint32_t)kPfBinCap) blists[row * kPfBinCap + slot] = make_uint2(key, (uint32_t)t);
-    } else {
-      atomicAdd(&hist[row * kHistBins + d2], 1u);
-    }
+    atomicAdd(&hist[row * (kHistBins / 2) + (d2 >> 1)], 1u << ((d2 & 1u) << 4));
+    const uint32_t slot = atomicAdd(&rbin[row], 1u);
+    if (slot < (uint32_t)kPfBinCap) blists[row * kPfBinCap + slot] = make_uint2(key, (uint32_t)t);
   };
   {
     const int mda = rmode[ra], mdb = rmode[rb];
@@ -529,10 +528,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
       const int r = warp;
       int bin;
       uint32_t ab;
-      if (lm)
-        warp_find_bin<true>(hist + r * (kHistBins / 2), rk1[r], bin, ab);
-      else
-        warp_find_bin<false>(hist + r * kHistBins, rk1[r], bin, ab);
+      warp_find_bin<true>(hist + r * (kHistBins / 2), rk1[r], bin, ab);
       if (lane == 0) {
         if (bin < 0) {
           atomicOr(p.status, TB_DEV_ERR_COUNT);
@@ -542,8 +538,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
         rb2[r] = (uint32_t)bin;
         rk2[r] = rk1[r] - ab;
         rabove[r] = ab;
-        rn2[r] = lm ? (hist[r * (kHistBins / 2) + (bin >> 1)] >> ((bin & 1) << 4)) & 0xFFFFu
-                    : hist[r * kHistBins + bin];
+        rn2[r] = (hist[r * (kHistBins / 2) + (bin >> 1)] >> ((bin & 1) << 4)) & 0xFFFFu;
       }
     }
     __syncthreads();
@@ -556,7 +551,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_rows_kernel(const Prefi
   // into the row's list
   if (any2) {
     // a row is resolved from its bin list when the list holds the whole bin
-    auto listed = [&](int r) { return lm && rbin[r] <= (uint32_t)kPfBinCap; };
+    auto listed = [&](int r) { return rbin[r] <= (uint32_t)kPfBinCap; };
     {  // keys of the listed rows' bins above the 22-bit prefix into the mask, keys at it into the row's list
       for (int e = tid; e < kPfRows * kPfBinCap; e += kPfThreads) {
         const int r = e / kPfBinCap, i = e % kPfBinCap;

@@ -1014,8 +1014,8 @@ TB_API tb_status tb_select_prefill(tb_ctx* ctx, int layer, const void* q_imp_row
   if (words_per_row < (need + 31) / 32) return TB_ERR_SHAPE;
   for (int b = 0; b < c.batch; ++b)
     if (ls.lens[b] < need) return TB_ERR_STATE;  // K_imp rows of the prefix must exist
+  if (need > kPfMaxPrefix) return TB_ERR_UNSUPPORTED;  // the one-row method keeps row scores in shared memory
   const size_t smem = (size_t)need * 4;
-  if (smem > 200 * 1024) return TB_ERR_UNSUPPORTED;  // row scores live in shared memory
   PrefillParams p{};
   p.q_imp = q_imp_rows;
   p.kimp = ls.kimp;

@@ -190,6 +190,21 @@ def test_prefill_rows_with_massive_ties_take_the_one_row_path():
             assert np.array_equal(np.nonzero(bits[:p + 1])[0], ref[h, p])
 
 
+def test_prefill_rows_longest_prefix_and_the_limit_beyond():
+    """Rows up to the accepted prefix of 51200 tokens select exactly; one
+    token more is refused before any launch (TB_ERR_UNSUPPORTED)."""
+    wl = PF_SMALL.with_(B=1, L=51200, n_layers=6)
+    _prefill_case(wl, layer=5, row0=51200 - 40, nrows=40, heads=[0, 3, 7], rows=[0, 7, 15, 16, 23, 24, 39])
+    cfg = config_of(wl.with_(L=51201), max_len=round_up(51201, 256))
+    ctx = TB.Context(cfg)
+    make_layer(ctx, wl.with_(L=51201), 5, [51201])
+    qrows = S.q_imp(wl, O.producer_of(5, wl.G), rows=(51201 - 16, 16))
+    masks = torch.zeros((1, wl.Hq, 16, (51201 + 31) // 32), dtype=torch.int32, device="cuda")
+    with pytest.raises(TB.TBError) as err:
+        ctx.select_prefill(5, to_dev(qrows, wl), 51201 - 16, 16, masks)
+    assert err.value.status == 7  # TB_ERR_UNSUPPORTED
+
+
 def test_prefill_rows_blocked_partial_block_and_mixed_budgets():
     """nrows not a multiple of the 16-row block, rows whose prefixes are
     shorter than sink + window next to rows with a real top-k."""
