@@ -27,8 +27,8 @@ struct AppendParams {
 // (all of them call it: it contains barriers): writes the K and V rows, then
 // K_imp[j] = sum_d K[d] W_K[d][j] in fp32 with W_K staged in shared memory;
 // the first 128 threads form 128 / d' partial sums per output column (over
-// D / parts dimensions each, ascending) that are added in a fixed order, so
-// the row is the same bits whichever kernel computes it.  `scratch` holds
+// D / parts dimensions each, as four interleaved chains) that are added in a
+// fixed order, so the row is the same bits whichever kernel computes it.  `scratch` holds
 // D * d' + 256 floats.
 constexpr int kAppendScratchFloats = 128 * 32 + 256;
 template <typename T>
@@ -41,6 +41,12 @@ __device__ __forceinline__ void append_row(const AppendParams& p, int g, int b, 
   const size_t row = kv_row(p.kl, b, g, p.Hkv, p.max_len, p.pos[b]);
   const T* W = reinterpret_cast<const T*>(p.w_k);
   const int nw = p.D * p.dimp;
+  // the new K and V elements are requested first: their latency overlaps W_K's
+  T kv = T(), vv = T();
+  if (tid < p.D) {
+    kv = reinterpret_cast<const T*>(p.k_new)[src + tid];
+    vv = reinterpret_cast<const T*>(p.v_new)[src + tid];
+  }
   constexpr int VEC = 16 / (int)sizeof(T);  // W_K staged with 16-byte loads, all in flight
   if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && nw % VEC == 0) {
 #pragma unroll 8
@@ -54,19 +60,24 @@ __device__ __forceinline__ void append_row(const AppendParams& p, int g, int b, 
     for (int e = tid; e < nw; e += nt) wsm[e] = to_f32(W[e]);
   }
   if (tid < p.D) {
-    const T kv = reinterpret_cast<const T*>(p.k_new)[src + tid];
     reinterpret_cast<T*>(p.k_cache)[row * p.D + tid] = kv;
-    reinterpret_cast<T*>(p.v_cache)[row * p.D + tid] = reinterpret_cast<const T*>(p.v_new)[src + tid];
+    reinterpret_cast<T*>(p.v_cache)[row * p.D + tid] = vv;
     krow[tid] = to_f32(kv);
   }
   __syncthreads();
   if (tid < 128) {
     const int parts = 128 / p.dimp;  // 4 (d'=32) or 8 (d'=16)
     const int j = tid % p.dimp, q = tid / p.dimp;
-    const int span = p.D / parts;
-    float acc = 0.f;
-    for (int d = q * span; d < (q + 1) * span; ++d) acc = fmaf(krow[d], wsm[d * p.dimp + j], acc);
-    part[tid] = acc;
+    const int span = p.D / parts;  // a multiple of 4
+    // four interleaved chains (dimensions d = 4i + u), added in a fixed order
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int d = q * span; d < (q + 1) * span; d += 4) {
+      a0 = fmaf(krow[d], wsm[d * p.dimp + j], a0);
+      a1 = fmaf(krow[d + 1], wsm[(d + 1) * p.dimp + j], a1);
+      a2 = fmaf(krow[d + 2], wsm[(d + 2) * p.dimp + j], a2);
+      a3 = fmaf(krow[d + 3], wsm[(d + 3) * p.dimp + j], a3);
+    }
+    part[tid] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();
   if (tid < p.dimp) {
