@@ -19,8 +19,9 @@
 //      thread double-buffered in registers; scores compared as floats with
 //      the bin's bounds) writes, per 32-token word, "kept for sure" (sink,
 //      window, keys above bin b1) into a shared copy of the CTA's mask words,
-//      and appends the keys of bin b1 (a few percent of the row) to a shared
-//      list while histogramming their second digit.
+//      and appends the scores of bin b1 (a few percent of the row) to a
+//      shared list; after the pass the list's scores become keys and their
+//      second digit is histogrammed (a convergent loop over the list).
 //   3. each CTA adds its histogram into the row's total in L2 (atomics);
 //      after a cluster barrier every CTA reads the total back: digit 2, then
 //      digit 3 over the list the same way, give T and the number `quota` of
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
     const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
     const float f_hi = hi_open ? 0.f : key_to_float((b1 + 1u) << 21);       // smallest key above it
-    // ---- one pass over the CTA's tokens: sure-keep words, the bin's keys, digit-2 histogram.
+    // ---- one pass over the CTA's tokens: sure-keep words and the bin's scores.
     // Float comparisons against the bin's bounds decide the same as the keys
     // (the key map is monotone and folds -0.0 onto +0.0, as IEEE comparison
     // does).  A lane's bin members of a batch (bit 4u + j: its load u,
@@ -304,10 +305,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if ((memb >> (4 * u + j)) & 1u) {
-            const uint32_t key = order_key(vv[j]);
-            if (pos < (uint32_t)kClListCap) sm.list[pos] = make_uint2(key, (uint32_t)(tv + j - c0));
-            atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
+          if ((memb >> (4 * u + j)) & 1u) {  // the raw score bits: keyed after the pass
+            if (pos < (uint32_t)kClListCap) sm.list[pos] = make_uint2(__float_as_uint(vv[j]), (uint32_t)(tv + j - c0));
             ++pos;
           }
       }
@@ -320,6 +319,20 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         if (w0 + 2 * WB < we) load_batch(va, w0 + 2 * WB);
         process(vb, w0 + WB);
       }
+    }
+    __syncthreads();
+    // the list's scores as keys, and their digit-2 histogram (from L2 when the list overflowed)
+    const uint32_t n1 = sm.n_list;
+    if (n1 <= (uint32_t)kClListCap) {
+      for (uint32_t i = tid; i < n1; i += kClThreads) {
+        const uint32_t key = order_key(__uint_as_float(sm.list[i].x));
+        sm.list[i].x = key;
+        atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
+      }
+    } else {
+      visit_candidates<NT>(srow, c0, c1, rs.lo, rs.hi, [&](int, uint32_t key) {
+        if ((key >> 21) == b1) atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
+      });
     }
     __syncthreads();
     hist_to_total<NT, kHistBins>(sm.hist, tot);
