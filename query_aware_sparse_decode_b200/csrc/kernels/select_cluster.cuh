@@ -79,7 +79,12 @@ struct ClusterSelectSmem {
   int bin;
   uint32_t above;
 };
-constexpr int kClSmem = (int)sizeof(ClusterSelectSmem);
+constexpr int kClSmem = ((int)sizeof(ClusterSelectSmem) + 15) / 16 * 16;
+// Dynamic shared memory of an NT-thread CTA: the struct, then the first
+// pass's staging area (float4 [kClBatch][NT]: a lane's batch of scores, read
+// back by the lane itself for its threshold-bin members).
+template <int NT>
+constexpr int cl_smem() { return kClSmem + kClBatch * NT * 16; }
 
 // Host: cluster size and chunk of a selection over rows of at most maxL
 // tokens, `nrows` rows in all.  max_active[i] is how many clusters of 2^i
@@ -202,6 +207,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint8_t cl_raw[];
   ClusterSelectSmem& sm = *reinterpret_cast<ClusterSelectSmem*>(cl_raw);
+  float4* stage = reinterpret_cast<float4*>(cl_raw + kClSmem);  // [kClBatch][NT]
   const int nc = (int)cluster.num_blocks();
   const int c = (int)cluster.block_rank();
   const int r = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -249,7 +255,9 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     // Float comparisons against the bin's bounds decide the same as the keys
     // (the key map is monotone and folds -0.0 onto +0.0, as IEEE comparison
     // does).  A lane's bin members of a batch (bit 4u + j: its load u,
-    // element j) are appended with one warp scan and one shared atomic.
+    // element j) are appended with one warp scan and one shared atomic; a
+    // lane with members stages its batch in shared memory and reads back
+    // only those.
     auto process = [&](const float4 (&v)[kClBatch], int w0) {
       const bool interior =
           w0 + 4 * kClBatch <= we && c0 + 32 * w0 >= rs.lo && c0 + 32 * (w0 + 4 * kClBatch) <= min(rs.hi, c1);
@@ -287,6 +295,10 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         memb |= mb << (4 * u);
       }
       if (!__any_sync(0xffffffffu, memb != 0u)) return;
+      if (memb) {  // stage the batch: the members are then read by index, not by an unrolled walk of all 16
+#pragma unroll
+        for (int u = 0; u < kClBatch; ++u) stage[u * NT + tid] = v[u];
+      }
       const uint32_t cnt = __popc(memb);
       uint32_t x = cnt;  // inclusive prefix over the lanes
 #pragma unroll
@@ -298,17 +310,13 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
       if (lane == 31) base = atomicAdd(&sm.n_list, x);
       base = __shfl_sync(0xffffffffu, base, 31);
       uint32_t pos = base + x - cnt;
-#pragma unroll
-      for (int u = 0; u < kClBatch; ++u) {
-        if (((memb >> (4 * u)) & 0xFu) == 0u) continue;
-        const int tv = c0 + 32 * (w0 + 4 * u + (lane >> 3)) + 4 * (lane & 7);
-        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if ((memb >> (4 * u + j)) & 1u) {  // the raw score bits: keyed after the pass
-            if (pos < (uint32_t)kClListCap) sm.list[pos] = make_uint2(__float_as_uint(vv[j]), (uint32_t)(tv + j - c0));
-            ++pos;
-          }
+      const float* sf = reinterpret_cast<const float*>(stage);
+      for (uint32_t m = memb; m != 0u; m &= m - 1u) {  // the raw score bits: keyed after the pass
+        const int bit = __ffs(m) - 1, u = bit >> 2, j = bit & 3;
+        const float sv = sf[(u * NT + tid) * 4 + j];
+        const int o = 32 * (w0 + 4 * u + (lane >> 3)) + 4 * (lane & 7) + j;  // token - c0
+        if (pos < (uint32_t)kClListCap) sm.list[pos] = make_uint2(__float_as_uint(sv), (uint32_t)o);
+        ++pos;
       }
     };
     constexpr int WB = 4 * kClBatch;  // words per batch

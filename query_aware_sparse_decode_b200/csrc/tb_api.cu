@@ -188,7 +188,7 @@ template <int NT>
 static void probe_cluster_select_nt(int (&active)[5]) {
   auto k = select_cluster_kernel<NT>;
   for (int i = 0; i < 5; ++i) active[i] = 0;
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kClSmem) != cudaSuccess ||
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, cl_smem<NT>()) != cudaSuccess ||
       cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
     return;
@@ -198,7 +198,7 @@ static void probe_cluster_select_nt(int (&active)[5]) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nc, 1, 1);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = kClSmem;
+    cfg.dynamicSmemBytes = cl_smem<NT>();
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = nc;
@@ -357,10 +357,10 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
     p.cslot = ctx->cslot;
     if (few)
       launch_pdl_cluster(select_cluster_kernel<kClThreadsFew>, dim3(nc, rows, c.batch), dim3(kClThreadsFew),
-                         (size_t)kClSmem, st, nc, p, chunk);
+                         (size_t)cl_smem<kClThreadsFew>(), st, nc, p, chunk);
     else
       launch_pdl_cluster(select_cluster_kernel<kClThreadsMany>, dim3(nc, rows, c.batch), dim3(kClThreadsMany),
-                         (size_t)kClSmem, st, nc, p, chunk);
+                         (size_t)cl_smem<kClThreadsMany>(), st, nc, p, chunk);
     ++ctx->launches;
     const tb_status s = cuda_status(cudaGetLastError());
     if (s == TB_OK) ctx->hist_clean = true;  // CTA 0 of every row clears the row's histogram
