@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     const uint32_t kleft = (uint32_t)rs.k - above;
     const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
     const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
-    const float f_hi = hi_open ? 0.f : key_to_float((b1 + 1u) << 21);       // smallest key above it
+    // smallest key above it; NaN when there is none (no score compares >= NaN)
+    const float f_hi = hi_open ? __int_as_float(0x7fc00000) : key_to_float((b1 + 1u) << 21);
     // ---- one pass over the CTA's tokens: sure-keep words and the bin's scores.
     // Float comparisons against the bin's bounds decide the same as the keys
     // (the key map is monotone and folds -0.0 onto +0.0, as IEEE comparison
@@ -258,14 +259,15 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     // element j) are appended with one warp scan and one shared atomic; a
     // lane with members stages its batch in shared memory and reads back
     // only those.
+    static_assert(kClBatch == 4, "the word exchange below assumes four loads per batch");
     auto process = [&](const float4 (&v)[kClBatch], int w0) {
       const bool interior =
           w0 + 4 * kClBatch <= we && c0 + 32 * w0 >= rs.lo && c0 + 32 * (w0 + 4 * kClBatch) <= min(rs.hi, c1);
-      uint32_t memb = 0;  // bit 4u + j
+      const int p8 = lane & 7;
+      uint32_t kx[kClBatch];  // load u's sure-keep nibble at bits 4 * p8 of its word
+      uint32_t memb = 0;     // bit 4u + j
 #pragma unroll
       for (int u = 0; u < kClBatch; ++u) {
-        const int w = w0 + 4 * u + (lane >> 3);
-        const int tv = c0 + 32 * w + 4 * (lane & 7);
         const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
         uint32_t keep = 0, mb = 0;
         if (interior) {  // every token a valid candidate
@@ -274,26 +276,38 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
             keep |= (uint32_t)(vv[j] >= f_hi) << j;
             mb |= (uint32_t)(vv[j] >= f_lo) << j;
           }
-          if (hi_open) keep = 0;
           mb &= ~keep;
         } else {
+          const int w = w0 + 4 * u + (lane >> 3);
+          const int tv = c0 + 32 * w + 4 * p8;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int t = tv + j;
             const bool valid = w < we && t < c1;
             const bool cand = t >= rs.lo && t < rs.hi;
-            const bool up = !hi_open && vv[j] >= f_hi;
+            const bool up = vv[j] >= f_hi;
             keep |= (uint32_t)(valid && (!cand || up)) << j;
             mb |= (uint32_t)(valid && cand && !up && vv[j] >= f_lo) << j;
           }
         }
-        uint32_t word = keep << (4 * (lane & 7));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        if ((lane & 7) == 0 && w < we) sm.mword[w] = word;
+        kx[u] = keep << (4 * p8);
         memb |= mb << (4 * u);
       }
+      // Each 8-lane group's four words, OR-ed over the group in three
+      // exchange rounds: over lane bit 2 a lane keeps two words and sends
+      // two, over bit 1 it keeps one and sends one, over bit 0 both lanes
+      // complete the same word.  Lane p8 ends with word u = 2 * (p8 >> 2 & 1)
+      // + (p8 >> 1 & 1); the even lane stores it.
+      const bool hb = (p8 & 4) != 0, mbit = (p8 & 2) != 0;
+      uint32_t k0 = hb ? kx[2] : kx[0], k1 = hb ? kx[3] : kx[1];
+      const uint32_t s0 = hb ? kx[0] : kx[2], s1 = hb ? kx[1] : kx[3];
+      k0 |= __shfl_xor_sync(0xffffffffu, s0, 4);
+      k1 |= __shfl_xor_sync(0xffffffffu, s1, 4);
+      uint32_t word = mbit ? k1 : k0;
+      word |= __shfl_xor_sync(0xffffffffu, mbit ? k0 : k1, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      const int wq = w0 + 4 * ((hb ? 2 : 0) + (mbit ? 1 : 0)) + (lane >> 3);
+      if ((p8 & 1) == 0 && wq < we) sm.mword[wq] = word;
       if (!__any_sync(0xffffffffu, memb != 0u)) return;
       if (memb) {  // stage the batch: the members are then read by index, not by an unrolled walk of all 16
 #pragma unroll
