@@ -136,14 +136,13 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// A cluster total (NB words in L2) read into shared memory, and the bin where
-// the running count from the top reaches k.  A histogram holding fewer than
-// k keys (inconsistent scores, e.g. NaN) records TB_DEV_ERR_COUNT and yields
-// bin 0, so every index stays in bounds.
+// The bin where the running count from the top of a histogram staged in
+// sm.tot (NB words, stored by the caller) reaches k.  A histogram holding
+// fewer than k keys (inconsistent scores, e.g. NaN) records TB_DEV_ERR_COUNT
+// and yields bin 0, so every index stays in bounds.
 template <int NT, int NB>
-__device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32_t k, ClusterSelectSmem& sm,
-                                                   uint32_t* status, uint32_t& above) {
-  for (int i = threadIdx.x; i < NB; i += NT) sm.tot[i] = __ldcg(total + i);
+__device__ __forceinline__ uint32_t find_staged_bin(uint32_t k, ClusterSelectSmem& sm, uint32_t* status,
+                                                    uint32_t& above) {
   if (threadIdx.x == 0) {
     sm.bin = -1;
     sm.above = 0;
@@ -158,6 +157,14 @@ __device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32
     return 0u;
   }
   return (uint32_t)bin;
+}
+
+// The same for a cluster total (NB words in L2), read into shared memory first.
+template <int NT, int NB>
+__device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32_t k, ClusterSelectSmem& sm,
+                                                   uint32_t* status, uint32_t& above) {
+  for (int i = threadIdx.x; i < NB; i += NT) sm.tot[i] = __ldcg(total + i);
+  return find_staged_bin<NT, NB>(k, sm, status, above);
 }
 
 // Adds this CTA's histogram into the row's total in L2 (non-empty bins only).
@@ -243,10 +250,17 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     };
-    if (wb < we) load_batch(va, wb);  // requested first: their latency overlaps the digit-1 search
-    // ---- digit 1 from the row's first-digit histogram; the bin's bounds as floats
+    // ---- digit 1 from the row's first-digit histogram; the bin's bounds as floats.
+    // The histogram is requested first, then the first batch of scores, whose
+    // latency overlaps the digit-1 search.
+    uint32_t h1[kHistBins / NT];
+#pragma unroll
+    for (int j = 0; j < kHistBins / NT; ++j) h1[j] = __ldcg(p.hist1 + row * kHistBins + tid + j * NT);
+    if (wb < we) load_batch(va, wb);
+#pragma unroll
+    for (int j = 0; j < kHistBins / NT; ++j) sm.tot[tid + j * NT] = h1[j];
     uint32_t above;
-    const uint32_t b1 = total_find_bin<NT, kHistBins>(p.hist1 + row * kHistBins, (uint32_t)rs.k, sm, p.status, above);
+    const uint32_t b1 = find_staged_bin<NT, kHistBins>((uint32_t)rs.k, sm, p.status, above);
     const uint32_t kleft = (uint32_t)rs.k - above;
     const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
     const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
