@@ -237,7 +237,9 @@ TB_API tb_status tb_sparse_attn_idx(tb_ctx* ctx, int layer, const void* q, const
  * attention, else score, select and sparse attention (TB_BUTLER per head,
  * TB_BUTLER_GROUP per KV group) or soft voting with a shared set
  * (TB_SOFTVOTE; q_imp_producer unused).  Uses the workspace for scores,
- * masks and split partials. */
+ * masks and split partials.  The workspace scores are dropped from L2
+ * without a write-back once the selection has read them (their contents are
+ * undefined after the call; the masks are kept). */
 TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const void* v_new, const void* q,
                                 const void* q_imp_producer, void* out, void* stream);
 

@@ -193,6 +193,13 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Drops the 128-byte line at p (128-byte aligned) from L2 without writing it
+// back: for intermediates that no later kernel reads, so that their dirty
+// lines do not cost HBM write bandwidth when they are evicted.
+__device__ __forceinline__ void discard_l2(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(__cvta_generic_to_global(p)) : "memory");
+}
+
 // ------------------------------------------------------------ block scans
 // Exclusive prefix sum over a block of NT threads (NT a multiple of 32,
 // NT <= 1024).  `sm` holds >= 32 words.  Every thread must call it.

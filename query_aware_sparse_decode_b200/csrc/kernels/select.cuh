@@ -65,6 +65,7 @@ struct SelectParams {
   const int32_t* sc_len;  // [B*rows] length of the cached selection
   uint32_t* sc_mask;      // [B*rows][mask_words] cached masks (refilled by fresh rows)
   int reuse_radius;
+  int discard_scores;     // 1: the scores are a dead intermediate after the selection (dropped from L2 unwritten)
   // cluster selection (select_cluster_kernel) only
   uint32_t* ctot;         // [B*rows][2048 + 1024] the cluster's digit-2 and digit-3 totals (zero between selections)
   uint32_t* cslot;        // [B*rows][32] per-CTA tie counts (0..15) and kept counts (16..31)

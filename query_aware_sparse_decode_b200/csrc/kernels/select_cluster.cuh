@@ -498,6 +498,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     gm[w] = x;
     if (refill) p.sc_mask[row * p.mask_words + (c0 >> 5) + w] = x;
     kept += __popc(x);
+    // every read of this CTA's scores is done: word w's 32 scores are one line
+    if (p.discard_scores) discard_l2(srow + c0 + 32 * w);
   }
   uint32_t kept_cta;
   (void)block_excl_scan<kClThreads>(kept, kept_cta, sm.scan);

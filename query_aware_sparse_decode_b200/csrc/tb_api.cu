@@ -308,7 +308,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
 // the first-digit histograms (and zeroed the candidate counters).
 static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool hist1_ready, int rows,
                                int32_t* idx, int idx_cap, int32_t* count, uint32_t* mask, cudaStream_t st,
-                               bool use_cache = false) {
+                               bool use_cache = false, bool scores_dead = false) {
   const tb_config& c = ctx->cfg;
   const LayerState& ls = ctx->layers[layer];
   SelectParams p{};
@@ -330,6 +330,7 @@ static tb_status launch_select(tb_ctx* ctx, int layer, const float* scores, bool
   p.keep_pct = c.keep_pct;
   p.sink = c.sink;
   p.window = c.window;
+  p.discard_scores = scores_dead ? 1 : 0;  // the decode step's workspace scores: no reader after the selection
   if (use_cache) {
     p.reuse = ctx->reuse;
     p.sc_len = ls.sc_len;
@@ -984,7 +985,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
     if (s != TB_OK) return s;
     trace_point(ctx, 2, st);
     s = launch_select(ctx, layer, ctx->scores, true, grouped ? c.n_kv_heads : c.n_q_heads, nullptr, 0, nullptr,
-                      ctx->mask, st, cached);
+                      ctx->mask, st, cached, true);
     if (s != TB_OK) return s;
     trace_point(ctx, 3, st);
     return launch_attn(ctx, layer, q, ctx->mask, grouped ? TB_MASK_GROUP : TB_MASK_PER_HEAD, out, nullptr, st);
@@ -994,7 +995,7 @@ TB_API tb_status tb_decode_step(tb_ctx* ctx, int layer, const void* k_new, const
   s = launch_softvote(ctx, layer, q, ctx->votes, ctx->hist, st);
   if (s != TB_OK) return s;
   trace_point(ctx, 2, st);
-  s = launch_select(ctx, layer, ctx->votes, true, 1, nullptr, 0, nullptr, ctx->mask, st);
+  s = launch_select(ctx, layer, ctx->votes, true, 1, nullptr, 0, nullptr, ctx->mask, st, false, true);
   if (s != TB_OK) return s;
   trace_point(ctx, 3, st);
   return launch_attn(ctx, layer, q, ctx->mask, TB_MASK_SHARED, out, nullptr, st);
