@@ -16,7 +16,8 @@
 // 2^(a - max)) pair per head and chunk.
 // softvote_reduce: merges each head's chunk pairs into (M, 1/Z) (every CTA,
 // while its first logits are in flight), then sums 2^(a - M) / Z over the
-// heads, one token per thread (logits are L2-resident).  Optionally it also
+// heads, one token per thread (logits are L2-resident), and drops the
+// CTA's logit lines from L2 unwritten (no reader follows).  Optionally it also
 // builds the first-digit histogram of the votes over the candidate range
 // [sink, len - window) for the selection that follows (warp-aggregated shared
 // atomics: votes crowd into few bins).
@@ -269,6 +270,13 @@ __global__ void __launch_bounds__(256) softvote_reduce_kernel(const VoteParams p
     }
     p.votes[(size_t)b * p.max_len + t] = v;
   }
+  // The logits are a dead intermediate once every thread has read its own:
+  // the CTA's lines (256 tokens = eight 128-byte lines per head) are dropped
+  // from L2 without a write-back.
+  __syncthreads();
+  for (int e = tid; e < p.Hq * (kVoteReduceTok / 32); e += 256)
+    discard_l2(p.logits + ((size_t)b * p.Hq + e / (kVoteReduceTok / 32)) * p.max_len + t_begin +
+               32 * (e % (kVoteReduceTok / 32)));
   if (p.hist1 == nullptr) return;
   const bool in = t < L && t >= p.sink && t < L - p.window;
   const uint32_t bin = in ? (order_key(v) >> 21) : 0xFFFFFFFFu;
