@@ -10,7 +10,8 @@
 // bf16 K_imp values): d' independent, coalesced loads, written as batches of
 // up to 16 loads ahead of their FMAs (fp32, dimension order j = 0..d'-1, the
 // group's query values broadcast from shared memory) so that many loads per
-// thread can be in flight.  The FMAs run on pairs of consecutive tokens
+// thread can be in flight; the next step's first batch is requested before
+// this step's stores and histogram updates.  The FMAs run on pairs of consecutive tokens
 // (fma.rn.f32x2: two independent round-to-nearest fp32 FMAs, the bits of two
 // fmaf).  A CTA covers `chunk` consecutive tokens (a multiple of 32, up to
 // `iters` steps of 256 threads' tokens; the launch uses 1, 2 or 4 whole
@@ -109,11 +110,24 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   constexpr int NB0 = GS * TPT > 32 ? kScoreLoadBatch / 2 : kScoreLoadBatch;
   static_assert(DIMP % NB0 == 0 || DIMP < NB0, "d' must be a multiple of the batch");
   constexpr int NB = DIMP < NB0 ? DIMP : NB0;
+  // The first batch of each iteration is requested before the previous
+  // iteration's stores and histogram updates, so those overlap its latency
+  // (when the accumulators are few enough to leave the registers for it).
+  constexpr bool AHEAD = GS * TPT <= 32;
+  uint4 v[NB];
+  auto load_batch = [&](int it, int j0) {
+    const int t0 = t_base + it * STEP + TPT * tid;
+    if (t0 < t_end) {
+      const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t0, DIMP, p.max_len);
+#pragma unroll
+      for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const uint4*>(K + (j0 + jj) * kKimpTile));
+    }
+  };
+  if (AHEAD) load_batch(0, 0);
 #pragma unroll 1
   for (int it = 0; it < p.iters; ++it) {
     const int t0 = t_base + it * STEP + TPT * tid;
     if (t0 < t_end) {
-      const KT* K = reinterpret_cast<const KT*>(p.kimp) + kimp_index(slab, 0, t0, DIMP, p.max_len);
       uint64_t acc2[GS][TPT / 2];  // token pairs (2u, 2u + 1)
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh)
@@ -121,9 +135,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
         for (int u = 0; u < TPT / 2; ++u) acc2[hh][u] = 0ull;
 #pragma unroll
       for (int j0 = 0; j0 < DIMP; j0 += NB) {
-        uint4 v[NB];
-#pragma unroll
-        for (int jj = 0; jj < NB; ++jj) v[jj] = __ldcs(reinterpret_cast<const uint4*>(K + (j0 + jj) * kKimpTile));
+        if (j0 > 0 || !AHEAD) load_batch(it, j0);
 #pragma unroll
         for (int jj = 0; jj < NB; ++jj) {
           uint64_t kv[TPT / 2];
@@ -137,6 +149,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
           }
         }
       }
+      if (AHEAD && it + 1 < p.iters) load_batch(it + 1, 0);
       float acc[GS][TPT];
 #pragma unroll
       for (int hh = 0; hh < GS; ++hh)
