@@ -178,10 +178,15 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
             if (t0 + u < L) srow[t0 + u] = acc[hh][u];
         }
         if (HIST) {
+          if (t0 >= p.sink && t0 + TPT <= L - p.window) {  // every token of the thread a candidate
 #pragma unroll
-          for (int u = 0; u < TPT; ++u) {
-            const int t = t0 + u;
-            if (t >= p.sink && t < L - p.window) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
+            for (int u = 0; u < TPT; ++u) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
+          } else {
+#pragma unroll
+            for (int u = 0; u < TPT; ++u) {
+              const int t = t0 + u;
+              if (t >= p.sink && t < L - p.window) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
+            }
           }
         }
       }

@@ -66,6 +66,7 @@ constexpr int kClMaxCluster = 16;
 constexpr int kClHist3 = 1024;                // bins of the 10-bit last digit
 constexpr int kClBatch = 4;                   // 16-byte loads per thread and batch of the first pass
 constexpr int kClTotWords = kHistBins + kClHist3 + 2;  // per row in ctot: totals, kept count, CTA ticket
+static_assert(kClTotWords % 2 == 0 && (kHistBins + kClHist3) % 2 == 0, "the (kept count, ticket) pair is one 8-byte word");
 constexpr int kClSlotWords = 2 * kClMaxCluster;    // per row in cslot
 
 struct ClusterSelectSmem {
@@ -75,7 +76,7 @@ struct ClusterSelectSmem {
   uint32_t hist[kHistBins];         // this CTA's digit-2 (then digit-3) histogram
   uint32_t tot[kHistBins];          // a cluster total read back from L2
   uint32_t scan[32];
-  uint32_t n_list, pre_ties, ntie_all, last;
+  uint32_t n_list, pre_ties, ntie_all, last, kept_total;
   int bin;
   uint32_t above;
 };
@@ -501,31 +502,35 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     // every read of this CTA's scores is done: word w's 32 scores are one line
     if (p.discard_scores) discard_l2(srow + c0 + 32 * w);
   }
-  uint32_t kept_cta;
-  (void)block_excl_scan<kClThreads>(kept, kept_cta, sm.scan);
+  // the CTA's kept count, complete in thread 0
+  uint32_t kept_cta = __reduce_add_sync(0xffffffffu, kept);
+  if (lane == 0) sm.scan[warp] = kept_cta;
+  __syncthreads();
+  if (warp == 0) kept_cta = __reduce_add_sync(0xffffffffu, lane < kClWarps ? sm.scan[lane] : 0u);
   const int sink_n = min(p.sink, rs.L);
   const uint32_t expect = (uint32_t)(sink_n + (rs.L - max(rs.L - p.window, sink_n)) + rs.k);
-  uint32_t* kept_sum = tot + kHistBins + kClHist3;  // then the CTA ticket
+  uint32_t* kept_sum = tot + kHistBins + kClHist3;  // 8-byte aligned: kept count (low word), CTA ticket (high)
   if (p.idx == nullptr) {
-    // The last CTA of the row to finish (a ticket taken after this CTA's
-    // count is added; nothing waits on it) checks the total, writes the
-    // count and clears the row's state: every CTA read the histograms and
-    // totals before taking its ticket.
+    // The last CTA of the row to finish (one 64-bit atomic adds this CTA's
+    // count and takes its ticket; nothing waits on it) checks the total,
+    // writes the count and clears the row's state: every CTA read the
+    // histograms and totals before taking its ticket.
     if (tid == 0) {
-      atomicAdd(kept_sum, kept_cta);
       __threadfence();
-      sm.last = atomicAdd(kept_sum + 1, 1u) == (uint32_t)(nc - 1) ? 1u : 0u;
+      const unsigned long long old =
+          atomicAdd(reinterpret_cast<unsigned long long*>(kept_sum), (1ull << 32) | kept_cta);
+      sm.last = (uint32_t)(old >> 32) == (uint32_t)(nc - 1) ? 1u : 0u;
+      sm.kept_total = (uint32_t)old + kept_cta;
     }
     __syncthreads();
     if (sm.last) {
       __threadfence();
       if (tid == 0) {
-        const uint32_t total = __ldcg(kept_sum);
+        const uint32_t total = sm.kept_total;
         if (p.count != nullptr) p.count[row] = (int32_t)total;
         // a reused set has the cached top-k's size, not this step's k
         if (!reused && total != expect) atomicOr(p.status, TB_DEV_ERR_COUNT);
       }
-      __syncthreads();  // the total is read before it is cleared
       for (int i = tid; i < kHistBins; i += kClThreads) p.hist1[row * kHistBins + i] = 0u;
       for (int i = tid; i < kClTotWords; i += kClThreads) tot[i] = 0u;
     }
