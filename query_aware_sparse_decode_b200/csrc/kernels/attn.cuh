@@ -45,26 +45,31 @@ struct AttnParams {
 };
 
 // Builds the CTA's gather list: the cache rows of the ascending union tokens
-// of [t0, t1) with a head bitmask each; pads to a multiple of 16 with
-// (row of t0, no head).
+// of [t0, t1) (at most kAttnMaxChunk tokens, 64 mask words) with a head
+// bitmask each; pads to a multiple of 16 with (row of t0, no head).  Warps 0
+// and 1 read the words (one per lane) and scan their counts; then each thread
+// expands half a word (16 tokens).
 template <int GS>
 __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int g, int t0, int t1, int32_t* list_idx,
                                                 uint8_t* list_hb, uint32_t* scan_sm) {
-  const int tid = threadIdx.x;
+  constexpr int NWM = kAttnMaxChunk / 32;
+  static_assert(NWM <= 64 && kAttnThreads == 2 * NWM, "two warps hold the words; a thread expands half a word");
+  __shared__ uint32_t s_u[NWM], s_excl[NWM], s_hm[GS][NWM];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwords = (t1 - t0 + 31) >> 5;
   const int w_base = t0 >> 5;
-  int base = 0;
-  for (int w0 = 0; w0 < nwords; w0 += kAttnThreads) {
-    const int w = w0 + tid;
+  const bool per_head = p.mask_mode == TB_MASK_PER_HEAD;
+  if (warp < 2) {
+    const int w = tid;
     uint32_t u = 0;
-    uint32_t hm[GS];
-#pragma unroll
-    for (int hh = 0; hh < GS; ++hh) hm[hh] = 0;
     if (w < nwords) {
-      if (p.mask_mode == TB_MASK_PER_HEAD) {
+      if (per_head) {
+        uint32_t hm[GS];
+#pragma unroll
+        for (int hh = 0; hh < GS; ++hh) hm[hh] = p.mask[((size_t)b * p.Hq + g * GS + hh) * p.mask_words + w_base + w];
 #pragma unroll
         for (int hh = 0; hh < GS; ++hh) {
-          hm[hh] = p.mask[((size_t)b * p.Hq + g * GS + hh) * p.mask_words + w_base + w];
+          s_hm[hh][w] = hm[hh];
           u |= hm[hh];
         }
       } else if (p.mask_mode == TB_MASK_SHARED) {
@@ -77,30 +82,48 @@ __device__ __forceinline__ int build_union_list(const AttnParams& p, int b, int 
       const int valid = t1 - (t0 + 32 * w);
       if (valid < 32) u &= (1u << valid) - 1u;
     }
-    uint32_t total;
-    int pos = base + (int)block_excl_scan<kAttnThreads>(__popc(u), total, scan_sm);
-    while (u) {
-      const int j = __ffs(u) - 1;
-      u &= u - 1u;
-      uint32_t hb = 0xFFu;
-      if (p.mask_mode == TB_MASK_PER_HEAD) {
-        hb = 0;
+    const uint32_t cnt = __popc(u);
+    uint32_t x = cnt;  // inclusive prefix over the warp's words
 #pragma unroll
-        for (int hh = 0; hh < GS; ++hh) hb |= ((hm[hh] >> j) & 1u) << hh;
-      }
-      list_idx[pos] = (int32_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, t0 + 32 * w + j);  // the token's cache row
-      list_hb[pos] = (uint8_t)hb;
-      ++pos;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    base += (int)total;
+    if (w < NWM) {
+      s_u[w] = u;
+      s_excl[w] = x - cnt;
+    }
+    if (lane == 31) scan_sm[warp] = x;
   }
-  const int padded = (base + kAttnTile - 1) / kAttnTile * kAttnTile;
-  for (int i = base + tid; i < padded; i += kAttnThreads) {
+  __syncthreads();
+  const uint32_t tot0 = scan_sm[0];
+  const int total = (int)(tot0 + (nwords > 32 ? scan_sm[1] : 0u));
+  {  // thread 2w + h expands half h (16 tokens) of word w
+    const int w = tid >> 1, h = tid & 1;
+    if (w < nwords) {
+      const uint32_t u = s_u[w];
+      int pos = (int)(s_excl[w] + (w >= 32 ? tot0 : 0u) + (h ? __popc(u & 0xFFFFu) : 0));
+      for (uint32_t x = h ? u >> 16 : u & 0xFFFFu; x != 0u; x &= x - 1u) {
+        const int j = 16 * h + __ffs(x) - 1;
+        uint32_t hb = 0xFFu;
+        if (per_head) {
+          hb = 0;
+#pragma unroll
+          for (int hh = 0; hh < GS; ++hh) hb |= ((s_hm[hh][w] >> j) & 1u) << hh;
+        }
+        list_idx[pos] = (int32_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, t0 + 32 * w + j);  // the token's cache row
+        list_hb[pos] = (uint8_t)hb;
+        ++pos;
+      }
+    }
+  }
+  const int padded = (total + kAttnTile - 1) / kAttnTile * kAttnTile;
+  for (int i = total + tid; i < padded; i += kAttnThreads) {
     list_idx[i] = (int32_t)kv_row(p.kl, b, g, p.Hkv, p.max_len, t0);
     list_hb[i] = 0;
   }
   __syncthreads();
-  return base;
+  return total;
 }
 
 // Writes the CTA's merged (m, l, o) partial for each head of the group from

@@ -193,6 +193,13 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Lanes below this one in the warp, as a bit mask.
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
 // Drops the 128-byte line at p (128-byte aligned) from L2 without writing it
 // back: for intermediates that no later kernel reads, so that their dirty
 // lines do not cost HBM write bandwidth when they are evicted.

@@ -46,6 +46,19 @@ struct ScoreParams {
   int lens[kMaxBatch];
 };
 
+// Copies of the fused first-digit histogram in shared memory: lane l adds
+// into copy l % copies, so that lanes whose scores fall into the same bin
+// collide less; the copies are summed when the CTA flushes.  With a bf16
+// K_imp (twice the tokens per load, so twice the updates per byte) as many
+// as fit 64 KB (nr rows of 2048 counters each); with an fp32 K_imp one (the
+// second copy measured no faster there).
+constexpr int score_hist_copies(int nr, bool kimp_bf16) {
+  return !kimp_bf16 || nr >= 8 ? 1 : 8 / nr > 4 ? 4 : 8 / nr;
+}
+constexpr size_t score_hist_smem(int nr, bool kimp_bf16) {
+  return (size_t)score_hist_copies(nr, kimp_bf16) * nr * kHistBins * 4;
+}
+
 // Packed fp32 pairs for fma.rn.f32x2.
 __device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) {
   uint64_t r;
@@ -81,7 +94,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   pdl_wait();
   pdl_trigger();
   __shared__ __align__(16) float qs[DIMP][GS];
-  extern __shared__ uint32_t hist[];  // [NR][2048] when HIST
+  constexpr int HC = score_hist_copies(NR, sizeof(KT) == 2);
+  extern __shared__ uint32_t hist[];  // [HC][NR][2048] when HIST
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int L = p.lens[b];
   const int t_base = chunk * p.chunk;
@@ -100,7 +114,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
     qs[j][hh] = to_f32(qi[(((size_t)b * p.Hq + g * GS + hh) * p.G + p.slot) * DIMP + j]);
   }
   if (HIST)
-    for (int e = tid; e < NR * kHistBins; e += kScoreThreads) hist[e] = 0;
+    for (int e = tid; e < HC * NR * kHistBins; e += kScoreThreads) hist[e] = 0;
   __syncthreads();
 
   const size_t slab = (size_t)b * p.Hkv + g;
@@ -178,14 +192,15 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
             if (t0 + u < L) srow[t0 + u] = acc[hh][u];
         }
         if (HIST) {
+          uint32_t* hrow = hist + ((tid & 31) % HC * NR + hh) * kHistBins;
           if (t0 >= p.sink && t0 + TPT <= L - p.window) {  // every token of the thread a candidate
 #pragma unroll
-            for (int u = 0; u < TPT; ++u) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
+            for (int u = 0; u < TPT; ++u) atomicAdd(&hrow[order_key(acc[hh][u]) >> 21], 1u);
           } else {
 #pragma unroll
             for (int u = 0; u < TPT; ++u) {
               const int t = t0 + u;
-              if (t >= p.sink && t < L - p.window) atomicAdd(&hist[hh * kHistBins + (order_key(acc[hh][u]) >> 21)], 1u);
+              if (t >= p.sink && t < L - p.window) atomicAdd(&hrow[order_key(acc[hh][u]) >> 21], 1u);
             }
           }
         }
@@ -195,7 +210,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
   if (HIST) {
     __syncthreads();
     for (int e = tid; e < NR * kHistBins; e += kScoreThreads) {
-      const uint32_t c = hist[e];
+      uint32_t c = 0;
+#pragma unroll
+      for (int cp = 0; cp < HC; ++cp) c += hist[cp * NR * kHistBins + e];
       if (c) atomicAdd(&p.hist[(row0 + e / kHistBins) * kHistBins + e % kHistBins], c);
     }
   }

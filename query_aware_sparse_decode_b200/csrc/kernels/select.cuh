@@ -109,12 +109,6 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
 struct RowShape {
   int L, lo, hi, k, mode;  // mode 0: no candidate kept, 1: all kept, 2: top-k by key
 };

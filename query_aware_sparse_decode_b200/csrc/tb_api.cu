@@ -259,7 +259,7 @@ static tb_status launch_score(tb_ctx* ctx, int layer, const void* q_imp, float* 
   if (maxL == 0) return cuda_status(cudaGetLastError());
   const int gs = c.n_q_heads / c.n_kv_heads;
   const bool grouped = c.variant == TB_BUTLER_GROUP;
-  const size_t smem = hist ? (size_t)(grouped ? 1 : gs) * kHistBins * 4 : 0;
+  const size_t smem = hist ? score_hist_smem(grouped ? 1 : gs, c.kimp_bf16 != 0) : 0;
   // the most tokens per CTA (up to 4 steps) that still gives about three
   // CTAs per SM; short or small batches get one step per CTA (a grid sized
   // to whole waves of exactly balanced chunks measured no faster)
