@@ -214,7 +214,7 @@ def gpu_ident(dev, local_rank: int) -> str:
 # from one ncu capture of it (B = 2, L = 131072, keep 30 %; summary under
 # profiles/).  Valid only for the kernel source it was measured on; any
 # change makes it null.
-ATTN_TRAFFIC = {"source_sha256_16": "ba858a51c5eef9bc", "bytes_per_union_row": (811.647488e6 + 7.071232e6) / 1581259}
+ATTN_TRAFFIC = {"source_sha256_16": "8da21a82852afdd5", "bytes_per_union_row": (811.624448e6 + 3.596544e6) / 1581259}
 
 
 def attn_traffic_per_row():
