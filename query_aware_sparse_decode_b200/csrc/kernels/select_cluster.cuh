@@ -22,10 +22,12 @@
 //      and appends the scores of bin b1 (a few percent of the row) to a
 //      shared list; after the pass the list's scores become keys and their
 //      second digit is histogrammed (a convergent loop over the list).
-//   3. each CTA adds its histogram into the row's total in L2 (atomics);
-//      after a cluster barrier every CTA reads the total back: digit 2, then
-//      digit 3 over the list the same way, give T and the number `quota` of
-//      keys equal to T that are kept.
+//   3. after a cluster barrier every CTA sums the cluster's digit-2
+//      histograms from their shared memory (distributed shared memory) and
+//      finds digit 2; for digit 3 (over the list) each CTA adds its histogram
+//      into the row's total in L2 (atomics) and reads it back after a
+//      cluster barrier.  Together they give T and the number `quota` of keys
+//      equal to T that are kept.
 //   4. ties at T go to the lowest indices.  When every key equal to T is
 //      kept (the usual case) each CTA keeps its own; otherwise each CTA posts
 //      its count, and after a barrier CTA c keeps the first
@@ -39,8 +41,10 @@
 //      counts are posted per CTA instead and a barrier gives every CTA its
 //      offset.
 // The cluster barriers (barrier.cluster arrive/release, wait/acquire) are the
-// only waits between CTAs, and every value they exchange goes through L2; no
-// CTA waits on a flag.  A CTA whose list overflows re-reads its tokens from
+// only waits between CTAs; the digit-2 histograms are read from the other
+// CTAs' shared memory (their digit-3 barrier keeps them alive until every
+// CTA has read them), everything else goes through L2; no CTA waits on a
+// flag.  A CTA whose list overflows re-reads its tokens from
 // L2 for steps 3-5 instead; the result is the same.  Rows that keep none or
 // all of their candidates, and rows reusing a cached selection, write their
 // words directly.
@@ -73,7 +77,8 @@ struct ClusterSelectSmem {
   uint32_t mword[kClWordsMax];      // the CTA's mask words
   uint32_t tbits[kClWordsMax];      // keys equal to T among the CTA's tokens
   uint2 list[kClListCap];           // (key, token - c0) of the threshold bin's keys
-  uint32_t hist[kHistBins];         // this CTA's digit-2 (then digit-3) histogram
+  uint32_t hist[kHistBins];         // this CTA's digit-2 histogram (read by the cluster's other CTAs)
+  uint32_t hist3[kClHist3];         // this CTA's digit-3 histogram
   uint32_t tot[kHistBins];          // a cluster total read back from L2
   uint32_t scan[32];
   uint32_t n_list, pre_ties, ntie_all, last, kept_total;
@@ -371,35 +376,39 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         if ((key >> 21) == b1) atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
       });
     }
-    __syncthreads();
-    hist_to_total<NT, kHistBins>(sm.hist, tot);
-    cluster.sync();  // the row's digit-2 total is complete in L2
-    // ---- digit 2
-    const uint32_t b2 = total_find_bin<NT, kHistBins>(tot, kleft, sm, p.status, above);
+    cluster.sync();  // every CTA's digit-2 histogram is complete in its shared memory
+    // ---- digit 2: the row's total summed from the cluster's shared histograms
+    for (int i = tid; i < kHistBins; i += kClThreads) {
+      uint32_t t = sm.hist[i];
+      for (int r = 0; r < nc; ++r)
+        if (r != c) t += *cluster.map_shared_rank(&sm.hist[i], r);
+      sm.tot[i] = t;
+    }
+    const uint32_t b2 = find_staged_bin<NT, kHistBins>(kleft, sm, p.status, above);
     const uint32_t kleft2 = kleft - above;
     const uint32_t prefix22 = (b1 << 11) | b2;
     const uint32_t n_list = sm.n_list;
     const bool overflow = n_list > (uint32_t)kClListCap;  // the list misses keys: re-read from L2
-    for (int i = tid; i < kClHist3; i += kClThreads) sm.hist[i] = 0u;
+    for (int i = tid; i < kClHist3; i += kClThreads) sm.hist3[i] = 0u;
     __syncthreads();
     if (!overflow) {
       for (uint32_t i = tid; i < n_list; i += kClThreads) {
         const uint32_t key = sm.list[i].x;
-        if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
+        if ((key >> 10) == prefix22) atomicAdd(&sm.hist3[key & (kClHist3 - 1)], 1u);
       }
     } else {
       visit_candidates<NT>(srow, c0, c1, rs.lo, rs.hi, [&](int, uint32_t key) {
-        if ((key >> 10) == prefix22) atomicAdd(&sm.hist[key & (kClHist3 - 1)], 1u);
+        if ((key >> 10) == prefix22) atomicAdd(&sm.hist3[key & (kClHist3 - 1)], 1u);
       });
     }
     __syncthreads();
-    hist_to_total<NT, kClHist3>(sm.hist, tot + kHistBins);
+    hist_to_total<NT, kClHist3>(sm.hist3, tot + kHistBins);
     cluster.sync();  // the row's digit-3 total is complete in L2
     // ---- digit 3: the k-th key T and the number of keys equal to T that are kept
     const uint32_t b3 = total_find_bin<NT, kClHist3>(tot + kHistBins, kleft2, sm, p.status, above);
     const uint32_t T = (prefix22 << 10) | b3;
     const uint32_t quota = kleft2 - above;
-    const uint32_t ntie_all = sm.tot[b3], my_ties = sm.hist[b3];
+    const uint32_t ntie_all = sm.tot[b3], my_ties = sm.hist3[b3];
     uint32_t q_c = my_ties;  // every key equal to T kept (the usual case: one key at T)
     if (ntie_all != quota) {  // the same decision in every CTA of the cluster
       if (tid == 0) slot[c] = my_ties;
