@@ -22,12 +22,12 @@
 //      and appends the scores of bin b1 (a few percent of the row) to a
 //      shared list; after the pass the list's scores become keys and their
 //      second digit is histogrammed (a convergent loop over the list).
-//   3. after a cluster barrier every CTA sums the cluster's digit-2
-//      histograms from their shared memory (distributed shared memory) and
-//      finds digit 2; for digit 3 (over the list) each CTA adds its histogram
-//      into the row's total in L2 (atomics) and reads it back after a
-//      cluster barrier.  Together they give T and the number `quota` of keys
-//      equal to T that are kept.
+//   3. in a cluster of two, after a cluster barrier each CTA adds the other
+//      CTA's digit-2 histogram from its shared memory (distributed shared
+//      memory) to its own; in larger clusters each CTA adds its histogram
+//      into the row's total in L2 (atomics) and reads the total back after a
+//      cluster barrier.  Digit 2, then digit 3 over the list through L2, give
+//      T and the number `quota` of keys equal to T that are kept.
 //   4. ties at T go to the lowest indices.  When every key equal to T is
 //      kept (the usual case) each CTA keeps its own; otherwise each CTA posts
 //      its count, and after a barrier CTA c keeps the first
@@ -41,9 +41,9 @@
 //      counts are posted per CTA instead and a barrier gives every CTA its
 //      offset.
 // The cluster barriers (barrier.cluster arrive/release, wait/acquire) are the
-// only waits between CTAs; the digit-2 histograms are read from the other
-// CTAs' shared memory (their digit-3 barrier keeps them alive until every
-// CTA has read them), everything else goes through L2; no CTA waits on a
+// only waits between CTAs; in a cluster of two the digit-2 histogram is read
+// from the other CTA's shared memory (the digit-3 barrier keeps it alive
+// until both have read), everything else goes through L2; no CTA waits on a
 // flag.  A CTA whose list overflows re-reads its tokens from
 // L2 for steps 3-5 instead; the result is the same.  Rows that keep none or
 // all of their candidates, and rows reusing a cached selection, write their
@@ -376,15 +376,21 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         if ((key >> 21) == b1) atomicAdd(&sm.hist[(key >> 10) & (kHistBins - 1)], 1u);
       });
     }
-    cluster.sync();  // every CTA's digit-2 histogram is complete in its shared memory
-    // ---- digit 2: the row's total summed from the cluster's shared histograms
-    for (int i = tid; i < kHistBins; i += kClThreads) {
-      uint32_t t = sm.hist[i];
-      for (int r = 0; r < nc; ++r)
-        if (r != c) t += *cluster.map_shared_rank(&sm.hist[i], r);
-      sm.tot[i] = t;
+    // ---- digit 2: the row's total, from the other CTA's shared histogram in
+    // a cluster of two, else through L2 (remote reads of many CTAs' 2048 bins
+    // cost more than the atomics and the read-back)
+    uint32_t b2;
+    if (nc <= 2) {
+      cluster.sync();  // every CTA's digit-2 histogram is complete in its shared memory
+      const uint32_t* other = nc == 2 ? cluster.map_shared_rank(sm.hist, c ^ 1) : nullptr;
+      for (int i = tid; i < kHistBins; i += kClThreads) sm.tot[i] = sm.hist[i] + (other ? other[i] : 0u);
+      b2 = find_staged_bin<NT, kHistBins>(kleft, sm, p.status, above);
+    } else {
+      __syncthreads();
+      hist_to_total<NT, kHistBins>(sm.hist, tot);
+      cluster.sync();  // the row's digit-2 total is complete in L2
+      b2 = total_find_bin<NT, kHistBins>(tot, kleft, sm, p.status, above);
     }
-    const uint32_t b2 = find_staged_bin<NT, kHistBins>(kleft, sm, p.status, above);
     const uint32_t kleft2 = kleft - above;
     const uint32_t prefix22 = (b1 << 11) | b2;
     const uint32_t n_list = sm.n_list;
