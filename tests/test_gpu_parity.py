@@ -255,6 +255,45 @@ def test_single_row_select_on_crowded_bins(kind, keep):
         assert np.array_equal(got_sets[b, 0], ref)
 
 
+@pytest.mark.parametrize("kind", [None, "two_digits", "three_values"])
+def test_select_clusters_of_two_exchange_digit_two_in_shared_memory(kind):
+    """128 rows just over 65536 tokens: clusters of two CTAs (512 threads),
+    the shape whose digit-2 histograms are summed through distributed shared
+    memory.  Exact sets and counts on identical fp32 scores, including rows
+    whose top two digits leave two bins (the exchanged histogram decides) and
+    rows where ties at the threshold take most of the budget."""
+    lens = (70000, 69001, 65537, 70000)
+    B, Hq, Hkv = len(lens), 32, 8
+    keep = 30
+    wl = S.Workload("sel_pair", n_layers=1, B=B, Hq=Hq, Hkv=Hkv, D=64, d_imp=16, G=1, L=max(lens), dtype="f32",
+                    keep_pct=keep, sink=16, window=64, plant="none", lens=lens)
+    cfg = config_of(wl)
+    Lmax = cfg.max_len
+    ctx = TB.Context(cfg)
+    dummy = torch.zeros((B, Hkv, Lmax, 64), device="cuda")
+    ctx.bind_layer(0, dummy, dummy.clone(), kimp_alloc(B, Hkv, 16, Lmax), torch.zeros((64, 16), device="cuda"))
+    ctx.set_seq_lens(0, lens)
+    if kind is None:
+        sc = _synthetic_scores(B, Hq, Lmax, 0, 907)
+    else:
+        sc = np.zeros((B, Hq, Lmax), np.float32)
+        for b, L in enumerate(lens):
+            for r in range(Hq):
+                sc[b, r, :L] = _crowded_scores(kind, L, 300 + 32 * b + r)
+    cnt = torch.full((B, Hq), -1, dtype=torch.int32, device="cuda")
+    mask = torch.zeros((B, Hq, Lmax // 32), dtype=torch.int32, device="cuda")
+    ctx.select(0, torch.from_numpy(sc).cuda(), Hq, count=cnt, mask=mask)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    cnt = cnt.cpu().numpy()
+    got_sets = sets_from_mask(mask, lens)
+    for b, L in enumerate(lens):
+        for r in range(Hq):
+            ref = O.select_tokens(sc[b, r].astype(np.float64), L, keep, wl.sink, wl.window)
+            assert cnt[b, r] == ref.size, f"b{b} r{r}"
+            assert np.array_equal(got_sets[b, r], ref), f"b{b} r{r}"
+
+
 @pytest.mark.parametrize("kind", [None, "two_digits"])
 def test_select_rows_beyond_one_cluster(kind):
     """Rows longer than a cluster of 16 CTAs of 65536 tokens (1048576) take
