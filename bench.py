@@ -163,9 +163,24 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def begin(self, timeout: float = 2.0):
+        """Waits (bounded) for the sampler's first line, then marks the start
+        of the timed region: only samples from here on are summarised."""
+        t_end = time.time() + timeout
+        while self.proc is not None and not self.lines and time.time() < t_end:
+            time.sleep(0.01)
+        self.first = len(self.lines)
+
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # a timed region shorter than the 200 ms period may see no sample: wait
+        # (bounded) for the one that follows it
+        first = getattr(self, "first", 0)
+        t_end = time.time() + 0.5
+        while len(self.lines) <= first and time.time() < t_end:
+            time.sleep(0.01)
+        self.lines = self.lines[first:]
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -421,6 +436,7 @@ def gpu_arm(args, rank, world, local_rank):
     # ---- device-timed region: inputs resident in HBM
     clocks = ClockSampler(gpu_ident(dev, local_rank))
     clocks.start()
+    clocks.begin()
     n0 = ctx.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -580,6 +596,7 @@ def shard_arm(args, rank, world, local_rank):
     barrier()
     clocks = ClockSampler(gpu_ident(dev, local_rank))
     clocks.start()
+    clocks.begin()
     n0 = ctx.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
