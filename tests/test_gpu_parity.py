@@ -294,6 +294,51 @@ def test_select_clusters_of_two_exchange_digit_two_in_shared_memory(kind):
             assert np.array_equal(got_sets[b, r], ref), f"b{b} r{r}"
 
 
+@pytest.mark.parametrize("kind", ["two_digits", "three_values"])
+def test_decode_step_on_controlled_scores_in_clusters_of_two(kind):
+    """The fused decode step (score kernel with its first-digit histogram,
+    clusters of two CTAs exchanging digit 2 in shared memory, the scores
+    dropped from L2 after the selection) on scores it computes exactly: the
+    importance query is the first unit vector and K_imp holds crowded values
+    in its first dimension (W_K = 0, so the appended token scores 0).  The
+    step's masks must be the oracle's sets exactly."""
+    lens0 = (69999, 69000, 65536, 69999)
+    B, Hq, Hkv, D, dimp = len(lens0), 32, 8, 64, 16
+    keep = 30
+    wl = S.Workload("step_ctl", n_layers=1, B=B, Hq=Hq, Hkv=Hkv, D=D, d_imp=dimp, G=1, L=max(lens0) + 1, dtype="f32",
+                    keep_pct=keep, sink=16, window=64, plant="none", lens=tuple(L + 1 for L in lens0))
+    cfg = config_of(wl)
+    Lmax = cfg.max_len
+    ctx = TB.Context(cfg)
+    k_cache = torch.zeros((B, Hkv, Lmax, D), device="cuda")
+    v_cache = torch.zeros_like(k_cache)
+    kimp = kimp_alloc(B, Hkv, dimp, Lmax)
+    vals = np.zeros((B, Hkv, Lmax), np.float32)
+    for b, L in enumerate(lens0):
+        for g in range(Hkv):
+            vals[b, g, :L] = _crowded_scores(kind, L, 500 + 8 * b + g)
+    kimp[:, :, :, 0, :] = torch.from_numpy(vals.reshape(B, Hkv, Lmax // 256, 256)).cuda()
+    ctx.bind_layer(0, k_cache, v_cache, kimp, torch.zeros((D, dimp), device="cuda"))
+    ctx.set_seq_lens(0, list(lens0))
+    q_imp = torch.zeros((B * Hq, 1, dimp), device="cuda")
+    q_imp[:, 0, 0] = 1.0
+    q = torch.from_numpy(S.fill_host(22, 3, 0, B * Hq, 0, D, 1, "f32").reshape(B, Hq, D)).cuda()
+    zero_row = torch.zeros((B, Hkv, D), device="cuda")
+    out = torch.empty((B, Hq, D), device="cuda")
+    ctx.decode_step(0, zero_row, zero_row.clone(), q, q_imp, out)
+    masks = ctx.step_masks(Hq)
+    torch.cuda.synchronize()
+    assert ctx.check_status() == 0
+    lens = ctx.seq_lens(0)
+    got_sets = sets_from_mask(masks, lens)
+    for b, L in enumerate(lens):
+        for h in range(Hq):
+            row = np.zeros(L, np.float64)
+            row[:L - 1] = vals[b, O.kv_head_of(h, Hq, Hkv), :L - 1]
+            ref = O.select_tokens(row, L, keep, wl.sink, wl.window)
+            assert np.array_equal(got_sets[b, h], ref), f"b{b} h{h}"
+
+
 @pytest.mark.parametrize("kind", [None, "two_digits"])
 def test_select_rows_beyond_one_cluster(kind):
     """Rows longer than a cluster of 16 CTAs of 65536 tokens (1048576) take
