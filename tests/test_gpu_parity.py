@@ -255,14 +255,18 @@ def test_single_row_select_on_crowded_bins(kind, keep):
         assert np.array_equal(got_sets[b, 0], ref)
 
 
-@pytest.mark.parametrize("kind", [None, "two_digits", "three_values"])
-def test_select_clusters_of_two_exchange_digit_two_in_shared_memory(kind):
+@pytest.mark.parametrize("kind,lens", [(None, (70000, 69001, 65537, 70000)),
+                                       ("two_digits", (70000, 69001, 65537, 70000)),
+                                       ("three_values", (70000, 69001, 65537, 70000)),
+                                       (None, (70000, 1000, 1, 65537))],
+                         ids=["random", "two_digits", "three_values", "ragged"])
+def test_select_clusters_of_two_exchange_digit_two_in_shared_memory(kind, lens):
     """128 rows just over 65536 tokens: clusters of two CTAs (512 threads),
     the shape whose digit-2 histograms are summed through distributed shared
     memory.  Exact sets and counts on identical fp32 scores, including rows
-    whose top two digits leave two bins (the exchanged histogram decides) and
-    rows where ties at the threshold take most of the budget."""
-    lens = (70000, 69001, 65537, 70000)
+    whose top two digits leave two bins (the exchanged histogram decides),
+    rows where ties at the threshold take most of the budget, and short rows
+    whose second CTA holds no token."""
     B, Hq, Hkv = len(lens), 32, 8
     keep = 30
     wl = S.Workload("sel_pair", n_layers=1, B=B, Hq=Hq, Hkv=Hkv, D=64, d_imp=16, G=1, L=max(lens), dtype="f32",
