@@ -72,6 +72,28 @@ struct SelectParams {
   int lens[kMaxBatch];
 };
 
+// Exclusive prefix sum over a block of NT threads with one barrier: a warp
+// scan, the warp totals through `sm` (>= NT / 32 words), and each warp's
+// base as a reduction over the totals before it.  `sm` may be written again
+// only after a later block barrier.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan_1b(uint32_t v, uint32_t& total, uint32_t* sm) {
+  constexpr int NW = NT / 32;
+  static_assert(NW >= 1 && NW <= 32, "1 to 32 warps");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm[warp] = x;
+  __syncthreads();
+  const uint32_t wt = lane < NW ? sm[lane] : 0u;
+  total = __reduce_add_sync(0xffffffffu, wt);
+  return __reduce_add_sync(0xffffffffu, lane < warp ? wt : 0u) + x - v;
+}
+
 // Find the bin b (scanning from the top) where the running count reaches k:
 // sum(bins > b) < k <= sum(bins >= b).  NB = PER * NT bins.
 template <int PER, int NT = kSelThreads>
@@ -87,7 +109,7 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t k, uint3
     local += c[j];
   }
   uint32_t total;
-  const uint32_t excl = block_excl_scan<NT>(local, total, scan_sm);
+  const uint32_t excl = block_excl_scan_1b<NT>(local, total, scan_sm);  // scan_sm is free again after the barrier below
   if (excl < k && k <= excl + local) {
     uint32_t run = excl;
 #pragma unroll
