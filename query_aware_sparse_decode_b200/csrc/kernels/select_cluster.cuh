@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
   if (topk) {
     for (int i = tid; i < nw; i += kClThreads) sm.tbits[i] = 0u;
     for (int i = tid; i < kHistBins; i += kClThreads) sm.hist[i] = 0u;
+    for (int i = tid; i < kClHist3; i += kClThreads) sm.hist3[i] = 0u;
     if (tid == 0) sm.n_list = 0u;
     // Warp w owns words [wb, we) and walks them in batches of 16 words: lane l
     // loads the 16 bytes at tokens 32 * (w0 + 4u + l / 8) + 4 * (l % 8),
@@ -395,9 +396,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     const uint32_t prefix22 = (b1 << 11) | b2;
     const uint32_t n_list = sm.n_list;
     const bool overflow = n_list > (uint32_t)kClListCap;  // the list misses keys: re-read from L2
-    for (int i = tid; i < kClHist3; i += kClThreads) sm.hist3[i] = 0u;
-    __syncthreads();
-    if (!overflow) {
+    if (!overflow) {  // (hist3 was zeroed at the start; the digit-2 search ended with a block barrier)
       for (uint32_t i = tid; i < n_list; i += kClThreads) {
         const uint32_t key = sm.list[i].x;
         if ((key >> 10) == prefix22) atomicAdd(&sm.hist3[key & (kClHist3 - 1)], 1u);
@@ -428,14 +427,18 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
       const uint32_t pre = sm.pre_ties;
       q_c = quota > pre ? min(quota - pre, my_ties) : 0u;
     }
-    // ---- keys of bin b1 above T into the words, keys equal to T into the tie bitmap
+    // ---- keys of bin b1 above T into the words; keys equal to T into the words
+    // too when this CTA keeps all of its ties (the usual case), else into the
+    // tie bitmap
+    const bool all_ties = q_c == my_ties;  // uniform in the CTA
+    uint32_t* tie_dst = all_ties ? sm.mword : sm.tbits;
     if (!overflow) {
       for (uint32_t i = tid; i < n_list; i += kClThreads) {
         const uint2 e = sm.list[i];
         if (e.x > T)
           atomicOr(&sm.mword[e.y >> 5], 1u << (e.y & 31));
         else if (e.x == T)
-          atomicOr(&sm.tbits[e.y >> 5], 1u << (e.y & 31));
+          atomicOr(&tie_dst[e.y >> 5], 1u << (e.y & 31));
       }
     } else {
       visit_candidates<NT>(srow, c0, c1, rs.lo, rs.hi, [&](int t, uint32_t key) {
@@ -443,14 +446,12 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         if (key > T && (key >> 21) == b1)
           atomicOr(&sm.mword[o >> 5], 1u << (o & 31));
         else if (key == T)
-          atomicOr(&sm.tbits[o >> 5], 1u << (o & 31));
+          atomicOr(&tie_dst[o >> 5], 1u << (o & 31));
       });
     }
-    __syncthreads();
     // ---- the first q_c ties of this CTA, in token order
-    if (q_c == my_ties) {
-      for (int w = tid; w < nw; w += kClThreads) sm.mword[w] |= sm.tbits[w];
-    } else if (q_c > 0) {  // uniform in the CTA
+    if (!all_ties && q_c > 0) {  // uniform in the CTA
+      __syncthreads();  // the tie bitmap is complete
       constexpr int WPT = kClWordsMax / kClThreads;
       const int w0 = tid * WPT;
       uint32_t cnt = 0;
