@@ -79,11 +79,10 @@ struct ClusterSelectSmem {
   uint2 list[kClListCap];           // (key, token - c0) of the threshold bin's keys
   uint32_t hist[kHistBins];         // this CTA's digit-2 histogram (read by the cluster's other CTAs)
   uint32_t hist3[kClHist3];         // this CTA's digit-3 histogram
-  uint32_t tot[kHistBins];          // a cluster total read back from L2
   uint32_t scan[32];
   uint32_t n_list, pre_ties, ntie_all, last, kept_total;
   int bin;
-  uint32_t above;
+  uint32_t above, bin_count;
 };
 constexpr int kClSmem = ((int)sizeof(ClusterSelectSmem) + 15) / 16 * 16;
 // Dynamic shared memory of an NT-thread CTA: the struct, then the first
@@ -142,35 +141,66 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// The bin where the running count from the top of a histogram staged in
-// sm.tot (NB words, stored by the caller) reaches k.  A histogram holding
-// fewer than k keys (inconsistent scores, e.g. NaN) records TB_DEV_ERR_COUNT
-// and yields bin 0, so every index stays in bounds.
-template <int NT, int NB>
-__device__ __forceinline__ uint32_t find_staged_bin(uint32_t k, ClusterSelectSmem& sm, uint32_t* status,
-                                                    uint32_t& above) {
-  if (threadIdx.x == 0) {
-    sm.bin = -1;
-    sm.above = 0;
+// The bin b where the running count from the top of an NB-bin histogram
+// reaches k (sum(bins > b) < k <= sum(bins >= b)), from the counts the
+// threads hold: thread t holds bins NB - 1 - (t * PER + j), j = 0..PER-1
+// (descending), so that no staging through shared memory is needed.  One
+// scan barrier and one closing barrier.  Also gives the bin's count.  A
+// histogram holding fewer than k keys (inconsistent scores, e.g. NaN)
+// records TB_DEV_ERR_COUNT and yields bin 0, so every index stays in bounds.
+template <int NT, int PER>
+__device__ __forceinline__ uint32_t find_bin_held(const uint32_t (&c)[PER], uint32_t k, ClusterSelectSmem& sm,
+                                                  uint32_t* status, uint32_t& above, uint32_t& count) {
+  constexpr int NB = PER * NT;
+  const int tid = threadIdx.x;
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) local += c[j];
+  if (tid == 0) sm.bin = -1;  // before the scan's barrier; the crossing thread writes after it
+  uint32_t total;
+  const uint32_t excl = block_excl_scan_1b<NT>(local, total, sm.scan);
+  if (excl < k && k <= excl + local) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      if (run + c[j] >= k) {
+        sm.bin = NB - 1 - (tid * PER + j);
+        sm.above = run;
+        sm.bin_count = c[j];
+        break;
+      }
+      run += c[j];
+    }
   }
   __syncthreads();
-  find_bin<NB / NT, NT>(sm.tot, k, sm.scan, &sm.bin, &sm.above);  // ends with a block barrier
   const int bin = sm.bin;
-  above = sm.above;
   if (bin < 0) {
-    if (threadIdx.x == 0) atomicOr(status, TB_DEV_ERR_COUNT);
+    if (tid == 0) atomicOr(status, TB_DEV_ERR_COUNT);
     above = 0;
+    count = 0;
     return 0u;
   }
+  above = sm.above;
+  count = sm.bin_count;
   return (uint32_t)bin;
 }
 
-// The same for a cluster total (NB words in L2), read into shared memory first.
-template <int NT, int NB>
-__device__ __forceinline__ uint32_t total_find_bin(const uint32_t* total, uint32_t k, ClusterSelectSmem& sm,
-                                                   uint32_t* status, uint32_t& above) {
-  for (int i = threadIdx.x; i < NB; i += NT) sm.tot[i] = __ldcg(total + i);
-  return find_staged_bin<NT, NB>(k, sm, status, above);
+// This thread's bins of an NB-word histogram in L2 (NB = PER * NT), in the
+// order find_bin_held wants: bins NB - 1 - (t * PER + j).
+template <int NT, int PER>
+__device__ __forceinline__ void load_bins_desc(const uint32_t* h, uint32_t (&c)[PER]) {
+  constexpr int NB = PER * NT;
+  const uint32_t* lo = h + NB - (threadIdx.x + 1) * PER;  // this thread's bins, ascending
+  if constexpr (PER == 4) {
+    const uint4 x = __ldcg(reinterpret_cast<const uint4*>(lo));
+    c[0] = x.w; c[1] = x.z; c[2] = x.y; c[3] = x.x;
+  } else if constexpr (PER == 2) {
+    const uint2 x = __ldcg(reinterpret_cast<const uint2*>(lo));
+    c[0] = x.y; c[1] = x.x;
+  } else {
+#pragma unroll
+    for (int j = 0; j < PER; ++j) c[j] = __ldcg(lo + PER - 1 - j);
+  }
 }
 
 // Adds this CTA's histogram into the row's total in L2 (non-empty bins only).
@@ -260,14 +290,12 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     // ---- digit 1 from the row's first-digit histogram; the bin's bounds as floats.
     // The histogram is requested first, then the first batch of scores, whose
     // latency overlaps the digit-1 search.
-    uint32_t h1[kHistBins / NT];
-#pragma unroll
-    for (int j = 0; j < kHistBins / NT; ++j) h1[j] = __ldcg(p.hist1 + row * kHistBins + tid + j * NT);
+    constexpr int P1 = kHistBins / NT;
+    uint32_t h1[P1];
+    load_bins_desc<NT, P1>(p.hist1 + row * kHistBins, h1);
     if (wb < we) load_batch(va, wb);
-#pragma unroll
-    for (int j = 0; j < kHistBins / NT; ++j) sm.tot[tid + j * NT] = h1[j];
-    uint32_t above;
-    const uint32_t b1 = find_staged_bin<NT, kHistBins>((uint32_t)rs.k, sm, p.status, above);
+    uint32_t above, bcount;
+    const uint32_t b1 = find_bin_held<NT, P1>(h1, (uint32_t)rs.k, sm, p.status, above, bcount);
     const uint32_t kleft = (uint32_t)rs.k - above;
     const bool hi_open = b1 == (uint32_t)(kHistBins - 1);                   // no key above the bin
     const float f_lo = key_to_float(b1 << 21);                              // smallest key of the bin
@@ -380,18 +408,22 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     // ---- digit 2: the row's total, from the other CTA's shared histogram in
     // a cluster of two, else through L2 (remote reads of many CTAs' 2048 bins
     // cost more than the atomics and the read-back)
-    uint32_t b2;
+    uint32_t h2[P1];
     if (nc <= 2) {
       cluster.sync();  // every CTA's digit-2 histogram is complete in its shared memory
       const uint32_t* other = nc == 2 ? cluster.map_shared_rank(sm.hist, c ^ 1) : nullptr;
-      for (int i = tid; i < kHistBins; i += kClThreads) sm.tot[i] = sm.hist[i] + (other ? other[i] : 0u);
-      b2 = find_staged_bin<NT, kHistBins>(kleft, sm, p.status, above);
+#pragma unroll
+      for (int j = 0; j < P1; ++j) {
+        const int bin = kHistBins - 1 - (tid * P1 + j);
+        h2[j] = sm.hist[bin] + (other ? other[bin] : 0u);
+      }
     } else {
       __syncthreads();
       hist_to_total<NT, kHistBins>(sm.hist, tot);
       cluster.sync();  // the row's digit-2 total is complete in L2
-      b2 = total_find_bin<NT, kHistBins>(tot, kleft, sm, p.status, above);
+      load_bins_desc<NT, P1>(tot, h2);
     }
+    const uint32_t b2 = find_bin_held<NT, P1>(h2, kleft, sm, p.status, above, bcount);
     const uint32_t kleft2 = kleft - above;
     const uint32_t prefix22 = (b1 << 11) | b2;
     const uint32_t n_list = sm.n_list;
@@ -410,10 +442,14 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     hist_to_total<NT, kClHist3>(sm.hist3, tot + kHistBins);
     cluster.sync();  // the row's digit-3 total is complete in L2
     // ---- digit 3: the k-th key T and the number of keys equal to T that are kept
-    const uint32_t b3 = total_find_bin<NT, kClHist3>(tot + kHistBins, kleft2, sm, p.status, above);
+    constexpr int P3 = kClHist3 / NT;
+    uint32_t h3[P3];
+    load_bins_desc<NT, P3>(tot + kHistBins, h3);
+    uint32_t ntie_all;
+    const uint32_t b3 = find_bin_held<NT, P3>(h3, kleft2, sm, p.status, above, ntie_all);
     const uint32_t T = (prefix22 << 10) | b3;
     const uint32_t quota = kleft2 - above;
-    const uint32_t ntie_all = sm.tot[b3], my_ties = sm.hist3[b3];
+    const uint32_t my_ties = sm.hist3[b3];
     uint32_t q_c = my_ties;  // every key equal to T kept (the usual case: one key at T)
     if (ntie_all != quota) {  // the same decision in every CTA of the cluster
       if (tid == 0) slot[c] = my_ties;
