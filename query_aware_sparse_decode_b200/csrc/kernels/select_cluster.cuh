@@ -412,11 +412,17 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
     if (nc <= 2) {
       cluster.sync();  // every CTA's digit-2 histogram is complete in its shared memory
       const uint32_t* other = nc == 2 ? cluster.map_shared_rank(sm.hist, c ^ 1) : nullptr;
+      const int lo = kHistBins - (tid + 1) * P1;  // this thread's bins, ascending
+      uint32_t o[P1];
+      if constexpr (P1 == 4) {  // one 16-byte read of the other CTA's shared memory
+        const uint4 x = other ? *reinterpret_cast<const uint4*>(other + lo) : make_uint4(0u, 0u, 0u, 0u);
+        o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+      } else {
 #pragma unroll
-      for (int j = 0; j < P1; ++j) {
-        const int bin = kHistBins - 1 - (tid * P1 + j);
-        h2[j] = sm.hist[bin] + (other ? other[bin] : 0u);
+        for (int j = 0; j < P1; ++j) o[j] = other ? other[lo + j] : 0u;
       }
+#pragma unroll
+      for (int j = 0; j < P1; ++j) h2[j] = sm.hist[lo + P1 - 1 - j] + o[P1 - 1 - j];
     } else {
       __syncthreads();
       hist_to_total<NT, kHistBins>(sm.hist, tot);
