@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
         if (!reused && total != expect) atomicOr(p.status, TB_DEV_ERR_COUNT);
       }
       for (int i = tid; i < kHistBins; i += kClThreads) p.hist1[row * kHistBins + i] = 0u;
-      for (int i = tid; i < kClTotWords; i += kClThreads) tot[i] = 0u;
+      for (int i = tid + (nc <= 2 ? kHistBins : 0); i < kClTotWords; i += kClThreads) tot[i] = 0u;  // digit-2 totals unused in pairs
     }
     return;
   }
@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_cluster_kernel(const Sel
   }
   if (c == 0) {  // every CTA read the histograms and totals before the last cluster barrier
     for (int i = tid; i < kHistBins; i += kClThreads) p.hist1[row * kHistBins + i] = 0u;
-    for (int i = tid; i < kClTotWords; i += kClThreads) tot[i] = 0u;
+    for (int i = tid + (nc <= 2 ? kHistBins : 0); i < kClTotWords; i += kClThreads) tot[i] = 0u;  // digit-2 totals unused in pairs
   }
 }
 
